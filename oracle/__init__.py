@@ -1,0 +1,131 @@
+"""Float64 CPU oracle of the GradLev scan (test infrastructure only).
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package. The product path (the CUDA library and
+``token_weight_scans_b200``) never does, and shares no code with it.
+
+The arithmetic lives in ``gradlev_oracle.cpp`` (serial token-by-token loops
+in double / complex<double>, see that file's header for the definition and
+its sources); this module only builds the shared object with g++ and marshals
+numpy arrays through ctypes.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gradlev_oracle.cpp")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with g++ (-O2, OpenMP, no fast-math). Returns the .so path."""
+    if (not force and os.path.exists(_LIB)
+            and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC)):
+        return _LIB
+    tmp = _LIB + f".tmp{os.getpid()}"
+    cmd = ["g++", "-O2", "-std=c++17", "-fopenmp", "-fPIC", "-shared",
+           "-fno-fast-math", "-ffp-contract=off", _SRC, "-o", tmp]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            P = ctypes.c_void_p
+            I = ctypes.c_int
+            lib.oracle_fwd_f64.argtypes = [I] * 5 + [P] * 6 + [I]
+            lib.oracle_fwd_c128.argtypes = [I] * 5 + [P] * 6 + [I]
+            lib.oracle_states_f64.argtypes = [I] * 3 + [P] * 7
+            lib.oracle_bwd_f64.argtypes = [I] * 5 + [P] * 11 + [I] * 3
+            lib.oracle_serial_f64.argtypes = [I] * 5 + [P] * 7 + [I]
+            lib.oracle_serial_c128.argtypes = [I] * 5 + [P] * 7 + [I]
+            lib.oracle_max_threads.restype = I
+            _lib = lib
+    return _lib
+
+
+def max_threads() -> int:
+    """Threads an oracle call uses when ``nthreads`` is 0 (OpenMP default)."""
+    return int(_load().oracle_max_threads())
+
+
+def _arr(a, dtype):
+    return np.ascontiguousarray(np.asarray(a), dtype=dtype)
+
+
+def _p(a):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dims(x, g):
+    B, H, T, din = x.shape
+    dout = g.shape[-1]
+    assert g.shape == (B, H, T, dout)
+    return B, H, T, din, dout
+
+
+def fwd(x, g, eta, alpha, W0, nthreads: int = 0):
+    """y [B,H,T,d_out] of the forward scan. Complex inputs run the complex instantiation."""
+    cplx = any(np.iscomplexobj(np.asarray(a)) for a in (x, g, eta, alpha, W0))
+    dt = np.complex128 if cplx else np.float64
+    x, g, eta, alpha, W0 = (_arr(a, dt) for a in (x, g, eta, alpha, W0))
+    B, H, T, din, dout = _dims(x, g)
+    assert eta.shape == alpha.shape == (B, H, T) and W0.shape == (H, dout, din)
+    y = np.empty((B, H, T, dout), dtype=dt)
+    f = _load().oracle_fwd_c128 if cplx else _load().oracle_fwd_f64
+    f(B, H, T, din, dout, _p(x), _p(g), _p(eta), _p(alpha), _p(W0), _p(y), int(nthreads))
+    return y
+
+
+def states(x, g, eta, alpha, W0):
+    """(y [T,d_out], S [T+1,d_out,d_in]) for ONE scan given as 2-D/1-D arrays."""
+    x, g, eta, alpha, W0 = (_arr(a, np.float64) for a in (x, g, eta, alpha, W0))
+    T, din = x.shape
+    dout = g.shape[1]
+    y = np.empty((T, dout))
+    S = np.empty((T + 1, dout, din))
+    _load().oracle_states_f64(T, din, dout, _p(x), _p(g), _p(eta), _p(alpha), _p(W0),
+                              _p(y), _p(S))
+    return y, S
+
+
+def bwd(x, g, eta, alpha, W0, dy, ckpt: int = 64, mutate: bool = False, nthreads: int = 0):
+    """Reverse scan. Returns dict dx, dg, deta, dalpha, dW0 (dW0 summed over b)."""
+    x, g, eta, alpha, W0, dy = (_arr(a, np.float64) for a in (x, g, eta, alpha, W0, dy))
+    B, H, T, din, dout = _dims(x, g)
+    assert dy.shape == g.shape and W0.shape == (H, dout, din)
+    out = dict(dx=np.empty_like(x), dg=np.empty_like(g), deta=np.empty_like(eta),
+               dalpha=np.empty_like(alpha), dW0=np.empty_like(W0))
+    _load().oracle_bwd_f64(B, H, T, din, dout, _p(x), _p(g), _p(eta), _p(alpha), _p(W0),
+                           _p(dy), _p(out["dx"]), _p(out["dg"]), _p(out["deta"]),
+                           _p(out["dalpha"]), _p(out["dW0"]), int(ckpt), 1 if mutate else 0,
+                           int(nthreads))
+    return out
+
+
+def serial(x, v, eta, alpha, W0, nthreads: int = 0):
+    """Serial online learner with inner loss 0.5||W x - v||^2: returns (y, g*)."""
+    cplx = any(np.iscomplexobj(np.asarray(a)) for a in (x, v, eta, alpha, W0))
+    dt = np.complex128 if cplx else np.float64
+    x, v, eta, alpha, W0 = (_arr(a, dt) for a in (x, v, eta, alpha, W0))
+    B, H, T, din, dout = _dims(x, v)
+    y = np.empty((B, H, T, dout), dtype=dt)
+    gs = np.empty((B, H, T, dout), dtype=dt)
+    f = _load().oracle_serial_c128 if cplx else _load().oracle_serial_f64
+    f(B, H, T, din, dout, _p(x), _p(v), _p(eta), _p(alpha), _p(W0), _p(y), _p(gs),
+      int(nthreads))
+    return y, gs

@@ -1,0 +1,307 @@
+// GradLev scan oracle: plain, serial, float64 CPU implementation.
+//
+// TEST INFRASTRUCTURE ONLY. Nothing in the product path (the CUDA library and
+// its Python binding) may include, link or call this file; only the tests,
+// the package's smoke check and the CPU-baseline leg of the benchmark do.
+// It shares no code, header or constant with the CUDA path.
+//
+// What it computes (one adaptive linear layer, per batch b and head h):
+//
+//   Cognaptus, "Parallelize the Training, Keep the Learning Serial", section
+//   "Once the gradient signals are known, the weight trajectory becomes
+//   parallelizable": a temporary weight W_t, initialised from the persistent
+//   weight W_0, is updated once per token with a centred rule driven by the
+//   layer input x_t, a step size eta_t, a retention gate alpha_t and the
+//   costate g_t (gradient of the token loss w.r.t. the layer output). The
+//   display equation is missing from the extracted page; the reading used here
+//   (the deviation D = W - W_0 decays by alpha and receives a rank-one
+//   gradient step) is:
+//
+//       D_0 = 0,   y_t = (W_0 + D_{t-1}) x_t,   D_t = alpha_t D_{t-1} - eta_t g_t x_t^T
+//
+//   in the page's 1-based notation. With 0-based tokens and S_t := the
+//   deviation BEFORE token t this is
+//
+//       S_0 = 0,   y_t = (W_0 + S_t) x_t,       S_{t+1} = alpha_t S_t - eta_t g_t x_t^T.
+//
+//   GradLev abstract (omanscience.com / scholarbro.com, "GradLev: Token-Parallel
+//   Test-Time Training Via Costate Prediction", Abstract): given inputs and
+//   costates, online gradient descent admits exact scans for forward
+//   evaluation and for reverse backpropagation. The backward here is the exact
+//   reverse-mode derivative of the recurrence above for the scalar objective
+//   L = sum_t <u_t, y_t> (u = dL/dy supplied by the caller), written as the
+//   adjoint recurrence of the state:
+//
+//       Lam_T = 0,   Lam_t = dL/dS_t = alpha_t Lam_{t+1} + u_t x_t^T
+//       dx_t     = (W_0 + S_t)^T u_t - eta_t Lam_{t+1}^T g_t
+//       dg_t     = -eta_t Lam_{t+1} x_t
+//       deta_t   = -g_t . (Lam_{t+1} x_t)
+//       dalpha_t = <Lam_{t+1}, S_t>_F
+//       dW_0     = sum over b and t of u_t x_t^T      (W_0 is one matrix per head)
+//
+// Everything is materialised token by token in double (or complex<double> for
+// the complex-step derivative checks); there is no chunking, no blocking and
+// no reordering beyond this serial definition. OpenMP is used only across the
+// independent (b, h) pairs; the token loop of each pair is serial.
+//
+// Layouts (row-major, contiguous):
+//   x, dx [B,H,T,d_in]   g, y, dy, dg [B,H,T,d_out]   eta, alpha, deta, dalpha [B,H,T]
+//   W0, dW0 [H,d_out,d_in]   (dW0 is summed over b in a fixed order b = 0..B-1)
+
+#include <complex>
+#include <cstddef>
+#include <cstdint>
+#include <cstring>
+#include <vector>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+namespace {
+
+using cplx = std::complex<double>;
+
+inline size_t at3(int b, int h, int t, int H, int T) {
+  return ((size_t)b * H + h) * (size_t)T + t;
+}
+
+// S <- alpha S - eta g x^T
+template <class R>
+void state_step(int din, int dout, R* S, R alpha, R eta, const R* g, const R* x) {
+  for (int n = 0; n < dout; ++n)
+    for (int k = 0; k < din; ++k)
+      S[(size_t)n * din + k] = alpha * S[(size_t)n * din + k] - eta * g[n] * x[k];
+}
+
+// Forward of one (b,h) scan. S_work holds d_out*d_in scalars. If S_traj is
+// non-null it receives S_0 .. S_T ((T+1)*d_out*d_in scalars).
+template <class R>
+void fwd_head(int T, int din, int dout, const R* x, const R* g, const R* eta,
+              const R* alpha, const R* W0, R* y, R* S_work, R* S_traj) {
+  const size_t dd = (size_t)din * dout;
+  for (size_t e = 0; e < dd; ++e) S_work[e] = R(0);
+  if (S_traj) std::memcpy(S_traj, S_work, dd * sizeof(R));
+  for (int t = 0; t < T; ++t) {
+    const R* xt = x + (size_t)t * din;
+    for (int n = 0; n < dout; ++n) {
+      R acc(0);
+      for (int k = 0; k < din; ++k)
+        acc += (W0[(size_t)n * din + k] + S_work[(size_t)n * din + k]) * xt[k];
+      y[(size_t)t * dout + n] = acc;
+    }
+    state_step(din, dout, S_work, alpha[t], eta[t], g + (size_t)t * dout, xt);
+    if (S_traj) std::memcpy(S_traj + (size_t)(t + 1) * dd, S_work, dd * sizeof(R));
+  }
+}
+
+// Backward of one (b,h) scan. S_t is needed in reverse order; the forward
+// sweep stores S at every `ckpt`-th token and each segment is re-run forward
+// from its checkpoint before it is walked backwards. dW0p receives this pair's
+// sum_t u_t x_t^T. `mutate` = 1 replaces (W_0 + S_t)^T by W_0^T in dx: the
+// negative control of the "synthetic test" section (persistent instead of
+// adapted weight in the backward reconstruction), used only by tests.
+void bwd_head(int T, int din, int dout, const double* x, const double* g,
+              const double* eta, const double* alpha, const double* W0,
+              const double* u, double* dx, double* dg, double* deta,
+              double* dalpha, double* dW0p, int ckpt, int mutate) {
+  const size_t dd = (size_t)din * dout;
+  if (ckpt < 1) ckpt = 1;
+  const int nseg = (T + ckpt - 1) / ckpt;
+  std::vector<double> ck((size_t)nseg * dd, 0.0);
+  std::vector<double> S(dd, 0.0);
+  for (int t = 0; t < T; ++t) {
+    if (t % ckpt == 0) std::memcpy(&ck[(size_t)(t / ckpt) * dd], S.data(), dd * sizeof(double));
+    state_step(din, dout, S.data(), alpha[t], eta[t], g + (size_t)t * dout, x + (size_t)t * din);
+  }
+  std::vector<double> seg((size_t)ckpt * dd);
+  std::vector<double> Lam(dd, 0.0), r(dout);
+  for (size_t e = 0; e < dd; ++e) dW0p[e] = 0.0;
+  for (int s = nseg - 1; s >= 0; --s) {
+    const int t0 = s * ckpt, t1 = (t0 + ckpt < T) ? t0 + ckpt : T;
+    std::memcpy(S.data(), &ck[(size_t)s * dd], dd * sizeof(double));
+    for (int t = t0; t < t1; ++t) {
+      std::memcpy(&seg[(size_t)(t - t0) * dd], S.data(), dd * sizeof(double));
+      state_step(din, dout, S.data(), alpha[t], eta[t], g + (size_t)t * dout, x + (size_t)t * din);
+    }
+    for (int t = t1 - 1; t >= t0; --t) {
+      const double* St = &seg[(size_t)(t - t0) * dd];  // S_t
+      const double* xt = x + (size_t)t * din;
+      const double* gt = g + (size_t)t * dout;
+      const double* ut = u + (size_t)t * dout;
+      // Lam currently holds Lam_{t+1}.
+      for (int n = 0; n < dout; ++n) {
+        double acc = 0.0;
+        for (int k = 0; k < din; ++k) acc += Lam[(size_t)n * din + k] * xt[k];
+        r[n] = acc;
+      }
+      double ge = 0.0;
+      for (int n = 0; n < dout; ++n) {
+        dg[(size_t)t * dout + n] = -eta[t] * r[n];
+        ge += gt[n] * r[n];
+      }
+      deta[t] = -ge;
+      double ip = 0.0;
+      for (size_t e = 0; e < dd; ++e) ip += Lam[e] * St[e];
+      dalpha[t] = ip;
+      for (int k = 0; k < din; ++k) {
+        double acc = 0.0;
+        for (int n = 0; n < dout; ++n) {
+          const double w = mutate ? W0[(size_t)n * din + k]
+                                  : W0[(size_t)n * din + k] + St[(size_t)n * din + k];
+          acc += w * ut[n] - eta[t] * Lam[(size_t)n * din + k] * gt[n];
+        }
+        dx[(size_t)t * din + k] = acc;
+      }
+      for (int n = 0; n < dout; ++n)
+        for (int k = 0; k < din; ++k) {
+          dW0p[(size_t)n * din + k] += ut[n] * xt[k];
+          Lam[(size_t)n * din + k] = alpha[t] * Lam[(size_t)n * din + k] + ut[n] * xt[k];
+        }
+    }
+  }
+}
+
+// Serial online learner with inner loss 0.5 ||W x_t - v_t||^2 (the learner
+// GradLev is meant to recover; "The predictor is constrained by the learner it
+// is supposed to reproduce"): y_t = W x_t, g*_t = y_t - v_t, then the same
+// centred update W <- W_0 + alpha_t (W - W_0) - eta_t g*_t x_t^T.
+template <class R>
+void serial_head(int T, int din, int dout, const R* x, const R* v, const R* eta,
+                 const R* alpha, const R* W0, R* y, R* gstar) {
+  const size_t dd = (size_t)din * dout;
+  std::vector<R> W(W0, W0 + dd);
+  for (int t = 0; t < T; ++t) {
+    const R* xt = x + (size_t)t * din;
+    for (int n = 0; n < dout; ++n) {
+      R acc(0);
+      for (int k = 0; k < din; ++k) acc += W[(size_t)n * din + k] * xt[k];
+      y[(size_t)t * dout + n] = acc;
+      gstar[(size_t)t * dout + n] = acc - v[(size_t)t * dout + n];
+    }
+    for (int n = 0; n < dout; ++n)
+      for (int k = 0; k < din; ++k) {
+        const size_t e = (size_t)n * din + k;
+        W[e] = W0[e] + alpha[t] * (W[e] - W0[e]) - eta[t] * gstar[(size_t)t * dout + n] * xt[k];
+      }
+  }
+}
+
+inline int pick_threads(int nthreads) {
+#ifdef _OPENMP
+  return nthreads > 0 ? nthreads : omp_get_max_threads();
+#else
+  (void)nthreads;
+  return 1;
+#endif
+}
+
+template <class R>
+void fwd_all(int B, int H, int T, int din, int dout, const R* x, const R* g, const R* eta,
+             const R* alpha, const R* W0, R* y, int nthreads) {
+  const int nt = pick_threads(nthreads);
+  const size_t dd = (size_t)din * dout;
+#pragma omp parallel num_threads(nt)
+  {
+    std::vector<R> S(dd);
+#pragma omp for schedule(dynamic, 1)
+    for (int bh = 0; bh < B * H; ++bh) {
+      const int b = bh / H, h = bh % H;
+      const size_t o = at3(b, h, 0, H, T);
+      fwd_head<R>(T, din, dout, x + o * din, g + o * dout, eta + o, alpha + o,
+                  W0 + (size_t)h * dd, y + o * dout, S.data(), nullptr);
+    }
+  }
+}
+
+template <class R>
+void serial_all(int B, int H, int T, int din, int dout, const R* x, const R* v, const R* eta,
+                const R* alpha, const R* W0, R* y, R* gstar, int nthreads) {
+  const int nt = pick_threads(nthreads);
+  const size_t dd = (size_t)din * dout;
+#pragma omp parallel for num_threads(nt) schedule(dynamic, 1)
+  for (int bh = 0; bh < B * H; ++bh) {
+    const int b = bh / H, h = bh % H;
+    const size_t o = at3(b, h, 0, H, T);
+    serial_head<R>(T, din, dout, x + o * din, v + o * dout, eta + o, alpha + o,
+                   W0 + (size_t)h * dd, y + o * dout, gstar + o * dout);
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+// y = forward scan (see file header). nthreads <= 0: OpenMP default.
+void oracle_fwd_f64(int B, int H, int T, int din, int dout, const double* x, const double* g,
+                    const double* eta, const double* alpha, const double* W0, double* y,
+                    int nthreads) {
+  fwd_all<double>(B, H, T, din, dout, x, g, eta, alpha, W0, y, nthreads);
+}
+
+// Same in complex arithmetic (arrays are interleaved re,im pairs). Used for
+// complex-step derivatives: Im f(a + i h v) / h = <df/da, v> + O(h^2).
+void oracle_fwd_c128(int B, int H, int T, int din, int dout, const double* x, const double* g,
+                     const double* eta, const double* alpha, const double* W0, double* y,
+                     int nthreads) {
+  fwd_all<cplx>(B, H, T, din, dout, reinterpret_cast<const cplx*>(x),
+                reinterpret_cast<const cplx*>(g), reinterpret_cast<const cplx*>(eta),
+                reinterpret_cast<const cplx*>(alpha), reinterpret_cast<const cplx*>(W0),
+                reinterpret_cast<cplx*>(y), nthreads);
+}
+
+// Whole state trajectory S_0..S_T of ONE scan (B = H = 1), for small tests.
+void oracle_states_f64(int T, int din, int dout, const double* x, const double* g,
+                       const double* eta, const double* alpha, const double* W0, double* y,
+                       double* S_traj) {
+  std::vector<double> S((size_t)din * dout);
+  fwd_head<double>(T, din, dout, x, g, eta, alpha, W0, y, S.data(), S_traj);
+}
+
+// Reverse scan (see file header). ckpt: checkpoint interval of the state
+// recompute (any value >= 1 gives the same result up to nothing: the recompute
+// is the same serial arithmetic). flags bit 0: negative-control mutation.
+void oracle_bwd_f64(int B, int H, int T, int din, int dout, const double* x, const double* g,
+                    const double* eta, const double* alpha, const double* W0, const double* dy,
+                    double* dx, double* dg, double* deta, double* dalpha, double* dW0,
+                    int ckpt, int flags, int nthreads) {
+  const int nt = pick_threads(nthreads);
+  const size_t dd = (size_t)din * dout;
+  std::vector<double> part((size_t)B * H * dd);
+#pragma omp parallel for num_threads(nt) schedule(dynamic, 1)
+  for (int bh = 0; bh < B * H; ++bh) {
+    const int b = bh / H, h = bh % H;
+    const size_t o = at3(b, h, 0, H, T);
+    bwd_head(T, din, dout, x + o * din, g + o * dout, eta + o, alpha + o, W0 + (size_t)h * dd,
+             dy + o * dout, dx + o * din, dg + o * dout, deta + o, dalpha + o,
+             &part[(size_t)bh * dd], ckpt, flags & 1);
+  }
+  for (int h = 0; h < H; ++h) {
+    double* out = dW0 + (size_t)h * dd;
+    for (size_t e = 0; e < dd; ++e) out[e] = 0.0;
+    for (int b = 0; b < B; ++b) {
+      const double* p = &part[((size_t)b * H + h) * dd];
+      for (size_t e = 0; e < dd; ++e) out[e] += p[e];
+    }
+  }
+}
+
+// Serial online learner (inner loss 0.5||W x - v||^2): outputs y and the true
+// serial costates g* = y - v.
+void oracle_serial_f64(int B, int H, int T, int din, int dout, const double* x, const double* v,
+                       const double* eta, const double* alpha, const double* W0, double* y,
+                       double* gstar, int nthreads) {
+  serial_all<double>(B, H, T, din, dout, x, v, eta, alpha, W0, y, gstar, nthreads);
+}
+
+void oracle_serial_c128(int B, int H, int T, int din, int dout, const double* x, const double* v,
+                        const double* eta, const double* alpha, const double* W0, double* y,
+                        double* gstar, int nthreads) {
+  serial_all<cplx>(B, H, T, din, dout, reinterpret_cast<const cplx*>(x),
+                   reinterpret_cast<const cplx*>(v), reinterpret_cast<const cplx*>(eta),
+                   reinterpret_cast<const cplx*>(alpha), reinterpret_cast<const cplx*>(W0),
+                   reinterpret_cast<cplx*>(y), reinterpret_cast<cplx*>(gstar), nthreads);
+}
+
+int oracle_max_threads(void) { return pick_threads(0); }
+
+}  // extern "C"

@@ -1,0 +1,300 @@
+"""Pins of the float64 oracle against facts that do not come from the oracle.
+
+Each test checks the oracle (oracle/gradlev_oracle.cpp) against an
+independent statement of what the GradLev scan must compute:
+
+* a hand-worked scalar example (tests/golden/scalar_T3.json);
+* the closed form of the state as a discounted sum of earlier rank-one
+  updates (Cognaptus, "Parallelize the Training, Keep the Learning Serial",
+  section "Once the gradient signals are known, the weight trajectory becomes
+  parallelizable"), evaluated by brute force on tiny inputs;
+* special cases that reduce to dense matrix products (alpha = 1 is strictly
+  causal linear attention, eta = 0 is the static layer, alpha = 0 keeps only
+  the previous token, T = 1);
+* exact recovery of the serial online learner when the true serial costates
+  are supplied (same page, sections "The predictor is constrained by the
+  learner it is supposed to reproduce" and "The synthetic test checks the
+  mechanism, not model quality"), including the learner's outer gradients
+  through the fixed-point adjoint;
+* derivative checks of every backward output: exact dot-product tests where
+  the output is affine in the argument, central differences where it is
+  quadratic (x), complex-step for the polynomial dependence on alpha;
+* the negative control of the synthetic-test section: using the persistent
+  weight instead of the adapted one in the backward must break the
+  gradients while leaving the forward unchanged.
+"""
+
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from token_weight_scans_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def rel(a, b):
+    a = np.asarray(a)
+    b = np.asarray(b)
+    den = max(np.max(np.abs(b)), 1e-300)
+    return float(np.max(np.abs(a - b)) / den)
+
+
+def tiny(B=2, H=2, T=12, d_in=5, d_out=4, seed=7, alpha_mode="sigmoid", with_v=False):
+    d = inputs.draw(B, H, T, d_in, d_out, dtype="f32", alpha_mode=alpha_mode, seed=seed,
+                    with_v=with_v)
+    return {k: v.astype(np.float64) for k, v in d.items()}
+
+
+# --------------------------------------------------------------------------- golden
+
+
+def test_golden_scalar_example():
+    gd = json.load(open(os.path.join(GOLDEN, "scalar_T3.json")))
+    i, e = gd["inputs"], gd["expected"]
+    x = np.array(i["x"]).reshape(1, 1, 3, 1)
+    g = np.array(i["g"]).reshape(1, 1, 3, 1)
+    eta = np.array(i["eta"]).reshape(1, 1, 3)
+    alpha = np.array(i["alpha"]).reshape(1, 1, 3)
+    W0 = np.array([[[i["W0"]]]])
+    dy = np.array(i["dy"]).reshape(1, 1, 3, 1)
+    y = oracle.fwd(x, g, eta, alpha, W0)
+    assert np.array_equal(y.ravel(), np.array(e["y"]))
+    o = oracle.bwd(x, g, eta, alpha, W0, dy, ckpt=2)
+    for k in ("dx", "dg", "deta", "dalpha"):
+        assert np.array_equal(o[k].ravel(), np.array(e[k])), k
+    assert o["dW0"].ravel()[0] == e["dW0"]
+
+
+# --------------------------------------------------------------------------- closed form
+
+
+def closed_form(x, g, eta, alpha, W0):
+    """S_t = -sum_{s<t} (prod_{r=s+1}^{t-1} alpha_r) eta_s g_s x_s^T, y_t = (W0 + S_t) x_t."""
+    T, din = x.shape
+    dout = g.shape[1]
+    y = np.zeros((T, dout))
+    S = np.zeros((T + 1, dout, din))
+    for t in range(T + 1):
+        acc = np.zeros((dout, din))
+        for s in range(t):
+            p = 1.0
+            for r in range(s + 1, t):
+                p *= alpha[r]
+            acc -= p * eta[s] * np.outer(g[s], x[s])
+        S[t] = acc
+        if t < T:
+            y[t] = (W0 + acc) @ x[t]
+    return y, S
+
+
+@pytest.mark.parametrize("alpha_mode", ["sigmoid", "log_uniform"])
+def test_closed_form_bruteforce(alpha_mode):
+    d = tiny(alpha_mode=alpha_mode)
+    y = oracle.fwd(d["x"], d["g"], d["eta"], d["alpha"], d["W0"])
+    B, H = d["x"].shape[:2]
+    for b in range(B):
+        for h in range(H):
+            yc, Sc = closed_form(d["x"][b, h], d["g"][b, h], d["eta"][b, h], d["alpha"][b, h],
+                                 d["W0"][h])
+            assert rel(y[b, h], yc) < 1e-13
+            y1, S1 = oracle.states(d["x"][b, h], d["g"][b, h], d["eta"][b, h],
+                                   d["alpha"][b, h], d["W0"][h])
+            assert rel(S1, Sc) < 1e-13
+            assert rel(y1, yc) < 1e-13
+
+
+def test_closed_form_random_gates_wide_range():
+    # gates spanning [0, 1] including exact zeros and ones
+    rng = np.random.default_rng(3)
+    T, din, dout = 15, 3, 6
+    x = rng.standard_normal((T, din))
+    g = rng.standard_normal((T, dout))
+    eta = rng.uniform(0, 1, T)
+    alpha = rng.choice([0.0, 1.0, 0.3, 0.99], T)
+    W0 = rng.standard_normal((dout, din))
+    yc, Sc = closed_form(x, g, eta, alpha, W0)
+    y1, S1 = oracle.states(x, g, eta, alpha, W0)
+    assert rel(y1, yc) < 1e-13 and rel(S1, Sc) < 1e-13
+
+
+# --------------------------------------------------------------------------- special cases
+
+
+def test_alpha_one_is_causal_linear_attention():
+    d = tiny(T=20)
+    d["alpha"][:] = 1.0
+    y = oracle.fwd(d["x"], d["g"], d["eta"], d["alpha"], d["W0"])
+    for b in range(2):
+        for h in range(2):
+            X, G, e = d["x"][b, h], d["g"][b, h], d["eta"][b, h]
+            ref = X @ d["W0"][h].T - np.tril(X @ X.T, -1) @ (e[:, None] * G)
+            assert rel(y[b, h], ref) < 1e-13
+
+
+def test_eta_zero_is_static_layer():
+    d = tiny()
+    d["eta"][:] = 0.0
+    y = oracle.fwd(d["x"], d["g"], d["eta"], d["alpha"], d["W0"])
+    ref = np.einsum("bhtk,hnk->bhtn", d["x"], d["W0"])
+    assert rel(y, ref) < 1e-14
+
+
+def test_alpha_zero_keeps_previous_token_only():
+    d = tiny()
+    d["alpha"][:] = 0.0
+    y = oracle.fwd(d["x"], d["g"], d["eta"], d["alpha"], d["W0"])
+    X, G, e = d["x"], d["g"], d["eta"]
+    ref = np.einsum("bhtk,hnk->bhtn", X, d["W0"])
+    dots = np.einsum("bhtk,bhtk->bht", X[:, :, 1:], X[:, :, :-1])
+    ref[:, :, 1:] -= (e[:, :, :-1] * dots)[..., None] * G[:, :, :-1]
+    assert rel(y, ref) < 1e-14
+
+
+def test_single_token():
+    d = tiny(T=1)
+    y = oracle.fwd(d["x"], d["g"], d["eta"], d["alpha"], d["W0"])
+    ref = np.einsum("bhtk,hnk->bhtn", d["x"], d["W0"])
+    assert np.array_equal(y, ref) or rel(y, ref) < 1e-15
+    o = oracle.bwd(d["x"], d["g"], d["eta"], d["alpha"], d["W0"], d["dy"])
+    assert np.all(o["dg"] == 0) and np.all(o["deta"] == 0) and np.all(o["dalpha"] == 0)
+    assert rel(o["dx"], np.einsum("bhtn,hnk->bhtk", d["dy"], d["W0"])) < 1e-14
+
+
+# --------------------------------------------------------------------------- exact recovery
+
+
+def test_exact_recovery_of_serial_learner():
+    d = tiny(T=40, d_in=6, d_out=5, with_v=True)
+    ys, gs = oracle.serial(d["x"], d["v"], d["eta"], d["alpha"], d["W0"])
+    y = oracle.fwd(d["x"], gs, d["eta"], d["alpha"], d["W0"])
+    assert rel(y, ys) < 1e-12
+    # the costates the scan's outputs imply equal the ones that were supplied
+    assert rel(y - d["v"], gs) < 1e-12
+
+
+def _scan_outer_grads(d, gs, u, mutate=False):
+    """Outer gradient of L = sum u.y of the serial learner, through the scan and the
+    fixed point g = y - v: nu = bwd(u + nu).dg iterated T+1 times (exact, since dg_t
+    only depends on upstream at later tokens)."""
+    T = d["x"].shape[2]
+    nu = np.zeros_like(u)
+    for _ in range(T + 1):
+        nu = oracle.bwd(d["x"], gs, d["eta"], d["alpha"], d["W0"], u + nu, mutate=mutate)["dg"]
+    o = oracle.bwd(d["x"], gs, d["eta"], d["alpha"], d["W0"], u + nu, mutate=mutate)
+    return dict(W0=o["dW0"], x=o["dx"], v=-nu, eta=o["deta"], alpha=o["dalpha"])
+
+
+def _serial_outer_grads(d, u, h=1e-30):
+    """Same gradient by complex-step through the serial learner, one entry at a time."""
+    out = {}
+    for name in ("W0", "x", "v", "eta", "alpha"):
+        base = d[name]
+        gr = np.zeros_like(base)
+        for idx in np.ndindex(base.shape):
+            args = {k: d[k].astype(np.complex128) for k in ("x", "v", "eta", "alpha", "W0")}
+            args[name][idx] += 1j * h
+            y, _ = oracle.serial(args["x"], args["v"], args["eta"], args["alpha"], args["W0"])
+            gr[idx] = np.sum(y * u).imag / h
+        out[name] = gr
+    return out
+
+
+def test_exact_recovery_outer_gradients():
+    d = tiny(B=2, H=1, T=7, d_in=3, d_out=2, with_v=True, seed=11)
+    u = d["dy"]
+    _, gs = oracle.serial(d["x"], d["v"], d["eta"], d["alpha"], d["W0"])
+    scan = _scan_outer_grads(d, gs, u)
+    ref = _serial_outer_grads(d, u)
+    for k in ref:
+        assert rel(scan[k], ref[k]) < 1e-12, k
+
+
+def test_negative_control_persistent_weight_in_backward():
+    """Persistent W0^T in place of the adapted weight in the backward: the forward is
+    untouched (it does not read the flag) but the gradients are far off."""
+    d = tiny(B=2, H=1, T=7, d_in=3, d_out=2, with_v=True, seed=11)
+    u = d["dy"]
+    _, gs = oracle.serial(d["x"], d["v"], d["eta"], d["alpha"], d["W0"])
+    ref = _serial_outer_grads(d, u)
+    good = _scan_outer_grads(d, gs, u)
+    bad = _scan_outer_grads(d, gs, u, mutate=True)
+    assert rel(good["x"], ref["x"]) < 1e-12
+    assert rel(bad["x"], ref["x"]) > 1e-3
+    # and the plain derivative pin below catches the mutation too
+    o_bad = oracle.bwd(d["x"], d["g"], d["eta"], d["alpha"], d["W0"], u, mutate=True)
+    fd = _fd_grad(d, "x", u)
+    assert rel(o_bad["dx"], fd) > 1e-3
+
+
+# --------------------------------------------------------------------------- derivatives
+
+
+def _L(d, u, **over):
+    a = {k: over.get(k, d[k]) for k in ("x", "g", "eta", "alpha", "W0")}
+    y = oracle.fwd(a["x"], a["g"], a["eta"], a["alpha"], a["W0"])
+    return np.sum(y * u)
+
+
+def _fd_grad(d, name, u):
+    """Elementwise derivative of L = sum u.y: exact two-point differences for the
+    affine arguments (g, eta, W0), central differences for x (L is quadratic in x,
+    so they carry no truncation error), complex step for alpha."""
+    base = d[name]
+    gr = np.zeros_like(base)
+    for idx in np.ndindex(base.shape):
+        if name == "alpha":
+            a = base.astype(np.complex128)
+            h = 1e-30
+            a[idx] += 1j * h
+            gr[idx] = np.imag(_L(d, u, alpha=a)) / h
+        elif name == "x":
+            h = 1e-3
+            p = base.copy(); p[idx] += h
+            m = base.copy(); m[idx] -= h
+            gr[idx] = (_L(d, u, x=p) - _L(d, u, x=m)) / (2 * h)
+        else:
+            h = 1.0
+            p = base.copy(); p[idx] += h
+            gr[idx] = _L(d, u, **{name: p}) - _L(d, u)
+    return gr
+
+
+@pytest.mark.parametrize("alpha_mode", ["sigmoid", "log_uniform"])
+def test_backward_matches_derivatives(alpha_mode):
+    d = tiny(B=2, H=2, T=9, d_in=5, d_out=4, seed=5, alpha_mode=alpha_mode)
+    u = d["dy"]
+    o = oracle.bwd(d["x"], d["g"], d["eta"], d["alpha"], d["W0"], u, ckpt=4)
+    names = dict(x="dx", g="dg", eta="deta", alpha="dalpha", W0="dW0")
+    for p, k in names.items():
+        fd = _fd_grad(d, p, u)
+        tol = 1e-9 if p == "x" else 1e-12
+        assert rel(o[k], fd) < tol, (p, rel(o[k], fd))
+
+
+def test_backward_with_degenerate_gates():
+    """alpha in {0, 1} and eta = 0 entries: the derivative is still exact."""
+    d = tiny(B=1, H=1, T=10, d_in=3, d_out=4, seed=9)
+    d["alpha"][0, 0, ::3] = 0.0
+    d["alpha"][0, 0, 1::3] = 1.0
+    d["eta"][0, 0, 2] = 0.0
+    u = d["dy"]
+    o = oracle.bwd(d["x"], d["g"], d["eta"], d["alpha"], d["W0"], u, ckpt=3)
+    for p, k in dict(x="dx", g="dg", eta="deta", alpha="dalpha", W0="dW0").items():
+        fd = _fd_grad(d, p, u)
+        assert rel(o[k], fd) < (1e-9 if p == "x" else 1e-12), p
+
+
+def test_structural_zeros_and_checkpoint_invariance():
+    d = tiny(B=2, H=3, T=17, d_in=4, d_out=3, seed=2)
+    outs = [oracle.bwd(d["x"], d["g"], d["eta"], d["alpha"], d["W0"], d["dy"], ckpt=c)
+            for c in (1, 5, 64)]
+    o = outs[0]
+    assert np.all(o["dg"][:, :, -1] == 0) and np.all(o["deta"][:, :, -1] == 0)
+    assert np.all(o["dalpha"][:, :, -1] == 0) and np.all(o["dalpha"][:, :, 0] == 0)
+    for other in outs[1:]:
+        for k in o:
+            assert np.array_equal(o[k], other[k]), k
