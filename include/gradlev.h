@@ -1,0 +1,143 @@
+/*
+ * gradlev.h - C ABI of the GradLev scan library (libgradlev.so, CUDA, sm_100a).
+ *
+ * The library evaluates the token-parallel scans of one GradLev adaptive
+ * linear layer on the GPU: the forward scan that rebuilds the centred
+ * fast-weight trajectory from the layer inputs, the gates and the costates,
+ * and the reverse scan that backpropagates an upstream gradient through it.
+ *
+ * Definition (Cognaptus, "Parallelize the Training, Keep the Learning Serial",
+ * section "Once the gradient signals are known, the weight trajectory becomes
+ * parallelizable"; GradLev abstract, "GradLev: Token-Parallel Test-Time
+ * Training Via Costate Prediction"). Per batch row b and head h, with 0-based
+ * tokens t and S_t the deviation of the temporary weight from the persistent
+ * weight W0 BEFORE token t:
+ *
+ *     S_0 = 0
+ *     y_t     = (W0 + S_t) x_t
+ *     S_{t+1} = alpha_t S_t - eta_t g_t x_t^T
+ *
+ * x_t is the layer input, eta_t the step size, alpha_t the retention gate and
+ * g_t the costate (gradient of the token loss with respect to the layer
+ * output). In the page's 1-based notation this is D_t = alpha_t D_{t-1} -
+ * eta_t g_t x_t^T, y_t = (W0 + D_{t-1}) x_t. The backward returns the exact
+ * gradients of L = sum_t <dy_t, y_t> with respect to x, g, eta, alpha and W0
+ * (W0 is one matrix per head, shared by all batch rows; dW0 sums over b).
+ *
+ * Layouts: contiguous, row-major, device memory.
+ *     x, dx          [B, H, T, d_in]     dtype
+ *     g, y, dy, dg   [B, H, T, d_out]    dtype
+ *     eta, alpha, d_eta, d_alpha [B, H, T]   float32 (all dtypes)
+ *     W0, dW0        [H, d_out, d_in]    float32 (all dtypes)
+ * dtype GRADLEV_F32: float32 I/O, float32 arithmetic (CUDA cores).
+ * dtype GRADLEV_BF16: bfloat16 I/O, bf16 tensor-core operands with float32
+ *     accumulation and float32 state.
+ *
+ * Ownership: the caller allocates every buffer (inputs, outputs, optional
+ * checkpoint buffer, workspace). The library allocates no device memory per
+ * call and keeps no per-call global state. Calls are asynchronous on `stream`
+ * (a cudaStream_t passed as void*; NULL = the legacy default stream). Outputs
+ * are overwritten, never accumulated.
+ *
+ * Errors: argument errors (null pointers, non-positive sizes, unsupported
+ * shapes, too-small workspace) are detected on the host and returned before
+ * any launch; nothing is written. Launch failures return GRADLEV_ERR_CUDA.
+ * Preconditions that are not checked (they would need a device read):
+ * 0 <= alpha <= 1 and finite inputs.
+ */
+#ifndef GRADLEV_H_
+#define GRADLEV_H_
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define GRADLEV_API __attribute__((visibility("default")))
+#else
+#define GRADLEV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GRADLEV_F32 = 0,  /* x, g, y, dy, dx, dg are float32 */
+  GRADLEV_BF16 = 1  /* x, g, y, dy, dx, dg are bfloat16 */
+} gradlev_dtype;
+
+typedef enum {
+  GRADLEV_OK = 0,
+  GRADLEV_ERR_INVALID_ARG = 1,  /* null pointer, size <= 0, unknown dtype */
+  GRADLEV_ERR_UNSUPPORTED = 2,  /* valid but unsupported shape for this dtype */
+  GRADLEV_ERR_WORKSPACE = 3,    /* workspace smaller than gradlev_scan_workspace_bytes() */
+  GRADLEV_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
+  GRADLEV_ERR_TIMEOUT = 5       /* a bounded device-side wait gave up (gradlev_device_status) */
+} gradlev_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+GRADLEV_API const char* gradlev_status_string(gradlev_status s);
+
+/* Whether (B, H, T, d_in, d_out, dt) is supported: GRADLEV_OK, or
+ * GRADLEV_ERR_INVALID_ARG / GRADLEV_ERR_UNSUPPORTED without touching the GPU.
+ * Supported: B, H, T >= 1 with B*H*T < 2^31; d_in % 4 == 0, d_out % 8 == 0,
+ * 8 <= d_in, d_out and d_in * d_out <= 16384. */
+GRADLEV_API gradlev_status gradlev_scan_supported(int B, int H, int T, int d_in, int d_out,
+                                      gradlev_dtype dt);
+
+/* Bytes of device workspace the forward (is_bwd = 0) or backward (is_bwd = 1)
+ * call needs for this shape; 0 if the shape is unsupported. The workspace is
+ * scratch: its contents on entry do not matter; on return its first 16 bytes
+ * hold the device status word read by gradlev_device_status() and the rest is
+ * unspecified. It is never smaller than 256 bytes. */
+GRADLEV_API size_t gradlev_scan_workspace_bytes(int B, int H, int T, int d_in, int d_out,
+                                    gradlev_dtype dt, int is_bwd);
+
+/* Bytes of the optional state-checkpoint buffer that gradlev_scan_fwd can fill
+ * and gradlev_scan_bwd can consume for the same shape and dtype; 0 if
+ * unsupported. Its contents are implementation-defined (the float32 scan state
+ * at fixed token intervals) and valid only for the inputs of the forward call
+ * that wrote them. */
+GRADLEV_API size_t gradlev_scan_ckpt_bytes(int B, int H, int T, int d_in, int d_out, gradlev_dtype dt);
+
+/* Forward scan: y_t = (W0 + S_t) x_t for every (b, h, t).
+ *   x [B,H,T,d_in], g [B,H,T,d_out] (dtype); eta, alpha [B,H,T] float32;
+ *   W0 [H,d_out,d_in] float32; y [B,H,T,d_out] (dtype) is written.
+ *   ckpt: NULL, or gradlev_scan_ckpt_bytes() bytes that receive the state
+ *   checkpoints for a later gradlev_scan_bwd on the same inputs.
+ *   workspace: at least gradlev_scan_workspace_bytes(..., 0) bytes. */
+GRADLEV_API gradlev_status gradlev_scan_fwd(int B, int H, int T, int d_in, int d_out, gradlev_dtype dt,
+                                const void* x, const void* g, const float* eta,
+                                const float* alpha, const float* W0, void* y, void* ckpt,
+                                void* workspace, size_t ws_bytes, void* stream);
+
+/* Reverse scan. With Lam_T = 0 and Lam_t = alpha_t Lam_{t+1} + dy_t x_t^T:
+ *   dx_t      = (W0 + S_t)^T dy_t - eta_t Lam_{t+1}^T g_t      [B,H,T,d_in]  (dtype)
+ *   dg_t      = -eta_t Lam_{t+1} x_t                            [B,H,T,d_out] (dtype)
+ *   d_eta_t   = -g_t . (Lam_{t+1} x_t)                          [B,H,T] float32
+ *   d_alpha_t = <Lam_{t+1}, S_t>_F                              [B,H,T] float32
+ *   dW0       = sum_{b,t} dy_t x_t^T                            [H,d_out,d_in] float32
+ *   ckpt: NULL (the call recomputes the states itself, in the workspace), or the
+ *   buffer a gradlev_scan_fwd call on the same inputs filled.
+ *   workspace: at least gradlev_scan_workspace_bytes(..., 1) bytes. */
+GRADLEV_API gradlev_status gradlev_scan_bwd(int B, int H, int T, int d_in, int d_out, gradlev_dtype dt,
+                                const void* x, const void* g, const float* eta,
+                                const float* alpha, const float* W0, const void* dy,
+                                void* dx, void* dg, float* d_eta, float* d_alpha, float* dW0,
+                                const void* ckpt, void* workspace, size_t ws_bytes,
+                                void* stream);
+
+/* Device status of the last call that used `workspace`: synchronises `stream`
+ * and reads the status word the kernels leave at the start of the workspace.
+ * GRADLEV_OK, GRADLEV_ERR_TIMEOUT if a bounded device-side wait gave up (the
+ * outputs of that call are then unspecified), or GRADLEV_ERR_CUDA. */
+GRADLEV_API gradlev_status gradlev_device_status(const void* workspace, void* stream);
+
+/* Number of kernels the last successful fwd / bwd call on this host thread
+ * launched (for launch accounting by benchmarks). */
+GRADLEV_API int gradlev_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GRADLEV_H_ */

@@ -1,0 +1,104 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every
+entry point include/gradlev.h declares, and rejects bad arguments before any launch."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import token_weight_scans_b200 as tw
+from token_weight_scans_b200 import build as tw_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gradlev.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    tw_build.build()
+    return tw.lib()
+
+
+def declared_entry_points():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"GRADLEV_API\s+[\w\s\*]+?\b(gradlev_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_entry_points()
+    for n in ("gradlev_scan_fwd", "gradlev_scan_bwd", "gradlev_scan_workspace_bytes",
+              "gradlev_status_string", "gradlev_scan_supported", "gradlev_scan_ckpt_bytes",
+              "gradlev_device_status", "gradlev_last_launch_count"):
+        assert n in names, n
+
+
+def test_library_exports_every_declared_symbol(L):
+    for n in declared_entry_points():
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    assert tw.gradlev_status_string(0) == "GRADLEV_OK"
+    assert tw.gradlev_status_string(3) == "GRADLEV_ERR_WORKSPACE"
+    assert tw.gradlev_status_string(99) == "GRADLEV_UNKNOWN_STATUS"
+
+
+@pytest.mark.parametrize("shape,dt,ok", [
+    ((1, 1, 256, 16, 16), 0, 0),
+    ((4, 8, 2048, 64, 64), 0, 0),
+    ((8, 16, 4096, 128, 128), 1, 0),
+    ((1, 1, 1, 8, 8), 1, 0),
+    ((0, 1, 4, 16, 16), 0, 1),
+    ((1, 1, 4, 16, 16), 7, 1),
+    ((1, 1, 4, 6, 16), 0, 2),
+    ((1, 1, 4, 16, 12), 0, 2),
+    ((1, 1, 4, 256, 256), 0, 2),
+])
+def test_supported_shapes(L, shape, dt, ok):
+    assert tw.gradlev_scan_supported(*shape, dt) == ok
+    ws = tw.gradlev_scan_workspace_bytes(*shape, dt, 1)
+    assert (ws >= 256) == (ok == 0)
+
+
+def test_bwd_workspace_covers_partials_and_states(L):
+    B, H, T, di, do = 2, 3, 100, 16, 24
+    ws_f = tw.gradlev_scan_workspace_bytes(B, H, T, di, do, 0, 0)
+    ws_b = tw.gradlev_scan_workspace_bytes(B, H, T, di, do, 0, 1)
+    ck = tw.gradlev_scan_ckpt_bytes(B, H, T, di, do, 0)
+    assert ws_f >= 256
+    assert ws_b >= 256 + B * H * di * do * 4 + ck
+    assert ck >= B * H * di * do * 4
+
+
+def test_argument_errors_return_before_launch(L):
+    P = ctypes.c_void_p
+    fake = P(4096)  # never dereferenced: validation fails first
+    # null input
+    st = L.gradlev_scan_fwd(1, 1, 8, 16, 16, 0, P(0), fake, fake, fake, fake, fake, P(0), fake,
+                            1 << 20, P(0))
+    assert st == 1
+    # unsupported shape
+    st = L.gradlev_scan_fwd(1, 1, 8, 16, 12, 0, fake, fake, fake, fake, fake, fake, P(0), fake,
+                            1 << 20, P(0))
+    assert st == 2
+    # workspace too small
+    st = L.gradlev_scan_fwd(1, 1, 8, 16, 16, 0, fake, fake, fake, fake, fake, fake, P(0), fake,
+                            16, P(0))
+    assert st == 3
+    st = L.gradlev_scan_bwd(1, 1, 8, 16, 16, 0, fake, fake, fake, fake, fake, fake, fake, fake,
+                            fake, fake, fake, P(0), fake, 16, P(0))
+    assert st == 3
+    # misaligned pointer
+    st = L.gradlev_scan_bwd(1, 1, 8, 16, 16, 0, P(4098), fake, fake, fake, fake, fake, fake,
+                            fake, fake, fake, fake, P(0), fake, 1 << 30, P(0))
+    assert st == 1
+    assert L.gradlev_device_status(P(0), P(0)) == 1
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(tw, "_lib", None)
+    monkeypatch.setattr(tw, "LIB_PATH", str(tmp_path / "nope.so"))
+    with pytest.raises(tw.GradlevError):
+        tw.lib()

@@ -1,0 +1,210 @@
+"""GPU parity: the CUDA scans (through the C ABI) against the float64 oracle.
+
+Inputs come from the seeded generator (token_weight_scans_b200.inputs); the
+oracle consumes the dtype-rounded values upcast to float64. Error metric: per
+output tensor, max |gpu - oracle| / max |oracle|, with the bars of
+tests/helpers.TOL (fp32 path 1e-5, bf16 path 2e-2).
+
+Small and mid-size cases are compared element by element on every output;
+the full-size workloads are run in the bench's launch configuration and
+compared on sampled (b, h) scans that the oracle evaluates one by one (dW0 on
+a sampled head, summed over all batch rows).
+"""
+
+import numpy as np
+import pytest
+
+import oracle
+from token_weight_scans_b200 import inputs
+from tests.helpers import TOL, heads_slice, rel_err, to_device, to_numpy
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+OUTS = ("dx", "dg", "deta", "dalpha", "dW0")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from token_weight_scans_b200 import build
+    build.build()
+    import token_weight_scans_b200 as tw
+    tw.lib()
+    yield
+
+
+def run_gpu(d, dtype, bwd=True, use_ckpt=False):
+    import token_weight_scans_b200 as tw
+    t = to_device(d, dtype)
+    ck = None
+    if use_ckpt:
+        B, H, T, di = t["x"].shape
+        do = t["g"].shape[-1]
+        code = tw.BF16 if dtype == "bf16" else tw.F32
+        ck = torch.empty(tw.gradlev_scan_ckpt_bytes(B, H, T, di, do, code), dtype=torch.uint8,
+                         device="cuda")
+    y = tw.gradlev_scan_fwd(t["x"], t["g"], t["eta"], t["alpha"], t["W0"], ckpt=ck)
+    out = {"y": y}
+    if bwd:
+        out.update(tw.gradlev_scan_bwd(t["x"], t["g"], t["eta"], t["alpha"], t["W0"], t["dy"],
+                                       ckpt=ck))
+    torch.cuda.synchronize()
+    return {k: to_numpy(v) for k, v in out.items()}
+
+
+def run_oracle(d, bwd=True):
+    d64 = {k: v.astype(np.float64) for k, v in d.items()}
+    out = {"y": oracle.fwd(d64["x"], d64["g"], d64["eta"], d64["alpha"], d64["W0"])}
+    if bwd:
+        out.update(oracle.bwd(d64["x"], d64["g"], d64["eta"], d64["alpha"], d64["W0"], d64["dy"]))
+    return out
+
+
+def assert_close(gpu, ref, dtype, keys, ctx=""):
+    errs = {k: rel_err(gpu[k], ref[k]) for k in keys}
+    bad = {k: e for k, e in errs.items() if not e <= TOL[dtype]}
+    assert not bad, f"{ctx} errors {errs} exceed {TOL[dtype]}"
+    return errs
+
+
+# ----------------------------------------------------------------- full configs, small ones
+
+
+@pytest.mark.parametrize("idx", [0, 1])
+def test_small_configs_full_compare(idx):
+    cfg = inputs.CONFIGS[idx]
+    d = inputs.draw_config(cfg)
+    gpu = run_gpu(d, cfg.dtype)
+    ref = run_oracle(d)
+    assert_close(gpu, ref, cfg.dtype, ("y",) + OUTS, cfg.name)
+
+
+# ----------------------------------------------------------------- mid sizes, ragged tails
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("T", [1, 15, 31, 32, 33, 64, 257])
+def test_ragged_lengths(dtype, T):
+    d = inputs.draw(2, 2, T, 64, 32, dtype=dtype, alpha_mode="sigmoid", seed=100 + T)
+    gpu = run_gpu(d, dtype)
+    ref = run_oracle(d)
+    assert_close(gpu, ref, dtype, ("y",) + OUTS, f"T={T}")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_mid_size_several_chunks(dtype):
+    d = inputs.draw(2, 3, 300, 128, 128, dtype=dtype, alpha_mode="log_uniform", seed=5)
+    gpu = run_gpu(d, dtype)
+    ref = run_oracle(d)
+    assert_close(gpu, ref, dtype, ("y",) + OUTS, "B2H3T300d128")
+
+
+@pytest.mark.parametrize("shape", [(1, 2, 70, 8, 64), (2, 1, 45, 96, 16), (1, 1, 40, 128, 64)])
+def test_rectangular(shape):
+    B, H, T, di, do = shape
+    d = inputs.draw(B, H, T, di, do, dtype="f32", seed=sum(shape))
+    gpu = run_gpu(d, "f32")
+    ref = run_oracle(d)
+    assert_close(gpu, ref, "f32", ("y",) + OUTS, str(shape))
+
+
+def test_degenerate_gates():
+    """alpha in {0, 1}, eta = 0 tokens: the decay products are formed exactly."""
+    d = inputs.draw(2, 2, 100, 32, 32, dtype="f32", seed=77)
+    d["alpha"][..., ::7] = 0.0
+    d["alpha"][..., 3::7] = 1.0
+    d["eta"][..., 5::11] = 0.0
+    gpu = run_gpu(d, "f32")
+    ref = run_oracle(d)
+    assert_close(gpu, ref, "f32", ("y",) + OUTS, "degenerate gates")
+
+
+def test_fwd_checkpoints_feed_bwd():
+    d = inputs.draw(2, 2, 130, 64, 64, dtype="bf16", seed=8)
+    a = run_gpu(d, "bf16", use_ckpt=False)
+    b = run_gpu(d, "bf16", use_ckpt=True)
+    for k in ("y",) + OUTS:
+        assert np.array_equal(a[k], b[k]), k
+
+
+def test_deterministic():
+    d = inputs.draw(2, 2, 200, 64, 64, dtype="bf16", seed=9)
+    a = run_gpu(d, "bf16")
+    b = run_gpu(d, "bf16")
+    for k in a:
+        assert np.array_equal(a[k], b[k]), k
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_bit_exact_integer_inputs(dtype):
+    """Small-integer x, g, dy, W0, eta = 1/8, alpha = 1: every intermediate is exactly
+    representable, so the GPU result must equal the oracle bit for bit (indexing, layout,
+    tails and structural zeros)."""
+    rng = np.random.default_rng(1)
+    B, H, T, di, do = 2, 2, 45, 16, 8
+    d = {
+        "x": (rng.integers(-1, 2, (B, H, T, di)) * (rng.random((B, H, T, di)) < 0.15)),
+        "g": (rng.integers(-1, 2, (B, H, T, do)) * (rng.random((B, H, T, do)) < 0.3)),
+        "eta": np.full((B, H, T), 0.125),
+        "alpha": np.ones((B, H, T)),
+        "W0": rng.integers(-1, 2, (H, do, di)) * (rng.random((H, do, di)) < 0.2),
+        "dy": (rng.integers(-1, 2, (B, H, T, do)) * (rng.random((B, H, T, do)) < 0.3)),
+    }
+    d = {k: v.astype(np.float32) for k, v in d.items()}
+    ref = run_oracle(d)
+    for k, v in ref.items():  # the chosen inputs keep every value a small dyadic rational
+        assert np.all(np.abs(v) < 2 ** 12) and np.all(v * 64 == np.round(v * 64)), k
+        if k in ("y", "dx", "dg"):  # outputs stored in the I/O dtype
+            assert np.array_equal(inputs.round_bf16(v).astype(np.float64), v), k
+    gpu = run_gpu(d, dtype)
+    for k in ("y",) + OUTS:
+        assert np.array_equal(gpu[k], ref[k]), (k, rel_err(gpu[k], ref[k]))
+
+
+def test_one_hot_layout():
+    """A single nonzero input at (b, h, t, k) reaches exactly the outputs the definition says."""
+    B, H, T, di, do = 2, 3, 40, 16, 8
+    z = lambda *s: np.zeros(s, np.float32)
+    d = {"x": z(B, H, T, di), "g": z(B, H, T, do), "eta": np.full((B, H, T), 0.5, np.float32),
+         "alpha": np.ones((B, H, T), np.float32), "W0": z(H, do, di), "dy": z(B, H, T, do)}
+    b, h, t = 1, 2, 33
+    d["x"][b, h, t, 5] = 1.0
+    d["W0"][h, 3, 5] = 2.0
+    d["dy"][b, h, t, 3] = 1.0
+    gpu = run_gpu(d, "f32")
+    ref = run_oracle(d)
+    for k in ("y",) + OUTS:
+        assert np.array_equal(gpu[k], ref[k]), k
+    assert gpu["y"][b, h, t, 3] == 2.0 and np.count_nonzero(gpu["y"]) == 1
+    assert gpu["dx"][b, h, t, 5] == 2.0 and np.count_nonzero(gpu["dx"]) == 1
+    assert gpu["dW0"][h, 3, 5] == 1.0 and np.count_nonzero(gpu["dW0"]) == 1
+
+
+# ----------------------------------------------------------------- full-size, sampled
+
+
+SAMPLED = {2: [(0, 0), (7, 15), (3, 9)], 3: [(0, 0), (7, 15), (4, 6)], 4: [(0, 0), (0, 15)]}
+
+
+@pytest.mark.parametrize("idx", [2, 3, 4])
+def test_full_size_sampled_heads(idx):
+    import token_weight_scans_b200 as tw
+    cfg = inputs.CONFIGS[idx]
+    code = tw.BF16 if cfg.dtype == "bf16" else tw.F32
+    if tw.gradlev_scan_supported(cfg.B, cfg.H, cfg.T, cfg.d_in, cfg.d_out, code) != 0:
+        pytest.xfail(f"{cfg.name}: shape not supported by this build")
+    d = inputs.draw_config(cfg)
+    do_bwd = "bwd" in cfg.passes
+    gpu = run_gpu(d, cfg.dtype, bwd=do_bwd, use_ckpt=True)
+    keys = ("y",) + (("dx", "dg", "deta", "dalpha") if do_bwd else ())
+    for b, h in SAMPLED[idx]:
+        ref = run_oracle(heads_slice(d, b, h), bwd=do_bwd)
+        g1 = {k: gpu[k][b:b + 1, h:h + 1] for k in keys}
+        assert_close(g1, ref, cfg.dtype, keys, f"{cfg.name} (b={b},h={h})")
+    if do_bwd:
+        h = SAMPLED[idx][-1][1]
+        sub = {k: (v[:, h:h + 1] if k != "W0" else v[h:h + 1]) for k, v in d.items()}
+        ref = run_oracle(sub, bwd=True)
+        assert rel_err(gpu["dW0"][h:h + 1], ref["dW0"]) <= TOL[cfg.dtype]

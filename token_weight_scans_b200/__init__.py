@@ -1,0 +1,207 @@
+"""Python binding of libgradlev.so, the B200 GradLev scan library.
+
+Argument marshalling only: every step of the scans runs in the library's CUDA
+kernels. PyTorch provides device memory and the stream. The functions carry
+the names of the C entry points declared in ``include/gradlev.h``.
+
+If the shared library is missing or cannot be loaded, every call raises
+``GradlevError``; there is no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "GradlevError", "lib", "gradlev_status_string", "gradlev_scan_supported",
+    "gradlev_scan_workspace_bytes", "gradlev_scan_ckpt_bytes", "gradlev_scan_fwd",
+    "gradlev_scan_bwd", "gradlev_device_status", "gradlev_last_launch_count",
+    "F32", "BF16", "LIB_PATH",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgradlev.so")
+F32 = 0
+BF16 = 1
+
+_ENTRY_POINTS = (
+    "gradlev_status_string", "gradlev_scan_supported", "gradlev_scan_workspace_bytes",
+    "gradlev_scan_ckpt_bytes", "gradlev_scan_fwd", "gradlev_scan_bwd",
+    "gradlev_device_status", "gradlev_last_launch_count",
+)
+
+
+class GradlevError(RuntimeError):
+    """A C entry point returned a non-OK status, or the library is unavailable."""
+
+    def __init__(self, msg, status=None):
+        super().__init__(msg)
+        self.status = status
+
+
+_lib = None
+
+
+def lib():
+    """The loaded ctypes library (loads it on first use; raises GradlevError if absent)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise GradlevError(f"libgradlev.so not built ({LIB_PATH}); run "
+                           "`python -m token_weight_scans_b200.build`")
+    try:
+        L = ctypes.CDLL(LIB_PATH)
+    except OSError as e:  # pragma: no cover - depends on the box
+        raise GradlevError(f"cannot load {LIB_PATH}: {e}") from e
+    I, Z, P = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
+    L.gradlev_status_string.argtypes = [I]
+    L.gradlev_status_string.restype = ctypes.c_char_p
+    L.gradlev_scan_supported.argtypes = [I] * 6
+    L.gradlev_scan_supported.restype = I
+    L.gradlev_scan_workspace_bytes.argtypes = [I] * 7
+    L.gradlev_scan_workspace_bytes.restype = Z
+    L.gradlev_scan_ckpt_bytes.argtypes = [I] * 6
+    L.gradlev_scan_ckpt_bytes.restype = Z
+    L.gradlev_scan_fwd.argtypes = [I] * 6 + [P] * 8 + [Z, P]
+    L.gradlev_scan_fwd.restype = I
+    L.gradlev_scan_bwd.argtypes = [I] * 6 + [P] * 13 + [Z, P]
+    L.gradlev_scan_bwd.restype = I
+    L.gradlev_device_status.argtypes = [P, P]
+    L.gradlev_device_status.restype = I
+    L.gradlev_last_launch_count.argtypes = []
+    L.gradlev_last_launch_count.restype = I
+    _lib = L
+    return L
+
+
+def gradlev_status_string(status: int) -> str:
+    return lib().gradlev_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise GradlevError(f"{what}: {gradlev_status_string(status)}", status)
+
+
+def _dt_code(dtype) -> int:
+    import torch
+    if dtype == torch.float32:
+        return F32
+    if dtype == torch.bfloat16:
+        return BF16
+    raise GradlevError(f"unsupported I/O dtype {dtype}")
+
+
+def gradlev_scan_supported(B, H, T, d_in, d_out, dt) -> int:
+    return int(lib().gradlev_scan_supported(B, H, T, d_in, d_out, dt))
+
+
+def gradlev_scan_workspace_bytes(B, H, T, d_in, d_out, dt, is_bwd) -> int:
+    return int(lib().gradlev_scan_workspace_bytes(B, H, T, d_in, d_out, dt, int(is_bwd)))
+
+
+def gradlev_scan_ckpt_bytes(B, H, T, d_in, d_out, dt) -> int:
+    return int(lib().gradlev_scan_ckpt_bytes(B, H, T, d_in, d_out, dt))
+
+
+def gradlev_last_launch_count() -> int:
+    return int(lib().gradlev_last_launch_count())
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream_ptr(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check_tensor(name, t, shape, dtype, device):
+    if t.shape != tuple(shape):
+        raise GradlevError(f"{name}: shape {tuple(t.shape)} != {tuple(shape)}")
+    if t.dtype != dtype:
+        raise GradlevError(f"{name}: dtype {t.dtype} != {dtype}")
+    if t.device != device:
+        raise GradlevError(f"{name}: device {t.device} != {device}")
+    if not t.is_contiguous():
+        raise GradlevError(f"{name}: must be contiguous")
+
+
+def _workspace(nbytes, device, workspace):
+    import torch
+    if workspace is None:
+        return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    if workspace.numel() * workspace.element_size() < nbytes:
+        raise GradlevError(f"workspace too small: {workspace.numel()} < {nbytes}")
+    return workspace
+
+
+def _dims(x, g):
+    if x.dim() != 4 or g.dim() != 4:
+        raise GradlevError("x and g must be [B,H,T,d] tensors")
+    B, H, T, d_in = x.shape
+    d_out = g.shape[-1]
+    return B, H, T, d_in, d_out
+
+
+def gradlev_scan_fwd(x, g, eta, alpha, W0, *, y=None, ckpt=None, workspace=None, stream=None):
+    """Forward scan on the GPU. Returns y [B,H,T,d_out] (dtype of x)."""
+    import torch
+    B, H, T, d_in, d_out = _dims(x, g)
+    dev, dt = x.device, x.dtype
+    f32 = torch.float32
+    _check_tensor("g", g, (B, H, T, d_out), dt, dev)
+    _check_tensor("eta", eta, (B, H, T), f32, dev)
+    _check_tensor("alpha", alpha, (B, H, T), f32, dev)
+    _check_tensor("W0", W0, (H, d_out, d_in), f32, dev)
+    _check_tensor("x", x, (B, H, T, d_in), dt, dev)
+    code = _dt_code(dt)
+    _check(gradlev_scan_supported(B, H, T, d_in, d_out, code), "gradlev_scan_fwd")
+    if y is None:
+        y = torch.empty((B, H, T, d_out), dtype=dt, device=dev)
+    _check_tensor("y", y, (B, H, T, d_out), dt, dev)
+    nws = gradlev_scan_workspace_bytes(B, H, T, d_in, d_out, code, 0)
+    ws = _workspace(nws, dev, workspace)
+    st = lib().gradlev_scan_fwd(B, H, T, d_in, d_out, code, _ptr(x), _ptr(g), _ptr(eta),
+                                _ptr(alpha), _ptr(W0), _ptr(y), _ptr(ckpt), _ptr(ws),
+                                ws.numel() * ws.element_size(), _stream_ptr(stream))
+    _check(st, "gradlev_scan_fwd")
+    return y
+
+
+def gradlev_scan_bwd(x, g, eta, alpha, W0, dy, *, ckpt=None, workspace=None, stream=None,
+                     out=None):
+    """Reverse scan on the GPU. Returns dict dx, dg, deta, dalpha, dW0."""
+    import torch
+    B, H, T, d_in, d_out = _dims(x, g)
+    dev, dt = x.device, x.dtype
+    f32 = torch.float32
+    _check_tensor("x", x, (B, H, T, d_in), dt, dev)
+    _check_tensor("g", g, (B, H, T, d_out), dt, dev)
+    _check_tensor("dy", dy, (B, H, T, d_out), dt, dev)
+    _check_tensor("eta", eta, (B, H, T), f32, dev)
+    _check_tensor("alpha", alpha, (B, H, T), f32, dev)
+    _check_tensor("W0", W0, (H, d_out, d_in), f32, dev)
+    code = _dt_code(dt)
+    _check(gradlev_scan_supported(B, H, T, d_in, d_out, code), "gradlev_scan_bwd")
+    if out is None:
+        out = dict(dx=torch.empty_like(x), dg=torch.empty_like(g),
+                   deta=torch.empty((B, H, T), dtype=f32, device=dev),
+                   dalpha=torch.empty((B, H, T), dtype=f32, device=dev),
+                   dW0=torch.empty((H, d_out, d_in), dtype=f32, device=dev))
+    nws = gradlev_scan_workspace_bytes(B, H, T, d_in, d_out, code, 1)
+    ws = _workspace(nws, dev, workspace)
+    st = lib().gradlev_scan_bwd(B, H, T, d_in, d_out, code, _ptr(x), _ptr(g), _ptr(eta),
+                                _ptr(alpha), _ptr(W0), _ptr(dy), _ptr(out["dx"]),
+                                _ptr(out["dg"]), _ptr(out["deta"]), _ptr(out["dalpha"]),
+                                _ptr(out["dW0"]), _ptr(ckpt), _ptr(ws),
+                                ws.numel() * ws.element_size(), _stream_ptr(stream))
+    _check(st, "gradlev_scan_bwd")
+    return out
+
+
+def gradlev_device_status(workspace, stream=None) -> int:
+    return int(lib().gradlev_device_status(_ptr(workspace), _stream_ptr(stream)))

@@ -1,0 +1,143 @@
+// Host side of the C ABI declared in include/gradlev.h: argument validation,
+// workspace sizing and kernel dispatch. No device memory is allocated here.
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "gradlev.h"
+#include "scan_ffma.h"
+
+namespace gradlev {
+
+static thread_local int t_launches = 0;
+void count_launch() { ++t_launches; }
+
+static constexpr size_t kStatusBytes = 256;  // status word + alignment pad
+
+static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+static gradlev_status check_shape(int B, int H, int T, int din, int dout, gradlev_dtype dt) {
+  if (B <= 0 || H <= 0 || T <= 0 || din <= 0 || dout <= 0) return GRADLEV_ERR_INVALID_ARG;
+  if (dt != GRADLEV_F32 && dt != GRADLEV_BF16) return GRADLEV_ERR_INVALID_ARG;
+  if ((long long)B * H * T >= (1LL << 31)) return GRADLEV_ERR_UNSUPPORTED;
+  if (!ffma::shape_ok(din, dout)) return GRADLEV_ERR_UNSUPPORTED;
+  return GRADLEV_OK;
+}
+
+static bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+}  // namespace gradlev
+
+using namespace gradlev;
+
+extern "C" {
+
+const char* gradlev_status_string(gradlev_status s) {
+  switch (s) {
+    case GRADLEV_OK: return "GRADLEV_OK";
+    case GRADLEV_ERR_INVALID_ARG: return "GRADLEV_ERR_INVALID_ARG";
+    case GRADLEV_ERR_UNSUPPORTED: return "GRADLEV_ERR_UNSUPPORTED";
+    case GRADLEV_ERR_WORKSPACE: return "GRADLEV_ERR_WORKSPACE";
+    case GRADLEV_ERR_CUDA: return "GRADLEV_ERR_CUDA";
+    case GRADLEV_ERR_TIMEOUT: return "GRADLEV_ERR_TIMEOUT";
+  }
+  return "GRADLEV_UNKNOWN_STATUS";
+}
+
+gradlev_status gradlev_scan_supported(int B, int H, int T, int d_in, int d_out, gradlev_dtype dt) {
+  return check_shape(B, H, T, d_in, d_out, dt);
+}
+
+size_t gradlev_scan_ckpt_bytes(int B, int H, int T, int d_in, int d_out, gradlev_dtype dt) {
+  if (check_shape(B, H, T, d_in, d_out, dt) != GRADLEV_OK) return 0;
+  return ffma::ckpt_bytes(B, H, T, d_in, d_out);
+}
+
+size_t gradlev_scan_workspace_bytes(int B, int H, int T, int d_in, int d_out, gradlev_dtype dt,
+                                    int is_bwd) {
+  if (check_shape(B, H, T, d_in, d_out, dt) != GRADLEV_OK) return 0;
+  size_t ws = kStatusBytes;
+  if (is_bwd) {
+    ws += align_up(ffma::dW0_part_bytes(B, H, d_in, d_out), 256);
+    ws += align_up(ffma::ckpt_bytes(B, H, T, d_in, d_out), 256);
+  }
+  return ws;
+}
+
+gradlev_status gradlev_scan_fwd(int B, int H, int T, int d_in, int d_out, gradlev_dtype dt,
+                                const void* x, const void* g, const float* eta,
+                                const float* alpha, const float* W0, void* y, void* ckpt,
+                                void* workspace, size_t ws_bytes, void* stream) {
+  gradlev_status s = check_shape(B, H, T, d_in, d_out, dt);
+  if (s != GRADLEV_OK) return s;
+  if (!x || !g || !eta || !alpha || !W0 || !y || !workspace) return GRADLEV_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(g, 16) || !aligned(y, 16) || !aligned(W0, 16) ||
+      !aligned(eta, 4) || !aligned(alpha, 4) || (ckpt && !aligned(ckpt, 16)) ||
+      !aligned(workspace, 16))
+    return GRADLEV_ERR_INVALID_ARG;
+  if (ws_bytes < gradlev_scan_workspace_bytes(B, H, T, d_in, d_out, dt, 0))
+    return GRADLEV_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  t_launches = 0;
+  if (cudaMemsetAsync(workspace, 0, sizeof(DeviceStatus), st) != cudaSuccess)
+    return GRADLEV_ERR_CUDA;
+  ffma::FwdArgs a{B, H, T, d_in, d_out, x, g, eta, alpha, W0, y, static_cast<float*>(ckpt)};
+  if (ffma::launch_fwd(a, dt == GRADLEV_BF16, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
+  return GRADLEV_OK;
+}
+
+gradlev_status gradlev_scan_bwd(int B, int H, int T, int d_in, int d_out, gradlev_dtype dt,
+                                const void* x, const void* g, const float* eta,
+                                const float* alpha, const float* W0, const void* dy, void* dx,
+                                void* dg, float* d_eta, float* d_alpha, float* dW0,
+                                const void* ckpt, void* workspace, size_t ws_bytes,
+                                void* stream) {
+  gradlev_status s = check_shape(B, H, T, d_in, d_out, dt);
+  if (s != GRADLEV_OK) return s;
+  if (!x || !g || !eta || !alpha || !W0 || !dy || !dx || !dg || !d_eta || !d_alpha || !dW0 ||
+      !workspace)
+    return GRADLEV_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(g, 16) || !aligned(dy, 16) || !aligned(dx, 16) ||
+      !aligned(dg, 16) || !aligned(W0, 16) || !aligned(dW0, 16) || !aligned(eta, 4) ||
+      !aligned(alpha, 4) || !aligned(d_eta, 4) || !aligned(d_alpha, 4) ||
+      (ckpt && !aligned(ckpt, 16)) || !aligned(workspace, 16))
+    return GRADLEV_ERR_INVALID_ARG;
+  if (ws_bytes < gradlev_scan_workspace_bytes(B, H, T, d_in, d_out, dt, 1))
+    return GRADLEV_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  t_launches = 0;
+  char* wsb = static_cast<char*>(workspace);
+  float* dW0_part = reinterpret_cast<float*>(wsb + kStatusBytes);
+  float* own_ckpt = reinterpret_cast<float*>(
+      wsb + kStatusBytes + align_up(ffma::dW0_part_bytes(B, H, d_in, d_out), 256));
+  if (cudaMemsetAsync(workspace, 0, sizeof(DeviceStatus), st) != cudaSuccess)
+    return GRADLEV_ERR_CUDA;
+  const bool bf16 = dt == GRADLEV_BF16;
+  const float* states = static_cast<const float*>(ckpt);
+  if (!states) {
+    ffma::FwdArgs f{B, H, T, d_in, d_out, x, g, eta, alpha, W0, nullptr, own_ckpt};
+    if (ffma::launch_fwd(f, bf16, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
+    states = own_ckpt;
+  }
+  ffma::BwdArgs a{B, H, T, d_in, d_out, x, g, eta, alpha, W0, dy, dx, dg, d_eta, d_alpha, dW0,
+                  states, dW0_part};
+  if (ffma::launch_bwd(a, bf16, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
+  return GRADLEV_OK;
+}
+
+gradlev_status gradlev_device_status(const void* workspace, void* stream) {
+  if (!workspace) return GRADLEV_ERR_INVALID_ARG;
+  DeviceStatus h;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return GRADLEV_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return GRADLEV_ERR_CUDA;
+  if (h.code == 0) return GRADLEV_OK;
+  return h.code == GRADLEV_ERR_TIMEOUT ? GRADLEV_ERR_TIMEOUT : GRADLEV_ERR_CUDA;
+}
+
+int gradlev_last_launch_count(void) { return t_launches; }
+
+}  // extern "C"

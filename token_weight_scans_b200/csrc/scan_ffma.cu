@@ -1,0 +1,586 @@
+// CUDA-core (FFMA) chunkwise GradLev scans: the float32 path of the library.
+//
+// Per (b, h) scan one CTA walks the sequence in chunks of FC = 32 tokens and
+// keeps the d_out x d_in float32 state in shared memory. Within a chunk the
+// recurrence S_{t+1} = alpha_t S_t - eta_t g_t x_t^T (Cognaptus, "Parallelize
+// the Training, Keep the Learning Serial", section "Once the gradient signals
+// are known, the weight trajectory becomes parallelizable") is unrolled into
+// its discounted-sum form, so every token of the chunk is evaluated in
+// parallel from the chunk-start state:
+//
+//   S_{c0+i} = D[i][-1] S_in + sum_{j<i} D[i][j] (-eta_j) g_j x_j^T,
+//   D[i][j]  = prod_{r=j+1}^{i-1} alpha_r          (chunk-local indices)
+//
+// and the chunk-to-chunk carry is the same formula at i = FC. The decay
+// products D are formed by direct multiplication (no logarithms), so alpha = 0
+// and alpha = 1 are exact.
+//
+// The reverse scan (GradLev abstract: exact scans for reverse
+// backpropagation) walks the chunks backwards carrying the state adjoint
+// Lam_t = alpha_t Lam_{t+1} + u_t x_t^T in shared memory, with the chunk-start
+// states S_in read back from checkpoints written by a forward sweep.
+// d_alpha_t = <Lam_{t+1}, S_t> is evaluated exactly per chunk as the four
+// cross terms of (chunk-end adjoint + intra-chunk adjoint) x (chunk-start state
+// + intra-chunk state), which avoids any division by alpha.
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "scan_ffma.h"
+
+namespace gradlev {
+namespace ffma {
+
+constexpr int FC = 32;    // tokens per chunk
+constexpr int FT = 256;   // threads per CTA
+constexpr int LDD = FC + 2;  // row stride of the decay table
+constexpr int LDC = FC + 1;  // row stride of FC x FC tables
+
+__device__ __forceinline__ float dot4(float4 a, float4 b) {
+  return a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w;
+}
+
+__device__ __forceinline__ void fma4(float4& acc, float s, float4 v) {
+  acc.x = fmaf(s, v.x, acc.x);
+  acc.y = fmaf(s, v.y, acc.y);
+  acc.z = fmaf(s, v.z, acc.z);
+  acc.w = fmaf(s, v.w, acc.w);
+}
+
+// Decay table Dt[i*LDD + (j+1)] = prod_{r=j+1}^{i-1} al[r] for i in [0, FC],
+// j in [-1, FC-1] (1 for the empty product, 0 where i <= j). Threads 0..FC.
+__device__ __forceinline__ void decay_table(float* Dt, const float* al, int tid) {
+  if (tid <= FC) {
+    const int jp = tid;
+    float pr = 1.f;
+    for (int i = 0; i <= FC; ++i) {
+      if (i < jp) {
+        Dt[i * LDD + jp] = 0.f;
+      } else {
+        Dt[i * LDD + jp] = pr;
+        if (i < FC) pr *= al[i];
+      }
+    }
+  }
+}
+
+template <typename Tio>
+__device__ __forceinline__ void load_rows(float* dst, int ld, const Tio* src, int n_rows,
+                                          int n_valid, int width, int tid) {
+  for (int e = tid; e < n_rows * width; e += FT) {
+    const int i = e / width, k = e - i * width;
+    dst[i * ld + k] = (i < n_valid) ? to_f32(src[(size_t)i * width + k]) : 0.f;
+  }
+}
+
+size_t fwd_smem_bytes(int din, int dout) {
+  const int LDI = din + 4, LDO = dout + 4;
+  return sizeof(float) * ((size_t)2 * dout * LDI + (size_t)FC * LDI + (size_t)FC * LDO +
+                          (size_t)FC * LDC + (size_t)(FC + 1) * LDD + 2 * FC);
+}
+
+// Forward scan. y may be null (state sweep only); ckpt may be null. ckpt layout:
+// float [B*H][n_chunks][d_out][d_in], the state at the start of each chunk.
+template <typename Tio>
+__global__ void __launch_bounds__(FT, 1) fwd_kernel(FwdArgs a) {
+  extern __shared__ float4 smem4[];
+  float* sm = reinterpret_cast<float*>(smem4);
+  const int din = a.din, dout = a.dout, tid = threadIdx.x;
+  const int LDI = din + 4, LDO = dout + 4;
+  float* S = sm;
+  float* W = S + dout * LDI;
+  float* X = W + dout * LDI;
+  float* G = X + FC * LDI;
+  float* P = G + FC * LDO;
+  float* Dt = P + FC * LDC;
+  float* et = Dt + (FC + 1) * LDD;
+  float* al = et + FC;
+
+  const int bh = blockIdx.x, h = bh % a.H;
+  const size_t tok0 = (size_t)bh * a.T;
+  const int nch = (a.T + FC - 1) / FC;
+  const Tio* xg = static_cast<const Tio*>(a.x);
+  const Tio* gg = static_cast<const Tio*>(a.g);
+  Tio* yg = static_cast<Tio*>(a.y);
+  const float* W0 = a.W0 + (size_t)h * dout * din;
+
+  for (int e = tid; e < dout * din; e += FT) {
+    const int n = e / din, k = e - n * din;
+    S[n * LDI + k] = 0.f;
+    W[n * LDI + k] = W0[e];
+  }
+  const int NG = dout / 4, NK4 = din / 4, NB = dout / 8;
+
+  for (int c = 0; c < nch; ++c) {
+    const int t0 = c * FC;
+    const int nt = min(FC, a.T - t0);
+    __syncthreads();
+    if (a.ckpt) {
+      float* dst = a.ckpt + ((size_t)bh * nch + c) * dout * din;
+      for (int e = tid; e < dout * din; e += FT) {
+        const int n = e / din, k = e - n * din;
+        dst[e] = S[n * LDI + k];
+      }
+    }
+    load_rows(X, LDI, xg + (tok0 + t0) * din, FC, nt, din, tid);
+    load_rows(G, LDO, gg + (tok0 + t0) * dout, FC, nt, dout, tid);
+    if (tid < FC) {
+      et[tid] = tid < nt ? a.eta[tok0 + t0 + tid] : 0.f;
+      al[tid] = tid < nt ? a.alpha[tok0 + t0 + tid] : 1.f;
+    }
+    __syncthreads();
+    decay_table(Dt, al, tid);
+    __syncthreads();
+
+    if (yg) {
+      // P_ij = (x_i . x_j) (-eta_j) D[i][j] for j < i (strictly causal), else 0
+      for (int e = tid; e < FC * FC; e += FT) {
+        const int i = e / FC, j = e - i * FC;
+        float v = 0.f;
+        if (j < i) {
+          float acc = 0.f;
+          for (int k = 0; k < din; k += 4)
+            acc += dot4(*reinterpret_cast<const float4*>(&X[i * LDI + k]),
+                        *reinterpret_cast<const float4*>(&X[j * LDI + k]));
+          v = acc * (-et[j]) * Dt[i * LDD + j + 1];
+        }
+        P[i * LDC + j] = v;
+      }
+      __syncthreads();
+      // y_i = W0 x_i + D[i][-1] S_in x_i + sum_j P_ij g_j; thread tile 4 tokens x 4 outputs
+      for (int tile = tid; tile < (FC / 4) * NG; tile += FT) {
+        const int ig = tile / NG, ng = tile - ig * NG;
+        float a1[4][4], a2[4][4], a3[4][4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int r = 0; r < 4; ++r) a1[q][r] = a2[q][r] = a3[q][r] = 0.f;
+        for (int k = 0; k < din; k += 4) {
+          float4 xv[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) xv[q] = *reinterpret_cast<const float4*>(&X[(ig * 4 + q) * LDI + k]);
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const float4 wv = *reinterpret_cast<const float4*>(&W[(ng + NG * r) * LDI + k]);
+            const float4 sv = *reinterpret_cast<const float4*>(&S[(ng + NG * r) * LDI + k]);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              a1[q][r] += dot4(xv[q], wv);
+              a2[q][r] += dot4(xv[q], sv);
+            }
+          }
+        }
+        for (int j = 0; j < FC; ++j) {
+          float gv[4];
+#pragma unroll
+          for (int r = 0; r < 4; ++r) gv[r] = G[j * LDO + ng + NG * r];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float pv = P[(ig * 4 + q) * LDC + j];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) a3[q][r] = fmaf(pv, gv[r], a3[q][r]);
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int i = ig * 4 + q;
+          if (i < nt) {
+            const float gam = Dt[i * LDD];
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+              yg[(tok0 + t0 + i) * dout + ng + NG * r] =
+                  from_f32<Tio>(a1[q][r] + gam * a2[q][r] + a3[q][r]);
+          }
+        }
+      }
+      __syncthreads();
+    }
+
+    // carry: S <- D[FC][-1] S + sum_j (-eta_j D[FC][j]) g_j x_j^T
+    const float gC = Dt[FC * LDD];
+    for (int item = tid; item < NB * NK4; item += FT) {
+      const int nb = item / NK4, k4 = item - nb * NK4;
+      float4 acc[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const float4 s = *reinterpret_cast<const float4*>(&S[(nb * 8 + r) * LDI + 4 * k4]);
+        acc[r] = make_float4(gC * s.x, gC * s.y, gC * s.z, gC * s.w);
+      }
+      for (int j = 0; j < nt; ++j) {
+        const float w = -et[j] * Dt[FC * LDD + j + 1];
+        const float4 xv = *reinterpret_cast<const float4*>(&X[j * LDI + 4 * k4]);
+#pragma unroll
+        for (int r = 0; r < 8; ++r) fma4(acc[r], w * G[j * LDO + nb * 8 + r], xv);
+      }
+#pragma unroll
+      for (int r = 0; r < 8; ++r) *reinterpret_cast<float4*>(&S[(nb * 8 + r) * LDI + 4 * k4]) = acc[r];
+    }
+  }
+}
+
+size_t bwd_smem_bytes(int din, int dout) {
+  const int LDI = din + 4, LDO = dout + 4;
+  const int NG = dout / 4, NK = din / 4;
+  return sizeof(float) *
+         ((size_t)2 * dout * LDI + (size_t)FC * LDI + (size_t)2 * FC * LDO + (size_t)5 * FC * LDC +
+          (size_t)(FC + 1) * LDD + 2 * FC + (size_t)FC * (2 * NG + NK) + FT + 2 * FC + 4);
+}
+
+// Reverse scan. ckpt holds the chunk-start states (float [B*H][n_chunks][d_out][d_in]).
+// dW0p receives this pair's sum_t u_t x_t^T (float [B*H][d_out][d_in]).
+template <typename Tio>
+__global__ void __launch_bounds__(FT, 1) bwd_kernel(BwdArgs a) {
+  extern __shared__ float4 smem4[];
+  float* sm = reinterpret_cast<float*>(smem4);
+  const int din = a.din, dout = a.dout, tid = threadIdx.x;
+  const int LDI = din + 4, LDO = dout + 4;
+  const int NG = dout / 4, NK = din / 4, NB = dout / 8, NK4 = din / 4;
+  float* L = sm;                    // Lam, [dout][LDI]
+  float* Sin = L + dout * LDI;      // chunk-start state
+  float* X = Sin + dout * LDI;      // [FC][LDI]
+  float* G = X + FC * LDI;          // [FC][LDO]
+  float* U = G + FC * LDO;          // [FC][LDO]
+  float* K = U + FC * LDO;          // x_i . x_j
+  float* Kug = K + FC * LDC;        // u_i . g_j
+  float* Ar = Kug + FC * LDC;       // r intra weights
+  float* Z = Ar + FC * LDC;         // dx intra weights
+  float* Q = Z + FC * LDC;          // (u_s.g_j)(x_s.x_j)
+  float* Dt = Q + FC * LDC;
+  float* et = Dt + (FC + 1) * LDD;
+  float* al = et + FC;
+  float* qpart = al + FC;           // [FC][NG]
+  float* epart = qpart + FC * NG;   // [FC][NG]
+  float* ppart = epart + FC * NG;   // [FC][NK]
+  float* red = ppart + FC * NK;     // [FT]
+  float* qv = red + FT;             // [FC]
+  float* pv = qv + FC;              // [FC]
+  float* Esh = pv + FC;             // [1]
+
+  const int bh = blockIdx.x, h = bh % a.H;
+  const size_t tok0 = (size_t)bh * a.T;
+  const int nch = (a.T + FC - 1) / FC;
+  const Tio* xg = static_cast<const Tio*>(a.x);
+  const Tio* gg = static_cast<const Tio*>(a.g);
+  const Tio* ug = static_cast<const Tio*>(a.dy);
+  Tio* dxg = static_cast<Tio*>(a.dx);
+  Tio* dgg = static_cast<Tio*>(a.dg);
+  const float* W0 = a.W0 + (size_t)h * dout * din;
+
+  for (int e = tid; e < dout * din; e += FT) {
+    const int n = e / din, k = e - n * din;
+    L[n * LDI + k] = 0.f;
+  }
+  float4 dw[2][8];
+#pragma unroll
+  for (int it = 0; it < 2; ++it)
+#pragma unroll
+    for (int r = 0; r < 8; ++r) dw[it][r] = make_float4(0.f, 0.f, 0.f, 0.f);
+
+  for (int c = nch - 1; c >= 0; --c) {
+    const int t0 = c * FC;
+    const int nt = min(FC, a.T - t0);
+    __syncthreads();
+    load_rows(X, LDI, xg + (tok0 + t0) * din, FC, nt, din, tid);
+    load_rows(G, LDO, gg + (tok0 + t0) * dout, FC, nt, dout, tid);
+    load_rows(U, LDO, ug + (tok0 + t0) * dout, FC, nt, dout, tid);
+    {
+      const float* src = a.ckpt + ((size_t)bh * nch + c) * dout * din;
+      for (int e = tid; e < dout * din; e += FT) {
+        const int n = e / din, k = e - n * din;
+        Sin[n * LDI + k] = src[e];
+      }
+    }
+    if (tid < FC) {
+      et[tid] = tid < nt ? a.eta[tok0 + t0 + tid] : 0.f;
+      al[tid] = tid < nt ? a.alpha[tok0 + t0 + tid] : 1.f;
+    }
+    __syncthreads();
+    decay_table(Dt, al, tid);
+    // Gram matrices of the chunk
+    for (int e = tid; e < 2 * FC * FC; e += FT) {
+      const int which = e / (FC * FC), ij = e - which * FC * FC;
+      const int i = ij / FC, j = ij - i * FC;
+      float acc = 0.f;
+      if (which == 0) {
+        for (int k = 0; k < din; k += 4)
+          acc += dot4(*reinterpret_cast<const float4*>(&X[i * LDI + k]),
+                      *reinterpret_cast<const float4*>(&X[j * LDI + k]));
+        K[i * LDC + j] = acc;
+      } else {
+        for (int n = 0; n < dout; n += 4)
+          acc += dot4(*reinterpret_cast<const float4*>(&U[i * LDO + n]),
+                      *reinterpret_cast<const float4*>(&G[j * LDO + n]));
+        Kug[i * LDC + j] = acc;
+      }
+    }
+    {  // <Lam_end, S_in>, fixed-order block reduction
+      float acc = 0.f;
+      for (int e = tid; e < dout * din; e += FT) {
+        const int n = e / din, k = e - n * din;
+        acc = fmaf(L[n * LDI + k], Sin[n * LDI + k], acc);
+      }
+      red[tid] = acc;
+    }
+    __syncthreads();
+    for (int e = tid; e < FC * FC; e += FT) {
+      const int i = e / FC, j = e - i * FC;
+      // r_i intra: sum_{s>i} D[s][i] K_si u_s
+      Ar[i * LDC + j] = (j > i) ? Dt[j * LDD + i + 1] * K[j * LDC + i] : 0.f;
+      float z = 0.f;
+      if (j < i) z = -et[j] * Dt[i * LDD + j + 1] * Kug[i * LDC + j];
+      else if (j > i) z = -et[i] * Dt[j * LDD + i + 1] * Kug[j * LDC + i];
+      Z[i * LDC + j] = z;
+      // Q[j][s] for j < s (here i plays j, j plays s)
+      Q[i * LDC + j] = (j > i) ? Kug[j * LDC + i] * K[j * LDC + i] : 0.f;
+    }
+    if (tid == 0) {
+      float s = 0.f;
+      for (int e = 0; e < FT; ++e) s += red[e];
+      Esh[0] = s;
+    }
+    __syncthreads();
+
+    // r = D[FC][i] (Lam_end x_i) + sum_{s>i} Ar[i][s] u_s ; dg = -eta r ; partial sums
+    for (int tile = tid; tile < (FC / 4) * NG; tile += FT) {
+      const int ig = tile / NG, ng = tile - ig * NG;
+      float r1[4][4], ri[4][4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) r1[q][r] = ri[q][r] = 0.f;
+      for (int k = 0; k < din; k += 4) {
+        float4 xv[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) xv[q] = *reinterpret_cast<const float4*>(&X[(ig * 4 + q) * LDI + k]);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const float4 lv = *reinterpret_cast<const float4*>(&L[(ng + NG * r) * LDI + k]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) r1[q][r] += dot4(xv[q], lv);
+        }
+      }
+      for (int s = 0; s < FC; ++s) {
+        float uv[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) uv[r] = U[s * LDO + ng + NG * r];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float w = Ar[(ig * 4 + q) * LDC + s];
+#pragma unroll
+          for (int r = 0; r < 4; ++r) ri[q][r] = fmaf(w, uv[r], ri[q][r]);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = ig * 4 + q;
+        const float dl = Dt[FC * LDD + i + 1];
+        float pe = 0.f, pq = 0.f;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int n = ng + NG * r;
+          const float rr = dl * r1[q][r] + ri[q][r];
+          const float gv = G[i * LDO + n];
+          pe = fmaf(gv, rr, pe);
+          pq = fmaf(gv, r1[q][r], pq);
+          if (i < nt) dgg[(tok0 + t0 + i) * dout + n] = from_f32<Tio>(-et[i] * rr);
+        }
+        epart[i * NG + ng] = pe;
+        qpart[i * NG + ng] = pq;
+      }
+    }
+
+    // dx_i = W0^T u_i + D[i][-1] S_in^T u_i - eta_i D[FC][i] Lam_end^T g_i + sum_j Z_ij x_j
+    for (int tile = tid; tile < (FC / 4) * NK; tile += FT) {
+      const int ig = tile / NK, kg = tile - ig * NK;
+      float aw[4][4], as[4][4], alm[4][4], az[4][4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) aw[q][r] = as[q][r] = alm[q][r] = az[q][r] = 0.f;
+      for (int n = 0; n < dout; ++n) {
+        float uq[4], gq[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uq[q] = U[(ig * 4 + q) * LDO + n];
+          gq[q] = G[(ig * 4 + q) * LDO + n];
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int k = kg + NK * r;
+          const float w0 = __ldg(&W0[(size_t)n * din + k]);
+          const float sv = Sin[n * LDI + k];
+          const float lv = L[n * LDI + k];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            aw[q][r] = fmaf(uq[q], w0, aw[q][r]);
+            as[q][r] = fmaf(uq[q], sv, as[q][r]);
+            alm[q][r] = fmaf(gq[q], lv, alm[q][r]);
+          }
+        }
+      }
+      for (int j = 0; j < FC; ++j) {
+        float xv[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) xv[r] = X[j * LDI + kg + NK * r];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float z = Z[(ig * 4 + q) * LDC + j];
+#pragma unroll
+          for (int r = 0; r < 4; ++r) az[q][r] = fmaf(z, xv[r], az[q][r]);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = ig * 4 + q;
+        const float gam = Dt[i * LDD];
+        const float ed = et[i] * Dt[FC * LDD + i + 1];
+        float pp = 0.f;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int k = kg + NK * r;
+          pp = fmaf(X[i * LDI + k], as[q][r], pp);
+          if (i < nt)
+            dxg[(tok0 + t0 + i) * din + k] =
+                from_f32<Tio>(aw[q][r] + gam * as[q][r] - ed * alm[q][r] + az[q][r]);
+        }
+        ppart[i * NK + kg] = pp;
+      }
+    }
+    __syncthreads();
+    if (tid < FC) {
+      const int i = tid;
+      float se = 0.f, sq = 0.f, sp = 0.f;
+      for (int e = 0; e < NG; ++e) {
+        se += epart[i * NG + e];
+        sq += qpart[i * NG + e];
+      }
+      for (int e = 0; e < NK; ++e) sp += ppart[i * NK + e];
+      qv[i] = sq;
+      pv[i] = sp;
+      if (i < nt) a.d_eta[tok0 + t0 + i] = -se;
+    }
+    __syncthreads();
+    if (tid < FC) {
+      // d_alpha_i = <Lam_{i+1}, S_i> as four cross terms (see file header)
+      const int i = tid;
+      const float gam = Dt[i * LDD], dl = Dt[FC * LDD + i + 1];
+      float t2 = 0.f, t3 = 0.f, t4 = 0.f;
+      for (int j = 0; j < i; ++j) {
+        const float aij = -et[j] * Dt[i * LDD + j + 1];
+        t2 = fmaf(aij, qv[j], t2);
+        float inner = 0.f;
+        for (int s = i + 1; s < FC; ++s) inner = fmaf(Dt[s * LDD + i + 1], Q[j * LDC + s], inner);
+        t4 = fmaf(aij, inner, t4);
+      }
+      for (int s = i + 1; s < FC; ++s) t3 = fmaf(Dt[s * LDD + i + 1], pv[s], t3);
+      const float h = gam * dl * Esh[0] + dl * t2 + gam * t3 + t4;
+      if (i < nt) a.d_alpha[tok0 + t0 + i] = h;
+    }
+    // Lam <- D[FC][-1] Lam + sum_s D[s][-1] u_s x_s^T ; dW0 += sum_s u_s x_s^T
+    const float gC = Dt[FC * LDD];
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+      const int item = tid + it * FT;
+      if (item < NB * NK4) {
+        const int nb = item / NK4, k4 = item - nb * NK4;
+        float4 acc[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const float4 l = *reinterpret_cast<const float4*>(&L[(nb * 8 + r) * LDI + 4 * k4]);
+          acc[r] = make_float4(gC * l.x, gC * l.y, gC * l.z, gC * l.w);
+        }
+        for (int s = 0; s < nt; ++s) {
+          const float gs = Dt[s * LDD];
+          const float4 xv = *reinterpret_cast<const float4*>(&X[s * LDI + 4 * k4]);
+#pragma unroll
+          for (int r = 0; r < 8; ++r) {
+            const float uv = U[s * LDO + nb * 8 + r];
+            fma4(acc[r], gs * uv, xv);
+            fma4(dw[it][r], uv, xv);
+          }
+        }
+#pragma unroll
+        for (int r = 0; r < 8; ++r) *reinterpret_cast<float4*>(&L[(nb * 8 + r) * LDI + 4 * k4]) = acc[r];
+      }
+    }
+  }
+  // this pair's dW0 partial
+  float* dst = a.dW0_part + (size_t)bh * dout * din;
+#pragma unroll
+  for (int it = 0; it < 2; ++it) {
+    const int item = tid + it * FT;
+    if (item < NB * NK4) {
+      const int nb = item / NK4, k4 = item - nb * NK4;
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        *reinterpret_cast<float4*>(&dst[(size_t)(nb * 8 + r) * din + 4 * k4]) = dw[it][r];
+    }
+  }
+}
+
+// dW0[h] = sum_{b=0..B-1} part[b][h] in a fixed order (deterministic).
+__global__ void reduce_dW0_kernel(const float* __restrict__ part, float* __restrict__ dW0, int B,
+                                  int H, int dd) {
+  const size_t n = (size_t)H * dd;
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+       e += (size_t)gridDim.x * blockDim.x) {
+    float s = 0.f;
+    for (int b = 0; b < B; ++b) s += part[(size_t)b * n + e];
+    dW0[e] = s;
+  }
+}
+
+template <typename Tio>
+static cudaError_t launch_fwd_t(const FwdArgs& a, cudaStream_t st) {
+  const size_t smem = fwd_smem_bytes(a.din, a.dout);
+  cudaError_t e = cudaFuncSetAttribute(fwd_kernel<Tio>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  fwd_kernel<Tio><<<a.B * a.H, FT, smem, st>>>(a);
+  count_launch();
+  return cudaGetLastError();
+}
+
+template <typename Tio>
+static cudaError_t launch_bwd_t(const BwdArgs& a, cudaStream_t st) {
+  const size_t smem = bwd_smem_bytes(a.din, a.dout);
+  cudaError_t e = cudaFuncSetAttribute(bwd_kernel<Tio>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  bwd_kernel<Tio><<<a.B * a.H, FT, smem, st>>>(a);
+  count_launch();
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int dd = a.din * a.dout;
+  const size_t n = (size_t)a.H * dd;
+  const int blocks = (int)((n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184);
+  reduce_dW0_kernel<<<blocks, 256, 0, st>>>(a.dW0_part, a.dW0, a.B, a.H, dd);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fwd(const FwdArgs& a, bool bf16, cudaStream_t st) {
+  return bf16 ? launch_fwd_t<__nv_bfloat16>(a, st) : launch_fwd_t<float>(a, st);
+}
+
+cudaError_t launch_bwd(const BwdArgs& a, bool bf16, cudaStream_t st) {
+  return bf16 ? launch_bwd_t<__nv_bfloat16>(a, st) : launch_bwd_t<float>(a, st);
+}
+
+size_t ckpt_bytes(int B, int H, int T, int din, int dout) {
+  const size_t nch = (size_t)(T + FC - 1) / FC;
+  return (size_t)B * H * nch * din * dout * sizeof(float);
+}
+
+size_t dW0_part_bytes(int B, int H, int din, int dout) {
+  return (size_t)B * H * din * dout * sizeof(float);
+}
+
+bool shape_ok(int din, int dout) {
+  return din % 4 == 0 && dout % 8 == 0 && din >= 8 && dout >= 8 && din * dout <= 16384 &&
+         bwd_smem_bytes(din, dout) <= 227 * 1024 && fwd_smem_bytes(din, dout) <= 227 * 1024;
+}
+
+}  // namespace ffma
+}  // namespace gradlev
