@@ -49,6 +49,9 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=15.0,
                    help="target CPU work of the oracle sample")
+    p.add_argument("--B", type=int, default=None, help="override B (reduced profiling case)")
+    p.add_argument("--H", type=int, default=None, help="override H (reduced profiling case)")
+    p.add_argument("--T", type=int, default=None, help="override T (reduced profiling case)")
     return p.parse_args()
 
 
@@ -226,6 +229,11 @@ def main():
     args = parse()
     from token_weight_scans_b200 import inputs
     cfg = inputs.CONFIGS[args.config]
+    over = {k: getattr(args, k) for k in ("B", "H", "T") if getattr(args, k) is not None}
+    if over:
+        import dataclasses
+        cfg = dataclasses.replace(cfg, name=cfg.name + " reduced to " + " ".join(
+            f"{k}={v}" for k, v in over.items()), **over)
     if args.impl == "reference":
         return run_reference(args, cfg)
 
