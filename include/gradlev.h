@@ -126,6 +126,37 @@ GRADLEV_API gradlev_status gradlev_scan_bwd(int B, int H, int T, int d_in, int d
                                 const void* ckpt, void* workspace, size_t ws_bytes,
                                 void* stream);
 
+/* Size of the static scratch array gradlev_scan_bwd_noalloc uses: 64 MiB,
+ * held by every GPU that loads the library until the process exits. */
+#define GRADLEV_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+/* gradlev_scan_bwd without a workspace argument, for callers that cannot
+ * allocate device memory: code running where the allocator is unavailable or
+ * must not grow (a fixed-pool serving runtime, a plugin that is handed only its
+ * tensors, a host binding without a CUDA allocator). The method has no
+ * counterpart of this call; it is a deployment convenience of this library.
+ *
+ * Same arguments, outputs and results as gradlev_scan_bwd minus `workspace`
+ * and `ws_bytes`. Scratch comes from one static device array of
+ * GRADLEV_NOALLOC_SCRATCH_BYTES on the current device. The call allocates
+ * nothing (no cudaMalloc, cudaFree or allocating library routine).
+ *   - Limit: it needs 256 + B*H*d_out*d_in*4 bytes (rounded up to 256) of
+ *     scratch, plus gradlev_scan_ckpt_bytes() (rounded up to 256) when ckpt is
+ *     NULL; a problem that needs more returns GRADLEV_ERR_WORKSPACE before any
+ *     launch. Shape errors return as in gradlev_scan_bwd.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *     first call before any stream capture.
+ *   - Every call on a device shares the one array, and it keeps the last
+ *     call's contents (each call clears the part that must start at zero).
+ *     Calls whose work overlaps on the GPU (different streams, or other host
+ *     threads) race on it and give wrong results: serialise them.
+ *   - gradlev_device_status() does not apply to this call. */
+GRADLEV_API gradlev_status gradlev_scan_bwd_noalloc(
+    int B, int H, int T, int d_in, int d_out, gradlev_dtype dt, const void* x, const void* g,
+    const float* eta, const float* alpha, const float* W0, const void* dy, void* dx, void* dg,
+    float* d_eta, float* d_alpha, float* dW0, const void* ckpt, void* stream);
+
 /* Device status of the last call that used `workspace`: synchronises `stream`
  * and reads the status word the kernels leave at the start of the workspace.
  * GRADLEV_OK, GRADLEV_ERR_TIMEOUT if a bounded device-side wait gave up (the
