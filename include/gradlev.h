@@ -167,6 +167,15 @@ GRADLEV_API gradlev_status gradlev_device_status(const void* workspace, void* st
  * launched (for launch accounting by benchmarks). */
 GRADLEV_API int gradlev_last_launch_count(void);
 
+/* Test hook for the failure-detection path (no GPU fault or hang is involved):
+ * with enable != 0, the next bf16 tensor-core gradlev_scan_fwd call withholds
+ * one internal completion signal, so one of the kernel's bounded waits runs out
+ * after timeout_ms; every CTA then unwinds (in-flight copies and matrix
+ * operations are drained, tensor memory is released) and the call's
+ * gradlev_device_status() reports GRADLEV_ERR_TIMEOUT. Host-global, one-shot,
+ * not thread-safe; for tests only. */
+GRADLEV_API void gradlev_debug_inject_timeout(int enable, int timeout_ms);
+
 #ifdef __cplusplus
 }
 #endif

@@ -8,11 +8,17 @@
 #include "common.cuh"
 #include "gradlev.h"
 #include "scan_ffma.h"
+#include "scan_tc.h"
 
 namespace gradlev {
 
 static thread_local int t_launches = 0;
 void count_launch() { ++t_launches; }
+
+// Test hook state (gradlev_debug_inject_timeout): consumed by the next fwd call.
+static int g_inject = 0;
+static uint64_t g_inject_timeout_ns = 0;
+static constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // bound of device-side waits
 
 static constexpr size_t kStatusBytes = 256;  // status word + alignment pad
 
@@ -83,6 +89,22 @@ gradlev_status gradlev_scan_fwd(int B, int H, int T, int d_in, int d_out, gradle
   t_launches = 0;
   if (cudaMemsetAsync(workspace, 0, sizeof(DeviceStatus), st) != cudaSuccess)
     return GRADLEV_ERR_CUDA;
+  if (dt == GRADLEV_BF16 && tc::fwd_shape_ok(d_in, d_out)) {
+    // tensor-core forward; the reverse scan of this build consumes the CUDA-core
+    // checkpoint format, which a state-only CUDA-core sweep writes when requested
+    const int inject = g_inject;
+    const uint64_t tmo = inject ? g_inject_timeout_ns : kWaitTimeoutNs;
+    g_inject = 0;
+    tc::TcFwdParams prm{B, H, T, d_in, d_out, eta, alpha, W0, static_cast<__nv_bfloat16*>(y),
+                        static_cast<DeviceStatus*>(workspace), tmo, inject};
+    if (tc::launch_fwd(prm, x, g, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
+    if (ckpt) {
+      ffma::FwdArgs a{B, H, T, d_in, d_out, x, g, eta, alpha, W0, nullptr,
+                      static_cast<float*>(ckpt)};
+      if (ffma::launch_fwd(a, true, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
+    }
+    return GRADLEV_OK;
+  }
   ffma::FwdArgs a{B, H, T, d_in, d_out, x, g, eta, alpha, W0, y, static_cast<float*>(ckpt)};
   if (ffma::launch_fwd(a, dt == GRADLEV_BF16, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
   return GRADLEV_OK;
@@ -139,5 +161,10 @@ gradlev_status gradlev_device_status(const void* workspace, void* stream) {
 }
 
 int gradlev_last_launch_count(void) { return t_launches; }
+
+void gradlev_debug_inject_timeout(int enable, int timeout_ms) {
+  g_inject = enable ? 1 : 0;
+  g_inject_timeout_ns = (uint64_t)(timeout_ms > 0 ? timeout_ms : 1) * 1000000ull;
+}
 
 }  // extern "C"

@@ -1,0 +1,475 @@
+// Tensor-core (tcgen05/TMEM) forward GradLev scan for bf16 I/O, d_in = 128 and
+// d_out a multiple of 128 (one CTA per (b, h, 128-wide slice of d_out)).
+//
+// Method (Cognaptus, "Parallelize the Training, Keep the Learning Serial",
+// section "Once the gradient signals are known, the weight trajectory becomes
+// parallelizable"; GradLev abstract): S_0 = 0, y_t = (W0 + S_t) x_t,
+// S_{t+1} = alpha_t S_t - eta_t g_t x_t^T. The deviation is a discounted sum
+// of rank-one updates, so within a chunk of C = 64 tokens starting at c0,
+// with L_j = sum_{r<=j} log2 alpha_{c0+r} (chunk-local):
+//
+//   y_i = W0 x_i + 2^{L_{i-1}} S x_i + sum_{j<i} (x_i.x_j) (-eta_j) 2^{L_{i-1}-L_j} g_j
+//   S'  = 2^{L_{C-1}} S + sum_j (-eta_j 2^{L_{C-1}-L_j}) g_j x_j^T
+//
+// All products are done transposed, with d_out on the 128 TMEM lanes:
+//   K    = X X^T                         (M=64 tokens, N=64, K=d_in)        -> TMEM
+//   P_ij = K_ij (-eta_j) 2^{L_{i-1}-L_j}  (j < i), bf16 in shared memory
+//   Y1^T = W0 X^T + G^T P^T               (M=128, N=64, K=d_in+C)            -> TMEM
+//   Y2^T = S X^T                          (M=128, N=64, K=d_in)              -> TMEM
+//   dS   = G^T Xhat, Xhat_j = w_j x_j     (M=128, N=d_in, K=C)               -> TMEM
+//   y_i  = Y1^T[:, i] + 2^{L_{i-1}} Y2^T[:, i]; S <- 2^{L_{C-1}} S + dS (fp32, registers)
+//
+// Warp roles (12 warps): 0 TMA producer, 1 MMA issuer (+TMEM owner), 2 gate
+// prep (log2 alpha cumulative sums), 3 scaled-X producer, 4..11 two math
+// warpgroups (mask, state update, output epilogue), warpgroup h handling
+// columns [64h, 64h+64) of the state and tokens [32h, 32h+32) of the output.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "scan_tc.h"
+#include "sm100.cuh"
+
+namespace gradlev {
+namespace tc {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int C = 64;          // tokens per chunk
+constexpr int NS = 3;          // TMA stages (X and G tiles)
+constexpr int GS = 4;          // gate slots
+constexpr int NTHREADS = 384;  // 12 warps
+constexpr int TILE = C * 128;  // bytes of one [64 rows x 128 B] swizzled block
+
+// TMEM columns (512 allocated)
+constexpr uint32_t COL_K0 = 0, COL_K1 = 64;      // K = X X^T (M=64 layout), double buffer
+constexpr uint32_t COL_Y1 = 128;                 // + 64 * buffer
+constexpr uint32_t COL_Y2 = 256;                 // + 64 * buffer
+constexpr uint32_t COL_DS = 384;                 // 128 columns
+
+struct GateSlot {
+  float L[C];     // chunk-local inclusive cumulative sum of log2 alpha
+  float eta[C];
+  float gam[C];   // 2^{L_{i-1}}
+  float w[C];     // -eta_j 2^{L_{C-1} - L_j}
+  float gC;       // 2^{L_{C-1}}
+  float pad[3];
+};
+
+struct Smem {
+  // 1024-byte aligned tiles first
+  uint8_t X[NS][2 * TILE];     // k-blocks [0,64), [64,128): 64 token rows x 128 B
+  uint8_t G[NS][2 * TILE];     // n-blocks of the slice: 64 token rows x 128 B
+  uint8_t W0[2][128 * 128];    // k-blocks: 128 n rows x 128 B (bf16 W0 slice)
+  uint8_t S[2][128 * 128];     // k-blocks: 128 n rows x 128 B (bf16 state)
+  uint8_t P[TILE];             // 64 token rows (i) x 128 B (j)
+  uint8_t Xh[2 * TILE];        // scaled X, same layout as X
+  GateSlot gates[GS];
+  uint64_t full[NS], empty[NS];
+  uint64_t gfull[GS], gempty[GS];
+  uint64_t kfull[2], kfree[2];
+  uint64_t yfull[2], yfree[2];
+  uint64_t pready, xready, dsfull, dsfree, sready, sfree, done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
+
+// where-codes of the bounded waits (role << 8 | site)
+enum : uint32_t {
+  W_TMA_EMPTY = 0x001, W_TMA_DRAIN = 0x002,
+  W_MMA_FULL = 0x101, W_MMA_KFREE, W_MMA_YFREE, W_MMA_XREADY, W_MMA_DSFREE, W_MMA_PREADY,
+  W_MMA_SREADY, W_MMA_DONE,
+  W_GATE_EMPTY = 0x201,
+  W_XH_FULL = 0x301, W_XH_GFULL, W_XH_DSFULL,
+  W_M_GFULL = 0x401, W_M_KFULL, W_M_DSFULL, W_M_SFREE, W_M_YFULL,
+};
+
+}  // namespace
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmG,
+               TcFwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nslice = p.dout >> 7;
+  const int bh = blockIdx.x / nslice, slice = blockIdx.x - bh * nslice;
+  const int h = bh % p.H;
+  const int n0 = slice * 128;
+  const int T = p.T;
+  const int nch = (T + C - 1) / C;
+  const WaitCtx wc{&sm.abort, p.status, p.timeout_ns};
+
+  if (threadIdx.x == 0) {
+    sm.abort = 0;
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
+    }
+    for (int g = 0; g < GS; ++g) {
+      mbar_init(&sm.gfull[g], 32);
+      mbar_init(&sm.gempty[g], 9);  // scaled-X warp + 8 math warps
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.kfull[b], 1);
+      mbar_init(&sm.kfree[b], 8);
+      mbar_init(&sm.yfull[b], 1);
+      mbar_init(&sm.yfree[b], 8);
+    }
+    mbar_init(&sm.pready, 8);
+    mbar_init(&sm.xready, 1);
+    mbar_init(&sm.dsfull, 1);
+    mbar_init(&sm.dsfree, 8);
+    mbar_init(&sm.sready, 8);
+    mbar_init(&sm.sfree, 1);
+    mbar_init(&sm.done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmX);
+    prefetch_tmap(&tmG);
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  // W0 slice -> bf16 swizzled K-major tiles; S_0 = 0
+  if (warp >= 4) {
+    const int t = threadIdx.x - 128;  // 0..255
+    const float* W0 = p.W0 + ((size_t)h * p.dout + n0) * 128;
+    for (int idx = t; idx < 128 * 16; idx += 256) {  // (row n, 16-byte chunk of 8 k)
+      const int n = idx >> 4, ck = idx & 15;
+      const int kb = ck >> 3, c = ck & 7;
+      const float4 a = *reinterpret_cast<const float4*>(W0 + (size_t)n * 128 + ck * 8);
+      const float4 b = *reinterpret_cast<const float4*>(W0 + (size_t)n * 128 + ck * 8 + 4);
+      st_shared_v4(smem_u32(sm.W0[kb]) + sw128_off(n, c), pack_bf16(a.x, a.y),
+                   pack_bf16(a.z, a.w), pack_bf16(b.x, b.y), pack_bf16(b.z, b.w));
+      st_shared_v4(smem_u32(sm.S[kb]) + sw128_off(n, c), 0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = sm.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    int issued = 0;
+    if (lane == 0) {
+      for (int c = 0; c < nch; ++c) {
+        const int s = c % NS;
+        if (!mbar_wait(&sm.empty[s], ((c / NS) & 1) ^ 1, wc, W_TMA_EMPTY)) break;
+        mbar_arrive_expect_tx(&sm.full[s], 4 * TILE);
+        tma_load_3d(sm.X[s], &tmX, &sm.full[s], 0, c * C, bh);
+        tma_load_3d(sm.X[s] + TILE, &tmX, &sm.full[s], 64, c * C, bh);
+        tma_load_3d(sm.G[s], &tmG, &sm.full[s], n0, c * C, bh);
+        tma_load_3d(sm.G[s] + TILE, &tmG, &sm.full[s], n0 + 64, c * C, bh);
+        issued = c + 1;
+      }
+      // teardown: let every load this thread issued land before the CTA exits
+      for (int c = issued > NS ? issued - NS : 0; c < issued; ++c)
+        mbar_drain(&sm.full[c % NS], (c / NS) & 1, wc, W_TMA_DRAIN);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t id_k = idesc_bf16(64, 64, false, false);
+      const uint32_t id_y = idesc_bf16(128, 64, false, false);
+      const uint32_t id_gp = idesc_bf16(128, 64, true, false);
+      const uint32_t id_ds = idesc_bf16(128, 128, true, true);
+      const uint32_t sW0 = smem_u32(sm.W0[0]), sS = smem_u32(sm.S[0]);
+      const uint32_t sP = smem_u32(sm.P), sXh = smem_u32(sm.Xh);
+      for (int c = 0; c < nch; ++c) {
+        const int s = c % NS, b = c & 1;
+        const uint32_t sX = smem_u32(sm.X[s]), sG = smem_u32(sm.G[s]);
+        if (!mbar_wait(&sm.full[s], (c / NS) & 1, wc, W_MMA_FULL)) break;
+        if (!mbar_wait(&sm.kfree[b], ((c >> 1) & 1) ^ 1, wc, W_MMA_KFREE)) break;
+        tc_fence_after();
+        // K = X X^T
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * TILE + (kk & 3) * 32;
+          umma_bf16(tbase + (b ? COL_K1 : COL_K0), sw128_desc(sX + off, 16, 1024),
+                    sw128_desc(sX + off, 16, 1024), id_k, kk > 0);
+        }
+        if (!(p.inject == 1 && c == 1)) umma_commit(&sm.kfull[b]);
+        if (!mbar_wait(&sm.yfree[b], ((c >> 1) & 1) ^ 1, wc, W_MMA_YFREE)) break;
+        tc_fence_after();
+        // Y1^T = W0 X^T
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t aoff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          const uint32_t boff = (kk >> 2) * TILE + (kk & 3) * 32;
+          umma_bf16(tbase + COL_Y1 + 64 * b, sw128_desc(sW0 + aoff, 16, 1024),
+                    sw128_desc(sX + boff, 16, 1024), id_y, kk > 0);
+        }
+        // dS = G^T Xhat
+        if (!mbar_wait(&sm.xready, c & 1, wc, W_MMA_XREADY)) break;
+        if (c > 0 && !mbar_wait(&sm.dsfree, (c - 1) & 1, wc, W_MMA_DSFREE)) break;
+        tc_fence_after();
+        for (int kk = 0; kk < 4; ++kk) {
+          umma_bf16(tbase + COL_DS, sw128_desc(sG + kk * 2048, TILE, 1024),
+                    sw128_desc(sXh + kk * 2048, TILE, 1024), id_ds, kk > 0);
+        }
+        umma_commit(&sm.dsfull);
+        // Y1^T += G^T P^T
+        if (!mbar_wait(&sm.pready, c & 1, wc, W_MMA_PREADY)) break;
+        tc_fence_after();
+        for (int kk = 0; kk < 4; ++kk) {
+          umma_bf16(tbase + COL_Y1 + 64 * b, sw128_desc(sG + kk * 2048, TILE, 1024),
+                    sw128_desc(sP + kk * 32, 16, 1024), id_gp, 1);
+        }
+        // Y2^T = S X^T
+        if (c > 0 && !mbar_wait(&sm.sready, (c - 1) & 1, wc, W_MMA_SREADY)) break;
+        tc_fence_after();
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t aoff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          const uint32_t boff = (kk >> 2) * TILE + (kk & 3) * 32;
+          umma_bf16(tbase + COL_Y2 + 64 * b, sw128_desc(sS + aoff, 16, 1024),
+                    sw128_desc(sX + boff, 16, 1024), id_y, kk > 0);
+        }
+        umma_commit(&sm.yfull[b]);
+        umma_commit(&sm.sfree);
+        umma_commit(&sm.empty[s]);
+      }
+      // teardown: every issued MMA completes before TMEM is released
+      umma_commit(&sm.done);
+      mbar_drain(&sm.done, 0, wc, W_MMA_DONE);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ gate prep
+    const size_t gbase = (size_t)bh * T;
+    for (int c = 0; c < nch; ++c) {
+      const int g = c % GS;
+      if (!mbar_wait(&sm.gempty[g], ((c / GS) & 1) ^ 1, wc, W_GATE_EMPTY)) break;
+      GateSlot& gs = sm.gates[g];
+      const int t0 = c * C + lane, t1 = t0 + 32;
+      const float a0 = t0 < T ? p.alpha[gbase + t0] : 1.f;
+      const float a1 = t1 < T ? p.alpha[gbase + t1] : 1.f;
+      const float e0 = t0 < T ? p.eta[gbase + t0] : 0.f;
+      const float e1 = t1 < T ? p.eta[gbase + t1] : 0.f;
+      float l0 = fmaxf(log2f(a0), -100.f), l1 = fmaxf(log2f(a1), -100.f);
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float u0 = __shfl_up_sync(0xffffffffu, l0, o);
+        const float u1 = __shfl_up_sync(0xffffffffu, l1, o);
+        if (lane >= o) {
+          l0 += u0;
+          l1 += u1;
+        }
+      }
+      l1 += __shfl_sync(0xffffffffu, l0, 31);
+      const float Lend = __shfl_sync(0xffffffffu, l1, 31);
+      const float pm0 = __shfl_up_sync(0xffffffffu, l0, 1);
+      const float pm1 = __shfl_up_sync(0xffffffffu, l1, 1);
+      const float last0 = __shfl_sync(0xffffffffu, l0, 31);
+      gs.L[lane] = l0;
+      gs.L[lane + 32] = l1;
+      gs.eta[lane] = e0;
+      gs.eta[lane + 32] = e1;
+      gs.gam[lane] = lane == 0 ? 1.f : exp2f(pm0);
+      gs.gam[lane + 32] = exp2f(lane == 0 ? last0 : pm1);
+      gs.w[lane] = -e0 * exp2f(Lend - l0);
+      gs.w[lane + 32] = -e1 * exp2f(Lend - l1);
+      if (lane == 0) gs.gC = exp2f(Lend);
+      __syncwarp();
+      mbar_arrive(&sm.gfull[g]);
+    }
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ scaled-X producer
+    for (int c = 0; c < nch; ++c) {
+      const int s = c % NS, g = c % GS;
+      if (!mbar_wait(&sm.full[s], (c / NS) & 1, wc, W_XH_FULL)) break;
+      if (!mbar_wait(&sm.gfull[g], (c / GS) & 1, wc, W_XH_GFULL)) break;
+      if (c > 0 && !mbar_wait(&sm.dsfull, (c - 1) & 1, wc, W_XH_DSFULL)) break;
+      const uint32_t src = smem_u32(sm.X[s]), dst = smem_u32(sm.Xh);
+      const float* w = sm.gates[g].w;
+#pragma unroll 4
+      for (int idx = lane; idx < 2 * TILE / 16; idx += 32) {
+        const uint32_t off = idx * 16;
+        const int j = (off & (TILE - 1)) >> 7;  // token row
+        const float wj = w[j];
+        const uint4 v = ld_shared_v4(src + off);
+        st_shared_v4(dst + off, pack_bf16(wj * bf16_lo(v.x), wj * bf16_hi(v.x)),
+                     pack_bf16(wj * bf16_lo(v.y), wj * bf16_hi(v.y)),
+                     pack_bf16(wj * bf16_lo(v.z), wj * bf16_hi(v.z)),
+                     pack_bf16(wj * bf16_lo(v.w), wj * bf16_hi(v.w)));
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&sm.xready);
+        mbar_arrive(&sm.gempty[g]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ math warpgroups
+    const int q = warp & 3;          // TMEM lane quadrant
+    const int hh = (warp - 4) >> 2;  // warpgroup: state columns [64hh, 64hh+64), tokens [32hh, +32)
+    const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+    const int n = 32 * q + lane;     // row of the d_out slice owned by this thread
+    float Sreg[64];
+#pragma unroll
+    for (int e = 0; e < 64; ++e) Sreg[e] = 0.f;
+    __nv_bfloat16* yout = p.y + (size_t)bh * T * p.dout + n0 + n;
+
+    for (int c = 0; c < nch; ++c) {
+      const int g = c % GS, b = c & 1;
+      const GateSlot& gs = sm.gates[g];
+      if (!mbar_wait(&sm.gfull[g], (c / GS) & 1, wc, W_M_GFULL)) break;
+
+      // ---- mask: P_ij = K_ij (-eta_j) 2^{L_{i-1} - L_j}, j < i
+      if (!mbar_wait(&sm.kfull[b], (c >> 1) & 1, wc, W_M_KFULL)) break;
+      tc_fence_after();
+      {
+        float v[32];
+        tmem_ld32(tbase + (b ? COL_K1 : COL_K0) + lane_off + 32 * hh, v);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.kfree[b]);
+        if (lane < 16) {
+          const int i = 16 * q + lane;
+          const float Lm1 = i == 0 ? 0.f : gs.L[i - 1];
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int j = 32 * hh + e;
+            const float p0 = (j < i) ? v[e] * (-gs.eta[j]) * exp2f(Lm1 - gs.L[j]) : 0.f;
+            const float p1 = (j + 1 < i) ? v[e + 1] * (-gs.eta[j + 1]) * exp2f(Lm1 - gs.L[j + 1]) : 0.f;
+            pk[e >> 1] = pack_bf16(p0, p1);
+          }
+          const uint32_t prow = smem_u32(sm.P);
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc)
+            st_shared_v4(prow + sw128_off(i, 4 * hh + cc), pk[4 * cc], pk[4 * cc + 1],
+                         pk[4 * cc + 2], pk[4 * cc + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.pready);
+      }
+
+      // ---- state: S <- 2^{L_{C-1}} S + dS ; bf16 copy for the next chunk
+      if (!mbar_wait(&sm.dsfull, c & 1, wc, W_M_DSFULL)) break;
+      if (!mbar_wait(&sm.sfree, c & 1, wc, W_M_SFREE)) break;
+      tc_fence_after();
+      {
+        float v0[32], v1[32];
+        tmem_ld32(tbase + COL_DS + lane_off + 64 * hh, v0);
+        tmem_ld32(tbase + COL_DS + lane_off + 64 * hh + 32, v1);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.dsfree);
+        const float gC = gs.gC;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          Sreg[e] = fmaf(gC, Sreg[e], v0[e]);
+          Sreg[32 + e] = fmaf(gC, Sreg[32 + e], v1[e]);
+        }
+        const uint32_t srow = smem_u32(sm.S[hh]);
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc)
+          st_shared_v4(srow + sw128_off(n, cc), pack_bf16(Sreg[8 * cc], Sreg[8 * cc + 1]),
+                       pack_bf16(Sreg[8 * cc + 2], Sreg[8 * cc + 3]),
+                       pack_bf16(Sreg[8 * cc + 4], Sreg[8 * cc + 5]),
+                       pack_bf16(Sreg[8 * cc + 6], Sreg[8 * cc + 7]));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.sready);
+      }
+
+      // ---- output: y_i = Y1^T[n][i] + 2^{L_{i-1}} Y2^T[n][i]
+      if (!mbar_wait(&sm.yfull[b], (c >> 1) & 1, wc, W_M_YFULL)) break;
+      tc_fence_after();
+      {
+        float a[32], s2[32];
+        tmem_ld32(tbase + COL_Y1 + 64 * b + lane_off + 32 * hh, a);
+        tmem_ld32(tbase + COL_Y2 + 64 * b + lane_off + 32 * hh, s2);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.yfree[b]);
+        const int ib = 32 * hh;
+        const int tb = c * C + ib;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          if (tb + e < T)
+            yout[(size_t)(tb + e) * p.dout] = __float2bfloat16_rn(fmaf(gs.gam[ib + e], s2[e], a[e]));
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.gempty[g]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 3-D bf16 map over [d2][d1][d0] (d0 innermost), box {64, box1, 1}, 128-byte swizzle.
+bool make_map_bf16_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                      uint32_t box1) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {64, box1, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool fwd_shape_ok(int din, int dout) { return din == 128 && dout % 128 == 0 && dout <= 256; }
+
+cudaError_t launch_fwd(const TcFwdParams& prm, const void* x, const void* g, cudaStream_t st) {
+  CUtensorMap mx, mg;
+  if (!make_map_bf16_3d(&mx, x, prm.din, prm.T, (uint64_t)prm.B * prm.H, C) ||
+      !make_map_bf16_3d(&mg, g, prm.dout, prm.T, (uint64_t)prm.B * prm.H, C))
+    return cudaErrorInvalidValue;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int grid = prm.B * prm.H * (prm.dout / 128);
+  fwd_kernel<<<grid, NTHREADS, kSmemBytes, st>>>(mx, mg, prm);
+  count_launch();
+  return cudaGetLastError();
+}
+
+size_t fwd_smem_bytes() { return kSmemBytes; }
+
+}  // namespace tc
+}  // namespace gradlev
