@@ -32,8 +32,9 @@ def _lib():
 def gpu_fwd(d):
     import token_weight_scans_b200 as tw
     t = to_device(d, "bf16")
-    y = tw.gradlev_scan_fwd(t["x"], t["g"], t["eta"], t["alpha"], t["W0"])
-    torch.cuda.synchronize()
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    y = tw.gradlev_scan_fwd(t["x"], t["g"], t["eta"], t["alpha"], t["W0"], workspace=ws)
+    assert tw.gradlev_device_status(ws) == 0, "device-side wait timed out"
     return to_numpy(y)
 
 

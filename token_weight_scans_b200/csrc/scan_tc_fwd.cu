@@ -20,9 +20,12 @@
 //   y_i  = Y1^T[:, i] + 2^{L_{i-1}} Y2^T[:, i]; S <- 2^{L_{C-1}} S + dS (fp32, registers)
 //
 // Warp roles (12 warps): 0 TMA producer, 1 MMA issuer (+TMEM owner), 2 gate
-// prep (log2 alpha cumulative sums), 3 scaled-X producer, 4..11 two math
-// warpgroups (mask, state update, output epilogue), warpgroup h handling
+// prep (log2 alpha cumulative sums, prefetched) and half of the scaled-X tile,
+// 3 the other half of the scaled-X tile, 4..11 two math warpgroups (state
+// update, mask of the next chunk, output epilogue), warpgroup h handling
 // columns [64h, 64h+64) of the state and tokens [32h, 32h+32) of the output.
+// The bf16 copy of the state is double-buffered so the state update of chunk
+// c overlaps the S X^T product of chunk c.
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -66,7 +69,7 @@ struct Smem {
   uint8_t X[NS][2 * TILE];     // k-blocks [0,64), [64,128): 64 token rows x 128 B
   uint8_t G[NS][2 * TILE];     // n-blocks of the slice: 64 token rows x 128 B
   uint8_t W0[2][128 * 128];    // k-blocks: 128 n rows x 128 B (bf16 W0 slice)
-  uint8_t S[2][128 * 128];     // k-blocks: 128 n rows x 128 B (bf16 state)
+  uint8_t S[2][2][128 * 128];  // [buffer][k-block]: 128 n rows x 128 B (bf16 state)
   uint8_t P[TILE];             // 64 token rows (i) x 128 B (j)
   uint8_t Xh[2 * TILE];        // scaled X, same layout as X
   GateSlot gates[GS];
@@ -74,7 +77,9 @@ struct Smem {
   uint64_t gfull[GS], gempty[GS];
   uint64_t kfull[2], kfree[2];
   uint64_t yfull[2], yfree[2];
-  uint64_t pready, xready, dsfull, dsfree, sready, sfree, done;
+  uint64_t sready[2], sfree[2];  // per bf16 state buffer
+  uint64_t pready, xready, dsfull, dsfree, done;
+  uint32_t pad_;
   uint32_t tmem_base;
   int abort;
 };
@@ -116,7 +121,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     for (int g = 0; g < GS; ++g) {
       mbar_init(&sm.gfull[g], 32);
-      mbar_init(&sm.gempty[g], 9);  // scaled-X warp + 8 math warps
+      mbar_init(&sm.gempty[g], 10);  // 2 scaled-X warps + 8 math warps
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.kfull[b], 1);
@@ -125,11 +130,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&sm.yfree[b], 8);
     }
     mbar_init(&sm.pready, 8);
-    mbar_init(&sm.xready, 1);
+    mbar_init(&sm.xready, 2);
     mbar_init(&sm.dsfull, 1);
     mbar_init(&sm.dsfree, 8);
-    mbar_init(&sm.sready, 8);
-    mbar_init(&sm.sfree, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.sready[b], 8);
+      mbar_init(&sm.sfree[b], 1);
+    }
     mbar_init(&sm.done, 1);
     fence_mbar_init();
   }
@@ -152,7 +159,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const float4 b = *reinterpret_cast<const float4*>(W0 + (size_t)n * 128 + ck * 8 + 4);
       st_shared_v4(smem_u32(sm.W0[kb]) + sw128_off(n, c), pack_bf16(a.x, a.y),
                    pack_bf16(a.z, a.w), pack_bf16(b.x, b.y), pack_bf16(b.z, b.w));
-      st_shared_v4(smem_u32(sm.S[kb]) + sw128_off(n, c), 0u, 0u, 0u, 0u);
+      st_shared_v4(smem_u32(sm.S[0][kb]) + sw128_off(n, c), 0u, 0u, 0u, 0u);
     }
     fence_proxy_async_smem();
   }
@@ -186,7 +193,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint32_t id_y = idesc_bf16(128, 64, false, false);
       const uint32_t id_gp = idesc_bf16(128, 64, true, false);
       const uint32_t id_ds = idesc_bf16(128, 128, true, true);
-      const uint32_t sW0 = smem_u32(sm.W0[0]), sS = smem_u32(sm.S[0]);
+      const uint32_t sW0 = smem_u32(sm.W0[0]);
       const uint32_t sP = smem_u32(sm.P), sXh = smem_u32(sm.Xh);
       for (int c = 0; c < nch; ++c) {
         const int s = c % NS, b = c & 1;
@@ -226,9 +233,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           umma_bf16(tbase + COL_Y1 + 64 * b, sw128_desc(sG + kk * 2048, TILE, 1024),
                     sw128_desc(sP + kk * 32, 16, 1024), id_gp, 1);
         }
-        // Y2^T = S X^T
-        if (c > 0 && !mbar_wait(&sm.sready, (c - 1) & 1, wc, W_MMA_SREADY)) break;
+        // Y2^T = S X^T (state buffer c & 1, written by the state update of chunk c - 1)
+        if (c > 0 && !mbar_wait(&sm.sready[b], ((c - 1) >> 1) & 1, wc, W_MMA_SREADY)) break;
         tc_fence_after();
+        const uint32_t sS = smem_u32(sm.S[b][0]);
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t aoff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
           const uint32_t boff = (kk >> 2) * TILE + (kk & 3) * 32;
@@ -236,77 +244,100 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     sw128_desc(sX + boff, 16, 1024), id_y, kk > 0);
         }
         umma_commit(&sm.yfull[b]);
-        umma_commit(&sm.sfree);
+        umma_commit(&sm.sfree[b]);
         umma_commit(&sm.empty[s]);
       }
       // teardown: every issued MMA completes before TMEM is released
       umma_commit(&sm.done);
       mbar_drain(&sm.done, 0, wc, W_MMA_DONE);
     }
-  } else if (warp == 2) {
-    // ------------------------------------------------------------ gate prep
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------------------------ gates + scaled X
+    // Warp 2 also prepares the gates of each chunk (alpha / eta prefetched PD chunks
+    // ahead so the global-load latency is off the chain); both warps then write
+    // half of Xhat = w (.) X with packed bf16 multiplies.
+    constexpr int PD = 4;
     const size_t gbase = (size_t)bh * T;
-    for (int c = 0; c < nch; ++c) {
-      const int g = c % GS;
-      if (!mbar_wait(&sm.gempty[g], ((c / GS) & 1) ^ 1, wc, W_GATE_EMPTY)) break;
-      GateSlot& gs = sm.gates[g];
-      const int t0 = c * C + lane, t1 = t0 + 32;
-      const float a0 = t0 < T ? p.alpha[gbase + t0] : 1.f;
-      const float a1 = t1 < T ? p.alpha[gbase + t1] : 1.f;
-      const float e0 = t0 < T ? p.eta[gbase + t0] : 0.f;
-      const float e1 = t1 < T ? p.eta[gbase + t1] : 0.f;
-      float l0 = fmaxf(log2f(a0), -100.f), l1 = fmaxf(log2f(a1), -100.f);
+    const bool gate_warp = warp == 2;
+    float ra[PD][2], re[PD][2];
+    if (gate_warp) {
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const float u0 = __shfl_up_sync(0xffffffffu, l0, o);
-        const float u1 = __shfl_up_sync(0xffffffffu, l1, o);
-        if (lane >= o) {
-          l0 += u0;
-          l1 += u1;
-        }
+      for (int k = 0; k < PD; ++k) {
+        const int t0 = k * C + lane, t1 = t0 + 32;
+        ra[k][0] = t0 < T ? p.alpha[gbase + t0] : 1.f;
+        ra[k][1] = t1 < T ? p.alpha[gbase + t1] : 1.f;
+        re[k][0] = t0 < T ? p.eta[gbase + t0] : 0.f;
+        re[k][1] = t1 < T ? p.eta[gbase + t1] : 0.f;
       }
-      l1 += __shfl_sync(0xffffffffu, l0, 31);
-      const float Lend = __shfl_sync(0xffffffffu, l1, 31);
-      const float pm0 = __shfl_up_sync(0xffffffffu, l0, 1);
-      const float pm1 = __shfl_up_sync(0xffffffffu, l1, 1);
-      const float last0 = __shfl_sync(0xffffffffu, l0, 31);
-      gs.L[lane] = l0;
-      gs.L[lane + 32] = l1;
-      gs.eta[lane] = e0;
-      gs.eta[lane + 32] = e1;
-      gs.gam[lane] = lane == 0 ? 1.f : exp2f(pm0);
-      gs.gam[lane + 32] = exp2f(lane == 0 ? last0 : pm1);
-      gs.w[lane] = -e0 * exp2f(Lend - l0);
-      gs.w[lane + 32] = -e1 * exp2f(Lend - l1);
-      if (lane == 0) gs.gC = exp2f(Lend);
-      __syncwarp();
-      mbar_arrive(&sm.gfull[g]);
     }
-  } else if (warp == 3) {
-    // ------------------------------------------------------------ scaled-X producer
-    for (int c = 0; c < nch; ++c) {
-      const int s = c % NS, g = c % GS;
-      if (!mbar_wait(&sm.full[s], (c / NS) & 1, wc, W_XH_FULL)) break;
-      if (!mbar_wait(&sm.gfull[g], (c / GS) & 1, wc, W_XH_GFULL)) break;
-      if (c > 0 && !mbar_wait(&sm.dsfull, (c - 1) & 1, wc, W_XH_DSFULL)) break;
-      const uint32_t src = smem_u32(sm.X[s]), dst = smem_u32(sm.Xh);
-      const float* w = sm.gates[g].w;
+    bool ok = true;
+    for (int cb = 0; cb < nch && ok; cb += PD) {
+#pragma unroll
+      for (int k = 0; k < PD; ++k) {
+        const int c = cb + k;
+        if (c >= nch) break;
+        const int s = c % NS, g = c % GS;
+        GateSlot& gs = sm.gates[g];
+        if (gate_warp) {
+          if (!mbar_wait(&sm.gempty[g], ((c / GS) & 1) ^ 1, wc, W_GATE_EMPTY)) { ok = false; break; }
+          const float a0 = ra[k][0], a1 = ra[k][1], e0 = re[k][0], e1 = re[k][1];
+          {  // prefetch the gates of chunk c + PD into this register slot
+            const int t0 = (c + PD) * C + lane, t1 = t0 + 32;
+            ra[k][0] = t0 < T ? p.alpha[gbase + t0] : 1.f;
+            ra[k][1] = t1 < T ? p.alpha[gbase + t1] : 1.f;
+            re[k][0] = t0 < T ? p.eta[gbase + t0] : 0.f;
+            re[k][1] = t1 < T ? p.eta[gbase + t1] : 0.f;
+          }
+          float l0 = fmaxf(log2f(a0), -100.f), l1 = fmaxf(log2f(a1), -100.f);
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const float u0 = __shfl_up_sync(0xffffffffu, l0, o);
+            const float u1 = __shfl_up_sync(0xffffffffu, l1, o);
+            if (lane >= o) {
+              l0 += u0;
+              l1 += u1;
+            }
+          }
+          const float last0 = __shfl_sync(0xffffffffu, l0, 31);
+          l1 += last0;
+          const float Lend = __shfl_sync(0xffffffffu, l1, 31);
+          const float pm0 = __shfl_up_sync(0xffffffffu, l0, 1);
+          const float pm1 = __shfl_up_sync(0xffffffffu, l1, 1);
+          gs.L[lane] = l0;
+          gs.L[lane + 32] = l1;
+          gs.eta[lane] = e0;
+          gs.eta[lane + 32] = e1;
+          gs.gam[lane] = lane == 0 ? 1.f : exp2f(pm0);
+          gs.gam[lane + 32] = exp2f(lane == 0 ? last0 : pm1);
+          gs.w[lane] = -e0 * exp2f(Lend - l0);
+          gs.w[lane + 32] = -e1 * exp2f(Lend - l1);
+          if (lane == 0) gs.gC = exp2f(Lend);
+          __syncwarp();
+          mbar_arrive(&sm.gfull[g]);
+        }
+        if (!mbar_wait(&sm.full[s], (c / NS) & 1, wc, W_XH_FULL)) { ok = false; break; }
+        if (!mbar_wait(&sm.gfull[g], (c / GS) & 1, wc, W_XH_GFULL)) { ok = false; break; }
+        if (c > 0 && !mbar_wait(&sm.dsfull, (c - 1) & 1, wc, W_XH_DSFULL)) { ok = false; break; }
+        const uint32_t src = smem_u32(sm.X[s]), dst = smem_u32(sm.Xh);
 #pragma unroll 4
-      for (int idx = lane; idx < 2 * TILE / 16; idx += 32) {
-        const uint32_t off = idx * 16;
-        const int j = (off & (TILE - 1)) >> 7;  // token row
-        const float wj = w[j];
-        const uint4 v = ld_shared_v4(src + off);
-        st_shared_v4(dst + off, pack_bf16(wj * bf16_lo(v.x), wj * bf16_hi(v.x)),
-                     pack_bf16(wj * bf16_lo(v.y), wj * bf16_hi(v.y)),
-                     pack_bf16(wj * bf16_lo(v.z), wj * bf16_hi(v.z)),
-                     pack_bf16(wj * bf16_lo(v.w), wj * bf16_hi(v.w)));
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&sm.xready);
-        mbar_arrive(&sm.gempty[g]);
+        for (int idx = (warp - 2) * 32 + lane; idx < 2 * TILE / 16; idx += 64) {
+          const uint32_t off = idx * 16;
+          const int j = (off & (TILE - 1)) >> 7;  // token row
+          const __nv_bfloat162 w2 = __float2bfloat162_rn(gs.w[j]);
+          const uint32_t wv = *reinterpret_cast<const uint32_t*>(&w2);
+          uint4 v = ld_shared_v4(src + off);
+          v.x = hmul2_bf16(v.x, wv);
+          v.y = hmul2_bf16(v.y, wv);
+          v.z = hmul2_bf16(v.z, wv);
+          v.w = hmul2_bf16(v.w, wv);
+          st_shared_v4(dst + off, v.x, v.y, v.z, v.w);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&sm.xready);
+          mbar_arrive(&sm.gempty[g]);
+        }
       }
     }
   } else {
@@ -320,46 +351,55 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     for (int e = 0; e < 64; ++e) Sreg[e] = 0.f;
     __nv_bfloat16* yout = p.y + (size_t)bh * T * p.dout + n0 + n;
 
-    for (int c = 0; c < nch; ++c) {
+    // mask of chunk c: P_ij = K_ij (-eta_j) 2^{L_{i-1} - L_j} for j < i
+    auto mask = [&](int c) -> bool {
       const int g = c % GS, b = c & 1;
       const GateSlot& gs = sm.gates[g];
-      if (!mbar_wait(&sm.gfull[g], (c / GS) & 1, wc, W_M_GFULL)) break;
-
-      // ---- mask: P_ij = K_ij (-eta_j) 2^{L_{i-1} - L_j}, j < i
-      if (!mbar_wait(&sm.kfull[b], (c >> 1) & 1, wc, W_M_KFULL)) break;
+      if (!mbar_wait(&sm.gfull[g], (c / GS) & 1, wc, W_M_GFULL)) return false;
+      if (!mbar_wait(&sm.kfull[b], (c >> 1) & 1, wc, W_M_KFULL)) return false;
       tc_fence_after();
-      {
-        float v[32];
-        tmem_ld32(tbase + (b ? COL_K1 : COL_K0) + lane_off + 32 * hh, v);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.kfree[b]);
-        if (lane < 16) {
-          const int i = 16 * q + lane;
-          const float Lm1 = i == 0 ? 0.f : gs.L[i - 1];
-          uint32_t pk[16];
+      float v[32];
+      tmem_ld32(tbase + (b ? COL_K1 : COL_K0) + lane_off + 32 * hh, v);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.kfree[b]);
+      if (lane < 16) {
+        const int i = 16 * q + lane;
+        const float Lm1 = i == 0 ? 0.f : gs.L[i - 1];
+        uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const int j = 32 * hh + e;
-            const float p0 = (j < i) ? v[e] * (-gs.eta[j]) * exp2f(Lm1 - gs.L[j]) : 0.f;
-            const float p1 = (j + 1 < i) ? v[e + 1] * (-gs.eta[j + 1]) * exp2f(Lm1 - gs.L[j + 1]) : 0.f;
-            pk[e >> 1] = pack_bf16(p0, p1);
-          }
-          const uint32_t prow = smem_u32(sm.P);
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc)
-            st_shared_v4(prow + sw128_off(i, 4 * hh + cc), pk[4 * cc], pk[4 * cc + 1],
-                         pk[4 * cc + 2], pk[4 * cc + 3]);
+        for (int e = 0; e < 32; e += 2) {
+          const int j = 32 * hh + e;
+          const float f0 = exp2f(fminf(Lm1 - gs.L[j], 0.f));
+          const float f1 = exp2f(fminf(Lm1 - gs.L[j + 1], 0.f));
+          const float p0 = (j < i) ? v[e] * (-gs.eta[j]) * f0 : 0.f;
+          const float p1 = (j + 1 < i) ? v[e + 1] * (-gs.eta[j + 1]) * f1 : 0.f;
+          pk[e >> 1] = pack_bf16(p0, p1);
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.pready);
+        const uint32_t prow = smem_u32(sm.P);
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+          st_shared_v4(prow + sw128_off(i, 4 * hh + cc), pk[4 * cc], pk[4 * cc + 1],
+                       pk[4 * cc + 2], pk[4 * cc + 3]);
       }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.pready);
+      return true;
+    };
 
-      // ---- state: S <- 2^{L_{C-1}} S + dS ; bf16 copy for the next chunk
+    bool ok = nch > 0 ? mask(0) : true;
+    for (int c = 0; c < nch && ok; ++c) {
+      const int g = c % GS, b = c & 1;
+      const GateSlot& gs = sm.gates[g];
+
+      // ---- state: S <- 2^{L_{C-1}} S + dS ; bf16 copy into buffer wb = (c+1)&1, which
+      //      the S X^T product of chunk c - 1 read (one barrier pair per buffer, so a
+      //      parity wait can never see a phase from the other buffer's traffic)
+      const int wb = (c + 1) & 1;
       if (!mbar_wait(&sm.dsfull, c & 1, wc, W_M_DSFULL)) break;
-      if (!mbar_wait(&sm.sfree, c & 1, wc, W_M_SFREE)) break;
+      if (c > 0 && !mbar_wait(&sm.sfree[wb], ((c - 1) >> 1) & 1, wc, W_M_SFREE)) break;
       tc_fence_after();
       {
         float v0[32], v1[32];
@@ -375,7 +415,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           Sreg[e] = fmaf(gC, Sreg[e], v0[e]);
           Sreg[32 + e] = fmaf(gC, Sreg[32 + e], v1[e]);
         }
-        const uint32_t srow = smem_u32(sm.S[hh]);
+        const uint32_t srow = smem_u32(sm.S[wb][hh]);
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc)
           st_shared_v4(srow + sw128_off(n, cc), pack_bf16(Sreg[8 * cc], Sreg[8 * cc + 1]),
@@ -384,8 +424,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                        pack_bf16(Sreg[8 * cc + 6], Sreg[8 * cc + 7]));
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.sready);
+        if (lane == 0) mbar_arrive(&sm.sready[wb]);
       }
+
+      // ---- mask of the next chunk (keeps the MMA stream fed while we store y)
+      if (c + 1 < nch && !mask(c + 1)) break;
 
       // ---- output: y_i = Y1^T[n][i] + 2^{L_{i-1}} Y2^T[n][i]
       if (!mbar_wait(&sm.yfull[b], (c >> 1) & 1, wc, W_M_YFULL)) break;
@@ -400,10 +443,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (lane == 0) mbar_arrive(&sm.yfree[b]);
         const int ib = 32 * hh;
         const int tb = c * C + ib;
+        if (tb + 32 <= T) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          if (tb + e < T)
+          for (int e = 0; e < 32; ++e)
             yout[(size_t)(tb + e) * p.dout] = __float2bfloat16_rn(fmaf(gs.gam[ib + e], s2[e], a[e]));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (tb + e < T)
+              yout[(size_t)(tb + e) * p.dout] =
+                  __float2bfloat16_rn(fmaf(gs.gam[ib + e], s2[e], a[e]));
         }
       }
       __syncwarp();
