@@ -98,3 +98,93 @@ def test_tc_fwd_timeout_path_reports_and_recovers():
     y = tw.gradlev_scan_fwd(t["x"], t["g"], t["eta"], t["alpha"], t["W0"], workspace=ws)
     assert tw.gradlev_device_status(ws) == 0
     assert rel_err(to_numpy(y), oracle_fwd(d)) <= TOL["bf16"]
+
+
+# ------------------------------------------------------------------ reverse scan
+
+BWD_OUTS = ("dx", "dg", "deta", "dalpha", "dW0")
+
+
+def gpu_fwd_bwd(d, use_ckpt=True):
+    import token_weight_scans_b200 as tw
+    t = to_device(d, "bf16")
+    B, H, T, di = t["x"].shape
+    do = t["g"].shape[-1]
+    ws = torch.empty(tw.gradlev_scan_workspace_bytes(B, H, T, di, do, tw.BF16, 1),
+                     dtype=torch.uint8, device="cuda")
+    ck = None
+    if use_ckpt:
+        ck = torch.empty(tw.gradlev_scan_ckpt_bytes(B, H, T, di, do, tw.BF16), dtype=torch.uint8,
+                         device="cuda")
+    y = tw.gradlev_scan_fwd(t["x"], t["g"], t["eta"], t["alpha"], t["W0"], ckpt=ck, workspace=ws)
+    assert tw.gradlev_device_status(ws) == 0
+    out = tw.gradlev_scan_bwd(t["x"], t["g"], t["eta"], t["alpha"], t["W0"], t["dy"], ckpt=ck,
+                              workspace=ws)
+    assert tw.gradlev_device_status(ws) == 0, "device-side wait timed out"
+    res = {k: to_numpy(v) for k, v in out.items()}
+    res["y"] = to_numpy(y)
+    return res
+
+
+def oracle_fwd_bwd(d):
+    d64 = {k: v.astype(np.float64) for k, v in d.items()}
+    o = oracle.bwd(d64["x"], d64["g"], d64["eta"], d64["alpha"], d64["W0"], d64["dy"])
+    o["y"] = oracle.fwd(d64["x"], d64["g"], d64["eta"], d64["alpha"], d64["W0"])
+    return o
+
+
+def check_all(got, ref, ctx):
+    errs = {k: rel_err(got[k], ref[k]) for k in ("y",) + BWD_OUTS}
+    bad = {k: e for k, e in errs.items() if not e <= TOL["bf16"]}
+    assert not bad, f"{ctx}: {errs}"
+
+
+@pytest.mark.parametrize("T", [1, 2, 63, 64, 65, 128, 200])
+def test_tc_bwd_ragged_lengths(T):
+    d = inputs.draw(2, 2, T, 128, 128, dtype="bf16", alpha_mode="log_uniform", seed=500 + T)
+    check_all(gpu_fwd_bwd(d), oracle_fwd_bwd(d), f"T={T}")
+
+
+@pytest.mark.parametrize("mode", ["sigmoid", "log_uniform"])
+def test_tc_bwd_several_chunks(mode):
+    d = inputs.draw(3, 2, 700, 128, 128, dtype="bf16", alpha_mode=mode, seed=51)
+    check_all(gpu_fwd_bwd(d), oracle_fwd_bwd(d), mode)
+
+
+def test_tc_bwd_degenerate_gates():
+    d = inputs.draw(2, 2, 300, 128, 128, dtype="bf16", seed=52)
+    d["alpha"][..., ::9] = 0.0
+    d["alpha"][..., 4::9] = 1.0
+    d["eta"][..., 7::13] = 0.0
+    check_all(gpu_fwd_bwd(d), oracle_fwd_bwd(d), "degenerate gates")
+
+
+def test_tc_bwd_own_state_sweep_matches_checkpoints():
+    d = inputs.draw(2, 2, 333, 128, 128, dtype="bf16", alpha_mode="log_uniform", seed=53)
+    a = gpu_fwd_bwd(d, use_ckpt=True)
+    b = gpu_fwd_bwd(d, use_ckpt=False)
+    for k in BWD_OUTS:
+        assert np.array_equal(a[k], b[k]), k
+
+
+def test_tc_bwd_deterministic():
+    d = inputs.draw(2, 3, 260, 128, 128, dtype="bf16", alpha_mode="log_uniform", seed=54)
+    a = gpu_fwd_bwd(d)
+    b = gpu_fwd_bwd(d)
+    for k in a:
+        assert np.array_equal(a[k], b[k]), k
+
+
+def test_tc_bwd_bit_exact_integer_inputs():
+    rng = np.random.default_rng(5)
+    B, H, T, di, do = 2, 2, 150, 128, 128
+    sp = lambda *s, p=0.03: (rng.integers(-1, 2, s) * (rng.random(s) < p)).astype(np.float32)
+    d = {"x": sp(B, H, T, di), "g": sp(B, H, T, do, p=0.05),
+         "eta": np.full((B, H, T), 0.125, np.float32), "alpha": np.ones((B, H, T), np.float32),
+         "W0": sp(H, do, di, p=0.05), "dy": sp(B, H, T, do, p=0.05)}
+    ref = oracle_fwd_bwd(d)
+    for k in ("y", "dx", "dg"):
+        assert np.array_equal(inputs.round_bf16(ref[k]).astype(np.float64), ref[k]), k
+    got = gpu_fwd_bwd(d)
+    for k in ("y",) + BWD_OUTS:
+        assert np.array_equal(got[k], ref[k]), (k, rel_err(got[k], ref[k]))

@@ -1,0 +1,29 @@
+// Internal dispatch shared by the C entry points (gradlev_abi.cu, gradlev_noalloc.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "gradlev.h"
+
+namespace gradlev {
+
+constexpr size_t kStatusBytes = 256;  // device status word + alignment pad
+
+// Which kernel family serves a shape: the tcgen05 kernels for bf16 with
+// d_in = d_out = 128, the CUDA-core kernels otherwise.
+bool use_tc(int din, int dout, gradlev_dtype dt);
+
+// Bytes of the reverse scan's scratch: status word, per-scan dW0 partials and,
+// when `own_states`, the chunk-start states of a forward state sweep.
+size_t bwd_scratch_bytes(int B, int H, int T, int din, int dout, gradlev_dtype dt,
+                         bool own_states);
+
+// Launch the reverse scan with its scratch at `ws` (bwd_scratch_bytes(.., ckpt == NULL)
+// bytes, 256-byte aligned). Shapes and pointers must already be validated.
+gradlev_status bwd_run(int B, int H, int T, int din, int dout, gradlev_dtype dt, const void* x,
+                       const void* g, const float* eta, const float* alpha, const float* W0,
+                       const void* dy, void* dx, void* dg, float* d_eta, float* d_alpha,
+                       float* dW0, const void* ckpt, char* ws, cudaStream_t st);
+
+}  // namespace gradlev

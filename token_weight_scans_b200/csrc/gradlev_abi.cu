@@ -1,11 +1,20 @@
 // Host side of the C ABI declared in include/gradlev.h: argument validation,
 // workspace sizing and kernel dispatch. No device memory is allocated here.
+//
+// Kernel families:
+//   * tcgen05 kernels (scan_tc_fwd.cu, scan_tc_bwd.cu): bf16 I/O, d_in = d_out = 128;
+//   * CUDA-core kernels (scan_ffma.cu): everything else that is supported
+//     (float32 I/O, or bf16 with d_in * d_out <= 16384).
+// The two families exchange state checkpoints in different formats; a
+// checkpoint buffer written by gradlev_scan_fwd is consumed by gradlev_scan_bwd
+// of the same shape and dtype, which always picks the same family.
 
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <string.h>
 
 #include "common.cuh"
+#include "dispatch.h"
 #include "gradlev.h"
 #include "scan_ffma.h"
 #include "scan_tc.h"
@@ -20,16 +29,78 @@ static int g_inject = 0;
 static uint64_t g_inject_timeout_ns = 0;
 static constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // bound of device-side waits
 
-static constexpr size_t kStatusBytes = 256;  // status word + alignment pad
-
 static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool use_tc(int din, int dout, gradlev_dtype dt) {
+  return dt == GRADLEV_BF16 && tc::bwd_shape_ok(din, dout);
+}
 
 static gradlev_status check_shape(int B, int H, int T, int din, int dout, gradlev_dtype dt) {
   if (B <= 0 || H <= 0 || T <= 0 || din <= 0 || dout <= 0) return GRADLEV_ERR_INVALID_ARG;
   if (dt != GRADLEV_F32 && dt != GRADLEV_BF16) return GRADLEV_ERR_INVALID_ARG;
   if ((long long)B * H * T >= (1LL << 31)) return GRADLEV_ERR_UNSUPPORTED;
-  if (!ffma::shape_ok(din, dout)) return GRADLEV_ERR_UNSUPPORTED;
+  if (!use_tc(din, dout, dt) && !ffma::shape_ok(din, dout)) return GRADLEV_ERR_UNSUPPORTED;
   return GRADLEV_OK;
+}
+
+static size_t ckpt_bytes_of(int B, int H, int T, int din, int dout, gradlev_dtype dt) {
+  return use_tc(din, dout, dt) ? tc::ckpt_bytes(B, H, T, din, dout)
+                               : ffma::ckpt_bytes(B, H, T, din, dout);
+}
+
+size_t bwd_scratch_bytes(int B, int H, int T, int din, int dout, gradlev_dtype dt,
+                         bool own_states) {
+  size_t ws = kStatusBytes + align_up((size_t)B * H * din * dout * sizeof(float), 256);
+  if (own_states) ws += align_up(ckpt_bytes_of(B, H, T, din, dout, dt), 256);
+  return ws;
+}
+
+static gradlev_status launch_fwd_impl(int B, int H, int T, int din, int dout, gradlev_dtype dt,
+                                      const void* x, const void* g, const float* eta,
+                                      const float* alpha, const float* W0, void* y, void* ckpt,
+                                      DeviceStatus* status, cudaStream_t st) {
+  if (use_tc(din, dout, dt)) {
+    const int inject = y ? g_inject : 0;
+    const uint64_t tmo = inject ? g_inject_timeout_ns : kWaitTimeoutNs;
+    if (y) g_inject = 0;
+    tc::TcFwdParams prm{B, H, T, din, dout, eta, alpha, W0, static_cast<__nv_bfloat16*>(y),
+                        static_cast<__nv_bfloat16*>(ckpt), status, tmo, inject};
+    return tc::launch_fwd(prm, x, g, st) == cudaSuccess ? GRADLEV_OK : GRADLEV_ERR_CUDA;
+  }
+  ffma::FwdArgs a{B, H, T, din, dout, x, g, eta, alpha, W0, y, static_cast<float*>(ckpt)};
+  return ffma::launch_fwd(a, dt == GRADLEV_BF16, st) == cudaSuccess ? GRADLEV_OK
+                                                                   : GRADLEV_ERR_CUDA;
+}
+
+gradlev_status bwd_run(int B, int H, int T, int din, int dout, gradlev_dtype dt, const void* x,
+                       const void* g, const float* eta, const float* alpha, const float* W0,
+                       const void* dy, void* dx, void* dg, float* d_eta, float* d_alpha,
+                       float* dW0, const void* ckpt, char* ws, cudaStream_t st) {
+  DeviceStatus* status = reinterpret_cast<DeviceStatus*>(ws);
+  float* dW0_part = reinterpret_cast<float*>(ws + kStatusBytes);
+  void* own = ws + kStatusBytes + align_up((size_t)B * H * din * dout * sizeof(float), 256);
+  if (cudaMemsetAsync(status, 0, sizeof(DeviceStatus), st) != cudaSuccess)
+    return GRADLEV_ERR_CUDA;
+  const void* states = ckpt;
+  if (!states) {
+    gradlev_status s = launch_fwd_impl(B, H, T, din, dout, dt, x, g, eta, alpha, W0, nullptr,
+                                       own, status, st);
+    if (s != GRADLEV_OK) return s;
+    states = own;
+  }
+  if (use_tc(din, dout, dt)) {
+    tc::TcBwdParams prm{B, H, T, din, dout, eta, alpha, W0,
+                        static_cast<__nv_bfloat16*>(dx), static_cast<__nv_bfloat16*>(dg),
+                        d_eta, d_alpha, dW0_part, status, kWaitTimeoutNs};
+    if (tc::launch_bwd(prm, x, g, dy, states, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
+    if (ffma::launch_reduce_dW0(dW0_part, dW0, B, H, din * dout, st) != cudaSuccess)
+      return GRADLEV_ERR_CUDA;
+    return GRADLEV_OK;
+  }
+  ffma::BwdArgs a{B, H, T, din, dout, x, g, eta, alpha, W0, dy, dx, dg, d_eta, d_alpha, dW0,
+                  static_cast<const float*>(states), dW0_part};
+  return ffma::launch_bwd(a, dt == GRADLEV_BF16, st) == cudaSuccess ? GRADLEV_OK
+                                                                   : GRADLEV_ERR_CUDA;
 }
 
 static bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
@@ -58,18 +129,13 @@ gradlev_status gradlev_scan_supported(int B, int H, int T, int d_in, int d_out, 
 
 size_t gradlev_scan_ckpt_bytes(int B, int H, int T, int d_in, int d_out, gradlev_dtype dt) {
   if (check_shape(B, H, T, d_in, d_out, dt) != GRADLEV_OK) return 0;
-  return ffma::ckpt_bytes(B, H, T, d_in, d_out);
+  return ckpt_bytes_of(B, H, T, d_in, d_out, dt);
 }
 
 size_t gradlev_scan_workspace_bytes(int B, int H, int T, int d_in, int d_out, gradlev_dtype dt,
                                     int is_bwd) {
   if (check_shape(B, H, T, d_in, d_out, dt) != GRADLEV_OK) return 0;
-  size_t ws = kStatusBytes;
-  if (is_bwd) {
-    ws += align_up(ffma::dW0_part_bytes(B, H, d_in, d_out), 256);
-    ws += align_up(ffma::ckpt_bytes(B, H, T, d_in, d_out), 256);
-  }
-  return ws;
+  return is_bwd ? bwd_scratch_bytes(B, H, T, d_in, d_out, dt, true) : kStatusBytes;
 }
 
 gradlev_status gradlev_scan_fwd(int B, int H, int T, int d_in, int d_out, gradlev_dtype dt,
@@ -87,27 +153,10 @@ gradlev_status gradlev_scan_fwd(int B, int H, int T, int d_in, int d_out, gradle
     return GRADLEV_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   t_launches = 0;
-  if (cudaMemsetAsync(workspace, 0, sizeof(DeviceStatus), st) != cudaSuccess)
+  DeviceStatus* status = static_cast<DeviceStatus*>(workspace);
+  if (cudaMemsetAsync(status, 0, sizeof(DeviceStatus), st) != cudaSuccess)
     return GRADLEV_ERR_CUDA;
-  if (dt == GRADLEV_BF16 && tc::fwd_shape_ok(d_in, d_out)) {
-    // tensor-core forward; the reverse scan of this build consumes the CUDA-core
-    // checkpoint format, which a state-only CUDA-core sweep writes when requested
-    const int inject = g_inject;
-    const uint64_t tmo = inject ? g_inject_timeout_ns : kWaitTimeoutNs;
-    g_inject = 0;
-    tc::TcFwdParams prm{B, H, T, d_in, d_out, eta, alpha, W0, static_cast<__nv_bfloat16*>(y),
-                        static_cast<DeviceStatus*>(workspace), tmo, inject};
-    if (tc::launch_fwd(prm, x, g, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
-    if (ckpt) {
-      ffma::FwdArgs a{B, H, T, d_in, d_out, x, g, eta, alpha, W0, nullptr,
-                      static_cast<float*>(ckpt)};
-      if (ffma::launch_fwd(a, true, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
-    }
-    return GRADLEV_OK;
-  }
-  ffma::FwdArgs a{B, H, T, d_in, d_out, x, g, eta, alpha, W0, y, static_cast<float*>(ckpt)};
-  if (ffma::launch_fwd(a, dt == GRADLEV_BF16, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
-  return GRADLEV_OK;
+  return launch_fwd_impl(B, H, T, d_in, d_out, dt, x, g, eta, alpha, W0, y, ckpt, status, st);
 }
 
 gradlev_status gradlev_scan_bwd(int B, int H, int T, int d_in, int d_out, gradlev_dtype dt,
@@ -128,25 +177,9 @@ gradlev_status gradlev_scan_bwd(int B, int H, int T, int d_in, int d_out, gradle
     return GRADLEV_ERR_INVALID_ARG;
   if (ws_bytes < gradlev_scan_workspace_bytes(B, H, T, d_in, d_out, dt, 1))
     return GRADLEV_ERR_WORKSPACE;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   t_launches = 0;
-  char* wsb = static_cast<char*>(workspace);
-  float* dW0_part = reinterpret_cast<float*>(wsb + kStatusBytes);
-  float* own_ckpt = reinterpret_cast<float*>(
-      wsb + kStatusBytes + align_up(ffma::dW0_part_bytes(B, H, d_in, d_out), 256));
-  if (cudaMemsetAsync(workspace, 0, sizeof(DeviceStatus), st) != cudaSuccess)
-    return GRADLEV_ERR_CUDA;
-  const bool bf16 = dt == GRADLEV_BF16;
-  const float* states = static_cast<const float*>(ckpt);
-  if (!states) {
-    ffma::FwdArgs f{B, H, T, d_in, d_out, x, g, eta, alpha, W0, nullptr, own_ckpt};
-    if (ffma::launch_fwd(f, bf16, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
-    states = own_ckpt;
-  }
-  ffma::BwdArgs a{B, H, T, d_in, d_out, x, g, eta, alpha, W0, dy, dx, dg, d_eta, d_alpha, dW0,
-                  states, dW0_part};
-  if (ffma::launch_bwd(a, bf16, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
-  return GRADLEV_OK;
+  return bwd_run(B, H, T, d_in, d_out, dt, x, g, eta, alpha, W0, dy, dx, dg, d_eta, d_alpha,
+                 dW0, ckpt, static_cast<char*>(workspace), static_cast<cudaStream_t>(stream));
 }
 
 gradlev_status gradlev_device_status(const void* workspace, void* stream) {

@@ -23,14 +23,13 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "dispatch.h"
 #include "gradlev.h"
-#include "scan_ffma.h"
 
 namespace gradlev {
 namespace {
 
 constexpr size_t kScratchBytes = GRADLEV_NOALLOC_SCRATCH_BYTES;
-constexpr size_t kStatus = 256;
 constexpr int kMaxDevices = 64;
 
 // The scratch itself. Every call on a device shares it; it keeps the last
@@ -39,8 +38,6 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 std::mutex g_mu;
 void* g_addr[kMaxDevices] = {};
-
-size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
 // Device address of g_noalloc_scratch on the current device (looked up once per device).
 gradlev_status scratch_address(void** out) {
@@ -72,9 +69,8 @@ extern "C" GRADLEV_API gradlev_status gradlev_scan_bwd_noalloc(
   // Shape and size checks first: they need no GPU and launch nothing.
   gradlev_status s = gradlev_scan_supported(B, H, T, d_in, d_out, dt);
   if (s != GRADLEV_OK) return s;
-  const size_t part = align256(ffma::dW0_part_bytes(B, H, d_in, d_out));
-  const size_t states = ckpt ? 0 : align256(ffma::ckpt_bytes(B, H, T, d_in, d_out));
-  if (kStatus + part + states > kScratchBytes) return GRADLEV_ERR_WORKSPACE;
+  if (bwd_scratch_bytes(B, H, T, d_in, d_out, dt, ckpt == nullptr) > kScratchBytes)
+    return GRADLEV_ERR_WORKSPACE;
   if (!x || !g || !eta || !alpha || !W0 || !dy || !dx || !dg || !d_eta || !d_alpha || !dW0)
     return GRADLEV_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(g, 16) || !aligned(dy, 16) || !aligned(dx, 16) ||
@@ -86,23 +82,8 @@ extern "C" GRADLEV_API gradlev_status gradlev_scan_bwd_noalloc(
   void* base = nullptr;
   s = scratch_address(&base);
   if (s != GRADLEV_OK) return s;
-  char* ws = static_cast<char*>(base);
-  float* dW0_part = reinterpret_cast<float*>(ws + kStatus);
-  float* own_states = reinterpret_cast<float*>(ws + kStatus + part);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-
-  // The status word must start at zero; the dW0 partials and the states are
+  // The status word is cleared by bwd_run; the dW0 partials and the states are
   // fully overwritten by the kernels before they are read.
-  if (cudaMemsetAsync(ws, 0, sizeof(DeviceStatus), st) != cudaSuccess) return GRADLEV_ERR_CUDA;
-  const bool bf16 = dt == GRADLEV_BF16;
-  const float* S = static_cast<const float*>(ckpt);
-  if (!S) {
-    ffma::FwdArgs f{B, H, T, d_in, d_out, x, g, eta, alpha, W0, nullptr, own_states};
-    if (ffma::launch_fwd(f, bf16, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
-    S = own_states;
-  }
-  ffma::BwdArgs a{B, H, T, d_in, d_out, x, g, eta, alpha, W0, dy, dx, dg, d_eta, d_alpha, dW0,
-                  S, dW0_part};
-  if (ffma::launch_bwd(a, bf16, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
-  return GRADLEV_OK;
+  return bwd_run(B, H, T, d_in, d_out, dt, x, g, eta, alpha, W0, dy, dx, dg, d_eta, d_alpha,
+                 dW0, ckpt, static_cast<char*>(base), static_cast<cudaStream_t>(stream));
 }

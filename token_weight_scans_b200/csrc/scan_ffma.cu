@@ -560,6 +560,15 @@ static cudaError_t launch_bwd_t(const BwdArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+cudaError_t launch_reduce_dW0(const float* part, float* dW0, int B, int H, int dd,
+                              cudaStream_t st) {
+  const size_t n = (size_t)H * dd;
+  const int blocks = (int)((n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184);
+  reduce_dW0_kernel<<<blocks, 256, 0, st>>>(part, dW0, B, H, dd);
+  count_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_fwd(const FwdArgs& a, bool bf16, cudaStream_t st) {
   return bf16 ? launch_fwd_t<__nv_bfloat16>(a, st) : launch_fwd_t<float>(a, st);
 }

@@ -40,6 +40,9 @@ size_t ckpt_bytes(int B, int H, int T, int din, int dout);
 size_t dW0_part_bytes(int B, int H, int din, int dout);
 cudaError_t launch_fwd(const FwdArgs& a, bool bf16, cudaStream_t st);
 cudaError_t launch_bwd(const BwdArgs& a, bool bf16, cudaStream_t st);
+// dW0[h] = sum over b of part[b][h] (fixed order); used by both kernel families
+cudaError_t launch_reduce_dW0(const float* part, float* dW0, int B, int H, int dd,
+                              cudaStream_t st);
 
 }  // namespace ffma
 }  // namespace gradlev

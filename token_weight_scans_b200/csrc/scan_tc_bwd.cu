@@ -1,0 +1,682 @@
+// Tensor-core (tcgen05/TMEM) reverse GradLev scan for bf16 I/O, d_in = d_out = 128.
+//
+// Reverse-mode derivative of S_{t+1} = alpha_t S_t - eta_t g_t x_t^T,
+// y_t = (W0 + S_t) x_t (Cognaptus, "Parallelize the Training, Keep the Learning
+// Serial", section "Once the gradient signals are known, the weight trajectory
+// becomes parallelizable"; GradLev abstract: the reverse backpropagation is a
+// scan too). With u = dL/dy and the state adjoint Lam_t = alpha_t Lam_{t+1} + u_t x_t^T:
+//   dx_t = (W0 + S_t)^T u_t - eta_t Lam_{t+1}^T g_t,  dg_t = -eta_t Lam_{t+1} x_t,
+//   deta_t = -g_t . Lam_{t+1} x_t,  dalpha_t = <Lam_{t+1}, S_t>,  dW0 = sum u_t x_t^T.
+//
+// One CTA per (b, h) walks the 64-token chunks backwards, carrying Lam (fp32 in
+// registers, bf16 copy in shared memory). The chunk-start state S_in comes from
+// the bf16 checkpoints of the forward scan. Inside a chunk (local i, with
+// L_j = sum_{r<=j} log2 alpha, gam_i = 2^{L_{i-1}}, del_i = 2^{L_{C-1}-L_i},
+// a_ij = -eta_j 2^{L_{i-1}-L_j} (j<i), b_is = 2^{L_{s-1}-L_i} (s>i)):
+//   r_i  = del_i Lam x_i + sum_{s>i} b_is (x_s.x_i) u_s
+//   dx_i = W0^T u_i + gam_i S_in^T u_i - eta_i del_i Lam^T g_i + sum_j Z_ij x_j
+//   Z_ij = a_ij (u_i.g_j) (j<i),  -eta_i b_ij (g_i.u_j) (j>i)
+//   deta_i = -(del_i q_i + t_i), q_i = g_i^T Lam x_i, t_i = sum_{s>i} b_is (x_i.x_s)(g_i.u_s)
+//   dalpha_i = gam_i del_i <Lam,S_in> + del_i sum_{j<i} a_ij q_j + gam_i sum_{s>i} b_is p_s
+//              + sum_{j<i} a_ij V_ij,  p_s = u_s^T S_in x_s,
+//   V_ij = sum_{s>i} b_is Q_js, Q_js = (u_s.g_j)(x_s.x_j) (j<s)
+//   Lam <- 2^{L_{C-1}} Lam + sum_s gam_s u_s x_s^T ;  dW0 += sum_s u_s x_s^T
+// (dalpha is the exact four-term expansion of <Lam_{i+1}, S_i>; no division by alpha.)
+//
+// Products (d on the 128 TMEM lanes, tokens on the columns; M=64 ones use the
+// two 16-lane halves of each TMEM sub-partition):
+//   phase 1: K = X X^T | Kug = U G^T (M=64), KugT = G U^T (M=64), dW0 += U^T X,
+//            DXb^T = S_in^T U^T, R1^T = Lam X^T
+//   phase 2: V^T = Bm Q^T (M=64), RI^T = U^T Ar^T, DXa^T = W0^T U^T + X^T Z^T + Lam^T Gs^T
+//   phase 3: dLam = U^T Xg
+// where Ar, Z, Q^T, Bm are built by the math warps from K, Kug, KugT into the
+// shared memory that held S_in, Gs = diag(-eta del) G and Xg = diag(gam) X are
+// written in place once their unscaled uses are over.
+//
+// Warp roles (12 warps): 0 TMA producer, 1 MMA issuer + TMEM owner, 2 gate
+// prep, 3 idle helper, 4..11 two math warpgroups (warpgroup h: tokens
+// [32h, 32h+32) of each chunk and state columns [64h, 64h+64)).
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "scan_tc.h"
+#include "sm100.cuh"
+
+namespace gradlev {
+namespace tc {
+
+bool make_map_bf16_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                      uint32_t box1);
+
+using namespace sm100;
+
+namespace {
+
+constexpr int C = kChunk;       // 64 tokens per chunk
+constexpr int NS = 2;           // stages of the X, G, U tiles
+constexpr int GS = 2;           // gate slots
+constexpr int NTHREADS = 384;
+constexpr int TILE = C * 128;   // [64 rows x 128 B] swizzled block
+constexpr int BIG = 128 * 128;  // [128 rows x 128 B] swizzled block
+
+// TMEM columns (512 allocated)
+constexpr uint32_t COL_KK = 0;    // K (lanes 0-15 of each sub-partition) | Kug (lanes 16-31)
+constexpr uint32_t COL_KT = 64;   // KugT (lanes 0-15) | V^T (lanes 16-31)
+constexpr uint32_t COL_R = 128;   // R1^T, then RI^T
+constexpr uint32_t COL_D = 192;   // DXb^T, then DXa^T
+constexpr uint32_t COL_DL = 256;  // dLam (128 columns)
+constexpr uint32_t COL_W = 384;   // dW0 accumulator (128 columns)
+constexpr uint32_t LANE16 = 16u << 16;
+
+// chunk-by-chunk matrices built by the math warps, aliased onto the S_in tile
+constexpr int CC_AR = 0, CC_Z = TILE, CC_QT = 2 * TILE, CC_BM = 3 * TILE;
+
+struct GateSlot {
+  float L[C];
+  float eta[C];
+  float gam[C];
+  float del[C];
+  float gC;
+  float pad[3];
+};
+
+struct Smem {
+  uint8_t X[NS][2 * TILE];    // [s rows][k]: k-blocks
+  uint8_t G[NS][2 * TILE];    // [s rows][n]: n-blocks
+  uint8_t U[NS][2 * TILE];    // [s rows][n]
+  uint8_t Sin[2 * BIG];       // [k-block][n rows x 128 B]; then Ar | Z | Q^T | Bm
+  uint8_t W0[2 * BIG];        // [k-block][n rows x 128 B]
+  uint8_t Lb[2 * BIG];        // bf16 Lam, [k-block][n rows x 128 B]
+  GateSlot gates[GS];
+  float redq[4][C], redp[4][C];
+  float tv[2][C], hv[2][C];
+  float qv[C], pv[C];
+  float ered[8];
+  uint64_t xfull[NS], xempty[NS];
+  uint64_t gfull[GS], gempty[GS];
+  uint64_t sfull, sempty;
+  uint64_t ccfull, b1full, b2full, b3full;
+  uint64_t m1done, m2done, m3done, xscaled, lbready, done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
+
+enum : uint32_t {
+  W_TMA_XEMPTY = 0x001, W_TMA_SEMPTY, W_TMA_DRAIN,
+  W_MMA_XFULL = 0x101, W_MMA_M2, W_MMA_SFULL, W_MMA_LB, W_MMA_M1, W_MMA_XS, W_MMA_M3,
+  W_MMA_DONE,
+  W_GATE_EMPTY = 0x201,
+  W_M_GFULL = 0x401, W_M_CC, W_M_B1, W_M_B2, W_M_B3,
+};
+
+__device__ __forceinline__ void named_sync_math() {
+  asm volatile("bar.sync 1, 256;" ::: "memory");
+}
+
+// Element (row, col) of a [rows x 128 B] swizzled bf16 block (col < 64).
+__device__ __forceinline__ uint32_t sw_elem(uint32_t base, uint32_t row, uint32_t col) {
+  return base + sw128_off(row, col >> 3) + ((col & 7) << 1);
+}
+
+__device__ __forceinline__ float lds_bf16(uint32_t addr) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr) : "memory");
+  return __uint_as_float(((uint32_t)v) << 16);
+}
+
+__device__ __forceinline__ void sts_bf16(uint32_t addr, float f) {
+  const __nv_bfloat16 b = __float2bfloat16_rn(f);
+  const unsigned short v = *reinterpret_cast<const unsigned short*>(&b);
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+}
+
+// Sum of v[0..31] over the 32 lanes of the warp; lane l returns the total of index l.
+__device__ __forceinline__ float reduce_scatter32(float (&v)[32], int lane) {
+  float w16[16], w8[8], w4[4], w2[2];
+  const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4, b1 = lane & 2, b0 = lane & 1;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const float send = b4 ? v[k] : v[k + 16];
+    const float keep = b4 ? v[k + 16] : v[k];
+    w16[k] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float send = b3 ? w16[k] : w16[k + 8];
+    const float keep = b3 ? w16[k + 8] : w16[k];
+    w8[k] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float send = b2 ? w8[k] : w8[k + 4];
+    const float keep = b2 ? w8[k + 4] : w8[k];
+    w4[k] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+  }
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const float send = b1 ? w4[k] : w4[k + 2];
+    const float keep = b1 ? w4[k + 2] : w4[k];
+    w2[k] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+  }
+  const float send = b0 ? w2[0] : w2[1];
+  const float keep = b0 ? w2[1] : w2[0];
+  return keep + __shfl_xor_sync(0xffffffffu, send, 1);
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    bwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmG,
+               const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmS,
+               TcBwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.x, h = bh % p.H;
+  const int T = p.T;
+  const int nch = (T + C - 1) / C;
+  const WaitCtx wc{&sm.abort, p.status, p.timeout_ns};
+
+  if (threadIdx.x == 0) {
+    sm.abort = 0;
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&sm.xfull[s], 1);
+      mbar_init(&sm.xempty[s], 1);
+    }
+    for (int g = 0; g < GS; ++g) {
+      mbar_init(&sm.gfull[g], 32);
+      mbar_init(&sm.gempty[g], 8);
+    }
+    mbar_init(&sm.sfull, 1);
+    mbar_init(&sm.sempty, 1);
+    mbar_init(&sm.ccfull, 1);
+    mbar_init(&sm.b1full, 1);
+    mbar_init(&sm.b2full, 1);
+    mbar_init(&sm.b3full, 1);
+    mbar_init(&sm.m1done, 8);
+    mbar_init(&sm.m2done, 8);
+    mbar_init(&sm.m3done, 8);
+    mbar_init(&sm.xscaled, 8);
+    mbar_init(&sm.lbready, 8);
+    mbar_init(&sm.done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmX);
+    prefetch_tmap(&tmG);
+    prefetch_tmap(&tmU);
+    prefetch_tmap(&tmS);
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (warp >= 4) {
+    // W0 -> bf16 swizzled [k-block][n rows]; Lam_T = 0
+    const int t = threadIdx.x - 128;
+    const float* W0 = p.W0 + (size_t)h * 128 * 128;
+    for (int idx = t; idx < 128 * 16; idx += 256) {
+      const int n = idx >> 4, ck = idx & 15;
+      const int kb = ck >> 3, c = ck & 7;
+      const float4 a = *reinterpret_cast<const float4*>(W0 + (size_t)n * 128 + ck * 8);
+      const float4 b = *reinterpret_cast<const float4*>(W0 + (size_t)n * 128 + ck * 8 + 4);
+      st_shared_v4(smem_u32(sm.W0 + kb * BIG) + sw128_off(n, c), pack_bf16(a.x, a.y),
+                   pack_bf16(a.z, a.w), pack_bf16(b.x, b.y), pack_bf16(b.z, b.w));
+      st_shared_v4(smem_u32(sm.Lb + kb * BIG) + sw128_off(n, c), 0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = sm.tmem_base;
+
+  if (warp < 4) {
+    if (warp == 0) {
+      // ---------------------------------------------------------- TMA producer
+      if (lane == 0) {
+        int xi = 0, si = 0;
+        for (int it = 0; it < nch; ++it) {
+          const int c = nch - 1 - it, st = it % NS;
+          if (!mbar_wait(&sm.xempty[st], ((it / NS) & 1) ^ 1, wc, W_TMA_XEMPTY)) break;
+          mbar_arrive_expect_tx(&sm.xfull[st], 6 * TILE);
+          tma_load_3d(sm.X[st], &tmX, &sm.xfull[st], 0, c * C, bh);
+          tma_load_3d(sm.X[st] + TILE, &tmX, &sm.xfull[st], 64, c * C, bh);
+          tma_load_3d(sm.G[st], &tmG, &sm.xfull[st], 0, c * C, bh);
+          tma_load_3d(sm.G[st] + TILE, &tmG, &sm.xfull[st], 64, c * C, bh);
+          tma_load_3d(sm.U[st], &tmU, &sm.xfull[st], 0, c * C, bh);
+          tma_load_3d(sm.U[st] + TILE, &tmU, &sm.xfull[st], 64, c * C, bh);
+          xi = it + 1;
+          if (!mbar_wait(&sm.sempty, (it & 1) ^ 1, wc, W_TMA_SEMPTY)) break;
+          mbar_arrive_expect_tx(&sm.sfull, 2 * BIG);
+          tma_load_3d(sm.Sin, &tmS, &sm.sfull, 0, 0, bh * nch + c);
+          tma_load_3d(sm.Sin + BIG, &tmS, &sm.sfull, 64, 0, bh * nch + c);
+          si = it + 1;
+        }
+        for (int it = xi > NS ? xi - NS : 0; it < xi; ++it)
+          mbar_drain(&sm.xfull[it % NS], (it / NS) & 1, wc, W_TMA_DRAIN);
+        if (si > 0) mbar_drain(&sm.sfull, (si - 1) & 1, wc, W_TMA_DRAIN);
+      }
+    } else if (warp == 1) {
+      // ---------------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        const uint32_t id_cc = idesc_bf16(64, 64, false, false);      // X X^T, U G^T, G U^T
+        const uint32_t id_w = idesc_bf16(128, 128, true, true);       // U^T X, U^T Xg
+        const uint32_t id_db = idesc_bf16(128, 64, true, false);      // S^T U^T, W0^T U^T, ...
+        const uint32_t id_r1 = idesc_bf16(128, 64, false, false);     // Lam X^T
+        const uint32_t id_v = idesc_bf16(64, 64, false, true);        // Bm Q^T
+        const uint32_t sS = smem_u32(sm.Sin), sW0 = smem_u32(sm.W0), sL = smem_u32(sm.Lb);
+        for (int it = 0; it < nch; ++it) {
+          const int st = it % NS;
+          const uint32_t sX = smem_u32(sm.X[st]), sG = smem_u32(sm.G[st]), sU = smem_u32(sm.U[st]);
+          if (!mbar_wait(&sm.xfull[st], (it / NS) & 1, wc, W_MMA_XFULL)) break;
+          if (it > 0 && !mbar_wait(&sm.m2done, (it - 1) & 1, wc, W_MMA_M2)) break;
+          tc_fence_after();
+          // ---- phase 1
+          for (int kk = 0; kk < 8; ++kk) {  // K = X X^T, Kug = U G^T, KugT = G U^T
+            const uint32_t off = (kk >> 2) * TILE + (kk & 3) * 32;
+            const uint64_t dX = sw128_desc(sX + off, 16, 1024);
+            const uint64_t dG = sw128_desc(sG + off, 16, 1024);
+            const uint64_t dU = sw128_desc(sU + off, 16, 1024);
+            umma_bf16(tbase + COL_KK, dX, dX, id_cc, kk > 0);
+            umma_bf16(tbase + COL_KK + LANE16, dU, dG, id_cc, kk > 0);
+            umma_bf16(tbase + COL_KT, dG, dU, id_cc, kk > 0);
+          }
+          umma_commit(&sm.ccfull);
+          for (int kk = 0; kk < 4; ++kk)  // dW0 += U^T X
+            umma_bf16(tbase + COL_W, sw128_desc(sU + kk * 2048, TILE, 1024),
+                      sw128_desc(sX + kk * 2048, TILE, 1024), id_w, (it > 0 || kk > 0));
+          if (!mbar_wait(&sm.sfull, it & 1, wc, W_MMA_SFULL)) break;
+          tc_fence_after();
+          for (int kk = 0; kk < 8; ++kk)  // DXb^T = S_in^T U^T
+            umma_bf16(tbase + COL_D, sw128_desc(sS + kk * 2048, BIG, 1024),
+                      sw128_desc(sU + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024), id_db, kk > 0);
+          if (it > 0 && !mbar_wait(&sm.lbready, (it - 1) & 1, wc, W_MMA_LB)) break;
+          tc_fence_after();
+          for (int kk = 0; kk < 8; ++kk)  // R1^T = Lam X^T
+            umma_bf16(tbase + COL_R, sw128_desc(sL + (kk >> 2) * BIG + (kk & 3) * 32, 16, 1024),
+                      sw128_desc(sX + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024), id_r1, kk > 0);
+          umma_commit(&sm.b1full);
+          // ---- phase 2
+          if (!mbar_wait(&sm.m1done, it & 1, wc, W_MMA_M1)) break;
+          tc_fence_after();
+          for (int kk = 0; kk < 4; ++kk)  // V^T = Bm Q^T
+            umma_bf16(tbase + COL_KT + LANE16, sw128_desc(sS + CC_BM + kk * 32, 16, 1024),
+                      sw128_desc(sS + CC_QT + kk * 2048, TILE, 1024), id_v, kk > 0);
+          for (int kk = 0; kk < 4; ++kk)  // RI^T = U^T Ar^T
+            umma_bf16(tbase + COL_R, sw128_desc(sU + kk * 2048, TILE, 1024),
+                      sw128_desc(sS + CC_AR + kk * 32, 16, 1024), id_db, kk > 0);
+          for (int kk = 0; kk < 8; ++kk)  // DXa^T = W0^T U^T
+            umma_bf16(tbase + COL_D, sw128_desc(sW0 + kk * 2048, BIG, 1024),
+                      sw128_desc(sU + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024), id_db, kk > 0);
+          for (int kk = 0; kk < 4; ++kk)  //      + X^T Z^T
+            umma_bf16(tbase + COL_D, sw128_desc(sX + kk * 2048, TILE, 1024),
+                      sw128_desc(sS + CC_Z + kk * 32, 16, 1024), id_db, 1);
+          for (int kk = 0; kk < 8; ++kk)  //      + Lam^T Gs^T
+            umma_bf16(tbase + COL_D, sw128_desc(sL + kk * 2048, BIG, 1024),
+                      sw128_desc(sG + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024), id_db, 1);
+          umma_commit(&sm.b2full);
+          umma_commit(&sm.sempty);
+          // ---- phase 3
+          if (!mbar_wait(&sm.xscaled, it & 1, wc, W_MMA_XS)) break;
+          if (it > 0 && !mbar_wait(&sm.m3done, (it - 1) & 1, wc, W_MMA_M3)) break;
+          tc_fence_after();
+          for (int kk = 0; kk < 4; ++kk)  // dLam = U^T Xg
+            umma_bf16(tbase + COL_DL, sw128_desc(sU + kk * 2048, TILE, 1024),
+                      sw128_desc(sX + kk * 2048, TILE, 1024), id_w, kk > 0);
+          umma_commit(&sm.b3full);
+          umma_commit(&sm.xempty[st]);
+        }
+        umma_commit(&sm.done);
+        mbar_drain(&sm.done, 0, wc, W_MMA_DONE);
+      }
+    } else if (warp == 2) {
+      // ---------------------------------------------------------- gate prep
+      const size_t gbase = (size_t)bh * T;
+      for (int it = 0; it < nch; ++it) {
+        const int c = nch - 1 - it, g = it % GS;
+        if (!mbar_wait_warp(&sm.gempty[g], ((it / GS) & 1) ^ 1, wc, W_GATE_EMPTY)) break;
+        GateSlot& gs = sm.gates[g];
+        const int t0 = c * C + lane, t1 = t0 + 32;
+        const float a0 = t0 < T ? p.alpha[gbase + t0] : 1.f;
+        const float a1 = t1 < T ? p.alpha[gbase + t1] : 1.f;
+        const float e0 = t0 < T ? p.eta[gbase + t0] : 0.f;
+        const float e1 = t1 < T ? p.eta[gbase + t1] : 0.f;
+        float l0 = fmaxf(log2f(a0), -100.f), l1 = fmaxf(log2f(a1), -100.f);
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const float u0 = __shfl_up_sync(0xffffffffu, l0, o);
+          const float u1 = __shfl_up_sync(0xffffffffu, l1, o);
+          if (lane >= o) {
+            l0 += u0;
+            l1 += u1;
+          }
+        }
+        const float last0 = __shfl_sync(0xffffffffu, l0, 31);
+        l1 += last0;
+        const float Lend = __shfl_sync(0xffffffffu, l1, 31);
+        const float pm0 = __shfl_up_sync(0xffffffffu, l0, 1);
+        const float pm1 = __shfl_up_sync(0xffffffffu, l1, 1);
+        gs.L[lane] = l0;
+        gs.L[lane + 32] = l1;
+        gs.eta[lane] = e0;
+        gs.eta[lane + 32] = e1;
+        gs.gam[lane] = lane == 0 ? 1.f : exp2f(pm0);
+        gs.gam[lane + 32] = exp2f(lane == 0 ? last0 : pm1);
+        gs.del[lane] = exp2f(Lend - l0);
+        gs.del[lane + 32] = exp2f(Lend - l1);
+        if (lane == 0) gs.gC = exp2f(Lend);
+        __syncwarp();
+        mbar_arrive(&sm.gfull[g]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ math warpgroups
+    const int q = warp & 3;          // TMEM lane quadrant
+    const int hh = (warp - 4) >> 2;  // token half [32hh, 32hh+32) / state columns [64hh, +64)
+    const int mt = threadIdx.x - 128;
+    const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+    const int n = 32 * q + lane;             // d row owned in the 128-lane products
+    const int ir = 16 * q + (lane & 15);     // chunk row owned in the 64-row products
+    const bool lo = lane < 16;
+    const uint32_t sS = smem_u32(sm.Sin);
+    float Lam[64];
+#pragma unroll
+    for (int e = 0; e < 64; ++e) Lam[e] = 0.f;
+
+    // Every math thread executes the same sequence of named barriers in every
+    // iteration, whatever happens to its waits: after a failed (timed-out or
+    // aborted) wait the warp skips the work but keeps the barrier schedule, so no
+    // warp can be left at a bar.sync that its peers never reach.
+    bool ok = true;
+    for (int it = 0; it < nch; ++it) {
+      const int c = nch - 1 - it, st = it % NS, g = it % GS;
+      const GateSlot& gs = sm.gates[g];
+      const int t0 = c * C;
+      const size_t tokbase = (size_t)bh * T + t0;
+      const uint32_t sX = smem_u32(sm.X[st]), sG = smem_u32(sm.G[st]);
+      ok = ok && mbar_wait_warp(&sm.gfull[g], (it / GS) & 1, wc, W_M_GFULL);
+      ok = ok && mbar_wait_warp(&sm.xfull[st], (it / NS) & 1, wc, W_M_GFULL);
+      ok = ok && mbar_wait_warp(&sm.sfull, it & 1, wc, W_M_GFULL);
+      ok = ok && mbar_wait_warp(&sm.ccfull, it & 1, wc, W_M_CC);
+      ok = ok && mbar_wait_warp(&sm.b1full, it & 1, wc, W_M_B1);
+      tc_fence_after();
+
+      // ---- <Lam_end, S_in>
+      if (ok) {
+        float acc = 0.f;
+        const uint32_t row = sS + hh * BIG;
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          const uint4 v = ld_shared_v4(row + sw128_off(n, cc));
+          acc = fmaf(Lam[8 * cc + 0], bf16_lo(v.x), acc);
+          acc = fmaf(Lam[8 * cc + 1], bf16_hi(v.x), acc);
+          acc = fmaf(Lam[8 * cc + 2], bf16_lo(v.y), acc);
+          acc = fmaf(Lam[8 * cc + 3], bf16_hi(v.y), acc);
+          acc = fmaf(Lam[8 * cc + 4], bf16_lo(v.z), acc);
+          acc = fmaf(Lam[8 * cc + 5], bf16_hi(v.z), acc);
+          acc = fmaf(Lam[8 * cc + 6], bf16_lo(v.w), acc);
+          acc = fmaf(Lam[8 * cc + 7], bf16_hi(v.w), acc);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) sm.ered[warp - 4] = acc;
+      }
+      named_sync_math();  // (A) S_in fully read: its buffer now receives Ar | Z | Q^T | Bm
+
+      float r1s[32], dxs[32];
+      if (ok) {
+        // ---- chunk matrices from K | Kug and KugT
+        {
+          float vkk[32], vkt[32];
+          tmem_ld32(tbase + COL_KK + lane_off + 32 * hh, vkk);
+          tmem_ld32(tbase + COL_KT + lane_off + 32 * hh, vkt);
+          tmem_ld_wait();
+          // lanes < 16 hold the K and KugT rows, lanes >= 16 the Kug row of the same i;
+          // each value is exchanged with the partner lane (l ^ 16) as it is consumed
+          const int i = ir;
+          const float Li = gs.L[i], Lim1 = i == 0 ? 0.f : gs.L[i - 1], eti = gs.eta[i];
+          const uint32_t b1 = sS + (lo ? CC_AR : CC_QT), b2 = sS + (lo ? CC_Z : CC_BM);
+          float tpart = 0.f;
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t m1[4], m2[4];
+#pragma unroll
+            for (int e2 = 0; e2 < 8; e2 += 2) {
+              float v0[2], v1[2];
+#pragma unroll
+              for (int d = 0; d < 2; ++d) {
+                const int e = 8 * cc + e2 + d;
+                const float o1 = __shfl_xor_sync(0xffffffffu, vkk[e], 16);
+                const float o2 = __shfl_xor_sync(0xffffffffu, vkt[e], 16);
+                const float kr = lo ? vkk[e] : o1;  // x_i . x_j
+                const float kg = lo ? o1 : vkk[e];  // u_i . g_j
+                const float kt = lo ? vkt[e] : o2;  // g_i . u_j
+                const int j = 32 * hh + e;
+                const float Ljm1 = j == 0 ? 0.f : gs.L[j - 1];
+                const float bij = exp2f(fminf(Ljm1 - Li, 0.f));                    // j > i
+                const float aij = -gs.eta[j] * exp2f(fminf(Lim1 - gs.L[j], 0.f));  // j < i
+                if (lo) {
+                  v0[d] = (j > i) ? bij * kr : 0.f;                                 // Ar
+                  v1[d] = (j < i) ? aij * kg : ((j > i) ? -eti * bij * kt : 0.f);   // Z
+                } else {
+                  v0[d] = (j < i) ? kg * kr : 0.f;  // Q^T
+                  v1[d] = (j > i) ? bij : 0.f;      // Bm
+                  if (j > i) tpart = fmaf(bij * kr, kt, tpart);
+                }
+              }
+              m1[e2 >> 1] = pack_bf16(v0[0], v0[1]);
+              m2[e2 >> 1] = pack_bf16(v1[0], v1[1]);
+            }
+            st_shared_v4(b1 + sw128_off(i, 4 * hh + cc), m1[0], m1[1], m1[2], m1[3]);
+            st_shared_v4(b2 + sw128_off(i, 4 * hh + cc), m2[0], m2[1], m2[2], m2[3]);
+          }
+          if (!lo) sm.tv[hh][i] = tpart;
+        }
+        // ---- q_j = g_j^T Lam x_j (from R1^T), then G <- diag(-eta del) G in place
+        {
+          float vr[32];
+          tmem_ld32(tbase + COL_R + lane_off + 32 * hh, vr);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int j = 32 * hh + e;
+            const uint32_t ga = sw_elem(sG + (n >> 6) * TILE, j, n & 63);
+            const float gv = lds_bf16(ga);
+            r1s[e] = gs.del[j] * vr[e];
+            vr[e] = gv * vr[e];  // partial product of q_j
+            sts_bf16(ga, -gs.eta[j] * gs.del[j] * gv);
+          }
+          sm.redq[q][32 * hh + lane] = reduce_scatter32(vr, lane);
+        }
+        // ---- p_s = x_s^T S_in^T u_s (from DXb^T)
+        {
+          float vd[32];
+          tmem_ld32(tbase + COL_D + lane_off + 32 * hh, vd);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int s = 32 * hh + e;
+            const float xv = lds_bf16(sw_elem(sX + (n >> 6) * TILE, s, n & 63));
+            dxs[e] = gs.gam[s] * vd[e];
+            vd[e] = xv * vd[e];  // partial product of p_s
+          }
+          sm.redp[q][32 * hh + lane] = reduce_scatter32(vd, lane);
+        }
+        tc_fence_before();
+        fence_proxy_async_smem();
+      }
+      named_sync_math();  // (B) chunk matrices, scaled G and the partial sums are complete
+      if (ok && lane == 0) mbar_arrive(&sm.m1done);
+      float E = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) E += sm.ered[w];
+      if (ok && mt < C) {
+        const int j = mt;
+        const float qj = sm.redq[0][j] + sm.redq[1][j] + sm.redq[2][j] + sm.redq[3][j];
+        const float pj = sm.redp[0][j] + sm.redp[1][j] + sm.redp[2][j] + sm.redp[3][j];
+        sm.qv[j] = qj;
+        sm.pv[j] = pj;
+        const float deta = -(gs.del[j] * qj + sm.tv[0][j] + sm.tv[1][j]);
+        if (t0 + j < T) p.d_eta[tokbase + j] = deta;
+      }
+
+      // ---- phase 2: r -> dg, dx, and the V part of dalpha
+      ok = ok && mbar_wait_warp(&sm.b2full, it & 1, wc, W_M_B2);
+      tc_fence_after();
+      if (ok) {
+        {
+          float vv[32], vri[32];
+          tmem_ld32(tbase + COL_KT + lane_off + 32 * hh, vv);
+          tmem_ld32(tbase + COL_R + lane_off + 32 * hh, vri);
+          tmem_ld_wait();
+          if (!lo) {
+            const int i = ir;
+            const float Lim1 = i == 0 ? 0.f : gs.L[i - 1];
+            float hpart = 0.f;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int j = 32 * hh + e;
+              const float aij = -gs.eta[j] * exp2f(fminf(Lim1 - gs.L[j], 0.f));
+              if (j < i) hpart = fmaf(aij, vv[e], hpart);
+            }
+            sm.hv[hh][i] = hpart;
+          }
+          __nv_bfloat16* dgo = p.dg + tokbase * 128 + n;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int i = 32 * hh + e;
+            if (t0 + i < T)
+              dgo[(size_t)i * 128] = __float2bfloat16_rn(-gs.eta[i] * (r1s[e] + vri[e]));
+          }
+        }
+        {
+          float vda[32];
+          tmem_ld32(tbase + COL_D + lane_off + 32 * hh, vda);
+          tmem_ld_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.m2done);
+          __nv_bfloat16* dxo = p.dx + tokbase * 128 + n;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int i = 32 * hh + e;
+            if (t0 + i < T) dxo[(size_t)i * 128] = __float2bfloat16_rn(vda[e] + dxs[e]);
+          }
+        }
+        // X <- diag(gam) X in place for dLam = U^T Xg
+#pragma unroll 8
+        for (int e = 0; e < 32; ++e) {
+          const int s = 32 * hh + e;
+          const uint32_t xa = sw_elem(sX + (n >> 6) * TILE, s, n & 63);
+          sts_bf16(xa, gs.gam[s] * lds_bf16(xa));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.xscaled);
+      }
+      named_sync_math();  // (C) hv of both halves written
+      if (ok && mt < C) {
+        const int i = mt;
+        const float Li = gs.L[i], Lim1 = i == 0 ? 0.f : gs.L[i - 1];
+        float t2 = 0.f, t3 = 0.f;
+        for (int j = 0; j < i; ++j)
+          t2 = fmaf(-gs.eta[j] * exp2f(fminf(Lim1 - gs.L[j], 0.f)), sm.qv[j], t2);
+        for (int s = i + 1; s < C; ++s)
+          t3 = fmaf(exp2f(fminf(gs.L[s - 1] - Li, 0.f)), sm.pv[s], t3);
+        const float da = gs.gam[i] * gs.del[i] * E + gs.del[i] * t2 + gs.gam[i] * t3 +
+                         sm.hv[0][i] + sm.hv[1][i];
+        if (t0 + i < T) p.d_alpha[tokbase + i] = da;
+      }
+
+      // ---- phase 3: Lam <- 2^{L_{C-1}} Lam + dLam
+      ok = ok && mbar_wait_warp(&sm.b3full, it & 1, wc, W_M_B3);
+      tc_fence_after();
+      if (ok) {
+        float v0[32], v1[32];
+        tmem_ld32(tbase + COL_DL + lane_off + 64 * hh, v0);
+        tmem_ld32(tbase + COL_DL + lane_off + 64 * hh + 32, v1);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.m3done);
+        const float gC = gs.gC;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          Lam[e] = fmaf(gC, Lam[e], v0[e]);
+          Lam[32 + e] = fmaf(gC, Lam[32 + e], v1[e]);
+        }
+        const uint32_t lrow = smem_u32(sm.Lb + hh * BIG);
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc)
+          st_shared_v4(lrow + sw128_off(n, cc), pack_bf16(Lam[8 * cc], Lam[8 * cc + 1]),
+                       pack_bf16(Lam[8 * cc + 2], Lam[8 * cc + 3]),
+                       pack_bf16(Lam[8 * cc + 4], Lam[8 * cc + 5]),
+                       pack_bf16(Lam[8 * cc + 6], Lam[8 * cc + 7]));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&sm.lbready);
+          mbar_arrive(&sm.gempty[g]);
+        }
+      }
+      named_sync_math();  // (D) per-chunk scratch consumed before the next chunk writes it
+    }
+
+    // ---- this scan's dW0 partial: the last b3full wait covered every product
+    {
+      if (ok) {
+        float v0[32], v1[32];
+        tmem_ld32(tbase + COL_W + lane_off + 64 * hh, v0);
+        tmem_ld32(tbase + COL_W + lane_off + 64 * hh + 32, v1);
+        tmem_ld_wait();
+        float4* dst = reinterpret_cast<float4*>(p.dW0_part + ((size_t)bh * 128 + n) * 128 + 64 * hh);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          dst[e] = make_float4(v0[4 * e], v0[4 * e + 1], v0[4 * e + 2], v0[4 * e + 3]);
+          dst[8 + e] = make_float4(v1[4 * e], v1[4 * e + 1], v1[4 * e + 2], v1[4 * e + 3]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+bool bwd_shape_ok(int din, int dout) { return din == 128 && dout == 128; }
+
+cudaError_t launch_bwd(const TcBwdParams& prm, const void* x, const void* g, const void* dy,
+                       const void* ckpt, cudaStream_t st) {
+  CUtensorMap mx, mg, mu, ms;
+  const uint64_t BH = (uint64_t)prm.B * prm.H;
+  const uint64_t nch = (uint64_t)(prm.T + C - 1) / C;
+  if (!make_map_bf16_3d(&mx, x, 128, prm.T, BH, C) || !make_map_bf16_3d(&mg, g, 128, prm.T, BH, C) ||
+      !make_map_bf16_3d(&mu, dy, 128, prm.T, BH, C) ||
+      !make_map_bf16_3d(&ms, ckpt, 128, 128, BH * nch, 128))
+    return cudaErrorInvalidValue;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  bwd_kernel<<<(int)BH, NTHREADS, kSmemBytes, st>>>(mx, mg, mu, ms, prm);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace tc
+}  // namespace gradlev

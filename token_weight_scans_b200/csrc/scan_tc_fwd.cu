@@ -279,7 +279,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int s = c % NS, g = c % GS;
         GateSlot& gs = sm.gates[g];
         if (gate_warp) {
-          if (!mbar_wait(&sm.gempty[g], ((c / GS) & 1) ^ 1, wc, W_GATE_EMPTY)) { ok = false; break; }
+          if (!mbar_wait_warp(&sm.gempty[g], ((c / GS) & 1) ^ 1, wc, W_GATE_EMPTY)) { ok = false; break; }
           const float a0 = ra[k][0], a1 = ra[k][1], e0 = re[k][0], e1 = re[k][1];
           {  // prefetch the gates of chunk c + PD into this register slot
             const int t0 = (c + PD) * C + lane, t1 = t0 + 32;
@@ -315,9 +315,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           __syncwarp();
           mbar_arrive(&sm.gfull[g]);
         }
-        if (!mbar_wait(&sm.full[s], (c / NS) & 1, wc, W_XH_FULL)) { ok = false; break; }
-        if (!mbar_wait(&sm.gfull[g], (c / GS) & 1, wc, W_XH_GFULL)) { ok = false; break; }
-        if (c > 0 && !mbar_wait(&sm.dsfull, (c - 1) & 1, wc, W_XH_DSFULL)) { ok = false; break; }
+        if (!mbar_wait_warp(&sm.full[s], (c / NS) & 1, wc, W_XH_FULL)) { ok = false; break; }
+        if (!mbar_wait_warp(&sm.gfull[g], (c / GS) & 1, wc, W_XH_GFULL)) { ok = false; break; }
+        if (c > 0 && !mbar_wait_warp(&sm.dsfull, (c - 1) & 1, wc, W_XH_DSFULL)) { ok = false; break; }
         const uint32_t src = smem_u32(sm.X[s]), dst = smem_u32(sm.Xh);
 #pragma unroll 4
         for (int idx = (warp - 2) * 32 + lane; idx < 2 * TILE / 16; idx += 64) {
@@ -349,14 +349,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     float Sreg[64];
 #pragma unroll
     for (int e = 0; e < 64; ++e) Sreg[e] = 0.f;
-    __nv_bfloat16* yout = p.y + (size_t)bh * T * p.dout + n0 + n;
+    __nv_bfloat16* yout = p.y ? p.y + (size_t)bh * T * p.dout + n0 + n : nullptr;
+    // chunk-start state checkpoints (bf16 [bh][chunk][dout][din]); S_0 = 0
+    uint4* ck_row = p.ckpt ? reinterpret_cast<uint4*>(p.ckpt + ((size_t)bh * nch * p.dout + n0 + n) * 128 + 64 * hh)
+                           : nullptr;
+    const size_t ck_stride = (size_t)p.dout * 128 / 8;  // uint4 per chunk
+    if (ck_row) {
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) ck_row[cc] = make_uint4(0u, 0u, 0u, 0u);
+    }
 
     // mask of chunk c: P_ij = K_ij (-eta_j) 2^{L_{i-1} - L_j} for j < i
     auto mask = [&](int c) -> bool {
       const int g = c % GS, b = c & 1;
       const GateSlot& gs = sm.gates[g];
-      if (!mbar_wait(&sm.gfull[g], (c / GS) & 1, wc, W_M_GFULL)) return false;
-      if (!mbar_wait(&sm.kfull[b], (c >> 1) & 1, wc, W_M_KFULL)) return false;
+      if (!mbar_wait_warp(&sm.gfull[g], (c / GS) & 1, wc, W_M_GFULL)) return false;
+      if (!mbar_wait_warp(&sm.kfull[b], (c >> 1) & 1, wc, W_M_KFULL)) return false;
       tc_fence_after();
       float v[32];
       tmem_ld32(tbase + (b ? COL_K1 : COL_K0) + lane_off + 32 * hh, v);
@@ -398,8 +406,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       //      the S X^T product of chunk c - 1 read (one barrier pair per buffer, so a
       //      parity wait can never see a phase from the other buffer's traffic)
       const int wb = (c + 1) & 1;
-      if (!mbar_wait(&sm.dsfull, c & 1, wc, W_M_DSFULL)) break;
-      if (c > 0 && !mbar_wait(&sm.sfree[wb], ((c - 1) >> 1) & 1, wc, W_M_SFREE)) break;
+      if (!mbar_wait_warp(&sm.dsfull, c & 1, wc, W_M_DSFULL)) break;
+      if (c > 0 && !mbar_wait_warp(&sm.sfree[wb], ((c - 1) >> 1) & 1, wc, W_M_SFREE)) break;
       tc_fence_after();
       {
         float v0[32], v1[32];
@@ -416,12 +424,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           Sreg[32 + e] = fmaf(gC, Sreg[32 + e], v1[e]);
         }
         const uint32_t srow = smem_u32(sm.S[wb][hh]);
+        uint4* ck = (ck_row && c + 1 < nch) ? ck_row + (size_t)(c + 1) * ck_stride : nullptr;
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc)
-          st_shared_v4(srow + sw128_off(n, cc), pack_bf16(Sreg[8 * cc], Sreg[8 * cc + 1]),
-                       pack_bf16(Sreg[8 * cc + 2], Sreg[8 * cc + 3]),
-                       pack_bf16(Sreg[8 * cc + 4], Sreg[8 * cc + 5]),
-                       pack_bf16(Sreg[8 * cc + 6], Sreg[8 * cc + 7]));
+        for (int cc = 0; cc < 8; ++cc) {
+          const uint4 pk = make_uint4(pack_bf16(Sreg[8 * cc], Sreg[8 * cc + 1]),
+                                      pack_bf16(Sreg[8 * cc + 2], Sreg[8 * cc + 3]),
+                                      pack_bf16(Sreg[8 * cc + 4], Sreg[8 * cc + 5]),
+                                      pack_bf16(Sreg[8 * cc + 6], Sreg[8 * cc + 7]));
+          st_shared_v4(srow + sw128_off(n, cc), pk.x, pk.y, pk.z, pk.w);
+          if (ck) ck[cc] = pk;
+        }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.sready[wb]);
@@ -431,7 +443,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (c + 1 < nch && !mask(c + 1)) break;
 
       // ---- output: y_i = Y1^T[n][i] + 2^{L_{i-1}} Y2^T[n][i]
-      if (!mbar_wait(&sm.yfull[b], (c >> 1) & 1, wc, W_M_YFULL)) break;
+      if (!mbar_wait_warp(&sm.yfull[b], (c >> 1) & 1, wc, W_M_YFULL)) break;
       tc_fence_after();
       {
         float a[32], s2[32];
@@ -443,7 +455,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (lane == 0) mbar_arrive(&sm.yfree[b]);
         const int ib = 32 * hh;
         const int tb = c * C + ib;
-        if (tb + 32 <= T) {
+        if (!yout) {
+        } else if (tb + 32 <= T) {
 #pragma unroll
           for (int e = 0; e < 32; ++e)
             yout[(size_t)(tb + e) * p.dout] = __float2bfloat16_rn(fmaf(gs.gam[ib + e], s2[e], a[e]));
@@ -499,6 +512,11 @@ bool make_map_bf16_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1
 }
 
 bool fwd_shape_ok(int din, int dout) { return din == 128 && dout % 128 == 0 && dout <= 256; }
+
+size_t ckpt_bytes(int B, int H, int T, int din, int dout) {
+  const size_t nch = (size_t)(T + C - 1) / C;
+  return (size_t)B * H * nch * dout * din * sizeof(__nv_bfloat16);
+}
 
 cudaError_t launch_fwd(const TcFwdParams& prm, const void* x, const void* g, cudaStream_t st) {
   CUtensorMap mx, mg;

@@ -66,7 +66,7 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, const WaitCtx& w,
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, const WaitCtx& w,
                                              uint32_t where, bool abortable) {
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
@@ -88,6 +88,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
                                           uint32_t where) {
   if (mbar_test(bar, parity)) return true;
   return mbar_wait_slow(bar, parity, w, where, true);
+}
+
+// Warp-uniform variant for warps that go on to execute warp-collective
+// instructions: every lane waits, and the warp proceeds only if all lanes succeeded.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, const WaitCtx& w,
+                                               uint32_t where) {
+  const bool ok = mbar_wait(bar, parity, w, where);
+  return __all_sync(0xffffffffu, ok);
 }
 
 // Same, but ignores the abort flag (teardown: wait for work already in flight).
