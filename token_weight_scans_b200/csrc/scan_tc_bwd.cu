@@ -28,19 +28,24 @@
 //   phase 1: K = X X^T | Kug = U G^T (M=64), KugT = G U^T (M=64), dW0 += U^T X,
 //            DXb^T = S_in^T U^T, R1^T = Lam X^T
 //   phase 2: V^T = Bm Q^T (M=64), RI^T = U^T Ar^T, DXa^T = W0^T U^T + X^T Z^T + Lam^T Gs^T
-//   phase 3: dLam = U^T Xg
+//   phase 3: Lam += U^T Xg
 // where Ar, Z, Q^T, Bm are built by the math warps from K, Kug, KugT into the
 // shared memory that held S_in, Gs = diag(-eta del) G and Xg = diag(gam) X are
-// written in place once their unscaled uses are over.
+// written in place once their unscaled uses are over. The fp32 adjoint Lam
+// lives in TMEM: the math warps scale it by 2^{L_{C-1}} in place and the MMA
+// accumulates U^T Xg onto it; likewise del (.) R1^T and gam (.) DXb^T are
+// written back so that RI^T and DXa^T accumulate onto them (r^T and dx^T).
 //
-// Warp roles (12 warps): 0 TMA producer, 1 MMA issuer + TMEM owner, 2 gate
-// prep, 3 idle helper, 4..11 two math warpgroups (warpgroup h: tokens
-// [32h, 32h+32) of each chunk and state columns [64h, 64h+64)).
+// Warp roles (20 warps): 0 TMA producer, 1 MMA issuer + TMEM owner, 2 gate
+// prep, 3 idle helper, 4..19 four math warpgroups (warpgroup w: tokens
+// [16w, 16w+16) of each chunk and state columns [32w, 32w+32)).
 
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
+
+#include <type_traits>
 
 #include "common.cuh"
 #include "scan_tc.h"
@@ -59,29 +64,38 @@ namespace {
 constexpr int C = kChunk;       // 64 tokens per chunk
 constexpr int NS = 2;           // stages of the X, G, U tiles
 constexpr int GS = 2;           // gate slots
-constexpr int NTHREADS = 384;
+constexpr int NMATH = 16;                   // math warps: 4 warpgroups
+constexpr int NTHREADS = 128 + 32 * NMATH;  // + TMA, MMA, gate and helper warps
 constexpr int TILE = C * 128;   // [64 rows x 128 B] swizzled block
 constexpr int BIG = 128 * 128;  // [128 rows x 128 B] swizzled block
 
 // TMEM columns (512 allocated)
 constexpr uint32_t COL_KK = 0;    // K (lanes 0-15 of each sub-partition) | Kug (lanes 16-31)
 constexpr uint32_t COL_KT = 64;   // KugT (lanes 0-15) | V^T (lanes 16-31)
-constexpr uint32_t COL_R = 128;   // R1^T, then RI^T
-constexpr uint32_t COL_D = 192;   // DXb^T, then DXa^T
-constexpr uint32_t COL_DL = 256;  // dLam (128 columns)
+constexpr uint32_t COL_R = 128;   // R1^T -> del (.) R1^T -> + RI^T = r^T
+constexpr uint32_t COL_D = 192;   // DXb^T -> gam (.) DXb^T -> + DXa^T = dx^T
+constexpr uint32_t COL_L = 256;   // Lam, fp32 (128 columns)
 constexpr uint32_t COL_W = 384;   // dW0 accumulator (128 columns)
 constexpr uint32_t LANE16 = 16u << 16;
 
 // chunk-by-chunk matrices built by the math warps, aliased onto the S_in tile
 constexpr int CC_AR = 0, CC_Z = TILE, CC_QT = 2 * TILE, CC_BM = 3 * TILE;
 
-struct GateSlot {
+// Per-chunk gate quantities (16-byte aligned rows for vector loads). With M = L_{31} (mid-chunk) the decay factors
+// split into row and column factors, a_ij = ra_i ca_j and b_ij = rb_i cb_j, as
+// long as every exponent stays inside fp32 range: fac = (|L_{C-1}| <= 120).
+struct alignas(16) GateSlot {
   float L[C];
   float eta[C];
   float gam[C];
   float del[C];
+  float ra[C];   // 2^{L_{i-1} - M}
+  float ca[C];   // -eta_j 2^{M - L_j}
+  float rb[C];   // 2^{M - L_i}
+  float cb[C];   // 2^{L_{j-1} - M}
   float gC;
-  float pad[3];
+  int fac;
+  float pad[2];
 };
 
 struct Smem {
@@ -93,14 +107,15 @@ struct Smem {
   uint8_t Lb[2 * BIG];        // bf16 Lam, [k-block][n rows x 128 B]
   GateSlot gates[GS];
   float redq[4][C], redp[4][C];
-  float tv[2][C], hv[2][C];
-  float qv[C], pv[C];
-  float ered[8];
+  float tv[4][C], t2v[4][C], t3v[4][C], hv[4][C];
+  alignas(16) float qv[C];
+  alignas(16) float pv[C];
+  float ered[NMATH];
   uint64_t xfull[NS], xempty[NS];
   uint64_t gfull[GS], gempty[GS];
   uint64_t sfull, sempty;
   uint64_t ccfull, b1full, b2full, b3full;
-  uint64_t m1done, m2done, m3done, xscaled, lbready, done;
+  uint64_t m1done, m2done, xscaled, lbready, done;
   uint32_t tmem_base;
   int abort;
 };
@@ -109,14 +124,13 @@ constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
 
 enum : uint32_t {
   W_TMA_XEMPTY = 0x001, W_TMA_SEMPTY, W_TMA_DRAIN,
-  W_MMA_XFULL = 0x101, W_MMA_M2, W_MMA_SFULL, W_MMA_LB, W_MMA_M1, W_MMA_XS, W_MMA_M3,
-  W_MMA_DONE,
+  W_MMA_XFULL = 0x101, W_MMA_M2, W_MMA_SFULL, W_MMA_LB, W_MMA_M1, W_MMA_XS, W_MMA_DONE,
   W_GATE_EMPTY = 0x201,
   W_M_GFULL = 0x401, W_M_CC, W_M_B1, W_M_B2, W_M_B3,
 };
 
 __device__ __forceinline__ void named_sync_math() {
-  asm volatile("bar.sync 1, 256;" ::: "memory");
+  asm volatile("bar.sync 1, %0;" ::"n"(32 * NMATH) : "memory");
 }
 
 // Element (row, col) of a [rows x 128 B] swizzled bf16 block (col < 64).
@@ -130,10 +144,38 @@ __device__ __forceinline__ float lds_bf16(uint32_t addr) {
   return __uint_as_float(((uint32_t)v) << 16);
 }
 
-__device__ __forceinline__ void sts_bf16(uint32_t addr, float f) {
+__device__ __forceinline__ void sts_u16(uint32_t addr, float f) {
   const __nv_bfloat16 b = __float2bfloat16_rn(f);
   const unsigned short v = *reinterpret_cast<const unsigned short*>(&b);
   asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+}
+
+// Sum of v[0..15] over the 32 lanes of the warp; lanes 2k and 2k+1 return the total of index k.
+__device__ __forceinline__ float reduce_scatter16(float (&v)[16], int lane) {
+  float w8[8], w4[4], w2[2];
+  const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float send = b4 ? v[k] : v[k + 8];
+    const float keep = b4 ? v[k + 8] : v[k];
+    w8[k] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float send = b3 ? w8[k] : w8[k + 4];
+    const float keep = b3 ? w8[k + 4] : w8[k];
+    w4[k] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const float send = b2 ? w4[k] : w4[k + 2];
+    const float keep = b2 ? w4[k + 2] : w4[k];
+    w2[k] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+  }
+  const float send = b1 ? w2[0] : w2[1];
+  const float keep = b1 ? w2[1] : w2[0];
+  float w1 = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+  return w1 + __shfl_xor_sync(0xffffffffu, w1, 1);
 }
 
 // Sum of v[0..31] over the 32 lanes of the warp; lane l returns the total of index l.
@@ -174,6 +216,7 @@ __device__ __forceinline__ float reduce_scatter32(float (&v)[32], int lane) {
 __global__ void __launch_bounds__(NTHREADS, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmG,
                const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmS,
+               const __grid_constant__ CUtensorMap tmDX, const __grid_constant__ CUtensorMap tmDG,
                TcBwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>(
@@ -192,7 +235,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     for (int g = 0; g < GS; ++g) {
       mbar_init(&sm.gfull[g], 32);
-      mbar_init(&sm.gempty[g], 8);
+      mbar_init(&sm.gempty[g], NMATH);
     }
     mbar_init(&sm.sfull, 1);
     mbar_init(&sm.sempty, 1);
@@ -200,11 +243,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(&sm.b1full, 1);
     mbar_init(&sm.b2full, 1);
     mbar_init(&sm.b3full, 1);
-    mbar_init(&sm.m1done, 8);
-    mbar_init(&sm.m2done, 8);
-    mbar_init(&sm.m3done, 8);
-    mbar_init(&sm.xscaled, 8);
-    mbar_init(&sm.lbready, 8);
+    mbar_init(&sm.m1done, NMATH);
+    mbar_init(&sm.m2done, NMATH);
+    mbar_init(&sm.xscaled, NMATH);
+    mbar_init(&sm.lbready, NMATH);
     mbar_init(&sm.done, 1);
     fence_mbar_init();
   }
@@ -213,6 +255,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     prefetch_tmap(&tmG);
     prefetch_tmap(&tmU);
     prefetch_tmap(&tmS);
+    prefetch_tmap(&tmDX);
+    prefetch_tmap(&tmDG);
   }
   if (warp == 1) {
     tmem_alloc(&sm.tmem_base, 512);
@@ -222,7 +266,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // W0 -> bf16 swizzled [k-block][n rows]; Lam_T = 0
     const int t = threadIdx.x - 128;
     const float* W0 = p.W0 + (size_t)h * 128 * 128;
-    for (int idx = t; idx < 128 * 16; idx += 256) {
+    for (int idx = t; idx < 128 * 16; idx += 32 * NMATH) {
       const int n = idx >> 4, ck = idx & 15;
       const int kb = ck >> 3, c = ck & 7;
       const float4 a = *reinterpret_cast<const float4*>(W0 + (size_t)n * 128 + ck * 8);
@@ -273,13 +317,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t id_r1 = idesc_bf16(128, 64, false, false);     // Lam X^T
         const uint32_t id_v = idesc_bf16(64, 64, false, true);        // Bm Q^T
         const uint32_t sS = smem_u32(sm.Sin), sW0 = smem_u32(sm.W0), sL = smem_u32(sm.Lb);
-        for (int it = 0; it < nch; ++it) {
+        // Software-pipelined order: the Gram products and dW0 of chunk it+1 are
+        // issued as soon as the math warps have read chunk it's phase-2 results,
+        // ahead of chunk it's Lam update; only Lam X^T waits for the new Lam.
+        auto xgu = [&](int it, uint32_t& sX, uint32_t& sG, uint32_t& sU) {
           const int st = it % NS;
-          const uint32_t sX = smem_u32(sm.X[st]), sG = smem_u32(sm.G[st]), sU = smem_u32(sm.U[st]);
-          if (!mbar_wait(&sm.xfull[st], (it / NS) & 1, wc, W_MMA_XFULL)) break;
-          if (it > 0 && !mbar_wait(&sm.m2done, (it - 1) & 1, wc, W_MMA_M2)) break;
+          sX = smem_u32(sm.X[st]);
+          sG = smem_u32(sm.G[st]);
+          sU = smem_u32(sm.U[st]);
+        };
+        auto phase1a = [&](int it) -> bool {  // K, Kug, KugT, dW0
+          uint32_t sX, sG, sU;
+          xgu(it, sX, sG, sU);
+          if (!mbar_wait(&sm.xfull[it % NS], (it / NS) & 1, wc, W_MMA_XFULL)) return false;
+          if (it > 0 && !mbar_wait(&sm.m2done, (it - 1) & 1, wc, W_MMA_M2)) return false;
           tc_fence_after();
-          // ---- phase 1
           for (int kk = 0; kk < 8; ++kk) {  // K = X X^T, Kug = U G^T, KugT = G U^T
             const uint32_t off = (kk >> 2) * TILE + (kk & 3) * 32;
             const uint64_t dX = sw128_desc(sX + off, 16, 1024);
@@ -293,29 +345,38 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int kk = 0; kk < 4; ++kk)  // dW0 += U^T X
             umma_bf16(tbase + COL_W, sw128_desc(sU + kk * 2048, TILE, 1024),
                       sw128_desc(sX + kk * 2048, TILE, 1024), id_w, (it > 0 || kk > 0));
-          if (!mbar_wait(&sm.sfull, it & 1, wc, W_MMA_SFULL)) break;
+          return true;
+        };
+        auto phase1b = [&](int it) -> bool {  // DXb^T, R1^T
+          uint32_t sX, sG, sU;
+          xgu(it, sX, sG, sU);
+          if (!mbar_wait(&sm.sfull, it & 1, wc, W_MMA_SFULL)) return false;
           tc_fence_after();
           for (int kk = 0; kk < 8; ++kk)  // DXb^T = S_in^T U^T
             umma_bf16(tbase + COL_D, sw128_desc(sS + kk * 2048, BIG, 1024),
                       sw128_desc(sU + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024), id_db, kk > 0);
-          if (it > 0 && !mbar_wait(&sm.lbready, (it - 1) & 1, wc, W_MMA_LB)) break;
+          if (it > 0 && !mbar_wait(&sm.lbready, (it - 1) & 1, wc, W_MMA_LB)) return false;
           tc_fence_after();
           for (int kk = 0; kk < 8; ++kk)  // R1^T = Lam X^T
             umma_bf16(tbase + COL_R, sw128_desc(sL + (kk >> 2) * BIG + (kk & 3) * 32, 16, 1024),
                       sw128_desc(sX + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024), id_r1, kk > 0);
           umma_commit(&sm.b1full);
-          // ---- phase 2
-          if (!mbar_wait(&sm.m1done, it & 1, wc, W_MMA_M1)) break;
+          return true;
+        };
+        auto phase2 = [&](int it) -> bool {
+          uint32_t sX, sG, sU;
+          xgu(it, sX, sG, sU);
+          if (!mbar_wait(&sm.m1done, it & 1, wc, W_MMA_M1)) return false;
           tc_fence_after();
           for (int kk = 0; kk < 4; ++kk)  // V^T = Bm Q^T
             umma_bf16(tbase + COL_KT + LANE16, sw128_desc(sS + CC_BM + kk * 32, 16, 1024),
                       sw128_desc(sS + CC_QT + kk * 2048, TILE, 1024), id_v, kk > 0);
-          for (int kk = 0; kk < 4; ++kk)  // RI^T = U^T Ar^T
+          for (int kk = 0; kk < 4; ++kk)  // r^T = del (.) R1^T + U^T Ar^T
             umma_bf16(tbase + COL_R, sw128_desc(sU + kk * 2048, TILE, 1024),
-                      sw128_desc(sS + CC_AR + kk * 32, 16, 1024), id_db, kk > 0);
-          for (int kk = 0; kk < 8; ++kk)  // DXa^T = W0^T U^T
+                      sw128_desc(sS + CC_AR + kk * 32, 16, 1024), id_db, 1);
+          for (int kk = 0; kk < 8; ++kk)  // dx^T = gam (.) DXb^T + W0^T U^T
             umma_bf16(tbase + COL_D, sw128_desc(sW0 + kk * 2048, BIG, 1024),
-                      sw128_desc(sU + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024), id_db, kk > 0);
+                      sw128_desc(sU + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024), id_db, 1);
           for (int kk = 0; kk < 4; ++kk)  //      + X^T Z^T
             umma_bf16(tbase + COL_D, sw128_desc(sX + kk * 2048, TILE, 1024),
                       sw128_desc(sS + CC_Z + kk * 32, 16, 1024), id_db, 1);
@@ -324,15 +385,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                       sw128_desc(sG + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024), id_db, 1);
           umma_commit(&sm.b2full);
           umma_commit(&sm.sempty);
-          // ---- phase 3
-          if (!mbar_wait(&sm.xscaled, it & 1, wc, W_MMA_XS)) break;
-          if (it > 0 && !mbar_wait(&sm.m3done, (it - 1) & 1, wc, W_MMA_M3)) break;
+          return true;
+        };
+        auto phase3 = [&](int it) -> bool {  // Lam += U^T Xg (Lam pre-scaled by the math warps)
+          uint32_t sX, sG, sU;
+          xgu(it, sX, sG, sU);
+          if (!mbar_wait(&sm.xscaled, it & 1, wc, W_MMA_XS)) return false;
           tc_fence_after();
-          for (int kk = 0; kk < 4; ++kk)  // dLam = U^T Xg
-            umma_bf16(tbase + COL_DL, sw128_desc(sU + kk * 2048, TILE, 1024),
-                      sw128_desc(sX + kk * 2048, TILE, 1024), id_w, kk > 0);
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tbase + COL_L, sw128_desc(sU + kk * 2048, TILE, 1024),
+                      sw128_desc(sX + kk * 2048, TILE, 1024), id_w, 1);
           umma_commit(&sm.b3full);
-          umma_commit(&sm.xempty[st]);
+          umma_commit(&sm.xempty[it % NS]);
+          return true;
+        };
+        bool ok = phase1a(0) && phase1b(0) && phase2(0);
+        for (int it = 0; it < nch && ok; ++it) {
+          if (it + 1 < nch) ok = phase1a(it + 1);
+          ok = ok && phase3(it);
+          if (it + 1 < nch) ok = ok && phase1b(it + 1) && phase2(it + 1);
         }
         umma_commit(&sm.done);
         mbar_drain(&sm.done, 0, wc, W_MMA_DONE);
@@ -372,7 +443,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         gs.gam[lane + 32] = exp2f(lane == 0 ? last0 : pm1);
         gs.del[lane] = exp2f(Lend - l0);
         gs.del[lane + 32] = exp2f(Lend - l1);
-        if (lane == 0) gs.gC = exp2f(Lend);
+        {
+          const float Mid = last0;  // L_{31}
+          const float lm0 = lane == 0 ? 0.f : pm0, lm1 = lane == 0 ? last0 : pm1;  // L_{i-1}
+          gs.ra[lane] = exp2f(lm0 - Mid);
+          gs.ra[lane + 32] = exp2f(lm1 - Mid);
+          gs.ca[lane] = -e0 * exp2f(Mid - l0);
+          gs.ca[lane + 32] = -e1 * exp2f(Mid - l1);
+          gs.rb[lane] = exp2f(Mid - l0);
+          gs.rb[lane + 32] = exp2f(Mid - l1);
+          gs.cb[lane] = exp2f(lm0 - Mid);
+          gs.cb[lane + 32] = exp2f(lm1 - Mid);
+        }
+        if (lane == 0) {
+          gs.gC = exp2f(Lend);
+          gs.fac = (Lend >= -120.f) ? 1 : 0;
+        }
         __syncwarp();
         mbar_arrive(&sm.gfull[g]);
       }
@@ -380,16 +466,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else {
     // ------------------------------------------------------------ math warpgroups
     const int q = warp & 3;          // TMEM lane quadrant
-    const int hh = (warp - 4) >> 2;  // token half [32hh, 32hh+32) / state columns [64hh, +64)
+    const int wg = (warp - 4) >> 2;  // warpgroup: tokens [16wg, +16), Lam columns [32wg, +32)
     const int mt = threadIdx.x - 128;
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
     const int n = 32 * q + lane;             // d row owned in the 128-lane products
     const int ir = 16 * q + (lane & 15);     // chunk row owned in the 64-row products
     const bool lo = lane < 16;
+    const int j0w = 16 * wg;                 // first chunk token / column of this warpgroup
     const uint32_t sS = smem_u32(sm.Sin);
-    float Lam[64];
+    const uint32_t tL = tbase + COL_L + lane_off + 32 * wg;  // this thread's Lam columns
+    const uint32_t sLb = smem_u32(sm.Lb);
+    {  // Lam_T = 0
+      float z[32];
 #pragma unroll
-    for (int e = 0; e < 64; ++e) Lam[e] = 0.f;
+      for (int e = 0; e < 32; ++e) z[e] = 0.f;
+      tmem_st32(tL, z);
+      tmem_st_wait();
+    }
 
     // Every math thread executes the same sequence of named barriers in every
     // iteration, whatever happens to its waits: after a failed (timed-out or
@@ -409,217 +502,289 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       ok = ok && mbar_wait_warp(&sm.b1full, it & 1, wc, W_M_B1);
       tc_fence_after();
 
-      // ---- <Lam_end, S_in>
       if (ok) {
-        float acc = 0.f;
-        const uint32_t row = sS + hh * BIG;
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          const uint4 v = ld_shared_v4(row + sw128_off(n, cc));
-          acc = fmaf(Lam[8 * cc + 0], bf16_lo(v.x), acc);
-          acc = fmaf(Lam[8 * cc + 1], bf16_hi(v.x), acc);
-          acc = fmaf(Lam[8 * cc + 2], bf16_lo(v.y), acc);
-          acc = fmaf(Lam[8 * cc + 3], bf16_hi(v.y), acc);
-          acc = fmaf(Lam[8 * cc + 4], bf16_lo(v.z), acc);
-          acc = fmaf(Lam[8 * cc + 5], bf16_hi(v.z), acc);
-          acc = fmaf(Lam[8 * cc + 6], bf16_lo(v.w), acc);
-          acc = fmaf(Lam[8 * cc + 7], bf16_hi(v.w), acc);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (lane == 0) sm.ered[warp - 4] = acc;
-      }
-      named_sync_math();  // (A) S_in fully read: its buffer now receives Ar | Z | Q^T | Bm
-
-      float r1s[32], dxs[32];
-      if (ok) {
-        // ---- chunk matrices from K | Kug and KugT
+        // ---- <Lam_end, S_in>, then Lam <- 2^{L_{C-1}} Lam in place
         {
-          float vkk[32], vkt[32];
-          tmem_ld32(tbase + COL_KK + lane_off + 32 * hh, vkk);
-          tmem_ld32(tbase + COL_KT + lane_off + 32 * hh, vkt);
+          const float gC = gs.gC;
+          const uint32_t row = sS + (wg >> 1) * BIG;
+          float v[32];
+          tmem_ld32(tL, v);
           tmem_ld_wait();
-          // lanes < 16 hold the K and KugT rows, lanes >= 16 the Kug row of the same i;
-          // each value is exchanged with the partner lane (l ^ 16) as it is consumed
-          const int i = ir;
-          const float Li = gs.L[i], Lim1 = i == 0 ? 0.f : gs.L[i - 1], eti = gs.eta[i];
-          const uint32_t b1 = sS + (lo ? CC_AR : CC_QT), b2 = sS + (lo ? CC_Z : CC_BM);
-          float tpart = 0.f;
+          float acc = 0.f;
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) {
+            const uint4 sv = ld_shared_v4(row + sw128_off(n, 4 * (wg & 1) + cc));
+            acc = fmaf(v[8 * cc + 0], bf16_lo(sv.x), acc);
+            acc = fmaf(v[8 * cc + 1], bf16_hi(sv.x), acc);
+            acc = fmaf(v[8 * cc + 2], bf16_lo(sv.y), acc);
+            acc = fmaf(v[8 * cc + 3], bf16_hi(sv.y), acc);
+            acc = fmaf(v[8 * cc + 4], bf16_lo(sv.z), acc);
+            acc = fmaf(v[8 * cc + 5], bf16_hi(sv.z), acc);
+            acc = fmaf(v[8 * cc + 6], bf16_lo(sv.w), acc);
+            acc = fmaf(v[8 * cc + 7], bf16_hi(sv.w), acc);
+          }
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] *= gC;
+          tmem_st32(tL, v);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+          if (lane == 0) sm.ered[warp - 4] = acc;
+        }
+        // ---- q_j = g_j^T Lam x_j from R1^T; del (.) R1^T back
+        {
+          float vr[16], sv[16];
+          tmem_ld16(tbase + COL_R + lane_off + j0w, vr);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int j = j0w + e;
+            const float gv = lds_bf16(sw_elem(sG + (n >> 6) * TILE, j, n & 63));
+            sv[e] = gs.del[j] * vr[e];
+            vr[e] = gv * vr[e];
+          }
+          tmem_st16(tbase + COL_R + lane_off + j0w, sv);
+          const float r = reduce_scatter16(vr, lane);
+          if (!(lane & 1)) sm.redq[q][j0w + (lane >> 1)] = r;
+        }
+        // ---- p_s = x_s^T S_in^T u_s from DXb^T; gam (.) DXb^T back
+        {
+          float vd[16], sv[16];
+          tmem_ld16(tbase + COL_D + lane_off + j0w, vd);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int s = j0w + e;
+            const float xv = lds_bf16(sw_elem(sX + (n >> 6) * TILE, s, n & 63));
+            sv[e] = gs.gam[s] * vd[e];
+            vd[e] = xv * vd[e];
+          }
+          tmem_st16(tbase + COL_D + lane_off + j0w, sv);
+          const float r = reduce_scatter16(vd, lane);
+          if (!(lane & 1)) sm.redp[q][j0w + (lane >> 1)] = r;
+        }
+        tmem_st_wait();
+      }
+      named_sync_math();  // (B1) S_in read; partial sums of q, p and E written; G read
+      if (ok) {  // G <- diag(-eta del) G, rows scaled with packed bf16 multiplies
+#pragma unroll
+        for (int k = 0; k < (2 * TILE / 16) / (32 * NMATH); ++k) {
+          const uint32_t off = (uint32_t)(mt + 32 * NMATH * k) * 16;
+          const int j = (off & (TILE - 1)) >> 7;
+          const __nv_bfloat162 f2 = __float2bfloat162_rn(-gs.eta[j] * gs.del[j]);
+          const uint32_t fv = *reinterpret_cast<const uint32_t*>(&f2);
+          uint4 v = ld_shared_v4(sG + off);
+          st_shared_v4(sG + off, hmul2_bf16(v.x, fv), hmul2_bf16(v.y, fv), hmul2_bf16(v.z, fv),
+                       hmul2_bf16(v.w, fv));
+        }
+      }
+      if (ok && mt < C) {
+        const int j = mt;
+        sm.qv[j] = sm.redq[0][j] + sm.redq[1][j] + sm.redq[2][j] + sm.redq[3][j];
+        sm.pv[j] = sm.redp[0][j] + sm.redp[1][j] + sm.redp[2][j] + sm.redp[3][j];
+      }
+      float E = 0.f;
+#pragma unroll
+      for (int w = 0; w < NMATH; ++w) E += sm.ered[w];
+      named_sync_math();  // (B2) q and p complete; the S_in buffer may be overwritten
+
+      if (ok) {
+        // ---- chunk matrices from K | Kug and KugT, plus the t, t2, t3 partial sums
+        float vkk[16], vkt[16];
+        tmem_ld16(tbase + COL_KK + lane_off + j0w, vkk);
+        tmem_ld16(tbase + COL_KT + lane_off + j0w, vkt);
+        tmem_ld_wait();
+        // lanes < 16 hold the K and KugT rows, lanes >= 16 the Kug row of the same i;
+        // each value is exchanged with the partner lane (l ^ 16) as it is consumed
+        const int i = ir;
+        const float Li = gs.L[i], Lim1 = i == 0 ? 0.f : gs.L[i - 1], eti = gs.eta[i];
+        const float rai = gs.ra[i], rbi = gs.rb[i];
+        const uint32_t b1 = sS + (lo ? CC_AR : CC_QT), b2 = sS + (lo ? CC_Z : CC_BM);
+        float tpart = 0.f, t2part = 0.f, t3part = 0.f;
+        auto build = [&](auto fac_tag) {
+          constexpr bool FAC = decltype(fac_tag)::value;
+          // Both lane halves run the same straight-line code on their own data
+          // (selects, no divergent branches): lanes < 16 produce Ar and Z and the t2
+          // sum, lanes >= 16 produce Q^T and Bm and the t and t3 sums.
+          const float selA = lo ? 1.f : 0.f, selB = 1.f - selA;
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
             uint32_t m1[4], m2[4];
 #pragma unroll
-            for (int e2 = 0; e2 < 8; e2 += 2) {
-              float v0[2], v1[2];
+            for (int e4 = 0; e4 < 8; e4 += 4) {
+              const int jb = j0w + 8 * cc + e4;
+              float4 cb4, ca4, L4, Lm4, et4;
+              if (FAC) {
+                cb4 = *reinterpret_cast<const float4*>(&gs.cb[jb]);
+                ca4 = *reinterpret_cast<const float4*>(&gs.ca[jb]);
+              } else {
+                L4 = *reinterpret_cast<const float4*>(&gs.L[jb]);
+                et4 = *reinterpret_cast<const float4*>(&gs.eta[jb]);
+                Lm4 = make_float4(jb == 0 ? 0.f : gs.L[jb - 1], L4.x, L4.y, L4.z);
+              }
+              const float4 q4 = *reinterpret_cast<const float4*>(&sm.qv[jb]);
+              const float4 p4 = *reinterpret_cast<const float4*>(&sm.pv[jb]);
+              const float cbv[4] = {cb4.x, cb4.y, cb4.z, cb4.w};
+              const float cav[4] = {ca4.x, ca4.y, ca4.z, ca4.w};
+              const float Lv[4] = {L4.x, L4.y, L4.z, L4.w};
+              const float Lmv[4] = {Lm4.x, Lm4.y, Lm4.z, Lm4.w};
+              const float etv[4] = {et4.x, et4.y, et4.z, et4.w};
+              const float qvv[4] = {q4.x, q4.y, q4.z, q4.w};
+              const float pvv[4] = {p4.x, p4.y, p4.z, p4.w};
+              float v0[4], v1[4];
 #pragma unroll
-              for (int d = 0; d < 2; ++d) {
-                const int e = 8 * cc + e2 + d;
+              for (int d = 0; d < 4; ++d) {
+                const int e = 8 * cc + e4 + d;
+                const int j = jb + d;
                 const float o1 = __shfl_xor_sync(0xffffffffu, vkk[e], 16);
                 const float o2 = __shfl_xor_sync(0xffffffffu, vkt[e], 16);
                 const float kr = lo ? vkk[e] : o1;  // x_i . x_j
                 const float kg = lo ? o1 : vkk[e];  // u_i . g_j
                 const float kt = lo ? vkt[e] : o2;  // g_i . u_j
-                const int j = 32 * hh + e;
-                const float Ljm1 = j == 0 ? 0.f : gs.L[j - 1];
-                const float bij = exp2f(fminf(Ljm1 - Li, 0.f));                    // j > i
-                const float aij = -gs.eta[j] * exp2f(fminf(Lim1 - gs.L[j], 0.f));  // j < i
-                if (lo) {
-                  v0[d] = (j > i) ? bij * kr : 0.f;                                 // Ar
-                  v1[d] = (j < i) ? aij * kg : ((j > i) ? -eti * bij * kt : 0.f);   // Z
+                float bij, aij;                     // b_ij (j > i), a_ij (j < i)
+                if (FAC) {
+                  bij = cbv[d] * rbi;
+                  aij = rai * cav[d];
                 } else {
-                  v0[d] = (j < i) ? kg * kr : 0.f;  // Q^T
-                  v1[d] = (j > i) ? bij : 0.f;      // Bm
-                  if (j > i) tpart = fmaf(bij * kr, kt, tpart);
+                  bij = exp2f(fminf(Lmv[d] - Li, 0.f));
+                  aij = -etv[d] * exp2f(fminf(Lim1 - Lv[d], 0.f));
                 }
+                const float lt = (j < i) ? 1.f : 0.f, gt = (j > i) ? 1.f : 0.f;
+                const float bg = gt * bij, al = lt * aij;
+                // lanes < 16: Ar = b kr, Z = a kg - eta_i b kt ; lanes >= 16: Q^T = kg kr, Bm = b
+                v0[d] = kr * (lo ? bg : lt * kg);
+                v1[d] = lo ? fmaf(al, kg, -eti * bg * kt) : bg;
+                t2part = fmaf(selA * al, qvv[d], t2part);
+                tpart = fmaf(selB * bg * kr, kt, tpart);
+                t3part = fmaf(selB * bg, pvv[d], t3part);
               }
-              m1[e2 >> 1] = pack_bf16(v0[0], v0[1]);
-              m2[e2 >> 1] = pack_bf16(v1[0], v1[1]);
+              m1[e4 >> 1] = pack_bf16(v0[0], v0[1]);
+              m1[(e4 >> 1) + 1] = pack_bf16(v0[2], v0[3]);
+              m2[e4 >> 1] = pack_bf16(v1[0], v1[1]);
+              m2[(e4 >> 1) + 1] = pack_bf16(v1[2], v1[3]);
             }
-            st_shared_v4(b1 + sw128_off(i, 4 * hh + cc), m1[0], m1[1], m1[2], m1[3]);
-            st_shared_v4(b2 + sw128_off(i, 4 * hh + cc), m2[0], m2[1], m2[2], m2[3]);
+            st_shared_v4(b1 + sw128_off(i, 2 * wg + cc), m1[0], m1[1], m1[2], m1[3]);
+            st_shared_v4(b2 + sw128_off(i, 2 * wg + cc), m2[0], m2[1], m2[2], m2[3]);
           }
-          if (!lo) sm.tv[hh][i] = tpart;
-        }
-        // ---- q_j = g_j^T Lam x_j (from R1^T), then G <- diag(-eta del) G in place
-        {
-          float vr[32];
-          tmem_ld32(tbase + COL_R + lane_off + 32 * hh, vr);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int j = 32 * hh + e;
-            const uint32_t ga = sw_elem(sG + (n >> 6) * TILE, j, n & 63);
-            const float gv = lds_bf16(ga);
-            r1s[e] = gs.del[j] * vr[e];
-            vr[e] = gv * vr[e];  // partial product of q_j
-            sts_bf16(ga, -gs.eta[j] * gs.del[j] * gv);
-          }
-          sm.redq[q][32 * hh + lane] = reduce_scatter32(vr, lane);
-        }
-        // ---- p_s = x_s^T S_in^T u_s (from DXb^T)
-        {
-          float vd[32];
-          tmem_ld32(tbase + COL_D + lane_off + 32 * hh, vd);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int s = 32 * hh + e;
-            const float xv = lds_bf16(sw_elem(sX + (n >> 6) * TILE, s, n & 63));
-            dxs[e] = gs.gam[s] * vd[e];
-            vd[e] = xv * vd[e];  // partial product of p_s
-          }
-          sm.redp[q][32 * hh + lane] = reduce_scatter32(vd, lane);
+        };
+        if (gs.fac) build(std::true_type{});
+        else build(std::false_type{});
+        if (lo) {
+          sm.t2v[wg][i] = t2part;
+        } else {
+          sm.tv[wg][i] = tpart;
+          sm.t3v[wg][i] = t3part;
         }
         tc_fence_before();
         fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.m1done);
       }
-      named_sync_math();  // (B) chunk matrices, scaled G and the partial sums are complete
-      if (ok && lane == 0) mbar_arrive(&sm.m1done);
-      float E = 0.f;
-#pragma unroll
-      for (int w = 0; w < 8; ++w) E += sm.ered[w];
+      named_sync_math();  // (B3) t complete
       if (ok && mt < C) {
         const int j = mt;
-        const float qj = sm.redq[0][j] + sm.redq[1][j] + sm.redq[2][j] + sm.redq[3][j];
-        const float pj = sm.redp[0][j] + sm.redp[1][j] + sm.redp[2][j] + sm.redp[3][j];
-        sm.qv[j] = qj;
-        sm.pv[j] = pj;
-        const float deta = -(gs.del[j] * qj + sm.tv[0][j] + sm.tv[1][j]);
+        const float deta =
+            -(gs.del[j] * sm.qv[j] + sm.tv[0][j] + sm.tv[1][j] + sm.tv[2][j] + sm.tv[3][j]);
         if (t0 + j < T) p.d_eta[tokbase + j] = deta;
       }
 
-      // ---- phase 2: r -> dg, dx, and the V part of dalpha
+      // ---- phase 2: dg from r^T, dx from dx^T, and the V part of dalpha
       ok = ok && mbar_wait_warp(&sm.b2full, it & 1, wc, W_M_B2);
       tc_fence_after();
       if (ok) {
         {
-          float vv[32], vri[32];
-          tmem_ld32(tbase + COL_KT + lane_off + 32 * hh, vv);
-          tmem_ld32(tbase + COL_R + lane_off + 32 * hh, vri);
+          float vv[16], vri[16];
+          tmem_ld16(tbase + COL_KT + lane_off + j0w, vv);
+          tmem_ld16(tbase + COL_R + lane_off + j0w, vri);
           tmem_ld_wait();
           if (!lo) {
             const int i = ir;
-            const float Lim1 = i == 0 ? 0.f : gs.L[i - 1];
             float hpart = 0.f;
+            if (gs.fac) {
+              const float rai = gs.ra[i];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int j = 32 * hh + e;
-              const float aij = -gs.eta[j] * exp2f(fminf(Lim1 - gs.L[j], 0.f));
-              if (j < i) hpart = fmaf(aij, vv[e], hpart);
+              for (int e = 0; e < 16; ++e) {
+                const int j = j0w + e;
+                if (j < i) hpart = fmaf(rai * gs.ca[j], vv[e], hpart);
+              }
+            } else {
+              const float Lim1 = i == 0 ? 0.f : gs.L[i - 1];
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                const int j = j0w + e;
+                const float aij = -gs.eta[j] * exp2f(fminf(Lim1 - gs.L[j], 0.f));
+                if (j < i) hpart = fmaf(aij, vv[e], hpart);
+              }
             }
-            sm.hv[hh][i] = hpart;
+            sm.hv[wg][i] = hpart;
           }
-          __nv_bfloat16* dgo = p.dg + tokbase * 128 + n;
+          // dg^T[n][i] = -eta_i r^T[n][i] -> staging tile [i rows][n] (the bf16 Lam tile is
+          // free until the Lam update: MMA2 has read it)
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int i = 32 * hh + e;
-            if (t0 + i < T)
-              dgo[(size_t)i * 128] = __float2bfloat16_rn(-gs.eta[i] * (r1s[e] + vri[e]));
+          for (int e = 0; e < 16; ++e) {
+            const int i = j0w + e;
+            sts_u16(sw_elem(sLb + (n >> 6) * TILE, i, n & 63), -gs.eta[i] * vri[e]);
           }
         }
         {
-          float vda[32];
-          tmem_ld32(tbase + COL_D + lane_off + 32 * hh, vda);
+          float vda[16];
+          tmem_ld16(tbase + COL_D + lane_off + j0w, vda);
           tmem_ld_wait();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sm.m2done);
-          __nv_bfloat16* dxo = p.dx + tokbase * 128 + n;
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int i = 32 * hh + e;
-            if (t0 + i < T) dxo[(size_t)i * 128] = __float2bfloat16_rn(vda[e] + dxs[e]);
-          }
+          for (int e = 0; e < 16; ++e)
+            sts_u16(sw_elem(sLb + 2 * TILE + (n >> 6) * TILE, j0w + e, n & 63), vda[e]);
         }
-        // X <- diag(gam) X in place for dLam = U^T Xg
-#pragma unroll 8
-        for (int e = 0; e < 32; ++e) {
-          const int s = 32 * hh + e;
-          const uint32_t xa = sw_elem(sX + (n >> 6) * TILE, s, n & 63);
-          sts_bf16(xa, gs.gam[s] * lds_bf16(xa));
+        // X <- diag(gam) X in place for Lam += U^T Xg (rows, packed bf16 multiplies)
+#pragma unroll
+        for (int k = 0; k < (2 * TILE / 16) / (32 * NMATH); ++k) {
+          const uint32_t off = (uint32_t)(mt + 32 * NMATH * k) * 16;
+          const int sr = (off & (TILE - 1)) >> 7;
+          const __nv_bfloat162 f2 = __float2bfloat162_rn(gs.gam[sr]);
+          const uint32_t fv = *reinterpret_cast<const uint32_t*>(&f2);
+          uint4 v = ld_shared_v4(sX + off);
+          st_shared_v4(sX + off, hmul2_bf16(v.x, fv), hmul2_bf16(v.y, fv), hmul2_bf16(v.z, fv),
+                       hmul2_bf16(v.w, fv));
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.xscaled);
       }
-      named_sync_math();  // (C) hv of both halves written
+      named_sync_math();  // (B4) hv of all warpgroups and the dg / dx staging tiles written
+      if (ok && mt == 0) {  // rows past T are clipped by the tensor maps
+        tma_store_3d(&tmDG, sm.Lb, 0, t0, bh);
+        tma_store_3d(&tmDG, sm.Lb + TILE, 64, t0, bh);
+        tma_store_3d(&tmDX, sm.Lb + 2 * TILE, 0, t0, bh);
+        tma_store_3d(&tmDX, sm.Lb + 3 * TILE, 64, t0, bh);
+        tma_store_commit();
+      }
       if (ok && mt < C) {
         const int i = mt;
-        const float Li = gs.L[i], Lim1 = i == 0 ? 0.f : gs.L[i - 1];
-        float t2 = 0.f, t3 = 0.f;
-        for (int j = 0; j < i; ++j)
-          t2 = fmaf(-gs.eta[j] * exp2f(fminf(Lim1 - gs.L[j], 0.f)), sm.qv[j], t2);
-        for (int s = i + 1; s < C; ++s)
-          t3 = fmaf(exp2f(fminf(gs.L[s - 1] - Li, 0.f)), sm.pv[s], t3);
-        const float da = gs.gam[i] * gs.del[i] * E + gs.del[i] * t2 + gs.gam[i] * t3 +
-                         sm.hv[0][i] + sm.hv[1][i];
+        const float t2 = sm.t2v[0][i] + sm.t2v[1][i] + sm.t2v[2][i] + sm.t2v[3][i];
+        const float t3 = sm.t3v[0][i] + sm.t3v[1][i] + sm.t3v[2][i] + sm.t3v[3][i];
+        const float h4 = sm.hv[0][i] + sm.hv[1][i] + sm.hv[2][i] + sm.hv[3][i];
+        const float da = gs.gam[i] * gs.del[i] * E + gs.del[i] * t2 + gs.gam[i] * t3 + h4;
         if (t0 + i < T) p.d_alpha[tokbase + i] = da;
       }
 
-      // ---- phase 3: Lam <- 2^{L_{C-1}} Lam + dLam
+      // ---- phase 3: bf16 copy of the new Lam for the next chunk's products
       ok = ok && mbar_wait_warp(&sm.b3full, it & 1, wc, W_M_B3);
       tc_fence_after();
+      if (mt == 0) tma_store_wait_read();  // the staging tiles are about to be overwritten
+      named_sync_math();  // (B4b)
       if (ok) {
-        float v0[32], v1[32];
-        tmem_ld32(tbase + COL_DL + lane_off + 64 * hh, v0);
-        tmem_ld32(tbase + COL_DL + lane_off + 64 * hh + 32, v1);
+        const uint32_t lrow = sLb + (wg >> 1) * BIG;
+        float v[32];
+        tmem_ld32(tL, v);
         tmem_ld_wait();
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+          st_shared_v4(lrow + sw128_off(n, 4 * (wg & 1) + cc), pack_bf16(v[8 * cc], v[8 * cc + 1]),
+                       pack_bf16(v[8 * cc + 2], v[8 * cc + 3]),
+                       pack_bf16(v[8 * cc + 4], v[8 * cc + 5]),
+                       pack_bf16(v[8 * cc + 6], v[8 * cc + 7]));
         tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.m3done);
-        const float gC = gs.gC;
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          Lam[e] = fmaf(gC, Lam[e], v0[e]);
-          Lam[32 + e] = fmaf(gC, Lam[32 + e], v1[e]);
-        }
-        const uint32_t lrow = smem_u32(sm.Lb + hh * BIG);
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc)
-          st_shared_v4(lrow + sw128_off(n, cc), pack_bf16(Lam[8 * cc], Lam[8 * cc + 1]),
-                       pack_bf16(Lam[8 * cc + 2], Lam[8 * cc + 3]),
-                       pack_bf16(Lam[8 * cc + 4], Lam[8 * cc + 5]),
-                       pack_bf16(Lam[8 * cc + 6], Lam[8 * cc + 7]));
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -627,23 +792,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           mbar_arrive(&sm.gempty[g]);
         }
       }
-      named_sync_math();  // (D) per-chunk scratch consumed before the next chunk writes it
+      named_sync_math();  // (B5) per-chunk scratch consumed before the next chunk writes it
     }
 
+    if (mt == 0) tma_store_wait_all();
     // ---- this scan's dW0 partial: the last b3full wait covered every product
-    {
-      if (ok) {
-        float v0[32], v1[32];
-        tmem_ld32(tbase + COL_W + lane_off + 64 * hh, v0);
-        tmem_ld32(tbase + COL_W + lane_off + 64 * hh + 32, v1);
-        tmem_ld_wait();
-        float4* dst = reinterpret_cast<float4*>(p.dW0_part + ((size_t)bh * 128 + n) * 128 + 64 * hh);
+    if (ok) {
+      float v[32];
+      tmem_ld32(tbase + COL_W + lane_off + 32 * wg, v);
+      tmem_ld_wait();
+      float4* dst = reinterpret_cast<float4*>(p.dW0_part + ((size_t)bh * 128 + n) * 128 + 32 * wg);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          dst[e] = make_float4(v0[4 * e], v0[4 * e + 1], v0[4 * e + 2], v0[4 * e + 3]);
-          dst[8 + e] = make_float4(v1[4 * e], v1[4 * e + 1], v1[4 * e + 2], v1[4 * e + 3]);
-        }
-      }
+      for (int e = 0; e < 8; ++e) dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
     }
   }
 
@@ -659,12 +819,14 @@ bool bwd_shape_ok(int din, int dout) { return din == 128 && dout == 128; }
 
 cudaError_t launch_bwd(const TcBwdParams& prm, const void* x, const void* g, const void* dy,
                        const void* ckpt, cudaStream_t st) {
-  CUtensorMap mx, mg, mu, ms;
+  CUtensorMap mx, mg, mu, ms, mdx, mdg;
   const uint64_t BH = (uint64_t)prm.B * prm.H;
   const uint64_t nch = (uint64_t)(prm.T + C - 1) / C;
   if (!make_map_bf16_3d(&mx, x, 128, prm.T, BH, C) || !make_map_bf16_3d(&mg, g, 128, prm.T, BH, C) ||
       !make_map_bf16_3d(&mu, dy, 128, prm.T, BH, C) ||
-      !make_map_bf16_3d(&ms, ckpt, 128, 128, BH * nch, 128))
+      !make_map_bf16_3d(&ms, ckpt, 128, 128, BH * nch, 128) ||
+      !make_map_bf16_3d(&mdx, prm.dx, 128, prm.T, BH, C) ||
+      !make_map_bf16_3d(&mdg, prm.dg, 128, prm.T, BH, C))
     return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!attr_set) {
@@ -673,7 +835,7 @@ cudaError_t launch_bwd(const TcBwdParams& prm, const void* x, const void* g, con
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  bwd_kernel<<<(int)BH, NTHREADS, kSmemBytes, st>>>(mx, mg, mu, ms, prm);
+  bwd_kernel<<<(int)BH, NTHREADS, kSmemBytes, st>>>(mx, mg, mu, ms, mdx, mdg, prm);
   count_launch();
   return cudaGetLastError();
 }

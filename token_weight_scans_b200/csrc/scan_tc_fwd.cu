@@ -55,13 +55,18 @@ constexpr uint32_t COL_Y1 = 128;                 // + 64 * buffer
 constexpr uint32_t COL_Y2 = 256;                 // + 64 * buffer
 constexpr uint32_t COL_DS = 384;                 // 128 columns
 
+// With M = L_{31}, the mask factor -eta_j 2^{L_{i-1} - L_j} = ra_i ca_j whenever
+// every exponent stays inside fp32 range: fac = (|L_{C-1}| <= 120).
 struct GateSlot {
   float L[C];     // chunk-local inclusive cumulative sum of log2 alpha
   float eta[C];
   float gam[C];   // 2^{L_{i-1}}
   float w[C];     // -eta_j 2^{L_{C-1} - L_j}
+  float ra[C];    // 2^{L_{i-1} - M}
+  float ca[C];    // -eta_j 2^{M - L_j}
   float gC;       // 2^{L_{C-1}}
-  float pad[3];
+  int fac;
+  float pad[2];
 };
 
 struct Smem {
@@ -311,7 +316,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           gs.gam[lane + 32] = exp2f(lane == 0 ? last0 : pm1);
           gs.w[lane] = -e0 * exp2f(Lend - l0);
           gs.w[lane + 32] = -e1 * exp2f(Lend - l1);
-          if (lane == 0) gs.gC = exp2f(Lend);
+          gs.ra[lane] = exp2f((lane == 0 ? 0.f : pm0) - last0);
+          gs.ra[lane + 32] = exp2f((lane == 0 ? last0 : pm1) - last0);
+          gs.ca[lane] = -e0 * exp2f(last0 - l0);
+          gs.ca[lane + 32] = -e1 * exp2f(last0 - l1);
+          if (lane == 0) {
+            gs.gC = exp2f(Lend);
+            gs.fac = (Lend >= -120.f) ? 1 : 0;
+          }
           __syncwarp();
           mbar_arrive(&sm.gfull[g]);
         }
@@ -376,14 +388,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int i = 16 * q + lane;
         const float Lm1 = i == 0 ? 0.f : gs.L[i - 1];
         uint32_t pk[16];
+        if (gs.fac) {
+          const float rai = gs.ra[i];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int j = 32 * hh + e;
-          const float f0 = exp2f(fminf(Lm1 - gs.L[j], 0.f));
-          const float f1 = exp2f(fminf(Lm1 - gs.L[j + 1], 0.f));
-          const float p0 = (j < i) ? v[e] * (-gs.eta[j]) * f0 : 0.f;
-          const float p1 = (j + 1 < i) ? v[e + 1] * (-gs.eta[j + 1]) * f1 : 0.f;
-          pk[e >> 1] = pack_bf16(p0, p1);
+          for (int e = 0; e < 32; e += 2) {
+            const int j = 32 * hh + e;
+            const float p0 = (j < i) ? v[e] * rai * gs.ca[j] : 0.f;
+            const float p1 = (j + 1 < i) ? v[e + 1] * rai * gs.ca[j + 1] : 0.f;
+            pk[e >> 1] = pack_bf16(p0, p1);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int j = 32 * hh + e;
+            const float f0 = exp2f(fminf(Lm1 - gs.L[j], 0.f));
+            const float f1 = exp2f(fminf(Lm1 - gs.L[j + 1], 0.f));
+            const float p0 = (j < i) ? v[e] * (-gs.eta[j]) * f0 : 0.f;
+            const float p1 = (j + 1 < i) ? v[e + 1] * (-gs.eta[j + 1]) * f1 : 0.f;
+            pk[e >> 1] = pack_bf16(p0, p1);
+          }
         }
         const uint32_t prow = smem_u32(sm.P);
 #pragma unroll
