@@ -79,8 +79,10 @@ GRADLEV_API const char* gradlev_status_string(gradlev_status s);
 
 /* Whether (B, H, T, d_in, d_out, dt) is supported: GRADLEV_OK, or
  * GRADLEV_ERR_INVALID_ARG / GRADLEV_ERR_UNSUPPORTED without touching the GPU.
- * Supported: B, H, T >= 1 with B*H*T < 2^31; d_in % 4 == 0, d_out % 8 == 0,
- * 8 <= d_in, d_out and d_in * d_out <= 16384. */
+ * Supported: B, H, T >= 1 with B*H*T < 2^31, and either
+ *   - GRADLEV_BF16 with d_in = 128 and d_out in {128, 256} (tensor-core kernels), or
+ *   - either dtype with d_in % 4 == 0, d_out % 8 == 0, 8 <= d_in, d_out and
+ *     d_in * d_out <= 16384 (CUDA-core kernels). */
 GRADLEV_API gradlev_status gradlev_scan_supported(int B, int H, int T, int d_in, int d_out,
                                       gradlev_dtype dt);
 

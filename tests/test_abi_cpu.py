@@ -55,6 +55,9 @@ def test_status_strings(L):
     ((1, 1, 4, 6, 16), 0, 2),
     ((1, 1, 4, 16, 12), 0, 2),
     ((1, 1, 4, 256, 256), 0, 2),
+    ((1, 16, 32768, 128, 256), 1, 0),
+    ((1, 16, 32768, 128, 256), 0, 2),
+    ((1, 1, 4, 128, 384), 1, 2),
 ])
 def test_supported_shapes(L, shape, dt, ok):
     assert tw.gradlev_scan_supported(*shape, dt) == ok

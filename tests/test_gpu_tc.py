@@ -188,3 +188,10 @@ def test_tc_bwd_bit_exact_integer_inputs():
     got = gpu_fwd_bwd(d)
     for k in ("y",) + BWD_OUTS:
         assert np.array_equal(got[k], ref[k]), (k, rel_err(got[k], ref[k]))
+
+
+@pytest.mark.parametrize("T", [70, 200])
+def test_tc_rectangular_dout256(T):
+    """d_out = 256: forward on two 128-row slices, backward as two slice problems."""
+    d = inputs.draw(2, 2, T, 128, 256, dtype="bf16", alpha_mode="log_uniform", seed=600 + T)
+    check_all(gpu_fwd_bwd(d), oracle_fwd_bwd(d), f"d_out=256 T={T}")

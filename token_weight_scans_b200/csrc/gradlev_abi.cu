@@ -2,7 +2,8 @@
 // workspace sizing and kernel dispatch. No device memory is allocated here.
 //
 // Kernel families:
-//   * tcgen05 kernels (scan_tc_fwd.cu, scan_tc_bwd.cu): bf16 I/O, d_in = d_out = 128;
+//   * tcgen05 kernels (scan_tc_fwd.cu, scan_tc_bwd.cu): bf16 I/O, d_in = 128 and
+//     d_out in {128, 256} (one 128-row slice of d_out per CTA / per backward launch);
 //   * CUDA-core kernels (scan_ffma.cu): everything else that is supported
 //     (float32 I/O, or bf16 with d_in * d_out <= 16384).
 // The two families exchange state checkpoints in different formats; a
@@ -89,10 +90,13 @@ gradlev_status bwd_run(int B, int H, int T, int din, int dout, gradlev_dtype dt,
     states = own;
   }
   if (use_tc(din, dout, dt)) {
-    tc::TcBwdParams prm{B, H, T, din, dout, eta, alpha, W0,
-                        static_cast<__nv_bfloat16*>(dx), static_cast<__nv_bfloat16*>(dg),
-                        d_eta, d_alpha, dW0_part, status, kWaitTimeoutNs};
-    if (tc::launch_bwd(prm, x, g, dy, states, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
+    // one launch per 128-row slice of d_out; later slices accumulate dx, d_eta, d_alpha
+    for (int n0 = 0; n0 < dout; n0 += 128) {
+      tc::TcBwdParams prm{B, H, T, din, dout, n0, n0 > 0 ? 1 : 0, eta, alpha, W0,
+                          static_cast<__nv_bfloat16*>(dx), static_cast<__nv_bfloat16*>(dg),
+                          d_eta, d_alpha, dW0_part, status, kWaitTimeoutNs};
+      if (tc::launch_bwd(prm, x, g, dy, states, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
+    }
     if (ffma::launch_reduce_dW0(dW0_part, dW0, B, H, din * dout, st) != cudaSuccess)
       return GRADLEV_ERR_CUDA;
     return GRADLEV_OK;

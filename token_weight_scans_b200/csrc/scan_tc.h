@@ -22,8 +22,14 @@ struct TcFwdParams {
   int inject;               // test hook: 1 = withhold one completion signal
 };
 
+// The reverse scan of one 128-row slice [n0, n0+128) of d_out: the rows of the
+// state and adjoint evolve independently, so a d_out = 256 problem is two
+// slice problems whose dx, d_eta and d_alpha add up (accumulate = 1 on the
+// second slice) and whose dg and dW0 rows are disjoint.
 struct TcBwdParams {
-  int B, H, T, din, dout;   // din == dout == 128
+  int B, H, T, din, dout;   // din == 128, dout in {128, 256}
+  int n0;                   // first d_out row of this slice
+  int accumulate;           // add dx, d_eta, d_alpha onto the values already there
   const float* eta;
   const float* alpha;
   const float* W0;          // [H,128,128] float32

@@ -1,4 +1,5 @@
-// Tensor-core (tcgen05/TMEM) reverse GradLev scan for bf16 I/O, d_in = d_out = 128.
+// Tensor-core (tcgen05/TMEM) reverse GradLev scan for bf16 I/O, d_in = 128 and
+// one 128-row slice of d_out per launch.
 //
 // Reverse-mode derivative of S_{t+1} = alpha_t S_t - eta_t g_t x_t^T,
 // y_t = (W0 + S_t) x_t (Cognaptus, "Parallelize the Training, Keep the Learning
@@ -178,39 +179,6 @@ __device__ __forceinline__ float reduce_scatter16(float (&v)[16], int lane) {
   return w1 + __shfl_xor_sync(0xffffffffu, w1, 1);
 }
 
-// Sum of v[0..31] over the 32 lanes of the warp; lane l returns the total of index l.
-__device__ __forceinline__ float reduce_scatter32(float (&v)[32], int lane) {
-  float w16[16], w8[8], w4[4], w2[2];
-  const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4, b1 = lane & 2, b0 = lane & 1;
-#pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    const float send = b4 ? v[k] : v[k + 16];
-    const float keep = b4 ? v[k + 16] : v[k];
-    w16[k] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-  }
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const float send = b3 ? w16[k] : w16[k + 8];
-    const float keep = b3 ? w16[k + 8] : w16[k];
-    w8[k] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-  }
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const float send = b2 ? w8[k] : w8[k + 4];
-    const float keep = b2 ? w8[k + 4] : w8[k];
-    w4[k] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-  }
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const float send = b1 ? w4[k] : w4[k + 2];
-    const float keep = b1 ? w4[k + 2] : w4[k];
-    w2[k] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-  }
-  const float send = b0 ? w2[0] : w2[1];
-  const float keep = b0 ? w2[1] : w2[0];
-  return keep + __shfl_xor_sync(0xffffffffu, send, 1);
-}
-
 }  // namespace
 
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -265,7 +233,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (warp >= 4) {
     // W0 -> bf16 swizzled [k-block][n rows]; Lam_T = 0
     const int t = threadIdx.x - 128;
-    const float* W0 = p.W0 + (size_t)h * 128 * 128;
+    const float* W0 = p.W0 + ((size_t)h * p.dout + p.n0) * 128;
     for (int idx = t; idx < 128 * 16; idx += 32 * NMATH) {
       const int n = idx >> 4, ck = idx & 15;
       const int kb = ck >> 3, c = ck & 7;
@@ -293,15 +261,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           mbar_arrive_expect_tx(&sm.xfull[st], 6 * TILE);
           tma_load_3d(sm.X[st], &tmX, &sm.xfull[st], 0, c * C, bh);
           tma_load_3d(sm.X[st] + TILE, &tmX, &sm.xfull[st], 64, c * C, bh);
-          tma_load_3d(sm.G[st], &tmG, &sm.xfull[st], 0, c * C, bh);
-          tma_load_3d(sm.G[st] + TILE, &tmG, &sm.xfull[st], 64, c * C, bh);
-          tma_load_3d(sm.U[st], &tmU, &sm.xfull[st], 0, c * C, bh);
-          tma_load_3d(sm.U[st] + TILE, &tmU, &sm.xfull[st], 64, c * C, bh);
+          tma_load_3d(sm.G[st], &tmG, &sm.xfull[st], p.n0, c * C, bh);
+          tma_load_3d(sm.G[st] + TILE, &tmG, &sm.xfull[st], p.n0 + 64, c * C, bh);
+          tma_load_3d(sm.U[st], &tmU, &sm.xfull[st], p.n0, c * C, bh);
+          tma_load_3d(sm.U[st] + TILE, &tmU, &sm.xfull[st], p.n0 + 64, c * C, bh);
           xi = it + 1;
           if (!mbar_wait(&sm.sempty, (it & 1) ^ 1, wc, W_TMA_SEMPTY)) break;
           mbar_arrive_expect_tx(&sm.sfull, 2 * BIG);
-          tma_load_3d(sm.Sin, &tmS, &sm.sfull, 0, 0, bh * nch + c);
-          tma_load_3d(sm.Sin + BIG, &tmS, &sm.sfull, 64, 0, bh * nch + c);
+          tma_load_3d(sm.Sin, &tmS, &sm.sfull, 0, p.n0, bh * nch + c);
+          tma_load_3d(sm.Sin + BIG, &tmS, &sm.sfull, 64, p.n0, bh * nch + c);
           si = it + 1;
         }
         for (int it = xi > NS ? xi - NS : 0; it < xi; ++it)
@@ -684,7 +652,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int j = mt;
         const float deta =
             -(gs.del[j] * sm.qv[j] + sm.tv[0][j] + sm.tv[1][j] + sm.tv[2][j] + sm.tv[3][j]);
-        if (t0 + j < T) p.d_eta[tokbase + j] = deta;
+        if (t0 + j < T) p.d_eta[tokbase + j] = p.accumulate ? p.d_eta[tokbase + j] + deta : deta;
       }
 
       // ---- phase 2: dg from r^T, dx from dx^T, and the V part of dalpha
@@ -732,6 +700,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sm.m2done);
+          if (p.accumulate) {  // add the dx of the slices already done
+            const __nv_bfloat16* dxo = p.dx + tokbase * 128 + n;
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              if (t0 + j0w + e < T) vda[e] += __bfloat162float(dxo[(size_t)(j0w + e) * 128]);
+          }
 #pragma unroll
           for (int e = 0; e < 16; ++e)
             sts_u16(sw_elem(sLb + 2 * TILE + (n >> 6) * TILE, j0w + e, n & 63), vda[e]);
@@ -753,8 +727,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       named_sync_math();  // (B4) hv of all warpgroups and the dg / dx staging tiles written
       if (ok && mt == 0) {  // rows past T are clipped by the tensor maps
-        tma_store_3d(&tmDG, sm.Lb, 0, t0, bh);
-        tma_store_3d(&tmDG, sm.Lb + TILE, 64, t0, bh);
+        tma_store_3d(&tmDG, sm.Lb, p.n0, t0, bh);
+        tma_store_3d(&tmDG, sm.Lb + TILE, p.n0 + 64, t0, bh);
         tma_store_3d(&tmDX, sm.Lb + 2 * TILE, 0, t0, bh);
         tma_store_3d(&tmDX, sm.Lb + 3 * TILE, 64, t0, bh);
         tma_store_commit();
@@ -765,7 +739,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const float t3 = sm.t3v[0][i] + sm.t3v[1][i] + sm.t3v[2][i] + sm.t3v[3][i];
         const float h4 = sm.hv[0][i] + sm.hv[1][i] + sm.hv[2][i] + sm.hv[3][i];
         const float da = gs.gam[i] * gs.del[i] * E + gs.del[i] * t2 + gs.gam[i] * t3 + h4;
-        if (t0 + i < T) p.d_alpha[tokbase + i] = da;
+        if (t0 + i < T) p.d_alpha[tokbase + i] = p.accumulate ? p.d_alpha[tokbase + i] + da : da;
       }
 
       // ---- phase 3: bf16 copy of the new Lam for the next chunk's products
@@ -801,7 +775,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       float v[32];
       tmem_ld32(tbase + COL_W + lane_off + 32 * wg, v);
       tmem_ld_wait();
-      float4* dst = reinterpret_cast<float4*>(p.dW0_part + ((size_t)bh * 128 + n) * 128 + 32 * wg);
+      float4* dst = reinterpret_cast<float4*>(p.dW0_part + ((size_t)bh * p.dout + p.n0 + n) * 128 + 32 * wg);
 #pragma unroll
       for (int e = 0; e < 8; ++e) dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
     }
@@ -815,18 +789,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
-bool bwd_shape_ok(int din, int dout) { return din == 128 && dout == 128; }
+bool bwd_shape_ok(int din, int dout) { return din == 128 && (dout == 128 || dout == 256); }
 
 cudaError_t launch_bwd(const TcBwdParams& prm, const void* x, const void* g, const void* dy,
                        const void* ckpt, cudaStream_t st) {
   CUtensorMap mx, mg, mu, ms, mdx, mdg;
   const uint64_t BH = (uint64_t)prm.B * prm.H;
   const uint64_t nch = (uint64_t)(prm.T + C - 1) / C;
-  if (!make_map_bf16_3d(&mx, x, 128, prm.T, BH, C) || !make_map_bf16_3d(&mg, g, 128, prm.T, BH, C) ||
-      !make_map_bf16_3d(&mu, dy, 128, prm.T, BH, C) ||
-      !make_map_bf16_3d(&ms, ckpt, 128, 128, BH * nch, 128) ||
+  const uint64_t D = (uint64_t)prm.dout;
+  if (!make_map_bf16_3d(&mx, x, 128, prm.T, BH, C) || !make_map_bf16_3d(&mg, g, D, prm.T, BH, C) ||
+      !make_map_bf16_3d(&mu, dy, D, prm.T, BH, C) ||
+      !make_map_bf16_3d(&ms, ckpt, 128, D, BH * nch, 128) ||
       !make_map_bf16_3d(&mdx, prm.dx, 128, prm.T, BH, C) ||
-      !make_map_bf16_3d(&mdg, prm.dg, 128, prm.T, BH, C))
+      !make_map_bf16_3d(&mdg, prm.dg, D, prm.T, BH, C))
     return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!attr_set) {
