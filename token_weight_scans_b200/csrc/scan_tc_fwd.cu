@@ -11,21 +11,23 @@
 //   y_i = W0 x_i + 2^{L_{i-1}} S x_i + sum_{j<i} (x_i.x_j) (-eta_j) 2^{L_{i-1}-L_j} g_j
 //   S'  = 2^{L_{C-1}} S + sum_j (-eta_j 2^{L_{C-1}-L_j}) g_j x_j^T
 //
-// All products are done transposed, with d_out on the 128 TMEM lanes:
+// Products (the output ones token-major, so that each epilogue thread owns a
+// contiguous piece of one output row):
 //   K    = X X^T                         (M=64 tokens, N=64, K=d_in)        -> TMEM
 //   P_ij = K_ij (-eta_j) 2^{L_{i-1}-L_j}  (j < i), bf16 in shared memory
-//   Y1^T = W0 X^T + G^T P^T               (M=128, N=64, K=d_in+C)            -> TMEM
-//   Y2^T = S X^T                          (M=128, N=64, K=d_in)              -> TMEM
+//   Y1   = X W0^T + P G                   (M=64 tokens, N=128, K=d_in+C)     -> TMEM
+//   Y2   = X S^T                          (M=64 tokens, N=128, K=d_in)       -> TMEM
 //   dS   = G^T Xhat, Xhat_j = w_j x_j     (M=128, N=d_in, K=C)               -> TMEM
-//   y_i  = Y1^T[:, i] + 2^{L_{i-1}} Y2^T[:, i]; S <- 2^{L_{C-1}} S + dS (fp32, registers)
+//   y_i  = Y1[i, :] + 2^{L_{i-1}} Y2[i, :]; S <- 2^{L_{C-1}} S + dS (fp32, registers)
 //
 // Warp roles (12 warps): 0 TMA producer, 1 MMA issuer (+TMEM owner), 2 gate
 // prep (log2 alpha cumulative sums, prefetched) and half of the scaled-X tile,
-// 3 the other half of the scaled-X tile, 4..11 two math warpgroups (state
-// update, mask of the next chunk, output epilogue), warpgroup h handling
-// columns [64h, 64h+64) of the state and tokens [32h, 32h+32) of the output.
-// The bf16 copy of the state is double-buffered so the state update of chunk
-// c overlaps the S X^T product of chunk c.
+// 3 the other half of the scaled-X tile (double-buffered, so these two warps
+// run a chunk ahead), 4..11 two math warpgroups (state update, mask of the
+// next chunk, output epilogue): warpgroup h owns state columns [64h, 64h+64)
+// and output columns [64h, 64h+64) of the slice. The bf16 copy of the state is
+// double-buffered so the state update of chunk c overlaps the S X^T product of
+// chunk c.
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -44,16 +46,18 @@ using namespace sm100;
 namespace {
 
 constexpr int C = 64;          // tokens per chunk
-constexpr int NS = 3;          // TMA stages (X and G tiles)
+constexpr int NS = 2;          // TMA stages (X and G tiles)
 constexpr int GS = 4;          // gate slots
 constexpr int NTHREADS = 384;  // 12 warps
 constexpr int TILE = C * 128;  // bytes of one [64 rows x 128 B] swizzled block
+constexpr int BIG = 128 * 128; // bytes of one [128 rows x 128 B] swizzled block
 
-// TMEM columns (512 allocated)
-constexpr uint32_t COL_K0 = 0, COL_K1 = 64;      // K = X X^T (M=64 layout), double buffer
-constexpr uint32_t COL_Y1 = 128;                 // + 64 * buffer
-constexpr uint32_t COL_Y2 = 256;                 // + 64 * buffer
-constexpr uint32_t COL_DS = 384;                 // 128 columns
+// TMEM columns (512 allocated). The M=64 products occupy lanes 0-15 of each
+// 32-lane sub-partition (row i at lane 32 (i / 16) + i % 16).
+constexpr uint32_t COL_K0 = 0, COL_K1 = 64;      // K = X X^T, double buffer
+constexpr uint32_t COL_Y1 = 128;                 // Y1 (128 columns)
+constexpr uint32_t COL_Y2 = 256;                 // Y2 (128 columns)
+constexpr uint32_t COL_DS = 384;                 // dS (128 columns, all 128 lanes)
 
 // With M = L_{31}, the mask factor -eta_j 2^{L_{i-1} - L_j} = ra_i ca_j whenever
 // every exponent stays inside fp32 range: fac = (|L_{C-1}| <= 120).
@@ -73,18 +77,17 @@ struct Smem {
   // 1024-byte aligned tiles first
   uint8_t X[NS][2 * TILE];     // k-blocks [0,64), [64,128): 64 token rows x 128 B
   uint8_t G[NS][2 * TILE];     // n-blocks of the slice: 64 token rows x 128 B
-  uint8_t W0[2][128 * 128];    // k-blocks: 128 n rows x 128 B (bf16 W0 slice)
-  uint8_t S[2][2][128 * 128];  // [buffer][k-block]: 128 n rows x 128 B (bf16 state)
+  uint8_t W0[2][BIG];          // k-blocks: 128 n rows x 128 B (bf16 W0 slice)
+  uint8_t S[2][2][BIG];        // [buffer][k-block]: 128 n rows x 128 B (bf16 state)
+  uint8_t Xh[2][2 * TILE];     // [buffer] scaled X, same layout as X
   uint8_t P[TILE];             // 64 token rows (i) x 128 B (j)
-  uint8_t Xh[2 * TILE];        // scaled X, same layout as X
   GateSlot gates[GS];
   uint64_t full[NS], empty[NS];
   uint64_t gfull[GS], gempty[GS];
   uint64_t kfull[2], kfree[2];
-  uint64_t yfull[2], yfree[2];
-  uint64_t sready[2], sfree[2];  // per bf16 state buffer
-  uint64_t pready, xready, dsfull, dsfree, done;
-  uint32_t pad_;
+  uint64_t xhready[2], xhfree[2];  // per scaled-X buffer
+  uint64_t sready[2], sfree[2];    // per bf16 state buffer
+  uint64_t yfull, yfree, pready, dsfull, dsfree, done;
   uint32_t tmem_base;
   int abort;
 };
@@ -97,7 +100,7 @@ enum : uint32_t {
   W_MMA_FULL = 0x101, W_MMA_KFREE, W_MMA_YFREE, W_MMA_XREADY, W_MMA_DSFREE, W_MMA_PREADY,
   W_MMA_SREADY, W_MMA_DONE,
   W_GATE_EMPTY = 0x201,
-  W_XH_FULL = 0x301, W_XH_GFULL, W_XH_DSFULL,
+  W_XH_FULL = 0x301, W_XH_GFULL, W_XH_FREE,
   W_M_GFULL = 0x401, W_M_KFULL, W_M_DSFULL, W_M_SFREE, W_M_YFULL,
 };
 
@@ -131,17 +134,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.kfull[b], 1);
       mbar_init(&sm.kfree[b], 8);
-      mbar_init(&sm.yfull[b], 1);
-      mbar_init(&sm.yfree[b], 8);
-    }
-    mbar_init(&sm.pready, 8);
-    mbar_init(&sm.xready, 2);
-    mbar_init(&sm.dsfull, 1);
-    mbar_init(&sm.dsfree, 8);
-    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.xhready[b], 2);
+      mbar_init(&sm.xhfree[b], 1);
       mbar_init(&sm.sready[b], 8);
       mbar_init(&sm.sfree[b], 1);
     }
+    mbar_init(&sm.yfull, 1);
+    mbar_init(&sm.yfree, 8);
+    mbar_init(&sm.pready, 8);
+    mbar_init(&sm.dsfull, 1);
+    mbar_init(&sm.dsfree, 8);
     mbar_init(&sm.done, 1);
     fence_mbar_init();
   }
@@ -194,15 +196,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t id_k = idesc_bf16(64, 64, false, false);
-      const uint32_t id_y = idesc_bf16(128, 64, false, false);
-      const uint32_t id_gp = idesc_bf16(128, 64, true, false);
-      const uint32_t id_ds = idesc_bf16(128, 128, true, true);
-      const uint32_t sW0 = smem_u32(sm.W0[0]);
-      const uint32_t sP = smem_u32(sm.P), sXh = smem_u32(sm.Xh);
+      const uint32_t id_k = idesc_bf16(64, 64, false, false);    // X X^T
+      const uint32_t id_y = idesc_bf16(64, 128, false, false);   // X W0^T, X S^T
+      const uint32_t id_pg = idesc_bf16(64, 128, false, true);   // P G (G n-contiguous)
+      const uint32_t id_ds = idesc_bf16(128, 128, true, true);   // G^T Xhat
+      const uint32_t sW0 = smem_u32(sm.W0[0]), sP = smem_u32(sm.P);
       for (int c = 0; c < nch; ++c) {
         const int s = c % NS, b = c & 1;
         const uint32_t sX = smem_u32(sm.X[s]), sG = smem_u32(sm.G[s]);
+        const uint32_t sXh = smem_u32(sm.Xh[b]), sS = smem_u32(sm.S[b][0]);
         if (!mbar_wait(&sm.full[s], (c / NS) & 1, wc, W_MMA_FULL)) break;
         if (!mbar_wait(&sm.kfree[b], ((c >> 1) & 1) ^ 1, wc, W_MMA_KFREE)) break;
         tc_fence_after();
@@ -213,43 +215,42 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     sw128_desc(sX + off, 16, 1024), id_k, kk > 0);
         }
         if (!(p.inject == 1 && c == 1)) umma_commit(&sm.kfull[b]);
-        if (!mbar_wait(&sm.yfree[b], ((c >> 1) & 1) ^ 1, wc, W_MMA_YFREE)) break;
-        tc_fence_after();
-        // Y1^T = W0 X^T
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t aoff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          const uint32_t boff = (kk >> 2) * TILE + (kk & 3) * 32;
-          umma_bf16(tbase + COL_Y1 + 64 * b, sw128_desc(sW0 + aoff, 16, 1024),
-                    sw128_desc(sX + boff, 16, 1024), id_y, kk > 0);
-        }
         // dS = G^T Xhat
-        if (!mbar_wait(&sm.xready, c & 1, wc, W_MMA_XREADY)) break;
+        if (!mbar_wait(&sm.xhready[b], (c >> 1) & 1, wc, W_MMA_XREADY)) break;
         if (c > 0 && !mbar_wait(&sm.dsfree, (c - 1) & 1, wc, W_MMA_DSFREE)) break;
         tc_fence_after();
-        for (int kk = 0; kk < 4; ++kk) {
+        for (int kk = 0; kk < 4; ++kk)
           umma_bf16(tbase + COL_DS, sw128_desc(sG + kk * 2048, TILE, 1024),
                     sw128_desc(sXh + kk * 2048, TILE, 1024), id_ds, kk > 0);
-        }
         umma_commit(&sm.dsfull);
-        // Y1^T += G^T P^T
-        if (!mbar_wait(&sm.pready, c & 1, wc, W_MMA_PREADY)) break;
+        umma_commit(&sm.xhfree[b]);
+        // Y1 = X W0^T (the epilogue of chunk c - 1 has read Y1 and Y2)
+        if (c > 0 && !mbar_wait(&sm.yfree, (c - 1) & 1, wc, W_MMA_YFREE)) break;
         tc_fence_after();
-        for (int kk = 0; kk < 4; ++kk) {
-          umma_bf16(tbase + COL_Y1 + 64 * b, sw128_desc(sG + kk * 2048, TILE, 1024),
-                    sw128_desc(sP + kk * 32, 16, 1024), id_gp, 1);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t aoff = (kk >> 2) * TILE + (kk & 3) * 32;
+          const uint32_t boff = (kk >> 2) * BIG + (kk & 3) * 32;
+          umma_bf16(tbase + COL_Y1, sw128_desc(sX + aoff, 16, 1024),
+                    sw128_desc(sW0 + boff, 16, 1024), id_y, kk > 0);
         }
-        // Y2^T = S X^T (state buffer c & 1, written by the state update of chunk c - 1)
+        // Y2 = X S^T (state buffer c & 1, written by the state update of chunk c - 1)
         if (c > 0 && !mbar_wait(&sm.sready[b], ((c - 1) >> 1) & 1, wc, W_MMA_SREADY)) break;
         tc_fence_after();
-        const uint32_t sS = smem_u32(sm.S[b][0]);
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t aoff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          const uint32_t boff = (kk >> 2) * TILE + (kk & 3) * 32;
-          umma_bf16(tbase + COL_Y2 + 64 * b, sw128_desc(sS + aoff, 16, 1024),
-                    sw128_desc(sX + boff, 16, 1024), id_y, kk > 0);
+          const uint32_t aoff = (kk >> 2) * TILE + (kk & 3) * 32;
+          const uint32_t boff = (kk >> 2) * BIG + (kk & 3) * 32;
+          umma_bf16(tbase + COL_Y2, sw128_desc(sX + aoff, 16, 1024),
+                    sw128_desc(sS + boff, 16, 1024), id_y, kk > 0);
         }
-        umma_commit(&sm.yfull[b]);
         umma_commit(&sm.sfree[b]);
+        // Y1 += P G. The mask of chunk c + 1 overwrites P only after the K product
+        // of chunk c + 1 has completed, which is committed after these.
+        if (!mbar_wait(&sm.pready, c & 1, wc, W_MMA_PREADY)) break;
+        tc_fence_after();
+        for (int kk = 0; kk < 4; ++kk)
+          umma_bf16(tbase + COL_Y1, sw128_desc(sP + kk * 32, 16, 1024),
+                    sw128_desc(sG + kk * 2048, TILE, 1024), id_pg, 1);
+        umma_commit(&sm.yfull);
         umma_commit(&sm.empty[s]);
       }
       // teardown: every issued MMA completes before TMEM is released
@@ -329,8 +330,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         if (!mbar_wait_warp(&sm.full[s], (c / NS) & 1, wc, W_XH_FULL)) { ok = false; break; }
         if (!mbar_wait_warp(&sm.gfull[g], (c / GS) & 1, wc, W_XH_GFULL)) { ok = false; break; }
-        if (c > 0 && !mbar_wait_warp(&sm.dsfull, (c - 1) & 1, wc, W_XH_DSFULL)) { ok = false; break; }
-        const uint32_t src = smem_u32(sm.X[s]), dst = smem_u32(sm.Xh);
+        if (!mbar_wait_warp(&sm.xhfree[c & 1], ((c >> 1) & 1) ^ 1, wc, W_XH_FREE)) { ok = false; break; }
+        const uint32_t src = smem_u32(sm.X[s]), dst = smem_u32(sm.Xh[c & 1]);
 #pragma unroll 4
         for (int idx = (warp - 2) * 32 + lane; idx < 2 * TILE / 16; idx += 64) {
           const uint32_t off = idx * 16;
@@ -347,7 +348,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&sm.xready);
+          mbar_arrive(&sm.xhready[c & 1]);
           mbar_arrive(&sm.gempty[g]);
         }
       }
@@ -355,13 +356,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else {
     // ------------------------------------------------------------ math warpgroups
     const int q = warp & 3;          // TMEM lane quadrant
-    const int hh = (warp - 4) >> 2;  // warpgroup: state columns [64hh, 64hh+64), tokens [32hh, +32)
+    const int hh = (warp - 4) >> 2;  // warpgroup: state and output columns [64hh, 64hh+64)
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
     const int n = 32 * q + lane;     // row of the d_out slice owned by this thread
     float Sreg[64];
 #pragma unroll
     for (int e = 0; e < 64; ++e) Sreg[e] = 0.f;
-    __nv_bfloat16* yout = p.y ? p.y + (size_t)bh * T * p.dout + n0 + n : nullptr;
+    __nv_bfloat16* yout = p.y ? p.y + (size_t)bh * T * p.dout + n0 + 64 * hh : nullptr;
     // chunk-start state checkpoints (bf16 [bh][chunk][dout][din]); S_0 = 0
     uint4* ck_row = p.ckpt ? reinterpret_cast<uint4*>(p.ckpt + ((size_t)bh * nch * p.dout + n0 + n) * 128 + 64 * hh)
                            : nullptr;
@@ -433,29 +434,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (c > 0 && !mbar_wait_warp(&sm.sfree[wb], ((c - 1) >> 1) & 1, wc, W_M_SFREE)) break;
       tc_fence_after();
       {
-        float v0[32], v1[32];
-        tmem_ld32(tbase + COL_DS + lane_off + 64 * hh, v0);
-        tmem_ld32(tbase + COL_DS + lane_off + 64 * hh + 32, v1);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.dsfree);
         const float gC = gs.gC;
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          Sreg[e] = fmaf(gC, Sreg[e], v0[e]);
-          Sreg[32 + e] = fmaf(gC, Sreg[32 + e], v1[e]);
-        }
         const uint32_t srow = smem_u32(sm.S[wb][hh]);
         uint4* ck = (ck_row && c + 1 < nch) ? ck_row + (size_t)(c + 1) * ck_stride : nullptr;
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          const uint4 pk = make_uint4(pack_bf16(Sreg[8 * cc], Sreg[8 * cc + 1]),
-                                      pack_bf16(Sreg[8 * cc + 2], Sreg[8 * cc + 3]),
-                                      pack_bf16(Sreg[8 * cc + 4], Sreg[8 * cc + 5]),
-                                      pack_bf16(Sreg[8 * cc + 6], Sreg[8 * cc + 7]));
-          st_shared_v4(srow + sw128_off(n, cc), pk.x, pk.y, pk.z, pk.w);
-          if (ck) ck[cc] = pk;
+        for (int hf = 0; hf < 2; ++hf) {
+          float v[32];
+          tmem_ld32(tbase + COL_DS + lane_off + 64 * hh + 32 * hf, v);
+          tmem_ld_wait();
+          if (hf == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.dsfree);
+          }
+#pragma unroll
+          for (int e = 0; e < 32; ++e) Sreg[32 * hf + e] = fmaf(gC, Sreg[32 * hf + e], v[e]);
+#pragma unroll
+          for (int cc = 4 * hf; cc < 4 * hf + 4; ++cc) {
+            const uint4 pk = make_uint4(pack_bf16(Sreg[8 * cc], Sreg[8 * cc + 1]),
+                                        pack_bf16(Sreg[8 * cc + 2], Sreg[8 * cc + 3]),
+                                        pack_bf16(Sreg[8 * cc + 4], Sreg[8 * cc + 5]),
+                                        pack_bf16(Sreg[8 * cc + 6], Sreg[8 * cc + 7]));
+            st_shared_v4(srow + sw128_off(n, cc), pk.x, pk.y, pk.z, pk.w);
+            if (ck) ck[cc] = pk;
+          }
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -465,30 +467,35 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // ---- mask of the next chunk (keeps the MMA stream fed while we store y)
       if (c + 1 < nch && !mask(c + 1)) break;
 
-      // ---- output: y_i = Y1^T[n][i] + 2^{L_{i-1}} Y2^T[n][i]
-      if (!mbar_wait_warp(&sm.yfull[b], (c >> 1) & 1, wc, W_M_YFULL)) break;
+      // ---- output: y_i = Y1[i] + 2^{L_{i-1}} Y2[i]; lanes 0-15 hold token rows
+      //      i = 16 q + lane of the M=64 products, 32 columns per load
+      if (!mbar_wait_warp(&sm.yfull, c & 1, wc, W_M_YFULL)) break;
       tc_fence_after();
       {
-        float a[32], s2[32];
-        tmem_ld32(tbase + COL_Y1 + 64 * b + lane_off + 32 * hh, a);
-        tmem_ld32(tbase + COL_Y2 + 64 * b + lane_off + 32 * hh, s2);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.yfree[b]);
-        const int ib = 32 * hh;
-        const int tb = c * C + ib;
-        if (!yout) {
-        } else if (tb + 32 <= T) {
+        const int i = 16 * q + (lane & 15);
+        const int tok = c * C + i;
+        const float gi = gs.gam[i];
+        const bool store = yout != nullptr && lane < 16 && tok < T;
+        uint4* dst = store ? reinterpret_cast<uint4*>(yout + (size_t)tok * p.dout) : nullptr;
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            yout[(size_t)(tb + e) * p.dout] = __float2bfloat16_rn(fmaf(gs.gam[ib + e], s2[e], a[e]));
-        } else {
+        for (int k = 0; k < 4; ++k) {
+          float a[16], s2[16];
+          tmem_ld16(tbase + COL_Y1 + lane_off + 64 * hh + 16 * k, a);
+          tmem_ld16(tbase + COL_Y2 + lane_off + 64 * hh + 16 * k, s2);
+          tmem_ld_wait();
+          if (k == 3) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.yfree);
+          }
+          uint32_t w[8];
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (tb + e < T)
-              yout[(size_t)(tb + e) * p.dout] =
-                  __float2bfloat16_rn(fmaf(gs.gam[ib + e], s2[e], a[e]));
+          for (int e = 0; e < 8; ++e)
+            w[e] = pack_bf16(fmaf(gi, s2[2 * e], a[2 * e]), fmaf(gi, s2[2 * e + 1], a[2 * e + 1]));
+          if (store) {
+            dst[2 * k] = make_uint4(w[0], w[1], w[2], w[3]);
+            dst[2 * k + 1] = make_uint4(w[4], w[5], w[6], w[7]);
+          }
         }
       }
       __syncwarp();
