@@ -81,6 +81,7 @@ struct Smem {
   uint8_t S[2][2][BIG];        // [buffer][k-block]: 128 n rows x 128 B (bf16 state)
   uint8_t Xh[2][2 * TILE];     // [buffer] scaled X, same layout as X
   uint8_t P[TILE];             // 64 token rows (i) x 128 B (j)
+  uint8_t Ys[2 * TILE];        // y staging: n-blocks of 64 token rows x 128 B (TMA store)
   GateSlot gates[GS];
   uint64_t full[NS], empty[NS];
   uint64_t gfull[GS], gempty[GS];
@@ -104,10 +105,21 @@ enum : uint32_t {
   W_M_GFULL = 0x401, W_M_KFULL, W_M_DSFULL, W_M_SFREE, W_M_YFULL,
 };
 
+// Barrier 1: the eight math warps only.
+__device__ __forceinline__ void named_sync_math() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+// Waits until at most n (0..2) of this thread's TMA store groups still read shared memory.
+__device__ __forceinline__ void store_reads_pending_at_most(int n) {
+  if (n <= 0) tma_store_wait_read_n<0>();
+  else if (n == 1) tma_store_wait_read_n<1>();
+  else tma_store_wait_read_n<2>();
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(NTHREADS, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmG,
+               const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmS,
                TcFwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>(
@@ -150,6 +162,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmX);
     prefetch_tmap(&tmG);
+    if (p.y) prefetch_tmap(&tmY);
+    if (p.ckpt) prefetch_tmap(&tmS);
   }
   if (warp == 1) {
     tmem_alloc(&sm.tmem_base, 512);
@@ -362,14 +376,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     float Sreg[64];
 #pragma unroll
     for (int e = 0; e < 64; ++e) Sreg[e] = 0.f;
-    __nv_bfloat16* yout = p.y ? p.y + (size_t)bh * T * p.dout + n0 + 64 * hh : nullptr;
-    // chunk-start state checkpoints (bf16 [bh][chunk][dout][din]); S_0 = 0
-    uint4* ck_row = p.ckpt ? reinterpret_cast<uint4*>(p.ckpt + ((size_t)bh * nch * p.dout + n0 + n) * 128 + 64 * hh)
-                           : nullptr;
-    const size_t ck_stride = (size_t)p.dout * 128 / 8;  // uint4 per chunk
-    if (ck_row) {
-#pragma unroll
-      for (int cc = 0; cc < 8; ++cc) ck_row[cc] = make_uint4(0u, 0u, 0u, 0u);
+    const int mt = threadIdx.x - 128;  // 0..255; thread 0 issues the TMA stores
+    const bool has_y = p.y != nullptr, has_ck = p.ckpt != nullptr;
+    // chunk-start state checkpoints (bf16 [bh][chunk][dout][din], tensor map tmS) are
+    // TMA-stored straight from the swizzled bf16 state tiles; S_0 = 0 is buffer 0
+    if (has_ck && mt == 0) {
+      tma_store_3d(&tmS, sm.S[0][0], 0, n0, bh * nch);
+      tma_store_3d(&tmS, sm.S[0][1], 64, n0, bh * nch);
+      tma_store_commit();
     }
 
     // mask of chunk c: P_ij = K_ij (-eta_j) 2^{L_{i-1} - L_j} for j < i
@@ -421,22 +435,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       return true;
     };
 
+    // Every math warp executes the same sequence of named barriers in every
+    // iteration, whatever happens to its waits: after a failed (timed-out or
+    // aborted) wait the warp skips the work but keeps the barrier schedule.
+    // Thread mt = 0 commits one TMA store group per checkpoint and per y tile, in
+    // the order CK_{c+1} (state update of chunk c), Y_c (epilogue of chunk c).
     bool ok = nch > 0 ? mask(0) : true;
-    for (int c = 0; c < nch && ok; ++c) {
-      const int g = c % GS, b = c & 1;
+    for (int c = 0; c < nch; ++c) {
+      const int g = c % GS;
       const GateSlot& gs = sm.gates[g];
 
       // ---- state: S <- 2^{L_{C-1}} S + dS ; bf16 copy into buffer wb = (c+1)&1, which
       //      the S X^T product of chunk c - 1 read (one barrier pair per buffer, so a
       //      parity wait can never see a phase from the other buffer's traffic)
       const int wb = (c + 1) & 1;
-      if (!mbar_wait_warp(&sm.dsfull, c & 1, wc, W_M_DSFULL)) break;
-      if (c > 0 && !mbar_wait_warp(&sm.sfree[wb], ((c - 1) >> 1) & 1, wc, W_M_SFREE)) break;
-      tc_fence_after();
-      {
+      ok = ok && mbar_wait_warp(&sm.dsfull, c & 1, wc, W_M_DSFULL);
+      ok = ok && (c == 0 || mbar_wait_warp(&sm.sfree[wb], ((c - 1) >> 1) & 1, wc, W_M_SFREE));
+      // the checkpoint store CK_c-1 that last read buffer wb is done reading: at most
+      // Y_{c-2}, CK_c, Y_{c-1} (or CK_1, Y_0 after CK_0) are newer than it
+      if (mt == 0 && has_ck) store_reads_pending_at_most(has_y ? 2 : 1);
+      named_sync_math();  // (F1)
+      if (ok) {
+        tc_fence_after();
         const float gC = gs.gC;
         const uint32_t srow = smem_u32(sm.S[wb][hh]);
-        uint4* ck = (ck_row && c + 1 < nch) ? ck_row + (size_t)(c + 1) * ck_stride : nullptr;
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
           float v[32];
@@ -450,33 +472,37 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) Sreg[32 * hf + e] = fmaf(gC, Sreg[32 * hf + e], v[e]);
 #pragma unroll
-          for (int cc = 4 * hf; cc < 4 * hf + 4; ++cc) {
-            const uint4 pk = make_uint4(pack_bf16(Sreg[8 * cc], Sreg[8 * cc + 1]),
-                                        pack_bf16(Sreg[8 * cc + 2], Sreg[8 * cc + 3]),
-                                        pack_bf16(Sreg[8 * cc + 4], Sreg[8 * cc + 5]),
-                                        pack_bf16(Sreg[8 * cc + 6], Sreg[8 * cc + 7]));
-            st_shared_v4(srow + sw128_off(n, cc), pk.x, pk.y, pk.z, pk.w);
-            if (ck) ck[cc] = pk;
-          }
+          for (int cc = 4 * hf; cc < 4 * hf + 4; ++cc)
+            st_shared_v4(srow + sw128_off(n, cc), pack_bf16(Sreg[8 * cc], Sreg[8 * cc + 1]),
+                         pack_bf16(Sreg[8 * cc + 2], Sreg[8 * cc + 3]),
+                         pack_bf16(Sreg[8 * cc + 4], Sreg[8 * cc + 5]),
+                         pack_bf16(Sreg[8 * cc + 6], Sreg[8 * cc + 7]));
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.sready[wb]);
       }
+      named_sync_math();  // (F2) the bf16 state S_{c+1} is complete in buffer wb
+      if (ok && mt == 0 && has_ck && c + 1 < nch) {
+        tma_store_3d(&tmS, sm.S[wb][0], 0, n0, bh * nch + c + 1);
+        tma_store_3d(&tmS, sm.S[wb][1], 64, n0, bh * nch + c + 1);
+        tma_store_commit();
+      }
 
       // ---- mask of the next chunk (keeps the MMA stream fed while we store y)
-      if (c + 1 < nch && !mask(c + 1)) break;
+      if (c + 1 < nch) ok = ok && mask(c + 1);
 
       // ---- output: y_i = Y1[i] + 2^{L_{i-1}} Y2[i]; lanes 0-15 hold token rows
-      //      i = 16 q + lane of the M=64 products, 32 columns per load
-      if (!mbar_wait_warp(&sm.yfull, c & 1, wc, W_M_YFULL)) break;
-      tc_fence_after();
-      {
+      //      i = 16 q + lane of the M=64 products; staged bf16 and TMA-stored
+      ok = ok && mbar_wait_warp(&sm.yfull, c & 1, wc, W_M_YFULL);
+      // the staging tile's previous store Y_{c-1} is done reading (only CK_{c+1} is newer)
+      if (mt == 0 && has_y) store_reads_pending_at_most((has_ck && c + 1 < nch) ? 1 : 0);
+      named_sync_math();  // (F3)
+      if (ok) {
+        tc_fence_after();
         const int i = 16 * q + (lane & 15);
-        const int tok = c * C + i;
         const float gi = gs.gam[i];
-        const bool store = yout != nullptr && lane < 16 && tok < T;
-        uint4* dst = store ? reinterpret_cast<uint4*>(yout + (size_t)tok * p.dout) : nullptr;
+        const uint32_t yrow = smem_u32(sm.Ys + hh * TILE);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           float a[16], s2[16];
@@ -492,15 +518,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             w[e] = pack_bf16(fmaf(gi, s2[2 * e], a[2 * e]), fmaf(gi, s2[2 * e + 1], a[2 * e + 1]));
-          if (store) {
-            dst[2 * k] = make_uint4(w[0], w[1], w[2], w[3]);
-            dst[2 * k + 1] = make_uint4(w[4], w[5], w[6], w[7]);
+          if (lane < 16 && has_y) {
+            st_shared_v4(yrow + sw128_off(i, 2 * k), w[0], w[1], w[2], w[3]);
+            st_shared_v4(yrow + sw128_off(i, 2 * k + 1), w[4], w[5], w[6], w[7]);
           }
         }
+        fence_proxy_async_smem();
+      }
+      named_sync_math();  // (F4) the y tile of chunk c is staged; rows past T are clipped
+      if (ok && mt == 0 && has_y) {
+        tma_store_3d(&tmY, sm.Ys, n0, c * C, bh);
+        tma_store_3d(&tmY, sm.Ys + TILE, n0 + 64, c * C, bh);
+        tma_store_commit();
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.gempty[g]);
+      if (ok && lane == 0) mbar_arrive(&sm.gempty[g]);
     }
+    if (mt == 0) tma_store_wait_all();
   }
 
   tc_fence_before();
@@ -549,9 +583,16 @@ size_t ckpt_bytes(int B, int H, int T, int din, int dout) {
 }
 
 cudaError_t launch_fwd(const TcFwdParams& prm, const void* x, const void* g, cudaStream_t st) {
-  CUtensorMap mx, mg;
-  if (!make_map_bf16_3d(&mx, x, prm.din, prm.T, (uint64_t)prm.B * prm.H, C) ||
-      !make_map_bf16_3d(&mg, g, prm.dout, prm.T, (uint64_t)prm.B * prm.H, C))
+  CUtensorMap mx, mg, my, ms;
+  const uint64_t BH = (uint64_t)prm.B * prm.H;
+  const uint64_t nch = (uint64_t)(prm.T + C - 1) / C;
+  // The y and checkpoint maps are only used when those outputs are requested; g
+  // stands in as a well-formed base otherwise.
+  if (!make_map_bf16_3d(&mx, x, prm.din, prm.T, BH, C) ||
+      !make_map_bf16_3d(&mg, g, prm.dout, prm.T, BH, C) ||
+      !make_map_bf16_3d(&my, prm.y ? (const void*)prm.y : g, prm.dout, prm.T, BH, C) ||
+      !make_map_bf16_3d(&ms, prm.ckpt ? (const void*)prm.ckpt : g, 128, prm.dout,
+                        prm.ckpt ? BH * nch : 1, 128))
     return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!attr_set) {
@@ -561,7 +602,7 @@ cudaError_t launch_fwd(const TcFwdParams& prm, const void* x, const void* g, cud
     attr_set = true;
   }
   const int grid = prm.B * prm.H * (prm.dout / 128);
-  fwd_kernel<<<grid, NTHREADS, kSmemBytes, st>>>(mx, mg, prm);
+  fwd_kernel<<<grid, NTHREADS, kSmemBytes, st>>>(mx, mg, my, ms, prm);
   count_launch();
   return cudaGetLastError();
 }
