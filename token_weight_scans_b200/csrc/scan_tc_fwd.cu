@@ -105,9 +105,6 @@ enum : uint32_t {
   W_M_GFULL = 0x401, W_M_KFULL, W_M_DSFULL, W_M_SFREE, W_M_YFULL,
 };
 
-// Barrier 1: the eight math warps only.
-__device__ __forceinline__ void named_sync_math() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-
 // Waits until at most n (0..2) of this thread's TMA store groups still read shared memory.
 __device__ __forceinline__ void store_reads_pending_at_most(int n) {
   if (n <= 0) tma_store_wait_read_n<0>();
@@ -376,13 +373,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     float Sreg[64];
 #pragma unroll
     for (int e = 0; e < 64; ++e) Sreg[e] = 0.f;
-    const int mt = threadIdx.x - 128;  // 0..255; thread 0 issues the TMA stores
     const bool has_y = p.y != nullptr, has_ck = p.ckpt != nullptr;
-    // chunk-start state checkpoints (bf16 [bh][chunk][dout][din], tensor map tmS) are
-    // TMA-stored straight from the swizzled bf16 state tiles; S_0 = 0 is buffer 0
-    if (has_ck && mt == 0) {
-      tma_store_3d(&tmS, sm.S[0][0], 0, n0, bh * nch);
-      tma_store_3d(&tmS, sm.S[0][1], 64, n0, bh * nch);
+    // Each warp TMA-stores what it wrote itself: its 32 rows of one k-block of the
+    // bf16 state (the chunk-start checkpoints, bf16 [bh][chunk][dout][din], box of
+    // 32 rows) and its 16 token rows of one n-block of y (box of 16 rows). S_0 = 0
+    // is buffer 0.
+    const uint32_t s_part = (uint32_t)(32 * q) * 128;  // byte offset of the warp's state rows
+    const uint32_t y_part = (uint32_t)(16 * q) * 128;  // byte offset of the warp's token rows
+    if (has_ck && lane == 0) {
+      tma_store_3d(&tmS, sm.S[0][hh] + s_part, 64 * hh, n0 + 32 * q, bh * nch);
       tma_store_commit();
     }
 
@@ -435,11 +434,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       return true;
     };
 
-    // Every math warp executes the same sequence of named barriers in every
-    // iteration, whatever happens to its waits: after a failed (timed-out or
-    // aborted) wait the warp skips the work but keeps the barrier schedule.
-    // Thread mt = 0 commits one TMA store group per checkpoint and per y tile, in
-    // the order CK_{c+1} (state update of chunk c), Y_c (epilogue of chunk c).
+    // Lane 0 of each math warp commits one TMA store group per checkpoint part and
+    // per y part, in the order CK_{c+1} (state update of chunk c), Y_c (epilogue of
+    // chunk c); before its rows of a buffer are rewritten it waits until the
+    // group that last read them is done reading.
     bool ok = nch > 0 ? mask(0) : true;
     for (int c = 0; c < nch; ++c) {
       const int g = c % GS;
@@ -451,10 +449,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int wb = (c + 1) & 1;
       ok = ok && mbar_wait_warp(&sm.dsfull, c & 1, wc, W_M_DSFULL);
       ok = ok && (c == 0 || mbar_wait_warp(&sm.sfree[wb], ((c - 1) >> 1) & 1, wc, W_M_SFREE));
-      // the checkpoint store CK_c-1 that last read buffer wb is done reading: at most
-      // Y_{c-2}, CK_c, Y_{c-1} (or CK_1, Y_0 after CK_0) are newer than it
-      if (mt == 0 && has_ck) store_reads_pending_at_most(has_y ? 2 : 1);
-      named_sync_math();  // (F1)
+      // CK_{c-1} last read these rows of buffer wb; at most Y_{c-2}, CK_c, Y_{c-1}
+      // (or CK_1, Y_0 after CK_0) are newer
+      if (lane == 0 && has_ck) store_reads_pending_at_most(has_y ? 2 : 1);
+      __syncwarp();
       if (ok) {
         tc_fence_after();
         const float gC = gs.gC;
@@ -480,13 +478,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.sready[wb]);
-      }
-      named_sync_math();  // (F2) the bf16 state S_{c+1} is complete in buffer wb
-      if (ok && mt == 0 && has_ck && c + 1 < nch) {
-        tma_store_3d(&tmS, sm.S[wb][0], 0, n0, bh * nch + c + 1);
-        tma_store_3d(&tmS, sm.S[wb][1], 64, n0, bh * nch + c + 1);
-        tma_store_commit();
+        if (lane == 0) {
+          mbar_arrive(&sm.sready[wb]);
+          if (has_ck && c + 1 < nch) {
+            tma_store_3d(&tmS, sm.S[wb][hh] + s_part, 64 * hh, n0 + 32 * q, bh * nch + c + 1);
+            tma_store_commit();
+          }
+        }
       }
 
       // ---- mask of the next chunk (keeps the MMA stream fed while we store y)
@@ -495,9 +493,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // ---- output: y_i = Y1[i] + 2^{L_{i-1}} Y2[i]; lanes 0-15 hold token rows
       //      i = 16 q + lane of the M=64 products; staged bf16 and TMA-stored
       ok = ok && mbar_wait_warp(&sm.yfull, c & 1, wc, W_M_YFULL);
-      // the staging tile's previous store Y_{c-1} is done reading (only CK_{c+1} is newer)
-      if (mt == 0 && has_y) store_reads_pending_at_most((has_ck && c + 1 < nch) ? 1 : 0);
-      named_sync_math();  // (F3)
+      // Y_{c-1} last read these staging rows; only CK_{c+1} is newer
+      if (lane == 0 && has_y) store_reads_pending_at_most((has_ck && c + 1 < nch) ? 1 : 0);
+      __syncwarp();
       if (ok) {
         tc_fence_after();
         const int i = 16 * q + (lane & 15);
@@ -524,17 +522,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
         }
         fence_proxy_async_smem();
+        __syncwarp();
+        // rows past T are clipped; a part that starts past T is not issued
+        if (lane == 0 && has_y && c * C + 16 * q < T) {
+          tma_store_3d(&tmY, sm.Ys + hh * TILE + y_part, n0 + 64 * hh, c * C + 16 * q, bh);
+          tma_store_commit();
+        }
+        if (lane == 0) mbar_arrive(&sm.gempty[g]);
       }
-      named_sync_math();  // (F4) the y tile of chunk c is staged; rows past T are clipped
-      if (ok && mt == 0 && has_y) {
-        tma_store_3d(&tmY, sm.Ys, n0, c * C, bh);
-        tma_store_3d(&tmY, sm.Ys + TILE, n0 + 64, c * C, bh);
-        tma_store_commit();
-      }
-      __syncwarp();
-      if (ok && lane == 0) mbar_arrive(&sm.gempty[g]);
     }
-    if (mt == 0) tma_store_wait_all();
+    if (lane == 0) tma_store_wait_all();
   }
 
   tc_fence_before();
@@ -590,9 +587,9 @@ cudaError_t launch_fwd(const TcFwdParams& prm, const void* x, const void* g, cud
   // stands in as a well-formed base otherwise.
   if (!make_map_bf16_3d(&mx, x, prm.din, prm.T, BH, C) ||
       !make_map_bf16_3d(&mg, g, prm.dout, prm.T, BH, C) ||
-      !make_map_bf16_3d(&my, prm.y ? (const void*)prm.y : g, prm.dout, prm.T, BH, C) ||
+      !make_map_bf16_3d(&my, prm.y ? (const void*)prm.y : g, prm.dout, prm.T, BH, 16) ||
       !make_map_bf16_3d(&ms, prm.ckpt ? (const void*)prm.ckpt : g, 128, prm.dout,
-                        prm.ckpt ? BH * nch : 1, 128))
+                        prm.ckpt ? BH * nch : 1, 32))
     return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!attr_set) {
