@@ -242,6 +242,7 @@ def main():
 
     import token_weight_scans_b200 as tw
     from token_weight_scans_b200 import build as tw_build
+    from token_weight_scans_b200 import multirank
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -270,7 +271,7 @@ def main():
 
     # inputs: each rank its own seeded batch (weak scaling)
     d = inputs.draw(B, H, T, di, do, dtype=cfg.dtype, alpha_mode=cfg.alpha_mode,
-                    seed=inputs.SEED_BASE + cfg.index + 1000 * rank)
+                    seed=multirank.rank_seed(cfg.index, rank))
     host = {}
     for k, v in d.items():
         t = torch.from_numpy(v)
@@ -300,8 +301,7 @@ def main():
             tw.gradlev_scan_bwd(src["x"], src["g"], src["eta"], src["alpha"], src["W0"],
                                 src["dy"], ckpt=ck, workspace=ws, out=gr)
             launches[0] += tw.gradlev_last_launch_count()
-            if world > 1:
-                dist.all_reduce(gr["dW0"])
+            multirank.allreduce_dW0(gr["dW0"], dist)
 
     for _ in range(args.warmup):
         step()
@@ -330,8 +330,8 @@ def main():
                                 ckpt=ck, workspace=ws, out=gr)
             launches[0] += tw.gradlev_last_launch_count()
         ev[i][2].record(stream)
-        if do_bwd and world > 1:
-            dist.all_reduce(gr["dW0"])
+        if do_bwd:
+            multirank.allreduce_dW0(gr["dW0"], dist)
     end.record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -340,10 +340,7 @@ def main():
     ms = start.elapsed_time(end)
     fwd_ms = float(np.mean([a.elapsed_time(b) for a, b, _ in ev]))
     bwd_ms = float(np.mean([b.elapsed_time(c) for _, b, c in ev])) if do_bwd else 0.0
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = multirank.max_over_ranks(ms, dist, device=dev)
     gpu_launches = launches[0]
 
     # e2e through the public API with host buffers: H2D inputs, scan, D2H outputs
@@ -379,11 +376,8 @@ def main():
         e2.record(stream)
         torch.cuda.synchronize()
         ems = s2.elapsed_time(e2) / e_steps
-        if world > 1:
-            t = torch.tensor([ems], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": cfg.tokens * world / (ems * 1e-3), "unit": "tokens/s",
+        ems = multirank.max_over_ranks(ems, dist, device=dev)
+        e2e = {"value": multirank.weak_scaling_value(cfg.tokens, world, 1, ems), "unit": "tokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": ems, "steps": e_steps}
 
@@ -402,7 +396,7 @@ def main():
         ms_step = ms / args.steps
         line = {
             "metric": METRIC,
-            "value": cfg.tokens * world * args.steps / (ms * 1e-3),
+            "value": multirank.weak_scaling_value(cfg.tokens, world, args.steps, ms),
             "unit": "tokens/s",
             "n_gpus": world,
             "steps": args.steps,
@@ -414,7 +408,7 @@ def main():
             "dtype": cfg.dtype,
             "data": "synthetic (seeded generator; no dataset or trained weights)",
             "config": {"workload": cfg.name, "B": B, "H": H, "T": T, "d_in": di, "d_out": do,
-                       "passes": "+".join(cfg.passes), "global_batch": B * world,
+                       "passes": "+".join(cfg.passes), "global_batch": multirank.global_batch(B, world),
                        "parallelism": f"independent batch per GPU x{world}" +
                                       (" + dW0 all-reduce" if world > 1 and do_bwd else ""),
                        "l2": "no flush: working set "
