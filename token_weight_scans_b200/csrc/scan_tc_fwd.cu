@@ -52,12 +52,15 @@ constexpr int NTHREADS = 384;  // 12 warps
 constexpr int TILE = C * 128;  // bytes of one [64 rows x 128 B] swizzled block
 constexpr int BIG = 128 * 128; // bytes of one [128 rows x 128 B] swizzled block
 
-// TMEM columns (512 allocated). The M=64 products occupy lanes 0-15 of each
-// 32-lane sub-partition (row i at lane 32 (i / 16) + i % 16).
-constexpr uint32_t COL_K0 = 0, COL_K1 = 64;      // K = X X^T, double buffer
-constexpr uint32_t COL_Y1 = 128;                 // Y1 (128 columns)
-constexpr uint32_t COL_Y2 = 256;                 // Y2 (128 columns)
+// TMEM columns (512 allocated). An M=64 product occupies 16 lanes of each
+// 32-lane sub-partition (row i at lane 32 (i / 16) + i % 16, plus 16 when its
+// address carries LANE16). Y1 and Y2 of one chunk share 128 columns, Y1 in the
+// lower and Y2 in the upper 16 lanes, so that one load gives a thread pair
+// (l, l + 16) both halves of the same token row; the pair is double-buffered.
+constexpr uint32_t COL_K0 = 0, COL_K1 = 64;      // K = X X^T, double buffer (lanes 0-15)
+constexpr uint32_t COL_Y = 128;                  // + 128 * buffer: Y1 | Y2 (128 columns)
 constexpr uint32_t COL_DS = 384;                 // dS (128 columns, all 128 lanes)
+constexpr uint32_t LANE16 = 16u << 16;
 
 // With M = L_{31}, the mask factor -eta_j 2^{L_{i-1} - L_j} = ra_i ca_j whenever
 // every exponent stays inside fp32 range: fac = (|L_{C-1}| <= 120).
@@ -88,7 +91,8 @@ struct Smem {
   uint64_t kfull[2], kfree[2];
   uint64_t xhready[2], xhfree[2];  // per scaled-X buffer
   uint64_t sready[2], sfree[2];    // per bf16 state buffer
-  uint64_t yfull, yfree, pready, dsfull, dsfree, done;
+  uint64_t yfull[2], yfree[2];    // per Y1 | Y2 buffer
+  uint64_t pready, dsfull, dsfree, done;
   uint32_t tmem_base;
   int abort;
 };
@@ -148,8 +152,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&sm.sready[b], 8);
       mbar_init(&sm.sfree[b], 1);
     }
-    mbar_init(&sm.yfull, 1);
-    mbar_init(&sm.yfree, 8);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.yfull[b], 1);
+      mbar_init(&sm.yfree[b], 8);
+    }
     mbar_init(&sm.pready, 8);
     mbar_init(&sm.dsfull, 1);
     mbar_init(&sm.dsfree, 8);
@@ -235,14 +241,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     sw128_desc(sXh + kk * 2048, TILE, 1024), id_ds, kk > 0);
         umma_commit(&sm.dsfull);
         umma_commit(&sm.xhfree[b]);
-        // Y1 = X W0^T (the epilogue of chunk c - 1 has read Y1 and Y2)
-        if (c > 0 && !mbar_wait(&sm.yfree, (c - 1) & 1, wc, W_MMA_YFREE)) break;
+        // Y1 = X W0^T into buffer b (the epilogue of chunk c - 2 has read it)
+        const uint32_t tY1 = tbase + COL_Y + 128 * b, tY2 = tY1 + LANE16;
+        if (!mbar_wait(&sm.yfree[b], ((c >> 1) & 1) ^ 1, wc, W_MMA_YFREE)) break;
         tc_fence_after();
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t aoff = (kk >> 2) * TILE + (kk & 3) * 32;
           const uint32_t boff = (kk >> 2) * BIG + (kk & 3) * 32;
-          umma_bf16(tbase + COL_Y1, sw128_desc(sX + aoff, 16, 1024),
-                    sw128_desc(sW0 + boff, 16, 1024), id_y, kk > 0);
+          umma_bf16(tY1, sw128_desc(sX + aoff, 16, 1024), sw128_desc(sW0 + boff, 16, 1024), id_y,
+                    kk > 0);
         }
         // Y2 = X S^T (state buffer c & 1, written by the state update of chunk c - 1)
         if (c > 0 && !mbar_wait(&sm.sready[b], ((c - 1) >> 1) & 1, wc, W_MMA_SREADY)) break;
@@ -250,8 +257,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t aoff = (kk >> 2) * TILE + (kk & 3) * 32;
           const uint32_t boff = (kk >> 2) * BIG + (kk & 3) * 32;
-          umma_bf16(tbase + COL_Y2, sw128_desc(sX + aoff, 16, 1024),
-                    sw128_desc(sS + boff, 16, 1024), id_y, kk > 0);
+          umma_bf16(tY2, sw128_desc(sX + aoff, 16, 1024), sw128_desc(sS + boff, 16, 1024), id_y,
+                    kk > 0);
         }
         umma_commit(&sm.sfree[b]);
         // Y1 += P G. The mask of chunk c + 1 overwrites P only after the K product
@@ -259,9 +266,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (!mbar_wait(&sm.pready, c & 1, wc, W_MMA_PREADY)) break;
         tc_fence_after();
         for (int kk = 0; kk < 4; ++kk)
-          umma_bf16(tbase + COL_Y1, sw128_desc(sP + kk * 32, 16, 1024),
+          umma_bf16(tY1, sw128_desc(sP + kk * 32, 16, 1024),
                     sw128_desc(sG + kk * 2048, TILE, 1024), id_pg, 1);
-        umma_commit(&sm.yfull);
+        umma_commit(&sm.yfull[b]);
         umma_commit(&sm.empty[s]);
       }
       // teardown: every issued MMA completes before TMEM is released
@@ -490,36 +497,41 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // ---- mask of the next chunk (keeps the MMA stream fed while we store y)
       if (c + 1 < nch) ok = ok && mask(c + 1);
 
-      // ---- output: y_i = Y1[i] + 2^{L_{i-1}} Y2[i]; lanes 0-15 hold token rows
-      //      i = 16 q + lane of the M=64 products; staged bf16 and TMA-stored
-      ok = ok && mbar_wait_warp(&sm.yfull, c & 1, wc, W_M_YFULL);
+      // ---- output: y_i = Y1[i] + 2^{L_{i-1}} Y2[i]. Lane l < 16 holds Y1 and lane l + 16
+      //      holds Y2 of token row i = 16 q + l; for each 16 columns the pair swaps
+      //      halves, so lane l forms columns 0-7 and lane l + 16 columns 8-15.
+      const int yb = c & 1;
+      ok = ok && mbar_wait_warp(&sm.yfull[yb], (c >> 1) & 1, wc, W_M_YFULL);
       // Y_{c-1} last read these staging rows; only CK_{c+1} is newer
       if (lane == 0 && has_y) store_reads_pending_at_most((has_ck && c + 1 < nch) ? 1 : 0);
       __syncwarp();
       if (ok) {
         tc_fence_after();
         const int i = 16 * q + (lane & 15);
+        const int hi = lane >> 4;
         const float gi = gs.gam[i];
         const uint32_t yrow = smem_u32(sm.Ys + hh * TILE);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          float a[16], s2[16];
-          tmem_ld16(tbase + COL_Y1 + lane_off + 64 * hh + 16 * k, a);
-          tmem_ld16(tbase + COL_Y2 + lane_off + 64 * hh + 16 * k, s2);
+          float v[16];
+          tmem_ld16(tbase + COL_Y + 128 * yb + lane_off + 64 * hh + 16 * k, v);
           tmem_ld_wait();
           if (k == 3) {
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.yfree);
+            if (lane == 0) mbar_arrive(&sm.yfree[yb]);
           }
-          uint32_t w[8];
+          uint32_t w[4];
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            w[e] = pack_bf16(fmaf(gi, s2[2 * e], a[2 * e]), fmaf(gi, s2[2 * e + 1], a[2 * e + 1]));
-          if (lane < 16 && has_y) {
-            st_shared_v4(yrow + sw128_off(i, 2 * k), w[0], w[1], w[2], w[3]);
-            st_shared_v4(yrow + sw128_off(i, 2 * k + 1), w[4], w[5], w[6], w[7]);
+          for (int e = 0; e < 8; e += 2) {
+            // lo lane sends Y1 columns 8-15, hi lane sends Y2 columns 0-7
+            const float r0 = __shfl_xor_sync(0xffffffffu, hi ? v[e] : v[8 + e], 16);
+            const float r1 = __shfl_xor_sync(0xffffffffu, hi ? v[e + 1] : v[9 + e], 16);
+            const float y0 = hi ? fmaf(gi, v[8 + e], r0) : fmaf(gi, r0, v[e]);
+            const float y1 = hi ? fmaf(gi, v[9 + e], r1) : fmaf(gi, r1, v[e + 1]);
+            w[e >> 1] = pack_bf16(y0, y1);
           }
+          if (has_y) st_shared_v4(yrow + sw128_off(i, 2 * k + hi), w[0], w[1], w[2], w[3]);
         }
         fence_proxy_async_smem();
         __syncwarp();
