@@ -116,7 +116,7 @@ struct Smem {
   uint64_t gfull[GS], gempty[GS];
   uint64_t sfull, sempty;
   uint64_t ccfull, b1full, b2full, b3full;
-  uint64_t m1done, m2done, xscaled, lbready, done;
+  uint64_t m1a, m1done, m2done, xscaled, lbready, done;
   uint32_t tmem_base;
   int abort;
 };
@@ -126,6 +126,7 @@ constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
 enum : uint32_t {
   W_TMA_XEMPTY = 0x001, W_TMA_SEMPTY, W_TMA_DRAIN,
   W_MMA_XFULL = 0x101, W_MMA_M2, W_MMA_SFULL, W_MMA_LB, W_MMA_M1, W_MMA_XS, W_MMA_DONE,
+  W_MMA_M1A,
   W_GATE_EMPTY = 0x201,
   W_M_GFULL = 0x401, W_M_CC, W_M_B1, W_M_B2, W_M_B3,
 };
@@ -211,6 +212,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(&sm.b1full, 1);
     mbar_init(&sm.b2full, 1);
     mbar_init(&sm.b3full, 1);
+    mbar_init(&sm.m1a, NMATH);
     mbar_init(&sm.m1done, NMATH);
     mbar_init(&sm.m2done, NMATH);
     mbar_init(&sm.xscaled, NMATH);
@@ -285,19 +287,37 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t id_r1 = idesc_bf16(128, 64, false, false);     // Lam X^T
         const uint32_t id_v = idesc_bf16(64, 64, false, true);        // Bm Q^T
         const uint32_t sS = smem_u32(sm.Sin), sW0 = smem_u32(sm.W0), sL = smem_u32(sm.Lb);
-        // Software-pipelined order: the Gram products and dW0 of chunk it+1 are
-        // issued as soon as the math warps have read chunk it's phase-2 results,
-        // ahead of chunk it's Lam update; only Lam X^T waits for the new Lam.
+        // Issue order per chunk: the products on the carried chain first (the Lam
+        // update of the previous chunk, then DXb and R1 = Lam X^T of this one), then
+        // the Gram products and dW0, which the tensor pipe works through while the
+        // math warps use R1 and DXb; the dx terms that need only scaled G and DXb
+        // next; last the three products that need the chunk matrices.
         auto xgu = [&](int it, uint32_t& sX, uint32_t& sG, uint32_t& sU) {
           const int st = it % NS;
           sX = smem_u32(sm.X[st]);
           sG = smem_u32(sm.G[st]);
           sU = smem_u32(sm.U[st]);
         };
-        auto phase1a = [&](int it) -> bool {  // K, Kug, KugT, dW0
+        auto phase1b = [&](int it) -> bool {  // DXb^T, R1^T
           uint32_t sX, sG, sU;
           xgu(it, sX, sG, sU);
           if (!mbar_wait(&sm.xfull[it % NS], (it / NS) & 1, wc, W_MMA_XFULL)) return false;
+          if (!mbar_wait(&sm.sfull, it & 1, wc, W_MMA_SFULL)) return false;
+          tc_fence_after();
+          for (int kk = 0; kk < 8; ++kk)  // DXb^T = S_in^T U^T
+            umma_bf16(tbase + COL_D, sw128_desc(sS + kk * 2048, BIG, 1024),
+                      sw128_desc(sU + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024), id_db, kk > 0);
+          if (it > 0 && !mbar_wait(&sm.lbready, (it - 1) & 1, wc, W_MMA_LB)) return false;
+          tc_fence_after();
+          for (int kk = 0; kk < 8; ++kk)  // R1^T = Lam X^T
+            umma_bf16(tbase + COL_R, sw128_desc(sL + (kk >> 2) * BIG + (kk & 3) * 32, 16, 1024),
+                      sw128_desc(sX + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024), id_r1, kk > 0);
+          umma_commit(&sm.b1full);
+          return true;
+        };
+        auto phase1a = [&](int it) -> bool {  // K, Kug, KugT, dW0
+          uint32_t sX, sG, sU;
+          xgu(it, sX, sG, sU);
           if (it > 0 && !mbar_wait(&sm.m2done, (it - 1) & 1, wc, W_MMA_M2)) return false;
           tc_fence_after();
           for (int kk = 0; kk < 8; ++kk) {  // K = X X^T, Kug = U G^T, KugT = G U^T
@@ -315,23 +335,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                       sw128_desc(sX + kk * 2048, TILE, 1024), id_w, (it > 0 || kk > 0));
           return true;
         };
-        auto phase1b = [&](int it) -> bool {  // DXb^T, R1^T
+        auto phase2a = [&](int it) -> bool {  // dx^T terms that need only Gs and gam (.) DXb^T
           uint32_t sX, sG, sU;
           xgu(it, sX, sG, sU);
-          if (!mbar_wait(&sm.sfull, it & 1, wc, W_MMA_SFULL)) return false;
+          if (!mbar_wait(&sm.m1a, it & 1, wc, W_MMA_M1A)) return false;
           tc_fence_after();
-          for (int kk = 0; kk < 8; ++kk)  // DXb^T = S_in^T U^T
-            umma_bf16(tbase + COL_D, sw128_desc(sS + kk * 2048, BIG, 1024),
-                      sw128_desc(sU + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024), id_db, kk > 0);
-          if (it > 0 && !mbar_wait(&sm.lbready, (it - 1) & 1, wc, W_MMA_LB)) return false;
-          tc_fence_after();
-          for (int kk = 0; kk < 8; ++kk)  // R1^T = Lam X^T
-            umma_bf16(tbase + COL_R, sw128_desc(sL + (kk >> 2) * BIG + (kk & 3) * 32, 16, 1024),
-                      sw128_desc(sX + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024), id_r1, kk > 0);
-          umma_commit(&sm.b1full);
+          for (int kk = 0; kk < 8; ++kk)  // dx^T = gam (.) DXb^T + W0^T U^T
+            umma_bf16(tbase + COL_D, sw128_desc(sW0 + kk * 2048, BIG, 1024),
+                      sw128_desc(sU + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024), id_db, 1);
+          for (int kk = 0; kk < 8; ++kk)  //      + Lam^T Gs^T
+            umma_bf16(tbase + COL_D, sw128_desc(sL + kk * 2048, BIG, 1024),
+                      sw128_desc(sG + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024), id_db, 1);
           return true;
         };
-        auto phase2 = [&](int it) -> bool {
+        auto phase2b = [&](int it) -> bool {  // the products of the chunk matrices
           uint32_t sX, sG, sU;
           xgu(it, sX, sG, sU);
           if (!mbar_wait(&sm.m1done, it & 1, wc, W_MMA_M1)) return false;
@@ -342,15 +359,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int kk = 0; kk < 4; ++kk)  // r^T = del (.) R1^T + U^T Ar^T
             umma_bf16(tbase + COL_R, sw128_desc(sU + kk * 2048, TILE, 1024),
                       sw128_desc(sS + CC_AR + kk * 32, 16, 1024), id_db, 1);
-          for (int kk = 0; kk < 8; ++kk)  // dx^T = gam (.) DXb^T + W0^T U^T
-            umma_bf16(tbase + COL_D, sw128_desc(sW0 + kk * 2048, BIG, 1024),
-                      sw128_desc(sU + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024), id_db, 1);
-          for (int kk = 0; kk < 4; ++kk)  //      + X^T Z^T
+          for (int kk = 0; kk < 4; ++kk)  // dx^T += X^T Z^T
             umma_bf16(tbase + COL_D, sw128_desc(sX + kk * 2048, TILE, 1024),
                       sw128_desc(sS + CC_Z + kk * 32, 16, 1024), id_db, 1);
-          for (int kk = 0; kk < 8; ++kk)  //      + Lam^T Gs^T
-            umma_bf16(tbase + COL_D, sw128_desc(sL + kk * 2048, BIG, 1024),
-                      sw128_desc(sG + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024), id_db, 1);
           umma_commit(&sm.b2full);
           umma_commit(&sm.sempty);
           return true;
@@ -367,11 +378,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           umma_commit(&sm.xempty[it % NS]);
           return true;
         };
-        bool ok = phase1a(0) && phase1b(0) && phase2(0);
+        auto chunk = [&](int it) -> bool {
+          return phase1b(it) && phase1a(it) && phase2a(it) && phase2b(it);
+        };
+        bool ok = chunk(0);
         for (int it = 0; it < nch && ok; ++it) {
-          if (it + 1 < nch) ok = phase1a(it + 1);
-          ok = ok && phase3(it);
-          if (it + 1 < nch) ok = ok && phase1b(it + 1) && phase2(it + 1);
+          ok = phase3(it);
+          if (it + 1 < nch) ok = ok && chunk(it + 1);
         }
         umma_commit(&sm.done);
         mbar_drain(&sm.done, 0, wc, W_MMA_DONE);
@@ -466,7 +479,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       ok = ok && mbar_wait_warp(&sm.gfull[g], (it / GS) & 1, wc, W_M_GFULL);
       ok = ok && mbar_wait_warp(&sm.xfull[st], (it / NS) & 1, wc, W_M_GFULL);
       ok = ok && mbar_wait_warp(&sm.sfull, it & 1, wc, W_M_GFULL);
-      ok = ok && mbar_wait_warp(&sm.ccfull, it & 1, wc, W_M_CC);
       ok = ok && mbar_wait_warp(&sm.b1full, it & 1, wc, W_M_B1);
       tc_fence_after();
 
@@ -533,6 +545,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tmem_st_wait();
       }
       named_sync_math();  // (B1) S_in read; partial sums of q, p and E written; G read
+      // the Gram products (which read G) are complete before G is scaled in place
+      ok = ok && mbar_wait_warp(&sm.ccfull, it & 1, wc, W_M_CC);
+      tc_fence_after();
       if (ok) {  // G <- diag(-eta del) G, rows scaled with packed bf16 multiplies
 #pragma unroll
         for (int k = 0; k < (2 * TILE / 16) / (32 * NMATH); ++k) {
@@ -544,6 +559,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           st_shared_v4(sG + off, hmul2_bf16(v.x, fv), hmul2_bf16(v.y, fv), hmul2_bf16(v.z, fv),
                        hmul2_bf16(v.w, fv));
         }
+        // Gs and gam (.) DXb^T are in place (the TMEM writes finished before B1)
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.m1a);
       }
       if (ok && mt < C) {
         const int j = mt;
