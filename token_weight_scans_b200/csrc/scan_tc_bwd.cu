@@ -654,11 +654,77 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             st_shared_v4(b2 + sw128_off(i, 2 * wg + cc), m2[0], m2[1], m2[2], m2[3]);
           }
         };
-        if (gs.fac) build(std::true_type{});
+        // With the factored decays, a warp whose 16 x 16 block lies wholly above
+        // (wg > q: every j > i) or below (wg < q: every j < i) the diagonal needs no
+        // masks, and fewer exchanges: above, each lane already holds what it needs
+        // (lanes < 16: K and KugT; lanes >= 16 produce only Bm and t3); below, one
+        // exchange gives both halves K_ij Kug_ij.
+        auto store_pair = [&](int cc, const float (&v0)[8], const float (&v1)[8]) {
+          st_shared_v4(b1 + sw128_off(i, 2 * wg + cc), pack_bf16(v0[0], v0[1]),
+                       pack_bf16(v0[2], v0[3]), pack_bf16(v0[4], v0[5]), pack_bf16(v0[6], v0[7]));
+          st_shared_v4(b2 + sw128_off(i, 2 * wg + cc), pack_bf16(v1[0], v1[1]),
+                       pack_bf16(v1[2], v1[3]), pack_bf16(v1[4], v1[5]), pack_bf16(v1[6], v1[7]));
+        };
+        auto build_above = [&]() {
+          const float neti = -eti;
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            float v0[8], v1[8];
+#pragma unroll
+            for (int e4 = 0; e4 < 8; e4 += 4) {
+              const int jb = j0w + 8 * cc + e4;
+              const float4 cb4 = *reinterpret_cast<const float4*>(&gs.cb[jb]);
+              const float4 p4 = *reinterpret_cast<const float4*>(&sm.pv[jb]);
+              const float cbv[4] = {cb4.x, cb4.y, cb4.z, cb4.w};
+              const float pvv[4] = {p4.x, p4.y, p4.z, p4.w};
+#pragma unroll
+              for (int d = 0; d < 4; ++d) {
+                const int e = 8 * cc + e4 + d;
+                const float bij = cbv[d] * rbi;
+                const float pa = bij * vkk[e];                  // lanes < 16: b_ij K_ij
+                v0[e4 + d] = lo ? pa : 0.f;                     // Ar | Q^T = 0
+                v1[e4 + d] = lo ? neti * bij * vkt[e] : bij;    // Z | Bm
+                tpart += lo ? pa * vkt[e] : 0.f;
+                t3part += lo ? 0.f : bij * pvv[d];
+              }
+            }
+            store_pair(cc, v0, v1);
+          }
+        };
+        auto build_below = [&]() {
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            float v0[8], v1[8];
+#pragma unroll
+            for (int e4 = 0; e4 < 8; e4 += 4) {
+              const int jb = j0w + 8 * cc + e4;
+              const float4 ca4 = *reinterpret_cast<const float4*>(&gs.ca[jb]);
+              const float4 q4 = *reinterpret_cast<const float4*>(&sm.qv[jb]);
+              const float cav[4] = {ca4.x, ca4.y, ca4.z, ca4.w};
+              const float qvv[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+              for (int d = 0; d < 4; ++d) {
+                const int e = 8 * cc + e4 + d;
+                const float o = __shfl_xor_sync(0xffffffffu, vkk[e], 16);  // the other half
+                const float aij = rai * cav[d];
+                v0[e4 + d] = lo ? 0.f : vkk[e] * o;  // Ar = 0 | Q^T = K Kug
+                v1[e4 + d] = lo ? aij * o : 0.f;     // Z = a Kug | Bm = 0
+                t2part += lo ? aij * qvv[d] : 0.f;
+              }
+            }
+            store_pair(cc, v0, v1);
+          }
+        };
+        if (gs.fac && wg > q) build_above();
+        else if (gs.fac && wg < q) build_below();
+        else if (gs.fac) build(std::true_type{});
         else build(std::false_type{});
+        // each partial is nonzero in one lane half only; combine the pair
+        tpart += __shfl_xor_sync(0xffffffffu, tpart, 16);
+        t2part += __shfl_xor_sync(0xffffffffu, t2part, 16);
+        t3part += __shfl_xor_sync(0xffffffffu, t3part, 16);
         if (lo) {
           sm.t2v[wg][i] = t2part;
-        } else {
           sm.tv[wg][i] = tpart;
           sm.t3v[wg][i] = t3part;
         }
