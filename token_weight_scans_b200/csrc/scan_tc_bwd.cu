@@ -111,7 +111,7 @@ struct Smem {
   float tv[4][C], t2v[4][C], t3v[4][C], hv[4][C];
   alignas(16) float qv[C];
   alignas(16) float pv[C];
-  float ered[NMATH];
+  alignas(16) float ered[NMATH];
   uint64_t xfull[NS], xempty[NS];
   uint64_t gfull[GS], gempty[GS];
   uint64_t sfull, sempty;
@@ -570,9 +570,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         sm.qv[j] = sm.redq[0][j] + sm.redq[1][j] + sm.redq[2][j] + sm.redq[3][j];
         sm.pv[j] = sm.redp[0][j] + sm.redp[1][j] + sm.redp[2][j] + sm.redp[3][j];
       }
-      float E = 0.f;
-#pragma unroll
-      for (int w = 0; w < NMATH; ++w) E += sm.ered[w];
       named_sync_math();  // (B2) q and p complete; the S_in buffer may be overwritten
 
       if (ok) {
@@ -753,7 +750,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (!lo) {
             const int i = ir;
             float hpart = 0.f;
-            if (gs.fac) {
+            if (gs.fac && wg > q) {
+              // every j > i in this block: no term
+            } else if (gs.fac && wg < q) {  // every j < i
+              float acc = 0.f;
+#pragma unroll
+              for (int e4 = 0; e4 < 16; e4 += 4) {
+                const float4 ca4 = *reinterpret_cast<const float4*>(&gs.ca[j0w + e4]);
+                acc = fmaf(ca4.x, vv[e4], acc);
+                acc = fmaf(ca4.y, vv[e4 + 1], acc);
+                acc = fmaf(ca4.z, vv[e4 + 2], acc);
+                acc = fmaf(ca4.w, vv[e4 + 3], acc);
+              }
+              hpart = gs.ra[i] * acc;
+            } else if (gs.fac) {
               const float rai = gs.ra[i];
 #pragma unroll
               for (int e = 0; e < 16; ++e) {
@@ -824,6 +834,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const float t2 = sm.t2v[0][i] + sm.t2v[1][i] + sm.t2v[2][i] + sm.t2v[3][i];
         const float t3 = sm.t3v[0][i] + sm.t3v[1][i] + sm.t3v[2][i] + sm.t3v[3][i];
         const float h4 = sm.hv[0][i] + sm.hv[1][i] + sm.hv[2][i] + sm.hv[3][i];
+        float E = 0.f;  // <Lam_end, S_in>: sum of the math warps' partials
+#pragma unroll
+        for (int w = 0; w < NMATH; w += 4) {
+          const float4 e4 = *reinterpret_cast<const float4*>(&sm.ered[w]);
+          E += (e4.x + e4.y) + (e4.z + e4.w);
+        }
         const float da = gs.gam[i] * gs.del[i] * E + gs.del[i] * t2 + gs.gam[i] * t3 + h4;
         if (t0 + i < T) p.d_alpha[tokbase + i] = p.accumulate ? p.d_alpha[tokbase + i] + da : da;
       }
