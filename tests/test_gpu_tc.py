@@ -32,7 +32,9 @@ def _lib():
 def gpu_fwd(d):
     import token_weight_scans_b200 as tw
     t = to_device(d, "bf16")
-    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    B, H, T, di = t["x"].shape
+    ws = torch.empty(tw.gradlev_scan_workspace_bytes(B, H, T, di, t["g"].shape[-1], tw.BF16, 0),
+                     dtype=torch.uint8, device="cuda")
     y = tw.gradlev_scan_fwd(t["x"], t["g"], t["eta"], t["alpha"], t["W0"], workspace=ws)
     assert tw.gradlev_device_status(ws) == 0, "device-side wait timed out"
     return to_numpy(y)
@@ -90,7 +92,8 @@ def test_tc_fwd_timeout_path_reports_and_recovers():
     import token_weight_scans_b200 as tw
     d = inputs.draw(2, 2, 256, 128, 128, dtype="bf16", seed=44)
     t = to_device(d, "bf16")
-    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(tw.gradlev_scan_workspace_bytes(2, 2, 256, 128, 128, tw.BF16, 0),
+                     dtype=torch.uint8, device="cuda")
     tw.lib().gradlev_debug_inject_timeout(1, 20)
     tw.gradlev_scan_fwd(t["x"], t["g"], t["eta"], t["alpha"], t["W0"], workspace=ws)
     assert tw.gradlev_device_status(ws) == 5  # GRADLEV_ERR_TIMEOUT

@@ -49,23 +49,101 @@ static size_t ckpt_bytes_of(int B, int H, int T, int din, int dout, gradlev_dtyp
                                : ffma::ckpt_bytes(B, H, T, din, dout);
 }
 
+// ---- segmented long scans (tensor-core path)
+//
+// When the scans of a call cannot fill the GPU, each scan is cut into segments
+// that separate CTAs walk at the same time. Forward: a summary pass gives each
+// segment's local state and log-decay, combine_segments turns them into the
+// segments' start states, and the main pass walks every segment from its start
+// state. Reverse: the same with the adjoint, walked backwards.
+struct SegPlan {
+  int nseg = 1, seg_chunks = 1 << 30;
+};
+
+static SegPlan fwd_plan(int B, int H, int T, int dout) {
+  SegPlan s;
+  tc::segment_plan(B * H * (dout / 128), (T + tc::kChunk - 1) / tc::kChunk, &s.nseg,
+                   &s.seg_chunks);
+  return s;
+}
+
+static SegPlan bwd_plan(int B, int H, int T) {
+  SegPlan s;
+  tc::segment_plan(B * H, (T + tc::kChunk - 1) / tc::kChunk, &s.nseg, &s.seg_chunks);
+  return s;
+}
+
+// Scratch of the segment passes: local summaries and combined states
+// ([B*H][nseg][dout][din] fp32 each) and the segment log-decays ([B*H][nseg]).
+static size_t seg_bytes(int B, int H, int din, int dout, int nseg) {
+  if (nseg <= 1) return 0;
+  const size_t mats = (size_t)B * H * nseg * dout * din * sizeof(float);
+  return 2 * align_up(mats, 256) + align_up((size_t)B * H * nseg * sizeof(float), 256);
+}
+
+struct SegBufs {
+  float *loc, *comb, *L;
+};
+
+static SegBufs seg_bufs(char* base, int B, int H, int din, int dout, int nseg) {
+  const size_t mats = align_up((size_t)B * H * nseg * dout * din * sizeof(float), 256);
+  return {reinterpret_cast<float*>(base), reinterpret_cast<float*>(base + mats),
+          reinterpret_cast<float*>(base + 2 * mats)};
+}
+
+static size_t fwd_scratch_bytes(int B, int H, int T, int din, int dout, gradlev_dtype dt) {
+  if (!use_tc(din, dout, dt)) return kStatusBytes;
+  return kStatusBytes + seg_bytes(B, H, din, dout, fwd_plan(B, H, T, dout).nseg);
+}
+
+static size_t dW0_part_bytes(int B, int H, int T, int din, int dout, gradlev_dtype dt) {
+  const int nseg = use_tc(din, dout, dt) ? bwd_plan(B, H, T).nseg : 1;
+  return align_up((size_t)B * H * nseg * din * dout * sizeof(float), 256);
+}
+
 size_t bwd_scratch_bytes(int B, int H, int T, int din, int dout, gradlev_dtype dt,
                          bool own_states) {
-  size_t ws = kStatusBytes + align_up((size_t)B * H * din * dout * sizeof(float), 256);
+  size_t ws = kStatusBytes + dW0_part_bytes(B, H, T, din, dout, dt);
   if (own_states) ws += align_up(ckpt_bytes_of(B, H, T, din, dout, dt), 256);
+  if (use_tc(din, dout, dt)) {
+    const size_t fseg = own_states ? seg_bytes(B, H, din, dout, fwd_plan(B, H, T, dout).nseg) : 0;
+    const size_t bseg = seg_bytes(B, H, din, dout, bwd_plan(B, H, T).nseg);
+    ws += fseg > bseg ? fseg : bseg;
+  }
   return ws;
 }
 
 static gradlev_status launch_fwd_impl(int B, int H, int T, int din, int dout, gradlev_dtype dt,
                                       const void* x, const void* g, const float* eta,
                                       const float* alpha, const float* W0, void* y, void* ckpt,
-                                      DeviceStatus* status, cudaStream_t st) {
+                                      DeviceStatus* status, char* seg_ws, cudaStream_t st) {
   if (use_tc(din, dout, dt)) {
     const int inject = y ? g_inject : 0;
     const uint64_t tmo = inject ? g_inject_timeout_ns : kWaitTimeoutNs;
     if (y) g_inject = 0;
+    const SegPlan sp = fwd_plan(B, H, T, dout);
     tc::TcFwdParams prm{B, H, T, din, dout, eta, alpha, W0, static_cast<__nv_bfloat16*>(y),
                         static_cast<__nv_bfloat16*>(ckpt), status, tmo, inject};
+    if (sp.nseg > 1) {
+      const SegBufs sb = seg_bufs(seg_ws, B, H, din, dout, sp.nseg);
+      tc::TcFwdParams sum = prm;  // each segment's local state and log-decay
+      sum.y = nullptr;
+      sum.ckpt = nullptr;
+      sum.inject = 0;
+      sum.timeout_ns = kWaitTimeoutNs;
+      sum.nseg = sp.nseg;
+      sum.seg_chunks = sp.seg_chunks;
+      sum.S_final = sb.loc;
+      sum.seg_L = sb.L;
+      sum.summary = 1;
+      if (tc::launch_fwd(sum, x, g, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
+      if (tc::combine_segments(sb.loc, sb.L, sb.comb, B * H, sp.nseg, dout * din, 0, st) !=
+          cudaSuccess)
+        return GRADLEV_ERR_CUDA;
+      prm.nseg = sp.nseg;
+      prm.seg_chunks = sp.seg_chunks;
+      prm.S_init = sb.comb;
+    }
     return tc::launch_fwd(prm, x, g, st) == cudaSuccess ? GRADLEV_OK : GRADLEV_ERR_CUDA;
   }
   ffma::FwdArgs a{B, H, T, din, dout, x, g, eta, alpha, W0, y, static_cast<float*>(ckpt)};
@@ -79,25 +157,50 @@ gradlev_status bwd_run(int B, int H, int T, int din, int dout, gradlev_dtype dt,
                        float* dW0, const void* ckpt, char* ws, cudaStream_t st) {
   DeviceStatus* status = reinterpret_cast<DeviceStatus*>(ws);
   float* dW0_part = reinterpret_cast<float*>(ws + kStatusBytes);
-  void* own = ws + kStatusBytes + align_up((size_t)B * H * din * dout * sizeof(float), 256);
+  char* own = ws + kStatusBytes + dW0_part_bytes(B, H, T, din, dout, dt);
+  char* seg_ws = own + (ckpt ? 0 : align_up(ckpt_bytes_of(B, H, T, din, dout, dt), 256));
   if (cudaMemsetAsync(status, 0, sizeof(DeviceStatus), st) != cudaSuccess)
     return GRADLEV_ERR_CUDA;
   const void* states = ckpt;
   if (!states) {
     gradlev_status s = launch_fwd_impl(B, H, T, din, dout, dt, x, g, eta, alpha, W0, nullptr,
-                                       own, status, st);
+                                       own, status, seg_ws, st);
     if (s != GRADLEV_OK) return s;
     states = own;
   }
   if (use_tc(din, dout, dt)) {
+    const SegPlan sp = bwd_plan(B, H, T);
+    const float* L_init = nullptr;
+    if (sp.nseg > 1) {
+      // each segment's local adjoint (walked backwards from zero) and log-decay, then the
+      // adjoint at each segment's end
+      const SegBufs sb = seg_bufs(seg_ws, B, H, din, dout, sp.nseg);
+      tc::TcFwdParams sum{B, H, T, din, dout, eta, alpha, W0, nullptr, nullptr, status,
+                          kWaitTimeoutNs, 0};
+      sum.nseg = sp.nseg;
+      sum.seg_chunks = sp.seg_chunks;
+      sum.S_final = sb.loc;
+      sum.seg_L = sb.L;
+      sum.summary = 1;
+      sum.reverse = 1;
+      if (tc::launch_fwd(sum, x, dy, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
+      if (tc::combine_segments(sb.loc, sb.L, sb.comb, B * H, sp.nseg, dout * din, 1, st) !=
+          cudaSuccess)
+        return GRADLEV_ERR_CUDA;
+      L_init = sb.comb;
+    }
     // one launch per 128-row slice of d_out; later slices accumulate dx, d_eta, d_alpha
     for (int n0 = 0; n0 < dout; n0 += 128) {
       tc::TcBwdParams prm{B, H, T, din, dout, n0, n0 > 0 ? 1 : 0, eta, alpha, W0,
                           static_cast<__nv_bfloat16*>(dx), static_cast<__nv_bfloat16*>(dg),
                           d_eta, d_alpha, dW0_part, status, kWaitTimeoutNs};
+      prm.nseg = sp.nseg;
+      prm.seg_chunks = sp.seg_chunks;
+      prm.L_init = L_init;
       if (tc::launch_bwd(prm, x, g, dy, states, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
     }
-    if (ffma::launch_reduce_dW0(dW0_part, dW0, B, H, din * dout, st) != cudaSuccess)
+    // partials are [B][nseg][H]: a fixed-order sum over b and the segments
+    if (ffma::launch_reduce_dW0(dW0_part, dW0, B * sp.nseg, H, din * dout, st) != cudaSuccess)
       return GRADLEV_ERR_CUDA;
     return GRADLEV_OK;
   }
@@ -139,7 +242,8 @@ size_t gradlev_scan_ckpt_bytes(int B, int H, int T, int d_in, int d_out, gradlev
 size_t gradlev_scan_workspace_bytes(int B, int H, int T, int d_in, int d_out, gradlev_dtype dt,
                                     int is_bwd) {
   if (check_shape(B, H, T, d_in, d_out, dt) != GRADLEV_OK) return 0;
-  return is_bwd ? bwd_scratch_bytes(B, H, T, d_in, d_out, dt, true) : kStatusBytes;
+  return is_bwd ? bwd_scratch_bytes(B, H, T, d_in, d_out, dt, true)
+                : fwd_scratch_bytes(B, H, T, d_in, d_out, dt);
 }
 
 gradlev_status gradlev_scan_fwd(int B, int H, int T, int d_in, int d_out, gradlev_dtype dt,
@@ -160,7 +264,8 @@ gradlev_status gradlev_scan_fwd(int B, int H, int T, int d_in, int d_out, gradle
   DeviceStatus* status = static_cast<DeviceStatus*>(workspace);
   if (cudaMemsetAsync(status, 0, sizeof(DeviceStatus), st) != cudaSuccess)
     return GRADLEV_ERR_CUDA;
-  return launch_fwd_impl(B, H, T, d_in, d_out, dt, x, g, eta, alpha, W0, y, ckpt, status, st);
+  return launch_fwd_impl(B, H, T, d_in, d_out, dt, x, g, eta, alpha, W0, y, ckpt, status,
+                         static_cast<char*>(workspace) + kStatusBytes, st);
 }
 
 gradlev_status gradlev_scan_bwd(int B, int H, int T, int d_in, int d_out, gradlev_dtype dt,

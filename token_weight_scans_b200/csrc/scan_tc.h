@@ -10,6 +10,14 @@
 namespace gradlev {
 namespace tc {
 
+// The forward kernel walks one segment of chunks per CTA: CTA (b, h, slice, seg)
+// covers chunks [seg * seg_chunks, min(n_chunks, (seg + 1) * seg_chunks)) of
+// its scan. With nseg > 1 the segments' start states come from S_init, which a
+// summary pass (summary = 1: the state carry alone, from a zero start, ending in
+// S_final and seg_L) and a combine pass (combine_segments) produce beforehand.
+// reverse = 1 walks the segment backwards and weights row j of the G-operand by
+// 2^{L_{j-1}} instead of -eta_j 2^{L_{C-1}-L_j}: with dy in place of g, that is the
+// adjoint recursion Lam <- 2^{L_{C-1}} Lam + sum_j 2^{L_{j-1}} u_j x_j^T.
 struct TcFwdParams {
   int B, H, T, din, dout;   // din == 128, dout % 128 == 0
   const float* eta;         // [B,H,T]
@@ -20,26 +28,40 @@ struct TcFwdParams {
   DeviceStatus* status;     // device status word (workspace head)
   uint64_t timeout_ns;      // bound of every wait inside the kernel
   int inject;               // test hook: 1 = withhold one completion signal
+  int nseg = 1;             // segments per scan
+  int seg_chunks = 1 << 30; // chunks per segment (the last one may be shorter)
+  const float* S_init = nullptr;  // [B*H][nseg][dout][din] segment start states, or null (= 0)
+  float* S_final = nullptr;       // [B*H][nseg][dout][din] state after the walk, or null
+  float* seg_L = nullptr;         // [B*H][nseg] sum of log2 alpha over the segment, or null
+  int summary = 0;          // 1: state carry only (no y, no checkpoints)
+  int reverse = 0;          // 1: adjoint summary (see above)
 };
 
 // The reverse scan of one 128-row slice [n0, n0+128) of d_out: the rows of the
 // state and adjoint evolve independently, so a d_out = 256 problem is two
 // slice problems whose dx, d_eta and d_alpha add up (accumulate = 1 on the
 // second slice) and whose dg and dW0 rows are disjoint.
+//
+// The reverse kernel walks one segment per CTA, like the forward one; L_init
+// holds the adjoint at each segment's end (zero for the last segment), from the
+// reverse summary and combine passes.
 struct TcBwdParams {
   int B, H, T, din, dout;   // din == 128, dout in {128, 256}
   int n0;                   // first d_out row of this slice
   int accumulate;           // add dx, d_eta, d_alpha onto the values already there
   const float* eta;
   const float* alpha;
-  const float* W0;          // [H,128,128] float32
+  const float* W0;          // [H,dout,128] float32
   __nv_bfloat16* dx;        // [B,H,T,128]
-  __nv_bfloat16* dg;        // [B,H,T,128]
+  __nv_bfloat16* dg;        // [B,H,T,dout]
   float* d_eta;             // [B,H,T]
   float* d_alpha;           // [B,H,T]
-  float* dW0_part;          // [B*H][128][128] float32 per-scan partials
+  float* dW0_part;          // [B][nseg][H][dout][128] float32 per-(scan, segment) partials
   DeviceStatus* status;
   uint64_t timeout_ns;
+  int nseg = 1;             // segments per scan
+  int seg_chunks = 1 << 30; // chunks per segment (the last one may be shorter)
+  const float* L_init = nullptr;  // [B*H][nseg][dout][din] adjoint at each segment's end, or null
 };
 
 constexpr int kChunk = 64;  // tokens per chunk of the tensor-core kernels
@@ -52,6 +74,12 @@ cudaError_t launch_fwd(const TcFwdParams& p, const void* x, const void* g, cudaS
 cudaError_t launch_bwd(const TcBwdParams& p, const void* x, const void* g, const void* dy,
                        const void* ckpt, cudaStream_t st);
 size_t fwd_smem_bytes();
+// Segments for `units` CTAs per segment index over a scan of n_chunks chunks.
+void segment_plan(int units, int n_chunks, int* nseg, int* seg_chunks);
+// The serial recursion over segment summaries (forward: start states; reverse:
+// end adjoints), element by element for `scans` scans of per_scan elements.
+cudaError_t combine_segments(const float* loc, const float* segL, float* out, int scans, int nseg,
+                             int per_scan, int reverse, cudaStream_t st);
 
 }  // namespace tc
 }  // namespace gradlev

@@ -191,9 +191,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   Smem& sm = *reinterpret_cast<Smem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.x, h = bh % p.H;
+  const int bh = blockIdx.x / p.nseg, seg = blockIdx.x - bh * p.nseg, h = bh % p.H;
   const int T = p.T;
-  const int nch = (T + C - 1) / C;
+  const int nch_all = (T + C - 1) / C;         // chunks of the whole sequence
+  const int c0 = seg * p.seg_chunks;           // this CTA's segment: chunks [c0, c1),
+  const int c1 = min(nch_all, c0 + p.seg_chunks);  // walked from c1 - 1 down to c0
+  const int nch = c1 - c0;
+  const size_t seg_row = (size_t)bh * p.nseg + seg;  // [bh][seg] index of the segment adjoints
   const WaitCtx wc{&sm.abort, p.status, p.timeout_ns};
 
   if (threadIdx.x == 0) {
@@ -233,7 +237,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tmem_relinquish();
   }
   if (warp >= 4) {
-    // W0 -> bf16 swizzled [k-block][n rows]; Lam_T = 0
+    // W0 -> bf16 swizzled [k-block][n rows]; the bf16 adjoint at the segment's end
+    // (Lam_T = 0 for the last segment)
     const int t = threadIdx.x - 128;
     const float* W0 = p.W0 + ((size_t)h * p.dout + p.n0) * 128;
     for (int idx = t; idx < 128 * 16; idx += 32 * NMATH) {
@@ -243,7 +248,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const float4 b = *reinterpret_cast<const float4*>(W0 + (size_t)n * 128 + ck * 8 + 4);
       st_shared_v4(smem_u32(sm.W0 + kb * BIG) + sw128_off(n, c), pack_bf16(a.x, a.y),
                    pack_bf16(a.z, a.w), pack_bf16(b.x, b.y), pack_bf16(b.z, b.w));
-      st_shared_v4(smem_u32(sm.Lb + kb * BIG) + sw128_off(n, c), 0u, 0u, 0u, 0u);
+      if (p.L_init) {
+        const float* li = p.L_init + (seg_row * p.dout + p.n0 + n) * 128 + ck * 8;
+        const float4 u = *reinterpret_cast<const float4*>(li);
+        const float4 v = *reinterpret_cast<const float4*>(li + 4);
+        st_shared_v4(smem_u32(sm.Lb + kb * BIG) + sw128_off(n, c), pack_bf16(u.x, u.y),
+                     pack_bf16(u.z, u.w), pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
+      } else {
+        st_shared_v4(smem_u32(sm.Lb + kb * BIG) + sw128_off(n, c), 0u, 0u, 0u, 0u);
+      }
     }
     fence_proxy_async_smem();
   }
@@ -258,7 +271,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (lane == 0) {
         int xi = 0, si = 0;
         for (int it = 0; it < nch; ++it) {
-          const int c = nch - 1 - it, st = it % NS;
+          const int c = c1 - 1 - it, st = it % NS;
           if (!mbar_wait(&sm.xempty[st], ((it / NS) & 1) ^ 1, wc, W_TMA_XEMPTY)) break;
           mbar_arrive_expect_tx(&sm.xfull[st], 6 * TILE);
           tma_load_3d(sm.X[st], &tmX, &sm.xfull[st], 0, c * C, bh);
@@ -270,8 +283,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           xi = it + 1;
           if (!mbar_wait(&sm.sempty, (it & 1) ^ 1, wc, W_TMA_SEMPTY)) break;
           mbar_arrive_expect_tx(&sm.sfull, 2 * BIG);
-          tma_load_3d(sm.Sin, &tmS, &sm.sfull, 0, p.n0, bh * nch + c);
-          tma_load_3d(sm.Sin + BIG, &tmS, &sm.sfull, 64, p.n0, bh * nch + c);
+          tma_load_3d(sm.Sin, &tmS, &sm.sfull, 0, p.n0, bh * nch_all + c);
+          tma_load_3d(sm.Sin + BIG, &tmS, &sm.sfull, 64, p.n0, bh * nch_all + c);
           si = it + 1;
         }
         for (int it = xi > NS ? xi - NS : 0; it < xi; ++it)
@@ -393,7 +406,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // ---------------------------------------------------------- gate prep
       const size_t gbase = (size_t)bh * T;
       for (int it = 0; it < nch; ++it) {
-        const int c = nch - 1 - it, g = it % GS;
+        const int c = c1 - 1 - it, g = it % GS;
         if (!mbar_wait_warp(&sm.gempty[g], ((it / GS) & 1) ^ 1, wc, W_GATE_EMPTY)) break;
         GateSlot& gs = sm.gates[g];
         const int t0 = c * C + lane, t1 = t0 + 32;
@@ -457,10 +470,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t sS = smem_u32(sm.Sin);
     const uint32_t tL = tbase + COL_L + lane_off + 32 * wg;  // this thread's Lam columns
     const uint32_t sLb = smem_u32(sm.Lb);
-    {  // Lam_T = 0
+    {  // the fp32 adjoint at the segment's end (Lam_T = 0 for the last segment)
       float z[32];
+      if (p.L_init) {
+        const float4* li = reinterpret_cast<const float4*>(
+            p.L_init + (seg_row * p.dout + p.n0 + n) * 128 + 32 * wg);
 #pragma unroll
-      for (int e = 0; e < 32; ++e) z[e] = 0.f;
+        for (int e = 0; e < 8; ++e) {
+          const float4 v = li[e];
+          z[4 * e] = v.x;
+          z[4 * e + 1] = v.y;
+          z[4 * e + 2] = v.z;
+          z[4 * e + 3] = v.w;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) z[e] = 0.f;
+      }
       tmem_st32(tL, z);
       tmem_st_wait();
     }
@@ -471,7 +497,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // warp can be left at a bar.sync that its peers never reach.
     bool ok = true;
     for (int it = 0; it < nch; ++it) {
-      const int c = nch - 1 - it, st = it % NS, g = it % GS;
+      const int c = c1 - 1 - it, st = it % NS, g = it % GS;
       const GateSlot& gs = sm.gates[g];
       const int t0 = c * C;
       const size_t tokbase = (size_t)bh * T + t0;
@@ -877,7 +903,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       float v[32];
       tmem_ld32(tbase + COL_W + lane_off + 32 * wg, v);
       tmem_ld_wait();
-      float4* dst = reinterpret_cast<float4*>(p.dW0_part + ((size_t)bh * p.dout + p.n0 + n) * 128 + 32 * wg);
+      // partial of (b, seg, h): the fixed-order reduction sums over b and seg
+      const size_t part = ((size_t)(bh / p.H) * p.nseg + seg) * p.H + h;
+      float4* dst = reinterpret_cast<float4*>(p.dW0_part + (part * p.dout + p.n0 + n) * 128 + 32 * wg);
 #pragma unroll
       for (int e = 0; e < 8; ++e) dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
     }
@@ -912,7 +940,7 @@ cudaError_t launch_bwd(const TcBwdParams& prm, const void* x, const void* g, con
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  bwd_kernel<<<(int)BH, NTHREADS, kSmemBytes, st>>>(mx, mg, mu, ms, mdx, mdg, prm);
+  bwd_kernel<<<(int)BH * prm.nseg, NTHREADS, kSmemBytes, st>>>(mx, mg, mu, ms, mdx, mdg, prm);
   count_launch();
   return cudaGetLastError();
 }

@@ -127,11 +127,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nslice = p.dout >> 7;
-  const int bh = blockIdx.x / nslice, slice = blockIdx.x - bh * nslice;
+  const int unit = blockIdx.x / p.nseg, seg = blockIdx.x - unit * p.nseg;
+  const int bh = unit / nslice, slice = unit - bh * nslice;
   const int h = bh % p.H;
   const int n0 = slice * 128;
   const int T = p.T;
-  const int nch = (T + C - 1) / C;
+  const int nch_all = (T + C - 1) / C;           // chunks of the whole sequence
+  const int c0 = seg * p.seg_chunks;             // this CTA's segment: chunks [c0, c1)
+  const int c1 = min(nch_all, c0 + p.seg_chunks);
+  const int nch = c1 - c0;                       // chunks this CTA walks
+  // global chunk of the c-th chunk walked (a reverse summary walks the segment backwards)
+  auto cg = [&](int c) { return p.reverse ? c1 - 1 - c : c0 + c; };
+  const size_t seg_row = (size_t)bh * p.nseg + seg;  // [bh][seg] index of the segment states
   const WaitCtx wc{&sm.abort, p.status, p.timeout_ns};
 
   if (threadIdx.x == 0) {
@@ -183,7 +190,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const float4 b = *reinterpret_cast<const float4*>(W0 + (size_t)n * 128 + ck * 8 + 4);
       st_shared_v4(smem_u32(sm.W0[kb]) + sw128_off(n, c), pack_bf16(a.x, a.y),
                    pack_bf16(a.z, a.w), pack_bf16(b.x, b.y), pack_bf16(b.z, b.w));
-      st_shared_v4(smem_u32(sm.S[0][kb]) + sw128_off(n, c), 0u, 0u, 0u, 0u);
+      if (p.S_init) {  // the segment's start state (rows of this slice), fp32 -> bf16
+        const float* si = p.S_init + (seg_row * p.dout + n0 + n) * 128 + ck * 8;
+        const float4 u = *reinterpret_cast<const float4*>(si);
+        const float4 v = *reinterpret_cast<const float4*>(si + 4);
+        st_shared_v4(smem_u32(sm.S[0][kb]) + sw128_off(n, c), pack_bf16(u.x, u.y),
+                     pack_bf16(u.z, u.w), pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
+      } else {
+        st_shared_v4(smem_u32(sm.S[0][kb]) + sw128_off(n, c), 0u, 0u, 0u, 0u);
+      }
     }
     fence_proxy_async_smem();
   }
@@ -200,10 +215,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int s = c % NS;
         if (!mbar_wait(&sm.empty[s], ((c / NS) & 1) ^ 1, wc, W_TMA_EMPTY)) break;
         mbar_arrive_expect_tx(&sm.full[s], 4 * TILE);
-        tma_load_3d(sm.X[s], &tmX, &sm.full[s], 0, c * C, bh);
-        tma_load_3d(sm.X[s] + TILE, &tmX, &sm.full[s], 64, c * C, bh);
-        tma_load_3d(sm.G[s], &tmG, &sm.full[s], n0, c * C, bh);
-        tma_load_3d(sm.G[s] + TILE, &tmG, &sm.full[s], n0 + 64, c * C, bh);
+        const int t0 = cg(c) * C;
+        tma_load_3d(sm.X[s], &tmX, &sm.full[s], 0, t0, bh);
+        tma_load_3d(sm.X[s] + TILE, &tmX, &sm.full[s], 64, t0, bh);
+        tma_load_3d(sm.G[s], &tmG, &sm.full[s], n0, t0, bh);
+        tma_load_3d(sm.G[s] + TILE, &tmG, &sm.full[s], n0 + 64, t0, bh);
         issued = c + 1;
       }
       // teardown: let every load this thread issued land before the CTA exits
@@ -223,15 +239,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t sX = smem_u32(sm.X[s]), sG = smem_u32(sm.G[s]);
         const uint32_t sXh = smem_u32(sm.Xh[b]), sS = smem_u32(sm.S[b][0]);
         if (!mbar_wait(&sm.full[s], (c / NS) & 1, wc, W_MMA_FULL)) break;
-        if (!mbar_wait(&sm.kfree[b], ((c >> 1) & 1) ^ 1, wc, W_MMA_KFREE)) break;
-        tc_fence_after();
-        // K = X X^T
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * TILE + (kk & 3) * 32;
-          umma_bf16(tbase + (b ? COL_K1 : COL_K0), sw128_desc(sX + off, 16, 1024),
-                    sw128_desc(sX + off, 16, 1024), id_k, kk > 0);
+        if (!p.summary) {
+          if (!mbar_wait(&sm.kfree[b], ((c >> 1) & 1) ^ 1, wc, W_MMA_KFREE)) break;
+          tc_fence_after();
+          // K = X X^T
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * TILE + (kk & 3) * 32;
+            umma_bf16(tbase + (b ? COL_K1 : COL_K0), sw128_desc(sX + off, 16, 1024),
+                      sw128_desc(sX + off, 16, 1024), id_k, kk > 0);
+          }
+          if (!(p.inject == 1 && c == 1)) umma_commit(&sm.kfull[b]);
         }
-        if (!(p.inject == 1 && c == 1)) umma_commit(&sm.kfull[b]);
         // dS = G^T Xhat
         if (!mbar_wait(&sm.xhready[b], (c >> 1) & 1, wc, W_MMA_XREADY)) break;
         if (c > 0 && !mbar_wait(&sm.dsfree, (c - 1) & 1, wc, W_MMA_DSFREE)) break;
@@ -241,6 +259,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     sw128_desc(sXh + kk * 2048, TILE, 1024), id_ds, kk > 0);
         umma_commit(&sm.dsfull);
         umma_commit(&sm.xhfree[b]);
+        if (p.summary) {  // state carry only: the stage is free once dS has read it
+          umma_commit(&sm.empty[s]);
+          continue;
+        }
         // Y1 = X W0^T into buffer b (the epilogue of chunk c - 2 has read it)
         const uint32_t tY1 = tbase + COL_Y + 128 * b, tY2 = tY1 + LANE16;
         if (!mbar_wait(&sm.yfree[b], ((c >> 1) & 1) ^ 1, wc, W_MMA_YFREE)) break;
@@ -284,15 +306,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const size_t gbase = (size_t)bh * T;
     const bool gate_warp = warp == 2;
     float ra[PD][2], re[PD][2];
+    float Lseg = 0.f;  // sum of log2 alpha over the walked chunks (lane-uniform)
+    // gates of the c-th walked chunk (alpha = 1, eta = 0 past the walk or past T)
+    auto gate_load = [&](int c, float (&a)[2], float (&e)[2]) {
+      const bool in = c < nch;
+      const int t0 = (in ? cg(c) : 0) * C + lane, t1 = t0 + 32;
+      a[0] = in && t0 < T ? p.alpha[gbase + t0] : 1.f;
+      a[1] = in && t1 < T ? p.alpha[gbase + t1] : 1.f;
+      e[0] = in && t0 < T ? p.eta[gbase + t0] : 0.f;
+      e[1] = in && t1 < T ? p.eta[gbase + t1] : 0.f;
+    };
     if (gate_warp) {
 #pragma unroll
-      for (int k = 0; k < PD; ++k) {
-        const int t0 = k * C + lane, t1 = t0 + 32;
-        ra[k][0] = t0 < T ? p.alpha[gbase + t0] : 1.f;
-        ra[k][1] = t1 < T ? p.alpha[gbase + t1] : 1.f;
-        re[k][0] = t0 < T ? p.eta[gbase + t0] : 0.f;
-        re[k][1] = t1 < T ? p.eta[gbase + t1] : 0.f;
-      }
+      for (int k = 0; k < PD; ++k) gate_load(k, ra[k], re[k]);
     }
     bool ok = true;
     for (int cb = 0; cb < nch && ok; cb += PD) {
@@ -305,13 +331,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (gate_warp) {
           if (!mbar_wait_warp(&sm.gempty[g], ((c / GS) & 1) ^ 1, wc, W_GATE_EMPTY)) { ok = false; break; }
           const float a0 = ra[k][0], a1 = ra[k][1], e0 = re[k][0], e1 = re[k][1];
-          {  // prefetch the gates of chunk c + PD into this register slot
-            const int t0 = (c + PD) * C + lane, t1 = t0 + 32;
-            ra[k][0] = t0 < T ? p.alpha[gbase + t0] : 1.f;
-            ra[k][1] = t1 < T ? p.alpha[gbase + t1] : 1.f;
-            re[k][0] = t0 < T ? p.eta[gbase + t0] : 0.f;
-            re[k][1] = t1 < T ? p.eta[gbase + t1] : 0.f;
-          }
+          gate_load(c + PD, ra[k], re[k]);  // prefetch chunk c + PD into this register slot
           float l0 = fmaxf(log2f(a0), -100.f), l1 = fmaxf(log2f(a1), -100.f);
 #pragma unroll
           for (int o = 1; o < 32; o <<= 1) {
@@ -325,6 +345,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const float last0 = __shfl_sync(0xffffffffu, l0, 31);
           l1 += last0;
           const float Lend = __shfl_sync(0xffffffffu, l1, 31);
+          Lseg += Lend;
           const float pm0 = __shfl_up_sync(0xffffffffu, l0, 1);
           const float pm1 = __shfl_up_sync(0xffffffffu, l1, 1);
           gs.L[lane] = l0;
@@ -354,7 +375,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int idx = (warp - 2) * 32 + lane; idx < 2 * TILE / 16; idx += 64) {
           const uint32_t off = idx * 16;
           const int j = (off & (TILE - 1)) >> 7;  // token row
-          const __nv_bfloat162 w2 = __float2bfloat162_rn(gs.w[j]);
+          // forward: -eta_j 2^{L_{C-1}-L_j}; reverse (adjoint) summary: 2^{L_{j-1}}
+          const __nv_bfloat162 w2 = __float2bfloat162_rn(p.reverse ? gs.gam[j] : gs.w[j]);
           const uint32_t wv = *reinterpret_cast<const uint32_t*>(&w2);
           uint4 v = ld_shared_v4(src + off);
           v.x = hmul2_bf16(v.x, wv);
@@ -371,24 +393,39 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
     }
+    if (ok && gate_warp && lane == 0 && p.seg_L && slice == 0) p.seg_L[seg_row] = Lseg;
   } else {
     // ------------------------------------------------------------ math warpgroups
     const int q = warp & 3;          // TMEM lane quadrant
     const int hh = (warp - 4) >> 2;  // warpgroup: state and output columns [64hh, 64hh+64)
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
     const int n = 32 * q + lane;     // row of the d_out slice owned by this thread
-    float Sreg[64];
+    float Sreg[64];  // fp32 state: row n, columns [64hh, 64hh+64)
+    if (p.S_init) {
+      const float4* si = reinterpret_cast<const float4*>(
+          p.S_init + (seg_row * p.dout + n0 + n) * 128 + 64 * hh);
 #pragma unroll
-    for (int e = 0; e < 64; ++e) Sreg[e] = 0.f;
-    const bool has_y = p.y != nullptr, has_ck = p.ckpt != nullptr;
+      for (int e = 0; e < 16; ++e) {
+        const float4 v = si[e];
+        Sreg[4 * e] = v.x;
+        Sreg[4 * e + 1] = v.y;
+        Sreg[4 * e + 2] = v.z;
+        Sreg[4 * e + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 64; ++e) Sreg[e] = 0.f;
+    }
+    const bool full = !p.summary;  // outputs, not just the state carry
+    const bool has_y = full && p.y != nullptr, has_ck = full && p.ckpt != nullptr;
     // Each warp TMA-stores what it wrote itself: its 32 rows of one k-block of the
     // bf16 state (the chunk-start checkpoints, bf16 [bh][chunk][dout][din], box of
     // 32 rows) and its 16 token rows of one n-block of y (box of 16 rows). S_0 = 0
     // is buffer 0.
     const uint32_t s_part = (uint32_t)(32 * q) * 128;  // byte offset of the warp's state rows
     const uint32_t y_part = (uint32_t)(16 * q) * 128;  // byte offset of the warp's token rows
-    if (has_ck && lane == 0) {
-      tma_store_3d(&tmS, sm.S[0][hh] + s_part, 64 * hh, n0 + 32 * q, bh * nch);
+    if (has_ck && lane == 0) {  // the checkpoint of the segment's first chunk
+      tma_store_3d(&tmS, sm.S[0][hh] + s_part, 64 * hh, n0 + 32 * q, bh * nch_all + c0);
       tma_store_commit();
     }
 
@@ -445,7 +482,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // per y part, in the order CK_{c+1} (state update of chunk c), Y_c (epilogue of
     // chunk c); before its rows of a buffer are rewritten it waits until the
     // group that last read them is done reading.
-    bool ok = nch > 0 ? mask(0) : true;
+    bool ok = (nch > 0 && full) ? mask(0) : true;
     for (int c = 0; c < nch; ++c) {
       const int g = c % GS;
       const GateSlot& gs = sm.gates[g];
@@ -455,7 +492,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       //      parity wait can never see a phase from the other buffer's traffic)
       const int wb = (c + 1) & 1;
       ok = ok && mbar_wait_warp(&sm.dsfull, c & 1, wc, W_M_DSFULL);
-      ok = ok && (c == 0 || mbar_wait_warp(&sm.sfree[wb], ((c - 1) >> 1) & 1, wc, W_M_SFREE));
+      ok = ok && (c == 0 || !full || mbar_wait_warp(&sm.sfree[wb], ((c - 1) >> 1) & 1, wc, W_M_SFREE));
       // CK_{c-1} last read these rows of buffer wb; at most Y_{c-2}, CK_c, Y_{c-1}
       // (or CK_1, Y_0 after CK_0) are newer
       if (lane == 0 && has_ck) store_reads_pending_at_most(has_y ? 2 : 1);
@@ -476,6 +513,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
 #pragma unroll
           for (int e = 0; e < 32; ++e) Sreg[32 * hf + e] = fmaf(gC, Sreg[32 * hf + e], v[e]);
+          if (!full) continue;
 #pragma unroll
           for (int cc = 4 * hf; cc < 4 * hf + 4; ++cc)
             st_shared_v4(srow + sw128_off(n, cc), pack_bf16(Sreg[8 * cc], Sreg[8 * cc + 1]),
@@ -485,13 +523,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) {
+        if (lane == 0 && full) {
           mbar_arrive(&sm.sready[wb]);
           if (has_ck && c + 1 < nch) {
-            tma_store_3d(&tmS, sm.S[wb][hh] + s_part, 64 * hh, n0 + 32 * q, bh * nch + c + 1);
+            tma_store_3d(&tmS, sm.S[wb][hh] + s_part, 64 * hh, n0 + 32 * q,
+                         bh * nch_all + cg(c) + 1);
             tma_store_commit();
           }
         }
+      }
+      if (!full) {  // state carry only
+        __syncwarp();
+        if (ok && lane == 0) mbar_arrive(&sm.gempty[g]);
+        continue;
       }
 
       // ---- mask of the next chunk (keeps the MMA stream fed while we store y)
@@ -536,14 +580,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         fence_proxy_async_smem();
         __syncwarp();
         // rows past T are clipped; a part that starts past T is not issued
-        if (lane == 0 && has_y && c * C + 16 * q < T) {
-          tma_store_3d(&tmY, sm.Ys + hh * TILE + y_part, n0 + 64 * hh, c * C + 16 * q, bh);
+        if (lane == 0 && has_y && cg(c) * C + 16 * q < T) {
+          tma_store_3d(&tmY, sm.Ys + hh * TILE + y_part, n0 + 64 * hh, cg(c) * C + 16 * q, bh);
           tma_store_commit();
         }
         if (lane == 0) mbar_arrive(&sm.gempty[g]);
       }
     }
     if (lane == 0) tma_store_wait_all();
+    if (ok && p.S_final) {  // the state after the walked chunks, fp32
+      float4* so = reinterpret_cast<float4*>(p.S_final + (seg_row * p.dout + n0 + n) * 128 + 64 * hh);
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        so[e] = make_float4(Sreg[4 * e], Sreg[4 * e + 1], Sreg[4 * e + 2], Sreg[4 * e + 3]);
+    }
   }
 
   tc_fence_before();
@@ -610,7 +660,7 @@ cudaError_t launch_fwd(const TcFwdParams& prm, const void* x, const void* g, cud
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const int grid = prm.B * prm.H * (prm.dout / 128);
+  const int grid = prm.B * prm.H * (prm.dout / 128) * prm.nseg;
   fwd_kernel<<<grid, NTHREADS, kSmemBytes, st>>>(mx, mg, my, ms, prm);
   count_launch();
   return cudaGetLastError();
