@@ -105,3 +105,21 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(tw, "LIB_PATH", str(tmp_path / "nope.so"))
     with pytest.raises(tw.GradlevError):
         tw.lib()
+
+
+def test_forward_workspace_grows_only_for_segmented_scans(L):
+    """Scans that fill the GPU run unsegmented and need only the status word;
+    few long scans are cut into segments, whose summaries live in the workspace."""
+    full = tw.gradlev_scan_workspace_bytes(8, 16, 4096, 128, 128, tw.BF16, 0)
+    few = tw.gradlev_scan_workspace_bytes(1, 2, 4096, 128, 128, tw.BF16, 0)
+    assert full == 256
+    # 2 scans -> segments; two fp32 [scan][seg][d_out][d_in] buffers at least
+    assert few >= 256 + 2 * 2 * 2 * 128 * 128 * 4
+    # the reverse scan's workspace covers its per-segment dW0 partials as well
+    bwd_few = tw.gradlev_scan_workspace_bytes(1, 2, 4096, 128, 128, tw.BF16, 1)
+    bwd_full = tw.gradlev_scan_workspace_bytes(8, 16, 4096, 128, 128, tw.BF16, 1)
+    assert bwd_few > tw.gradlev_scan_ckpt_bytes(1, 2, 4096, 128, 128, tw.BF16) + 2 * 128 * 128 * 4
+    assert bwd_full >= 256 + 8 * 16 * 128 * 128 * 4 + \
+        tw.gradlev_scan_ckpt_bytes(8, 16, 4096, 128, 128, tw.BF16)
+    # one chunk: nothing to split
+    assert tw.gradlev_scan_workspace_bytes(1, 1, 64, 128, 128, tw.BF16, 0) == 256
