@@ -31,14 +31,15 @@
 //   phase 2: V^T = Bm Q^T (M=64), RI^T = U^T Ar^T, DXa^T = W0^T U^T + X^T Z^T + Lam^T Gs^T
 //   phase 3: Lam += U^T Xg
 // where Ar, Z, Q^T, Bm are built by the math warps from K, Kug, KugT into the
-// shared memory that held S_in, Gs = diag(-eta del) G and Xg = diag(gam) X are
-// written in place once their unscaled uses are over. The fp32 adjoint Lam
+// shared memory that held S_in, Gs = diag(-eta del) G is written in place once
+// the unscaled G has been used, and Xg = diag(gam) X is a tile of its own that
+// warp 3 writes as soon as X arrives. The fp32 adjoint Lam
 // lives in TMEM: the math warps scale it by 2^{L_{C-1}} in place and the MMA
 // accumulates U^T Xg onto it; likewise del (.) R1^T and gam (.) DXb^T are
 // written back so that RI^T and DXa^T accumulate onto them (r^T and dx^T).
 //
 // Warp roles (20 warps): 0 TMA producer, 1 MMA issuer + TMEM owner, 2 gate
-// prep, 3 idle helper, 4..19 four math warpgroups (warpgroup w: tokens
+// prep, 3 writes Xg = diag(gam) X, 4..19 four math warpgroups (warpgroup w: tokens
 // [16w, 16w+16) of each chunk and state columns [32w, 32w+32)).
 
 #include <cuda.h>
@@ -106,6 +107,7 @@ struct Smem {
   uint8_t Sin[2 * BIG];       // [k-block][n rows x 128 B]; then Ar | Z | Q^T | Bm
   uint8_t W0[2 * BIG];        // [k-block][n rows x 128 B]
   uint8_t Lb[2 * BIG];        // bf16 Lam, [k-block][n rows x 128 B]
+  uint8_t Xg[2 * TILE];       // diag(gam) X for the Lam update, same layout as X
   GateSlot gates[GS];
   float redq[4][C], redp[4][C];
   float tv[4][C], t2v[4][C], t3v[4][C], hv[4][C];
@@ -116,18 +118,19 @@ struct Smem {
   uint64_t gfull[GS], gempty[GS];
   uint64_t sfull, sempty;
   uint64_t ccfull, b1full, b2full, b3full;
-  uint64_t m1a, m1done, m2done, xscaled, lbready, done;
+  uint64_t m1a, m1done, m2done, lscaled, xgready, xgfree, lbready, done;
   uint32_t tmem_base;
   int abort;
 };
 
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
+static_assert(kSmemBytes <= 227 * 1024, "over the 227 KB of shared memory a CTA may use");
 
 enum : uint32_t {
   W_TMA_XEMPTY = 0x001, W_TMA_SEMPTY, W_TMA_DRAIN,
   W_MMA_XFULL = 0x101, W_MMA_M2, W_MMA_SFULL, W_MMA_LB, W_MMA_M1, W_MMA_XS, W_MMA_DONE,
   W_MMA_M1A,
-  W_GATE_EMPTY = 0x201,
+  W_GATE_EMPTY = 0x201, W_XG_FULL, W_XG_GFULL, W_XG_FREE,
   W_M_GFULL = 0x401, W_M_CC, W_M_B1, W_M_B2, W_M_B3,
 };
 
@@ -219,7 +222,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(&sm.m1a, NMATH);
     mbar_init(&sm.m1done, NMATH);
     mbar_init(&sm.m2done, NMATH);
-    mbar_init(&sm.xscaled, NMATH);
+    mbar_init(&sm.lscaled, NMATH);
+    mbar_init(&sm.xgready, 1);
+    mbar_init(&sm.xgfree, 1);
     mbar_init(&sm.lbready, NMATH);
     mbar_init(&sm.done, 1);
     fence_mbar_init();
@@ -316,6 +321,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           xgu(it, sX, sG, sU);
           if (!mbar_wait(&sm.xfull[it % NS], (it / NS) & 1, wc, W_MMA_XFULL)) return false;
           if (!mbar_wait(&sm.sfull, it & 1, wc, W_MMA_SFULL)) return false;
+          // DXb^T and R1^T overwrite the dx^T and r^T accumulators of the previous chunk,
+          // which its output phase has read by m2done
+          if (it > 0 && !mbar_wait(&sm.m2done, (it - 1) & 1, wc, W_MMA_M2)) return false;
           tc_fence_after();
           for (int kk = 0; kk < 8; ++kk)  // DXb^T = S_in^T U^T
             umma_bf16(tbase + COL_D, sw128_desc(sS + kk * 2048, BIG, 1024),
@@ -377,30 +385,55 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                       sw128_desc(sS + CC_Z + kk * 32, 16, 1024), id_db, 1);
           umma_commit(&sm.b2full);
           umma_commit(&sm.sempty);
+          umma_commit(&sm.xempty[it % NS]);  // the last products reading X, G and U
           return true;
         };
         auto phase3 = [&](int it) -> bool {  // Lam += U^T Xg (Lam pre-scaled by the math warps)
           uint32_t sX, sG, sU;
           xgu(it, sX, sG, sU);
-          if (!mbar_wait(&sm.xscaled, it & 1, wc, W_MMA_XS)) return false;
+          if (!mbar_wait(&sm.lscaled, it & 1, wc, W_MMA_XS)) return false;
+          if (!mbar_wait(&sm.xgready, it & 1, wc, W_MMA_XS)) return false;
           tc_fence_after();
+          const uint32_t sXg = smem_u32(sm.Xg);
           for (int kk = 0; kk < 4; ++kk)
             umma_bf16(tbase + COL_L, sw128_desc(sU + kk * 2048, TILE, 1024),
-                      sw128_desc(sX + kk * 2048, TILE, 1024), id_w, 1);
+                      sw128_desc(sXg + kk * 2048, TILE, 1024), id_w, 1);
           umma_commit(&sm.b3full);
-          umma_commit(&sm.xempty[it % NS]);
+          umma_commit(&sm.xgfree);
           return true;
         };
-        auto chunk = [&](int it) -> bool {
-          return phase1b(it) && phase1a(it) && phase2a(it) && phase2b(it);
-        };
-        bool ok = chunk(0);
-        for (int it = 0; it < nch && ok; ++it) {
-          ok = phase3(it);
-          if (it + 1 < nch) ok = ok && chunk(it + 1);
-        }
+        // the Lam update is issued as soon as the math warps have scaled Lam, so that it
+        // runs while they build the chunk matrices
+        bool ok = true;
+        for (int it = 0; it < nch && ok; ++it)
+          ok = phase1b(it) && phase1a(it) && phase3(it) && phase2a(it) && phase2b(it);
         umma_commit(&sm.done);
         mbar_drain(&sm.done, 0, wc, W_MMA_DONE);
+      }
+    } else if (warp == 3) {
+      // ---------------------------------------------------------- Xg = diag(gam) X
+      bool ok = true;
+      for (int it = 0; it < nch && ok; ++it) {
+        const int st = it % NS, g = it % GS;
+        ok = ok && mbar_wait_warp(&sm.xfull[st], (it / NS) & 1, wc, W_XG_FULL);
+        ok = ok && mbar_wait_warp(&sm.gfull[g], (it / GS) & 1, wc, W_XG_GFULL);
+        ok = ok && (it == 0 || mbar_wait_warp(&sm.xgfree, (it - 1) & 1, wc, W_XG_FREE));
+        if (!ok) break;
+        const GateSlot& gs = sm.gates[g];
+        const uint32_t src = smem_u32(sm.X[st]), dst = smem_u32(sm.Xg);
+#pragma unroll 4
+        for (int idx = lane; idx < 2 * TILE / 16; idx += 32) {
+          const uint32_t off = (uint32_t)idx * 16;
+          const int sr = (off & (TILE - 1)) >> 7;  // token row
+          const __nv_bfloat162 f2 = __float2bfloat162_rn(gs.gam[sr]);
+          const uint32_t fv = *reinterpret_cast<const uint32_t*>(&f2);
+          const uint4 v = ld_shared_v4(src + off);
+          st_shared_v4(dst + off, hmul2_bf16(v.x, fv), hmul2_bf16(v.y, fv), hmul2_bf16(v.z, fv),
+                       hmul2_bf16(v.w, fv));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.xgready);
       }
     } else if (warp == 2) {
       // ---------------------------------------------------------- gate prep
@@ -535,6 +568,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
           if (lane == 0) sm.ered[warp - 4] = acc;
+          // the scaled Lam is in place: the Lam update of this chunk may be issued
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.lscaled);
         }
         // ---- q_j = g_j^T Lam x_j from R1^T; del (.) R1^T back
         {
@@ -832,20 +870,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int e = 0; e < 16; ++e)
             sts_u16(sw_elem(sLb + 2 * TILE + (n >> 6) * TILE, j0w + e, n & 63), vda[e]);
         }
-        // X <- diag(gam) X in place for Lam += U^T Xg (rows, packed bf16 multiplies)
-#pragma unroll
-        for (int k = 0; k < (2 * TILE / 16) / (32 * NMATH); ++k) {
-          const uint32_t off = (uint32_t)(mt + 32 * NMATH * k) * 16;
-          const int sr = (off & (TILE - 1)) >> 7;
-          const __nv_bfloat162 f2 = __float2bfloat162_rn(gs.gam[sr]);
-          const uint32_t fv = *reinterpret_cast<const uint32_t*>(&f2);
-          uint4 v = ld_shared_v4(sX + off);
-          st_shared_v4(sX + off, hmul2_bf16(v.x, fv), hmul2_bf16(v.y, fv), hmul2_bf16(v.z, fv),
-                       hmul2_bf16(v.w, fv));
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.xscaled);
       }
       named_sync_math();  // (B4) hv of all warpgroups and the dg / dx staging tiles written
       if (ok && mt == 0) {  // rows past T are clipped by the tensor maps

@@ -98,6 +98,7 @@ struct Smem {
 };
 
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
+static_assert(kSmemBytes <= 227 * 1024, "over the 227 KB of shared memory a CTA may use");
 
 // where-codes of the bounded waits (role << 8 | site)
 enum : uint32_t {
