@@ -27,16 +27,16 @@
 // Products (d on the 128 TMEM lanes, tokens on the columns; M=64 ones use the
 // two 16-lane halves of each TMEM sub-partition):
 //   phase 1: K = X X^T | Kug = U G^T (M=64), KugT = G U^T (M=64), dW0 += U^T X,
-//            DXb^T = S_in^T U^T, R1^T = Lam X^T
-//   phase 2: V^T = Bm Q^T (M=64), RI^T = U^T Ar^T, DXa^T = W0^T U^T + X^T Z^T + Lam^T Gs^T
+//            DXb = U S_in, R1 = X Lam^T (M=64, token-major)
+//   phase 2: V^T = Bm Q^T (M=64), r += Ar U, dx += U W0 + Z X + Gs Lam (token-major)
 //   phase 3: Lam += U^T Xg
 // where Ar, Z, Q^T, Bm are built by the math warps from K, Kug, KugT into the
 // shared memory that held S_in, Gs = diag(-eta del) G is written in place once
 // the unscaled G has been used, and Xg = diag(gam) X is a tile of its own that
 // warp 3 writes as soon as X arrives. The fp32 adjoint Lam
 // lives in TMEM: the math warps scale it by 2^{L_{C-1}} in place and the MMA
-// accumulates U^T Xg onto it; likewise del (.) R1^T and gam (.) DXb^T are
-// written back so that RI^T and DXa^T accumulate onto them (r^T and dx^T).
+// accumulates U^T Xg onto it; likewise the rows del_i R1_i and gam_i DXb_i are
+// written back so that the remaining terms accumulate onto them (r and dx).
 //
 // Warp roles (20 warps): 0 TMA producer, 1 MMA issuer + TMEM owner, 2 gate
 // prep, 3 writes Xg = diag(gam) X, 4..19 four math warpgroups (warpgroup w: tokens
@@ -74,8 +74,10 @@ constexpr int BIG = 128 * 128;  // [128 rows x 128 B] swizzled block
 // TMEM columns (512 allocated)
 constexpr uint32_t COL_KK = 0;    // K (lanes 0-15 of each sub-partition) | Kug (lanes 16-31)
 constexpr uint32_t COL_KT = 64;   // KugT (lanes 0-15) | V^T (lanes 16-31)
-constexpr uint32_t COL_R = 128;   // R1^T -> del (.) R1^T -> + RI^T = r^T
-constexpr uint32_t COL_D = 192;   // DXb^T -> gam (.) DXb^T -> + DXa^T = dx^T
+// r and dx are token-major M=64 products (token row i at lane 32 (i/16) + i%16):
+// r in the lower 16 lanes and dx in the upper 16 lanes of the same 128 columns, so
+// one load gives a warp the r and dx rows of the same tokens.
+constexpr uint32_t COL_RX = 128;  // R1 -> del (.) R1 -> + Ar U = r  |  DXb -> gam (.) DXb -> + ... = dx
 constexpr uint32_t COL_L = 256;   // Lam, fp32 (128 columns)
 constexpr uint32_t COL_W = 384;   // dW0 accumulator (128 columns)
 constexpr uint32_t LANE16 = 16u << 16;
@@ -301,8 +303,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (lane == 0) {
         const uint32_t id_cc = idesc_bf16(64, 64, false, false);      // X X^T, U G^T, G U^T
         const uint32_t id_w = idesc_bf16(128, 128, true, true);       // U^T X, U^T Xg
-        const uint32_t id_db = idesc_bf16(128, 64, true, false);      // S^T U^T, W0^T U^T, ...
-        const uint32_t id_r1 = idesc_bf16(128, 64, false, false);     // Lam X^T
+        const uint32_t id_tb = idesc_bf16(64, 128, false, true);      // U S_in, U W0, Ar U, ...
+        const uint32_t id_r1 = idesc_bf16(64, 128, false, false);     // X Lam^T
         const uint32_t id_v = idesc_bf16(64, 64, false, true);        // Bm Q^T
         const uint32_t sS = smem_u32(sm.Sin), sW0 = smem_u32(sm.W0), sL = smem_u32(sm.Lb);
         // Issue order per chunk: the products on the carried chain first (the Lam
@@ -316,23 +318,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           sG = smem_u32(sm.G[st]);
           sU = smem_u32(sm.U[st]);
         };
-        auto phase1b = [&](int it) -> bool {  // DXb^T, R1^T
+        auto phase1b = [&](int it) -> bool {  // DXb, R1
           uint32_t sX, sG, sU;
           xgu(it, sX, sG, sU);
           if (!mbar_wait(&sm.xfull[it % NS], (it / NS) & 1, wc, W_MMA_XFULL)) return false;
           if (!mbar_wait(&sm.sfull, it & 1, wc, W_MMA_SFULL)) return false;
-          // DXb^T and R1^T overwrite the dx^T and r^T accumulators of the previous chunk,
+          // DXb and R1 overwrite the dx and r accumulators of the previous chunk,
           // which its output phase has read by m2done
           if (it > 0 && !mbar_wait(&sm.m2done, (it - 1) & 1, wc, W_MMA_M2)) return false;
           tc_fence_after();
-          for (int kk = 0; kk < 8; ++kk)  // DXb^T = S_in^T U^T
-            umma_bf16(tbase + COL_D, sw128_desc(sS + kk * 2048, BIG, 1024),
-                      sw128_desc(sU + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024), id_db, kk > 0);
+          for (int kk = 0; kk < 8; ++kk)  // DXb = U S_in
+            umma_bf16(tbase + COL_RX + LANE16, sw128_desc(sU + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024),
+                      sw128_desc(sS + kk * 2048, BIG, 1024), id_tb, kk > 0);
           if (it > 0 && !mbar_wait(&sm.lbready, (it - 1) & 1, wc, W_MMA_LB)) return false;
           tc_fence_after();
-          for (int kk = 0; kk < 8; ++kk)  // R1^T = Lam X^T
-            umma_bf16(tbase + COL_R, sw128_desc(sL + (kk >> 2) * BIG + (kk & 3) * 32, 16, 1024),
-                      sw128_desc(sX + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024), id_r1, kk > 0);
+          for (int kk = 0; kk < 8; ++kk)  // R1 = X Lam^T
+            umma_bf16(tbase + COL_RX, sw128_desc(sX + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024),
+                      sw128_desc(sL + (kk >> 2) * BIG + (kk & 3) * 32, 16, 1024), id_r1, kk > 0);
           umma_commit(&sm.b1full);
           return true;
         };
@@ -356,17 +358,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                       sw128_desc(sX + kk * 2048, TILE, 1024), id_w, (it > 0 || kk > 0));
           return true;
         };
-        auto phase2a = [&](int it) -> bool {  // dx^T terms that need only Gs and gam (.) DXb^T
+        auto phase2a = [&](int it) -> bool {  // dx terms that need only Gs and gam (.) DXb
           uint32_t sX, sG, sU;
           xgu(it, sX, sG, sU);
           if (!mbar_wait(&sm.m1a, it & 1, wc, W_MMA_M1A)) return false;
           tc_fence_after();
-          for (int kk = 0; kk < 8; ++kk)  // dx^T = gam (.) DXb^T + W0^T U^T
-            umma_bf16(tbase + COL_D, sw128_desc(sW0 + kk * 2048, BIG, 1024),
-                      sw128_desc(sU + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024), id_db, 1);
-          for (int kk = 0; kk < 8; ++kk)  //      + Lam^T Gs^T
-            umma_bf16(tbase + COL_D, sw128_desc(sL + kk * 2048, BIG, 1024),
-                      sw128_desc(sG + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024), id_db, 1);
+          for (int kk = 0; kk < 8; ++kk)  // dx = gam (.) DXb + U W0
+            umma_bf16(tbase + COL_RX + LANE16, sw128_desc(sU + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024),
+                      sw128_desc(sW0 + kk * 2048, BIG, 1024), id_tb, 1);
+          for (int kk = 0; kk < 8; ++kk)  //      + Gs Lam
+            umma_bf16(tbase + COL_RX + LANE16, sw128_desc(sG + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024),
+                      sw128_desc(sL + kk * 2048, BIG, 1024), id_tb, 1);
           return true;
         };
         auto phase2b = [&](int it) -> bool {  // the products of the chunk matrices
@@ -377,12 +379,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int kk = 0; kk < 4; ++kk)  // V^T = Bm Q^T
             umma_bf16(tbase + COL_KT + LANE16, sw128_desc(sS + CC_BM + kk * 32, 16, 1024),
                       sw128_desc(sS + CC_QT + kk * 2048, TILE, 1024), id_v, kk > 0);
-          for (int kk = 0; kk < 4; ++kk)  // r^T = del (.) R1^T + U^T Ar^T
-            umma_bf16(tbase + COL_R, sw128_desc(sU + kk * 2048, TILE, 1024),
-                      sw128_desc(sS + CC_AR + kk * 32, 16, 1024), id_db, 1);
-          for (int kk = 0; kk < 4; ++kk)  // dx^T += X^T Z^T
-            umma_bf16(tbase + COL_D, sw128_desc(sX + kk * 2048, TILE, 1024),
-                      sw128_desc(sS + CC_Z + kk * 32, 16, 1024), id_db, 1);
+          for (int kk = 0; kk < 4; ++kk)  // r = del (.) R1 + Ar U
+            umma_bf16(tbase + COL_RX, sw128_desc(sS + CC_AR + kk * 32, 16, 1024),
+                      sw128_desc(sU + kk * 2048, TILE, 1024), id_tb, 1);
+          for (int kk = 0; kk < 4; ++kk)  // dx += Z X
+            umma_bf16(tbase + COL_RX + LANE16, sw128_desc(sS + CC_Z + kk * 32, 16, 1024),
+                      sw128_desc(sX + kk * 2048, TILE, 1024), id_tb, 1);
           umma_commit(&sm.b2full);
           umma_commit(&sm.sempty);
           umma_commit(&sm.xempty[it % NS]);  // the last products reading X, G and U
@@ -574,37 +576,34 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&sm.lscaled);
         }
-        // ---- q_j = g_j^T Lam x_j from R1^T; del (.) R1^T back
+        // ---- one pass for q and p: lanes 0-15 hold row i of R1 (q_i = g_i . R1_i,
+        //      then R1_i <- del_i R1_i), lanes 16-31 row i of DXb (p_i = x_i . DXb_i,
+        //      then DXb_i <- gam_i DXb_i); this warp covers columns [32 wg, 32 wg + 32)
         {
-          float vr[16], sv[16];
-          tmem_ld16(tbase + COL_R + lane_off + j0w, vr);
+          float v[32];
+          tmem_ld32(tbase + COL_RX + lane_off + 32 * wg, v);
           tmem_ld_wait();
+          const int i = ir;
+          const uint32_t row = (lo ? sG : sX) + (wg >> 1) * TILE;
+          float acc = 0.f;
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int j = j0w + e;
-            const float gv = lds_bf16(sw_elem(sG + (n >> 6) * TILE, j, n & 63));
-            sv[e] = gs.del[j] * vr[e];
-            vr[e] = gv * vr[e];
+          for (int cc = 0; cc < 4; ++cc) {
+            const uint4 sv = ld_shared_v4(row + sw128_off(i, 4 * (wg & 1) + cc));
+            acc = fmaf(v[8 * cc + 0], bf16_lo(sv.x), acc);
+            acc = fmaf(v[8 * cc + 1], bf16_hi(sv.x), acc);
+            acc = fmaf(v[8 * cc + 2], bf16_lo(sv.y), acc);
+            acc = fmaf(v[8 * cc + 3], bf16_hi(sv.y), acc);
+            acc = fmaf(v[8 * cc + 4], bf16_lo(sv.z), acc);
+            acc = fmaf(v[8 * cc + 5], bf16_hi(sv.z), acc);
+            acc = fmaf(v[8 * cc + 6], bf16_lo(sv.w), acc);
+            acc = fmaf(v[8 * cc + 7], bf16_hi(sv.w), acc);
           }
-          tmem_st16(tbase + COL_R + lane_off + j0w, sv);
-          const float r = reduce_scatter16(vr, lane);
-          if (!(lane & 1)) sm.redq[q][j0w + (lane >> 1)] = r;
-        }
-        // ---- p_s = x_s^T S_in^T u_s from DXb^T; gam (.) DXb^T back
-        {
-          float vd[16], sv[16];
-          tmem_ld16(tbase + COL_D + lane_off + j0w, vd);
-          tmem_ld_wait();
+          const float sc = lo ? gs.del[i] : gs.gam[i];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int s = j0w + e;
-            const float xv = lds_bf16(sw_elem(sX + (n >> 6) * TILE, s, n & 63));
-            sv[e] = gs.gam[s] * vd[e];
-            vd[e] = xv * vd[e];
-          }
-          tmem_st16(tbase + COL_D + lane_off + j0w, sv);
-          const float r = reduce_scatter16(vd, lane);
-          if (!(lane & 1)) sm.redp[q][j0w + (lane >> 1)] = r;
+          for (int e = 0; e < 32; ++e) v[e] *= sc;
+          tmem_st32(tbase + COL_RX + lane_off + 32 * wg, v);
+          if (lo) sm.redq[wg][i] = acc;
+          else sm.redp[wg][i] = acc;
         }
         tmem_st_wait();
       }
@@ -623,7 +622,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           st_shared_v4(sG + off, hmul2_bf16(v.x, fv), hmul2_bf16(v.y, fv), hmul2_bf16(v.z, fv),
                        hmul2_bf16(v.w, fv));
         }
-        // Gs and gam (.) DXb^T are in place (the TMEM writes finished before B1)
+        // Gs and gam (.) DXb are in place (the TMEM writes finished before B1)
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
@@ -802,14 +801,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (t0 + j < T) p.d_eta[tokbase + j] = p.accumulate ? p.d_eta[tokbase + j] + deta : deta;
       }
 
-      // ---- phase 2: dg from r^T, dx from dx^T, and the V part of dalpha
+      // ---- phase 2: dg from r, dx from dx, and the V part of dalpha
       ok = ok && mbar_wait_warp(&sm.b2full, it & 1, wc, W_M_B2);
       tc_fence_after();
       if (ok) {
         {
-          float vv[16], vri[16];
+          float vv[16];
           tmem_ld16(tbase + COL_KT + lane_off + j0w, vv);
-          tmem_ld16(tbase + COL_R + lane_off + j0w, vri);
           tmem_ld_wait();
           if (!lo) {
             const int i = ir;
@@ -845,30 +843,44 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             sm.hv[wg][i] = hpart;
           }
-          // dg^T[n][i] = -eta_i r^T[n][i] -> staging tile [i rows][n] (the bf16 Lam tile is
-          // free until the Lam update: MMA2 has read it)
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int i = j0w + e;
-            sts_u16(sw_elem(sLb + (n >> 6) * TILE, i, n & 63), -gs.eta[i] * vri[e]);
-          }
         }
         {
-          float vda[16];
-          tmem_ld16(tbase + COL_D + lane_off + j0w, vda);
+          // dg_i = -eta_i r_i (lanes 0-15) and dx_i (lanes 16-31) -> staging tiles [i rows][d]
+          // in the bf16 Lam tile, free until the Lam update: the products have read it
+          float v[32];
+          tmem_ld32(tbase + COL_RX + lane_off + 32 * wg, v);
           tmem_ld_wait();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sm.m2done);
-          if (p.accumulate) {  // add the dx of the slices already done
-            const __nv_bfloat16* dxo = p.dx + tokbase * 128 + n;
+          const int i = ir;
+          if (lo) {
+            const float ne = -gs.eta[i];
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              if (t0 + j0w + e < T) vda[e] += __bfloat162float(dxo[(size_t)(j0w + e) * 128]);
+            for (int e = 0; e < 32; ++e) v[e] *= ne;
+          } else if (p.accumulate && t0 + i < T) {  // add the dx of the slices already done
+            const uint4* dxo = reinterpret_cast<const uint4*>(p.dx + (tokbase + i) * 128 + 32 * wg);
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              const uint4 o = dxo[cc];
+              v[8 * cc + 0] += bf16_lo(o.x);
+              v[8 * cc + 1] += bf16_hi(o.x);
+              v[8 * cc + 2] += bf16_lo(o.y);
+              v[8 * cc + 3] += bf16_hi(o.y);
+              v[8 * cc + 4] += bf16_lo(o.z);
+              v[8 * cc + 5] += bf16_hi(o.z);
+              v[8 * cc + 6] += bf16_lo(o.w);
+              v[8 * cc + 7] += bf16_hi(o.w);
+            }
           }
+          const uint32_t trow = sLb + (lo ? 0 : 2 * TILE) + (wg >> 1) * TILE;
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            sts_u16(sw_elem(sLb + 2 * TILE + (n >> 6) * TILE, j0w + e, n & 63), vda[e]);
+          for (int cc = 0; cc < 4; ++cc)
+            st_shared_v4(trow + sw128_off(i, 4 * (wg & 1) + cc), pack_bf16(v[8 * cc], v[8 * cc + 1]),
+                         pack_bf16(v[8 * cc + 2], v[8 * cc + 3]),
+                         pack_bf16(v[8 * cc + 4], v[8 * cc + 5]),
+                         pack_bf16(v[8 * cc + 6], v[8 * cc + 7]));
+          fence_proxy_async_smem();
         }
       }
       named_sync_math();  // (B4) hv of all warpgroups and the dg / dx staging tiles written
