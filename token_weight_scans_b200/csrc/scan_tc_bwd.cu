@@ -540,11 +540,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       ok = ok && mbar_wait_warp(&sm.gfull[g], (it / GS) & 1, wc, W_M_GFULL);
       ok = ok && mbar_wait_warp(&sm.xfull[st], (it / NS) & 1, wc, W_M_GFULL);
       ok = ok && mbar_wait_warp(&sm.sfull, it & 1, wc, W_M_GFULL);
-      ok = ok && mbar_wait_warp(&sm.b1full, it & 1, wc, W_M_B1);
       tc_fence_after();
 
       if (ok) {
-        // ---- <Lam_end, S_in>, then Lam <- 2^{L_{C-1}} Lam in place
+        // ---- <Lam_end, S_in>, then Lam <- 2^{L_{C-1}} Lam in place (Lam_end is complete
+        //      since the previous chunk's b3full; this overlaps the R1 and DXb products)
         {
           const float gC = gs.gC;
           const uint32_t row = sS + (wg >> 1) * BIG;
@@ -576,6 +576,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&sm.lscaled);
         }
+      }
+      ok = ok && mbar_wait_warp(&sm.b1full, it & 1, wc, W_M_B1);
+      tc_fence_after();
+      if (ok) {
         // ---- one pass for q and p: lanes 0-15 hold row i of R1 (q_i = g_i . R1_i,
         //      then R1_i <- del_i R1_i), lanes 16-31 row i of DXb (p_i = x_i . DXb_i,
         //      then DXb_i <- gam_i DXb_i); this warp covers columns [32 wg, 32 wg + 32)
@@ -793,13 +797,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.m1done);
       }
-      named_sync_math();  // (B3) t complete
-      if (ok && mt < C) {
-        const int j = mt;
-        const float deta =
-            -(gs.del[j] * sm.qv[j] + sm.tv[0][j] + sm.tv[1][j] + sm.tv[2][j] + sm.tv[3][j]);
-        if (t0 + j < T) p.d_eta[tokbase + j] = p.accumulate ? p.d_eta[tokbase + j] + deta : deta;
-      }
 
       // ---- phase 2: dg from r, dx from dx, and the V part of dalpha
       ok = ok && mbar_wait_warp(&sm.b2full, it & 1, wc, W_M_B2);
@@ -883,7 +880,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           fence_proxy_async_smem();
         }
       }
-      named_sync_math();  // (B4) hv of all warpgroups and the dg / dx staging tiles written
+      named_sync_math();  // (B4) t, hv of all warpgroups and the dg / dx staging tiles written
       if (ok && mt == 0) {  // rows past T are clipped by the tensor maps
         tma_store_3d(&tmDG, sm.Lb, p.n0, t0, bh);
         tma_store_3d(&tmDG, sm.Lb + TILE, p.n0 + 64, t0, bh);
@@ -891,8 +888,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tma_store_3d(&tmDX, sm.Lb + 3 * TILE, 64, t0, bh);
         tma_store_commit();
       }
-      if (ok && mt < C) {
-        const int i = mt;
+      if (ok && mt < C) {  // d_eta_j = -(del_j q_j + t_j)
+        const int j = mt;
+        const float deta =
+            -(gs.del[j] * sm.qv[j] + sm.tv[0][j] + sm.tv[1][j] + sm.tv[2][j] + sm.tv[3][j]);
+        if (t0 + j < T) p.d_eta[tokbase + j] = p.accumulate ? p.d_eta[tokbase + j] + deta : deta;
+      }
+      if (ok && mt >= C && mt < 2 * C) {
+        const int i = mt - C;
         const float t2 = sm.t2v[0][i] + sm.t2v[1][i] + sm.t2v[2][i] + sm.t2v[3][i];
         const float t3 = sm.t3v[0][i] + sm.t3v[1][i] + sm.t3v[2][i] + sm.t3v[3][i];
         const float h4 = sm.hv[0][i] + sm.hv[1][i] + sm.hv[2][i] + sm.hv[3][i];
@@ -930,7 +933,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           mbar_arrive(&sm.gempty[g]);
         }
       }
-      named_sync_math();  // (B5) per-chunk scratch consumed before the next chunk writes it
+      // No barrier is needed here: every read of this chunk's scratch (partial sums,
+      // gates) happened before B4b, and the next chunk's products wait for lbready
+      // from every math warp.
     }
 
     if (mt == 0) tma_store_wait_all();
