@@ -327,14 +327,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           // which its output phase has read by m2done
           if (it > 0 && !mbar_wait(&sm.m2done, (it - 1) & 1, wc, W_MMA_M2)) return false;
           tc_fence_after();
+          #pragma unroll
           for (int kk = 0; kk < 8; ++kk)  // DXb = U S_in
-            umma_bf16(tbase + COL_RX + LANE16, sw128_desc(sU + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024),
-                      sw128_desc(sS + kk * 2048, BIG, 1024), id_tb, kk > 0);
+            umma_bf16(tbase + COL_RX + LANE16, desc_at(sw128_desc(sU, 16, 1024), (kk >> 2) * TILE + (kk & 3) * 32),
+                      desc_at(sw128_desc(sS, BIG, 1024), kk * 2048), id_tb, kk > 0);
           if (it > 0 && !mbar_wait(&sm.lbready, (it - 1) & 1, wc, W_MMA_LB)) return false;
           tc_fence_after();
+          #pragma unroll
           for (int kk = 0; kk < 8; ++kk)  // R1 = X Lam^T
-            umma_bf16(tbase + COL_RX, sw128_desc(sX + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024),
-                      sw128_desc(sL + (kk >> 2) * BIG + (kk & 3) * 32, 16, 1024), id_r1, kk > 0);
+            umma_bf16(tbase + COL_RX, desc_at(sw128_desc(sX, 16, 1024), (kk >> 2) * TILE + (kk & 3) * 32),
+                      desc_at(sw128_desc(sL, 16, 1024), (kk >> 2) * BIG + (kk & 3) * 32), id_r1, kk > 0);
           umma_commit(&sm.b1full);
           return true;
         };
@@ -343,19 +345,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           xgu(it, sX, sG, sU);
           if (it > 0 && !mbar_wait(&sm.m2done, (it - 1) & 1, wc, W_MMA_M2)) return false;
           tc_fence_after();
+          #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {  // K = X X^T, Kug = U G^T, KugT = G U^T
             const uint32_t off = (kk >> 2) * TILE + (kk & 3) * 32;
-            const uint64_t dX = sw128_desc(sX + off, 16, 1024);
-            const uint64_t dG = sw128_desc(sG + off, 16, 1024);
-            const uint64_t dU = sw128_desc(sU + off, 16, 1024);
+            const uint64_t dX = desc_at(sw128_desc(sX, 16, 1024), off);
+            const uint64_t dG = desc_at(sw128_desc(sG, 16, 1024), off);
+            const uint64_t dU = desc_at(sw128_desc(sU, 16, 1024), off);
             umma_bf16(tbase + COL_KK, dX, dX, id_cc, kk > 0);
             umma_bf16(tbase + COL_KK + LANE16, dU, dG, id_cc, kk > 0);
             umma_bf16(tbase + COL_KT, dG, dU, id_cc, kk > 0);
           }
           umma_commit(&sm.ccfull);
+          #pragma unroll
           for (int kk = 0; kk < 4; ++kk)  // dW0 += U^T X
-            umma_bf16(tbase + COL_W, sw128_desc(sU + kk * 2048, TILE, 1024),
-                      sw128_desc(sX + kk * 2048, TILE, 1024), id_w, (it > 0 || kk > 0));
+            umma_bf16(tbase + COL_W, desc_at(sw128_desc(sU, TILE, 1024), kk * 2048),
+                      desc_at(sw128_desc(sX, TILE, 1024), kk * 2048), id_w, (it > 0 || kk > 0));
           return true;
         };
         auto phase2a = [&](int it) -> bool {  // dx terms that need only Gs and gam (.) DXb
@@ -363,12 +367,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           xgu(it, sX, sG, sU);
           if (!mbar_wait(&sm.m1a, it & 1, wc, W_MMA_M1A)) return false;
           tc_fence_after();
+          #pragma unroll
           for (int kk = 0; kk < 8; ++kk)  // dx = gam (.) DXb + U W0
-            umma_bf16(tbase + COL_RX + LANE16, sw128_desc(sU + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024),
-                      sw128_desc(sW0 + kk * 2048, BIG, 1024), id_tb, 1);
+            umma_bf16(tbase + COL_RX + LANE16, desc_at(sw128_desc(sU, 16, 1024), (kk >> 2) * TILE + (kk & 3) * 32),
+                      desc_at(sw128_desc(sW0, BIG, 1024), kk * 2048), id_tb, 1);
+          #pragma unroll
           for (int kk = 0; kk < 8; ++kk)  //      + Gs Lam
-            umma_bf16(tbase + COL_RX + LANE16, sw128_desc(sG + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024),
-                      sw128_desc(sL + kk * 2048, BIG, 1024), id_tb, 1);
+            umma_bf16(tbase + COL_RX + LANE16, desc_at(sw128_desc(sG, 16, 1024), (kk >> 2) * TILE + (kk & 3) * 32),
+                      desc_at(sw128_desc(sL, BIG, 1024), kk * 2048), id_tb, 1);
           return true;
         };
         auto phase2b = [&](int it) -> bool {  // the products of the chunk matrices
@@ -376,15 +382,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           xgu(it, sX, sG, sU);
           if (!mbar_wait(&sm.m1done, it & 1, wc, W_MMA_M1)) return false;
           tc_fence_after();
+          #pragma unroll
           for (int kk = 0; kk < 4; ++kk)  // V^T = Bm Q^T
-            umma_bf16(tbase + COL_KT + LANE16, sw128_desc(sS + CC_BM + kk * 32, 16, 1024),
-                      sw128_desc(sS + CC_QT + kk * 2048, TILE, 1024), id_v, kk > 0);
+            umma_bf16(tbase + COL_KT + LANE16, desc_at(sw128_desc(sS, 16, 1024), CC_BM + kk * 32),
+                      desc_at(sw128_desc(sS, TILE, 1024), CC_QT + kk * 2048), id_v, kk > 0);
+          #pragma unroll
           for (int kk = 0; kk < 4; ++kk)  // r = del (.) R1 + Ar U
-            umma_bf16(tbase + COL_RX, sw128_desc(sS + CC_AR + kk * 32, 16, 1024),
-                      sw128_desc(sU + kk * 2048, TILE, 1024), id_tb, 1);
+            umma_bf16(tbase + COL_RX, desc_at(sw128_desc(sS, 16, 1024), CC_AR + kk * 32),
+                      desc_at(sw128_desc(sU, TILE, 1024), kk * 2048), id_tb, 1);
+          #pragma unroll
           for (int kk = 0; kk < 4; ++kk)  // dx += Z X
-            umma_bf16(tbase + COL_RX + LANE16, sw128_desc(sS + CC_Z + kk * 32, 16, 1024),
-                      sw128_desc(sX + kk * 2048, TILE, 1024), id_tb, 1);
+            umma_bf16(tbase + COL_RX + LANE16, desc_at(sw128_desc(sS, 16, 1024), CC_Z + kk * 32),
+                      desc_at(sw128_desc(sX, TILE, 1024), kk * 2048), id_tb, 1);
           umma_commit(&sm.b2full);
           umma_commit(&sm.sempty);
           umma_commit(&sm.xempty[it % NS]);  // the last products reading X, G and U
@@ -397,9 +406,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (!mbar_wait(&sm.xgready, it & 1, wc, W_MMA_XS)) return false;
           tc_fence_after();
           const uint32_t sXg = smem_u32(sm.Xg);
+          #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            umma_bf16(tbase + COL_L, sw128_desc(sU + kk * 2048, TILE, 1024),
-                      sw128_desc(sXg + kk * 2048, TILE, 1024), id_w, 1);
+            umma_bf16(tbase + COL_L, desc_at(sw128_desc(sU, TILE, 1024), kk * 2048),
+                      desc_at(sw128_desc(sXg, TILE, 1024), kk * 2048), id_w, 1);
           umma_commit(&sm.b3full);
           umma_commit(&sm.xgfree);
           return true;

@@ -244,10 +244,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (!mbar_wait(&sm.kfree[b], ((c >> 1) & 1) ^ 1, wc, W_MMA_KFREE)) break;
           tc_fence_after();
           // K = X X^T
+          #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = (kk >> 2) * TILE + (kk & 3) * 32;
-            umma_bf16(tbase + (b ? COL_K1 : COL_K0), sw128_desc(sX + off, 16, 1024),
-                      sw128_desc(sX + off, 16, 1024), id_k, kk > 0);
+            umma_bf16(tbase + (b ? COL_K1 : COL_K0), desc_at(sw128_desc(sX, 16, 1024), off),
+                      desc_at(sw128_desc(sX, 16, 1024), off), id_k, kk > 0);
           }
           if (!(p.inject == 1 && c == 1)) umma_commit(&sm.kfull[b]);
         }
@@ -255,9 +256,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (!mbar_wait(&sm.xhready[b], (c >> 1) & 1, wc, W_MMA_XREADY)) break;
         if (c > 0 && !mbar_wait(&sm.dsfree, (c - 1) & 1, wc, W_MMA_DSFREE)) break;
         tc_fence_after();
+        #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_bf16(tbase + COL_DS, sw128_desc(sG + kk * 2048, TILE, 1024),
-                    sw128_desc(sXh + kk * 2048, TILE, 1024), id_ds, kk > 0);
+          umma_bf16(tbase + COL_DS, desc_at(sw128_desc(sG, TILE, 1024), kk * 2048),
+                    desc_at(sw128_desc(sXh, TILE, 1024), kk * 2048), id_ds, kk > 0);
         umma_commit(&sm.dsfull);
         umma_commit(&sm.xhfree[b]);
         if (p.summary) {  // state carry only: the stage is free once dS has read it
@@ -268,19 +270,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t tY1 = tbase + COL_Y + 128 * b, tY2 = tY1 + LANE16;
         if (!mbar_wait(&sm.yfree[b], ((c >> 1) & 1) ^ 1, wc, W_MMA_YFREE)) break;
         tc_fence_after();
+        #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t aoff = (kk >> 2) * TILE + (kk & 3) * 32;
           const uint32_t boff = (kk >> 2) * BIG + (kk & 3) * 32;
-          umma_bf16(tY1, sw128_desc(sX + aoff, 16, 1024), sw128_desc(sW0 + boff, 16, 1024), id_y,
+          umma_bf16(tY1, desc_at(sw128_desc(sX, 16, 1024), aoff), desc_at(sw128_desc(sW0, 16, 1024), boff), id_y,
                     kk > 0);
         }
         // Y2 = X S^T (state buffer c & 1, written by the state update of chunk c - 1)
         if (c > 0 && !mbar_wait(&sm.sready[b], ((c - 1) >> 1) & 1, wc, W_MMA_SREADY)) break;
         tc_fence_after();
+        #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t aoff = (kk >> 2) * TILE + (kk & 3) * 32;
           const uint32_t boff = (kk >> 2) * BIG + (kk & 3) * 32;
-          umma_bf16(tY2, sw128_desc(sX + aoff, 16, 1024), sw128_desc(sS + boff, 16, 1024), id_y,
+          umma_bf16(tY2, desc_at(sw128_desc(sX, 16, 1024), aoff), desc_at(sw128_desc(sS, 16, 1024), boff), id_y,
                     kk > 0);
         }
         umma_commit(&sm.sfree[b]);
@@ -288,9 +292,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // of chunk c + 1 has completed, which is committed after these.
         if (!mbar_wait(&sm.pready, c & 1, wc, W_MMA_PREADY)) break;
         tc_fence_after();
+        #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_bf16(tY1, sw128_desc(sP + kk * 32, 16, 1024),
-                    sw128_desc(sG + kk * 2048, TILE, 1024), id_pg, 1);
+          umma_bf16(tY1, desc_at(sw128_desc(sP, 16, 1024), kk * 32),
+                    desc_at(sw128_desc(sG, TILE, 1024), kk * 2048), id_pg, 1);
         umma_commit(&sm.yfull[b]);
         umma_commit(&sm.empty[s]);
       }

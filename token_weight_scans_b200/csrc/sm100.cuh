@@ -263,6 +263,15 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uin
   return d;
 }
 
+// The descriptor of the tile `byte_off` bytes past the one `base` describes: the
+// start address is the low 14-bit field (address >> 4), and shared-memory
+// addresses stay below 256 KB, so the offset adds without a carry out of the field.
+// With the base hoisted out of an unrolled K loop, each MMA's descriptors cost one
+// add apiece.
+__device__ __forceinline__ uint64_t desc_at(uint64_t base, uint32_t byte_off) {
+  return base + (uint64_t)(byte_off >> 4);
+}
+
 // Instruction descriptor of tcgen05.mma kind::f16: bf16 A and B, fp32 accumulator.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
   return (1u << 4)                      // D format: f32
