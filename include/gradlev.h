@@ -90,15 +90,19 @@ GRADLEV_API gradlev_status gradlev_scan_supported(int B, int H, int T, int d_in,
  * call needs for this shape; 0 if the shape is unsupported. The workspace is
  * scratch: its contents on entry do not matter; on return its first 16 bytes
  * hold the device status word read by gradlev_device_status() and the rest is
- * unspecified. It is never smaller than 256 bytes. */
+ * unspecified. It is never smaller than 256 bytes. It grows with the shape: the
+ * backward keeps per-scan dW0 partials there, and calls whose scans are too few
+ * to fill the GPU cut each scan into segments whose fp32 summaries live there
+ * (a few 64 KB matrices per scan and segment). */
 GRADLEV_API size_t gradlev_scan_workspace_bytes(int B, int H, int T, int d_in, int d_out,
                                     gradlev_dtype dt, int is_bwd);
 
 /* Bytes of the optional state-checkpoint buffer that gradlev_scan_fwd can fill
  * and gradlev_scan_bwd can consume for the same shape and dtype; 0 if
- * unsupported. Its contents are implementation-defined (the float32 scan state
- * at fixed token intervals) and valid only for the inputs of the forward call
- * that wrote them. */
+ * unsupported. Its contents are implementation-defined (the scan state at fixed
+ * token intervals: bfloat16 every 64 tokens for bf16 I/O with d_in = 128 and
+ * d_out in {128, 256}, float32 every 32 tokens otherwise) and valid only for the
+ * inputs of the forward call that wrote them. */
 GRADLEV_API size_t gradlev_scan_ckpt_bytes(int B, int H, int T, int d_in, int d_out, gradlev_dtype dt);
 
 /* Forward scan: y_t = (W0 + S_t) x_t for every (b, h, t).
