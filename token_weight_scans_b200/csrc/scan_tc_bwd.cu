@@ -115,12 +115,13 @@ struct Smem {
   float tv[4][C], t2v[4][C], t3v[4][C], hv[4][C];
   alignas(16) float qv[C];
   alignas(16) float pv[C];
-  alignas(16) float ered[NMATH];
+  alignas(16) float ered[2][NMATH];  // by chunk parity: the d_alpha of chunk it reads its
+                                     // slots while faster warps start chunk it + 1
   uint64_t xfull[NS], xempty[NS];
   uint64_t gfull[GS], gempty[GS];
-  uint64_t sfull, sempty;
+  uint64_t sfull, sempty;  // S_in tile loaded | S_in / chunk-matrix tile read by its last products
   uint64_t ccfull, b1full, b2full, b3full;
-  uint64_t m1a, m1done, m2done, lscaled, xgready, xgfree, lbready, done;
+  uint64_t m1a, m1done, m2done, lscaled, xgready, xgfree, lbfree, lbready, done;
   uint32_t tmem_base;
   int abort;
 };
@@ -209,7 +210,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     sm.abort = 0;
     for (int s = 0; s < NS; ++s) {
       mbar_init(&sm.xfull[s], 1);
-      mbar_init(&sm.xempty[s], 1);
+      mbar_init(&sm.xempty[s], 2);  // the last products on X, G, U + the dg / dx stores' read
     }
     for (int g = 0; g < GS; ++g) {
       mbar_init(&sm.gfull[g], 32);
@@ -217,6 +218,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     mbar_init(&sm.sfull, 1);
     mbar_init(&sm.sempty, 1);
+    mbar_init(&sm.lbfree, 1);
     mbar_init(&sm.ccfull, 1);
     mbar_init(&sm.b1full, 1);
     mbar_init(&sm.b2full, 1);
@@ -288,6 +290,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tma_load_3d(sm.U[st], &tmU, &sm.xfull[st], p.n0, c * C, bh);
           tma_load_3d(sm.U[st] + TILE, &tmU, &sm.xfull[st], p.n0 + 64, c * C, bh);
           xi = it + 1;
+          // the S_in tile doubles as the chunk-matrix scratch: load once the previous
+          // chunk's products on the chunk matrices have completed
           if (!mbar_wait(&sm.sempty, (it & 1) ^ 1, wc, W_TMA_SEMPTY)) break;
           mbar_arrive_expect_tx(&sm.sfull, 2 * BIG);
           tma_load_3d(sm.Sin, &tmS, &sm.sfull, 0, p.n0, bh * nch_all + c);
@@ -307,44 +311,47 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t id_r1 = idesc_bf16(64, 128, false, false);     // X Lam^T
         const uint32_t id_v = idesc_bf16(64, 64, false, true);        // Bm Q^T
         const uint32_t sS = smem_u32(sm.Sin), sW0 = smem_u32(sm.W0), sL = smem_u32(sm.Lb);
-        // Issue order per chunk: the products on the carried chain first (the Lam
-        // update of the previous chunk, then DXb and R1 = Lam X^T of this one), then
-        // the Gram products and dW0, which the tensor pipe works through while the
-        // math warps use R1 and DXb; the dx terms that need only scaled G and DXb
-        // next; last the three products that need the chunk matrices.
+        // Issue order per chunk: R1 = X Lam^T and the Gram products and dW0 as soon as
+        // the previous chunk's output phase has read its accumulators, DXb when S_in
+        // lands, the Lam update once the math warps have scaled Lam, the dx terms that
+        // need only scaled G and DXb, and last the three products that need the chunk
+        // matrices.
         auto xgu = [&](int it, uint32_t& sX, uint32_t& sG, uint32_t& sU) {
           const int st = it % NS;
           sX = smem_u32(sm.X[st]);
           sG = smem_u32(sm.G[st]);
           sU = smem_u32(sm.U[st]);
         };
-        auto phase1b = [&](int it) -> bool {  // DXb, R1
+        auto phase1r = [&](int it) -> bool {  // R1 = X Lam^T
           uint32_t sX, sG, sU;
           xgu(it, sX, sG, sU);
           if (!mbar_wait(&sm.xfull[it % NS], (it / NS) & 1, wc, W_MMA_XFULL)) return false;
-          if (!mbar_wait(&sm.sfull, it & 1, wc, W_MMA_SFULL)) return false;
-          // DXb and R1 overwrite the dx and r accumulators of the previous chunk,
-          // which its output phase has read by m2done
+          // R1 and DXb overwrite the r and dx accumulators of the previous chunk, which
+          // its output phase has read by m2done
           if (it > 0 && !mbar_wait(&sm.m2done, (it - 1) & 1, wc, W_MMA_M2)) return false;
-          tc_fence_after();
-          #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)  // DXb = U S_in
-            umma_bf16(tbase + COL_RX + LANE16, desc_at(sw128_desc(sU, 16, 1024), (kk >> 2) * TILE + (kk & 3) * 32),
-                      desc_at(sw128_desc(sS, BIG, 1024), kk * 2048), id_tb, kk > 0);
           if (it > 0 && !mbar_wait(&sm.lbready, (it - 1) & 1, wc, W_MMA_LB)) return false;
           tc_fence_after();
           #pragma unroll
           for (int kk = 0; kk < 8; ++kk)  // R1 = X Lam^T
             umma_bf16(tbase + COL_RX, desc_at(sw128_desc(sX, 16, 1024), (kk >> 2) * TILE + (kk & 3) * 32),
                       desc_at(sw128_desc(sL, 16, 1024), (kk >> 2) * BIG + (kk & 3) * 32), id_r1, kk > 0);
-          umma_commit(&sm.b1full);
           return true;
         };
-        auto phase1a = [&](int it) -> bool {  // K, Kug, KugT, dW0
+        auto phase1b = [&](int it) -> bool {  // DXb = U S_in, once S_in has landed
           uint32_t sX, sG, sU;
           xgu(it, sX, sG, sU);
-          if (it > 0 && !mbar_wait(&sm.m2done, (it - 1) & 1, wc, W_MMA_M2)) return false;
+          if (!mbar_wait(&sm.sfull, it & 1, wc, W_MMA_SFULL)) return false;
           tc_fence_after();
+          #pragma unroll
+          for (int kk = 0; kk < 8; ++kk)  // DXb = U S_in
+            umma_bf16(tbase + COL_RX + LANE16, desc_at(sw128_desc(sU, 16, 1024), (kk >> 2) * TILE + (kk & 3) * 32),
+                      desc_at(sw128_desc(sS, BIG, 1024), kk * 2048), id_tb, kk > 0);
+          umma_commit(&sm.b1full);  // R1, the Gram products, dW0 and DXb
+          return true;
+        };
+        auto phase1a = [&](int it) -> bool {  // K, Kug, KugT, dW0 (after phase1r's waits)
+          uint32_t sX, sG, sU;
+          xgu(it, sX, sG, sU);
           #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {  // K = X X^T, Kug = U G^T, KugT = G U^T
             const uint32_t off = (kk >> 2) * TILE + (kk & 3) * 32;
@@ -375,6 +382,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int kk = 0; kk < 8; ++kk)  //      + Gs Lam
             umma_bf16(tbase + COL_RX + LANE16, desc_at(sw128_desc(sG, 16, 1024), (kk >> 2) * TILE + (kk & 3) * 32),
                       desc_at(sw128_desc(sL, BIG, 1024), kk * 2048), id_tb, 1);
+          umma_commit(&sm.lbfree);  // the last product reading the bf16 Lam of this chunk
           return true;
         };
         auto phase2b = [&](int it) -> bool {  // the products of the chunk matrices
@@ -395,7 +403,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             umma_bf16(tbase + COL_RX + LANE16, desc_at(sw128_desc(sS, 16, 1024), CC_Z + kk * 32),
                       desc_at(sw128_desc(sX, TILE, 1024), kk * 2048), id_tb, 1);
           umma_commit(&sm.b2full);
-          umma_commit(&sm.sempty);
+          umma_commit(&sm.sempty);           // the last products reading S_in / the chunk matrices
           umma_commit(&sm.xempty[it % NS]);  // the last products reading X, G and U
           return true;
         };
@@ -415,10 +423,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           return true;
         };
         // the Lam update is issued as soon as the math warps have scaled Lam, so that it
-        // runs while they build the chunk matrices
+        // runs while they build the chunk matrices. R1 and the Gram products need only
+        // the previous chunk's output phase and the new Lam, so they run while the next
+        // S_in tile is still being loaded; DXb follows when it lands.
         bool ok = true;
         for (int it = 0; it < nch && ok; ++it)
-          ok = phase1b(it) && phase1a(it) && phase3(it) && phase2a(it) && phase2b(it);
+          ok = phase1r(it) && phase1a(it) && phase1b(it) && phase3(it) && phase2a(it) &&
+               phase2b(it);
         umma_commit(&sm.done);
         mbar_drain(&sm.done, 0, wc, W_MMA_DONE);
       }
@@ -579,7 +590,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tmem_st32(tL, v);
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-          if (lane == 0) sm.ered[warp - 4] = acc;
+          if (lane == 0) sm.ered[it & 1][warp - 4] = acc;
           // the scaled Lam is in place: the Lam update of this chunk may be issued
           tmem_st_wait();
           tc_fence_before();
@@ -808,6 +819,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (lane == 0) mbar_arrive(&sm.m1done);
       }
 
+      // ---- bf16 copy of the updated Lam for the next chunk's products, as soon as the Lam
+      //      update is done and this chunk's last reader of the bf16 Lam (Gs Lam) has run
+      ok = ok && mbar_wait_warp(&sm.b3full, it & 1, wc, W_M_B3);
+      ok = ok && mbar_wait_warp(&sm.lbfree, it & 1, wc, W_M_B3);
+      tc_fence_after();
+      if (ok && it + 1 < nch) {
+        const uint32_t lrow = sLb + (wg >> 1) * BIG;
+        float v[32];
+        tmem_ld32(tL, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+          st_shared_v4(lrow + sw128_off(n, 4 * (wg & 1) + cc), pack_bf16(v[8 * cc], v[8 * cc + 1]),
+                       pack_bf16(v[8 * cc + 2], v[8 * cc + 3]),
+                       pack_bf16(v[8 * cc + 4], v[8 * cc + 5]),
+                       pack_bf16(v[8 * cc + 6], v[8 * cc + 7]));
+        tc_fence_before();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.lbready);
+      }
+
       // ---- phase 2: dg from r, dx from dx, and the V part of dalpha
       ok = ok && mbar_wait_warp(&sm.b2full, it & 1, wc, W_M_B2);
       tc_fence_after();
@@ -853,7 +886,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         {
           // dg_i = -eta_i r_i (lanes 0-15) and dx_i (lanes 16-31) -> staging tiles [i rows][d]
-          // in the bf16 Lam tile, free until the Lam update: the products have read it
+          // in this chunk's G and U tiles: every product that reads them has completed
           float v[32];
           tmem_ld32(tbase + COL_RX + lane_off + 32 * wg, v);
           tmem_ld_wait();
@@ -880,7 +913,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               v[8 * cc + 7] += bf16_hi(o.w);
             }
           }
-          const uint32_t trow = sLb + (lo ? 0 : 2 * TILE) + (wg >> 1) * TILE;
+          const uint32_t trow = smem_u32(lo ? sm.G[st] : sm.U[st]) + (wg >> 1) * TILE;
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc)
             st_shared_v4(trow + sw128_off(i, 4 * (wg & 1) + cc), pack_bf16(v[8 * cc], v[8 * cc + 1]),
@@ -892,10 +925,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       named_sync_math();  // (B4) t, hv of all warpgroups and the dg / dx staging tiles written
       if (ok && mt == 0) {  // rows past T are clipped by the tensor maps
-        tma_store_3d(&tmDG, sm.Lb, p.n0, t0, bh);
-        tma_store_3d(&tmDG, sm.Lb + TILE, p.n0 + 64, t0, bh);
-        tma_store_3d(&tmDX, sm.Lb + 2 * TILE, 0, t0, bh);
-        tma_store_3d(&tmDX, sm.Lb + 3 * TILE, 64, t0, bh);
+        tma_store_3d(&tmDG, sm.G[st], p.n0, t0, bh);
+        tma_store_3d(&tmDG, sm.G[st] + TILE, p.n0 + 64, t0, bh);
+        tma_store_3d(&tmDX, sm.U[st], 0, t0, bh);
+        tma_store_3d(&tmDX, sm.U[st] + TILE, 64, t0, bh);
         tma_store_commit();
       }
       if (ok && mt < C) {  // d_eta_j = -(del_j q_j + t_j)
@@ -912,44 +945,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         float E = 0.f;  // <Lam_end, S_in>: sum of the math warps' partials
 #pragma unroll
         for (int w = 0; w < NMATH; w += 4) {
-          const float4 e4 = *reinterpret_cast<const float4*>(&sm.ered[w]);
+          const float4 e4 = *reinterpret_cast<const float4*>(&sm.ered[it & 1][w]);
           E += (e4.x + e4.y) + (e4.z + e4.w);
         }
         const float da = gs.gam[i] * gs.del[i] * E + gs.del[i] * t2 + gs.gam[i] * t3 + h4;
         if (t0 + i < T) p.d_alpha[tokbase + i] = p.accumulate ? p.d_alpha[tokbase + i] + da : da;
       }
 
-      // ---- phase 3: bf16 copy of the new Lam for the next chunk's products
-      ok = ok && mbar_wait_warp(&sm.b3full, it & 1, wc, W_M_B3);
-      tc_fence_after();
-      if (mt == 0) tma_store_wait_read();  // the staging tiles are about to be overwritten
-      named_sync_math();  // (B4b)
-      if (ok) {
-        const uint32_t lrow = sLb + (wg >> 1) * BIG;
-        float v[32];
-        tmem_ld32(tL, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
-          st_shared_v4(lrow + sw128_off(n, 4 * (wg & 1) + cc), pack_bf16(v[8 * cc], v[8 * cc + 1]),
-                       pack_bf16(v[8 * cc + 2], v[8 * cc + 3]),
-                       pack_bf16(v[8 * cc + 4], v[8 * cc + 5]),
-                       pack_bf16(v[8 * cc + 6], v[8 * cc + 7]));
-        tc_fence_before();
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&sm.lbready);
-          mbar_arrive(&sm.gempty[g]);
-        }
+      // ---- the staging tiles are read: the stage may take the X, G, U of chunk it + NS
+      if (mt == 0) {
+        tma_store_wait_read();
+        mbar_arrive(&sm.xempty[st]);
       }
-      // No barrier is needed here: every read of this chunk's scratch (partial sums,
-      // gates) happened before B4b, and the next chunk's products wait for lbready
-      // from every math warp.
+      __syncwarp();
+      if (ok && lane == 0) mbar_arrive(&sm.gempty[g]);  // this chunk's gates are read
+      // No barrier is needed here. Faster warps may start the next chunk while warps
+      // 4-7 finish the scalars above, but what those read is rewritten only later:
+      // q by warps 4-5 themselves, the t, t2, t3 and h partials after the next B2
+      // (which warps 4-7 must reach), the E partials in the other parity slot, and
+      // the gates only after every math warp has arrived on gempty. The next tiles of
+      // this stage land in the staging tiles only after their stores have read them.
     }
 
     if (mt == 0) tma_store_wait_all();
-    // ---- this scan's dW0 partial: the last b3full wait covered every product
+    // ---- this scan's dW0 partial: the last b2full wait covered every product
     if (ok) {
       float v[32];
       tmem_ld32(tbase + COL_W + lane_off + 32 * wg, v);
