@@ -106,9 +106,12 @@ struct Smem {
   uint8_t X[NS][2 * TILE];    // [s rows][k]: k-blocks
   uint8_t G[NS][2 * TILE];    // [s rows][n]: n-blocks
   uint8_t U[NS][2 * TILE];    // [s rows][n]
-  uint8_t Sin[2 * BIG];       // [k-block][n rows x 128 B]; then Ar | Z | Q^T | Bm
+  // Two regions that swap roles every chunk. Chunk it loads S_in into SL[it & 1], builds
+  // its chunk matrices (Ar | Z | Q^T | Bm) there once S_in is read, and leaves the bf16
+  // Lam for the next chunk there once those are read; it reads the bf16 Lam of the chunk
+  // before from SL[(it & 1) ^ 1], which then takes the next S_in.
+  uint8_t SL[2][2 * BIG];     // [k-block][n rows x 128 B]
   uint8_t W0[2 * BIG];        // [k-block][n rows x 128 B]
-  uint8_t Lb[2 * BIG];        // bf16 Lam, [k-block][n rows x 128 B]
   uint8_t Xg[2 * TILE];       // diag(gam) X for the Lam update, same layout as X
   GateSlot gates[GS];
   float redq[4][C], redp[4][C];
@@ -119,8 +122,8 @@ struct Smem {
                                      // slots while faster warps start chunk it + 1
   uint64_t xfull[NS], xempty[NS];
   uint64_t gfull[GS], gempty[GS];
-  uint64_t sfull, sempty;  // S_in tile loaded | S_in / chunk-matrix tile read by its last products
-  uint64_t ccfull, b1full, b2full, b3full;
+  uint64_t sfull;  // S_in tile loaded
+  uint64_t ccfull, b1full, b2full;
   uint64_t m1a, m1done, m2done, lscaled, xgready, xgfree, lbfree, lbready, done;
   uint32_t tmem_base;
   int abort;
@@ -134,57 +137,13 @@ enum : uint32_t {
   W_MMA_XFULL = 0x101, W_MMA_M2, W_MMA_SFULL, W_MMA_LB, W_MMA_M1, W_MMA_XS, W_MMA_DONE,
   W_MMA_M1A,
   W_GATE_EMPTY = 0x201, W_XG_FULL, W_XG_GFULL, W_XG_FREE,
-  W_M_GFULL = 0x401, W_M_CC, W_M_B1, W_M_B2, W_M_B3,
+  W_M_GFULL = 0x401, W_M_CC, W_M_B1, W_M_B2,
 };
 
 __device__ __forceinline__ void named_sync_math() {
   asm volatile("bar.sync 1, %0;" ::"n"(32 * NMATH) : "memory");
 }
 
-// Element (row, col) of a [rows x 128 B] swizzled bf16 block (col < 64).
-__device__ __forceinline__ uint32_t sw_elem(uint32_t base, uint32_t row, uint32_t col) {
-  return base + sw128_off(row, col >> 3) + ((col & 7) << 1);
-}
-
-__device__ __forceinline__ float lds_bf16(uint32_t addr) {
-  unsigned short v;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr) : "memory");
-  return __uint_as_float(((uint32_t)v) << 16);
-}
-
-__device__ __forceinline__ void sts_u16(uint32_t addr, float f) {
-  const __nv_bfloat16 b = __float2bfloat16_rn(f);
-  const unsigned short v = *reinterpret_cast<const unsigned short*>(&b);
-  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
-}
-
-// Sum of v[0..15] over the 32 lanes of the warp; lanes 2k and 2k+1 return the total of index k.
-__device__ __forceinline__ float reduce_scatter16(float (&v)[16], int lane) {
-  float w8[8], w4[4], w2[2];
-  const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const float send = b4 ? v[k] : v[k + 8];
-    const float keep = b4 ? v[k + 8] : v[k];
-    w8[k] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-  }
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const float send = b3 ? w8[k] : w8[k + 4];
-    const float keep = b3 ? w8[k + 4] : w8[k];
-    w4[k] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-  }
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const float send = b2 ? w4[k] : w4[k + 2];
-    const float keep = b2 ? w4[k + 2] : w4[k];
-    w2[k] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-  }
-  const float send = b1 ? w2[0] : w2[1];
-  const float keep = b1 ? w2[1] : w2[0];
-  float w1 = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-  return w1 + __shfl_xor_sync(0xffffffffu, w1, 1);
-}
 
 }  // namespace
 
@@ -217,12 +176,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&sm.gempty[g], NMATH);
     }
     mbar_init(&sm.sfull, 1);
-    mbar_init(&sm.sempty, 1);
     mbar_init(&sm.lbfree, 1);
     mbar_init(&sm.ccfull, 1);
     mbar_init(&sm.b1full, 1);
     mbar_init(&sm.b2full, 1);
-    mbar_init(&sm.b3full, 1);
     mbar_init(&sm.m1a, NMATH);
     mbar_init(&sm.m1done, NMATH);
     mbar_init(&sm.m2done, NMATH);
@@ -261,10 +218,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const float* li = p.L_init + (seg_row * p.dout + p.n0 + n) * 128 + ck * 8;
         const float4 u = *reinterpret_cast<const float4*>(li);
         const float4 v = *reinterpret_cast<const float4*>(li + 4);
-        st_shared_v4(smem_u32(sm.Lb + kb * BIG) + sw128_off(n, c), pack_bf16(u.x, u.y),
+        st_shared_v4(smem_u32(sm.SL[1] + kb * BIG) + sw128_off(n, c), pack_bf16(u.x, u.y),
                      pack_bf16(u.z, u.w), pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
       } else {
-        st_shared_v4(smem_u32(sm.Lb + kb * BIG) + sw128_off(n, c), 0u, 0u, 0u, 0u);
+        st_shared_v4(smem_u32(sm.SL[1] + kb * BIG) + sw128_off(n, c), 0u, 0u, 0u, 0u);
       }
     }
     fence_proxy_async_smem();
@@ -290,12 +247,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tma_load_3d(sm.U[st], &tmU, &sm.xfull[st], p.n0, c * C, bh);
           tma_load_3d(sm.U[st] + TILE, &tmU, &sm.xfull[st], p.n0 + 64, c * C, bh);
           xi = it + 1;
-          // the S_in tile doubles as the chunk-matrix scratch: load once the previous
-          // chunk's products on the chunk matrices have completed
-          if (!mbar_wait(&sm.sempty, (it & 1) ^ 1, wc, W_TMA_SEMPTY)) break;
+          // S_in goes to SL[it & 1], which last held the bf16 Lam that chunk it - 1 read:
+          // load once that chunk's last products on it have completed
+          if (it > 0 && !mbar_wait(&sm.lbfree, (it - 1) & 1, wc, W_TMA_SEMPTY)) break;
           mbar_arrive_expect_tx(&sm.sfull, 2 * BIG);
-          tma_load_3d(sm.Sin, &tmS, &sm.sfull, 0, p.n0, bh * nch_all + c);
-          tma_load_3d(sm.Sin + BIG, &tmS, &sm.sfull, 64, p.n0, bh * nch_all + c);
+          tma_load_3d(sm.SL[it & 1], &tmS, &sm.sfull, 0, p.n0, bh * nch_all + c);
+          tma_load_3d(sm.SL[it & 1] + BIG, &tmS, &sm.sfull, 64, p.n0, bh * nch_all + c);
           si = it + 1;
         }
         for (int it = xi > NS ? xi - NS : 0; it < xi; ++it)
@@ -310,29 +267,58 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t id_tb = idesc_bf16(64, 128, false, true);      // U S_in, U W0, Ar U, ...
         const uint32_t id_r1 = idesc_bf16(64, 128, false, false);     // X Lam^T
         const uint32_t id_v = idesc_bf16(64, 64, false, true);        // Bm Q^T
-        const uint32_t sS = smem_u32(sm.Sin), sW0 = smem_u32(sm.W0), sL = smem_u32(sm.Lb);
-        // Issue order per chunk: R1 = X Lam^T and the Gram products and dW0 as soon as
-        // the previous chunk's output phase has read its accumulators, DXb when S_in
-        // lands, the Lam update once the math warps have scaled Lam, the dx terms that
-        // need only scaled G and DXb, and last the three products that need the chunk
-        // matrices.
+        const uint32_t sW0 = smem_u32(sm.W0);
+        // Issue order per chunk: K, Kug and dW0 as soon as X, G, U land (their accumulators
+        // were last read by the previous chunk's matrix build); KugT and R1 once the previous
+        // chunk's output phase has read its accumulators and left the bf16 Lam; DXb when S_in
+        // lands; the Lam update once the math warps have scaled Lam; the dx terms that need
+        // only scaled G and DXb; and last the three products that need the chunk matrices.
         auto xgu = [&](int it, uint32_t& sX, uint32_t& sG, uint32_t& sU) {
           const int st = it % NS;
           sX = smem_u32(sm.X[st]);
           sG = smem_u32(sm.G[st]);
           sU = smem_u32(sm.U[st]);
         };
-        auto phase1r = [&](int it) -> bool {  // R1 = X Lam^T
+        // this chunk's S_in / chunk-matrix region, and the bf16 Lam of the chunk before
+        auto region_s = [&](int it) { return smem_u32(sm.SL[it & 1]); };
+        auto region_l = [&](int it) { return smem_u32(sm.SL[(it & 1) ^ 1]); };
+        auto phase1a = [&](int it) -> bool {  // K = X X^T, Kug = U G^T, dW0 += U^T X
           uint32_t sX, sG, sU;
           xgu(it, sX, sG, sU);
           if (!mbar_wait(&sm.xfull[it % NS], (it / NS) & 1, wc, W_MMA_XFULL)) return false;
-          // R1 and DXb overwrite the r and dx accumulators of the previous chunk, which
-          // its output phase has read by m2done
+          tc_fence_after();
+          #pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * TILE + (kk & 3) * 32;
+            const uint64_t dX = desc_at(sw128_desc(sX, 16, 1024), off);
+            umma_bf16(tbase + COL_KK, dX, dX, id_cc, kk > 0);
+            umma_bf16(tbase + COL_KK + LANE16, desc_at(sw128_desc(sU, 16, 1024), off),
+                      desc_at(sw128_desc(sG, 16, 1024), off), id_cc, kk > 0);
+          }
+          #pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tbase + COL_W, desc_at(sw128_desc(sU, TILE, 1024), kk * 2048),
+                      desc_at(sw128_desc(sX, TILE, 1024), kk * 2048), id_w, (it > 0 || kk > 0));
+          return true;
+        };
+        auto phase1r = [&](int it) -> bool {  // KugT = G U^T, R1 = X Lam^T
+          uint32_t sX, sG, sU;
+          xgu(it, sX, sG, sU);
+          // KugT, R1 (and DXb after them) overwrite accumulators that the previous chunk's
+          // output phase reads until m2done: V^T's neighbour lanes, r and dx
           if (it > 0 && !mbar_wait(&sm.m2done, (it - 1) & 1, wc, W_MMA_M2)) return false;
           if (it > 0 && !mbar_wait(&sm.lbready, (it - 1) & 1, wc, W_MMA_LB)) return false;
           tc_fence_after();
+          const uint32_t sL = region_l(it);
           #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)  // R1 = X Lam^T
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * TILE + (kk & 3) * 32;
+            umma_bf16(tbase + COL_KT, desc_at(sw128_desc(sG, 16, 1024), off),
+                      desc_at(sw128_desc(sU, 16, 1024), off), id_cc, kk > 0);
+          }
+          umma_commit(&sm.ccfull);  // the Gram products (the last readers of unscaled G)
+          #pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
             umma_bf16(tbase + COL_RX, desc_at(sw128_desc(sX, 16, 1024), (kk >> 2) * TILE + (kk & 3) * 32),
                       desc_at(sw128_desc(sL, 16, 1024), (kk >> 2) * BIG + (kk & 3) * 32), id_r1, kk > 0);
           return true;
@@ -342,6 +328,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           xgu(it, sX, sG, sU);
           if (!mbar_wait(&sm.sfull, it & 1, wc, W_MMA_SFULL)) return false;
           tc_fence_after();
+          const uint32_t sS = region_s(it);
           #pragma unroll
           for (int kk = 0; kk < 8; ++kk)  // DXb = U S_in
             umma_bf16(tbase + COL_RX + LANE16, desc_at(sw128_desc(sU, 16, 1024), (kk >> 2) * TILE + (kk & 3) * 32),
@@ -349,31 +336,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           umma_commit(&sm.b1full);  // R1, the Gram products, dW0 and DXb
           return true;
         };
-        auto phase1a = [&](int it) -> bool {  // K, Kug, KugT, dW0 (after phase1r's waits)
-          uint32_t sX, sG, sU;
-          xgu(it, sX, sG, sU);
-          #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {  // K = X X^T, Kug = U G^T, KugT = G U^T
-            const uint32_t off = (kk >> 2) * TILE + (kk & 3) * 32;
-            const uint64_t dX = desc_at(sw128_desc(sX, 16, 1024), off);
-            const uint64_t dG = desc_at(sw128_desc(sG, 16, 1024), off);
-            const uint64_t dU = desc_at(sw128_desc(sU, 16, 1024), off);
-            umma_bf16(tbase + COL_KK, dX, dX, id_cc, kk > 0);
-            umma_bf16(tbase + COL_KK + LANE16, dU, dG, id_cc, kk > 0);
-            umma_bf16(tbase + COL_KT, dG, dU, id_cc, kk > 0);
-          }
-          umma_commit(&sm.ccfull);
-          #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)  // dW0 += U^T X
-            umma_bf16(tbase + COL_W, desc_at(sw128_desc(sU, TILE, 1024), kk * 2048),
-                      desc_at(sw128_desc(sX, TILE, 1024), kk * 2048), id_w, (it > 0 || kk > 0));
-          return true;
-        };
         auto phase2a = [&](int it) -> bool {  // dx terms that need only Gs and gam (.) DXb
           uint32_t sX, sG, sU;
           xgu(it, sX, sG, sU);
           if (!mbar_wait(&sm.m1a, it & 1, wc, W_MMA_M1A)) return false;
           tc_fence_after();
+          const uint32_t sL = region_l(it);
           #pragma unroll
           for (int kk = 0; kk < 8; ++kk)  // dx = gam (.) DXb + U W0
             umma_bf16(tbase + COL_RX + LANE16, desc_at(sw128_desc(sU, 16, 1024), (kk >> 2) * TILE + (kk & 3) * 32),
@@ -382,7 +350,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int kk = 0; kk < 8; ++kk)  //      + Gs Lam
             umma_bf16(tbase + COL_RX + LANE16, desc_at(sw128_desc(sG, 16, 1024), (kk >> 2) * TILE + (kk & 3) * 32),
                       desc_at(sw128_desc(sL, BIG, 1024), kk * 2048), id_tb, 1);
-          umma_commit(&sm.lbfree);  // the last product reading the bf16 Lam of this chunk
+          umma_commit(&sm.lbfree);  // the last product reading the bf16 Lam of the chunk before
           return true;
         };
         auto phase2b = [&](int it) -> bool {  // the products of the chunk matrices
@@ -390,6 +358,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           xgu(it, sX, sG, sU);
           if (!mbar_wait(&sm.m1done, it & 1, wc, W_MMA_M1)) return false;
           tc_fence_after();
+          const uint32_t sS = region_s(it);
           #pragma unroll
           for (int kk = 0; kk < 4; ++kk)  // V^T = Bm Q^T
             umma_bf16(tbase + COL_KT + LANE16, desc_at(sw128_desc(sS, 16, 1024), CC_BM + kk * 32),
@@ -402,8 +371,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int kk = 0; kk < 4; ++kk)  // dx += Z X
             umma_bf16(tbase + COL_RX + LANE16, desc_at(sw128_desc(sS, 16, 1024), CC_Z + kk * 32),
                       desc_at(sw128_desc(sX, TILE, 1024), kk * 2048), id_tb, 1);
-          umma_commit(&sm.b2full);
-          umma_commit(&sm.sempty);           // the last products reading S_in / the chunk matrices
+          umma_commit(&sm.b2full);           // every product of this chunk, the Lam update included
           umma_commit(&sm.xempty[it % NS]);  // the last products reading X, G and U
           return true;
         };
@@ -418,17 +386,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int kk = 0; kk < 4; ++kk)
             umma_bf16(tbase + COL_L, desc_at(sw128_desc(sU, TILE, 1024), kk * 2048),
                       desc_at(sw128_desc(sXg, TILE, 1024), kk * 2048), id_w, 1);
-          umma_commit(&sm.b3full);
           umma_commit(&sm.xgfree);
           return true;
         };
-        // the Lam update is issued as soon as the math warps have scaled Lam, so that it
-        // runs while they build the chunk matrices. R1 and the Gram products need only
-        // the previous chunk's output phase and the new Lam, so they run while the next
-        // S_in tile is still being loaded; DXb follows when it lands.
+        // K, Kug and dW0 run while the previous chunk's output phase reads its accumulators;
+        // R1 and DXb follow, and the Lam update is issued as soon as the math warps have
+        // scaled Lam, so that it runs while they build the chunk matrices.
         bool ok = true;
         for (int it = 0; it < nch && ok; ++it)
-          ok = phase1r(it) && phase1a(it) && phase1b(it) && phase3(it) && phase2a(it) &&
+          ok = phase1a(it) && phase1r(it) && phase1b(it) && phase3(it) && phase2a(it) &&
                phase2b(it);
         umma_commit(&sm.done);
         mbar_drain(&sm.done, 0, wc, W_MMA_DONE);
@@ -523,9 +489,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int ir = 16 * q + (lane & 15);     // chunk row owned in the 64-row products
     const bool lo = lane < 16;
     const int j0w = 16 * wg;                 // first chunk token / column of this warpgroup
-    const uint32_t sS = smem_u32(sm.Sin);
     const uint32_t tL = tbase + COL_L + lane_off + 32 * wg;  // this thread's Lam columns
-    const uint32_t sLb = smem_u32(sm.Lb);
     {  // the fp32 adjoint at the segment's end (Lam_T = 0 for the last segment)
       float z[32];
       if (p.L_init) {
@@ -558,6 +522,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int t0 = c * C;
       const size_t tokbase = (size_t)bh * T + t0;
       const uint32_t sX = smem_u32(sm.X[st]), sG = smem_u32(sm.G[st]);
+      const uint32_t sS = smem_u32(sm.SL[it & 1]);  // S_in, then the chunk matrices
       ok = ok && mbar_wait_warp(&sm.gfull[g], (it / GS) & 1, wc, W_M_GFULL);
       ok = ok && mbar_wait_warp(&sm.xfull[st], (it / NS) & 1, wc, W_M_GFULL);
       ok = ok && mbar_wait_warp(&sm.sfull, it & 1, wc, W_M_GFULL);
@@ -565,7 +530,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
       if (ok) {
         // ---- <Lam_end, S_in>, then Lam <- 2^{L_{C-1}} Lam in place (Lam_end is complete
-        //      since the previous chunk's b3full; this overlaps the R1 and DXb products)
+        //      since the previous chunk's b2full; this overlaps the R1 and DXb products)
         {
           const float gC = gs.gC;
           const uint32_t row = sS + (wg >> 1) * BIG;
@@ -819,13 +784,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (lane == 0) mbar_arrive(&sm.m1done);
       }
 
-      // ---- bf16 copy of the updated Lam for the next chunk's products, as soon as the Lam
-      //      update is done and this chunk's last reader of the bf16 Lam (Gs Lam) has run
-      ok = ok && mbar_wait_warp(&sm.b3full, it & 1, wc, W_M_B3);
-      ok = ok && mbar_wait_warp(&sm.lbfree, it & 1, wc, W_M_B3);
+      // ---- phase 2: dg from r, dx from dx, and the V part of dalpha
+      ok = ok && mbar_wait_warp(&sm.b2full, it & 1, wc, W_M_B2);
       tc_fence_after();
       if (ok && it + 1 < nch) {
-        const uint32_t lrow = sLb + (wg >> 1) * BIG;
+        // bf16 copy of the updated Lam for the next chunk's products, into this chunk's
+        // region: b2full covers the Lam update and the last products on the chunk matrices
+        const uint32_t lrow = sS + (wg >> 1) * BIG;
         float v[32];
         tmem_ld32(tL, v);
         tmem_ld_wait();
@@ -840,10 +805,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.lbready);
       }
-
-      // ---- phase 2: dg from r, dx from dx, and the V part of dalpha
-      ok = ok && mbar_wait_warp(&sm.b2full, it & 1, wc, W_M_B2);
-      tc_fence_after();
       if (ok) {
         {
           float vv[16];
