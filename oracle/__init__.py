@@ -51,6 +51,9 @@ def _load():
             lib.oracle_fwd_c128.argtypes = [I] * 5 + [P] * 6 + [I]
             lib.oracle_states_f64.argtypes = [I] * 3 + [P] * 7
             lib.oracle_bwd_f64.argtypes = [I] * 5 + [P] * 11 + [I] * 3
+            lib.oracle_fwd_state_f64.argtypes = [I] * 5 + [P] * 8 + [I]
+            lib.oracle_fwd_state_c128.argtypes = [I] * 5 + [P] * 8 + [I]
+            lib.oracle_bwd_state_f64.argtypes = [I] * 5 + [P] * 14 + [I] * 3
             lib.oracle_serial_f64.argtypes = [I] * 5 + [P] * 7 + [I]
             lib.oracle_serial_c128.argtypes = [I] * 5 + [P] * 7 + [I]
             lib.oracle_max_threads.restype = I
@@ -89,6 +92,58 @@ def fwd(x, g, eta, alpha, W0, nthreads: int = 0):
     f = _load().oracle_fwd_c128 if cplx else _load().oracle_fwd_f64
     f(B, H, T, din, dout, _p(x), _p(g), _p(eta), _p(alpha), _p(W0), _p(y), int(nthreads))
     return y
+
+
+def _state_arg(S, dt, B, H, din, dout):
+    if S is None:
+        return None
+    S = _arr(S, dt)
+    assert S.shape == (B, H, dout, din), S.shape
+    return S
+
+
+def _pn(a):
+    return _p(a) if a is not None else None
+
+
+def fwd_state(x, g, eta, alpha, W0, S0=None, nthreads: int = 0):
+    """Forward scan continuing from the start deviation S0 ([B,H,d_out,d_in], None = 0).
+
+    Returns (y [B,H,T,d_out], S_T [B,H,d_out,d_in]). Complex inputs run the complex
+    instantiation."""
+    cplx = any(np.iscomplexobj(np.asarray(a)) for a in (x, g, eta, alpha, W0)
+               if a is not None) or (S0 is not None and np.iscomplexobj(np.asarray(S0)))
+    dt = np.complex128 if cplx else np.float64
+    x, g, eta, alpha, W0 = (_arr(a, dt) for a in (x, g, eta, alpha, W0))
+    B, H, T, din, dout = _dims(x, g)
+    assert eta.shape == alpha.shape == (B, H, T) and W0.shape == (H, dout, din)
+    S0 = _state_arg(S0, dt, B, H, din, dout)
+    y = np.empty((B, H, T, dout), dtype=dt)
+    ST = np.empty((B, H, dout, din), dtype=dt)
+    f = _load().oracle_fwd_state_c128 if cplx else _load().oracle_fwd_state_f64
+    f(B, H, T, din, dout, _p(x), _p(g), _p(eta), _p(alpha), _p(W0), _pn(S0), _p(y), _p(ST),
+      int(nthreads))
+    return y, ST
+
+
+def bwd_state(x, g, eta, alpha, W0, dy, S0=None, LamT=None, ckpt: int = 64,
+              mutate: bool = False, nthreads: int = 0):
+    """Reverse scan with the carried state: S0 is the start deviation the forward began
+    from, LamT the gradient of the objective with respect to S_T (both [B,H,d_out,d_in],
+    None = 0). Returns dict dx, dg, deta, dalpha, dW0, dS0."""
+    x, g, eta, alpha, W0, dy = (_arr(a, np.float64) for a in (x, g, eta, alpha, W0, dy))
+    B, H, T, din, dout = _dims(x, g)
+    assert dy.shape == g.shape and W0.shape == (H, dout, din)
+    S0 = _state_arg(S0, np.float64, B, H, din, dout)
+    LamT = _state_arg(LamT, np.float64, B, H, din, dout)
+    out = dict(dx=np.empty_like(x), dg=np.empty_like(g), deta=np.empty_like(eta),
+               dalpha=np.empty_like(alpha), dW0=np.empty_like(W0),
+               dS0=np.empty((B, H, dout, din)))
+    _load().oracle_bwd_state_f64(B, H, T, din, dout, _p(x), _p(g), _p(eta), _p(alpha), _p(W0),
+                                 _pn(S0), _p(dy), _pn(LamT), _p(out["dx"]), _p(out["dg"]),
+                                 _p(out["deta"]), _p(out["dalpha"]), _p(out["dW0"]),
+                                 _p(out["dS0"]), int(ckpt), 1 if mutate else 0, int(nthreads))
+    return out
 
 
 def states(x, g, eta, alpha, W0):

@@ -39,6 +39,19 @@
 //       dalpha_t = <Lam_{t+1}, S_t>_F
 //       dW_0     = sum over b and t of u_t x_t^T      (W_0 is one matrix per head)
 //
+// Carried state (a sequence split across calls). The same section notes that
+// the recurrence is affine, so partial results combine: the second part of a
+// split sequence continues from the deviation the first part left. The
+// streaming entry points take that start deviation S_0 (zero for a fresh
+// sequence) and return the end deviation S_T; in reverse they take the
+// objective's gradient with respect to S_T (Lam_T, the adjoint flowing in
+// from the later part) and return dL/dS_0:
+//
+//       L = sum_t <u_t, y_t> + <Lam_T, S_T>_F,   dS_0 = Lam_0
+//
+// with the adjoint recurrence above started from that Lam_T. Every other
+// output keeps its formula, with S_t now including the carried S_0.
+//
 // Everything is materialised token by token in double (or complex<double> for
 // the complex-step derivative checks); there is no chunking, no blocking and
 // no reordering beyond this serial definition. OpenMP is used only across the
@@ -73,13 +86,15 @@ void state_step(int din, int dout, R* S, R alpha, R eta, const R* g, const R* x)
       S[(size_t)n * din + k] = alpha * S[(size_t)n * din + k] - eta * g[n] * x[k];
 }
 
-// Forward of one (b,h) scan. S_work holds d_out*d_in scalars. If S_traj is
-// non-null it receives S_0 .. S_T ((T+1)*d_out*d_in scalars).
+// Forward of one (b,h) scan. S_work holds d_out*d_in scalars. S0 (or null for
+// zero) is the start deviation; if S_traj is non-null it receives S_0 .. S_T
+// ((T+1)*d_out*d_in scalars); if ST is non-null it receives S_T.
 template <class R>
 void fwd_head(int T, int din, int dout, const R* x, const R* g, const R* eta,
-              const R* alpha, const R* W0, R* y, R* S_work, R* S_traj) {
+              const R* alpha, const R* W0, R* y, R* S_work, R* S_traj,
+              const R* S0 = nullptr, R* ST = nullptr) {
   const size_t dd = (size_t)din * dout;
-  for (size_t e = 0; e < dd; ++e) S_work[e] = R(0);
+  for (size_t e = 0; e < dd; ++e) S_work[e] = S0 ? S0[e] : R(0);
   if (S_traj) std::memcpy(S_traj, S_work, dd * sizeof(R));
   for (int t = 0; t < T; ++t) {
     const R* xt = x + (size_t)t * din;
@@ -92,6 +107,7 @@ void fwd_head(int T, int din, int dout, const R* x, const R* g, const R* eta,
     state_step(din, dout, S_work, alpha[t], eta[t], g + (size_t)t * dout, xt);
     if (S_traj) std::memcpy(S_traj + (size_t)(t + 1) * dd, S_work, dd * sizeof(R));
   }
+  if (ST) std::memcpy(ST, S_work, dd * sizeof(R));
 }
 
 // Backward of one (b,h) scan. S_t is needed in reverse order; the forward
@@ -100,21 +116,27 @@ void fwd_head(int T, int din, int dout, const R* x, const R* g, const R* eta,
 // sum_t u_t x_t^T. `mutate` = 1 replaces (W_0 + S_t)^T by W_0^T in dx: the
 // negative control of the "synthetic test" section (persistent instead of
 // adapted weight in the backward reconstruction), used only by tests.
+// S0 / LamT (null for zero): the carried start deviation and the adjoint
+// flowing in at the end; dS0 (if non-null) receives Lam_0.
 void bwd_head(int T, int din, int dout, const double* x, const double* g,
               const double* eta, const double* alpha, const double* W0,
               const double* u, double* dx, double* dg, double* deta,
-              double* dalpha, double* dW0p, int ckpt, int mutate) {
+              double* dalpha, double* dW0p, int ckpt, int mutate,
+              const double* S0 = nullptr, const double* LamT = nullptr,
+              double* dS0 = nullptr) {
   const size_t dd = (size_t)din * dout;
   if (ckpt < 1) ckpt = 1;
   const int nseg = (T + ckpt - 1) / ckpt;
   std::vector<double> ck((size_t)nseg * dd, 0.0);
   std::vector<double> S(dd, 0.0);
+  if (S0) std::memcpy(S.data(), S0, dd * sizeof(double));
   for (int t = 0; t < T; ++t) {
     if (t % ckpt == 0) std::memcpy(&ck[(size_t)(t / ckpt) * dd], S.data(), dd * sizeof(double));
     state_step(din, dout, S.data(), alpha[t], eta[t], g + (size_t)t * dout, x + (size_t)t * din);
   }
   std::vector<double> seg((size_t)ckpt * dd);
   std::vector<double> Lam(dd, 0.0), r(dout);
+  if (LamT) std::memcpy(Lam.data(), LamT, dd * sizeof(double));
   for (size_t e = 0; e < dd; ++e) dW0p[e] = 0.0;
   for (int s = nseg - 1; s >= 0; --s) {
     const int t0 = s * ckpt, t1 = (t0 + ckpt < T) ? t0 + ckpt : T;
@@ -159,6 +181,7 @@ void bwd_head(int T, int din, int dout, const double* x, const double* g,
         }
     }
   }
+  if (dS0) std::memcpy(dS0, Lam.data(), dd * sizeof(double));
 }
 
 // Serial online learner with inner loss 0.5 ||W x_t - v_t||^2 (the learner
@@ -195,9 +218,11 @@ inline int pick_threads(int nthreads) {
 #endif
 }
 
+// S0, ST: null, or [B,H,d_out,d_in] start / end deviations.
 template <class R>
 void fwd_all(int B, int H, int T, int din, int dout, const R* x, const R* g, const R* eta,
-             const R* alpha, const R* W0, R* y, int nthreads) {
+             const R* alpha, const R* W0, R* y, int nthreads, const R* S0 = nullptr,
+             R* ST = nullptr) {
   const int nt = pick_threads(nthreads);
   const size_t dd = (size_t)din * dout;
 #pragma omp parallel num_threads(nt)
@@ -208,7 +233,8 @@ void fwd_all(int B, int H, int T, int din, int dout, const R* x, const R* g, con
       const int b = bh / H, h = bh % H;
       const size_t o = at3(b, h, 0, H, T);
       fwd_head<R>(T, din, dout, x + o * din, g + o * dout, eta + o, alpha + o,
-                  W0 + (size_t)h * dd, y + o * dout, S.data(), nullptr);
+                  W0 + (size_t)h * dd, y + o * dout, S.data(), nullptr,
+                  S0 ? S0 + (size_t)bh * dd : nullptr, ST ? ST + (size_t)bh * dd : nullptr);
     }
   }
 }
@@ -249,6 +275,26 @@ void oracle_fwd_c128(int B, int H, int T, int din, int dout, const double* x, co
                 reinterpret_cast<cplx*>(y), nthreads);
 }
 
+// Forward with the carried state (see file header): S0 may be null (zero), ST
+// may be null (not written); both [B,H,d_out,d_in].
+void oracle_fwd_state_f64(int B, int H, int T, int din, int dout, const double* x,
+                          const double* g, const double* eta, const double* alpha,
+                          const double* W0, const double* S0, double* y, double* ST,
+                          int nthreads) {
+  fwd_all<double>(B, H, T, din, dout, x, g, eta, alpha, W0, y, nthreads, S0, ST);
+}
+
+void oracle_fwd_state_c128(int B, int H, int T, int din, int dout, const double* x,
+                           const double* g, const double* eta, const double* alpha,
+                           const double* W0, const double* S0, double* y, double* ST,
+                           int nthreads) {
+  fwd_all<cplx>(B, H, T, din, dout, reinterpret_cast<const cplx*>(x),
+                reinterpret_cast<const cplx*>(g), reinterpret_cast<const cplx*>(eta),
+                reinterpret_cast<const cplx*>(alpha), reinterpret_cast<const cplx*>(W0),
+                reinterpret_cast<cplx*>(y), nthreads, reinterpret_cast<const cplx*>(S0),
+                reinterpret_cast<cplx*>(ST));
+}
+
 // Whole state trajectory S_0..S_T of ONE scan (B = H = 1), for small tests.
 void oracle_states_f64(int T, int din, int dout, const double* x, const double* g,
                        const double* eta, const double* alpha, const double* W0, double* y,
@@ -260,10 +306,29 @@ void oracle_states_f64(int T, int din, int dout, const double* x, const double* 
 // Reverse scan (see file header). ckpt: checkpoint interval of the state
 // recompute (any value >= 1 gives the same result up to nothing: the recompute
 // is the same serial arithmetic). flags bit 0: negative-control mutation.
+void oracle_bwd_state_f64(int B, int H, int T, int din, int dout, const double* x,
+                          const double* g, const double* eta, const double* alpha,
+                          const double* W0, const double* S0, const double* dy,
+                          const double* LamT, double* dx, double* dg, double* deta,
+                          double* dalpha, double* dW0, double* dS0, int ckpt, int flags,
+                          int nthreads);
+
 void oracle_bwd_f64(int B, int H, int T, int din, int dout, const double* x, const double* g,
                     const double* eta, const double* alpha, const double* W0, const double* dy,
                     double* dx, double* dg, double* deta, double* dalpha, double* dW0,
                     int ckpt, int flags, int nthreads) {
+  oracle_bwd_state_f64(B, H, T, din, dout, x, g, eta, alpha, W0, nullptr, dy, nullptr, dx, dg,
+                       deta, dalpha, dW0, nullptr, ckpt, flags, nthreads);
+}
+
+// Reverse scan with the carried state (see file header): S0 and LamT may be null
+// (zero), dS0 may be null (not written); all three are [B,H,d_out,d_in].
+void oracle_bwd_state_f64(int B, int H, int T, int din, int dout, const double* x,
+                          const double* g, const double* eta, const double* alpha,
+                          const double* W0, const double* S0, const double* dy,
+                          const double* LamT, double* dx, double* dg, double* deta,
+                          double* dalpha, double* dW0, double* dS0, int ckpt, int flags,
+                          int nthreads) {
   const int nt = pick_threads(nthreads);
   const size_t dd = (size_t)din * dout;
   std::vector<double> part((size_t)B * H * dd);
@@ -273,7 +338,8 @@ void oracle_bwd_f64(int B, int H, int T, int din, int dout, const double* x, con
     const size_t o = at3(b, h, 0, H, T);
     bwd_head(T, din, dout, x + o * din, g + o * dout, eta + o, alpha + o, W0 + (size_t)h * dd,
              dy + o * dout, dx + o * din, dg + o * dout, deta + o, dalpha + o,
-             &part[(size_t)bh * dd], ckpt, flags & 1);
+             &part[(size_t)bh * dd], ckpt, flags & 1, S0 ? S0 + (size_t)bh * dd : nullptr,
+             LamT ? LamT + (size_t)bh * dd : nullptr, dS0 ? dS0 + (size_t)bh * dd : nullptr);
   }
   for (int h = 0; h < H; ++h) {
     double* out = dW0 + (size_t)h * dd;

@@ -21,7 +21,15 @@ independent statement of what the GradLev scan must compute:
   quadratic (x), complex-step for the polynomial dependence on alpha;
 * the negative control of the synthetic-test section: using the persistent
   weight instead of the adapted one in the backward must break the
-  gradients while leaving the forward unchanged.
+  gradients while leaving the forward unchanged;
+* the carried state of a split sequence (same page, same section: the
+  recurrence is affine, so partial results combine). This is pinned by
+  - the closed form with the start deviation S_0;
+  - running the two parts with S_T -> S_0 and dS_0 -> Lam_T handed across,
+    which must equal the whole sequence;
+  - derivative checks of every output, dS_0 included, for the objective
+    with the <Lam_T, S_T> term;
+  - closed-form special cases (static gates; alpha_0 = 0 cuts S_0 off).
 """
 
 import json
@@ -298,3 +306,139 @@ def test_structural_zeros_and_checkpoint_invariance():
     for other in outs[1:]:
         for k in o:
             assert np.array_equal(o[k], other[k]), k
+
+
+# --------------------------------------------------------------------------- carried state
+
+
+def closed_form_state(x, g, eta, alpha, W0, S0):
+    """The closed form above plus the carried start deviation:
+    S_t = (prod_{r<t} alpha_r) S_0 - sum_{s<t} (prod_{r=s+1}^{t-1} alpha_r) eta_s g_s x_s^T."""
+    _, S = closed_form(x, g, eta, alpha, W0)
+    T = x.shape[0]
+    y = np.zeros((T, g.shape[1]))
+    for t in range(T + 1):
+        p = 1.0
+        for r in range(t):
+            p *= alpha[r]
+        S[t] = S[t] + p * S0
+        if t < T:
+            y[t] = (W0 + S[t]) @ x[t]
+    return y, S
+
+
+def _state_inputs(B=1, H=2, T=11, d_in=4, d_out=3, seed=21, alpha_mode="sigmoid"):
+    d = tiny(B=B, H=H, T=T, d_in=d_in, d_out=d_out, seed=seed, alpha_mode=alpha_mode)
+    rng = np.random.default_rng(seed + 1000)
+    S0 = rng.standard_normal((B, H, d_out, d_in))
+    LamT = rng.standard_normal((B, H, d_out, d_in))
+    return d, S0, LamT
+
+
+@pytest.mark.parametrize("alpha_mode", ["sigmoid", "log_uniform"])
+def test_state_closed_form_bruteforce(alpha_mode):
+    d, S0, _ = _state_inputs(B=2, alpha_mode=alpha_mode)
+    y, ST = oracle.fwd_state(d["x"], d["g"], d["eta"], d["alpha"], d["W0"], S0)
+    B, H = d["x"].shape[:2]
+    for b in range(B):
+        for h in range(H):
+            yc, Sc = closed_form_state(d["x"][b, h], d["g"][b, h], d["eta"][b, h],
+                                       d["alpha"][b, h], d["W0"][h], S0[b, h])
+            assert rel(y[b, h], yc) < 1e-13
+            assert rel(ST[b, h], Sc[-1]) < 1e-13
+    # no start state is the zero start state, and matches the stateless forward bit for bit
+    y0, _ = oracle.fwd_state(d["x"], d["g"], d["eta"], d["alpha"], d["W0"])
+    yz, _ = oracle.fwd_state(d["x"], d["g"], d["eta"], d["alpha"], d["W0"], np.zeros_like(S0))
+    assert np.array_equal(y0, oracle.fwd(d["x"], d["g"], d["eta"], d["alpha"], d["W0"]))
+    assert np.array_equal(y0, yz)
+
+
+def _cut(d, t0, t1):
+    return {k: (v[:, :, t0:t1] if k != "W0" else v) for k, v in d.items()}
+
+
+@pytest.mark.parametrize("split", [1, 5, 10])
+def test_split_sequence_equals_whole(split):
+    d, S0, LamT = _state_inputs(B=2, H=2, T=11)
+    T = d["x"].shape[2]
+    a, b = _cut(d, 0, split), _cut(d, split, T)
+    args = lambda p: (p["x"], p["g"], p["eta"], p["alpha"], p["W0"])
+    yw, STw = oracle.fwd_state(*args(d), S0)
+    y1, S1 = oracle.fwd_state(*args(a), S0)
+    y2, S2 = oracle.fwd_state(*args(b), S1)
+    # the same serial arithmetic in the same order: bit for bit
+    assert np.array_equal(np.concatenate([y1, y2], axis=2), yw)
+    assert np.array_equal(S2, STw)
+    w = oracle.bwd_state(*args(d), d["dy"], S0=S0, LamT=LamT, ckpt=3)
+    o2 = oracle.bwd_state(*args(b), b["dy"], S0=S1, LamT=LamT, ckpt=3)
+    o1 = oracle.bwd_state(*args(a), a["dy"], S0=S0, LamT=o2["dS0"], ckpt=3)
+    for k in ("dx", "dg", "deta", "dalpha"):
+        assert np.array_equal(np.concatenate([o1[k], o2[k]], axis=2), w[k]), k
+    assert np.array_equal(o1["dS0"], w["dS0"])
+    assert rel(o1["dW0"] + o2["dW0"], w["dW0"]) < 1e-14
+
+
+def _L_state(d, u, S0, LamT, over=None):
+    over = over or {}
+    a = {k: over.get(k, d[k]) for k in ("x", "g", "eta", "alpha", "W0")}
+    S0 = over.get("S0", S0)
+    y, ST = oracle.fwd_state(a["x"], a["g"], a["eta"], a["alpha"], a["W0"], S0)
+    return np.sum(y * u) + np.sum(ST * LamT)
+
+
+def _fd_grad_state(d, S0, LamT, name, u):
+    """Derivatives of L = sum u.y + <Lam_T, S_T>: complex step for alpha, central
+    differences for x (quadratic), exact two-point differences for the affine rest."""
+    base = S0 if name == "S0" else d[name]
+    gr = np.zeros_like(base)
+    for idx in np.ndindex(base.shape):
+        if name == "alpha":
+            a = base.astype(np.complex128)
+            h = 1e-30
+            a[idx] += 1j * h
+            gr[idx] = np.imag(_L_state(d, u, S0, LamT, {"alpha": a})) / h
+        elif name == "x":
+            h = 1e-3
+            p = base.copy(); p[idx] += h
+            m = base.copy(); m[idx] -= h
+            gr[idx] = (_L_state(d, u, S0, LamT, {"x": p}) - _L_state(d, u, S0, LamT, {"x": m})) / (2 * h)
+        else:
+            p = base.copy(); p[idx] += 1.0
+            gr[idx] = _L_state(d, u, S0, LamT, {name: p}) - _L_state(d, u, S0, LamT)
+    return gr
+
+
+@pytest.mark.parametrize("alpha_mode", ["sigmoid", "log_uniform"])
+def test_state_backward_matches_derivatives(alpha_mode):
+    d, S0, LamT = _state_inputs(B=1, H=2, T=7, d_in=3, d_out=2, seed=31, alpha_mode=alpha_mode)
+    u = d["dy"]
+    o = oracle.bwd_state(d["x"], d["g"], d["eta"], d["alpha"], d["W0"], u, S0=S0, LamT=LamT,
+                         ckpt=3)
+    names = dict(x="dx", g="dg", eta="deta", alpha="dalpha", W0="dW0", S0="dS0")
+    for p, k in names.items():
+        fd = _fd_grad_state(d, S0, LamT, p, u)
+        tol = 1e-9 if p == "x" else 1e-12
+        assert rel(o[k], fd) < tol, (p, rel(o[k], fd))
+
+
+def test_state_special_cases_closed_form():
+    d, S0, LamT = _state_inputs(B=1, H=1, T=6, d_in=3, d_out=2, seed=41)
+    x, u = d["x"][0, 0], d["dy"][0, 0]
+    # static gates (alpha = 1, eta = 0): y_t = (W0 + S0) x_t, S_T = S0,
+    # dS0 = Lam_T + sum_t u_t x_t^T
+    st = dict(d, alpha=np.ones_like(d["alpha"]), eta=np.zeros_like(d["eta"]))
+    y, ST = oracle.fwd_state(st["x"], st["g"], st["eta"], st["alpha"], st["W0"], S0)
+    assert rel(y[0, 0], x @ (st["W0"][0] + S0[0, 0]).T) < 1e-14
+    assert np.array_equal(ST, S0)
+    o = oracle.bwd_state(st["x"], st["g"], st["eta"], st["alpha"], st["W0"], st["dy"], S0=S0,
+                         LamT=LamT)
+    assert rel(o["dS0"][0, 0], LamT[0, 0] + u.T @ x) < 1e-14
+    # alpha_0 = 0 forgets S0 after the first token: only y_0 sees it
+    cut = dict(d, alpha=d["alpha"].copy())
+    cut["alpha"][0, 0, 0] = 0.0
+    y1, ST1 = oracle.fwd_state(cut["x"], cut["g"], cut["eta"], cut["alpha"], cut["W0"], S0)
+    y2, ST2 = oracle.fwd_state(cut["x"], cut["g"], cut["eta"], cut["alpha"], cut["W0"])
+    assert np.array_equal(y1[:, :, 1:], y2[:, :, 1:]) and np.array_equal(ST1, ST2)
+    o = oracle.bwd_state(cut["x"], cut["g"], cut["eta"], cut["alpha"], cut["W0"], cut["dy"],
+                         S0=S0, LamT=LamT)
+    assert rel(o["dS0"][0, 0], np.outer(u[0], x[0])) < 1e-14
