@@ -132,6 +132,54 @@ GRADLEV_API gradlev_status gradlev_scan_bwd(int B, int H, int T, int d_in, int d
                                 const void* ckpt, void* workspace, size_t ws_bytes,
                                 void* stream);
 
+/* Split sequences: the carried state.
+ *
+ * Cognaptus, "Parallelize the Training, Keep the Learning Serial", section "Once
+ * the gradient signals are known, the weight trajectory becomes parallelizable":
+ * the recurrence is affine, so partial results combine. A sequence cut into
+ * consecutive parts can be scanned one call per part, each continuing from the
+ * deviation the previous part left.
+ *
+ * Forward with a carried state: the same as gradlev_scan_fwd, except that the
+ * deviation before the first token is S0 instead of 0, and the deviation after
+ * the last token is returned:
+ *   S_0 = S0,  y_t = (W0 + S_t) x_t,  S_{t+1} = alpha_t S_t - eta_t g_t x_t^T,
+ *   ST = S_T.
+ *   S0: NULL (zero), or [B,H,d_out,d_in] float32, read only.
+ *   ST: NULL (not written), or [B,H,d_out,d_in] float32, written. It may not
+ *       alias S0.
+ *   Both are 16-byte aligned (else GRADLEV_ERR_INVALID_ARG) and owned by the
+ *   caller. Every other argument, the workspace size and the checkpoints are as
+ *   in gradlev_scan_fwd; the checkpoints then hold states that include S0. */
+GRADLEV_API gradlev_status gradlev_scan_fwd_state(int B, int H, int T, int d_in, int d_out,
+                                      gradlev_dtype dt, const void* x, const void* g,
+                                      const float* eta, const float* alpha, const float* W0,
+                                      const float* S0, void* y, float* ST, void* ckpt,
+                                      void* workspace, size_t ws_bytes, void* stream);
+
+/* Reverse scan with a carried state: the derivative of
+ *   L = sum_t <dy_t, y_t> + <LamT, S_T>_F
+ * for the forward above. The adjoint recurrence starts from Lam_T = LamT instead
+ * of 0, every output of gradlev_scan_bwd keeps its formula (with S_t including
+ * S0), and the adjoint at the first token is returned:
+ *   dS0 = Lam_0 = dL/dS_0.
+ *   S0: NULL (zero), or the start deviation the forward began from. It is read
+ *       only when ckpt is NULL (the call then recomputes the states from it);
+ *       checkpoints from gradlev_scan_fwd_state already include it.
+ *   LamT: NULL (zero), or [B,H,d_out,d_in] float32. When this part is followed
+ *       by another, LamT is the dS0 the later part's call returned.
+ *   dS0: NULL (not written), or [B,H,d_out,d_in] float32.
+ *   All three are 16-byte aligned and owned by the caller. dS0 may not alias
+ *   another argument. Every other argument, the workspace size and the errors
+ *   are as in gradlev_scan_bwd. */
+GRADLEV_API gradlev_status gradlev_scan_bwd_state(int B, int H, int T, int d_in, int d_out,
+                                      gradlev_dtype dt, const void* x, const void* g,
+                                      const float* eta, const float* alpha, const float* W0,
+                                      const float* S0, const void* dy, const float* LamT,
+                                      void* dx, void* dg, float* d_eta, float* d_alpha,
+                                      float* dW0, float* dS0, const void* ckpt,
+                                      void* workspace, size_t ws_bytes, void* stream);
+
 /* Size of the static scratch array gradlev_scan_bwd_noalloc uses: 64 MiB,
  * held by every GPU that loads the library until the process exits. */
 #define GRADLEV_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)

@@ -30,7 +30,8 @@ def test_header_declares_the_entry_points():
     names = declared_entry_points()
     for n in ("gradlev_scan_fwd", "gradlev_scan_bwd", "gradlev_scan_workspace_bytes",
               "gradlev_status_string", "gradlev_scan_supported", "gradlev_scan_ckpt_bytes",
-              "gradlev_device_status", "gradlev_last_launch_count"):
+              "gradlev_device_status", "gradlev_last_launch_count", "gradlev_scan_fwd_state",
+              "gradlev_scan_bwd_state"):
         assert n in names, n
 
 
@@ -123,3 +124,28 @@ def test_forward_workspace_grows_only_for_segmented_scans(L):
         tw.gradlev_scan_ckpt_bytes(8, 16, 4096, 128, 128, tw.BF16)
     # one chunk: nothing to split
     assert tw.gradlev_scan_workspace_bytes(1, 1, 64, 128, 128, tw.BF16, 0) == 256
+
+
+def test_state_entry_points_validate_before_launch(L):
+    """The carried-state calls check their extra pointers on the host, like the rest."""
+    P = ctypes.c_void_p
+    fake = P(4096)  # never dereferenced: validation fails first
+    I = ctypes.c_int
+    L.gradlev_scan_fwd_state.restype = I
+    L.gradlev_scan_bwd_state.restype = I
+    fwd = lambda S0, ST, ws=1 << 20, d_out=16: L.gradlev_scan_fwd_state(
+        1, 1, 8, 16, d_out, 0, fake, fake, fake, fake, fake, S0, fake, ST, P(0), fake, ws, P(0))
+    bwd = lambda S0, LamT, dS0, ws=1 << 30: L.gradlev_scan_bwd_state(
+        1, 1, 8, 16, 16, 0, fake, fake, fake, fake, fake, S0, fake, LamT, fake, fake, fake, fake,
+        fake, dS0, P(0), fake, ws, P(0))
+    assert fwd(P(4100), P(0)) == 1  # misaligned S0
+    assert fwd(P(0), P(4104)) == 1  # misaligned ST
+    assert fwd(P(0), P(0), d_out=12) == 2  # unsupported shape
+    assert fwd(P(0), P(0), ws=16) == 3  # workspace too small
+    assert bwd(P(4100), P(0), P(0)) == 1
+    assert bwd(P(0), P(4100), P(0)) == 1
+    assert bwd(P(0), P(0), P(4100)) == 1
+    assert bwd(P(0), P(0), P(0), ws=16) == 3
+    # the required pointers are still required
+    assert L.gradlev_scan_fwd_state(1, 1, 8, 16, 16, 0, P(0), fake, fake, fake, fake, P(0), fake,
+                                    P(0), P(0), fake, 1 << 20, P(0)) == 1

@@ -16,8 +16,8 @@ import os
 __all__ = [
     "GradlevError", "lib", "gradlev_status_string", "gradlev_scan_supported",
     "gradlev_scan_workspace_bytes", "gradlev_scan_ckpt_bytes", "gradlev_scan_fwd",
-    "gradlev_scan_bwd", "gradlev_device_status", "gradlev_last_launch_count",
-    "F32", "BF16", "LIB_PATH",
+    "gradlev_scan_bwd", "gradlev_scan_fwd_state", "gradlev_scan_bwd_state",
+    "gradlev_device_status", "gradlev_last_launch_count", "F32", "BF16", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgradlev.so")
@@ -27,7 +27,8 @@ BF16 = 1
 _ENTRY_POINTS = (
     "gradlev_status_string", "gradlev_scan_supported", "gradlev_scan_workspace_bytes",
     "gradlev_scan_ckpt_bytes", "gradlev_scan_fwd", "gradlev_scan_bwd",
-    "gradlev_device_status", "gradlev_last_launch_count",
+    "gradlev_scan_fwd_state", "gradlev_scan_bwd_state", "gradlev_device_status",
+    "gradlev_last_launch_count",
 )
 
 
@@ -67,6 +68,10 @@ def lib():
     L.gradlev_scan_fwd.restype = I
     L.gradlev_scan_bwd.argtypes = [I] * 6 + [P] * 13 + [Z, P]
     L.gradlev_scan_bwd.restype = I
+    L.gradlev_scan_fwd_state.argtypes = [I] * 6 + [P] * 10 + [Z, P]
+    L.gradlev_scan_fwd_state.restype = I
+    L.gradlev_scan_bwd_state.argtypes = [I] * 6 + [P] * 16 + [Z, P]
+    L.gradlev_scan_bwd_state.restype = I
     L.gradlev_device_status.argtypes = [P, P]
     L.gradlev_device_status.restype = I
     L.gradlev_last_launch_count.argtypes = []
@@ -200,6 +205,83 @@ def gradlev_scan_bwd(x, g, eta, alpha, W0, dy, *, ckpt=None, workspace=None, str
                                 _ptr(out["dW0"]), _ptr(ckpt), _ptr(ws),
                                 ws.numel() * ws.element_size(), _stream_ptr(stream))
     _check(st, "gradlev_scan_bwd")
+    return out
+
+
+def _state_tensor(name, t, B, H, d_in, d_out, dev):
+    import torch
+    if t is not None:
+        _check_tensor(name, t, (B, H, d_out, d_in), torch.float32, dev)
+    return t
+
+
+def gradlev_scan_fwd_state(x, g, eta, alpha, W0, S0=None, *, y=None, ST=None, ckpt=None,
+                           workspace=None, stream=None):
+    """Forward scan continuing from the carried deviation S0 ([B,H,d_out,d_in] float32,
+    None = 0). Returns (y, ST), ST the deviation after the last token."""
+    import torch
+    B, H, T, d_in, d_out = _dims(x, g)
+    dev, dt = x.device, x.dtype
+    f32 = torch.float32
+    _check_tensor("x", x, (B, H, T, d_in), dt, dev)
+    _check_tensor("g", g, (B, H, T, d_out), dt, dev)
+    _check_tensor("eta", eta, (B, H, T), f32, dev)
+    _check_tensor("alpha", alpha, (B, H, T), f32, dev)
+    _check_tensor("W0", W0, (H, d_out, d_in), f32, dev)
+    _state_tensor("S0", S0, B, H, d_in, d_out, dev)
+    code = _dt_code(dt)
+    _check(gradlev_scan_supported(B, H, T, d_in, d_out, code), "gradlev_scan_fwd_state")
+    if y is None:
+        y = torch.empty((B, H, T, d_out), dtype=dt, device=dev)
+    _check_tensor("y", y, (B, H, T, d_out), dt, dev)
+    if ST is None:
+        ST = torch.empty((B, H, d_out, d_in), dtype=f32, device=dev)
+    _state_tensor("ST", ST, B, H, d_in, d_out, dev)
+    nws = gradlev_scan_workspace_bytes(B, H, T, d_in, d_out, code, 0)
+    ws = _workspace(nws, dev, workspace)
+    st = lib().gradlev_scan_fwd_state(B, H, T, d_in, d_out, code, _ptr(x), _ptr(g), _ptr(eta),
+                                      _ptr(alpha), _ptr(W0), _ptr(S0), _ptr(y), _ptr(ST),
+                                      _ptr(ckpt), _ptr(ws), ws.numel() * ws.element_size(),
+                                      _stream_ptr(stream))
+    _check(st, "gradlev_scan_fwd_state")
+    return y, ST
+
+
+def gradlev_scan_bwd_state(x, g, eta, alpha, W0, dy, S0=None, LamT=None, *, ckpt=None,
+                           workspace=None, stream=None, out=None):
+    """Reverse scan with the carried state: S0 the start deviation of the forward (read only
+    without ckpt), LamT the adjoint flowing in after the last token (both [B,H,d_out,d_in]
+    float32, None = 0). Returns dict dx, dg, deta, dalpha, dW0, dS0."""
+    import torch
+    B, H, T, d_in, d_out = _dims(x, g)
+    dev, dt = x.device, x.dtype
+    f32 = torch.float32
+    _check_tensor("x", x, (B, H, T, d_in), dt, dev)
+    _check_tensor("g", g, (B, H, T, d_out), dt, dev)
+    _check_tensor("dy", dy, (B, H, T, d_out), dt, dev)
+    _check_tensor("eta", eta, (B, H, T), f32, dev)
+    _check_tensor("alpha", alpha, (B, H, T), f32, dev)
+    _check_tensor("W0", W0, (H, d_out, d_in), f32, dev)
+    _state_tensor("S0", S0, B, H, d_in, d_out, dev)
+    _state_tensor("LamT", LamT, B, H, d_in, d_out, dev)
+    code = _dt_code(dt)
+    _check(gradlev_scan_supported(B, H, T, d_in, d_out, code), "gradlev_scan_bwd_state")
+    if out is None:
+        out = dict(dx=torch.empty_like(x), dg=torch.empty_like(g),
+                   deta=torch.empty((B, H, T), dtype=f32, device=dev),
+                   dalpha=torch.empty((B, H, T), dtype=f32, device=dev),
+                   dW0=torch.empty((H, d_out, d_in), dtype=f32, device=dev),
+                   dS0=torch.empty((B, H, d_out, d_in), dtype=f32, device=dev))
+    _state_tensor("dS0", out["dS0"], B, H, d_in, d_out, dev)
+    nws = gradlev_scan_workspace_bytes(B, H, T, d_in, d_out, code, 1)
+    ws = _workspace(nws, dev, workspace)
+    st = lib().gradlev_scan_bwd_state(B, H, T, d_in, d_out, code, _ptr(x), _ptr(g), _ptr(eta),
+                                      _ptr(alpha), _ptr(W0), _ptr(S0), _ptr(dy), _ptr(LamT),
+                                      _ptr(out["dx"]), _ptr(out["dg"]), _ptr(out["deta"]),
+                                      _ptr(out["dalpha"]), _ptr(out["dW0"]), _ptr(out["dS0"]),
+                                      _ptr(ckpt), _ptr(ws), ws.numel() * ws.element_size(),
+                                      _stream_ptr(stream))
+    _check(st, "gradlev_scan_bwd_state")
     return out
 
 

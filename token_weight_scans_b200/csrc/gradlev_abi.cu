@@ -116,7 +116,8 @@ size_t bwd_scratch_bytes(int B, int H, int T, int din, int dout, gradlev_dtype d
 static gradlev_status launch_fwd_impl(int B, int H, int T, int din, int dout, gradlev_dtype dt,
                                       const void* x, const void* g, const float* eta,
                                       const float* alpha, const float* W0, void* y, void* ckpt,
-                                      DeviceStatus* status, char* seg_ws, cudaStream_t st) {
+                                      DeviceStatus* status, char* seg_ws, cudaStream_t st,
+                                      const float* S0, float* ST) {
   if (use_tc(din, dout, dt)) {
     const int inject = y ? g_inject : 0;
     const uint64_t tmo = inject ? g_inject_timeout_ns : kWaitTimeoutNs;
@@ -137,16 +138,22 @@ static gradlev_status launch_fwd_impl(int B, int H, int T, int din, int dout, gr
       sum.seg_L = sb.L;
       sum.summary = 1;
       if (tc::launch_fwd(sum, x, g, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
-      if (tc::combine_segments(sb.loc, sb.L, sb.comb, B * H, sp.nseg, dout * din, 0, st) !=
+      // the first segment starts from the carried state S0
+      if (tc::combine_segments(sb.loc, sb.L, S0, sb.comb, B * H, sp.nseg, dout * din, 0, st) !=
           cudaSuccess)
         return GRADLEV_ERR_CUDA;
       prm.nseg = sp.nseg;
       prm.seg_chunks = sp.seg_chunks;
       prm.S_init = sb.comb;
+    } else {
+      prm.S_init = S0;  // [B*H][1][dout][din]: the one segment's start state
     }
+    prm.S_last = ST;
     return tc::launch_fwd(prm, x, g, st) == cudaSuccess ? GRADLEV_OK : GRADLEV_ERR_CUDA;
   }
   ffma::FwdArgs a{B, H, T, din, dout, x, g, eta, alpha, W0, y, static_cast<float*>(ckpt)};
+  a.S0 = S0;
+  a.ST = ST;
   return ffma::launch_fwd(a, dt == GRADLEV_BF16, st) == cudaSuccess ? GRADLEV_OK
                                                                    : GRADLEV_ERR_CUDA;
 }
@@ -154,7 +161,8 @@ static gradlev_status launch_fwd_impl(int B, int H, int T, int din, int dout, gr
 gradlev_status bwd_run(int B, int H, int T, int din, int dout, gradlev_dtype dt, const void* x,
                        const void* g, const float* eta, const float* alpha, const float* W0,
                        const void* dy, void* dx, void* dg, float* d_eta, float* d_alpha,
-                       float* dW0, const void* ckpt, char* ws, cudaStream_t st) {
+                       float* dW0, const void* ckpt, char* ws, cudaStream_t st,
+                       const StateIO& io) {
   DeviceStatus* status = reinterpret_cast<DeviceStatus*>(ws);
   float* dW0_part = reinterpret_cast<float*>(ws + kStatusBytes);
   char* own = ws + kStatusBytes + dW0_part_bytes(B, H, T, din, dout, dt);
@@ -164,13 +172,13 @@ gradlev_status bwd_run(int B, int H, int T, int din, int dout, gradlev_dtype dt,
   const void* states = ckpt;
   if (!states) {
     gradlev_status s = launch_fwd_impl(B, H, T, din, dout, dt, x, g, eta, alpha, W0, nullptr,
-                                       own, status, seg_ws, st);
+                                       own, status, seg_ws, st, io.S0, nullptr);
     if (s != GRADLEV_OK) return s;
     states = own;
   }
   if (use_tc(din, dout, dt)) {
     const SegPlan sp = bwd_plan(B, H, T);
-    const float* L_init = nullptr;
+    const float* L_init = io.LamT;  // one segment: it ends where the adjoint flows in
     if (sp.nseg > 1) {
       // each segment's local adjoint (walked backwards from zero) and log-decay, then the
       // adjoint at each segment's end
@@ -184,8 +192,9 @@ gradlev_status bwd_run(int B, int H, int T, int din, int dout, gradlev_dtype dt,
       sum.summary = 1;
       sum.reverse = 1;
       if (tc::launch_fwd(sum, x, dy, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
-      if (tc::combine_segments(sb.loc, sb.L, sb.comb, B * H, sp.nseg, dout * din, 1, st) !=
-          cudaSuccess)
+      // the last segment ends where the adjoint LamT flows in
+      if (tc::combine_segments(sb.loc, sb.L, io.LamT, sb.comb, B * H, sp.nseg, dout * din, 1,
+                               st) != cudaSuccess)
         return GRADLEV_ERR_CUDA;
       L_init = sb.comb;
     }
@@ -197,6 +206,7 @@ gradlev_status bwd_run(int B, int H, int T, int din, int dout, gradlev_dtype dt,
       prm.nseg = sp.nseg;
       prm.seg_chunks = sp.seg_chunks;
       prm.L_init = L_init;
+      prm.L_first = io.dS0;
       if (tc::launch_bwd(prm, x, g, dy, states, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
     }
     // partials are [B][nseg][H]: a fixed-order sum over b and the segments
@@ -206,6 +216,8 @@ gradlev_status bwd_run(int B, int H, int T, int din, int dout, gradlev_dtype dt,
   }
   ffma::BwdArgs a{B, H, T, din, dout, x, g, eta, alpha, W0, dy, dx, dg, d_eta, d_alpha, dW0,
                   static_cast<const float*>(states), dW0_part};
+  a.LamT = io.LamT;
+  a.dS0 = io.dS0;
   return ffma::launch_bwd(a, dt == GRADLEV_BF16, st) == cudaSuccess ? GRADLEV_OK
                                                                    : GRADLEV_ERR_CUDA;
 }
@@ -246,16 +258,21 @@ size_t gradlev_scan_workspace_bytes(int B, int H, int T, int d_in, int d_out, gr
                 : fwd_scratch_bytes(B, H, T, d_in, d_out, dt);
 }
 
-gradlev_status gradlev_scan_fwd(int B, int H, int T, int d_in, int d_out, gradlev_dtype dt,
+}  // extern "C"
+
+namespace gradlev {
+
+static gradlev_status fwd_entry(int B, int H, int T, int d_in, int d_out, gradlev_dtype dt,
                                 const void* x, const void* g, const float* eta,
-                                const float* alpha, const float* W0, void* y, void* ckpt,
-                                void* workspace, size_t ws_bytes, void* stream) {
+                                const float* alpha, const float* W0, const float* S0, void* y,
+                                float* ST, void* ckpt, void* workspace, size_t ws_bytes,
+                                void* stream) {
   gradlev_status s = check_shape(B, H, T, d_in, d_out, dt);
   if (s != GRADLEV_OK) return s;
   if (!x || !g || !eta || !alpha || !W0 || !y || !workspace) return GRADLEV_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(g, 16) || !aligned(y, 16) || !aligned(W0, 16) ||
       !aligned(eta, 4) || !aligned(alpha, 4) || (ckpt && !aligned(ckpt, 16)) ||
-      !aligned(workspace, 16))
+      (S0 && !aligned(S0, 16)) || (ST && !aligned(ST, 16)) || !aligned(workspace, 16))
     return GRADLEV_ERR_INVALID_ARG;
   if (ws_bytes < gradlev_scan_workspace_bytes(B, H, T, d_in, d_out, dt, 0))
     return GRADLEV_ERR_WORKSPACE;
@@ -265,15 +282,15 @@ gradlev_status gradlev_scan_fwd(int B, int H, int T, int d_in, int d_out, gradle
   if (cudaMemsetAsync(status, 0, sizeof(DeviceStatus), st) != cudaSuccess)
     return GRADLEV_ERR_CUDA;
   return launch_fwd_impl(B, H, T, d_in, d_out, dt, x, g, eta, alpha, W0, y, ckpt, status,
-                         static_cast<char*>(workspace) + kStatusBytes, st);
+                         static_cast<char*>(workspace) + kStatusBytes, st, S0, ST);
 }
 
-gradlev_status gradlev_scan_bwd(int B, int H, int T, int d_in, int d_out, gradlev_dtype dt,
+static gradlev_status bwd_entry(int B, int H, int T, int d_in, int d_out, gradlev_dtype dt,
                                 const void* x, const void* g, const float* eta,
                                 const float* alpha, const float* W0, const void* dy, void* dx,
                                 void* dg, float* d_eta, float* d_alpha, float* dW0,
-                                const void* ckpt, void* workspace, size_t ws_bytes,
-                                void* stream) {
+                                const void* ckpt, void* workspace, size_t ws_bytes, void* stream,
+                                const StateIO& io) {
   gradlev_status s = check_shape(B, H, T, d_in, d_out, dt);
   if (s != GRADLEV_OK) return s;
   if (!x || !g || !eta || !alpha || !W0 || !dy || !dx || !dg || !d_eta || !d_alpha || !dW0 ||
@@ -282,13 +299,61 @@ gradlev_status gradlev_scan_bwd(int B, int H, int T, int d_in, int d_out, gradle
   if (!aligned(x, 16) || !aligned(g, 16) || !aligned(dy, 16) || !aligned(dx, 16) ||
       !aligned(dg, 16) || !aligned(W0, 16) || !aligned(dW0, 16) || !aligned(eta, 4) ||
       !aligned(alpha, 4) || !aligned(d_eta, 4) || !aligned(d_alpha, 4) ||
-      (ckpt && !aligned(ckpt, 16)) || !aligned(workspace, 16))
+      (ckpt && !aligned(ckpt, 16)) || (io.S0 && !aligned(io.S0, 16)) ||
+      (io.LamT && !aligned(io.LamT, 16)) || (io.dS0 && !aligned(io.dS0, 16)) ||
+      !aligned(workspace, 16))
     return GRADLEV_ERR_INVALID_ARG;
   if (ws_bytes < gradlev_scan_workspace_bytes(B, H, T, d_in, d_out, dt, 1))
     return GRADLEV_ERR_WORKSPACE;
   t_launches = 0;
   return bwd_run(B, H, T, d_in, d_out, dt, x, g, eta, alpha, W0, dy, dx, dg, d_eta, d_alpha,
-                 dW0, ckpt, static_cast<char*>(workspace), static_cast<cudaStream_t>(stream));
+                 dW0, ckpt, static_cast<char*>(workspace), static_cast<cudaStream_t>(stream), io);
+}
+
+}  // namespace gradlev
+
+extern "C" {
+
+gradlev_status gradlev_scan_fwd(int B, int H, int T, int d_in, int d_out, gradlev_dtype dt,
+                                const void* x, const void* g, const float* eta,
+                                const float* alpha, const float* W0, void* y, void* ckpt,
+                                void* workspace, size_t ws_bytes, void* stream) {
+  return fwd_entry(B, H, T, d_in, d_out, dt, x, g, eta, alpha, W0, nullptr, y, nullptr, ckpt,
+                   workspace, ws_bytes, stream);
+}
+
+gradlev_status gradlev_scan_fwd_state(int B, int H, int T, int d_in, int d_out, gradlev_dtype dt,
+                                      const void* x, const void* g, const float* eta,
+                                      const float* alpha, const float* W0, const float* S0,
+                                      void* y, float* ST, void* ckpt, void* workspace,
+                                      size_t ws_bytes, void* stream) {
+  return fwd_entry(B, H, T, d_in, d_out, dt, x, g, eta, alpha, W0, S0, y, ST, ckpt, workspace,
+                   ws_bytes, stream);
+}
+
+gradlev_status gradlev_scan_bwd(int B, int H, int T, int d_in, int d_out, gradlev_dtype dt,
+                                const void* x, const void* g, const float* eta,
+                                const float* alpha, const float* W0, const void* dy, void* dx,
+                                void* dg, float* d_eta, float* d_alpha, float* dW0,
+                                const void* ckpt, void* workspace, size_t ws_bytes,
+                                void* stream) {
+  return bwd_entry(B, H, T, d_in, d_out, dt, x, g, eta, alpha, W0, dy, dx, dg, d_eta, d_alpha,
+                   dW0, ckpt, workspace, ws_bytes, stream, StateIO{});
+}
+
+gradlev_status gradlev_scan_bwd_state(int B, int H, int T, int d_in, int d_out, gradlev_dtype dt,
+                                      const void* x, const void* g, const float* eta,
+                                      const float* alpha, const float* W0, const float* S0,
+                                      const void* dy, const float* LamT, void* dx, void* dg,
+                                      float* d_eta, float* d_alpha, float* dW0, float* dS0,
+                                      const void* ckpt, void* workspace, size_t ws_bytes,
+                                      void* stream) {
+  StateIO io;
+  io.S0 = S0;
+  io.LamT = LamT;
+  io.dS0 = dS0;
+  return bwd_entry(B, H, T, d_in, d_out, dt, x, g, eta, alpha, W0, dy, dx, dg, d_eta, d_alpha,
+                   dW0, ckpt, workspace, ws_bytes, stream, io);
 }
 
 gradlev_status gradlev_device_status(const void* workspace, void* stream) {

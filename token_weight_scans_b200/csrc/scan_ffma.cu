@@ -105,9 +105,10 @@ __global__ void __launch_bounds__(FT, 1) fwd_kernel(FwdArgs a) {
   Tio* yg = static_cast<Tio*>(a.y);
   const float* W0 = a.W0 + (size_t)h * dout * din;
 
+  const float* S0 = a.S0 ? a.S0 + (size_t)bh * dout * din : nullptr;
   for (int e = tid; e < dout * din; e += FT) {
     const int n = e / din, k = e - n * din;
-    S[n * LDI + k] = 0.f;
+    S[n * LDI + k] = S0 ? S0[e] : 0.f;
     W[n * LDI + k] = W0[e];
   }
   const int NG = dout / 4, NK4 = din / 4, NB = dout / 8;
@@ -217,6 +218,14 @@ __global__ void __launch_bounds__(FT, 1) fwd_kernel(FwdArgs a) {
       for (int r = 0; r < 8; ++r) *reinterpret_cast<float4*>(&S[(nb * 8 + r) * LDI + 4 * k4]) = acc[r];
     }
   }
+  if (a.ST) {  // the state after the last token (padded tokens left it unchanged)
+    __syncthreads();
+    float* dst = a.ST + (size_t)bh * dout * din;
+    for (int e = tid; e < dout * din; e += FT) {
+      const int n = e / din, k = e - n * din;
+      dst[e] = S[n * LDI + k];
+    }
+  }
 }
 
 size_t bwd_smem_bytes(int din, int dout) {
@@ -267,9 +276,10 @@ __global__ void __launch_bounds__(FT, 1) bwd_kernel(BwdArgs a) {
   Tio* dgg = static_cast<Tio*>(a.dg);
   const float* W0 = a.W0 + (size_t)h * dout * din;
 
+  const float* LamT = a.LamT ? a.LamT + (size_t)bh * dout * din : nullptr;
   for (int e = tid; e < dout * din; e += FT) {
     const int n = e / din, k = e - n * din;
-    L[n * LDI + k] = 0.f;
+    L[n * LDI + k] = LamT ? LamT[e] : 0.f;
   }
   float4 dw[2][8];
 #pragma unroll
@@ -503,6 +513,14 @@ __global__ void __launch_bounds__(FT, 1) bwd_kernel(BwdArgs a) {
 #pragma unroll
         for (int r = 0; r < 8; ++r) *reinterpret_cast<float4*>(&L[(nb * 8 + r) * LDI + 4 * k4]) = acc[r];
       }
+    }
+  }
+  if (a.dS0) {  // the adjoint at the first token
+    __syncthreads();
+    float* ds = a.dS0 + (size_t)bh * dout * din;
+    for (int e = tid; e < dout * din; e += FT) {
+      const int n = e / din, k = e - n * din;
+      ds[e] = L[n * LDI + k];
     }
   }
   // this pair's dW0 partial

@@ -16,6 +16,8 @@ struct FwdArgs {
   const float* W0;    // [H,dout,din]
   void* y;            // [B,H,T,dout] or null (state sweep only)
   float* ckpt;        // [B*H][n_chunks][dout][din] or null
+  const float* S0 = nullptr;  // [B*H][dout][din] carried start state, or null (zero)
+  float* ST = nullptr;        // [B*H][dout][din] receives the state after the last token, or null
 };
 
 struct BwdArgs {
@@ -33,6 +35,8 @@ struct BwdArgs {
   float* dW0;         // [H,dout,din]
   const float* ckpt;  // chunk-start states written by the forward sweep
   float* dW0_part;    // [B*H][dout][din] scratch
+  const float* LamT = nullptr;  // [B*H][dout][din] adjoint flowing in at the end, or null (zero)
+  float* dS0 = nullptr;         // [B*H][dout][din] receives the adjoint at the first token, or null
 };
 
 bool shape_ok(int din, int dout);

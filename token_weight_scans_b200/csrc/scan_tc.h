@@ -35,6 +35,8 @@ struct TcFwdParams {
   float* seg_L = nullptr;         // [B*H][nseg] sum of log2 alpha over the segment, or null
   int summary = 0;          // 1: state carry only (no y, no checkpoints)
   int reverse = 0;          // 1: adjoint summary (see above)
+  float* S_last = nullptr;  // [B*H][dout][din] the state after the scan's last token, or null
+                            // (written by the last segment's CTAs; not in summary mode)
 };
 
 // The reverse scan of one 128-row slice [n0, n0+128) of d_out: the rows of the
@@ -62,6 +64,8 @@ struct TcBwdParams {
   int nseg = 1;             // segments per scan
   int seg_chunks = 1 << 30; // chunks per segment (the last one may be shorter)
   const float* L_init = nullptr;  // [B*H][nseg][dout][din] adjoint at each segment's end, or null
+  float* L_first = nullptr;  // [B*H][dout][din] the adjoint at the scan's first token (dL/dS_0),
+                             // or null (written by segment 0's CTAs)
 };
 
 constexpr int kChunk = 64;  // tokens per chunk of the tensor-core kernels
@@ -77,9 +81,11 @@ size_t fwd_smem_bytes();
 // Segments for `units` CTAs per segment index over a scan of n_chunks chunks.
 void segment_plan(int units, int n_chunks, int* nseg, int* seg_chunks);
 // The serial recursion over segment summaries (forward: start states; reverse:
-// end adjoints), element by element for `scans` scans of per_scan elements.
-cudaError_t combine_segments(const float* loc, const float* segL, float* out, int scans, int nseg,
-                             int per_scan, int reverse, cudaStream_t st);
+// end adjoints), element by element for `scans` scans of per_scan elements. `init`
+// ([scans][per_scan], or null for zero) is the value entering the first segment walked:
+// the carried start state forward, the adjoint flowing in at the end in reverse.
+cudaError_t combine_segments(const float* loc, const float* segL, const float* init, float* out,
+                             int scans, int nseg, int per_scan, int reverse, cudaStream_t st);
 
 }  // namespace tc
 }  // namespace gradlev

@@ -940,6 +940,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
       for (int e = 0; e < 8; ++e) dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
     }
+    // ---- the adjoint at the scan's first token, dL/dS_0 (segment 0 ends there)
+    if (ok && p.L_first && seg == 0) {
+      float v[32];
+      tmem_ld32(tL, v);
+      tmem_ld_wait();
+      float4* dst = reinterpret_cast<float4*>(p.L_first + ((size_t)bh * p.dout + p.n0 + n) * 128 + 32 * wg);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+    }
   }
 
   tc_fence_before();

@@ -600,6 +600,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int e = 0; e < 16; ++e)
         so[e] = make_float4(Sreg[4 * e], Sreg[4 * e + 1], Sreg[4 * e + 2], Sreg[4 * e + 3]);
     }
+    if (ok && full && p.S_last && seg == p.nseg - 1) {  // S_T: padded tokens left it unchanged
+      float4* so = reinterpret_cast<float4*>(p.S_last + ((size_t)bh * p.dout + n0 + n) * 128 + 64 * hh);
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        so[e] = make_float4(Sreg[4 * e], Sreg[4 * e + 1], Sreg[4 * e + 2], Sreg[4 * e + 3]);
+    }
   }
 
   tc_fence_before();

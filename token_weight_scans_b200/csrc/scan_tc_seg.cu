@@ -12,7 +12,9 @@
 //   reverse (adjoint Lam): Lam_end(nseg-1) = 0,
 //                          Lam_end(k) = 2^{L_{k+1}} Lam_end(k+1) + Lloc_{k+1}
 // The recursion runs element by element in fp32: one thread per element of the
-// d_out x d_in matrix, looping over the segments of its scan.
+// d_out x d_in matrix, looping over the segments of its scan. A carried start
+// state (forward) or an adjoint flowing in at the sequence's end (reverse)
+// replaces the zero that enters the first segment walked.
 
 #include <cuda_runtime.h>
 
@@ -23,12 +25,13 @@ namespace gradlev {
 namespace tc {
 
 __global__ void combine_kernel(const float* __restrict__ loc, const float* __restrict__ segL,
-                               float* __restrict__ out, int nseg, int per_scan, int reverse) {
+                               const float* __restrict__ init, float* __restrict__ out, int nseg,
+                               int per_scan, int reverse) {
   const int scan = blockIdx.y;
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= per_scan) return;
   const size_t base = (size_t)scan * nseg;
-  float acc = 0.f;
+  float acc = init ? init[(size_t)scan * per_scan + e] : 0.f;
   for (int i = 0; i < nseg; ++i) {
     const int k = reverse ? nseg - 1 - i : i;
     const size_t at = (base + k) * per_scan + e;
@@ -38,10 +41,10 @@ __global__ void combine_kernel(const float* __restrict__ loc, const float* __res
   }
 }
 
-cudaError_t combine_segments(const float* loc, const float* segL, float* out, int scans, int nseg,
-                             int per_scan, int reverse, cudaStream_t st) {
+cudaError_t combine_segments(const float* loc, const float* segL, const float* init, float* out,
+                             int scans, int nseg, int per_scan, int reverse, cudaStream_t st) {
   const dim3 grid((per_scan + 255) / 256, scans);
-  combine_kernel<<<grid, 256, 0, st>>>(loc, segL, out, nseg, per_scan, reverse);
+  combine_kernel<<<grid, 256, 0, st>>>(loc, segL, init, out, nseg, per_scan, reverse);
   count_launch();
   return cudaGetLastError();
 }
