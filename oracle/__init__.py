@@ -56,6 +56,7 @@ def _load():
             lib.oracle_bwd_state_f64.argtypes = [I] * 5 + [P] * 14 + [I] * 3
             lib.oracle_serial_f64.argtypes = [I] * 5 + [P] * 7 + [I]
             lib.oracle_serial_c128.argtypes = [I] * 5 + [P] * 7 + [I]
+            lib.oracle_decode_f64.argtypes = [I] * 5 + [P] * 8 + [I]
             lib.oracle_max_threads.restype = I
             _lib = lib
     return _lib
@@ -184,3 +185,20 @@ def serial(x, v, eta, alpha, W0, nthreads: int = 0):
     f(B, H, T, din, dout, _p(x), _p(v), _p(eta), _p(alpha), _p(W0), _p(y), _p(gs),
       int(nthreads))
     return y, gs
+
+
+def decode(x, v, eta, alpha, W0, S, nthreads: int = 0):
+    """Deployment decode of T tokens from the carried deviation S ([B,H,d_out,d_in]).
+
+    Returns (y, g, S_after): outputs and costates [B,H,T,d_out], and the deviation after the
+    last token. S itself is not modified."""
+    x, v, eta, alpha, W0 = (_arr(a, np.float64) for a in (x, v, eta, alpha, W0))
+    B, H, T, din, dout = _dims(x, v)
+    assert eta.shape == alpha.shape == (B, H, T) and W0.shape == (H, dout, din)
+    S = np.array(S, dtype=np.float64, copy=True, order="C")
+    assert S.shape == (B, H, dout, din)
+    y = np.empty((B, H, T, dout))
+    g = np.empty((B, H, T, dout))
+    _load().oracle_decode_f64(B, H, T, din, dout, _p(x), _p(v), _p(eta), _p(alpha), _p(W0),
+                              _p(S), _p(y), _p(g), int(nthreads))
+    return y, g, S

@@ -209,6 +209,30 @@ void serial_head(int T, int din, int dout, const R* x, const R* v, const R* eta,
   }
 }
 
+// Deployment decode of one (b,h) pair (GradLev abstract: at deployment the
+// auxiliary predictor is discarded and the model updates itself by
+// token-by-token forward and backward passes; Cognaptus, same page, opening
+// section: deployment still runs a forward pass, a backward pass and a weight
+// update per token). For the single adapted layer with the synthetic test's
+// inner loss 0.5 ||W x_t - v_t||^2, one token is
+//     y_t = (W_0 + S) x_t,   g_t = y_t - v_t,   S <- alpha_t S - eta_t g_t x_t^T
+// with S the deviation carried between calls (in/out).
+template <class R>
+void decode_head(int T, int din, int dout, const R* x, const R* v, const R* eta,
+                 const R* alpha, const R* W0, R* S, R* y, R* g) {
+  for (int t = 0; t < T; ++t) {
+    const R* xt = x + (size_t)t * din;
+    for (int n = 0; n < dout; ++n) {
+      R acc(0);
+      for (int k = 0; k < din; ++k)
+        acc += (W0[(size_t)n * din + k] + S[(size_t)n * din + k]) * xt[k];
+      y[(size_t)t * dout + n] = acc;
+      g[(size_t)t * dout + n] = acc - v[(size_t)t * dout + n];
+    }
+    state_step(din, dout, S, alpha[t], eta[t], g + (size_t)t * dout, xt);
+  }
+}
+
 inline int pick_threads(int nthreads) {
 #ifdef _OPENMP
   return nthreads > 0 ? nthreads : omp_get_max_threads();
@@ -366,6 +390,23 @@ void oracle_serial_c128(int B, int H, int T, int din, int dout, const double* x,
                    reinterpret_cast<const cplx*>(v), reinterpret_cast<const cplx*>(eta),
                    reinterpret_cast<const cplx*>(alpha), reinterpret_cast<const cplx*>(W0),
                    reinterpret_cast<cplx*>(y), reinterpret_cast<cplx*>(gstar), nthreads);
+}
+
+// Deployment decode of T tokens per pair (see decode_head): S [B,H,d_out,d_in]
+// is read and overwritten with the deviation after the last token; y and g
+// [B,H,T,d_out] receive the outputs and the costates.
+void oracle_decode_f64(int B, int H, int T, int din, int dout, const double* x, const double* v,
+                       const double* eta, const double* alpha, const double* W0, double* S,
+                       double* y, double* g, int nthreads) {
+  const int nt = pick_threads(nthreads);
+  const size_t dd = (size_t)din * dout;
+#pragma omp parallel for num_threads(nt) schedule(dynamic, 1)
+  for (int bh = 0; bh < B * H; ++bh) {
+    const int b = bh / H, h = bh % H;
+    const size_t o = at3(b, h, 0, H, T);
+    decode_head<double>(T, din, dout, x + o * din, v + o * dout, eta + o, alpha + o,
+                        W0 + (size_t)h * dd, S + (size_t)bh * dd, y + o * dout, g + o * dout);
+  }
 }
 
 int oracle_max_threads(void) { return pick_threads(0); }

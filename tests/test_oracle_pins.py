@@ -29,7 +29,14 @@ independent statement of what the GradLev scan must compute:
     which must equal the whole sequence;
   - derivative checks of every output, dS_0 included, for the objective
     with the <Lam_T, S_T> term;
-  - closed-form special cases (static gates; alpha_0 = 0 cuts S_0 off).
+  - closed-form special cases (static gates; alpha_0 = 0 cuts S_0 off);
+* the deployment decode (GradLev abstract: token-by-token forward and backward
+  passes at deployment). It is pinned by
+  - the serial learner, which reaches the same numbers in a different form;
+  - the closed form of one step;
+  - token-by-token calls, which must equal one call;
+  - exact recovery: the scan given the decode's costates reproduces its
+    outputs and end state.
 """
 
 import json
@@ -442,3 +449,56 @@ def test_state_special_cases_closed_form():
     o = oracle.bwd_state(cut["x"], cut["g"], cut["eta"], cut["alpha"], cut["W0"], cut["dy"],
                          S0=S0, LamT=LamT)
     assert rel(o["dS0"][0, 0], np.outer(u[0], x[0])) < 1e-14
+
+
+# --------------------------------------------------------------------------- deployment decode
+
+
+def _decode_inputs(B=2, H=2, T=9, d_in=5, d_out=4, seed=61):
+    d = tiny(B=B, H=H, T=T, d_in=d_in, d_out=d_out, seed=seed, with_v=True)
+    S0 = np.random.default_rng(seed + 7).standard_normal((B, H, d_out, d_in)) * 0.3
+    return d, S0
+
+
+def test_decode_equals_serial_learner():
+    d, _ = _decode_inputs()
+    B, H, T, din = d["x"].shape
+    zero = np.zeros((B, H, d["v"].shape[-1], din))
+    y, g, _ = oracle.decode(d["x"], d["v"], d["eta"], d["alpha"], d["W0"], zero)
+    ys, gs = oracle.serial(d["x"], d["v"], d["eta"], d["alpha"], d["W0"])
+    assert rel(y, ys) < 1e-14 and rel(g, gs) < 1e-14
+
+
+def test_decode_single_step_closed_form():
+    d, S0 = _decode_inputs(T=1)
+    y, g, S1 = oracle.decode(d["x"], d["v"], d["eta"], d["alpha"], d["W0"], S0)
+    B, H = S0.shape[:2]
+    for b in range(B):
+        for h in range(H):
+            x, v = d["x"][b, h, 0], d["v"][b, h, 0]
+            yc = (d["W0"][h] + S0[b, h]) @ x
+            gc = yc - v
+            Sc = d["alpha"][b, h, 0] * S0[b, h] - d["eta"][b, h, 0] * np.outer(gc, x)
+            assert rel(y[b, h, 0], yc) < 1e-15 and rel(g[b, h, 0], gc) < 1e-14
+            assert rel(S1[b, h], Sc) < 1e-15
+
+
+def test_decode_token_by_token_equals_one_call():
+    d, S0 = _decode_inputs(T=7)
+    y, g, S = oracle.decode(d["x"], d["v"], d["eta"], d["alpha"], d["W0"], S0)
+    St = S0
+    for t in range(7):
+        sl = lambda a: a[:, :, t:t + 1]
+        yt, gt, St = oracle.decode(sl(d["x"]), sl(d["v"]), sl(d["eta"]), sl(d["alpha"]),
+                                   d["W0"], St)
+        assert np.array_equal(yt, y[:, :, t:t + 1]) and np.array_equal(gt, g[:, :, t:t + 1])
+    assert np.array_equal(St, S)
+
+
+def test_scan_with_decode_costates_recovers_decode():
+    """Exact recovery with a carried state: the scan driven by the decode's own costates
+    reproduces its outputs and its end deviation."""
+    d, S0 = _decode_inputs(T=13)
+    y, g, S = oracle.decode(d["x"], d["v"], d["eta"], d["alpha"], d["W0"], S0)
+    ys, Ss = oracle.fwd_state(d["x"], g, d["eta"], d["alpha"], d["W0"], S0)
+    assert rel(ys, y) < 1e-13 and rel(Ss, S) < 1e-13
