@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--config IDX] [--no-e2e] [--no-cpu-baseline]
+    python bench.py --decode [--steps K] [--warmup W] [--T TOKENS_PER_CALL]
 
 One step = one forward scan (with state checkpoints) + one reverse scan over
 one batch of the workload, i.e. every step of the hot path. The default
@@ -16,6 +17,12 @@ over the batch). Time is taken on the device with CUDA events, max over ranks.
 
 ``--impl reference`` times the float64 CPU oracle on a bounded sample of the
 same workload on rank 0 (other ranks exit at once).
+
+``--decode`` measures the deployment decode step instead and prints its own
+line. The shape is B8 H16 d128 bf16, one token per call unless --T says more.
+The states and weights of 16 layers are rotated, 134 MB in all, more than the
+L2. The call loop is captured in a CUDA graph; the plain-launch time is
+reported beside it.
 """
 
 from __future__ import annotations
@@ -52,6 +59,7 @@ def parse():
     p.add_argument("--B", type=int, default=None, help="override B (reduced profiling case)")
     p.add_argument("--H", type=int, default=None, help="override H (reduced profiling case)")
     p.add_argument("--T", type=int, default=None, help="override T (reduced profiling case)")
+    p.add_argument("--decode", action="store_true", help="time the deployment decode step")
     return p.parse_args()
 
 
@@ -225,8 +233,96 @@ def run_reference(args, cfg):
     print(json.dumps(line), flush=True)
 
 
+def run_decode(args):
+    """Deployment decode: one gradlev_decode_step call per layer per token."""
+    import torch
+
+    import token_weight_scans_b200 as tw
+    from token_weight_scans_b200 import build as tw_build
+    from token_weight_scans_b200 import inputs
+    torch.cuda.set_device(0)
+    tw_build.build()
+    tw.lib()
+    B, H, d = args.B or 8, args.H or 16, 128
+    T = args.T or 1
+    layers = 16
+    dev = torch.device("cuda", 0)
+    lay = []
+    for l in range(layers):
+        dr = inputs.draw(B, H, T, d, d, dtype="bf16", alpha_mode="sigmoid", seed=5000 + l,
+                         with_v=True)
+        t = {k: torch.from_numpy(v).to(dev) for k, v in dr.items()}
+        for k in ("x", "v"):
+            t[k] = t[k].to(torch.bfloat16)
+        t["S"] = torch.zeros((B, H, d, d), dtype=torch.float32, device=dev)
+        t["y"] = torch.empty((B, H, T, d), dtype=torch.bfloat16, device=dev)
+        t["g"] = torch.empty_like(t["y"])
+        lay.append(t)
+
+    def call(t):
+        tw.gradlev_decode_step(t["x"], t["v"], t["eta"], t["alpha"], t["W0"], t["S"], y=t["y"],
+                               g=t["g"])
+
+    K = max(1, args.steps) * layers
+    for i in range(max(3, args.warmup) * layers):
+        call(lay[i % layers])
+    torch.cuda.synchronize()
+    s0, e0 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record()
+    for i in range(K):
+        call(lay[i % layers])
+    e0.record()
+    torch.cuda.synchronize()
+    plain_us = s0.elapsed_time(e0) * 1e3 / K
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            for i in range(K):
+                call(lay[i % layers])
+    torch.cuda.current_stream().wait_stream(side)
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    s1, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 5
+    s1.record()
+    for _ in range(reps):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    us = s1.elapsed_time(e1) * 1e3 / (reps * K)
+    peaks, peak_src = load_peaks()
+    # algorithmic bytes of one call: S read and written, W0 read, the token vectors
+    byt = B * H * d * d * 4 * 2 + H * d * d * 4 + B * H * T * d * 2 * 4 + B * H * T * 8
+    gbs = byt / (us * 1e-6) / 1e9
+    line = {"metric": "GradLev deployment decode: tokens/s through 16 adapted layers on 1 B200 "
+                      f"(B{B} H{H} d{d} bf16, {T} token(s) per call)",
+            "value": B * T / (us * 1e-6 * layers), "unit": "tokens/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "us_per_call": us,
+            "us_per_call_plain_launch": plain_us, "higher_is_better": True,
+            "dtype": "bf16", "data": "synthetic (seeded generator)",
+            "config": {"workload": "decode", "B": B, "H": H, "T_per_call": T, "d_in": d,
+                       "d_out": d, "layers": layers, "cuda_graph": True,
+                       "l2": f"no flush: {layers} layers' S and W0 "
+                             f"({layers * (B * H + H) * d * d * 4 / 1e6:.0f} MB) > 126 MB L2"},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                         "alg_bytes_per_launch": byt, "kernel": "decode_kernel",
+                         "peak_source": peak_src},
+            "clocks": clk, "gpu_launches": reps * K}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
+    if args.decode:
+        return run_decode(args)
     from token_weight_scans_b200 import inputs
     cfg = inputs.CONFIGS[args.config]
     over = {k: getattr(args, k) for k in ("B", "H", "T") if getattr(args, k) is not None}

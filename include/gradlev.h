@@ -180,6 +180,35 @@ GRADLEV_API gradlev_status gradlev_scan_bwd_state(int B, int H, int T, int d_in,
                                       float* dW0, float* dS0, const void* ckpt,
                                       void* workspace, size_t ws_bytes, void* stream);
 
+/* Deployment decode: T tokens of the token-by-token learner, in order.
+ *
+ * The GradLev abstract states that the auxiliary predictor is discarded at
+ * deployment, and the model then updates itself with token-by-token forward and
+ * backward passes. Cognaptus, "Parallelize the Training, Keep the Learning
+ * Serial", opening section, says the same: each token costs a forward pass, a
+ * backward pass and a weight update. For one adapted linear layer with the inner
+ * loss 0.5 ||W x_t - v_t||^2 of the pages' synthetic test, each token is
+ *   y_t = (W0 + S) x_t,   g_t = y_t - v_t,   S <- alpha_t S - eta_t g_t x_t^T.
+ * S is the deviation from W0, carried between calls. With S = 0 before the
+ * first token, this reproduces the serial online learner the scans recover.
+ *
+ *   x [B,H,T,d_in], v [B,H,T,d_out] (targets), y and g [B,H,T,d_out]: dtype.
+ *   eta, alpha [B,H,T]: float32. W0 [H,d_out,d_in]: float32.
+ *   S [B,H,d_out,d_in]: float32, read and overwritten with the deviation after
+ *     the last token.
+ *   g: NULL (costates not written), or the buffer that receives them.
+ * Constraints:
+ *   - d_in must be a multiple of 4 and at most 256, else
+ *     GRADLEV_ERR_UNSUPPORTED. Any d_out >= 1 is accepted.
+ *   - Alignment, else GRADLEV_ERR_INVALID_ARG: x to 4 elements; v, y and g to
+ *     one element; W0 and S to 16 bytes.
+ *   - One launch; no workspace; no device waits; nothing is allocated.
+ *   - The buffers are the caller's. y and g may not alias the inputs. */
+GRADLEV_API gradlev_status gradlev_decode_step(int B, int H, int T, int d_in, int d_out,
+                                   gradlev_dtype dt, const void* x, const void* v,
+                                   const float* eta, const float* alpha, const float* W0,
+                                   float* S, void* y, void* g, void* stream);
+
 /* Size of the static scratch array gradlev_scan_bwd_noalloc uses: 64 MiB,
  * held by every GPU that loads the library until the process exits. */
 #define GRADLEV_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)

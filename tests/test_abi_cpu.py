@@ -31,7 +31,7 @@ def test_header_declares_the_entry_points():
     for n in ("gradlev_scan_fwd", "gradlev_scan_bwd", "gradlev_scan_workspace_bytes",
               "gradlev_status_string", "gradlev_scan_supported", "gradlev_scan_ckpt_bytes",
               "gradlev_device_status", "gradlev_last_launch_count", "gradlev_scan_fwd_state",
-              "gradlev_scan_bwd_state"):
+              "gradlev_scan_bwd_state", "gradlev_decode_step"):
         assert n in names, n
 
 
@@ -149,3 +149,17 @@ def test_state_entry_points_validate_before_launch(L):
     # the required pointers are still required
     assert L.gradlev_scan_fwd_state(1, 1, 8, 16, 16, 0, P(0), fake, fake, fake, fake, P(0), fake,
                                     P(0), P(0), fake, 1 << 20, P(0)) == 1
+
+
+def test_decode_step_validates_before_launch(L):
+    P = ctypes.c_void_p
+    fake = P(4096)
+    L.gradlev_decode_step.restype = ctypes.c_int
+    call = lambda d_in=16, d_out=8, x=fake, S=fake, T=1: L.gradlev_decode_step(
+        1, 1, T, d_in, d_out, 1, x, fake, fake, fake, fake, S, fake, P(0), P(0))
+    assert call(d_in=18) == 2            # d_in not a multiple of 4
+    assert call(d_in=260) == 2           # d_in above 256
+    assert call(T=0) == 1                # empty
+    assert call(x=P(0)) == 1             # missing input
+    assert call(x=P(4098)) == 1          # bf16 x not aligned to 4 elements
+    assert call(S=P(4104)) == 1          # S not 16-byte aligned

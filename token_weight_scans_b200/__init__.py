@@ -17,7 +17,7 @@ __all__ = [
     "GradlevError", "lib", "gradlev_status_string", "gradlev_scan_supported",
     "gradlev_scan_workspace_bytes", "gradlev_scan_ckpt_bytes", "gradlev_scan_fwd",
     "gradlev_scan_bwd", "gradlev_scan_fwd_state", "gradlev_scan_bwd_state",
-    "gradlev_device_status", "gradlev_last_launch_count", "F32", "BF16", "LIB_PATH",
+    "gradlev_decode_step", "gradlev_device_status", "gradlev_last_launch_count", "F32", "BF16", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgradlev.so")
@@ -27,8 +27,8 @@ BF16 = 1
 _ENTRY_POINTS = (
     "gradlev_status_string", "gradlev_scan_supported", "gradlev_scan_workspace_bytes",
     "gradlev_scan_ckpt_bytes", "gradlev_scan_fwd", "gradlev_scan_bwd",
-    "gradlev_scan_fwd_state", "gradlev_scan_bwd_state", "gradlev_device_status",
-    "gradlev_last_launch_count",
+    "gradlev_scan_fwd_state", "gradlev_scan_bwd_state", "gradlev_decode_step",
+    "gradlev_device_status", "gradlev_last_launch_count",
 )
 
 
@@ -72,6 +72,8 @@ def lib():
     L.gradlev_scan_fwd_state.restype = I
     L.gradlev_scan_bwd_state.argtypes = [I] * 6 + [P] * 16 + [Z, P]
     L.gradlev_scan_bwd_state.restype = I
+    L.gradlev_decode_step.argtypes = [I] * 6 + [P] * 9
+    L.gradlev_decode_step.restype = I
     L.gradlev_device_status.argtypes = [P, P]
     L.gradlev_device_status.restype = I
     L.gradlev_last_launch_count.argtypes = []
@@ -283,6 +285,34 @@ def gradlev_scan_bwd_state(x, g, eta, alpha, W0, dy, S0=None, LamT=None, *, ckpt
                                       _stream_ptr(stream))
     _check(st, "gradlev_scan_bwd_state")
     return out
+
+
+def gradlev_decode_step(x, v, eta, alpha, W0, S, *, y=None, g=None, want_g=True, stream=None):
+    """Deployment decode of the T tokens of x in order, from the carried deviation S
+    ([B,H,d_out,d_in] float32, updated in place). Returns (y, g): outputs and costates
+    [B,H,T,d_out] (g is None when want_g is False and no buffer is given)."""
+    import torch
+    B, H, T, d_in, d_out = _dims(x, v)
+    dev, dt = x.device, x.dtype
+    f32 = torch.float32
+    _check_tensor("x", x, (B, H, T, d_in), dt, dev)
+    _check_tensor("v", v, (B, H, T, d_out), dt, dev)
+    _check_tensor("eta", eta, (B, H, T), f32, dev)
+    _check_tensor("alpha", alpha, (B, H, T), f32, dev)
+    _check_tensor("W0", W0, (H, d_out, d_in), f32, dev)
+    _check_tensor("S", S, (B, H, d_out, d_in), f32, dev)
+    if y is None:
+        y = torch.empty((B, H, T, d_out), dtype=dt, device=dev)
+    _check_tensor("y", y, (B, H, T, d_out), dt, dev)
+    if g is None and want_g:
+        g = torch.empty((B, H, T, d_out), dtype=dt, device=dev)
+    if g is not None:
+        _check_tensor("g", g, (B, H, T, d_out), dt, dev)
+    st = lib().gradlev_decode_step(B, H, T, d_in, d_out, _dt_code(dt), _ptr(x), _ptr(v),
+                                   _ptr(eta), _ptr(alpha), _ptr(W0), _ptr(S), _ptr(y), _ptr(g),
+                                   _stream_ptr(stream))
+    _check(st, "gradlev_decode_step")
+    return y, g
 
 
 def gradlev_device_status(workspace, stream=None) -> int:

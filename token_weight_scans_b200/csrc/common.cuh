@@ -26,7 +26,9 @@ struct DeviceStatus {
   unsigned int pad[2];
 };
 
-// Launch accounting for gradlev_last_launch_count().
+// Launch accounting for gradlev_last_launch_count(): every entry point resets the
+// count, every kernel launch adds one.
 void count_launch();
+void reset_launch_count();
 
 }  // namespace gradlev

@@ -24,6 +24,7 @@ namespace gradlev {
 
 static thread_local int t_launches = 0;
 void count_launch() { ++t_launches; }
+void reset_launch_count() { t_launches = 0; }
 
 // Test hook state (gradlev_debug_inject_timeout): consumed by the next fwd call.
 static int g_inject = 0;
