@@ -202,3 +202,35 @@ def decode(x, v, eta, alpha, W0, S, nthreads: int = 0):
     _load().oracle_decode_f64(B, H, T, din, dout, _p(x), _p(v), _p(eta), _p(alpha), _p(W0),
                               _p(S), _p(y), _p(g), int(nthreads))
     return y, g, S
+
+
+def consistency(x, ghat, eta, alpha, W0, v, lam: float = 1.0, nthreads: int = 0):
+    """One GradLev training step of the single adapted layer, given predicted costates.
+
+    Cognaptus, "Parallelize the Training, Keep the Learning Serial", section "The
+    predictor is constrained by the learner it is supposed to reproduce":
+    - the forward runs on the predicted costates ghat;
+    - the costates the proposed trajectory implies are reconstructed by
+      backpropagating through the layer. For the synthetic test's inner loss
+      0.5 ||y - v||^2 that is gtil_t = y_t - v_t;
+    - training combines the token loss with a consistency term that pushes ghat
+      toward gtil.
+
+    The term's formula is missing from the page. Read as written, with gtil as the
+    target (no gradient through it):
+        L = sum_t 0.5 ||gtil_t||^2 + lam ||ghat_t - gtil_t||^2.
+    The token loss's output gradient is gtil itself, so its gradients are the reverse
+    scan with dy = gtil. The consistency term adds 2 lam (ghat - gtil) to d ghat.
+
+    Returns a dict with:
+    - y, gtil, r = ghat - gtil;
+    - loss_tok and loss_c, per token [B,H,T];
+    - dx, dghat, deta, dalpha, dW0, and dv = -gtil."""
+    x, ghat, eta, alpha, W0, v = (_arr(a, np.float64) for a in (x, ghat, eta, alpha, W0, v))
+    y = fwd(x, ghat, eta, alpha, W0, nthreads=nthreads)
+    gtil = y - v
+    r = ghat - gtil
+    o = bwd(x, ghat, eta, alpha, W0, gtil, nthreads=nthreads)
+    return dict(y=y, gtil=gtil, r=r, loss_tok=0.5 * np.sum(gtil * gtil, axis=-1),
+                loss_c=np.sum(r * r, axis=-1), dx=o["dx"], dghat=o["dg"] + 2.0 * lam * r,
+                deta=o["deta"], dalpha=o["dalpha"], dW0=o["dW0"], dv=-gtil)

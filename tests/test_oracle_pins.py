@@ -36,7 +36,13 @@ independent statement of what the GradLev scan must compute:
   - the closed form of one step;
   - token-by-token calls, which must equal one call;
   - exact recovery: the scan given the decode's costates reproduces its
-    outputs and end state.
+    outputs and end state;
+* the consistency step (section "The predictor is constrained by the learner
+  it is supposed to reproduce"). It is pinned by
+  - the fixed point: with the serial learner's true costates the residual,
+    the consistency loss and its gradient vanish;
+  - complex-step derivatives of the token loss;
+  - the closed form of one token.
 """
 
 import json
@@ -502,3 +508,64 @@ def test_scan_with_decode_costates_recovers_decode():
     y, g, S = oracle.decode(d["x"], d["v"], d["eta"], d["alpha"], d["W0"], S0)
     ys, Ss = oracle.fwd_state(d["x"], g, d["eta"], d["alpha"], d["W0"], S0)
     assert rel(ys, y) < 1e-13 and rel(Ss, S) < 1e-13
+
+
+# --------------------------------------------------------------------------- consistency step
+
+
+def test_consistency_vanishes_at_the_serial_costates():
+    """Exact consistency: feeding the serial learner's true costates as the prediction
+    gives a zero residual, so the consistency term and its gradient vanish."""
+    d = tiny(B=2, H=2, T=15, d_in=5, d_out=4, seed=71, with_v=True)
+    _, gstar = oracle.serial(d["x"], d["v"], d["eta"], d["alpha"], d["W0"])
+    c = oracle.consistency(d["x"], gstar, d["eta"], d["alpha"], d["W0"], d["v"], lam=3.0)
+    scale = np.max(np.abs(gstar))
+    assert np.max(np.abs(c["r"])) < 1e-14 * scale
+    assert np.max(c["loss_c"]) < 1e-27 * scale ** 2
+    tok = oracle.bwd(d["x"], gstar, d["eta"], d["alpha"], d["W0"], c["gtil"])["dg"]
+    assert np.max(np.abs(c["dghat"] - tok)) < 1e-13 * max(np.max(np.abs(tok)), 1.0)
+    # and away from the fixed point the residual is not small
+    c2 = oracle.consistency(d["x"], gstar * 0.5, d["eta"], d["alpha"], d["W0"], d["v"])
+    assert np.max(np.abs(c2["r"])) > 1e-2 * scale
+
+
+def _token_loss(d, ghat, over=None):
+    over = over or {}
+    a = {k: over.get(k, d[k]) for k in ("x", "eta", "alpha", "W0", "v")}
+    gh = over.get("ghat", ghat)
+    y = oracle.fwd(a["x"], gh, a["eta"], a["alpha"], a["W0"])
+    gt = y - a["v"]
+    return 0.5 * np.sum(gt * gt)
+
+
+def test_consistency_token_loss_gradients_complex_step():
+    d = tiny(B=1, H=2, T=6, d_in=3, d_out=2, seed=73, with_v=True)
+    ghat = np.random.default_rng(74).standard_normal(d["v"].shape)
+    lam = 0.7
+    c = oracle.consistency(d["x"], ghat, d["eta"], d["alpha"], d["W0"], d["v"], lam=lam)
+    names = dict(x="dx", ghat="dghat", eta="deta", alpha="dalpha", W0="dW0", v="dv")
+    for p, k in names.items():
+        base = ghat if p == "ghat" else d[p]
+        gr = np.zeros_like(base)
+        for idx in np.ndindex(base.shape):
+            z = base.astype(np.complex128)
+            z[idx] += 1e-30j
+            gr[idx] = np.imag(_token_loss(d, ghat, {p: z})) / 1e-30
+        got = c[k] - (2.0 * lam * c["r"] if p == "ghat" else 0.0)  # the stop-gradient term
+        assert rel(got, gr) < 1e-12, (p, rel(got, gr))
+
+
+def test_consistency_single_token_closed_form():
+    d = tiny(B=1, H=1, T=1, d_in=4, d_out=3, seed=75, with_v=True)
+    ghat = np.random.default_rng(76).standard_normal(d["v"].shape)
+    c = oracle.consistency(d["x"], ghat, d["eta"], d["alpha"], d["W0"], d["v"], lam=2.0)
+    x, v, W0 = d["x"][0, 0, 0], d["v"][0, 0, 0], d["W0"][0]
+    gt = W0 @ x - v                      # S_0 = 0: y_0 = W0 x_0
+    r = ghat[0, 0, 0] - gt
+    assert rel(c["gtil"][0, 0, 0], gt) < 1e-15
+    assert abs(c["loss_tok"][0, 0, 0] - 0.5 * gt @ gt) < 1e-14 * (gt @ gt)
+    assert abs(c["loss_c"][0, 0, 0] - r @ r) < 1e-14 * (r @ r)
+    # one token: dx = W0^T gtil, d ghat = 2 lam r (g only feeds later tokens), dW0 = gtil x^T
+    assert rel(c["dx"][0, 0, 0], W0.T @ gt) < 1e-15
+    assert rel(c["dghat"][0, 0, 0], 4.0 * r) < 1e-15
+    assert rel(c["dW0"][0], np.outer(gt, x)) < 1e-15
