@@ -3,6 +3,7 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--config IDX] [--no-e2e] [--no-cpu-baseline]
     python bench.py --decode [--steps K] [--warmup W] [--T TOKENS_PER_CALL]
+    python bench.py --consistency [--steps K] [--warmup W] [--config IDX]
 
 One step = one forward scan (with state checkpoints) + one reverse scan over
 one batch of the workload, i.e. every step of the hot path. The default
@@ -23,6 +24,11 @@ line. The shape is B8 H16 d128 bf16, one token per call unless --T says more.
 The states and weights of 16 layers are rotated, 134 MB in all, more than the
 L2. The call loop is captured in a CUDA graph; the plain-launch time is
 reported beside it.
+
+``--consistency`` times gradlev_consistency_step on the workload's shape. One
+call is a whole training step from predicted costates: the forward, the
+reconstructed costates and losses, the reverse scan, and the consistency
+gradient. It prints its own line.
 """
 
 from __future__ import annotations
@@ -60,6 +66,8 @@ def parse():
     p.add_argument("--H", type=int, default=None, help="override H (reduced profiling case)")
     p.add_argument("--T", type=int, default=None, help="override T (reduced profiling case)")
     p.add_argument("--decode", action="store_true", help="time the deployment decode step")
+    p.add_argument("--consistency", action="store_true",
+                   help="time the consistency training step")
     return p.parse_args()
 
 
@@ -319,10 +327,79 @@ def run_decode(args):
     print(json.dumps(line), flush=True)
 
 
+def run_consistency(args):
+    """gradlev_consistency_step on the workload's shape (inputs resident in HBM)."""
+    import torch
+
+    import token_weight_scans_b200 as tw
+    from token_weight_scans_b200 import build as tw_build
+    from token_weight_scans_b200 import inputs
+    torch.cuda.set_device(0)
+    tw_build.build()
+    tw.lib()
+    cfg = inputs.CONFIGS[args.config]
+    B, H, T, di, do = cfg.B, cfg.H, cfg.T, cfg.d_in, cfg.d_out
+    tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    es = 2 if cfg.dtype == "bf16" else 4
+    d = inputs.draw(B, H, T, di, do, dtype=cfg.dtype, alpha_mode=cfg.alpha_mode, seed=77,
+                    with_v=True)
+    t = {k: torch.from_numpy(v).cuda() for k, v in d.items()}
+    for k in ("x", "g", "v"):
+        t[k] = t[k].to(tdt)
+    code = tw.BF16 if cfg.dtype == "bf16" else tw.F32
+    ws = torch.empty(tw.gradlev_consistency_workspace_bytes(B, H, T, di, do, code),
+                     dtype=torch.uint8, device="cuda")
+    out = None
+
+    def step():
+        nonlocal out
+        out = tw.gradlev_consistency_step(t["x"], t["g"], t["eta"], t["alpha"], t["W0"], t["v"],
+                                          1.0, workspace=ws, out=out)
+        return tw.gradlev_last_launch_count()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    s0, e0 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches = 0
+    s0.record()
+    for _ in range(args.steps):
+        launches += step()
+    e0.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = s0.elapsed_time(e0) / args.steps
+    peaks, peak_src = load_peaks()
+    N = B * H * T
+    ab = alg_bytes(cfg, es)
+    # residual: y, ghat, v read, gtil and dv written, two losses; finish: dg, ghat, gtil
+    # read, dg written
+    extra = N * do * es * (5 + 4) + N * 8
+    byt = ab["fwd"] + ab["bwd"] + extra
+    gbs = byt / (ms * 1e-3) / 1e9
+    line = {"metric": f"GradLev consistency training step tokens/s on 1 B200 ({cfg.name})",
+            "value": B * T / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "dtype": cfg.dtype, "data": "synthetic (seeded generator)",
+            "config": {"workload": "consistency step, " + cfg.name, "B": B, "H": H, "T": T,
+                       "d_in": di, "d_out": do,
+                       "l2": f"no flush: {byt / 1e6:.0f} MB per step > 126 MB L2"},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                         "alg_bytes_per_step": byt, "peak_source": peak_src},
+            "clocks": clk, "gpu_launches": launches}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.decode:
         return run_decode(args)
+    if args.consistency:
+        return run_consistency(args)
     from token_weight_scans_b200 import inputs
     cfg = inputs.CONFIGS[args.config]
     over = {k: getattr(args, k) for k in ("B", "H", "T") if getattr(args, k) is not None}

@@ -209,6 +209,49 @@ GRADLEV_API gradlev_status gradlev_decode_step(int B, int H, int T, int d_in, in
                                    const float* eta, const float* alpha, const float* W0,
                                    float* S, void* y, void* g, void* stream);
 
+/* One training step of the adapted layer from predicted costates: the forward
+ * scan, the reconstructed costates, the token and consistency losses, and every
+ * gradient of their sum.
+ *
+ * Cognaptus, "Parallelize the Training, Keep the Learning Serial", section "The
+ * predictor is constrained by the learner it is supposed to reproduce":
+ *   - the forward runs on the predicted costates ghat;
+ *   - the costates the proposed trajectory implies are reconstructed from it;
+ *   - training combines the token loss with a term that pushes ghat toward them.
+ * For the synthetic test's inner loss 0.5 ||y - v||^2 the reconstruction is
+ * gtil = y - v. The consistency term's formula is missing from the page; this
+ * call reads it as lam ||ghat - gtil||^2 with gtil the target (no gradient
+ * flows through gtil):
+ *   L = sum_t 0.5 ||gtil_t||^2 + lam ||ghat_t - gtil_t||^2.
+ *
+ * Outputs (all written):
+ *   y, gtil [B,H,T,d_out] (dtype)    loss_tok, loss_c [B,H,T] float32 (per token)
+ *   dx [B,H,T,d_in] (dtype)          dghat [B,H,T,d_out] (dtype): gradient w.r.t. ghat
+ *   d_eta, d_alpha [B,H,T] float32   dW0 [H,d_out,d_in] float32
+ *   dv [B,H,T,d_out] (dtype) = -gtil, or NULL (not written).
+ * The token loss's output gradient is gtil, so dx, d_eta, d_alpha and dW0 are
+ * the reverse scan with dy = gtil. The consistency term adds 2 lam (ghat - gtil)
+ * to dghat.
+ *
+ * Requirements, else the status shown:
+ *   - d_out a multiple of 4, and the shapes of gradlev_scan_fwd
+ *     (GRADLEV_ERR_UNSUPPORTED);
+ *   - workspace at least gradlev_consistency_workspace_bytes() bytes
+ *     (GRADLEV_ERR_WORKSPACE);
+ *   - alignment (GRADLEV_ERR_INVALID_ARG): workspace 256 bytes; x, ghat, y,
+ *     gtil, dx, dghat, W0 and dW0 16 bytes; v and dv 4 elements.
+ * Outputs may not alias inputs. gradlev_device_status(workspace) reports the
+ * bounded waits of all its launches. */
+GRADLEV_API size_t gradlev_consistency_workspace_bytes(int B, int H, int T, int d_in, int d_out,
+                                           gradlev_dtype dt);
+GRADLEV_API gradlev_status gradlev_consistency_step(int B, int H, int T, int d_in, int d_out,
+                                        gradlev_dtype dt, const void* x, const void* ghat,
+                                        const float* eta, const float* alpha, const float* W0,
+                                        const void* v, float lam, void* y, void* gtil,
+                                        float* loss_tok, float* loss_c, void* dx, void* dghat,
+                                        float* d_eta, float* d_alpha, float* dW0, void* dv,
+                                        void* workspace, size_t ws_bytes, void* stream);
+
 /* Size of the static scratch array gradlev_scan_bwd_noalloc uses: 64 MiB,
  * held by every GPU that loads the library until the process exits. */
 #define GRADLEV_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)

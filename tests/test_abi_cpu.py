@@ -31,7 +31,8 @@ def test_header_declares_the_entry_points():
     for n in ("gradlev_scan_fwd", "gradlev_scan_bwd", "gradlev_scan_workspace_bytes",
               "gradlev_status_string", "gradlev_scan_supported", "gradlev_scan_ckpt_bytes",
               "gradlev_device_status", "gradlev_last_launch_count", "gradlev_scan_fwd_state",
-              "gradlev_scan_bwd_state", "gradlev_decode_step"):
+              "gradlev_scan_bwd_state", "gradlev_decode_step", "gradlev_consistency_step",
+              "gradlev_consistency_workspace_bytes"):
         assert n in names, n
 
 
@@ -163,3 +164,27 @@ def test_decode_step_validates_before_launch(L):
     assert call(x=P(0)) == 1             # missing input
     assert call(x=P(4098)) == 1          # bf16 x not aligned to 4 elements
     assert call(S=P(4104)) == 1          # S not 16-byte aligned
+
+
+def test_consistency_step_validates_before_launch(L):
+    P = ctypes.c_void_p
+    fake = P(4096)
+    I, Z = ctypes.c_int, ctypes.c_size_t
+    L.gradlev_consistency_workspace_bytes.restype = Z
+    L.gradlev_consistency_workspace_bytes.argtypes = [I] * 6
+    L.gradlev_consistency_step.restype = I
+    L.gradlev_consistency_step.argtypes = [I] * 6 + [P] * 6 + [ctypes.c_float] + [P] * 11 + [Z, P]
+    nws = L.gradlev_consistency_workspace_bytes(2, 2, 100, 16, 16, 0)
+    # the reverse scan's scratch with its own states, plus the forward's checkpoints
+    assert nws >= L.gradlev_scan_workspace_bytes(2, 2, 100, 16, 16, 0, 1)
+    assert L.gradlev_consistency_workspace_bytes(2, 2, 100, 16, 18, 0) == 0  # d_out % 4
+    call = lambda v=fake, ws=fake, nbytes=1 << 30, d_out=16, dv=P(0): \
+        L.gradlev_consistency_step(2, 2, 100, 16, d_out, 0, fake, fake, fake, fake, fake, v, 1.0,
+                                   fake, fake, fake, fake, fake, fake, fake, fake, fake, dv, ws,
+                                   nbytes, P(0))
+    assert call(d_out=18) == 2           # d_out not a multiple of 4
+    assert call(v=P(0)) == 1             # missing input
+    assert call(v=P(4100)) == 1          # f32 v not 16-byte aligned
+    assert call(dv=P(4100)) == 1
+    assert call(ws=P(4096 + 16)) == 1    # workspace not 256-byte aligned
+    assert call(nbytes=16) == 3          # workspace too small

@@ -17,7 +17,8 @@ __all__ = [
     "GradlevError", "lib", "gradlev_status_string", "gradlev_scan_supported",
     "gradlev_scan_workspace_bytes", "gradlev_scan_ckpt_bytes", "gradlev_scan_fwd",
     "gradlev_scan_bwd", "gradlev_scan_fwd_state", "gradlev_scan_bwd_state",
-    "gradlev_decode_step", "gradlev_device_status", "gradlev_last_launch_count", "F32", "BF16", "LIB_PATH",
+    "gradlev_decode_step", "gradlev_consistency_workspace_bytes", "gradlev_consistency_step",
+    "gradlev_device_status", "gradlev_last_launch_count", "F32", "BF16", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgradlev.so")
@@ -28,6 +29,7 @@ _ENTRY_POINTS = (
     "gradlev_status_string", "gradlev_scan_supported", "gradlev_scan_workspace_bytes",
     "gradlev_scan_ckpt_bytes", "gradlev_scan_fwd", "gradlev_scan_bwd",
     "gradlev_scan_fwd_state", "gradlev_scan_bwd_state", "gradlev_decode_step",
+    "gradlev_consistency_workspace_bytes", "gradlev_consistency_step",
     "gradlev_device_status", "gradlev_last_launch_count",
 )
 
@@ -74,6 +76,11 @@ def lib():
     L.gradlev_scan_bwd_state.restype = I
     L.gradlev_decode_step.argtypes = [I] * 6 + [P] * 9
     L.gradlev_decode_step.restype = I
+    L.gradlev_consistency_workspace_bytes.argtypes = [I] * 6
+    L.gradlev_consistency_workspace_bytes.restype = Z
+    L.gradlev_consistency_step.argtypes = ([I] * 6 + [P] * 6 + [ctypes.c_float] + [P] * 11 +
+                                           [Z, P])
+    L.gradlev_consistency_step.restype = I
     L.gradlev_device_status.argtypes = [P, P]
     L.gradlev_device_status.restype = I
     L.gradlev_last_launch_count.argtypes = []
@@ -313,6 +320,49 @@ def gradlev_decode_step(x, v, eta, alpha, W0, S, *, y=None, g=None, want_g=True,
                                    _stream_ptr(stream))
     _check(st, "gradlev_decode_step")
     return y, g
+
+
+def gradlev_consistency_workspace_bytes(B, H, T, d_in, d_out, dt) -> int:
+    return int(lib().gradlev_consistency_workspace_bytes(B, H, T, d_in, d_out, dt))
+
+
+def gradlev_consistency_step(x, ghat, eta, alpha, W0, v, lam=1.0, *, want_dv=True,
+                             workspace=None, stream=None, out=None):
+    """One training step of the adapted layer from predicted costates ghat (see
+    include/gradlev.h). Returns dict y, gtil, loss_tok, loss_c, dx, dghat, deta, dalpha, dW0
+    and dv (None when want_dv is False)."""
+    import torch
+    B, H, T, d_in, d_out = _dims(x, ghat)
+    dev, dt = x.device, x.dtype
+    f32 = torch.float32
+    _check_tensor("x", x, (B, H, T, d_in), dt, dev)
+    _check_tensor("ghat", ghat, (B, H, T, d_out), dt, dev)
+    _check_tensor("v", v, (B, H, T, d_out), dt, dev)
+    _check_tensor("eta", eta, (B, H, T), f32, dev)
+    _check_tensor("alpha", alpha, (B, H, T), f32, dev)
+    _check_tensor("W0", W0, (H, d_out, d_in), f32, dev)
+    code = _dt_code(dt)
+    nws = gradlev_consistency_workspace_bytes(B, H, T, d_in, d_out, code)
+    if nws == 0:
+        raise GradlevError("gradlev_consistency_step: unsupported shape", 2)
+    if out is None:
+        out = dict(y=torch.empty_like(ghat), gtil=torch.empty_like(ghat),
+                   loss_tok=torch.empty((B, H, T), dtype=f32, device=dev),
+                   loss_c=torch.empty((B, H, T), dtype=f32, device=dev),
+                   dx=torch.empty_like(x), dghat=torch.empty_like(ghat),
+                   deta=torch.empty((B, H, T), dtype=f32, device=dev),
+                   dalpha=torch.empty((B, H, T), dtype=f32, device=dev),
+                   dW0=torch.empty((H, d_out, d_in), dtype=f32, device=dev),
+                   dv=torch.empty_like(ghat) if want_dv else None)
+    ws = _workspace(nws, dev, workspace)
+    st = lib().gradlev_consistency_step(
+        B, H, T, d_in, d_out, code, _ptr(x), _ptr(ghat), _ptr(eta), _ptr(alpha), _ptr(W0),
+        _ptr(v), float(lam), _ptr(out["y"]), _ptr(out["gtil"]), _ptr(out["loss_tok"]),
+        _ptr(out["loss_c"]), _ptr(out["dx"]), _ptr(out["dghat"]), _ptr(out["deta"]),
+        _ptr(out["dalpha"]), _ptr(out["dW0"]), _ptr(out.get("dv")), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream_ptr(stream))
+    _check(st, "gradlev_consistency_step")
+    return out
 
 
 def gradlev_device_status(workspace, stream=None) -> int:

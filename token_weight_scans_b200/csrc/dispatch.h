@@ -33,10 +33,12 @@ struct StateIO {
 // Launch the reverse scan with its scratch at `ws` (bwd_scratch_bytes(.., ckpt == NULL)
 // bytes, 256-byte aligned). Shapes and pointers must already be validated. io.S0 is read
 // only when ckpt is null (the forward sweep that recomputes the states starts from it).
+// clear_status = false keeps what earlier launches of the same call wrote into the
+// status word at the start of `ws`.
 gradlev_status bwd_run(int B, int H, int T, int din, int dout, gradlev_dtype dt, const void* x,
                        const void* g, const float* eta, const float* alpha, const float* W0,
                        const void* dy, void* dx, void* dg, float* d_eta, float* d_alpha,
                        float* dW0, const void* ckpt, char* ws, cudaStream_t st,
-                       const StateIO& io = StateIO{});
+                       const StateIO& io = StateIO{}, bool clear_status = true);
 
 }  // namespace gradlev

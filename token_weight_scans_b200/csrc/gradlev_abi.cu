@@ -17,6 +17,7 @@
 #include "common.cuh"
 #include "dispatch.h"
 #include "gradlev.h"
+#include "consistency.h"
 #include "scan_ffma.h"
 #include "scan_tc.h"
 
@@ -163,12 +164,12 @@ gradlev_status bwd_run(int B, int H, int T, int din, int dout, gradlev_dtype dt,
                        const void* g, const float* eta, const float* alpha, const float* W0,
                        const void* dy, void* dx, void* dg, float* d_eta, float* d_alpha,
                        float* dW0, const void* ckpt, char* ws, cudaStream_t st,
-                       const StateIO& io) {
+                       const StateIO& io, bool clear_status) {
   DeviceStatus* status = reinterpret_cast<DeviceStatus*>(ws);
   float* dW0_part = reinterpret_cast<float*>(ws + kStatusBytes);
   char* own = ws + kStatusBytes + dW0_part_bytes(B, H, T, din, dout, dt);
   char* seg_ws = own + (ckpt ? 0 : align_up(ckpt_bytes_of(B, H, T, din, dout, dt), 256));
-  if (cudaMemsetAsync(status, 0, sizeof(DeviceStatus), st) != cudaSuccess)
+  if (clear_status && cudaMemsetAsync(status, 0, sizeof(DeviceStatus), st) != cudaSuccess)
     return GRADLEV_ERR_CUDA;
   const void* states = ckpt;
   if (!states) {
@@ -355,6 +356,63 @@ gradlev_status gradlev_scan_bwd_state(int B, int H, int T, int d_in, int d_out, 
   io.dS0 = dS0;
   return bwd_entry(B, H, T, d_in, d_out, dt, x, g, eta, alpha, W0, dy, dx, dg, d_eta, d_alpha,
                    dW0, ckpt, workspace, ws_bytes, stream, io);
+}
+
+size_t gradlev_consistency_workspace_bytes(int B, int H, int T, int d_in, int d_out,
+                                           gradlev_dtype dt) {
+  if (check_shape(B, H, T, d_in, d_out, dt) != GRADLEV_OK || d_out % 4 != 0) return 0;
+  // the reverse scan's scratch, then the forward's checkpoints that it consumes
+  return bwd_scratch_bytes(B, H, T, d_in, d_out, dt, true) +
+         align_up(ckpt_bytes_of(B, H, T, d_in, d_out, dt), 256);
+}
+
+gradlev_status gradlev_consistency_step(int B, int H, int T, int d_in, int d_out,
+                                        gradlev_dtype dt, const void* x, const void* ghat,
+                                        const float* eta, const float* alpha, const float* W0,
+                                        const void* v, float lam, void* y, void* gtil,
+                                        float* loss_tok, float* loss_c, void* dx, void* dghat,
+                                        float* d_eta, float* d_alpha, float* dW0, void* dv,
+                                        void* workspace, size_t ws_bytes, void* stream) {
+  gradlev_status s = check_shape(B, H, T, d_in, d_out, dt);
+  if (s != GRADLEV_OK) return s;
+  if (d_out % 4 != 0) return GRADLEV_ERR_UNSUPPORTED;
+  if (!x || !ghat || !eta || !alpha || !W0 || !v || !y || !gtil || !loss_tok || !loss_c || !dx ||
+      !dghat || !d_eta || !d_alpha || !dW0 || !workspace)
+    return GRADLEV_ERR_INVALID_ARG;
+  const size_t ea = dt == GRADLEV_BF16 ? 8 : 16;  // 4-element vectors of the residual pass
+  if (!aligned(x, 16) || !aligned(ghat, 16) || !aligned(y, 16) || !aligned(dx, 16) ||
+      !aligned(dghat, 16) || !aligned(W0, 16) || !aligned(dW0, 16) || !aligned(v, ea) ||
+      !aligned(gtil, 16) || (dv && !aligned(dv, ea)) || !aligned(eta, 4) ||
+      !aligned(alpha, 4) || !aligned(d_eta, 4) || !aligned(d_alpha, 4) ||
+      !aligned(loss_tok, 4) || !aligned(loss_c, 4) || !aligned(workspace, 256))
+    return GRADLEV_ERR_INVALID_ARG;
+  if (ws_bytes < gradlev_consistency_workspace_bytes(B, H, T, d_in, d_out, dt))
+    return GRADLEV_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  t_launches = 0;
+  char* ws = static_cast<char*>(workspace);
+  DeviceStatus* status = reinterpret_cast<DeviceStatus*>(ws);
+  void* ckpt = ws + bwd_scratch_bytes(B, H, T, d_in, d_out, dt, true);
+  if (cudaMemsetAsync(status, 0, sizeof(DeviceStatus), st) != cudaSuccess)
+    return GRADLEV_ERR_CUDA;
+  // 1. forward on the predicted costates, checkpoints for the reverse scan
+  s = launch_fwd_impl(B, H, T, d_in, d_out, dt, x, ghat, eta, alpha, W0, y, ckpt, status,
+                      ws + kStatusBytes, st, nullptr, nullptr);
+  if (s != GRADLEV_OK) return s;
+  // 2. reconstructed costates gtil = y - v (the token loss's output gradient), the losses
+  const size_t ntok = (size_t)B * H * T;
+  consistency::ResidualArgs ra{ntok, d_out, y, ghat, v, gtil, dv, loss_tok, loss_c};
+  if (consistency::launch_residual(ra, dt == GRADLEV_BF16, st) != cudaSuccess)
+    return GRADLEV_ERR_CUDA;
+  // 3. the token loss's gradients: the reverse scan with dy = gtil
+  s = bwd_run(B, H, T, d_in, d_out, dt, x, ghat, eta, alpha, W0, gtil, dx, dghat, d_eta, d_alpha,
+              dW0, ckpt, ws, st, StateIO{}, false);
+  if (s != GRADLEV_OK) return s;
+  // 4. the consistency term pushes ghat toward gtil: d ghat += 2 lam (ghat - gtil)
+  if (consistency::launch_finish(dghat, ghat, gtil, lam, ntok * d_out, dt == GRADLEV_BF16, st) !=
+      cudaSuccess)
+    return GRADLEV_ERR_CUDA;
+  return GRADLEV_OK;
 }
 
 gradlev_status gradlev_device_status(const void* workspace, void* stream) {
