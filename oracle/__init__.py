@@ -57,6 +57,8 @@ def _load():
             lib.oracle_serial_f64.argtypes = [I] * 5 + [P] * 7 + [I]
             lib.oracle_serial_c128.argtypes = [I] * 5 + [P] * 7 + [I]
             lib.oracle_decode_f64.argtypes = [I] * 5 + [P] * 8 + [I]
+            lib.oracle_mlp2_serial_f64.argtypes = [I] * 6 + [P] * 9 + [I]
+            lib.oracle_mlp2_recon_f64.argtypes = [I] * 6 + [P] * 8 + [I] + [P] * 6 + [I]
             lib.oracle_max_threads.restype = I
             _lib = lib
     return _lib
@@ -234,3 +236,42 @@ def consistency(x, ghat, eta, alpha, W0, v, lam: float = 1.0, nthreads: int = 0)
     return dict(y=y, gtil=gtil, r=r, loss_tok=0.5 * np.sum(gtil * gtil, axis=-1),
                 loss_c=np.sum(r * r, axis=-1), dx=o["dx"], dghat=o["dg"] + 2.0 * lam * r,
                 deta=o["deta"], dalpha=o["dalpha"], dW0=o["dW0"], dv=-gtil)
+
+
+def _mlp2_dims(x, v, W1):
+    B, H, T, dx = x.shape
+    dy = v.shape[-1]
+    dh = W1.shape[1]
+    assert v.shape == (B, H, T, dy) and W1.shape == (H, dh, dx)
+    return B, H, T, dx, dh, dy
+
+
+def mlp2_serial(x, v, eta, alpha, W1, W2, nthreads: int = 0):
+    """Two-layer adapted MLP, serial test-time backpropagation (tanh hidden layer):
+    returns (y [B,H,T,dy], g1 [B,H,T,dh], g2 [B,H,T,dy]) - outputs and true costates."""
+    x, v, eta, alpha, W1, W2 = (_arr(a, np.float64) for a in (x, v, eta, alpha, W1, W2))
+    B, H, T, dx, dh, dy = _mlp2_dims(x, v, W1)
+    assert W2.shape == (H, dy, dh)
+    y = np.empty((B, H, T, dy))
+    g1 = np.empty((B, H, T, dh))
+    g2 = np.empty((B, H, T, dy))
+    _load().oracle_mlp2_serial_f64(B, H, T, dx, dh, dy, _p(x), _p(v), _p(eta), _p(alpha),
+                                   _p(W1), _p(W2), _p(y), _p(g1), _p(g2), int(nthreads))
+    return y, g1, g2
+
+
+def mlp2_recon(x, g1hat, g2hat, v, eta, alpha, W1, W2, control: bool = False,
+               nthreads: int = 0):
+    """Parallel reconstruction of the two-layer adapted MLP from given costates. Returns
+    dict a, h, y, g2til, g1til, dW1 (dW1 = sum_t g1til_t x_t^T per pair)."""
+    x, g1hat, g2hat, v, eta, alpha, W1, W2 = (
+        _arr(a, np.float64) for a in (x, g1hat, g2hat, v, eta, alpha, W1, W2))
+    B, H, T, dx, dh, dy = _mlp2_dims(x, v, W1)
+    out = dict(a=np.empty((B, H, T, dh)), h=np.empty((B, H, T, dh)), y=np.empty((B, H, T, dy)),
+               g2til=np.empty((B, H, T, dy)), g1til=np.empty((B, H, T, dh)),
+               dW1=np.empty((B, H, dh, dx)))
+    _load().oracle_mlp2_recon_f64(B, H, T, dx, dh, dy, _p(x), _p(g1hat), _p(g2hat), _p(v),
+                                  _p(eta), _p(alpha), _p(W1), _p(W2), 1 if control else 0,
+                                  _p(out["a"]), _p(out["h"]), _p(out["y"]), _p(out["g2til"]),
+                                  _p(out["g1til"]), _p(out["dW1"]), int(nthreads))
+    return out

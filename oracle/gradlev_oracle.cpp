@@ -61,6 +61,7 @@
 //   x, dx [B,H,T,d_in]   g, y, dy, dg [B,H,T,d_out]   eta, alpha, deta, dalpha [B,H,T]
 //   W0, dW0 [H,d_out,d_in]   (dW0 is summed over b in a fixed order b = 0..B-1)
 
+#include <cmath>
 #include <complex>
 #include <cstddef>
 #include <cstdint>
@@ -230,6 +231,87 @@ void decode_head(int T, int din, int dout, const R* x, const R* v, const R* eta,
       g[(size_t)t * dout + n] = acc - v[(size_t)t * dout + n];
     }
     state_step(din, dout, S, alpha[t], eta[t], g + (size_t)t * dout, xt);
+  }
+}
+
+// Two-layer adapted MLP of the synthetic test (Cognaptus, same page, section
+// "The synthetic test checks the mechanism, not model quality"). Both matrices
+// adapt with the centred rule; the pages do not name the nonlinearity, and tanh
+// is used here. Shared gates eta_t, alpha_t drive both layers. Per token:
+//   a_t = (W1 + S1) x_t,  h_t = tanh(a_t),  y_t = (W2 + S2) h_t,
+//   g2_t = y_t - v_t,     g1_t = (1 - h_t^2) (.) ((W2 + S2)^T g2_t),
+//   S1 <- alpha_t S1 - eta_t g1_t x_t^T,  S2 <- alpha_t S2 - eta_t g2_t h_t^T,
+// i.e. serial test-time backpropagation of the token loss 0.5 ||y_t - v_t||^2.
+// Shapes: x [T,dx], v/y/g2 [T,dy], g1 [T,dh], W1 [dh,dx], W2 [dy,dh].
+template <class R>
+void mlp2_serial_head(int T, int dx, int dh, int dy, const R* x, const R* v, const R* eta,
+                      const R* alpha, const R* W1, const R* W2, R* y, R* g1, R* g2) {
+  std::vector<R> S1((size_t)dh * dx, R(0)), S2((size_t)dy * dh, R(0)), a(dh), h(dh), q(dh);
+  for (int t = 0; t < T; ++t) {
+    const R* xt = x + (size_t)t * dx;
+    for (int k = 0; k < dh; ++k) {
+      R acc(0);
+      for (int m = 0; m < dx; ++m) acc += (W1[(size_t)k * dx + m] + S1[(size_t)k * dx + m]) * xt[m];
+      a[k] = acc;
+      h[k] = std::tanh(acc);
+    }
+    R* g2t = g2 + (size_t)t * dy;
+    for (int n = 0; n < dy; ++n) {
+      R acc(0);
+      for (int k = 0; k < dh; ++k) acc += (W2[(size_t)n * dh + k] + S2[(size_t)n * dh + k]) * h[k];
+      y[(size_t)t * dy + n] = acc;
+      g2t[n] = acc - v[(size_t)t * dy + n];
+    }
+    R* g1t = g1 + (size_t)t * dh;
+    for (int k = 0; k < dh; ++k) {
+      R acc(0);
+      for (int n = 0; n < dy; ++n) acc += (W2[(size_t)n * dh + k] + S2[(size_t)n * dh + k]) * g2t[n];
+      g1t[k] = (R(1) - h[k] * h[k]) * acc;
+    }
+    state_step(dx, dh, S1.data(), alpha[t], eta[t], g1t, xt);
+    state_step(dh, dy, S2.data(), alpha[t], eta[t], g2t, h.data());
+  }
+}
+
+// The parallel reconstruction of the same two layers from given costates g1hat,
+// g2hat, as the pages describe it: both layers' forwards are scans driven by the
+// given costates, and the costates the trajectory implies are then reconstructed
+// by backpropagating each token's loss through the adapted weights of that token:
+//   a = scan(x; g1hat, W1),  h = tanh(a),  y = scan(h; g2hat, W2),
+//   g2til_t = y_t - v_t,  g1til_t = (1 - h_t^2) (.) ((W2 + S2_t)^T g2til_t),
+//   dW1 = sum_t g1til_t x_t^T   (the first matrix's gradient over the sequence).
+// control = 1 replaces the adapted W2 + S2_t by the persistent W2 in the
+// reconstruction: the control of the synthetic-test section.
+void mlp2_recon_head(int T, int dx, int dh, int dy, const double* x, const double* g1hat,
+                     const double* g2hat, const double* v, const double* eta,
+                     const double* alpha, const double* W1, const double* W2, int control,
+                     double* a, double* h, double* y, double* g2til, double* g1til,
+                     double* dW1) {
+  std::vector<double> S1((size_t)dh * dx), S2((size_t)dy * dh, 0.0);
+  fwd_head<double>(T, dx, dh, x, g1hat, eta, alpha, W1, a, S1.data(), nullptr);
+  for (size_t e = 0; e < (size_t)T * dh; ++e) h[e] = std::tanh(a[e]);
+  for (size_t e = 0; e < (size_t)dh * dx; ++e) dW1[e] = 0.0;
+  for (int t = 0; t < T; ++t) {
+    const double* ht = h + (size_t)t * dh;
+    double* g2t = g2til + (size_t)t * dy;
+    for (int n = 0; n < dy; ++n) {
+      double acc = 0.0;
+      for (int k = 0; k < dh; ++k) acc += (W2[(size_t)n * dh + k] + S2[(size_t)n * dh + k]) * ht[k];
+      y[(size_t)t * dy + n] = acc;
+      g2t[n] = acc - v[(size_t)t * dy + n];
+    }
+    double* g1t = g1til + (size_t)t * dh;
+    for (int k = 0; k < dh; ++k) {
+      double acc = 0.0;
+      for (int n = 0; n < dy; ++n) {
+        const double w = control ? W2[(size_t)n * dh + k]
+                                 : W2[(size_t)n * dh + k] + S2[(size_t)n * dh + k];
+        acc += w * g2t[n];
+      }
+      g1t[k] = (1.0 - ht[k] * ht[k]) * acc;
+      for (int m = 0; m < dx; ++m) dW1[(size_t)k * dx + m] += g1t[k] * x[(size_t)t * dx + m];
+    }
+    state_step(dh, dy, S2.data(), alpha[t], eta[t], g2hat + (size_t)t * dy, ht);
   }
 }
 
@@ -406,6 +488,42 @@ void oracle_decode_f64(int B, int H, int T, int din, int dout, const double* x, 
     const size_t o = at3(b, h, 0, H, T);
     decode_head<double>(T, din, dout, x + o * din, v + o * dout, eta + o, alpha + o,
                         W0 + (size_t)h * dd, S + (size_t)bh * dd, y + o * dout, g + o * dout);
+  }
+}
+
+// Two-layer serial learner (see mlp2_serial_head): y, g1, g2 for every pair.
+// x [B,H,T,dx], v/y/g2 [B,H,T,dy], g1 [B,H,T,dh], W1 [H,dh,dx], W2 [H,dy,dh].
+void oracle_mlp2_serial_f64(int B, int H, int T, int dx, int dh, int dy, const double* x,
+                            const double* v, const double* eta, const double* alpha,
+                            const double* W1, const double* W2, double* y, double* g1,
+                            double* g2, int nthreads) {
+  const int nt = pick_threads(nthreads);
+#pragma omp parallel for num_threads(nt) schedule(dynamic, 1)
+  for (int bh = 0; bh < B * H; ++bh) {
+    const int h = bh % H;
+    const size_t o = (size_t)bh * T;
+    mlp2_serial_head<double>(T, dx, dh, dy, x + o * dx, v + o * dy, eta + o, alpha + o,
+                             W1 + (size_t)h * dh * dx, W2 + (size_t)h * dy * dh, y + o * dy,
+                             g1 + o * dh, g2 + o * dy);
+  }
+}
+
+// Two-layer parallel reconstruction (see mlp2_recon_head). a, h, g1til [B,H,T,dh];
+// y, g2til [B,H,T,dy]; dW1 [B,H,dh,dx].
+void oracle_mlp2_recon_f64(int B, int H, int T, int dx, int dh, int dy, const double* x,
+                           const double* g1hat, const double* g2hat, const double* v,
+                           const double* eta, const double* alpha, const double* W1,
+                           const double* W2, int control, double* a, double* hh, double* y,
+                           double* g2til, double* g1til, double* dW1, int nthreads) {
+  const int nt = pick_threads(nthreads);
+#pragma omp parallel for num_threads(nt) schedule(dynamic, 1)
+  for (int bh = 0; bh < B * H; ++bh) {
+    const int h = bh % H;
+    const size_t o = (size_t)bh * T;
+    mlp2_recon_head(T, dx, dh, dy, x + o * dx, g1hat + o * dh, g2hat + o * dy, v + o * dy,
+                    eta + o, alpha + o, W1 + (size_t)h * dh * dx, W2 + (size_t)h * dy * dh,
+                    control, a + o * dh, hh + o * dh, y + o * dy, g2til + o * dy,
+                    g1til + o * dh, dW1 + (size_t)bh * dh * dx);
   }
 }
 

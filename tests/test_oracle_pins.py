@@ -42,7 +42,15 @@ independent statement of what the GradLev scan must compute:
   - the fixed point: with the serial learner's true costates the residual,
     the consistency loss and its gradient vanish;
   - complex-step derivatives of the token loss;
-  - the closed form of one token.
+  - the closed form of one token;
+* the two-layer adapted MLP of the synthetic test (section "The synthetic
+  test checks the mechanism, not model quality"). It is pinned by
+  - exact recovery of the serial learner's outputs, hidden costates and
+    first-matrix gradient;
+  - the control (persistent second matrix in the reconstruction): outputs
+    unchanged, costates and gradient far off;
+  - the closed form of two tokens;
+  - the hidden costate as the complex-step gradient of the token loss.
 """
 
 import json
@@ -569,3 +577,66 @@ def test_consistency_single_token_closed_form():
     assert rel(c["dx"][0, 0, 0], W0.T @ gt) < 1e-15
     assert rel(c["dghat"][0, 0, 0], 4.0 * r) < 1e-15
     assert rel(c["dW0"][0], np.outer(gt, x)) < 1e-15
+
+
+# --------------------------------------------------------------------------- two-layer MLP
+
+
+def _mlp2_inputs(B=1, H=2, T=20, dx=5, dh=4, dy=3, seed=81):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((B, H, T, dx))
+    v = rng.standard_normal((B, H, T, dy))
+    eta = rng.uniform(0.0, 0.5, (B, H, T))
+    alpha = rng.uniform(0.5, 1.0, (B, H, T))
+    W1 = 0.5 * rng.standard_normal((H, dh, dx))
+    W2 = 0.5 * rng.standard_normal((H, dy, dh))
+    return x, v, eta, alpha, W1, W2
+
+
+def test_mlp2_exact_recovery_of_serial_learner():
+    """The mechanism of the synthetic test: with the serial learner's costates supplied,
+    the parallel reconstruction gives its outputs, hidden costates and first-matrix
+    gradient back (the pages report rounding-scale differences)."""
+    x, v, eta, alpha, W1, W2 = _mlp2_inputs()
+    y, g1, g2 = oracle.mlp2_serial(x, v, eta, alpha, W1, W2)
+    r = oracle.mlp2_recon(x, g1, g2, v, eta, alpha, W1, W2)
+    assert rel(r["y"], y) < 1e-14 and rel(r["g2til"], g2) < 1e-14 and rel(r["g1til"], g1) < 1e-14
+    dW1 = np.einsum("bhtk,bhtm->bhkm", g1, x)
+    assert rel(r["dW1"], dW1) < 1e-14
+
+
+def test_mlp2_control_breaks_the_backward_only():
+    x, v, eta, alpha, W1, W2 = _mlp2_inputs(seed=83)
+    y, g1, g2 = oracle.mlp2_serial(x, v, eta, alpha, W1, W2)
+    r = oracle.mlp2_recon(x, g1, g2, v, eta, alpha, W1, W2)
+    c = oracle.mlp2_recon(x, g1, g2, v, eta, alpha, W1, W2, control=True)
+    assert np.array_equal(c["y"], r["y"]) and np.array_equal(c["g2til"], r["g2til"])
+    assert rel(c["g1til"], g1) > 0.05 and rel(c["dW1"], r["dW1"]) > 0.05
+
+
+def test_mlp2_two_tokens_closed_form():
+    x, v, eta, alpha, W1, W2 = _mlp2_inputs(B=1, H=1, T=2, seed=85)
+    y, g1, g2 = oracle.mlp2_serial(x, v, eta, alpha, W1, W2)
+    X, V, e, al, A, Bm = x[0, 0], v[0, 0], eta[0, 0], alpha[0, 0], W1[0], W2[0]
+    # token 0 from the persistent weights
+    h0 = np.tanh(A @ X[0]); y0 = Bm @ h0; q0 = y0 - V[0]; p0 = (1 - h0 ** 2) * (Bm.T @ q0)
+    # both deviations after token 0
+    S1 = -e[0] * np.outer(p0, X[0]); S2 = -e[0] * np.outer(q0, h0)
+    h1 = np.tanh((A + S1) @ X[1]); y1 = (Bm + S2) @ h1; q1 = y1 - V[1]
+    p1 = (1 - h1 ** 2) * ((Bm + S2).T @ q1)
+    assert rel(y[0, 0], np.stack([y0, y1])) < 1e-15
+    assert rel(g2[0, 0], np.stack([q0, q1])) < 1e-15
+    assert rel(g1[0, 0], np.stack([p0, p1])) < 1e-14
+
+
+def test_mlp2_hidden_costate_is_the_token_gradient():
+    """g1 is the derivative of the token loss with respect to the hidden pre-activation,
+    the weights held at their values for that token (complex step on a_0)."""
+    x, v, eta, alpha, W1, W2 = _mlp2_inputs(B=1, H=1, T=1, seed=87)
+    _, g1, _ = oracle.mlp2_serial(x, v, eta, alpha, W1, W2)
+    a0 = W1[0] @ x[0, 0, 0]
+    for k in range(a0.size):
+        z = a0.astype(np.complex128)
+        z[k] += 1e-30j
+        r = W2[0] @ np.tanh(z) - v[0, 0, 0]
+        assert abs(np.imag(0.5 * np.sum(r * r)) / 1e-30 - g1[0, 0, 0, k]) < 1e-14
