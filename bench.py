@@ -4,6 +4,7 @@
                     [--config IDX] [--no-e2e] [--no-cpu-baseline]
     python bench.py --decode [--steps K] [--warmup W] [--T TOKENS_PER_CALL]
     python bench.py --consistency [--steps K] [--warmup W] [--config IDX]
+    python bench.py --mlp2 [--steps K] [--warmup W]
 
 One step = one forward scan (with state checkpoints) + one reverse scan over
 one batch of the workload, i.e. every step of the hot path. The default
@@ -29,6 +30,10 @@ reported beside it.
 call is a whole training step from predicted costates: the forward, the
 reconstructed costates and losses, the reverse scan, and the consistency
 gradient. It prints its own line.
+
+``--mlp2`` times gradlev_mlp2_recon, the two-layer reconstruction of the
+synthetic test, at bf16 B8 H16 T4096 with d_x = d_h = d_y = 128, and prints
+its own line.
 """
 
 from __future__ import annotations
@@ -68,6 +73,7 @@ def parse():
     p.add_argument("--decode", action="store_true", help="time the deployment decode step")
     p.add_argument("--consistency", action="store_true",
                    help="time the consistency training step")
+    p.add_argument("--mlp2", action="store_true", help="time the two-layer reconstruction")
     return p.parse_args()
 
 
@@ -394,8 +400,75 @@ def run_consistency(args):
     print(json.dumps(line), flush=True)
 
 
+def run_mlp2(args):
+    """gradlev_mlp2_recon at bf16 B8 H16 T4096, d_x = d_h = d_y = 128."""
+    import torch
+
+    import token_weight_scans_b200 as tw
+    from token_weight_scans_b200 import build as tw_build
+    torch.cuda.set_device(0)
+    tw_build.build()
+    tw.lib()
+    B, H, T = args.B or 8, args.H or 16, args.T or 4096
+    d = 128
+    g = torch.Generator(device="cuda").manual_seed(91)
+    rn = lambda *s: torch.randn(*s, generator=g, device="cuda")
+    bf = torch.bfloat16
+    x, v = rn(B, H, T, d).to(bf), rn(B, H, T, d).to(bf)
+    g1, g2 = (0.1 * rn(B, H, T, d)).to(bf), (0.1 * rn(B, H, T, d)).to(bf)
+    eta = 0.5 / d * torch.rand(B, H, T, generator=g, device="cuda")
+    alpha = 0.9 + 0.099 * torch.rand(B, H, T, generator=g, device="cuda")
+    W1, W2 = rn(H, d, d) / d ** 0.5, rn(H, d, d) / d ** 0.5
+    ws = torch.empty(tw.gradlev_mlp2_workspace_bytes(B, H, T, d, d, d, tw.BF16),
+                     dtype=torch.uint8, device="cuda")
+    out = None
+
+    def step():
+        nonlocal out
+        out = tw.gradlev_mlp2_recon(x, g1, g2, v, eta, alpha, W1, W2, workspace=ws, out=out)
+        return tw.gradlev_last_launch_count()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    s0, e0 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches = 0
+    s0.record()
+    for _ in range(args.steps):
+        launches += step()
+    e0.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = s0.elapsed_time(e0) / args.steps
+    N = B * H * T
+    # algorithmic bytes: two forward scans (x, g1hat, a; h, g2hat, y), tanh (a in, h out),
+    # the reconstruction (x, h, g2hat, y, v in; g2til, g1til out) and dW1
+    byt = N * d * 2 * (3 + 3 + 2 + 7) + 4 * N * 8 + 2 * H * d * d * 4 + B * H * d * d * 4
+    flops = 2 * N * d * d * (2 + 2) + 2 * N * d * d * 4  # scans, then W2^T u, S2^T u, carry, dW1
+    peaks, peak_src = load_peaks()
+    line = {"metric": "GradLev two-layer reconstruction tokens/s on 1 B200 "
+                      f"(B{B} H{H} T{T} d128 bf16)",
+            "value": B * T / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "dtype": "bf16", "data": "synthetic (seeded generator)",
+            "config": {"workload": "mlp2 reconstruction", "B": B, "H": H, "T": T, "d_x": d,
+                       "d_h": d, "d_y": d},
+            "roofline": {"bound": "hbm", "achieved": byt / (ms * 1e-3) / 1e9,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": byt / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                         "alg_bytes_per_step": byt, "alg_flops_per_step": flops,
+                         "peak_source": peak_src},
+            "clocks": clk, "gpu_launches": launches}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
+    if args.mlp2:
+        return run_mlp2(args)
     if args.decode:
         return run_decode(args)
     if args.consistency:

@@ -252,6 +252,47 @@ GRADLEV_API gradlev_status gradlev_consistency_step(int B, int H, int T, int d_i
                                         float* d_eta, float* d_alpha, float* dW0, void* dv,
                                         void* workspace, size_t ws_bytes, void* stream);
 
+/* Parallel reconstruction of the two-layer adapted MLP of the synthetic test.
+ *
+ * Cognaptus, "Parallelize the Training, Keep the Learning Serial", section "The
+ * synthetic test checks the mechanism, not model quality". Both matrices adapt
+ * with the centred rule under the shared gates eta, alpha; the hidden layer is
+ * tanh (the pages name no nonlinearity). Given costates g1hat and g2hat for the
+ * two layers:
+ *   a = scan(x; g1hat, W1)          [B,H,T,d_h]   (the forward scan, d_in = d_x)
+ *   h = tanh(a)                      [B,H,T,d_h]
+ *   y = scan(h; g2hat, W2)          [B,H,T,d_y]
+ *   g2til_t = y_t - v_t              [B,H,T,d_y]
+ *   g1til_t = (1 - h_t^2) (.) ((W2 + S2_t)^T g2til_t)   [B,H,T,d_h]
+ *   dW1 = sum_t g1til_t x_t^T         [B,H,d_h,d_x] float32
+ * S2_t is the second layer's deviation before token t. control = 1 uses the
+ * persistent W2 instead of W2 + S2_t: the control of the same section, which
+ * leaves y unchanged and breaks g1til and dW1. With the serial learner's costates
+ * supplied, the outputs are the serial learner's outputs, hidden costates and
+ * first-matrix gradient.
+ *
+ * Arguments:
+ *   W1 [H,d_h,d_x], W2 [H,d_y,d_h], eta and alpha [B,H,T]: float32.
+ *   x, g1hat, g2hat, v and every output except dW1: dtype.
+ * Requirements, else the status shown:
+ *   - (d_x -> d_h) and (d_h -> d_y) must each be a supported scan shape; d_x a
+ *     multiple of 4; d_h and d_y multiples of 8; d_h * d_x <= 16384
+ *     (GRADLEV_ERR_UNSUPPORTED);
+ *   - workspace at least gradlev_mlp2_workspace_bytes() bytes
+ *     (GRADLEV_ERR_WORKSPACE);
+ *   - alignment (GRADLEV_ERR_INVALID_ARG): x, g1hat, g2hat, a, h, y, W1, W2,
+ *     dW1 and workspace 16 bytes; v, g2til, g1til one element.
+ * Outputs may not alias inputs. */
+GRADLEV_API size_t gradlev_mlp2_workspace_bytes(int B, int H, int T, int d_x, int d_h, int d_y,
+                                    gradlev_dtype dt);
+GRADLEV_API gradlev_status gradlev_mlp2_recon(int B, int H, int T, int d_x, int d_h, int d_y,
+                                  gradlev_dtype dt, const void* x, const void* g1hat,
+                                  const void* g2hat, const void* v, const float* eta,
+                                  const float* alpha, const float* W1, const float* W2,
+                                  int control, void* a, void* h, void* y, void* g2til,
+                                  void* g1til, float* dW1, void* workspace, size_t ws_bytes,
+                                  void* stream);
+
 /* Size of the static scratch array gradlev_scan_bwd_noalloc uses: 64 MiB,
  * held by every GPU that loads the library until the process exits. */
 #define GRADLEV_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)

@@ -32,7 +32,8 @@ def test_header_declares_the_entry_points():
               "gradlev_status_string", "gradlev_scan_supported", "gradlev_scan_ckpt_bytes",
               "gradlev_device_status", "gradlev_last_launch_count", "gradlev_scan_fwd_state",
               "gradlev_scan_bwd_state", "gradlev_decode_step", "gradlev_consistency_step",
-              "gradlev_consistency_workspace_bytes"):
+              "gradlev_consistency_workspace_bytes", "gradlev_mlp2_recon",
+              "gradlev_mlp2_workspace_bytes"):
         assert n in names, n
 
 
@@ -188,3 +189,23 @@ def test_consistency_step_validates_before_launch(L):
     assert call(dv=P(4100)) == 1
     assert call(ws=P(4096 + 16)) == 1    # workspace not 256-byte aligned
     assert call(nbytes=16) == 3          # workspace too small
+
+
+def test_mlp2_recon_validates_before_launch(L):
+    P = ctypes.c_void_p
+    fake = P(4096)
+    I, Z = ctypes.c_int, ctypes.c_size_t
+    L.gradlev_mlp2_workspace_bytes.restype = Z
+    L.gradlev_mlp2_workspace_bytes.argtypes = [I] * 7
+    L.gradlev_mlp2_recon.restype = I
+    L.gradlev_mlp2_recon.argtypes = [I] * 7 + [P] * 8 + [I] + [P] * 7 + [Z, P]
+    assert L.gradlev_mlp2_workspace_bytes(2, 2, 64, 16, 32, 8, 0) > 0
+    assert L.gradlev_mlp2_workspace_bytes(2, 2, 64, 16, 30, 8, 0) == 0   # d_h % 8
+    assert L.gradlev_mlp2_workspace_bytes(2, 2, 64, 256, 128, 8, 0) == 0  # d_h * d_x too big
+    call = lambda d_h=32, x=fake, ws=1 << 30, dW1=fake: L.gradlev_mlp2_recon(
+        2, 2, 64, 16, d_h, 8, 0, x, fake, fake, fake, fake, fake, fake, fake, 0, fake, fake,
+        fake, fake, fake, dW1, fake, ws, P(0))
+    assert call(d_h=30) == 2
+    assert call(x=P(0)) == 1
+    assert call(dW1=P(4100)) == 1
+    assert call(ws=16) == 3

@@ -18,7 +18,7 @@ __all__ = [
     "gradlev_scan_workspace_bytes", "gradlev_scan_ckpt_bytes", "gradlev_scan_fwd",
     "gradlev_scan_bwd", "gradlev_scan_fwd_state", "gradlev_scan_bwd_state",
     "gradlev_decode_step", "gradlev_consistency_workspace_bytes", "gradlev_consistency_step",
-    "gradlev_device_status", "gradlev_last_launch_count", "F32", "BF16", "LIB_PATH",
+    "gradlev_mlp2_workspace_bytes", "gradlev_mlp2_recon", "gradlev_device_status", "gradlev_last_launch_count", "F32", "BF16", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgradlev.so")
@@ -30,7 +30,8 @@ _ENTRY_POINTS = (
     "gradlev_scan_ckpt_bytes", "gradlev_scan_fwd", "gradlev_scan_bwd",
     "gradlev_scan_fwd_state", "gradlev_scan_bwd_state", "gradlev_decode_step",
     "gradlev_consistency_workspace_bytes", "gradlev_consistency_step",
-    "gradlev_device_status", "gradlev_last_launch_count",
+    "gradlev_mlp2_workspace_bytes", "gradlev_mlp2_recon", "gradlev_device_status",
+    "gradlev_last_launch_count",
 )
 
 
@@ -81,6 +82,10 @@ def lib():
     L.gradlev_consistency_step.argtypes = ([I] * 6 + [P] * 6 + [ctypes.c_float] + [P] * 11 +
                                            [Z, P])
     L.gradlev_consistency_step.restype = I
+    L.gradlev_mlp2_workspace_bytes.argtypes = [I] * 7
+    L.gradlev_mlp2_workspace_bytes.restype = Z
+    L.gradlev_mlp2_recon.argtypes = [I] * 7 + [P] * 8 + [I] + [P] * 7 + [Z, P]
+    L.gradlev_mlp2_recon.restype = I
     L.gradlev_device_status.argtypes = [P, P]
     L.gradlev_device_status.restype = I
     L.gradlev_last_launch_count.argtypes = []
@@ -362,6 +367,48 @@ def gradlev_consistency_step(x, ghat, eta, alpha, W0, v, lam=1.0, *, want_dv=Tru
         _ptr(out["dalpha"]), _ptr(out["dW0"]), _ptr(out.get("dv")), _ptr(ws),
         ws.numel() * ws.element_size(), _stream_ptr(stream))
     _check(st, "gradlev_consistency_step")
+    return out
+
+
+def gradlev_mlp2_workspace_bytes(B, H, T, d_x, d_h, d_y, dt) -> int:
+    return int(lib().gradlev_mlp2_workspace_bytes(B, H, T, d_x, d_h, d_y, dt))
+
+
+def gradlev_mlp2_recon(x, g1hat, g2hat, v, eta, alpha, W1, W2, control=False, *,
+                       workspace=None, stream=None, out=None):
+    """Parallel reconstruction of the two-layer adapted MLP from given costates (see
+    include/gradlev.h). Returns dict a, h, y, g2til, g1til, dW1."""
+    import torch
+    if x.dim() != 4 or v.dim() != 4 or W1.dim() != 3:
+        raise GradlevError("x, v must be [B,H,T,d] and W1 [H,d_h,d_x]")
+    B, H, T, d_x = x.shape
+    d_y = v.shape[-1]
+    d_h = W1.shape[1]
+    dev, dt = x.device, x.dtype
+    f32 = torch.float32
+    _check_tensor("x", x, (B, H, T, d_x), dt, dev)
+    _check_tensor("g1hat", g1hat, (B, H, T, d_h), dt, dev)
+    _check_tensor("g2hat", g2hat, (B, H, T, d_y), dt, dev)
+    _check_tensor("v", v, (B, H, T, d_y), dt, dev)
+    _check_tensor("eta", eta, (B, H, T), f32, dev)
+    _check_tensor("alpha", alpha, (B, H, T), f32, dev)
+    _check_tensor("W1", W1, (H, d_h, d_x), f32, dev)
+    _check_tensor("W2", W2, (H, d_y, d_h), f32, dev)
+    code = _dt_code(dt)
+    nws = gradlev_mlp2_workspace_bytes(B, H, T, d_x, d_h, d_y, code)
+    if nws == 0:
+        raise GradlevError("gradlev_mlp2_recon: unsupported shape", 2)
+    if out is None:
+        out = dict(a=torch.empty_like(g1hat), h=torch.empty_like(g1hat), y=torch.empty_like(v),
+                   g2til=torch.empty_like(v), g1til=torch.empty_like(g1hat),
+                   dW1=torch.empty((B, H, d_h, d_x), dtype=f32, device=dev))
+    ws = _workspace(nws, dev, workspace)
+    st = lib().gradlev_mlp2_recon(
+        B, H, T, d_x, d_h, d_y, code, _ptr(x), _ptr(g1hat), _ptr(g2hat), _ptr(v), _ptr(eta),
+        _ptr(alpha), _ptr(W1), _ptr(W2), 1 if control else 0, _ptr(out["a"]), _ptr(out["h"]),
+        _ptr(out["y"]), _ptr(out["g2til"]), _ptr(out["g1til"]), _ptr(out["dW1"]), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream_ptr(stream))
+    _check(st, "gradlev_mlp2_recon")
     return out
 
 

@@ -18,6 +18,7 @@
 #include "dispatch.h"
 #include "gradlev.h"
 #include "consistency.h"
+#include "mlp2.h"
 #include "scan_ffma.h"
 #include "scan_tc.h"
 
@@ -413,6 +414,62 @@ gradlev_status gradlev_consistency_step(int B, int H, int T, int d_in, int d_out
       cudaSuccess)
     return GRADLEV_ERR_CUDA;
   return GRADLEV_OK;
+}
+
+size_t gradlev_mlp2_workspace_bytes(int B, int H, int T, int d_x, int d_h, int d_y,
+                                    gradlev_dtype dt) {
+  if (check_shape(B, H, T, d_x, d_h, dt) != GRADLEV_OK ||
+      check_shape(B, H, T, d_h, d_y, dt) != GRADLEV_OK || !mlp2::shape_ok(d_x, d_h, d_y))
+    return 0;
+  const size_t a = fwd_scratch_bytes(B, H, T, d_x, d_h, dt);
+  const size_t b = fwd_scratch_bytes(B, H, T, d_h, d_y, dt);
+  return a > b ? a : b;  // the two forward scans run one after the other
+}
+
+gradlev_status gradlev_mlp2_recon(int B, int H, int T, int d_x, int d_h, int d_y,
+                                  gradlev_dtype dt, const void* x, const void* g1hat,
+                                  const void* g2hat, const void* v, const float* eta,
+                                  const float* alpha, const float* W1, const float* W2,
+                                  int control, void* a, void* h, void* y, void* g2til,
+                                  void* g1til, float* dW1, void* workspace, size_t ws_bytes,
+                                  void* stream) {
+  gradlev_status s = check_shape(B, H, T, d_x, d_h, dt);
+  if (s != GRADLEV_OK) return s;
+  s = check_shape(B, H, T, d_h, d_y, dt);
+  if (s != GRADLEV_OK) return s;
+  if (!mlp2::shape_ok(d_x, d_h, d_y)) return GRADLEV_ERR_UNSUPPORTED;
+  if (!x || !g1hat || !g2hat || !v || !eta || !alpha || !W1 || !W2 || !a || !h || !y ||
+      !g2til || !g1til || !dW1 || !workspace)
+    return GRADLEV_ERR_INVALID_ARG;
+  const size_t es = dt == GRADLEV_BF16 ? 2 : 4;
+  if (!aligned(x, 16) || !aligned(g1hat, 16) || !aligned(g2hat, 16) || !aligned(a, 16) ||
+      !aligned(h, 16) || !aligned(y, 16) || !aligned(W1, 16) || !aligned(W2, 16) ||
+      !aligned(dW1, 16) || !aligned(v, es) || !aligned(g2til, es) || !aligned(g1til, es) ||
+      !aligned(eta, 4) || !aligned(alpha, 4) || !aligned(workspace, 16))
+    return GRADLEV_ERR_INVALID_ARG;
+  if (ws_bytes < gradlev_mlp2_workspace_bytes(B, H, T, d_x, d_h, d_y, dt))
+    return GRADLEV_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  t_launches = 0;
+  char* ws = static_cast<char*>(workspace);
+  DeviceStatus* status = reinterpret_cast<DeviceStatus*>(ws);
+  if (cudaMemsetAsync(status, 0, sizeof(DeviceStatus), st) != cudaSuccess)
+    return GRADLEV_ERR_CUDA;
+  // first layer: a = scan(x; g1hat, W1), h = tanh(a)
+  s = launch_fwd_impl(B, H, T, d_x, d_h, dt, x, g1hat, eta, alpha, W1, a, nullptr, status,
+                      ws + kStatusBytes, st, nullptr, nullptr);
+  if (s != GRADLEV_OK) return s;
+  const size_t nh = (size_t)B * H * T * d_h;
+  if (mlp2::launch_tanh(a, h, nh, dt == GRADLEV_BF16, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
+  // second layer: y = scan(h; g2hat, W2)
+  s = launch_fwd_impl(B, H, T, d_h, d_y, dt, h, g2hat, eta, alpha, W2, y, nullptr, status,
+                      ws + kStatusBytes, st, nullptr, nullptr);
+  if (s != GRADLEV_OK) return s;
+  // reconstruction through the second layer's adapted weights
+  mlp2::TqueryArgs ta{B, H, T, d_x, d_h, d_y, control ? 1 : 0, x, h, g2hat, y, v, eta, alpha,
+                      W2, g2til, g1til, dW1};
+  return mlp2::launch_tquery(ta, dt == GRADLEV_BF16, st) == cudaSuccess ? GRADLEV_OK
+                                                                       : GRADLEV_ERR_CUDA;
 }
 
 gradlev_status gradlev_device_status(const void* workspace, void* stream) {
