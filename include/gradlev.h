@@ -280,9 +280,13 @@ GRADLEV_API gradlev_status gradlev_consistency_step(int B, int H, int T, int d_i
  *     (GRADLEV_ERR_UNSUPPORTED);
  *   - workspace at least gradlev_mlp2_workspace_bytes() bytes
  *     (GRADLEV_ERR_WORKSPACE);
- *   - alignment (GRADLEV_ERR_INVALID_ARG): x, g1hat, g2hat, a, h, y, W1, W2,
- *     dW1 and workspace 16 bytes; v, g2til, g1til one element.
- * Outputs may not alias inputs. */
+ *   - alignment (GRADLEV_ERR_INVALID_ARG): workspace 256 bytes; x, g1hat,
+ *     g2hat, a, h, y, g2til, g1til, W1, W2 and dW1 16 bytes; v one element.
+ * Outputs may not alias inputs.
+ * Routes: with a tensor-core second layer (bf16, d_h = 128, d_y in {128, 256})
+ * and no control, g1til comes from the reverse-scan kernel in its hidden-costate
+ * mode, i.e. dx without the adjoint terms, times (1 - h^2). Every other case uses
+ * a CUDA-core reconstruction kernel. */
 GRADLEV_API size_t gradlev_mlp2_workspace_bytes(int B, int H, int T, int d_x, int d_h, int d_y,
                                     gradlev_dtype dt);
 GRADLEV_API gradlev_status gradlev_mlp2_recon(int B, int H, int T, int d_x, int d_h, int d_y,

@@ -416,14 +416,48 @@ gradlev_status gradlev_consistency_step(int B, int H, int T, int d_in, int d_out
   return GRADLEV_OK;
 }
 
+}  // extern "C"
+
+namespace gradlev {
+
+// Workspace of the two-layer reconstruction. The tensor-core route (second layer a
+// tensor-core shape, no control) lays it out as:
+//   [0, r0)  status word, the forward scans' segment scratch, the reverse scan's partials
+//   ckpt     the second layer's checkpoints
+//   dg, de, da  scratch for the reverse scan's outputs that this call does not return
+// The CUDA-core route needs only the first part.
+struct Mlp2Ws {
+  size_t r0, ckpt, dg, de, da, total;
+};
+
+static Mlp2Ws mlp2_ws(int B, int H, int T, int dx, int dh, int dy, gradlev_dtype dt) {
+  Mlp2Ws w{};
+  const size_t f1 = fwd_scratch_bytes(B, H, T, dx, dh, dt);
+  const size_t f2 = fwd_scratch_bytes(B, H, T, dh, dy, dt);
+  w.r0 = f1 > f2 ? f1 : f2;
+  if (use_tc(dh, dy, dt)) {
+    const size_t b = bwd_scratch_bytes(B, H, T, dh, dy, dt, false);
+    w.r0 = align_up(w.r0 > b ? w.r0 : b, 256);
+    const size_t es = dt == GRADLEV_BF16 ? 2 : 4;
+    const size_t ntok = (size_t)B * H * T;
+    w.ckpt = align_up(ckpt_bytes_of(B, H, T, dh, dy, dt), 256);
+    w.dg = align_up(ntok * dy * es, 256);
+    w.de = w.da = align_up(ntok * 4, 256);
+  }
+  w.total = w.r0 + w.ckpt + w.dg + w.de + w.da;
+  return w;
+}
+
+}  // namespace gradlev
+
+extern "C" {
+
 size_t gradlev_mlp2_workspace_bytes(int B, int H, int T, int d_x, int d_h, int d_y,
                                     gradlev_dtype dt) {
   if (check_shape(B, H, T, d_x, d_h, dt) != GRADLEV_OK ||
       check_shape(B, H, T, d_h, d_y, dt) != GRADLEV_OK || !mlp2::shape_ok(d_x, d_h, d_y))
     return 0;
-  const size_t a = fwd_scratch_bytes(B, H, T, d_x, d_h, dt);
-  const size_t b = fwd_scratch_bytes(B, H, T, d_h, d_y, dt);
-  return a > b ? a : b;  // the two forward scans run one after the other
+  return mlp2_ws(B, H, T, d_x, d_h, d_y, dt).total;
 }
 
 gradlev_status gradlev_mlp2_recon(int B, int H, int T, int d_x, int d_h, int d_y,
@@ -444,32 +478,54 @@ gradlev_status gradlev_mlp2_recon(int B, int H, int T, int d_x, int d_h, int d_y
   const size_t es = dt == GRADLEV_BF16 ? 2 : 4;
   if (!aligned(x, 16) || !aligned(g1hat, 16) || !aligned(g2hat, 16) || !aligned(a, 16) ||
       !aligned(h, 16) || !aligned(y, 16) || !aligned(W1, 16) || !aligned(W2, 16) ||
-      !aligned(dW1, 16) || !aligned(v, es) || !aligned(g2til, es) || !aligned(g1til, es) ||
-      !aligned(eta, 4) || !aligned(alpha, 4) || !aligned(workspace, 16))
+      !aligned(dW1, 16) || !aligned(v, es) || !aligned(g2til, 16) || !aligned(g1til, 16) ||
+      !aligned(eta, 4) || !aligned(alpha, 4) || !aligned(workspace, 256))
     return GRADLEV_ERR_INVALID_ARG;
-  if (ws_bytes < gradlev_mlp2_workspace_bytes(B, H, T, d_x, d_h, d_y, dt))
-    return GRADLEV_ERR_WORKSPACE;
+  const Mlp2Ws w = mlp2_ws(B, H, T, d_x, d_h, d_y, dt);
+  if (ws_bytes < w.total) return GRADLEV_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   t_launches = 0;
   char* ws = static_cast<char*>(workspace);
   DeviceStatus* status = reinterpret_cast<DeviceStatus*>(ws);
   if (cudaMemsetAsync(status, 0, sizeof(DeviceStatus), st) != cudaSuccess)
     return GRADLEV_ERR_CUDA;
+  const bool bf = dt == GRADLEV_BF16;
+  const bool tc_route = use_tc(d_h, d_y, dt) && !control;
+  char* ckpt = tc_route ? ws + w.r0 : nullptr;
   // first layer: a = scan(x; g1hat, W1), h = tanh(a)
   s = launch_fwd_impl(B, H, T, d_x, d_h, dt, x, g1hat, eta, alpha, W1, a, nullptr, status,
                       ws + kStatusBytes, st, nullptr, nullptr);
   if (s != GRADLEV_OK) return s;
-  const size_t nh = (size_t)B * H * T * d_h;
-  if (mlp2::launch_tanh(a, h, nh, dt == GRADLEV_BF16, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
-  // second layer: y = scan(h; g2hat, W2)
-  s = launch_fwd_impl(B, H, T, d_h, d_y, dt, h, g2hat, eta, alpha, W2, y, nullptr, status,
+  const size_t ntok = (size_t)B * H * T;
+  if (mlp2::launch_tanh(a, h, ntok * d_h, bf, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
+  // second layer: y = scan(h; g2hat, W2), with its checkpoints on the tensor-core route
+  s = launch_fwd_impl(B, H, T, d_h, d_y, dt, h, g2hat, eta, alpha, W2, y, ckpt, status,
                       ws + kStatusBytes, st, nullptr, nullptr);
   if (s != GRADLEV_OK) return s;
-  // reconstruction through the second layer's adapted weights
-  mlp2::TqueryArgs ta{B, H, T, d_x, d_h, d_y, control ? 1 : 0, x, h, g2hat, y, v, eta, alpha,
-                      W2, g2til, g1til, dW1};
-  return mlp2::launch_tquery(ta, dt == GRADLEV_BF16, st) == cudaSuccess ? GRADLEV_OK
-                                                                       : GRADLEV_ERR_CUDA;
+  if (!tc_route) {
+    // the reconstruction kernel on CUDA cores (every shape, and the control)
+    mlp2::TqueryArgs ta{B, H, T, d_x, d_h, d_y, control ? 1 : 0, x, h, g2hat, y, v, eta, alpha,
+                        W2, g2til, g1til, dW1};
+    return mlp2::launch_tquery(ta, bf, st) == cudaSuccess ? GRADLEV_OK : GRADLEV_ERR_CUDA;
+  }
+  // tensor-core route: g2til = y - v, then the reverse scan of the second layer in its
+  // hidden-costate mode gives g1til = (1 - h^2) (.) (W2 + S2_t)^T g2til directly
+  if (mlp2::launch_sub(y, v, g2til, ntok * d_y, bf, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
+  char* dg = ckpt + w.ckpt;
+  float* de = reinterpret_cast<float*>(dg + w.dg);
+  float* da = reinterpret_cast<float*>(dg + w.dg + w.de);
+  float* parts = reinterpret_cast<float*>(ws + kStatusBytes);
+  for (int n0 = 0; n0 < d_y; n0 += 128) {
+    tc::TcBwdParams prm{B, H, T, d_h, d_y, n0, n0 > 0 ? 1 : 0, eta, alpha, W2,
+                        static_cast<__nv_bfloat16*>(g1til), reinterpret_cast<__nv_bfloat16*>(dg),
+                        de, da, parts, status, kWaitTimeoutNs};
+    prm.local = 1;
+    if (tc::launch_bwd(prm, h, g2hat, g2til, ckpt, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
+  }
+  // the first matrix's gradient over the sequence
+  return mlp2::launch_outer_sum(g1til, x, dW1, B * H, T, d_h, d_x, bf, st) == cudaSuccess
+             ? GRADLEV_OK
+             : GRADLEV_ERR_CUDA;
 }
 
 gradlev_status gradlev_device_status(const void* workspace, void* stream) {

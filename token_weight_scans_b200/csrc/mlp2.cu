@@ -301,6 +301,106 @@ cudaError_t launch_tanh(const void* a, void* h, size_t elems, bool bf16, cudaStr
 }
 
 template <typename Tio>
+__global__ void sub_kernel(const Tio* __restrict__ y, const Tio* __restrict__ v,
+                           Tio* __restrict__ out, size_t n) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x)
+    out[i] = from_f32<Tio>(to_f32(y[i]) - to_f32(v[i]));
+}
+
+// dW1 = sum_t g1_t x_t^T for one (b,h) per CTA: chunks of FC tokens are staged in
+// shared memory and every thread accumulates up to two 8 x 4 blocks in registers.
+template <typename Tio>
+__global__ void __launch_bounds__(FT, 1) outer_sum_kernel(const Tio* __restrict__ g1,
+                                                          const Tio* __restrict__ x,
+                                                          float* __restrict__ dW1, int T, int dh,
+                                                          int dx) {
+  extern __shared__ float4 smem4[];
+  float* Gs = reinterpret_cast<float*>(smem4);      // [FC][dh + 4]
+  const int LDH = dh + 4, LDX = dx + 4;
+  float* Xs = Gs + (size_t)FC * LDH;                // [FC][dx + 4]
+  const int tid = threadIdx.x, bh = blockIdx.x;
+  const size_t tok0 = (size_t)bh * T;
+  const int NKX4 = dx / 4, NBH = dh / 8;
+  float4 dw[2][8];
+#pragma unroll
+  for (int it = 0; it < 2; ++it)
+#pragma unroll
+    for (int r = 0; r < 8; ++r) dw[it][r] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int t0 = 0; t0 < T; t0 += FC) {
+    const int nt = min(FC, T - t0);
+    __syncthreads();
+    load_rows(Gs, LDH, g1 + (tok0 + t0) * dh, nt, dh, tid);
+    load_rows(Xs, LDX, x + (tok0 + t0) * dx, nt, dx, tid);
+    __syncthreads();
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+      const int item = tid + it * FT;
+      if (item < NBH * NKX4) {
+        const int nb = item / NKX4, k4 = item - nb * NKX4;
+        for (int i = 0; i < nt; ++i) {
+          const float4 xv = *reinterpret_cast<const float4*>(&Xs[i * LDX + 4 * k4]);
+#pragma unroll
+          for (int r = 0; r < 8; ++r) {
+            const float gv = Gs[i * LDH + nb * 8 + r];
+            dw[it][r].x = fmaf(gv, xv.x, dw[it][r].x);
+            dw[it][r].y = fmaf(gv, xv.y, dw[it][r].y);
+            dw[it][r].z = fmaf(gv, xv.z, dw[it][r].z);
+            dw[it][r].w = fmaf(gv, xv.w, dw[it][r].w);
+          }
+        }
+      }
+    }
+  }
+  float* dst = dW1 + (size_t)bh * dh * dx;
+#pragma unroll
+  for (int it = 0; it < 2; ++it) {
+    const int item = tid + it * FT;
+    if (item < NBH * NKX4) {
+      const int nb = item / NKX4, k4 = item - nb * NKX4;
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        *reinterpret_cast<float4*>(&dst[(size_t)(nb * 8 + r) * dx + 4 * k4]) = dw[it][r];
+    }
+  }
+}
+
+cudaError_t launch_sub(const void* y, const void* v, void* out, size_t elems, bool bf16,
+                       cudaStream_t st) {
+  const size_t want = (elems + 255) / 256;
+  const unsigned grid = (unsigned)(want < 148 * 16 ? (want > 0 ? want : 1) : 148 * 16);
+  if (bf16)
+    sub_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(y),
+                                                   static_cast<const __nv_bfloat16*>(v),
+                                                   static_cast<__nv_bfloat16*>(out), elems);
+  else
+    sub_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(y),
+                                           static_cast<const float*>(v),
+                                           static_cast<float*>(out), elems);
+  count_launch();
+  return cudaGetLastError();
+}
+
+template <typename Tio>
+static cudaError_t launch_outer_sum_t(const void* g1, const void* x, float* dW1, int BH, int T,
+                                      int dh, int dx, cudaStream_t st) {
+  const size_t smem = sizeof(float) * (size_t)FC * ((dh + 4) + (dx + 4));
+  cudaError_t e = cudaFuncSetAttribute(outer_sum_kernel<Tio>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  outer_sum_kernel<Tio><<<BH, FT, smem, st>>>(static_cast<const Tio*>(g1),
+                                              static_cast<const Tio*>(x), dW1, T, dh, dx);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_outer_sum(const void* g1, const void* x, float* dW1, int BH, int T, int dh,
+                             int dx, bool bf16, cudaStream_t st) {
+  return bf16 ? launch_outer_sum_t<__nv_bfloat16>(g1, x, dW1, BH, T, dh, dx, st)
+              : launch_outer_sum_t<float>(g1, x, dW1, BH, T, dh, dx, st);
+}
+
+template <typename Tio>
 static cudaError_t launch_tquery_t(const TqueryArgs& a, cudaStream_t st) {
   const size_t smem = layout(a.dx, a.dh, a.dy).total * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(tquery_kernel<Tio>,

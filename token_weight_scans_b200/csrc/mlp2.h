@@ -26,6 +26,12 @@ struct TqueryArgs {
 bool shape_ok(int dx, int dh, int dy);
 cudaError_t launch_tanh(const void* a, void* h, size_t elems, bool bf16, cudaStream_t st);
 cudaError_t launch_tquery(const TqueryArgs& a, bool bf16, cudaStream_t st);
+// out = y - v over `elems` elements (a multiple of 4)
+cudaError_t launch_sub(const void* y, const void* v, void* out, size_t elems, bool bf16,
+                       cudaStream_t st);
+// dW1[bh] = sum_t g1[bh][t] x[bh][t]^T, [dh][dx] fp32 per (b,h); shape_ok() limits apply
+cudaError_t launch_outer_sum(const void* g1, const void* x, float* dW1, int BH, int T, int dh,
+                             int dx, bool bf16, cudaStream_t st);
 
 }  // namespace mlp2
 }  // namespace gradlev

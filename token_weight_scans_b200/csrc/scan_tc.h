@@ -66,6 +66,10 @@ struct TcBwdParams {
   const float* L_init = nullptr;  // [B*H][nseg][dout][din] adjoint at each segment's end, or null
   float* L_first = nullptr;  // [B*H][dout][din] the adjoint at the scan's first token (dL/dS_0),
                              // or null (written by segment 0's CTAs)
+  // Hidden-costate mode: dx_t = (1 - x_t^2) (.) ((W0 + S_t)^T dy_t), the layer's input
+  // gradient at frozen weights through tanh (no adjoint terms). dg, d_eta, d_alpha and
+  // the dW0 partials are then scratch.
+  int local = 0;
 };
 
 constexpr int kChunk = 64;  // tokens per chunk of the tensor-core kernels

@@ -346,10 +346,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int kk = 0; kk < 8; ++kk)  // dx = gam (.) DXb + U W0
             umma_bf16(tbase + COL_RX + LANE16, desc_at(sw128_desc(sU, 16, 1024), (kk >> 2) * TILE + (kk & 3) * 32),
                       desc_at(sw128_desc(sW0, BIG, 1024), kk * 2048), id_tb, 1);
-          #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)  //      + Gs Lam
-            umma_bf16(tbase + COL_RX + LANE16, desc_at(sw128_desc(sG, 16, 1024), (kk >> 2) * TILE + (kk & 3) * 32),
-                      desc_at(sw128_desc(sL, BIG, 1024), kk * 2048), id_tb, 1);
+          if (!p.local) {
+            #pragma unroll
+            for (int kk = 0; kk < 8; ++kk)  //      + Gs Lam
+              umma_bf16(tbase + COL_RX + LANE16, desc_at(sw128_desc(sG, 16, 1024), (kk >> 2) * TILE + (kk & 3) * 32),
+                        desc_at(sw128_desc(sL, BIG, 1024), kk * 2048), id_tb, 1);
+          }
           umma_commit(&sm.lbfree);  // the last product reading the bf16 Lam of the chunk before
           return true;
         };
@@ -635,6 +637,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // each value is exchanged with the partner lane (l ^ 16) as it is consumed
         const int i = ir;
         const float Li = gs.L[i], Lim1 = i == 0 ? 0.f : gs.L[i - 1], eti = gs.eta[i];
+        const float zb = p.local ? 0.f : 1.f;  // keeps the adjoint's intra-chunk term of Z
         const float rai = gs.ra[i], rbi = gs.rb[i];
         const uint32_t b1 = sS + (lo ? CC_AR : CC_QT), b2 = sS + (lo ? CC_Z : CC_BM);
         float tpart = 0.f, t2part = 0.f, t3part = 0.f;
@@ -690,7 +693,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const float bg = gt * bij, al = lt * aij;
                 // lanes < 16: Ar = b kr, Z = a kg - eta_i b kt ; lanes >= 16: Q^T = kg kr, Bm = b
                 v0[d] = kr * (lo ? bg : lt * kg);
-                v1[d] = lo ? fmaf(al, kg, -eti * bg * kt) : bg;
+                v1[d] = lo ? fmaf(al, kg, -zb * eti * bg * kt) : bg;
                 t2part = fmaf(selA * al, qvv[d], t2part);
                 tpart = fmaf(selB * bg * kr, kt, tpart);
                 t3part = fmaf(selB * bg, pvv[d], t3part);
@@ -716,7 +719,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                        pack_bf16(v1[2], v1[3]), pack_bf16(v1[4], v1[5]), pack_bf16(v1[6], v1[7]));
         };
         auto build_above = [&]() {
-          const float neti = -eti;
+          const float neti = -zb * eti;  // the j > i part of Z (zero in hidden-costate mode)
 #pragma unroll
           for (int cc = 0; cc < 2; ++cc) {
             float v0[8], v1[8];
@@ -859,7 +862,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const float ne = -gs.eta[i];
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] *= ne;
-          } else if (p.accumulate && t0 + i < T) {  // add the dx of the slices already done
+          } else if (p.local) {  // hidden-costate mode: (1 - x^2) (.) (W0 + S)^T dy
+            const uint32_t xrow = smem_u32(sm.X[st]) + (wg >> 1) * TILE;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              const uint4 xv = ld_shared_v4(xrow + sw128_off(i, 4 * (wg & 1) + cc));
+              const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const float a0 = bf16_lo(xw[k]), a1 = bf16_hi(xw[k]);
+                v[8 * cc + 2 * k] *= 1.f - a0 * a0;
+                v[8 * cc + 2 * k + 1] *= 1.f - a1 * a1;
+              }
+            }
+          }
+          if (!lo && p.accumulate && t0 + i < T) {  // add the dx of the slices already done
             const uint4* dxo = reinterpret_cast<const uint4*>(p.dx + (tokbase + i) * 128 + 32 * wg);
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
