@@ -44,6 +44,8 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <atomic>
+
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
@@ -990,12 +992,16 @@ cudaError_t launch_bwd(const TcBwdParams& prm, const void* x, const void* g, con
       !make_map_bf16_3d(&mdx, prm.dx, 128, prm.T, BH, C) ||
       !make_map_bf16_3d(&mdg, prm.dg, D, prm.T, BH, C))
     return cudaErrorInvalidValue;
-  static bool attr_set = false;
-  if (!attr_set) {
+  // The shared-memory opt-in is a per-device attribute: set it once on each device.
+  static std::atomic<uint64_t> attr_set{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
+  if (!bit || !(attr_set.load() & bit)) {
     cudaError_t e = cudaFuncSetAttribute(bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_set.fetch_or(bit);
   }
   bwd_kernel<<<(int)BH * prm.nseg, NTHREADS, kSmemBytes, st>>>(mx, mg, mu, ms, mdx, mdg, prm);
   count_launch();

@@ -31,6 +31,8 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <atomic>
+
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
@@ -665,12 +667,16 @@ cudaError_t launch_fwd(const TcFwdParams& prm, const void* x, const void* g, cud
       !make_map_bf16_3d(&ms, prm.ckpt ? (const void*)prm.ckpt : g, 128, prm.dout,
                         prm.ckpt ? BH * nch : 1, 32))
     return cudaErrorInvalidValue;
-  static bool attr_set = false;
-  if (!attr_set) {
+  // The shared-memory opt-in is a per-device attribute: set it once on each device.
+  static std::atomic<uint64_t> attr_set{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
+  if (!bit || !(attr_set.load() & bit)) {
     cudaError_t e = cudaFuncSetAttribute(fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_set.fetch_or(bit);
   }
   const int grid = prm.B * prm.H * (prm.dout / 128) * prm.nseg;
   fwd_kernel<<<grid, NTHREADS, kSmemBytes, st>>>(mx, mg, my, ms, prm);
