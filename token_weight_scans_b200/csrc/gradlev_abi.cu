@@ -522,10 +522,12 @@ gradlev_status gradlev_mlp2_recon(int B, int H, int T, int d_x, int d_h, int d_y
     prm.local = 1;
     if (tc::launch_bwd(prm, h, g2hat, g2til, ckpt, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
   }
-  // the first matrix's gradient over the sequence
-  return mlp2::launch_outer_sum(g1til, x, dW1, B * H, T, d_h, d_x, bf, st) == cudaSuccess
-             ? GRADLEV_OK
-             : GRADLEV_ERR_CUDA;
+  // the first matrix's gradient over the sequence (tensor cores when d_x = 128 too)
+  const cudaError_t e =
+      mlp2::outer_tc_ok(d_h, d_x)
+          ? mlp2::launch_outer_tc(g1til, x, dW1, B * H, T, status, st)
+          : mlp2::launch_outer_sum(g1til, x, dW1, B * H, T, d_h, d_x, bf, st);
+  return e == cudaSuccess ? GRADLEV_OK : GRADLEV_ERR_CUDA;
 }
 
 gradlev_status gradlev_device_status(const void* workspace, void* stream) {

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stddef.h>
 
+#include "common.cuh"
+
 namespace gradlev {
 namespace mlp2 {
 
@@ -32,6 +34,11 @@ cudaError_t launch_sub(const void* y, const void* v, void* out, size_t elems, bo
 // dW1[bh] = sum_t g1[bh][t] x[bh][t]^T, [dh][dx] fp32 per (b,h); shape_ok() limits apply
 cudaError_t launch_outer_sum(const void* g1, const void* x, float* dW1, int BH, int T, int dh,
                              int dx, bool bf16, cudaStream_t st);
+// The same sum on the tensor cores for bf16 with dh = dx = 128 (TMA tiles, tcgen05 MMAs,
+// bounded waits reported through `status`).
+bool outer_tc_ok(int dh, int dx);
+cudaError_t launch_outer_tc(const void* g1, const void* x, float* dW1, int BH, int T,
+                            DeviceStatus* status, cudaStream_t st);
 
 }  // namespace mlp2
 }  // namespace gradlev
