@@ -280,15 +280,45 @@ __global__ void __launch_bounds__(FT, 1) tquery_kernel(TqueryArgs a) {
   }
 }
 
+// 16-byte vectors of the I/O type: 8 bf16 or 4 float per lane-load.
+__device__ __forceinline__ float vget(uint32_t w, int hi) {
+  return __uint_as_float(hi ? (w & 0xffff0000u) : (w << 16));
+}
+__device__ __forceinline__ uint32_t vpack(float lo, float hi) {
+  const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&b);
+}
+
+template <typename Tio, typename F>
+__device__ __forceinline__ uint4 vmap(uint4 u, F f) {
+  if constexpr (sizeof(Tio) == 2) {
+    u.x = vpack(f(vget(u.x, 0)), f(vget(u.x, 1)));
+    u.y = vpack(f(vget(u.y, 0)), f(vget(u.y, 1)));
+    u.z = vpack(f(vget(u.z, 0)), f(vget(u.z, 1)));
+    u.w = vpack(f(vget(u.w, 0)), f(vget(u.w, 1)));
+  } else {
+    u.x = __float_as_uint(f(__uint_as_float(u.x)));
+    u.y = __float_as_uint(f(__uint_as_float(u.y)));
+    u.z = __float_as_uint(f(__uint_as_float(u.z)));
+    u.w = __float_as_uint(f(__uint_as_float(u.w)));
+  }
+  return u;
+}
+
+// h = tanh(a): 16-byte vectors, then a scalar tail
 template <typename Tio>
 __global__ void tanh_kernel(const Tio* __restrict__ a, Tio* __restrict__ h, size_t n) {
-  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-       i += (size_t)gridDim.x * blockDim.x)
-    h[i] = from_f32<Tio>(tanhf(to_f32(a[i])));
+  constexpr int V = 16 / sizeof(Tio);
+  const size_t nv = n / V, stride = (size_t)gridDim.x * blockDim.x;
+  const size_t t = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  for (size_t i = t; i < nv; i += stride)
+    reinterpret_cast<uint4*>(h)[i] =
+        vmap<Tio>(reinterpret_cast<const uint4*>(a)[i], [](float x) { return tanhf(x); });
+  for (size_t i = nv * V + t; i < n; i += stride) h[i] = from_f32<Tio>(tanhf(to_f32(a[i])));
 }
 
 cudaError_t launch_tanh(const void* a, void* h, size_t elems, bool bf16, cudaStream_t st) {
-  const size_t want = (elems + 255) / 256;
+  const size_t want = (elems / (bf16 ? 8 : 4) + 255) / 256;
   const unsigned grid = (unsigned)(want < 148 * 16 ? (want > 0 ? want : 1) : 148 * 16);
   if (bf16)
     tanh_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(a),
@@ -300,11 +330,31 @@ cudaError_t launch_tanh(const void* a, void* h, size_t elems, bool bf16, cudaStr
   return cudaGetLastError();
 }
 
+// out = y - v: 16-byte vectors, then a scalar tail
 template <typename Tio>
 __global__ void sub_kernel(const Tio* __restrict__ y, const Tio* __restrict__ v,
                            Tio* __restrict__ out, size_t n) {
-  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-       i += (size_t)gridDim.x * blockDim.x)
+  constexpr int V = 16 / sizeof(Tio);
+  const size_t nv = n / V, stride = (size_t)gridDim.x * blockDim.x;
+  const size_t t = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  for (size_t i = t; i < nv; i += stride) {
+    const uint4 a = reinterpret_cast<const uint4*>(y)[i];
+    const uint4 b = reinterpret_cast<const uint4*>(v)[i];
+    uint4 r;
+    if constexpr (sizeof(Tio) == 2) {
+      r.x = vpack(vget(a.x, 0) - vget(b.x, 0), vget(a.x, 1) - vget(b.x, 1));
+      r.y = vpack(vget(a.y, 0) - vget(b.y, 0), vget(a.y, 1) - vget(b.y, 1));
+      r.z = vpack(vget(a.z, 0) - vget(b.z, 0), vget(a.z, 1) - vget(b.z, 1));
+      r.w = vpack(vget(a.w, 0) - vget(b.w, 0), vget(a.w, 1) - vget(b.w, 1));
+    } else {
+      r.x = __float_as_uint(__uint_as_float(a.x) - __uint_as_float(b.x));
+      r.y = __float_as_uint(__uint_as_float(a.y) - __uint_as_float(b.y));
+      r.z = __float_as_uint(__uint_as_float(a.z) - __uint_as_float(b.z));
+      r.w = __float_as_uint(__uint_as_float(a.w) - __uint_as_float(b.w));
+    }
+    reinterpret_cast<uint4*>(out)[i] = r;
+  }
+  for (size_t i = nv * V + t; i < n; i += stride)
     out[i] = from_f32<Tio>(to_f32(y[i]) - to_f32(v[i]));
 }
 
@@ -367,7 +417,7 @@ __global__ void __launch_bounds__(FT, 1) outer_sum_kernel(const Tio* __restrict_
 
 cudaError_t launch_sub(const void* y, const void* v, void* out, size_t elems, bool bf16,
                        cudaStream_t st) {
-  const size_t want = (elems + 255) / 256;
+  const size_t want = (elems / (bf16 ? 8 : 4) + 255) / 256;
   const unsigned grid = (unsigned)(want < 148 * 16 ? (want > 0 ? want : 1) : 148 * 16);
   if (bf16)
     sub_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(y),
