@@ -513,7 +513,7 @@ def main():
     do_bwd = "bwd" in cfg.passes
     B, H, T, di, do = cfg.B, cfg.H, cfg.T, cfg.d_in, cfg.d_out
     if tw.gradlev_scan_supported(B, H, T, di, do, code) != 0:
-        raise SystemExit(f"workload {cfg.name} is not supported by this build")
+        raise SystemExit(f"workload {cfg.name} is not supported by the library")
 
     # inputs: each rank its own seeded batch (weak scaling)
     d = inputs.draw(B, H, T, di, do, dtype=cfg.dtype, alpha_mode=cfg.alpha_mode,
