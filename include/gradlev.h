@@ -4,7 +4,13 @@
  * The library evaluates the token-parallel scans of one GradLev adaptive
  * linear layer on the GPU: the forward scan that rebuilds the centred
  * fast-weight trajectory from the layer inputs, the gates and the costates,
- * and the reverse scan that backpropagates an upstream gradient through it.
+ * and the reverse scan that backpropagates an upstream gradient through it
+ * (gradlev_scan_fwd, gradlev_scan_bwd). Around them:
+ *   gradlev_scan_fwd_state / _bwd_state   one part of a split sequence (carried state)
+ *   gradlev_decode_step                   deployment: token-by-token forward, costate, update
+ *   gradlev_consistency_step              a training step from predicted costates
+ *   gradlev_mlp2_recon                    the two-layer reconstruction of the synthetic test
+ *   gradlev_scan_bwd_noalloc              the reverse scan without a workspace argument
  *
  * Definition (Cognaptus, "Parallelize the Training, Keep the Learning Serial",
  * section "Once the gradient signals are known, the weight trajectory becomes
