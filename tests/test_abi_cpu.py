@@ -209,3 +209,26 @@ def test_mlp2_recon_validates_before_launch(L):
     assert call(x=P(0)) == 1
     assert call(dW1=P(4100)) == 1
     assert call(ws=16) == 3
+
+
+def test_binding_refuses_host_tensors():
+    """Host tensors never reach the library: its kernels would dereference them on the GPU."""
+    torch = pytest.importorskip("torch")
+    import token_weight_scans_b200 as tw
+    B, H, T, d = 1, 1, 8, 16
+    x = torch.zeros(B, H, T, d)
+    gates = torch.zeros(B, H, T)
+    W = torch.zeros(H, d, d)
+    S = torch.zeros(B, H, d, d)
+    calls = [
+        lambda: tw.gradlev_scan_fwd(x, x, gates, gates, W),
+        lambda: tw.gradlev_scan_bwd(x, x, gates, gates, W, x),
+        lambda: tw.gradlev_scan_fwd_state(x, x, gates, gates, W, S),
+        lambda: tw.gradlev_scan_bwd_state(x, x, gates, gates, W, x, S, S),
+        lambda: tw.gradlev_decode_step(x, x, gates, gates, W, S),
+        lambda: tw.gradlev_consistency_step(x, x, gates, gates, W, x),
+        lambda: tw.gradlev_mlp2_recon(x, x, x, x, gates, gates, W, W),
+    ]
+    for c in calls:
+        with pytest.raises(tw.GradlevError, match="CUDA device"):
+            c()

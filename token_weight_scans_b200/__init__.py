@@ -138,6 +138,14 @@ def _stream_ptr(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _cuda_device(x):
+    """The device of x, which must be a CUDA device: the library's kernels dereference
+    every pointer on the GPU, so host memory is refused here, before any call."""
+    if not getattr(x, "is_cuda", False):
+        raise GradlevError(f"tensors must be on a CUDA device, got {getattr(x, 'device', type(x))}")
+    return x.device
+
+
 def _check_tensor(name, t, shape, dtype, device):
     if t.shape != tuple(shape):
         raise GradlevError(f"{name}: shape {tuple(t.shape)} != {tuple(shape)}")
@@ -149,13 +157,40 @@ def _check_tensor(name, t, shape, dtype, device):
         raise GradlevError(f"{name}: must be contiguous")
 
 
+def _check_buffer(name, t, nbytes, device):
+    """A caller's byte buffer (workspace, checkpoints): on the call's device, contiguous,
+    at least nbytes long."""
+    if t.device != device:
+        raise GradlevError(f"{name}: device {t.device} != {device}")
+    if not t.is_contiguous():
+        raise GradlevError(f"{name}: must be contiguous")
+    if t.numel() * t.element_size() < nbytes:
+        raise GradlevError(f"{name} too small: {t.numel() * t.element_size()} < {nbytes} bytes")
+
+
 def _workspace(nbytes, device, workspace):
     import torch
     if workspace is None:
         return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
-    if workspace.numel() * workspace.element_size() < nbytes:
-        raise GradlevError(f"workspace too small: {workspace.numel()} < {nbytes}")
+    _check_buffer("workspace", workspace, nbytes, device)
     return workspace
+
+
+def _check_ckpt(ckpt, B, H, T, d_in, d_out, code, device):
+    if ckpt is not None:
+        _check_buffer("ckpt", ckpt, gradlev_scan_ckpt_bytes(B, H, T, d_in, d_out, code), device)
+
+
+def _check_out(out, spec, device):
+    """Caller-supplied outputs: every tensor of `spec` (name -> (shape, dtype)) present and
+    matching; None entries allowed only where spec says so (dtype None)."""
+    for k, (shape, dtype) in spec.items():
+        t = out.get(k)
+        if t is None:
+            if dtype is None:
+                continue
+            raise GradlevError(f"out[{k!r}] missing")
+        _check_tensor(f"out[{k!r}]", t, shape, t.dtype if dtype is None else dtype, device)
 
 
 def _dims(x, g):
@@ -170,7 +205,7 @@ def gradlev_scan_fwd(x, g, eta, alpha, W0, *, y=None, ckpt=None, workspace=None,
     """Forward scan on the GPU. Returns y [B,H,T,d_out] (dtype of x)."""
     import torch
     B, H, T, d_in, d_out = _dims(x, g)
-    dev, dt = x.device, x.dtype
+    dev, dt = _cuda_device(x), x.dtype
     f32 = torch.float32
     _check_tensor("g", g, (B, H, T, d_out), dt, dev)
     _check_tensor("eta", eta, (B, H, T), f32, dev)
@@ -182,6 +217,7 @@ def gradlev_scan_fwd(x, g, eta, alpha, W0, *, y=None, ckpt=None, workspace=None,
     if y is None:
         y = torch.empty((B, H, T, d_out), dtype=dt, device=dev)
     _check_tensor("y", y, (B, H, T, d_out), dt, dev)
+    _check_ckpt(ckpt, B, H, T, d_in, d_out, code, dev)
     nws = gradlev_scan_workspace_bytes(B, H, T, d_in, d_out, code, 0)
     ws = _workspace(nws, dev, workspace)
     st = lib().gradlev_scan_fwd(B, H, T, d_in, d_out, code, _ptr(x), _ptr(g), _ptr(eta),
@@ -196,7 +232,7 @@ def gradlev_scan_bwd(x, g, eta, alpha, W0, dy, *, ckpt=None, workspace=None, str
     """Reverse scan on the GPU. Returns dict dx, dg, deta, dalpha, dW0."""
     import torch
     B, H, T, d_in, d_out = _dims(x, g)
-    dev, dt = x.device, x.dtype
+    dev, dt = _cuda_device(x), x.dtype
     f32 = torch.float32
     _check_tensor("x", x, (B, H, T, d_in), dt, dev)
     _check_tensor("g", g, (B, H, T, d_out), dt, dev)
@@ -211,6 +247,10 @@ def gradlev_scan_bwd(x, g, eta, alpha, W0, dy, *, ckpt=None, workspace=None, str
                    deta=torch.empty((B, H, T), dtype=f32, device=dev),
                    dalpha=torch.empty((B, H, T), dtype=f32, device=dev),
                    dW0=torch.empty((H, d_out, d_in), dtype=f32, device=dev))
+    _check_out(out, dict(dx=((B, H, T, d_in), dt), dg=((B, H, T, d_out), dt),
+                         deta=((B, H, T), f32), dalpha=((B, H, T), f32),
+                         dW0=((H, d_out, d_in), f32)), dev)
+    _check_ckpt(ckpt, B, H, T, d_in, d_out, code, dev)
     nws = gradlev_scan_workspace_bytes(B, H, T, d_in, d_out, code, 1)
     ws = _workspace(nws, dev, workspace)
     st = lib().gradlev_scan_bwd(B, H, T, d_in, d_out, code, _ptr(x), _ptr(g), _ptr(eta),
@@ -235,7 +275,7 @@ def gradlev_scan_fwd_state(x, g, eta, alpha, W0, S0=None, *, y=None, ST=None, ck
     None = 0). Returns (y, ST), ST the deviation after the last token."""
     import torch
     B, H, T, d_in, d_out = _dims(x, g)
-    dev, dt = x.device, x.dtype
+    dev, dt = _cuda_device(x), x.dtype
     f32 = torch.float32
     _check_tensor("x", x, (B, H, T, d_in), dt, dev)
     _check_tensor("g", g, (B, H, T, d_out), dt, dev)
@@ -251,6 +291,7 @@ def gradlev_scan_fwd_state(x, g, eta, alpha, W0, S0=None, *, y=None, ST=None, ck
     if ST is None:
         ST = torch.empty((B, H, d_out, d_in), dtype=f32, device=dev)
     _state_tensor("ST", ST, B, H, d_in, d_out, dev)
+    _check_ckpt(ckpt, B, H, T, d_in, d_out, code, dev)
     nws = gradlev_scan_workspace_bytes(B, H, T, d_in, d_out, code, 0)
     ws = _workspace(nws, dev, workspace)
     st = lib().gradlev_scan_fwd_state(B, H, T, d_in, d_out, code, _ptr(x), _ptr(g), _ptr(eta),
@@ -268,7 +309,7 @@ def gradlev_scan_bwd_state(x, g, eta, alpha, W0, dy, S0=None, LamT=None, *, ckpt
     float32, None = 0). Returns dict dx, dg, deta, dalpha, dW0, dS0."""
     import torch
     B, H, T, d_in, d_out = _dims(x, g)
-    dev, dt = x.device, x.dtype
+    dev, dt = _cuda_device(x), x.dtype
     f32 = torch.float32
     _check_tensor("x", x, (B, H, T, d_in), dt, dev)
     _check_tensor("g", g, (B, H, T, d_out), dt, dev)
@@ -286,7 +327,10 @@ def gradlev_scan_bwd_state(x, g, eta, alpha, W0, dy, S0=None, LamT=None, *, ckpt
                    dalpha=torch.empty((B, H, T), dtype=f32, device=dev),
                    dW0=torch.empty((H, d_out, d_in), dtype=f32, device=dev),
                    dS0=torch.empty((B, H, d_out, d_in), dtype=f32, device=dev))
-    _state_tensor("dS0", out["dS0"], B, H, d_in, d_out, dev)
+    _check_out(out, dict(dx=((B, H, T, d_in), dt), dg=((B, H, T, d_out), dt),
+                         deta=((B, H, T), f32), dalpha=((B, H, T), f32),
+                         dW0=((H, d_out, d_in), f32), dS0=((B, H, d_out, d_in), f32)), dev)
+    _check_ckpt(ckpt, B, H, T, d_in, d_out, code, dev)
     nws = gradlev_scan_workspace_bytes(B, H, T, d_in, d_out, code, 1)
     ws = _workspace(nws, dev, workspace)
     st = lib().gradlev_scan_bwd_state(B, H, T, d_in, d_out, code, _ptr(x), _ptr(g), _ptr(eta),
@@ -305,7 +349,7 @@ def gradlev_decode_step(x, v, eta, alpha, W0, S, *, y=None, g=None, want_g=True,
     [B,H,T,d_out] (g is None when want_g is False and no buffer is given)."""
     import torch
     B, H, T, d_in, d_out = _dims(x, v)
-    dev, dt = x.device, x.dtype
+    dev, dt = _cuda_device(x), x.dtype
     f32 = torch.float32
     _check_tensor("x", x, (B, H, T, d_in), dt, dev)
     _check_tensor("v", v, (B, H, T, d_out), dt, dev)
@@ -338,7 +382,7 @@ def gradlev_consistency_step(x, ghat, eta, alpha, W0, v, lam=1.0, *, want_dv=Tru
     and dv (None when want_dv is False)."""
     import torch
     B, H, T, d_in, d_out = _dims(x, ghat)
-    dev, dt = x.device, x.dtype
+    dev, dt = _cuda_device(x), x.dtype
     f32 = torch.float32
     _check_tensor("x", x, (B, H, T, d_in), dt, dev)
     _check_tensor("ghat", ghat, (B, H, T, d_out), dt, dev)
@@ -359,6 +403,13 @@ def gradlev_consistency_step(x, ghat, eta, alpha, W0, v, lam=1.0, *, want_dv=Tru
                    dalpha=torch.empty((B, H, T), dtype=f32, device=dev),
                    dW0=torch.empty((H, d_out, d_in), dtype=f32, device=dev),
                    dv=torch.empty_like(ghat) if want_dv else None)
+    _check_out(out, dict(y=((B, H, T, d_out), dt), gtil=((B, H, T, d_out), dt),
+                         loss_tok=((B, H, T), f32), loss_c=((B, H, T), f32),
+                         dx=((B, H, T, d_in), dt), dghat=((B, H, T, d_out), dt),
+                         deta=((B, H, T), f32), dalpha=((B, H, T), f32),
+                         dW0=((H, d_out, d_in), f32)), dev)
+    if out.get("dv") is not None:
+        _check_tensor("out['dv']", out["dv"], (B, H, T, d_out), dt, dev)
     ws = _workspace(nws, dev, workspace)
     st = lib().gradlev_consistency_step(
         B, H, T, d_in, d_out, code, _ptr(x), _ptr(ghat), _ptr(eta), _ptr(alpha), _ptr(W0),
@@ -384,7 +435,7 @@ def gradlev_mlp2_recon(x, g1hat, g2hat, v, eta, alpha, W1, W2, control=False, *,
     B, H, T, d_x = x.shape
     d_y = v.shape[-1]
     d_h = W1.shape[1]
-    dev, dt = x.device, x.dtype
+    dev, dt = _cuda_device(x), x.dtype
     f32 = torch.float32
     _check_tensor("x", x, (B, H, T, d_x), dt, dev)
     _check_tensor("g1hat", g1hat, (B, H, T, d_h), dt, dev)
@@ -402,6 +453,9 @@ def gradlev_mlp2_recon(x, g1hat, g2hat, v, eta, alpha, W1, W2, control=False, *,
         out = dict(a=torch.empty_like(g1hat), h=torch.empty_like(g1hat), y=torch.empty_like(v),
                    g2til=torch.empty_like(v), g1til=torch.empty_like(g1hat),
                    dW1=torch.empty((B, H, d_h, d_x), dtype=f32, device=dev))
+    _check_out(out, dict(a=((B, H, T, d_h), dt), h=((B, H, T, d_h), dt),
+                         y=((B, H, T, d_y), dt), g2til=((B, H, T, d_y), dt),
+                         g1til=((B, H, T, d_h), dt), dW1=((B, H, d_h, d_x), f32)), dev)
     ws = _workspace(nws, dev, workspace)
     st = lib().gradlev_mlp2_recon(
         B, H, T, d_x, d_h, d_y, code, _ptr(x), _ptr(g1hat), _ptr(g2hat), _ptr(v), _ptr(eta),
