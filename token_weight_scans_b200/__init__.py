@@ -132,10 +132,15 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
 
 
-def _stream_ptr(stream):
+def _stream_ptr(stream, device=None):
+    """The stream as a cudaStream_t: the given one, which must belong to `device`, or the
+    current stream of `device` (of the current device when `device` is None)."""
     import torch
-    s = torch.cuda.current_stream() if stream is None else stream
-    return ctypes.c_void_p(s.cuda_stream)
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    if device is not None and stream.device != device:
+        raise GradlevError(f"stream is on {stream.device}, the tensors on {device}")
+    return ctypes.c_void_p(stream.cuda_stream)
 
 
 def _cuda_device(x):
@@ -220,9 +225,10 @@ def gradlev_scan_fwd(x, g, eta, alpha, W0, *, y=None, ckpt=None, workspace=None,
     _check_ckpt(ckpt, B, H, T, d_in, d_out, code, dev)
     nws = gradlev_scan_workspace_bytes(B, H, T, d_in, d_out, code, 0)
     ws = _workspace(nws, dev, workspace)
-    st = lib().gradlev_scan_fwd(B, H, T, d_in, d_out, code, _ptr(x), _ptr(g), _ptr(eta),
-                                _ptr(alpha), _ptr(W0), _ptr(y), _ptr(ckpt), _ptr(ws),
-                                ws.numel() * ws.element_size(), _stream_ptr(stream))
+    with torch.cuda.device(dev):  # launches go to the tensors' device
+        st = lib().gradlev_scan_fwd(B, H, T, d_in, d_out, code, _ptr(x), _ptr(g), _ptr(eta),
+                                    _ptr(alpha), _ptr(W0), _ptr(y), _ptr(ckpt), _ptr(ws),
+                                    ws.numel() * ws.element_size(), _stream_ptr(stream, dev))
     _check(st, "gradlev_scan_fwd")
     return y
 
@@ -253,11 +259,12 @@ def gradlev_scan_bwd(x, g, eta, alpha, W0, dy, *, ckpt=None, workspace=None, str
     _check_ckpt(ckpt, B, H, T, d_in, d_out, code, dev)
     nws = gradlev_scan_workspace_bytes(B, H, T, d_in, d_out, code, 1)
     ws = _workspace(nws, dev, workspace)
-    st = lib().gradlev_scan_bwd(B, H, T, d_in, d_out, code, _ptr(x), _ptr(g), _ptr(eta),
-                                _ptr(alpha), _ptr(W0), _ptr(dy), _ptr(out["dx"]),
-                                _ptr(out["dg"]), _ptr(out["deta"]), _ptr(out["dalpha"]),
-                                _ptr(out["dW0"]), _ptr(ckpt), _ptr(ws),
-                                ws.numel() * ws.element_size(), _stream_ptr(stream))
+    with torch.cuda.device(dev):  # launches go to the tensors' device
+        st = lib().gradlev_scan_bwd(B, H, T, d_in, d_out, code, _ptr(x), _ptr(g), _ptr(eta),
+                                    _ptr(alpha), _ptr(W0), _ptr(dy), _ptr(out["dx"]),
+                                    _ptr(out["dg"]), _ptr(out["deta"]), _ptr(out["dalpha"]),
+                                    _ptr(out["dW0"]), _ptr(ckpt), _ptr(ws),
+                                    ws.numel() * ws.element_size(), _stream_ptr(stream, dev))
     _check(st, "gradlev_scan_bwd")
     return out
 
@@ -294,10 +301,11 @@ def gradlev_scan_fwd_state(x, g, eta, alpha, W0, S0=None, *, y=None, ST=None, ck
     _check_ckpt(ckpt, B, H, T, d_in, d_out, code, dev)
     nws = gradlev_scan_workspace_bytes(B, H, T, d_in, d_out, code, 0)
     ws = _workspace(nws, dev, workspace)
-    st = lib().gradlev_scan_fwd_state(B, H, T, d_in, d_out, code, _ptr(x), _ptr(g), _ptr(eta),
-                                      _ptr(alpha), _ptr(W0), _ptr(S0), _ptr(y), _ptr(ST),
-                                      _ptr(ckpt), _ptr(ws), ws.numel() * ws.element_size(),
-                                      _stream_ptr(stream))
+    with torch.cuda.device(dev):  # launches go to the tensors' device
+        st = lib().gradlev_scan_fwd_state(B, H, T, d_in, d_out, code, _ptr(x), _ptr(g), _ptr(eta),
+                                          _ptr(alpha), _ptr(W0), _ptr(S0), _ptr(y), _ptr(ST),
+                                          _ptr(ckpt), _ptr(ws), ws.numel() * ws.element_size(),
+                                          _stream_ptr(stream, dev))
     _check(st, "gradlev_scan_fwd_state")
     return y, ST
 
@@ -333,12 +341,13 @@ def gradlev_scan_bwd_state(x, g, eta, alpha, W0, dy, S0=None, LamT=None, *, ckpt
     _check_ckpt(ckpt, B, H, T, d_in, d_out, code, dev)
     nws = gradlev_scan_workspace_bytes(B, H, T, d_in, d_out, code, 1)
     ws = _workspace(nws, dev, workspace)
-    st = lib().gradlev_scan_bwd_state(B, H, T, d_in, d_out, code, _ptr(x), _ptr(g), _ptr(eta),
-                                      _ptr(alpha), _ptr(W0), _ptr(S0), _ptr(dy), _ptr(LamT),
-                                      _ptr(out["dx"]), _ptr(out["dg"]), _ptr(out["deta"]),
-                                      _ptr(out["dalpha"]), _ptr(out["dW0"]), _ptr(out["dS0"]),
-                                      _ptr(ckpt), _ptr(ws), ws.numel() * ws.element_size(),
-                                      _stream_ptr(stream))
+    with torch.cuda.device(dev):  # launches go to the tensors' device
+        st = lib().gradlev_scan_bwd_state(B, H, T, d_in, d_out, code, _ptr(x), _ptr(g), _ptr(eta),
+                                          _ptr(alpha), _ptr(W0), _ptr(S0), _ptr(dy), _ptr(LamT),
+                                          _ptr(out["dx"]), _ptr(out["dg"]), _ptr(out["deta"]),
+                                          _ptr(out["dalpha"]), _ptr(out["dW0"]), _ptr(out["dS0"]),
+                                          _ptr(ckpt), _ptr(ws), ws.numel() * ws.element_size(),
+                                          _stream_ptr(stream, dev))
     _check(st, "gradlev_scan_bwd_state")
     return out
 
@@ -364,9 +373,10 @@ def gradlev_decode_step(x, v, eta, alpha, W0, S, *, y=None, g=None, want_g=True,
         g = torch.empty((B, H, T, d_out), dtype=dt, device=dev)
     if g is not None:
         _check_tensor("g", g, (B, H, T, d_out), dt, dev)
-    st = lib().gradlev_decode_step(B, H, T, d_in, d_out, _dt_code(dt), _ptr(x), _ptr(v),
-                                   _ptr(eta), _ptr(alpha), _ptr(W0), _ptr(S), _ptr(y), _ptr(g),
-                                   _stream_ptr(stream))
+    with torch.cuda.device(dev):  # launches go to the tensors' device
+        st = lib().gradlev_decode_step(B, H, T, d_in, d_out, _dt_code(dt), _ptr(x), _ptr(v),
+                                       _ptr(eta), _ptr(alpha), _ptr(W0), _ptr(S), _ptr(y), _ptr(g),
+                                       _stream_ptr(stream, dev))
     _check(st, "gradlev_decode_step")
     return y, g
 
@@ -411,12 +421,13 @@ def gradlev_consistency_step(x, ghat, eta, alpha, W0, v, lam=1.0, *, want_dv=Tru
     if out.get("dv") is not None:
         _check_tensor("out['dv']", out["dv"], (B, H, T, d_out), dt, dev)
     ws = _workspace(nws, dev, workspace)
-    st = lib().gradlev_consistency_step(
-        B, H, T, d_in, d_out, code, _ptr(x), _ptr(ghat), _ptr(eta), _ptr(alpha), _ptr(W0),
-        _ptr(v), float(lam), _ptr(out["y"]), _ptr(out["gtil"]), _ptr(out["loss_tok"]),
-        _ptr(out["loss_c"]), _ptr(out["dx"]), _ptr(out["dghat"]), _ptr(out["deta"]),
-        _ptr(out["dalpha"]), _ptr(out["dW0"]), _ptr(out.get("dv")), _ptr(ws),
-        ws.numel() * ws.element_size(), _stream_ptr(stream))
+    with torch.cuda.device(dev):  # launches go to the tensors' device
+        st = lib().gradlev_consistency_step(
+            B, H, T, d_in, d_out, code, _ptr(x), _ptr(ghat), _ptr(eta), _ptr(alpha), _ptr(W0),
+            _ptr(v), float(lam), _ptr(out["y"]), _ptr(out["gtil"]), _ptr(out["loss_tok"]),
+            _ptr(out["loss_c"]), _ptr(out["dx"]), _ptr(out["dghat"]), _ptr(out["deta"]),
+            _ptr(out["dalpha"]), _ptr(out["dW0"]), _ptr(out.get("dv")), _ptr(ws),
+            ws.numel() * ws.element_size(), _stream_ptr(stream, dev))
     _check(st, "gradlev_consistency_step")
     return out
 
@@ -457,14 +468,18 @@ def gradlev_mlp2_recon(x, g1hat, g2hat, v, eta, alpha, W1, W2, control=False, *,
                          y=((B, H, T, d_y), dt), g2til=((B, H, T, d_y), dt),
                          g1til=((B, H, T, d_h), dt), dW1=((B, H, d_h, d_x), f32)), dev)
     ws = _workspace(nws, dev, workspace)
-    st = lib().gradlev_mlp2_recon(
-        B, H, T, d_x, d_h, d_y, code, _ptr(x), _ptr(g1hat), _ptr(g2hat), _ptr(v), _ptr(eta),
-        _ptr(alpha), _ptr(W1), _ptr(W2), 1 if control else 0, _ptr(out["a"]), _ptr(out["h"]),
-        _ptr(out["y"]), _ptr(out["g2til"]), _ptr(out["g1til"]), _ptr(out["dW1"]), _ptr(ws),
-        ws.numel() * ws.element_size(), _stream_ptr(stream))
+    with torch.cuda.device(dev):  # launches go to the tensors' device
+        st = lib().gradlev_mlp2_recon(
+            B, H, T, d_x, d_h, d_y, code, _ptr(x), _ptr(g1hat), _ptr(g2hat), _ptr(v), _ptr(eta),
+            _ptr(alpha), _ptr(W1), _ptr(W2), 1 if control else 0, _ptr(out["a"]), _ptr(out["h"]),
+            _ptr(out["y"]), _ptr(out["g2til"]), _ptr(out["g1til"]), _ptr(out["dW1"]), _ptr(ws),
+            ws.numel() * ws.element_size(), _stream_ptr(stream, dev))
     _check(st, "gradlev_mlp2_recon")
     return out
 
 
 def gradlev_device_status(workspace, stream=None) -> int:
-    return int(lib().gradlev_device_status(_ptr(workspace), _stream_ptr(stream)))
+    import torch
+    with torch.cuda.device(workspace.device):
+        return int(lib().gradlev_device_status(_ptr(workspace),
+                                               _stream_ptr(stream, workspace.device)))
