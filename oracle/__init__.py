@@ -6,8 +6,10 @@ Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 
 The arithmetic lives in ``gradlev_oracle.cpp`` (serial token-by-token loops
 in double / complex<double>, see that file's header for the definition and
-its sources); this module only builds the shared object with g++ and marshals
-numpy arrays through ctypes.
+its sources); this module builds the shared object with g++ and marshals
+numpy arrays through ctypes. The one exception is ``consistency``, which
+composes the C++ forward and reverse scans with a few lines of numpy (the
+residual, the losses and the consistency term's gradient), written out there.
 """
 
 from __future__ import annotations
