@@ -11,6 +11,8 @@
  *   gradlev_consistency_step              a training step from predicted costates
  *   gradlev_mlp2_recon                    the two-layer reconstruction of the synthetic test
  *   gradlev_scan_bwd_noalloc              the reverse scan without a workspace argument
+ *   gradlev_scan_bwd_noalloc_scratch_bytes  its scratch need
+ *   gradlev_noalloc_device_status         its device status word
  *
  * Definition (Cognaptus, "Parallelize the Training, Keep the Learning Serial",
  * section "Once the gradient signals are known, the weight trajectory becomes
@@ -317,10 +319,15 @@ GRADLEV_API gradlev_status gradlev_mlp2_recon(int B, int H, int T, int d_x, int 
  * and `ws_bytes`. Scratch comes from one static device array of
  * GRADLEV_NOALLOC_SCRATCH_BYTES on the current device. The call allocates
  * nothing (no cudaMalloc, cudaFree or allocating library routine).
- *   - Limit: it needs 256 + B*H*d_out*d_in*4 bytes (rounded up to 256) of
- *     scratch, plus gradlev_scan_ckpt_bytes() (rounded up to 256) when ckpt is
- *     NULL; a problem that needs more returns GRADLEV_ERR_WORKSPACE before any
- *     launch. Shape errors return as in gradlev_scan_bwd.
+ *   - Limit: the call needs gradlev_scan_bwd_noalloc_scratch_bytes() of
+ *     scratch. That is the status word and the per-scan dW0 partials
+ *     (B*H*d_out*d_in*4 bytes, times the number of segments per scan when the
+ *     tensor-core path cuts few long scans into segments, plus the segment
+ *     summaries), and, when ckpt is NULL, the chunk-start states as well; with
+ *     ckpt NULL it equals gradlev_scan_workspace_bytes(.., is_bwd = 1). A
+ *     problem that needs more than GRADLEV_NOALLOC_SCRATCH_BYTES returns
+ *     GRADLEV_ERR_WORKSPACE before any launch. Shape errors return as in
+ *     gradlev_scan_bwd.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current) and caches it; make that
  *     first call before any stream capture.
@@ -328,11 +335,27 @@ GRADLEV_API gradlev_status gradlev_mlp2_recon(int B, int H, int T, int d_x, int 
  *     call's contents (each call clears the part that must start at zero).
  *     Calls whose work overlaps on the GPU (different streams, or other host
  *     threads) race on it and give wrong results: serialise them.
- *   - gradlev_device_status() does not apply to this call. */
+ *   - The device status word of the call lives at the start of the array:
+ *     read it with gradlev_noalloc_device_status(), not gradlev_device_status(). */
 GRADLEV_API gradlev_status gradlev_scan_bwd_noalloc(
     int B, int H, int T, int d_in, int d_out, gradlev_dtype dt, const void* x, const void* g,
     const float* eta, const float* alpha, const float* W0, const void* dy, void* dx, void* dg,
     float* d_eta, float* d_alpha, float* dW0, const void* ckpt, void* stream);
+
+/* Scratch bytes gradlev_scan_bwd_noalloc needs for this problem (has_ckpt != 0:
+ * the caller passes checkpoints), or 0 for an unsupported shape. No GPU call.
+ * The method has no counterpart of this call. */
+GRADLEV_API size_t gradlev_scan_bwd_noalloc_scratch_bytes(int B, int H, int T, int d_in,
+                                                         int d_out, gradlev_dtype dt,
+                                                         int has_ckpt);
+
+/* Device status of the last gradlev_scan_bwd_noalloc call on the current
+ * device: synchronises `stream` and reads the status word the kernels leave at
+ * the start of the static scratch array. GRADLEV_OK, GRADLEV_ERR_TIMEOUT if a
+ * bounded device-side wait gave up (that call's outputs are then unspecified),
+ * or GRADLEV_ERR_CUDA. Allocates nothing. The method has no counterpart of
+ * this call. */
+GRADLEV_API gradlev_status gradlev_noalloc_device_status(void* stream);
 
 /* Device status of the last call that used `workspace`: synchronises `stream`
  * and reads the status word the kernels leave at the start of the workspace.

@@ -15,6 +15,10 @@
 // is looked up once per device with cudaGetSymbolAddress, with that device
 // current, the first time the entry point runs on it, and cached.
 //
+// A bounded device-side wait that gives up writes its status word into the
+// start of the array, as it would into a workspace; gradlev_noalloc_device_status
+// reads it back.
+//
 // Nothing here calls cudaMalloc, cudaFree or any allocating routine.
 
 #include <cuda_runtime.h>
@@ -82,8 +86,29 @@ extern "C" GRADLEV_API gradlev_status gradlev_scan_bwd_noalloc(
   void* base = nullptr;
   s = scratch_address(&base);
   if (s != GRADLEV_OK) return s;
+  reset_launch_count();
   // The status word is cleared by bwd_run; the dW0 partials and the states are
   // fully overwritten by the kernels before they are read.
   return bwd_run(B, H, T, d_in, d_out, dt, x, g, eta, alpha, W0, dy, dx, dg, d_eta, d_alpha,
                  dW0, ckpt, static_cast<char*>(base), static_cast<cudaStream_t>(stream));
+}
+
+extern "C" GRADLEV_API size_t gradlev_scan_bwd_noalloc_scratch_bytes(int B, int H, int T, int d_in,
+                                                                   int d_out, gradlev_dtype dt,
+                                                                   int has_ckpt) {
+  if (gradlev_scan_supported(B, H, T, d_in, d_out, dt) != GRADLEV_OK) return 0;
+  return bwd_scratch_bytes(B, H, T, d_in, d_out, dt, has_ckpt == 0);
+}
+
+extern "C" GRADLEV_API gradlev_status gradlev_noalloc_device_status(void* stream) {
+  void* base = nullptr;
+  const gradlev_status s = scratch_address(&base);
+  if (s != GRADLEV_OK) return s;
+  DeviceStatus h;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&h, base, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return GRADLEV_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return GRADLEV_ERR_CUDA;
+  if (h.code == 0) return GRADLEV_OK;
+  return h.code == GRADLEV_ERR_TIMEOUT ? GRADLEV_ERR_TIMEOUT : GRADLEV_ERR_CUDA;
 }
