@@ -368,13 +368,18 @@ GRADLEV_API gradlev_status gradlev_device_status(const void* workspace, void* st
 GRADLEV_API int gradlev_last_launch_count(void);
 
 /* Test hook for the failure-detection path (no GPU fault or hang is involved):
- * with enable != 0, the next bf16 tensor-core gradlev_scan_fwd call withholds
- * one internal completion signal, so one of the kernel's bounded waits runs out
- * after timeout_ms; every CTA then unwinds (in-flight copies and matrix
- * operations are drained, tensor memory is released) and the call's
- * gradlev_device_status() reports GRADLEV_ERR_TIMEOUT. Host-global, one-shot,
- * not thread-safe; for tests only. */
-GRADLEV_API void gradlev_debug_inject_timeout(int enable, int timeout_ms);
+ * the next tensor-core launch at `site` withholds one internal completion
+ * signal, so one of the kernel's bounded waits runs out after timeout_ms; every
+ * CTA then unwinds (in-flight copies and matrix operations are drained, tensor
+ * memory is released) and the call's gradlev_device_status() reports
+ * GRADLEV_ERR_TIMEOUT. Sites (bf16 tensor-core shapes only):
+ *   1  the forward scan's main pass (gradlev_scan_fwd and the calls built on it)
+ *   2  the reverse scan's main kernel
+ *   3  the forward's segment-summary pass (few long scans, cut into segments)
+ *   4  the reverse scan's segment-summary pass
+ *   0  off
+ * Host-global, one-shot, not thread-safe; for tests only. */
+GRADLEV_API void gradlev_debug_inject_timeout(int site, int timeout_ms);
 
 #ifdef __cplusplus
 }

@@ -5,10 +5,8 @@ oracle consumes the dtype-rounded values upcast to float64. Error metric: per
 output tensor, max |gpu - oracle| / max |oracle|, with the bars of
 tests/helpers.TOL (fp32 path 1e-5, bf16 path 2e-2).
 
-Small and mid-size cases are compared element by element on every output;
-the full-size workloads are run in the bench's launch configuration and
-compared on sampled (b, h) scans that the oracle evaluates one by one (dW0 on
-a sampled head, summed over all batch rows).
+Every case, the full-size workloads included, is compared element by element
+on every output.
 """
 
 import numpy as np
@@ -16,7 +14,7 @@ import pytest
 
 import oracle
 from token_weight_scans_b200 import inputs
-from tests.helpers import TOL, heads_slice, rel_err, to_device, to_numpy
+from tests.helpers import TOL, rel_err, to_device, to_numpy
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -182,14 +180,18 @@ def test_one_hot_layout():
     assert gpu["dW0"][h, 3, 5] == 1.0 and np.count_nonzero(gpu["dW0"]) == 1
 
 
-# ----------------------------------------------------------------- full-size, sampled
-
-
-SAMPLED = {2: [(0, 0), (7, 15), (3, 9)], 3: [(0, 0), (7, 15), (4, 6)], 4: [(0, 0), (0, 15)]}
+# ----------------------------------------------------------------- full size, every head
 
 
 @pytest.mark.parametrize("idx", [2, 3, 4])
-def test_full_size_sampled_heads(idx):
+def test_full_size_every_output(idx):
+    """The full-size workloads in the bench's launch configuration (forward writing
+    checkpoints, reverse scan reading them), every output of every (b, h) scan and the
+    whole dW0 against the oracle. The achieved errors are printed (and appended to the
+    file named by GRADLEV_MARGINS_OUT, when set) so that the margins under the bar are on
+    record."""
+    import json
+    import os
     import token_weight_scans_b200 as tw
     cfg = inputs.CONFIGS[idx]
     code = tw.BF16 if cfg.dtype == "bf16" else tw.F32
@@ -198,13 +200,13 @@ def test_full_size_sampled_heads(idx):
     d = inputs.draw_config(cfg)
     do_bwd = "bwd" in cfg.passes
     gpu = run_gpu(d, cfg.dtype, bwd=do_bwd, use_ckpt=True)
-    keys = ("y",) + (("dx", "dg", "deta", "dalpha") if do_bwd else ())
-    for b, h in SAMPLED[idx]:
-        ref = run_oracle(heads_slice(d, b, h), bwd=do_bwd)
-        g1 = {k: gpu[k][b:b + 1, h:h + 1] for k in keys}
-        assert_close(g1, ref, cfg.dtype, keys, f"{cfg.name} (b={b},h={h})")
-    if do_bwd:
-        h = SAMPLED[idx][-1][1]
-        sub = {k: (v[:, h:h + 1] if k != "W0" else v[h:h + 1]) for k, v in d.items()}
-        ref = run_oracle(sub, bwd=True)
-        assert rel_err(gpu["dW0"][h:h + 1], ref["dW0"]) <= TOL[cfg.dtype]
+    ref = run_oracle(d, bwd=do_bwd)
+    keys = ("y",) + (OUTS if do_bwd else ())
+    errs = {k: rel_err(gpu[k], ref[k]) for k in keys}
+    line = json.dumps({"workload": cfg.name, "errors": errs, "bar": TOL[cfg.dtype]})
+    print("MARGINS " + line)
+    out = os.environ.get("GRADLEV_MARGINS_OUT")
+    if out:
+        with open(out, "a") as f:
+            f.write(line + "\n")
+    assert_close(gpu, ref, cfg.dtype, keys, cfg.name)

@@ -215,3 +215,52 @@ def test_tc_segmented_scan_matches_unsegmented():
     assert rel_err(a["dW0"], b["dW0"][:1]) <= 1e-2
     ref = oracle_fwd_bwd(lone)
     check_all(a, ref, "segmented lone scan")
+
+
+# ------------------------------------------------------------------ bounded-wait failure path
+# Each site of the test hook withholds one completion signal of one kernel family: the
+# kernel's bounded wait runs out, every CTA unwinds, the device status reports
+# GRADLEV_ERR_TIMEOUT, and the next call on the same context is correct. No fault, trap
+# or hang is involved.
+
+TIMEOUT = 5  # GRADLEV_ERR_TIMEOUT
+
+
+def _timeout_then_recover(site, B, H, T):
+    import token_weight_scans_b200 as tw
+    d = inputs.draw(B, H, T, 128, 128, dtype="bf16", alpha_mode="log_uniform", seed=70 + site)
+    t = to_device(d, "bf16")
+    ws = torch.zeros(tw.gradlev_scan_workspace_bytes(B, H, T, 128, 128, tw.BF16, 1),
+                     dtype=torch.uint8, device="cuda")
+    ck = torch.empty(tw.gradlev_scan_ckpt_bytes(B, H, T, 128, 128, tw.BF16), dtype=torch.uint8,
+                     device="cuda")
+    fwd = lambda: tw.gradlev_scan_fwd(t["x"], t["g"], t["eta"], t["alpha"], t["W0"], ckpt=ck,
+                                      workspace=ws)
+    bwd = lambda: tw.gradlev_scan_bwd(t["x"], t["g"], t["eta"], t["alpha"], t["W0"], t["dy"],
+                                      ckpt=ck, workspace=ws)
+    if site in (2, 4):  # the reverse scan needs good checkpoints first
+        fwd()
+        assert tw.gradlev_device_status(ws) == 0
+    tw.lib().gradlev_debug_inject_timeout(site, 20)
+    fwd() if site in (1, 3) else bwd()
+    assert tw.gradlev_device_status(ws) == TIMEOUT
+    # the context is intact: normal calls right after succeed and are correct
+    y = fwd()
+    assert tw.gradlev_device_status(ws) == 0
+    out = bwd()
+    assert tw.gradlev_device_status(ws) == 0
+    got = {k: to_numpy(v) for k, v in out.items()}
+    got["y"] = to_numpy(y)
+    check_all(got, oracle_fwd_bwd(d), f"after a timeout at site {site}")
+
+
+def test_tc_bwd_timeout_path_reports_and_recovers():
+    _timeout_then_recover(2, 2, 2, 256)
+
+
+@pytest.mark.parametrize("site", [3, 4], ids=["fwd-summary", "bwd-summary"])
+def test_tc_segment_summary_timeout_reports_and_recovers(site):
+    import token_weight_scans_b200 as tw
+    # one lone long scan: cut into segments, so the summary passes run
+    assert tw.gradlev_scan_workspace_bytes(1, 1, 1024, 128, 128, tw.BF16, 0) > 256
+    _timeout_then_recover(site, 1, 1, 1024)

@@ -24,14 +24,28 @@
 
 namespace gradlev {
 
+static constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // bound of device-side waits
+
 static thread_local int t_launches = 0;
 void count_launch() { ++t_launches; }
 void reset_launch_count() { t_launches = 0; }
 
-// Test hook state (gradlev_debug_inject_timeout): consumed by the next fwd call.
-static int g_inject = 0;
+// Test hook state (gradlev_debug_inject_timeout): the site of the next launch that
+// withholds one completion signal (0 = none), consumed by that launch.
+enum InjectSite { INJ_NONE = 0, INJ_FWD = 1, INJ_BWD = 2, INJ_FWD_SUMMARY = 3, INJ_BWD_SUMMARY = 4 };
+static int g_inject = INJ_NONE;
 static uint64_t g_inject_timeout_ns = 0;
-static constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // bound of device-side waits
+
+// The kernel's inject code and wait bound for a launch at `site` (one-shot).
+static int take_inject(int site, int code, uint64_t* timeout_ns) {
+  if (g_inject != site) {
+    *timeout_ns = kWaitTimeoutNs;
+    return 0;
+  }
+  g_inject = INJ_NONE;
+  *timeout_ns = g_inject_timeout_ns;
+  return code;
+}
 
 static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -122,9 +136,8 @@ static gradlev_status launch_fwd_impl(int B, int H, int T, int din, int dout, gr
                                       DeviceStatus* status, char* seg_ws, cudaStream_t st,
                                       const float* S0, float* ST) {
   if (use_tc(din, dout, dt)) {
-    const int inject = y ? g_inject : 0;
-    const uint64_t tmo = inject ? g_inject_timeout_ns : kWaitTimeoutNs;
-    if (y) g_inject = 0;
+    uint64_t tmo = kWaitTimeoutNs;
+    const int inject = y ? take_inject(INJ_FWD, 1, &tmo) : 0;
     const SegPlan sp = fwd_plan(B, H, T, dout);
     tc::TcFwdParams prm{B, H, T, din, dout, eta, alpha, W0, static_cast<__nv_bfloat16*>(y),
                         static_cast<__nv_bfloat16*>(ckpt), status, tmo, inject};
@@ -133,8 +146,7 @@ static gradlev_status launch_fwd_impl(int B, int H, int T, int din, int dout, gr
       tc::TcFwdParams sum = prm;  // each segment's local state and log-decay
       sum.y = nullptr;
       sum.ckpt = nullptr;
-      sum.inject = 0;
-      sum.timeout_ns = kWaitTimeoutNs;
+      sum.inject = take_inject(INJ_FWD_SUMMARY, 3, &sum.timeout_ns);
       sum.nseg = sp.nseg;
       sum.seg_chunks = sp.seg_chunks;
       sum.S_final = sb.loc;
@@ -188,6 +200,7 @@ gradlev_status bwd_run(int B, int H, int T, int din, int dout, gradlev_dtype dt,
       const SegBufs sb = seg_bufs(seg_ws, B, H, din, dout, sp.nseg);
       tc::TcFwdParams sum{B, H, T, din, dout, eta, alpha, W0, nullptr, nullptr, status,
                           kWaitTimeoutNs, 0};
+      sum.inject = take_inject(INJ_BWD_SUMMARY, 3, &sum.timeout_ns);
       sum.nseg = sp.nseg;
       sum.seg_chunks = sp.seg_chunks;
       sum.S_final = sb.loc;
@@ -210,6 +223,7 @@ gradlev_status bwd_run(int B, int H, int T, int din, int dout, gradlev_dtype dt,
       prm.seg_chunks = sp.seg_chunks;
       prm.L_init = L_init;
       prm.L_first = io.dS0;
+      prm.inject = take_inject(INJ_BWD, 2, &prm.timeout_ns);
       if (tc::launch_bwd(prm, x, g, dy, states, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
     }
     // partials are [B][nseg][H]: a fixed-order sum over b and the segments
@@ -543,8 +557,8 @@ gradlev_status gradlev_device_status(const void* workspace, void* stream) {
 
 int gradlev_last_launch_count(void) { return t_launches; }
 
-void gradlev_debug_inject_timeout(int enable, int timeout_ms) {
-  g_inject = enable ? 1 : 0;
+void gradlev_debug_inject_timeout(int site, int timeout_ms) {
+  g_inject = (site >= INJ_FWD && site <= INJ_BWD_SUMMARY) ? site : INJ_NONE;
   g_inject_timeout_ns = (uint64_t)(timeout_ms > 0 ? timeout_ms : 1) * 1000000ull;
 }
 

@@ -27,7 +27,8 @@ struct TcFwdParams {
   __nv_bfloat16* ckpt;      // [B*H][n_chunks][dout][din] chunk-start states, or null
   DeviceStatus* status;     // device status word (workspace head)
   uint64_t timeout_ns;      // bound of every wait inside the kernel
-  int inject;               // test hook: 1 = withhold one completion signal
+  int inject;               // test hook: 1 = withhold one completion signal of the main
+                            // pass, 3 = of the state carry (summary passes)
   int nseg = 1;             // segments per scan
   int seg_chunks = 1 << 30; // chunks per segment (the last one may be shorter)
   const float* S_init = nullptr;  // [B*H][nseg][dout][din] segment start states, or null (= 0)
@@ -70,6 +71,7 @@ struct TcBwdParams {
   // gradient at frozen weights through tanh (no adjoint terms). dg, d_eta, d_alpha and
   // the dW0 partials are then scratch.
   int local = 0;
+  int inject = 0;           // test hook: 2 = withhold one completion signal
 };
 
 constexpr int kChunk = 64;  // tokens per chunk of the tensor-core kernels

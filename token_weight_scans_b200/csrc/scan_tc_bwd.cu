@@ -335,7 +335,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int kk = 0; kk < 8; ++kk)  // DXb = U S_in
             umma_bf16(tbase + COL_RX + LANE16, desc_at(sw128_desc(sU, 16, 1024), (kk >> 2) * TILE + (kk & 3) * 32),
                       desc_at(sw128_desc(sS, BIG, 1024), kk * 2048), id_tb, kk > 0);
-          umma_commit(&sm.b1full);  // R1, the Gram products, dW0 and DXb
+          if (!(p.inject == 2 && it == 1)) umma_commit(&sm.b1full);  // R1, Gram, dW0, DXb
           return true;
         };
         auto phase2a = [&](int it) -> bool {  // dx terms that need only Gs and gam (.) DXb
