@@ -11,30 +11,23 @@
 //   y_i = W0 x_i + 2^{L_{i-1}} S x_i + sum_{j<i} (x_i.x_j) (-eta_j) 2^{L_{i-1}-L_j} g_j
 //   S'  = 2^{L_{C-1}} S + sum_j (-eta_j 2^{L_{C-1}-L_j}) g_j x_j^T
 //
-// Products (the output ones d-major: d_out on the 128 TMEM lanes, the chunk's
-// tokens on the columns, so that every product but the Gram one has M = 128):
-//   K     = X X^T                        (M=64 tokens, N=64, K=d_in)        -> TMEM
-//   P_ij  = K_ij (-eta_j) 2^{L_{i-1}-L_j} (j < i), bf16 in shared memory
-//   Y1^T  = W0 X^T + G^T P^T             (M=128, N=64, K=d_in then C; W0 is a
-//                                         bf16 A operand kept in TMEM)      -> TMEM
-//   Y2^T  = S X^T                        (M=128, N=64, K=d_in)              -> TMEM
-//   dS    = G^T Xhat, Xhat_j = w_j x_j   (M=128, N=d_in, K=C)               -> TMEM
-//   y_i   = Y1^T[:, i] + 2^{L_{i-1}} Y2^T[:, i];  S <- 2^{L_{C-1}} S + dS (fp32, registers)
+// Products (the output ones token-major, so that each epilogue thread owns a
+// contiguous piece of one output row):
+//   K    = X X^T                         (M=64 tokens, N=64, K=d_in)        -> TMEM
+//   P_ij = K_ij (-eta_j) 2^{L_{i-1}-L_j}  (j < i), bf16 in shared memory
+//   Y1   = X W0^T + P G                   (M=64 tokens, N=128, K=d_in+C)     -> TMEM
+//   Y2   = X S^T                          (M=64 tokens, N=128, K=d_in)       -> TMEM
+//   dS   = G^T Xhat, Xhat_j = w_j x_j     (M=128, N=d_in, K=C)               -> TMEM
+//   y_i  = Y1[i, :] + 2^{L_{i-1}} Y2[i, :]; S <- 2^{L_{C-1}} S + dS (fp32, registers)
 //
-// Warp roles (20 warps), each running through the chunks on its own, tied by
-// mbarriers so that the roles overlap across chunks:
-//   0      TMA producer (X and G tiles, 4 stages)
-//   1      MMA issuer and TMEM owner
-//   2      gate prep (log2 alpha cumulative sums, prefetched) + half of Xhat
-//   3      the other half of Xhat (double-buffered)
-//   4..7   mask: K -> P for each chunk, a chunk ahead of the output products
-//   8..15  state: the fp32 state in registers (warpgroup h owns columns
-//          [64h, 64h+64)), its bf16 copy for the S X^T product and the
-//          chunk-start checkpoints (TMA-stored from that copy)
-//   16..19 output epilogue: y from Y1^T and Y2^T, transposed into the chunk's
-//          X tile (free by then) and TMA-stored
-// Without y (state-carry summaries, checkpoint-only sweeps) only the producer,
-// MMA, gate/Xhat and state roles run.
+// Warp roles (12 warps): 0 TMA producer, 1 MMA issuer (+TMEM owner), 2 gate
+// prep (log2 alpha cumulative sums, prefetched) and half of the scaled-X tile,
+// 3 the other half of the scaled-X tile (double-buffered, so these two warps
+// run a chunk ahead), 4..11 two math warpgroups (state update, mask of the
+// next chunk, output epilogue): warpgroup h owns state columns [64h, 64h+64)
+// and output columns [64h, 64h+64) of the slice. The bf16 copy of the state is
+// double-buffered so the state update of chunk c overlaps the S X^T product of
+// chunk c.
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -55,21 +48,21 @@ using namespace sm100;
 namespace {
 
 constexpr int C = 64;          // tokens per chunk
-constexpr int NS = 4;          // TMA stages (X and G tiles)
+constexpr int NS = 2;          // TMA stages (X and G tiles)
 constexpr int GS = 4;          // gate slots
-constexpr int NTHREADS = 640;  // 20 warps
+constexpr int NTHREADS = 384;  // 12 warps
 constexpr int TILE = C * 128;  // bytes of one [64 rows x 128 B] swizzled block
 constexpr int BIG = 128 * 128; // bytes of one [128 rows x 128 B] swizzled block
 
-// TMEM columns (512 allocated).
-//   [0, 64)    K, an M=64 product: rows in lanes 0-15 of each 32-lane sub-partition
-//   [64, 128)  W0 slice as a bf16 A operand (lane n = row n, two k per column)
-//   [128, 384) two output buffers of 128 columns: Y1^T in the first 64, Y2^T in the next 64
-//   [384, 512) dS
-constexpr uint32_t COL_K = 0;
-constexpr uint32_t COL_W0 = 64;
-constexpr uint32_t COL_Y = 128;
-constexpr uint32_t COL_DS = 384;
+// TMEM columns (512 allocated). An M=64 product occupies 16 lanes of each
+// 32-lane sub-partition (row i at lane 32 (i / 16) + i % 16, plus 16 when its
+// address carries LANE16). Y1 and Y2 of one chunk share 128 columns, Y1 in the
+// lower and Y2 in the upper 16 lanes, so that one load gives a thread pair
+// (l, l + 16) both halves of the same token row; the pair is double-buffered.
+constexpr uint32_t COL_K0 = 0, COL_K1 = 64;      // K = X X^T, double buffer (lanes 0-15)
+constexpr uint32_t COL_Y = 128;                  // + 128 * buffer: Y1 | Y2 (128 columns)
+constexpr uint32_t COL_DS = 384;                 // dS (128 columns, all 128 lanes)
+constexpr uint32_t LANE16 = 16u << 16;
 
 // With M = L_{31}, the mask factor -eta_j 2^{L_{i-1} - L_j} = ra_i ca_j whenever
 // every exponent stays inside fp32 range: fac = (|L_{C-1}| <= 120).
@@ -87,20 +80,21 @@ struct GateSlot {
 
 struct Smem {
   // 1024-byte aligned tiles first
-  uint8_t X[NS][2 * TILE];     // k-blocks [0,64), [64,128): 64 token rows x 128 B; after the
-                               // chunk's products, the y staging tile (n-blocks of the slice)
+  uint8_t X[NS][2 * TILE];     // k-blocks [0,64), [64,128): 64 token rows x 128 B
   uint8_t G[NS][2 * TILE];     // n-blocks of the slice: 64 token rows x 128 B
-  uint8_t S[2][BIG];           // [k-block]: 128 n rows x 128 B (bf16 state)
+  uint8_t W0[2][BIG];          // k-blocks: 128 n rows x 128 B (bf16 W0 slice)
+  uint8_t S[2][2][BIG];        // [buffer][k-block]: 128 n rows x 128 B (bf16 state)
   uint8_t Xh[2][2 * TILE];     // [buffer] scaled X, same layout as X
-  uint8_t P[2][TILE];          // [buffer] 64 token rows (i) x 128 B (j)
+  uint8_t P[TILE];             // 64 token rows (i) x 128 B (j)
+  uint8_t Ys[2 * TILE];        // y staging: n-blocks of 64 token rows x 128 B (TMA store)
   GateSlot gates[GS];
   uint64_t full[NS], empty[NS];
   uint64_t gfull[GS], gempty[GS];
-  uint64_t kfull, kfree;
-  uint64_t xhready[2], xhfree[2];
-  uint64_t pready[2], pfree[2];
-  uint64_t yfull[2], yfree[2];
-  uint64_t dsfull, dsfree, sready, sfree, done;
+  uint64_t kfull[2], kfree[2];
+  uint64_t xhready[2], xhfree[2];  // per scaled-X buffer
+  uint64_t sready[2], sfree[2];    // per bf16 state buffer
+  uint64_t yfull[2], yfree[2];    // per Y1 | Y2 buffer
+  uint64_t pready, dsfull, dsfree, done;
   uint32_t tmem_base;
   int abort;
 };
@@ -115,12 +109,15 @@ enum : uint32_t {
   W_MMA_SREADY, W_MMA_DONE,
   W_GATE_EMPTY = 0x201,
   W_XH_FULL = 0x301, W_XH_GFULL, W_XH_FREE,
-  W_K_GFULL = 0x401, W_K_KFULL, W_K_PFREE,
-  W_S_DSFULL = 0x501, W_S_SFREE,
-  W_E_YFULL = 0x601, W_E_GFULL,
+  W_M_GFULL = 0x401, W_M_KFULL, W_M_DSFULL, W_M_SFREE, W_M_YFULL,
 };
 
-constexpr uint32_t BAR_EPI = 2;  // named barrier of the four epilogue warps
+// Waits until at most n (0..2) of this thread's TMA store groups still read shared memory.
+__device__ __forceinline__ void store_reads_pending_at_most(int n) {
+  if (n <= 0) tma_store_wait_read_n<0>();
+  else if (n == 1) tma_store_wait_read_n<1>();
+  else tma_store_wait_read_n<2>();
+}
 
 }  // namespace
 
@@ -146,9 +143,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   auto cg = [&](int c) { return p.reverse ? c1 - 1 - c : c0 + c; };
   const size_t seg_row = (size_t)bh * p.nseg + seg;  // [bh][seg] index of the segment states
   const WaitCtx wc{&sm.abort, p.status, p.timeout_ns};
-  // y outputs (and with them the Gram, mask, output products and epilogue)
-  const bool yout = !p.summary && p.y != nullptr;
-  const bool has_ck = !p.summary && p.ckpt != nullptr;
 
   if (threadIdx.x == 0) {
     sm.abort = 0;
@@ -158,64 +152,63 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     for (int g = 0; g < GS; ++g) {
       mbar_init(&sm.gfull[g], 32);
-      // Xhat warps (2) + state warps (8) [+ mask warps (4) + epilogue warps (4)]
-      mbar_init(&sm.gempty[g], yout ? 18 : 10);
+      mbar_init(&sm.gempty[g], 10);  // 2 scaled-X warps + 8 math warps
     }
-    mbar_init(&sm.kfull, 1);
-    mbar_init(&sm.kfree, 4);
     for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.kfull[b], 1);
+      mbar_init(&sm.kfree[b], 8);
       mbar_init(&sm.xhready[b], 2);
       mbar_init(&sm.xhfree[b], 1);
-      mbar_init(&sm.pready[b], 4);
-      mbar_init(&sm.pfree[b], 1);
-      mbar_init(&sm.yfull[b], 1);
-      mbar_init(&sm.yfree[b], 4);
+      mbar_init(&sm.sready[b], 8);
+      mbar_init(&sm.sfree[b], 1);
     }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.yfull[b], 1);
+      mbar_init(&sm.yfree[b], 8);
+    }
+    mbar_init(&sm.pready, 8);
     mbar_init(&sm.dsfull, 1);
     mbar_init(&sm.dsfree, 8);
-    mbar_init(&sm.sready, 8);
-    mbar_init(&sm.sfree, 1);
     mbar_init(&sm.done, 1);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmX);
     prefetch_tmap(&tmG);
-    if (yout) prefetch_tmap(&tmY);
-    if (has_ck) prefetch_tmap(&tmS);
+    if (p.y) prefetch_tmap(&tmY);
+    if (p.ckpt) prefetch_tmap(&tmS);
   }
   if (warp == 1) {
     tmem_alloc(&sm.tmem_base, 512);
     tmem_relinquish();
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tbase = sm.tmem_base;
-  if (yout && warp >= 4 && warp < 8) {
-    // the bf16 W0 slice into TMEM (A operand of W0 X^T): lane n = row n, column c holds
-    // elements 2c and 2c + 1
-    const int q = warp & 3, n = 32 * q + lane;
-    const float* W0r = p.W0 + ((size_t)h * p.dout + n0 + n) * 128;
-#pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-      float v[32];
-#pragma unroll
-      for (int e = 0; e < 32; e += 4) {
-        const float4 a = *reinterpret_cast<const float4*>(W0r + 64 * hf + 2 * e);
-        const float4 b = *reinterpret_cast<const float4*>(W0r + 64 * hf + 2 * e + 4);
-        v[e] = __uint_as_float(pack_bf16(a.x, a.y));
-        v[e + 1] = __uint_as_float(pack_bf16(a.z, a.w));
-        v[e + 2] = __uint_as_float(pack_bf16(b.x, b.y));
-        v[e + 3] = __uint_as_float(pack_bf16(b.z, b.w));
+  // W0 slice -> bf16 swizzled K-major tiles; S_0 = 0
+  if (warp >= 4) {
+    const int t = threadIdx.x - 128;  // 0..255
+    const float* W0 = p.W0 + ((size_t)h * p.dout + n0) * 128;
+    for (int idx = t; idx < 128 * 16; idx += 256) {  // (row n, 16-byte chunk of 8 k)
+      const int n = idx >> 4, ck = idx & 15;
+      const int kb = ck >> 3, c = ck & 7;
+      const float4 a = *reinterpret_cast<const float4*>(W0 + (size_t)n * 128 + ck * 8);
+      const float4 b = *reinterpret_cast<const float4*>(W0 + (size_t)n * 128 + ck * 8 + 4);
+      st_shared_v4(smem_u32(sm.W0[kb]) + sw128_off(n, c), pack_bf16(a.x, a.y),
+                   pack_bf16(a.z, a.w), pack_bf16(b.x, b.y), pack_bf16(b.z, b.w));
+      if (p.S_init) {  // the segment's start state (rows of this slice), fp32 -> bf16
+        const float* si = p.S_init + (seg_row * p.dout + n0 + n) * 128 + ck * 8;
+        const float4 u = *reinterpret_cast<const float4*>(si);
+        const float4 v = *reinterpret_cast<const float4*>(si + 4);
+        st_shared_v4(smem_u32(sm.S[0][kb]) + sw128_off(n, c), pack_bf16(u.x, u.y),
+                     pack_bf16(u.z, u.w), pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
+      } else {
+        st_shared_v4(smem_u32(sm.S[0][kb]) + sw128_off(n, c), 0u, 0u, 0u, 0u);
       }
-      tmem_st32(tbase + COL_W0 + ((uint32_t)(32 * q) << 16) + 32 * hf, v);
     }
-    tmem_st_wait();
+    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  const uint32_t tbase = sm.tmem_base;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -240,86 +233,73 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t id_k = idesc_bf16(64, 64, false, false);    // X X^T
-      const uint32_t id_y = idesc_bf16(128, 64, false, false);   // W0 X^T (W0 in TMEM), S X^T
-      const uint32_t id_gp = idesc_bf16(128, 64, true, false);   // G^T P^T (G n-contiguous)
+      const uint32_t id_y = idesc_bf16(64, 128, false, false);   // X W0^T, X S^T
+      const uint32_t id_pg = idesc_bf16(64, 128, false, true);   // P G (G n-contiguous)
       const uint32_t id_ds = idesc_bf16(128, 128, true, true);   // G^T Xhat
-      const uint32_t sS = smem_u32(sm.S[0]);
-      // K_c (the mask warps have read K_{c-1})
-      auto issue_k = [&](int c) -> bool {
-        const int s = c % NS;
-        if (!mbar_wait(&sm.full[s], (c / NS) & 1, wc, W_MMA_FULL)) return false;
-        if (!mbar_wait(&sm.kfree, (c & 1) ^ 1, wc, W_MMA_KFREE)) return false;
-        tc_fence_after();
-        const uint32_t sX = smem_u32(sm.X[s]);
-        const uint64_t dX = sw128_desc(sX, 16, 1024);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * TILE + (kk & 3) * 32;
-          umma_bf16(tbase + COL_K, desc_at(dX, off), desc_at(dX, off), id_k, kk > 0);
-        }
-        if (!(p.inject == 1 && c == 1)) umma_commit(&sm.kfull);
-        return true;
-      };
-      bool ok = true;
-      if (yout && nch > 0) ok = issue_k(0);
-      for (int c = 0; c < nch && ok; ++c) {
+      const uint32_t sW0 = smem_u32(sm.W0[0]), sP = smem_u32(sm.P);
+      for (int c = 0; c < nch; ++c) {
         const int s = c % NS, b = c & 1;
         const uint32_t sX = smem_u32(sm.X[s]), sG = smem_u32(sm.G[s]);
-        const uint32_t sXh = smem_u32(sm.Xh[b]);
-        // ---- dS_c = G^T Xhat (the state warps have read dS_{c-1})
-        if (!(ok = mbar_wait(&sm.full[s], (c / NS) & 1, wc, W_MMA_FULL))) break;
-        if (!(ok = mbar_wait(&sm.xhready[b], (c >> 1) & 1, wc, W_MMA_XREADY))) break;
-        if (!(ok = mbar_wait(&sm.dsfree, (c & 1) ^ 1, wc, W_MMA_DSFREE))) break;
-        tc_fence_after();
-        {
-          const uint64_t dG = sw128_desc(sG, TILE, 1024), dXh = sw128_desc(sXh, TILE, 1024);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_bf16(tbase + COL_DS, desc_at(dG, kk * 2048), desc_at(dXh, kk * 2048), id_ds,
-                      kk > 0);
+        const uint32_t sXh = smem_u32(sm.Xh[b]), sS = smem_u32(sm.S[b][0]);
+        if (!mbar_wait(&sm.full[s], (c / NS) & 1, wc, W_MMA_FULL)) break;
+        if (!p.summary) {
+          if (!mbar_wait(&sm.kfree[b], ((c >> 1) & 1) ^ 1, wc, W_MMA_KFREE)) break;
+          tc_fence_after();
+          // K = X X^T
+          #pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * TILE + (kk & 3) * 32;
+            umma_bf16(tbase + (b ? COL_K1 : COL_K0), desc_at(sw128_desc(sX, 16, 1024), off),
+                      desc_at(sw128_desc(sX, 16, 1024), off), id_k, kk > 0);
+          }
+          if (!(p.inject == 1 && c == 1)) umma_commit(&sm.kfull[b]);
         }
+        // dS = G^T Xhat
+        if (!mbar_wait(&sm.xhready[b], (c >> 1) & 1, wc, W_MMA_XREADY)) break;
+        if (c > 0 && !mbar_wait(&sm.dsfree, (c - 1) & 1, wc, W_MMA_DSFREE)) break;
+        tc_fence_after();
+        #pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_bf16(tbase + COL_DS, desc_at(sw128_desc(sG, TILE, 1024), kk * 2048),
+                    desc_at(sw128_desc(sXh, TILE, 1024), kk * 2048), id_ds, kk > 0);
         if (!(p.inject == 3 && c == 1)) umma_commit(&sm.dsfull);
         umma_commit(&sm.xhfree[b]);
-        if (!yout) {  // state carry only: the stage is free once dS has read it
+        if (p.summary) {  // state carry only: the stage is free once dS has read it
           umma_commit(&sm.empty[s]);
           continue;
         }
-        // ---- K of the next chunk (the mask warps build its P while chunk c's products run)
-        if (c + 1 < nch && !(ok = issue_k(c + 1))) break;
-        // ---- Y1^T_c = W0 X^T + G^T P^T into buffer b (the epilogue of chunk c - 2 read it)
-        const uint32_t tY1 = tbase + COL_Y + 128 * b, tY2 = tY1 + 64;
-        if (!(ok = mbar_wait(&sm.yfree[b], ((c >> 1) & 1) ^ 1, wc, W_MMA_YFREE))) break;
+        // Y1 = X W0^T into buffer b (the epilogue of chunk c - 2 has read it)
+        const uint32_t tY1 = tbase + COL_Y + 128 * b, tY2 = tY1 + LANE16;
+        if (!mbar_wait(&sm.yfree[b], ((c >> 1) & 1) ^ 1, wc, W_MMA_YFREE)) break;
         tc_fence_after();
-        {
-          const uint64_t dX = sw128_desc(sX, 16, 1024);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            umma_bf16_tmem_a(tY1, tbase + COL_W0 + 8 * kk,
-                             desc_at(dX, (kk >> 2) * TILE + (kk & 3) * 32), id_y, kk > 0);
+        #pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t aoff = (kk >> 2) * TILE + (kk & 3) * 32;
+          const uint32_t boff = (kk >> 2) * BIG + (kk & 3) * 32;
+          umma_bf16(tY1, desc_at(sw128_desc(sX, 16, 1024), aoff), desc_at(sw128_desc(sW0, 16, 1024), boff), id_y,
+                    kk > 0);
         }
-        if (!(ok = mbar_wait(&sm.pready[b], (c >> 1) & 1, wc, W_MMA_PREADY))) break;
+        // Y2 = X S^T (state buffer c & 1, written by the state update of chunk c - 1)
+        if (c > 0 && !mbar_wait(&sm.sready[b], ((c - 1) >> 1) & 1, wc, W_MMA_SREADY)) break;
         tc_fence_after();
-        {
-          const uint64_t dG = sw128_desc(sG, TILE, 1024), dP = sw128_desc(smem_u32(sm.P[b]), 16, 1024);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_bf16(tY1, desc_at(dG, kk * 2048), desc_at(dP, kk * 32), id_gp, 1);
+        #pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t aoff = (kk >> 2) * TILE + (kk & 3) * 32;
+          const uint32_t boff = (kk >> 2) * BIG + (kk & 3) * 32;
+          umma_bf16(tY2, desc_at(sw128_desc(sX, 16, 1024), aoff), desc_at(sw128_desc(sS, 16, 1024), boff), id_y,
+                    kk > 0);
         }
-        umma_commit(&sm.pfree[b]);
-        // ---- Y2^T_c = S_c X^T (S_c written by the state update of chunk c - 1)
-        if (!(ok = mbar_wait(&sm.sready, c & 1, wc, W_MMA_SREADY))) break;
+        umma_commit(&sm.sfree[b]);
+        // Y1 += P G. The mask of chunk c + 1 overwrites P only after the K product
+        // of chunk c + 1 has completed, which is committed after these.
+        if (!mbar_wait(&sm.pready, c & 1, wc, W_MMA_PREADY)) break;
         tc_fence_after();
-        {
-          const uint64_t dX = sw128_desc(sX, 16, 1024), dS = sw128_desc(sS, 16, 1024);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t aoff = (kk >> 2) * BIG + (kk & 3) * 32;
-            const uint32_t boff = (kk >> 2) * TILE + (kk & 3) * 32;
-            umma_bf16(tY2, desc_at(dS, aoff), desc_at(dX, boff), id_y, kk > 0);
-          }
-        }
-        umma_commit(&sm.sfree);
+        #pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_bf16(tY1, desc_at(sw128_desc(sP, 16, 1024), kk * 32),
+                    desc_at(sw128_desc(sG, TILE, 1024), kk * 2048), id_pg, 1);
         umma_commit(&sm.yfull[b]);
+        umma_commit(&sm.empty[s]);
       }
       // teardown: every issued MMA completes before TMEM is released
       umma_commit(&sm.done);
@@ -422,77 +402,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
     }
     if (ok && gate_warp && lane == 0 && p.seg_L && slice == 0) p.seg_L[seg_row] = Lseg;
-  } else if (warp < 8) {
-    // ------------------------------------------------------------ mask warps
-    // Warp q: token rows [16q, 16q+16) of K, in lanes 0-15 of its sub-partition.
-    const int q = warp & 3;
-    const uint32_t lane_off = (uint32_t)(32 * q) << 16;
-    bool ok = true;
-    for (int c = 0; c < nch && yout && ok; ++c) {
-      const int g = c % GS, b = c & 1;
-      const GateSlot& gs = sm.gates[g];
-      ok = ok && mbar_wait_warp(&sm.gfull[g], (c / GS) & 1, wc, W_K_GFULL);
-      ok = ok && mbar_wait_warp(&sm.kfull, c & 1, wc, W_K_KFULL);
-      // P buffer b was last read by the G^T P^T product of chunk c - 2
-      ok = ok && mbar_wait_warp(&sm.pfree[b], ((c >> 1) & 1) ^ 1, wc, W_K_PFREE);
-      if (!ok) break;
-      tc_fence_after();
-      const bool mine = lane < 16;
-      const int i = 16 * q + (lane & 15);
-      const uint32_t prow = smem_u32(sm.P[b]);
-      const float Lm1 = i == 0 ? 0.f : gs.L[i - 1];
-      const float rai = gs.ra[i];
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        float v[32];
-        tmem_ld32(tbase + COL_K + lane_off + 32 * hf, v);
-        tmem_ld_wait();
-        if (hf == 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.kfree);
-        }
-        if (mine) {
-          uint32_t pk[16];
-          if (gs.fac) {
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const int j = 32 * hf + e;
-              const float p0 = (j < i) ? v[e] * rai * gs.ca[j] : 0.f;
-              const float p1 = (j + 1 < i) ? v[e + 1] * rai * gs.ca[j + 1] : 0.f;
-              pk[e >> 1] = pack_bf16(p0, p1);
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const int j = 32 * hf + e;
-              const float f0 = exp2f(fminf(Lm1 - gs.L[j], 0.f));
-              const float f1 = exp2f(fminf(Lm1 - gs.L[j + 1], 0.f));
-              const float p0 = (j < i) ? v[e] * (-gs.eta[j]) * f0 : 0.f;
-              const float p1 = (j + 1 < i) ? v[e + 1] * (-gs.eta[j + 1]) * f1 : 0.f;
-              pk[e >> 1] = pack_bf16(p0, p1);
-            }
-          }
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc)
-            st_shared_v4(prow + sw128_off(i, 4 * hf + cc), pk[4 * cc], pk[4 * cc + 1],
-                         pk[4 * cc + 2], pk[4 * cc + 3]);
-        }
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&sm.pready[b]);
-        mbar_arrive(&sm.gempty[g]);
-      }
-    }
-  } else if (warp < 16) {
-    // ------------------------------------------------------------ state warps
+  } else {
+    // ------------------------------------------------------------ math warpgroups
     const int q = warp & 3;          // TMEM lane quadrant
-    const int hh = (warp - 8) >> 2;  // warpgroup: state columns [64hh, 64hh+64)
+    const int hh = (warp - 4) >> 2;  // warpgroup: state and output columns [64hh, 64hh+64)
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
     const int n = 32 * q + lane;     // row of the d_out slice owned by this thread
-    const uint32_t srow = smem_u32(sm.S[hh]);
     float Sreg[64];  // fp32 state: row n, columns [64hh, 64hh+64)
     if (p.S_init) {
       const float4* si = reinterpret_cast<const float4*>(
@@ -509,64 +424,176 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
       for (int e = 0; e < 64; ++e) Sreg[e] = 0.f;
     }
-    const bool copy = yout || has_ck;  // the bf16 copy feeds S X^T and the checkpoints
-    // bf16 copy of the state (row n, this warpgroup's k-block) into the S tile
-    auto write_copy = [&]() {
+    const bool full = !p.summary;  // outputs, not just the state carry
+    const bool has_y = full && p.y != nullptr, has_ck = full && p.ckpt != nullptr;
+    // Each warp TMA-stores what it wrote itself: its 32 rows of one k-block of the
+    // bf16 state (the chunk-start checkpoints, bf16 [bh][chunk][dout][din], box of
+    // 32 rows) and its 16 token rows of one n-block of y (box of 16 rows). S_0 = 0
+    // is buffer 0.
+    const uint32_t s_part = (uint32_t)(32 * q) * 128;  // byte offset of the warp's state rows
+    const uint32_t y_part = (uint32_t)(16 * q) * 128;  // byte offset of the warp's token rows
+    if (has_ck && lane == 0) {  // the checkpoint of the segment's first chunk
+      tma_store_3d(&tmS, sm.S[0][hh] + s_part, 64 * hh, n0 + 32 * q, bh * nch_all + c0);
+      tma_store_commit();
+    }
+
+    // mask of chunk c: P_ij = K_ij (-eta_j) 2^{L_{i-1} - L_j} for j < i
+    auto mask = [&](int c) -> bool {
+      const int g = c % GS, b = c & 1;
+      const GateSlot& gs = sm.gates[g];
+      if (!mbar_wait_warp(&sm.gfull[g], (c / GS) & 1, wc, W_M_GFULL)) return false;
+      if (!mbar_wait_warp(&sm.kfull[b], (c >> 1) & 1, wc, W_M_KFULL)) return false;
+      tc_fence_after();
+      float v[32];
+      tmem_ld32(tbase + (b ? COL_K1 : COL_K0) + lane_off + 32 * hh, v);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.kfree[b]);
+      if (lane < 16) {
+        const int i = 16 * q + lane;
+        const float Lm1 = i == 0 ? 0.f : gs.L[i - 1];
+        uint32_t pk[16];
+        if (gs.fac) {
+          const float rai = gs.ra[i];
 #pragma unroll
-      for (int cc = 0; cc < 8; ++cc)
-        st_shared_v4(srow + sw128_off(n, cc), pack_bf16(Sreg[8 * cc], Sreg[8 * cc + 1]),
-                     pack_bf16(Sreg[8 * cc + 2], Sreg[8 * cc + 3]),
-                     pack_bf16(Sreg[8 * cc + 4], Sreg[8 * cc + 5]),
-                     pack_bf16(Sreg[8 * cc + 6], Sreg[8 * cc + 7]));
+          for (int e = 0; e < 32; e += 2) {
+            const int j = 32 * hh + e;
+            const float p0 = (j < i) ? v[e] * rai * gs.ca[j] : 0.f;
+            const float p1 = (j + 1 < i) ? v[e + 1] * rai * gs.ca[j + 1] : 0.f;
+            pk[e >> 1] = pack_bf16(p0, p1);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int j = 32 * hh + e;
+            const float f0 = exp2f(fminf(Lm1 - gs.L[j], 0.f));
+            const float f1 = exp2f(fminf(Lm1 - gs.L[j + 1], 0.f));
+            const float p0 = (j < i) ? v[e] * (-gs.eta[j]) * f0 : 0.f;
+            const float p1 = (j + 1 < i) ? v[e + 1] * (-gs.eta[j + 1]) * f1 : 0.f;
+            pk[e >> 1] = pack_bf16(p0, p1);
+          }
+        }
+        const uint32_t prow = smem_u32(sm.P);
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+          st_shared_v4(prow + sw128_off(i, 4 * hh + cc), pk[4 * cc], pk[4 * cc + 1],
+                       pk[4 * cc + 2], pk[4 * cc + 3]);
+      }
       fence_proxy_async_smem();
       __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.pready);
+      return true;
     };
-    // Each warp TMA-stores the 32 rows it wrote, one k-block wide, as its part of the
-    // chunk-start checkpoint (bf16 [bh][chunk][dout][din], box of 32 rows).
-    auto store_ck = [&](int gchunk) {
-      if (lane == 0) {
-        tma_store_3d(&tmS, sm.S[hh] + (uint32_t)(32 * q) * 128, 64 * hh, n0 + 32 * q,
-                     bh * nch_all + gchunk);
-        tma_store_commit();
-      }
-    };
-    if (copy) {  // S at the segment's first chunk
-      write_copy();
-      if (lane == 0) mbar_arrive(&sm.sready);
-      if (has_ck) store_ck(c0);
-    }
-    bool ok = true;
+
+    // Lane 0 of each math warp commits one TMA store group per checkpoint part and
+    // per y part, in the order CK_{c+1} (state update of chunk c), Y_c (epilogue of
+    // chunk c); before its rows of a buffer are rewritten it waits until the
+    // group that last read them is done reading.
+    bool ok = (nch > 0 && full) ? mask(0) : true;
     for (int c = 0; c < nch; ++c) {
       const int g = c % GS;
       const GateSlot& gs = sm.gates[g];
-      ok = ok && mbar_wait_warp(&sm.dsfull, c & 1, wc, W_S_DSFULL);
-      if (!ok) break;
-      tc_fence_after();
-      const float gC = gs.gC;
-#pragma unroll
-      for (int qq = 0; qq < 4; ++qq) {
-        float v[16];
-        tmem_ld16(tbase + COL_DS + lane_off + 64 * hh + 16 * qq, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 16; ++e) Sreg[16 * qq + e] = fmaf(gC, Sreg[16 * qq + e], v[e]);
-      }
-      tc_fence_before();
+
+      // ---- state: S <- 2^{L_{C-1}} S + dS ; bf16 copy into buffer wb = (c+1)&1, which
+      //      the S X^T product of chunk c - 1 read (one barrier pair per buffer, so a
+      //      parity wait can never see a phase from the other buffer's traffic)
+      const int wb = (c + 1) & 1;
+      ok = ok && mbar_wait_warp(&sm.dsfull, c & 1, wc, W_M_DSFULL);
+      ok = ok && (c == 0 || !full || mbar_wait_warp(&sm.sfree[wb], ((c - 1) >> 1) & 1, wc, W_M_SFREE));
+      // CK_{c-1} last read these rows of buffer wb; at most Y_{c-2}, CK_c, Y_{c-1}
+      // (or CK_1, Y_0 after CK_0) are newer
+      if (lane == 0 && has_ck) store_reads_pending_at_most(has_y ? 2 : 1);
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&sm.dsfree);
-        mbar_arrive(&sm.gempty[g]);
+      if (ok) {
+        tc_fence_after();
+        const float gC = gs.gC;
+        const uint32_t srow = smem_u32(sm.S[wb][hh]);
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          float v[32];
+          tmem_ld32(tbase + COL_DS + lane_off + 64 * hh + 32 * hf, v);
+          tmem_ld_wait();
+          if (hf == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.dsfree);
+          }
+#pragma unroll
+          for (int e = 0; e < 32; ++e) Sreg[32 * hf + e] = fmaf(gC, Sreg[32 * hf + e], v[e]);
+          if (!full) continue;
+#pragma unroll
+          for (int cc = 4 * hf; cc < 4 * hf + 4; ++cc)
+            st_shared_v4(srow + sw128_off(n, cc), pack_bf16(Sreg[8 * cc], Sreg[8 * cc + 1]),
+                         pack_bf16(Sreg[8 * cc + 2], Sreg[8 * cc + 3]),
+                         pack_bf16(Sreg[8 * cc + 4], Sreg[8 * cc + 5]),
+                         pack_bf16(Sreg[8 * cc + 6], Sreg[8 * cc + 7]));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && full) {
+          mbar_arrive(&sm.sready[wb]);
+          if (has_ck && c + 1 < nch) {
+            tma_store_3d(&tmS, sm.S[wb][hh] + s_part, 64 * hh, n0 + 32 * q,
+                         bh * nch_all + cg(c) + 1);
+            tma_store_commit();
+          }
+        }
       }
-      if (!copy || c + 1 == nch) continue;  // no copy after the last chunk
-      // the S X^T product of chunk c has read the old copy, and so has the last
-      // checkpoint store from it
-      if (yout) ok = ok && mbar_wait_warp(&sm.sfree, c & 1, wc, W_S_SFREE);
-      if (!ok) break;
-      if (has_ck && lane == 0) tma_store_wait_read();
+      if (!full) {  // state carry only
+        __syncwarp();
+        if (ok && lane == 0) mbar_arrive(&sm.gempty[g]);
+        continue;
+      }
+
+      // ---- mask of the next chunk (keeps the MMA stream fed while we store y)
+      if (c + 1 < nch) ok = ok && mask(c + 1);
+
+      // ---- output: y_i = Y1[i] + 2^{L_{i-1}} Y2[i]. Lane l < 16 holds Y1 and lane l + 16
+      //      holds Y2 of token row i = 16 q + l; for each 16 columns the pair swaps
+      //      halves, so lane l forms columns 0-7 and lane l + 16 columns 8-15.
+      const int yb = c & 1;
+      ok = ok && mbar_wait_warp(&sm.yfull[yb], (c >> 1) & 1, wc, W_M_YFULL);
+      // Y_{c-1} last read these staging rows; only CK_{c+1} is newer
+      if (lane == 0 && has_y) store_reads_pending_at_most((has_ck && c + 1 < nch) ? 1 : 0);
       __syncwarp();
-      write_copy();
-      if (lane == 0) mbar_arrive(&sm.sready);
-      if (has_ck) store_ck(cg(c) + 1);
+      if (ok) {
+        tc_fence_after();
+        const int i = 16 * q + (lane & 15);
+        const int hi = lane >> 4;
+        const float gi = gs.gam[i];
+        const uint32_t yrow = smem_u32(sm.Ys + hh * TILE);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          float v[16];
+          tmem_ld16(tbase + COL_Y + 128 * yb + lane_off + 64 * hh + 16 * k, v);
+          tmem_ld_wait();
+          if (k == 3) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.yfree[yb]);
+          }
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) {
+            // lo lane sends Y1 columns 8-15, hi lane sends Y2 columns 0-7
+            const float r0 = __shfl_xor_sync(0xffffffffu, hi ? v[e] : v[8 + e], 16);
+            const float r1 = __shfl_xor_sync(0xffffffffu, hi ? v[e + 1] : v[9 + e], 16);
+            const float y0 = hi ? fmaf(gi, v[8 + e], r0) : fmaf(gi, r0, v[e]);
+            const float y1 = hi ? fmaf(gi, v[9 + e], r1) : fmaf(gi, r1, v[e + 1]);
+            w[e >> 1] = pack_bf16(y0, y1);
+          }
+          if (has_y) st_shared_v4(yrow + sw128_off(i, 2 * k + hi), w[0], w[1], w[2], w[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        // rows past T are clipped; a part that starts past T is not issued
+        if (lane == 0 && has_y && cg(c) * C + 16 * q < T) {
+          tma_store_3d(&tmY, sm.Ys + hh * TILE + y_part, n0 + 64 * hh, cg(c) * C + 16 * q, bh);
+          tma_store_commit();
+        }
+        if (lane == 0) mbar_arrive(&sm.gempty[g]);
+      }
     }
     if (lane == 0) tma_store_wait_all();
     if (ok && p.S_final) {  // the state after the walked chunks, fp32
@@ -575,83 +602,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int e = 0; e < 16; ++e)
         so[e] = make_float4(Sreg[4 * e], Sreg[4 * e + 1], Sreg[4 * e + 2], Sreg[4 * e + 3]);
     }
-    if (ok && !p.summary && p.S_last && seg == p.nseg - 1) {  // S_T: padded tokens left it unchanged
+    if (ok && full && p.S_last && seg == p.nseg - 1) {  // S_T: padded tokens left it unchanged
       float4* so = reinterpret_cast<float4*>(p.S_last + ((size_t)bh * p.dout + n0 + n) * 128 + 64 * hh);
 #pragma unroll
       for (int e = 0; e < 16; ++e)
         so[e] = make_float4(Sreg[4 * e], Sreg[4 * e + 1], Sreg[4 * e + 2], Sreg[4 * e + 3]);
-    }
-  } else {
-    // ------------------------------------------------------------ output epilogue
-    // Thread (q, lane) owns output row n = 32q + lane of the slice: Y1^T and Y2^T hold
-    // y_i[n] for the chunk's 64 tokens i in its TMEM lane. y_i[n] is staged into
-    // row i of the chunk's X tile (free once the chunk's products are done): lanes
-    // n and n^1 exchange one value per token pair, so each writes a bf16 pair.
-    // Every epilogue warp runs every iteration and reaches the named barrier, also
-    // after a failed wait, so that none is left waiting at it.
-    const int q = warp & 3;
-    const uint32_t lane_off = (uint32_t)(32 * q) << 16;
-    const int n = 32 * q + lane;
-    const bool odd = lane & 1;
-    const int ne = n & ~1;                       // the pair's first column
-    const uint32_t nb = (uint32_t)(ne >> 6) * TILE;  // n-block of the staging tile
-    const uint32_t cb = (uint32_t)((ne & 63) * 2);   // byte offset inside the 128-byte row
-    const bool leader = warp == 16 && lane == 0;
-    bool ok = true;
-    int prev_s = -1;  // stage whose y store is still reading it
-    for (int c = 0; c < nch && yout; ++c) {
-      const int s = c % NS, g = c % GS, b = c & 1;
-      const GateSlot& gs = sm.gates[g];
-      if (leader && prev_s >= 0) {  // the last chunk's y store has read its stage
-        tma_store_wait_read();
-        mbar_arrive(&sm.empty[prev_s]);
-        prev_s = -1;
-      }
-      ok = ok && mbar_wait_warp(&sm.gfull[g], (c / GS) & 1, wc, W_E_GFULL);
-      ok = ok && mbar_wait_warp(&sm.yfull[b], (c >> 1) & 1, wc, W_E_YFULL);
-      if (ok) {
-        tc_fence_after();
-        const uint32_t tY = tbase + COL_Y + 128 * b + lane_off;
-        const uint32_t xs = smem_u32(sm.X[s]) + nb;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          float v1[16], v2[16];
-          tmem_ld16(tY + 16 * k, v1);
-          tmem_ld16(tY + 64 + 16 * k, v2);
-          tmem_ld_wait();
-          if (k == 3) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.yfree[b]);
-          }
-#pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            const int i0 = 16 * k + e;
-            const float ya = fmaf(gs.gam[i0], v2[e], v1[e]);          // y_{i0}[n]
-            const float yb = fmaf(gs.gam[i0 + 1], v2[e + 1], v1[e + 1]);  // y_{i0+1}[n]
-            // the even lane keeps token i0 and receives y_{i0}[n+1]; the odd lane keeps
-            // token i0 + 1 and receives y_{i0+1}[n-1]
-            const float r = __shfl_xor_sync(0xffffffffu, odd ? ya : yb, 1);
-            const int row = odd ? i0 + 1 : i0;
-            const uint32_t w = odd ? pack_bf16(r, yb) : pack_bf16(ya, r);
-            st_shared_b32(xs + row * 128 + ((((cb >> 4) ^ (row & 7)) << 4) | (cb & 15)), w);
-          }
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.gempty[g]);
-      }
-      named_bar_sync(BAR_EPI, 128);
-      if (leader && ok) {  // the stage goes back to the producer once this store has read it
-        tma_store_3d(&tmY, sm.X[s], n0, cg(c) * C, bh);
-        tma_store_3d(&tmY, sm.X[s] + TILE, n0 + 64, cg(c) * C, bh);
-        tma_store_commit();
-        prev_s = s;
-      }
-    }
-    if (leader) {
-      tma_store_wait_all();
-      if (prev_s >= 0) mbar_arrive(&sm.empty[prev_s]);
     }
   }
 
@@ -708,7 +663,7 @@ cudaError_t launch_fwd(const TcFwdParams& prm, const void* x, const void* g, cud
   // stands in as a well-formed base otherwise.
   if (!make_map_bf16_3d(&mx, x, prm.din, prm.T, BH, C) ||
       !make_map_bf16_3d(&mg, g, prm.dout, prm.T, BH, C) ||
-      !make_map_bf16_3d(&my, prm.y ? (const void*)prm.y : g, prm.dout, prm.T, BH, C) ||
+      !make_map_bf16_3d(&my, prm.y ? (const void*)prm.y : g, prm.dout, prm.T, BH, 16) ||
       !make_map_bf16_3d(&ms, prm.ckpt ? (const void*)prm.ckpt : g, 128, prm.dout,
                         prm.ckpt ? BH * nch : 1, 32))
     return cudaErrorInvalidValue;
