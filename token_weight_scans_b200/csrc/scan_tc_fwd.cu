@@ -17,17 +17,26 @@
 //   P_ij = K_ij (-eta_j) 2^{L_{i-1}-L_j}  (j < i), bf16 in shared memory
 //   Y1   = X W0^T + P G                   (M=64 tokens, N=128, K=d_in+C)     -> TMEM
 //   Y2   = X S^T                          (M=64 tokens, N=128, K=d_in)       -> TMEM
-//   dS   = G^T Xhat, Xhat_j = w_j x_j     (M=128, N=d_in, K=C)               -> TMEM
-//   y_i  = Y1[i, :] + 2^{L_{i-1}} Y2[i, :]; S <- 2^{L_{C-1}} S + dS (fp32, registers)
+//   S   += G^T Xhat, Xhat_j = w_j x_j     (M=128, N=d_in, K=C)               -> TMEM
+//   y_i  = Y1[i, :] + 2^{L_{i-1}} Y2[i, :]
+// The fp32 state lives in TMEM: the state warps scale it by 2^{L_{C-1}} in place
+// and the tensor core accumulates G^T Xhat onto it, so no thread carries it.
 //
-// Warp roles (12 warps): 0 TMA producer, 1 MMA issuer (+TMEM owner), 2 gate
-// prep (log2 alpha cumulative sums, prefetched) and half of the scaled-X tile,
-// 3 the other half of the scaled-X tile (double-buffered, so these two warps
-// run a chunk ahead), 4..11 two math warpgroups (state update, mask of the
-// next chunk, output epilogue): warpgroup h owns state columns [64h, 64h+64)
-// and output columns [64h, 64h+64) of the slice. The bf16 copy of the state is
-// double-buffered so the state update of chunk c overlaps the S X^T product of
-// chunk c.
+// Warp roles (20 warps): 0 TMA producer, 1 and 2 MMA issuers (1 owns TMEM),
+// 3 gate prep (log2 alpha cumulative sums, prefetched), 4..11 two state
+// warpgroups (bf16 copy of the chunk-start state for the S X^T product and the
+// checkpoint, then the in-place decay, then the scaled-X tile of the next chunk,
+// which is double-buffered), 12..19 two output warpgroups (the mask of the next
+// chunk, then the output epilogue). Warpgroup h of each pair owns state columns,
+// mask columns and output columns [64h, 64h+64) (mask: [32h, 32h+32)).
+//
+// A tcgen05.mma is issued by one thread, and that thread shares its scheduler
+// with the math warps of its TMEM lane quadrant; its issue rate drops several-
+// fold while they are busy. So the products are split between two issuers on
+// different schedulers: warp 1 issues K, the state update (right after K, so
+// that nothing queues ahead of it on the state chain), X W0^T and P G; warp 2
+// issues X S^T. Y is complete when both have committed, a stage is free when
+// both have read it.
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -50,7 +59,7 @@ namespace {
 constexpr int C = 64;          // tokens per chunk
 constexpr int NS = 2;          // TMA stages (X and G tiles)
 constexpr int GS = 4;          // gate slots
-constexpr int NTHREADS = 384;  // 12 warps
+constexpr int NTHREADS = 640;  // 20 warps
 constexpr int TILE = C * 128;  // bytes of one [64 rows x 128 B] swizzled block
 constexpr int BIG = 128 * 128; // bytes of one [128 rows x 128 B] swizzled block
 
@@ -61,7 +70,7 @@ constexpr int BIG = 128 * 128; // bytes of one [128 rows x 128 B] swizzled block
 // (l, l + 16) both halves of the same token row; the pair is double-buffered.
 constexpr uint32_t COL_K0 = 0, COL_K1 = 64;      // K = X X^T, double buffer (lanes 0-15)
 constexpr uint32_t COL_Y = 128;                  // + 128 * buffer: Y1 | Y2 (128 columns)
-constexpr uint32_t COL_DS = 384;                 // dS (128 columns, all 128 lanes)
+constexpr uint32_t COL_S = 384;                  // fp32 state (128 columns, all 128 lanes)
 constexpr uint32_t LANE16 = 16u << 16;
 
 // With M = L_{31}, the mask factor -eta_j 2^{L_{i-1} - L_j} = ra_i ca_j whenever
@@ -83,7 +92,7 @@ struct Smem {
   uint8_t X[NS][2 * TILE];     // k-blocks [0,64), [64,128): 64 token rows x 128 B
   uint8_t G[NS][2 * TILE];     // n-blocks of the slice: 64 token rows x 128 B
   uint8_t W0[2][BIG];          // k-blocks: 128 n rows x 128 B (bf16 W0 slice)
-  uint8_t S[2][2][BIG];        // [buffer][k-block]: 128 n rows x 128 B (bf16 state)
+  uint8_t S[2][2][BIG];        // [buffer][k-block]: 128 n rows x 128 B (bf16 chunk-start state)
   uint8_t Xh[2][2 * TILE];     // [buffer] scaled X, same layout as X
   uint8_t P[TILE];             // 64 token rows (i) x 128 B (j)
   uint8_t Ys[2 * TILE];        // y staging: n-blocks of 64 token rows x 128 B (TMA store)
@@ -93,8 +102,8 @@ struct Smem {
   uint64_t kfull[2], kfree[2];
   uint64_t xhready[2], xhfree[2];  // per scaled-X buffer
   uint64_t sready[2], sfree[2];    // per bf16 state buffer
-  uint64_t yfull[2], yfree[2];    // per Y1 | Y2 buffer
-  uint64_t pready, dsfull, dsfree, done;
+  uint64_t yfull[2], yfree[2];     // per Y1 | Y2 buffer
+  uint64_t pready, dsfull, sscaled, done[2];
   uint32_t tmem_base;
   int abort;
 };
@@ -105,19 +114,13 @@ static_assert(kSmemBytes <= 227 * 1024, "over the 227 KB of shared memory a CTA 
 // where-codes of the bounded waits (role << 8 | site)
 enum : uint32_t {
   W_TMA_EMPTY = 0x001, W_TMA_DRAIN = 0x002,
-  W_MMA_FULL = 0x101, W_MMA_KFREE, W_MMA_YFREE, W_MMA_XREADY, W_MMA_DSFREE, W_MMA_PREADY,
+  W_MMA_FULL = 0x101, W_MMA_KFREE, W_MMA_YFREE, W_MMA_XREADY, W_MMA_SSCALED, W_MMA_PREADY,
   W_MMA_SREADY, W_MMA_DONE,
   W_GATE_EMPTY = 0x201,
   W_XH_FULL = 0x301, W_XH_GFULL, W_XH_FREE,
-  W_M_GFULL = 0x401, W_M_KFULL, W_M_DSFULL, W_M_SFREE, W_M_YFULL,
+  W_M_GFULL = 0x401, W_M_KFULL, W_M_YFULL,
+  W_S_GFULL = 0x501, W_S_DSFULL, W_S_SFREE,
 };
-
-// Waits until at most n (0..2) of this thread's TMA store groups still read shared memory.
-__device__ __forceinline__ void store_reads_pending_at_most(int n) {
-  if (n <= 0) tma_store_wait_read_n<0>();
-  else if (n == 1) tma_store_wait_read_n<1>();
-  else tma_store_wait_read_n<2>();
-}
 
 }  // namespace
 
@@ -143,33 +146,34 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   auto cg = [&](int c) { return p.reverse ? c1 - 1 - c : c0 + c; };
   const size_t seg_row = (size_t)bh * p.nseg + seg;  // [bh][seg] index of the segment states
   const WaitCtx wc{&sm.abort, p.status, p.timeout_ns};
+  const bool full = !p.summary;  // outputs, not just the state carry
 
   if (threadIdx.x == 0) {
     sm.abort = 0;
     for (int s = 0; s < NS; ++s) {
       mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], 1);
+      mbar_init(&sm.empty[s], full ? 2 : 1);  // the issuers that read the stage
     }
     for (int g = 0; g < GS; ++g) {
       mbar_init(&sm.gfull[g], 32);
-      mbar_init(&sm.gempty[g], 10);  // 2 scaled-X warps + 8 math warps
+      // 8 state warps (+ 8 output warps when there are outputs)
+      mbar_init(&sm.gempty[g], full ? 16 : 8);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.kfull[b], 1);
       mbar_init(&sm.kfree[b], 8);
-      mbar_init(&sm.xhready[b], 2);
+      mbar_init(&sm.xhready[b], 8);  // the state warps
       mbar_init(&sm.xhfree[b], 1);
       mbar_init(&sm.sready[b], 8);
       mbar_init(&sm.sfree[b], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&sm.yfull[b], 1);
+      mbar_init(&sm.yfull[b], 2);  // both issuers write Y
       mbar_init(&sm.yfree[b], 8);
     }
     mbar_init(&sm.pready, 8);
     mbar_init(&sm.dsfull, 1);
-    mbar_init(&sm.dsfree, 8);
-    mbar_init(&sm.done, 1);
+    mbar_init(&sm.sscaled, 8);
+    mbar_init(&sm.done[0], 1);
+    mbar_init(&sm.done[1], 1);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -182,26 +186,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tmem_alloc(&sm.tmem_base, 512);
     tmem_relinquish();
   }
-  // W0 slice -> bf16 swizzled K-major tiles; S_0 = 0
-  if (warp >= 4) {
-    const int t = threadIdx.x - 128;  // 0..255
+  // W0 slice -> bf16 swizzled K-major tiles
+  if (warp >= 4 && full) {
+    const int t = threadIdx.x - 128;
     const float* W0 = p.W0 + ((size_t)h * p.dout + n0) * 128;
-    for (int idx = t; idx < 128 * 16; idx += 256) {  // (row n, 16-byte chunk of 8 k)
+    for (int idx = t; idx < 128 * 16; idx += NTHREADS - 128) {  // (row n, 16-byte chunk of 8 k)
       const int n = idx >> 4, ck = idx & 15;
       const int kb = ck >> 3, c = ck & 7;
       const float4 a = *reinterpret_cast<const float4*>(W0 + (size_t)n * 128 + ck * 8);
       const float4 b = *reinterpret_cast<const float4*>(W0 + (size_t)n * 128 + ck * 8 + 4);
       st_shared_v4(smem_u32(sm.W0[kb]) + sw128_off(n, c), pack_bf16(a.x, a.y),
                    pack_bf16(a.z, a.w), pack_bf16(b.x, b.y), pack_bf16(b.z, b.w));
-      if (p.S_init) {  // the segment's start state (rows of this slice), fp32 -> bf16
-        const float* si = p.S_init + (seg_row * p.dout + n0 + n) * 128 + ck * 8;
-        const float4 u = *reinterpret_cast<const float4*>(si);
-        const float4 v = *reinterpret_cast<const float4*>(si + 4);
-        st_shared_v4(smem_u32(sm.S[0][kb]) + sw128_off(n, c), pack_bf16(u.x, u.y),
-                     pack_bf16(u.z, u.w), pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
-      } else {
-        st_shared_v4(smem_u32(sm.S[0][kb]) + sw128_off(n, c), 0u, 0u, 0u, 0u);
-      }
     }
     fence_proxy_async_smem();
   }
@@ -229,9 +224,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int c = issued > NS ? issued - NS : 0; c < issued; ++c)
         mbar_drain(&sm.full[c % NS], (c / NS) & 1, wc, W_TMA_DRAIN);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------ MMA issuers
+    const int ii = warp - 1;  // 0: K, the state update, X W0^T, P G; 1: X S^T
+    // (the state carry alone has no work for issuer 1)
+    if (lane == 0 && (ii == 0 || full)) {
       const uint32_t id_k = idesc_bf16(64, 64, false, false);    // X X^T
       const uint32_t id_y = idesc_bf16(64, 128, false, false);   // X W0^T, X S^T
       const uint32_t id_pg = idesc_bf16(64, 128, false, true);   // P G (G n-contiguous)
@@ -241,78 +238,83 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int s = c % NS, b = c & 1;
         const uint32_t sX = smem_u32(sm.X[s]), sG = smem_u32(sm.G[s]);
         const uint32_t sXh = smem_u32(sm.Xh[b]), sS = smem_u32(sm.S[b][0]);
+        const uint32_t tY1 = tbase + COL_Y + 128 * b, tY2 = tY1 + LANE16;
         if (!mbar_wait(&sm.full[s], (c / NS) & 1, wc, W_MMA_FULL)) break;
-        if (!p.summary) {
-          if (!mbar_wait(&sm.kfree[b], ((c >> 1) & 1) ^ 1, wc, W_MMA_KFREE)) break;
+        if (ii == 0) {
+          if (full) {
+            // K = X X^T into buffer b (the mask of chunk c - 2 has read it)
+            if (!mbar_wait(&sm.kfree[b], ((c >> 1) & 1) ^ 1, wc, W_MMA_KFREE)) break;
+            tc_fence_after();
+            #pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t off = (kk >> 2) * TILE + (kk & 3) * 32;
+              umma_bf16(tbase + (b ? COL_K1 : COL_K0), desc_at(sw128_desc(sX, 16, 1024), off),
+                        desc_at(sw128_desc(sX, 16, 1024), off), id_k, kk > 0);
+            }
+            if (!(p.inject == 1 && c == 1)) umma_commit(&sm.kfull[b]);
+          }
+          // S += G^T Xhat onto the state that the state warps have scaled in place
+          if (!mbar_wait(&sm.xhready[b], (c >> 1) & 1, wc, W_MMA_XREADY)) break;
+          if (!mbar_wait(&sm.sscaled, c & 1, wc, W_MMA_SSCALED)) break;
           tc_fence_after();
-          // K = X X^T
+          #pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tbase + COL_S, desc_at(sw128_desc(sG, TILE, 1024), kk * 2048),
+                      desc_at(sw128_desc(sXh, TILE, 1024), kk * 2048), id_ds, 1);
+          if (!(p.inject == 3 && c == 1)) umma_commit(&sm.dsfull);
+          umma_commit(&sm.xhfree[b]);
+          if (!full) {  // state carry only: the stage is free once the update has read it
+            umma_commit(&sm.empty[s]);
+            continue;
+          }
+          // Y1 = X W0^T into buffer b (the epilogue of chunk c - 2 has read it)
+          if (!mbar_wait(&sm.yfree[b], ((c >> 1) & 1) ^ 1, wc, W_MMA_YFREE)) break;
+          tc_fence_after();
           #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * TILE + (kk & 3) * 32;
-            umma_bf16(tbase + (b ? COL_K1 : COL_K0), desc_at(sw128_desc(sX, 16, 1024), off),
-                      desc_at(sw128_desc(sX, 16, 1024), off), id_k, kk > 0);
+            const uint32_t aoff = (kk >> 2) * TILE + (kk & 3) * 32;
+            const uint32_t boff = (kk >> 2) * BIG + (kk & 3) * 32;
+            umma_bf16(tY1, desc_at(sw128_desc(sX, 16, 1024), aoff),
+                      desc_at(sw128_desc(sW0, 16, 1024), boff), id_y, kk > 0);
           }
-          if (!(p.inject == 1 && c == 1)) umma_commit(&sm.kfull[b]);
-        }
-        // dS = G^T Xhat
-        if (!mbar_wait(&sm.xhready[b], (c >> 1) & 1, wc, W_MMA_XREADY)) break;
-        if (c > 0 && !mbar_wait(&sm.dsfree, (c - 1) & 1, wc, W_MMA_DSFREE)) break;
-        tc_fence_after();
-        #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_bf16(tbase + COL_DS, desc_at(sw128_desc(sG, TILE, 1024), kk * 2048),
-                    desc_at(sw128_desc(sXh, TILE, 1024), kk * 2048), id_ds, kk > 0);
-        if (!(p.inject == 3 && c == 1)) umma_commit(&sm.dsfull);
-        umma_commit(&sm.xhfree[b]);
-        if (p.summary) {  // state carry only: the stage is free once dS has read it
+          // Y1 += P G. The mask of chunk c + 1 overwrites P only after the K product
+          // of chunk c + 1 has completed, which this thread commits after these.
+          if (!mbar_wait(&sm.pready, c & 1, wc, W_MMA_PREADY)) break;
+          tc_fence_after();
+          #pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tY1, desc_at(sw128_desc(sP, 16, 1024), kk * 32),
+                      desc_at(sw128_desc(sG, TILE, 1024), kk * 2048), id_pg, 1);
+          umma_commit(&sm.yfull[b]);
           umma_commit(&sm.empty[s]);
-          continue;
+        } else {
+          // Y2 = X S^T (bf16 chunk-start state in buffer b) into buffer b
+          if (!mbar_wait(&sm.sready[b], (c >> 1) & 1, wc, W_MMA_SREADY)) break;
+          if (!mbar_wait(&sm.yfree[b], ((c >> 1) & 1) ^ 1, wc, W_MMA_YFREE)) break;
+          tc_fence_after();
+          #pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t aoff = (kk >> 2) * TILE + (kk & 3) * 32;
+            const uint32_t boff = (kk >> 2) * BIG + (kk & 3) * 32;
+            umma_bf16(tY2, desc_at(sw128_desc(sX, 16, 1024), aoff),
+                      desc_at(sw128_desc(sS, 16, 1024), boff), id_y, kk > 0);
+          }
+          umma_commit(&sm.sfree[b]);
+          umma_commit(&sm.yfull[b]);
+          umma_commit(&sm.empty[s]);
         }
-        // Y1 = X W0^T into buffer b (the epilogue of chunk c - 2 has read it)
-        const uint32_t tY1 = tbase + COL_Y + 128 * b, tY2 = tY1 + LANE16;
-        if (!mbar_wait(&sm.yfree[b], ((c >> 1) & 1) ^ 1, wc, W_MMA_YFREE)) break;
-        tc_fence_after();
-        #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t aoff = (kk >> 2) * TILE + (kk & 3) * 32;
-          const uint32_t boff = (kk >> 2) * BIG + (kk & 3) * 32;
-          umma_bf16(tY1, desc_at(sw128_desc(sX, 16, 1024), aoff), desc_at(sw128_desc(sW0, 16, 1024), boff), id_y,
-                    kk > 0);
-        }
-        // Y2 = X S^T (state buffer c & 1, written by the state update of chunk c - 1)
-        if (c > 0 && !mbar_wait(&sm.sready[b], ((c - 1) >> 1) & 1, wc, W_MMA_SREADY)) break;
-        tc_fence_after();
-        #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t aoff = (kk >> 2) * TILE + (kk & 3) * 32;
-          const uint32_t boff = (kk >> 2) * BIG + (kk & 3) * 32;
-          umma_bf16(tY2, desc_at(sw128_desc(sX, 16, 1024), aoff), desc_at(sw128_desc(sS, 16, 1024), boff), id_y,
-                    kk > 0);
-        }
-        umma_commit(&sm.sfree[b]);
-        // Y1 += P G. The mask of chunk c + 1 overwrites P only after the K product
-        // of chunk c + 1 has completed, which is committed after these.
-        if (!mbar_wait(&sm.pready, c & 1, wc, W_MMA_PREADY)) break;
-        tc_fence_after();
-        #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_bf16(tY1, desc_at(sw128_desc(sP, 16, 1024), kk * 32),
-                    desc_at(sw128_desc(sG, TILE, 1024), kk * 2048), id_pg, 1);
-        umma_commit(&sm.yfull[b]);
-        umma_commit(&sm.empty[s]);
       }
-      // teardown: every issued MMA completes before TMEM is released
-      umma_commit(&sm.done);
-      mbar_drain(&sm.done, 0, wc, W_MMA_DONE);
+      // teardown: every MMA this thread issued completes before TMEM is released
+      umma_commit(&sm.done[ii]);
+      mbar_drain(&sm.done[ii], 0, wc, W_MMA_DONE);
     }
-  } else if (warp == 2 || warp == 3) {
-    // ------------------------------------------------------------ gates + scaled X
-    // Warp 2 also prepares the gates of each chunk (alpha / eta prefetched PD chunks
-    // ahead so the global-load latency is off the chain); both warps then write
-    // half of Xhat = w (.) X with packed bf16 multiplies.
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ gates
+    // The gates of each chunk (alpha / eta prefetched PD chunks ahead so the
+    // global-load latency is off the chain).
     constexpr int PD = 4;
     const size_t gbase = (size_t)bh * T;
-    const bool gate_warp = warp == 2;
+    constexpr bool gate_warp = true;
     float ra[PD][2], re[PD][2];
     float Lseg = 0.f;  // sum of log2 alpha over the walked chunks (lane-uniform)
     // gates of the c-th walked chunk (alpha = 1, eta = 0 past the walk or past T)
@@ -334,7 +336,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int k = 0; k < PD; ++k) {
         const int c = cb + k;
         if (c >= nch) break;
-        const int s = c % NS, g = c % GS;
+        const int g = c % GS;
         GateSlot& gs = sm.gates[g];
         if (gate_warp) {
           if (!mbar_wait_warp(&sm.gempty[g], ((c / GS) & 1) ^ 1, wc, W_GATE_EMPTY)) { ok = false; break; }
@@ -375,67 +377,155 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           __syncwarp();
           mbar_arrive(&sm.gfull[g]);
         }
-        if (!mbar_wait_warp(&sm.full[s], (c / NS) & 1, wc, W_XH_FULL)) { ok = false; break; }
-        if (!mbar_wait_warp(&sm.gfull[g], (c / GS) & 1, wc, W_XH_GFULL)) { ok = false; break; }
-        if (!mbar_wait_warp(&sm.xhfree[c & 1], ((c >> 1) & 1) ^ 1, wc, W_XH_FREE)) { ok = false; break; }
-        const uint32_t src = smem_u32(sm.X[s]), dst = smem_u32(sm.Xh[c & 1]);
-#pragma unroll 4
-        for (int idx = (warp - 2) * 32 + lane; idx < 2 * TILE / 16; idx += 64) {
-          const uint32_t off = idx * 16;
-          const int j = (off & (TILE - 1)) >> 7;  // token row
-          // forward: -eta_j 2^{L_{C-1}-L_j}; reverse (adjoint) summary: 2^{L_{j-1}}
-          const __nv_bfloat162 w2 = __float2bfloat162_rn(p.reverse ? gs.gam[j] : gs.w[j]);
-          const uint32_t wv = *reinterpret_cast<const uint32_t*>(&w2);
-          uint4 v = ld_shared_v4(src + off);
-          v.x = hmul2_bf16(v.x, wv);
-          v.y = hmul2_bf16(v.y, wv);
-          v.z = hmul2_bf16(v.z, wv);
-          v.w = hmul2_bf16(v.w, wv);
-          st_shared_v4(dst + off, v.x, v.y, v.z, v.w);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&sm.xhready[c & 1]);
-          mbar_arrive(&sm.gempty[g]);
-        }
       }
     }
     if (ok && gate_warp && lane == 0 && p.seg_L && slice == 0) p.seg_L[seg_row] = Lseg;
-  } else {
-    // ------------------------------------------------------------ math warpgroups
+  } else if (warp < 12) {
+    // ------------------------------------------------------------ state warpgroups
     const int q = warp & 3;          // TMEM lane quadrant
-    const int hh = (warp - 4) >> 2;  // warpgroup: state and output columns [64hh, 64hh+64)
+    const int hh = (warp - 4) >> 2;  // warpgroup: state columns [64hh, 64hh+64)
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
     const int n = 32 * q + lane;     // row of the d_out slice owned by this thread
-    float Sreg[64];  // fp32 state: row n, columns [64hh, 64hh+64)
-    if (p.S_init) {
-      const float4* si = reinterpret_cast<const float4*>(
-          p.S_init + (seg_row * p.dout + n0 + n) * 128 + 64 * hh);
+    const uint32_t tS = tbase + COL_S + lane_off + 64 * hh;
+    const bool has_ck = full && p.ckpt != nullptr;
+    // S_0 (the segment's start state, or zero) into TMEM
+    {
+      float v[32];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const float4 v = si[e];
-        Sreg[4 * e] = v.x;
-        Sreg[4 * e + 1] = v.y;
-        Sreg[4 * e + 2] = v.z;
-        Sreg[4 * e + 3] = v.w;
+      for (int hf = 0; hf < 2; ++hf) {
+        if (p.S_init) {
+          const float4* si = reinterpret_cast<const float4*>(
+              p.S_init + (seg_row * p.dout + n0 + n) * 128 + 64 * hh + 32 * hf);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float4 u = si[e];
+            v[4 * e] = u.x;
+            v[4 * e + 1] = u.y;
+            v[4 * e + 2] = u.z;
+            v[4 * e + 3] = u.w;
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = 0.f;
+        }
+        tmem_st32(tS + 32 * hf, v);
       }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 64; ++e) Sreg[e] = 0.f;
+      tmem_st_wait();
     }
-    const bool full = !p.summary;  // outputs, not just the state carry
-    const bool has_y = full && p.y != nullptr, has_ck = full && p.ckpt != nullptr;
     // Each warp TMA-stores what it wrote itself: its 32 rows of one k-block of the
-    // bf16 state (the chunk-start checkpoints, bf16 [bh][chunk][dout][din], box of
-    // 32 rows) and its 16 token rows of one n-block of y (box of 16 rows). S_0 = 0
-    // is buffer 0.
+    // bf16 chunk-start state (bf16 [bh][chunk][dout][din], box of 32 rows).
     const uint32_t s_part = (uint32_t)(32 * q) * 128;  // byte offset of the warp's state rows
-    const uint32_t y_part = (uint32_t)(16 * q) * 128;  // byte offset of the warp's token rows
-    if (has_ck && lane == 0) {  // the checkpoint of the segment's first chunk
-      tma_store_3d(&tmS, sm.S[0][hh] + s_part, 64 * hh, n0 + 32 * q, bh * nch_all + c0);
-      tma_store_commit();
+    // Xhat of the c-th walked chunk, w_j x_j (forward) or 2^{L_{j-1}} x_j (adjoint
+    // summary), with packed bf16 multiplies; each state thread writes 4 of its 1024
+    // 16-byte pieces. Written a chunk ahead, into the buffer the update of chunk c - 2 read.
+    const int st = threadIdx.x - 128;  // 0..255 over the state warps
+    auto scaled_x = [&](int c) -> bool {
+      const int s = c % NS, g = c % GS, b = c & 1;
+      if (!mbar_wait_warp(&sm.full[s], (c / NS) & 1, wc, W_XH_FULL)) return false;
+      if (!mbar_wait_warp(&sm.gfull[g], (c / GS) & 1, wc, W_XH_GFULL)) return false;
+      if (!mbar_wait_warp(&sm.xhfree[b], ((c >> 1) & 1) ^ 1, wc, W_XH_FREE)) return false;
+      const GateSlot& gs = sm.gates[g];
+      const uint32_t src = smem_u32(sm.X[s]), dst = smem_u32(sm.Xh[b]);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t off = (uint32_t)(st + 256 * k) * 16;
+        const int j = (off & (TILE - 1)) >> 7;  // token row
+        const __nv_bfloat162 w2 = __float2bfloat162_rn(p.reverse ? gs.gam[j] : gs.w[j]);
+        const uint32_t wv = *reinterpret_cast<const uint32_t*>(&w2);
+        uint4 v = ld_shared_v4(src + off);
+        st_shared_v4(dst + off, hmul2_bf16(v.x, wv), hmul2_bf16(v.y, wv), hmul2_bf16(v.z, wv),
+                     hmul2_bf16(v.w, wv));
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.xhready[b]);
+      return true;
+    };
+    bool ok = nch > 0 ? scaled_x(0) : true;
+    for (int c = 0; c < nch && ok; ++c) {
+      const int g = c % GS, b = c & 1;
+      const GateSlot& gs = sm.gates[g];
+      ok = ok && mbar_wait_warp(&sm.gfull[g], (c / GS) & 1, wc, W_S_GFULL);
+      // S_c is complete: the update of chunk c - 1 has accumulated onto it
+      ok = ok && (c == 0 || mbar_wait_warp(&sm.dsfull, (c - 1) & 1, wc, W_S_DSFULL));
+      // buffer b was last read by the S X^T product and the checkpoint store of chunk c - 2
+      ok = ok && (!full || c < 2 || mbar_wait_warp(&sm.sfree[b], ((c - 2) >> 1) & 1, wc, W_S_SFREE));
+      if (lane == 0 && has_ck) tma_store_wait_read_n<1>();
+      __syncwarp();
+      if (!ok) break;
+      tc_fence_after();
+      // S_c -> bf16 (kept packed), S <- 2^{L_{C-1}} S in place; the update of chunk c
+      // may then accumulate, and the bf16 copy goes to buffer b (outputs only)
+      const float gC = gs.gC;
+      uint32_t pk[32];
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        float v[32];
+        tmem_ld32(tS + 32 * hf, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) pk[16 * hf + e] = pack_bf16(v[2 * e], v[2 * e + 1]);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] *= gC;
+        tmem_st32(tS + 32 * hf, v);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.sscaled);  // the update of chunk c may accumulate
+      if (full) {
+        const uint32_t srow = smem_u32(sm.S[b][hh]);
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc)
+          st_shared_v4(srow + sw128_off(n, cc), pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+        fence_proxy_async_smem();
+      }
+      __syncwarp();
+      if (lane == 0) {
+        if (full) {
+          mbar_arrive(&sm.sready[b]);  // the S X^T product of chunk c may read buffer b
+          if (has_ck) {  // the checkpoint of chunk c: the state at its first token
+            tma_store_3d(&tmS, sm.S[b][hh] + s_part, 64 * hh, n0 + 32 * q, bh * nch_all + cg(c));
+            tma_store_commit();
+          }
+        }
+      }
+      // the scaled X of the next chunk, while the update of this one runs
+      if (c + 1 < nch && !scaled_x(c + 1)) ok = false;
+      if (lane == 0) mbar_arrive(&sm.gempty[g]);
     }
+    if (lane == 0) tma_store_wait_all();
+    // the state after the walked chunks, fp32
+    const bool last = full && p.S_last && seg == p.nseg - 1;  // S_T: padded tokens left it unchanged
+    if (ok && (p.S_final || last) &&
+        (nch == 0 || mbar_wait_warp(&sm.dsfull, (nch - 1) & 1, wc, W_S_DSFULL))) {
+      tc_fence_after();
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        float v[32];
+        tmem_ld32(tS + 32 * hf, v);
+        tmem_ld_wait();
+        const size_t col = (size_t)64 * hh + 32 * hf;
+        if (p.S_final) {
+          float4* so = reinterpret_cast<float4*>(p.S_final + (seg_row * p.dout + n0 + n) * 128 + col);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) so[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+        }
+        if (last) {
+          float4* so = reinterpret_cast<float4*>(p.S_last + ((size_t)bh * p.dout + n0 + n) * 128 + col);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) so[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+        }
+      }
+    }
+  } else if (full) {
+    // ------------------------------------------------------------ output warpgroups
+    const int q = warp & 3;           // TMEM lane quadrant
+    const int hh = (warp - 12) >> 2;  // warpgroup: mask columns [32hh, +32), outputs [64hh, +64)
+    const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+    const bool has_y = p.y != nullptr;
+    // Each warp TMA-stores its 16 token rows of one n-block of y (box of 16 rows).
+    const uint32_t y_part = (uint32_t)(16 * q) * 128;  // byte offset of the warp's token rows
 
     // mask of chunk c: P_ij = K_ij (-eta_j) 2^{L_{i-1} - L_j} for j < i
     auto mask = [&](int c) -> bool {
@@ -486,67 +576,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       return true;
     };
 
-    // Lane 0 of each math warp commits one TMA store group per checkpoint part and
-    // per y part, in the order CK_{c+1} (state update of chunk c), Y_c (epilogue of
-    // chunk c); before its rows of a buffer are rewritten it waits until the
-    // group that last read them is done reading.
-    bool ok = (nch > 0 && full) ? mask(0) : true;
+    bool ok = nch > 0 ? mask(0) : true;
     for (int c = 0; c < nch; ++c) {
       const int g = c % GS;
       const GateSlot& gs = sm.gates[g];
-
-      // ---- state: S <- 2^{L_{C-1}} S + dS ; bf16 copy into buffer wb = (c+1)&1, which
-      //      the S X^T product of chunk c - 1 read (one barrier pair per buffer, so a
-      //      parity wait can never see a phase from the other buffer's traffic)
-      const int wb = (c + 1) & 1;
-      ok = ok && mbar_wait_warp(&sm.dsfull, c & 1, wc, W_M_DSFULL);
-      ok = ok && (c == 0 || !full || mbar_wait_warp(&sm.sfree[wb], ((c - 1) >> 1) & 1, wc, W_M_SFREE));
-      // CK_{c-1} last read these rows of buffer wb; at most Y_{c-2}, CK_c, Y_{c-1}
-      // (or CK_1, Y_0 after CK_0) are newer
-      if (lane == 0 && has_ck) store_reads_pending_at_most(has_y ? 2 : 1);
-      __syncwarp();
-      if (ok) {
-        tc_fence_after();
-        const float gC = gs.gC;
-        const uint32_t srow = smem_u32(sm.S[wb][hh]);
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          float v[32];
-          tmem_ld32(tbase + COL_DS + lane_off + 64 * hh + 32 * hf, v);
-          tmem_ld_wait();
-          if (hf == 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.dsfree);
-          }
-#pragma unroll
-          for (int e = 0; e < 32; ++e) Sreg[32 * hf + e] = fmaf(gC, Sreg[32 * hf + e], v[e]);
-          if (!full) continue;
-#pragma unroll
-          for (int cc = 4 * hf; cc < 4 * hf + 4; ++cc)
-            st_shared_v4(srow + sw128_off(n, cc), pack_bf16(Sreg[8 * cc], Sreg[8 * cc + 1]),
-                         pack_bf16(Sreg[8 * cc + 2], Sreg[8 * cc + 3]),
-                         pack_bf16(Sreg[8 * cc + 4], Sreg[8 * cc + 5]),
-                         pack_bf16(Sreg[8 * cc + 6], Sreg[8 * cc + 7]));
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0 && full) {
-          mbar_arrive(&sm.sready[wb]);
-          if (has_ck && c + 1 < nch) {
-            tma_store_3d(&tmS, sm.S[wb][hh] + s_part, 64 * hh, n0 + 32 * q,
-                         bh * nch_all + cg(c) + 1);
-            tma_store_commit();
-          }
-        }
-      }
-      if (!full) {  // state carry only
-        __syncwarp();
-        if (ok && lane == 0) mbar_arrive(&sm.gempty[g]);
-        continue;
-      }
-
-      // ---- mask of the next chunk (keeps the MMA stream fed while we store y)
+      // the mask of the next chunk first: it keeps the P G product of the MMA stream fed
       if (c + 1 < nch) ok = ok && mask(c + 1);
 
       // ---- output: y_i = Y1[i] + 2^{L_{i-1}} Y2[i]. Lane l < 16 holds Y1 and lane l + 16
@@ -554,8 +588,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       //      halves, so lane l forms columns 0-7 and lane l + 16 columns 8-15.
       const int yb = c & 1;
       ok = ok && mbar_wait_warp(&sm.yfull[yb], (c >> 1) & 1, wc, W_M_YFULL);
-      // Y_{c-1} last read these staging rows; only CK_{c+1} is newer
-      if (lane == 0 && has_y) store_reads_pending_at_most((has_ck && c + 1 < nch) ? 1 : 0);
+      // Y_{c-1} last read these staging rows
+      if (lane == 0 && has_y) tma_store_wait_read_n<0>();
       __syncwarp();
       if (ok) {
         tc_fence_after();
@@ -596,18 +630,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
     }
     if (lane == 0) tma_store_wait_all();
-    if (ok && p.S_final) {  // the state after the walked chunks, fp32
-      float4* so = reinterpret_cast<float4*>(p.S_final + (seg_row * p.dout + n0 + n) * 128 + 64 * hh);
-#pragma unroll
-      for (int e = 0; e < 16; ++e)
-        so[e] = make_float4(Sreg[4 * e], Sreg[4 * e + 1], Sreg[4 * e + 2], Sreg[4 * e + 3]);
-    }
-    if (ok && full && p.S_last && seg == p.nseg - 1) {  // S_T: padded tokens left it unchanged
-      float4* so = reinterpret_cast<float4*>(p.S_last + ((size_t)bh * p.dout + n0 + n) * 128 + 64 * hh);
-#pragma unroll
-      for (int e = 0; e < 16; ++e)
-        so[e] = make_float4(Sreg[4 * e], Sreg[4 * e + 1], Sreg[4 * e + 2], Sreg[4 * e + 3]);
-    }
   }
 
   tc_fence_before();
