@@ -33,14 +33,21 @@
 // where Ar, Z, Q^T, Bm are built by the math warps from K, Kug, KugT into the
 // shared memory that held S_in, Gs = diag(-eta del) G is written in place once
 // the unscaled G has been used, and Xg = diag(gam) X is a tile of its own that
-// warp 3 writes as soon as X arrives. The fp32 adjoint Lam
+// the math warps write as soon as X arrives. The fp32 adjoint Lam
 // lives in TMEM: the math warps scale it by 2^{L_{C-1}} in place and the MMA
 // accumulates U^T Xg onto it; likewise the rows del_i R1_i and gam_i DXb_i are
 // written back so that the remaining terms accumulate onto them (r and dx).
 //
-// Warp roles (20 warps): 0 TMA producer, 1 MMA issuer + TMEM owner, 2 gate
-// prep, 3 writes Xg = diag(gam) X, 4..19 four math warpgroups (warpgroup w: tokens
-// [16w, 16w+16) of each chunk and state columns [32w, 32w+32)).
+// Warp roles (20 warps): 0 TMA producer and gate prep, 1..3 three MMA issuers
+// (1 owns TMEM), 4..19 four math warpgroups (warpgroup w: tokens [16w, 16w+16) of
+// each chunk and state columns [32w, 32w+32)).
+//
+// A tcgen05.mma is issued by one thread, and that thread shares its scheduler
+// with the math warps of its TMEM lane quadrant: with those warps busy, one
+// thread's issue rate drops several-fold. The 76 products of a chunk are
+// therefore split over three issuers on three schedulers (A: the Gram products,
+// dW0, V^T; B: the r accumulator and the Lam update; C: the dx accumulator), so
+// that each accumulator has a single issuer.
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -123,10 +130,11 @@ struct Smem {
   alignas(16) float ered[2][NMATH];  // by chunk parity: the d_alpha of chunk it reads its
                                      // slots while faster warps start chunk it + 1
   uint64_t xfull[NS], xempty[NS];
+  uint64_t staged[NS];  // the dg / dx staging tiles of the stage are written
   uint64_t gfull[GS], gempty[GS];
   uint64_t sfull;  // S_in tile loaded
   uint64_t ccfull, b1full, b2full;
-  uint64_t m1a, m1done, m2done, lscaled, xgready, xgfree, lbfree, lbready, done;
+  uint64_t m1a, m1done, m2done, lscaled, xgready, lbfree, lbready, done[3];
   uint32_t tmem_base;
   int abort;
 };
@@ -135,7 +143,7 @@ constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
 static_assert(kSmemBytes <= 227 * 1024, "over the 227 KB of shared memory a CTA may use");
 
 enum : uint32_t {
-  W_TMA_XEMPTY = 0x001, W_TMA_SEMPTY, W_TMA_DRAIN,
+  W_TMA_XEMPTY = 0x001, W_TMA_SEMPTY, W_TMA_DRAIN, W_TMA_STAGED,
   W_MMA_XFULL = 0x101, W_MMA_M2, W_MMA_SFULL, W_MMA_LB, W_MMA_M1, W_MMA_XS, W_MMA_DONE,
   W_MMA_M1A,
   W_GATE_EMPTY = 0x201, W_XG_FULL, W_XG_GFULL, W_XG_FREE,
@@ -171,25 +179,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     sm.abort = 0;
     for (int s = 0; s < NS; ++s) {
       mbar_init(&sm.xfull[s], 1);
-      mbar_init(&sm.xempty[s], 2);  // the last products on X, G, U + the dg / dx stores' read
+      mbar_init(&sm.xempty[s], 4);  // the three issuers' last products on X, G, U + the dg / dx stores' read
+      mbar_init(&sm.staged[s], 1);
     }
     for (int g = 0; g < GS; ++g) {
       mbar_init(&sm.gfull[g], 32);
       mbar_init(&sm.gempty[g], NMATH);
     }
     mbar_init(&sm.sfull, 1);
-    mbar_init(&sm.lbfree, 1);
+    mbar_init(&sm.lbfree, 2);  // R1 (issuer B) and Gs Lam (issuer C)
     mbar_init(&sm.ccfull, 1);
-    mbar_init(&sm.b1full, 1);
-    mbar_init(&sm.b2full, 1);
+    mbar_init(&sm.b1full, 2);  // R1 (B) and DXb (C)
+    mbar_init(&sm.b2full, 3);  // all three issuers
     mbar_init(&sm.m1a, NMATH);
     mbar_init(&sm.m1done, NMATH);
     mbar_init(&sm.m2done, NMATH);
     mbar_init(&sm.lscaled, NMATH);
-    mbar_init(&sm.xgready, 1);
-    mbar_init(&sm.xgfree, 1);
+    mbar_init(&sm.xgready, NMATH);
     mbar_init(&sm.lbready, NMATH);
-    mbar_init(&sm.done, 1);
+    for (int i = 0; i < 3; ++i) mbar_init(&sm.done[i], 1);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -235,212 +243,73 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   if (warp < 4) {
     if (warp == 0) {
-      // ---------------------------------------------------------- TMA producer
-      if (lane == 0) {
-        int xi = 0, si = 0;
-        for (int it = 0; it < nch; ++it) {
-          const int c = c1 - 1 - it, st = it % NS;
-          if (!mbar_wait(&sm.xempty[st], ((it / NS) & 1) ^ 1, wc, W_TMA_XEMPTY)) break;
-          mbar_arrive_expect_tx(&sm.xfull[st], 6 * TILE);
-          tma_load_3d(sm.X[st], &tmX, &sm.xfull[st], 0, c * C, bh);
-          tma_load_3d(sm.X[st] + TILE, &tmX, &sm.xfull[st], 64, c * C, bh);
-          tma_load_3d(sm.G[st], &tmG, &sm.xfull[st], p.n0, c * C, bh);
-          tma_load_3d(sm.G[st] + TILE, &tmG, &sm.xfull[st], p.n0 + 64, c * C, bh);
-          tma_load_3d(sm.U[st], &tmU, &sm.xfull[st], p.n0, c * C, bh);
-          tma_load_3d(sm.U[st] + TILE, &tmU, &sm.xfull[st], p.n0 + 64, c * C, bh);
-          xi = it + 1;
-          // S_in goes to SL[it & 1], which last held the bf16 Lam that chunk it - 1 read:
-          // load once that chunk's last products on it have completed
-          if (it > 0 && !mbar_wait(&sm.lbfree, (it - 1) & 1, wc, W_TMA_SEMPTY)) break;
-          mbar_arrive_expect_tx(&sm.sfull, 2 * BIG);
-          tma_load_3d(sm.SL[it & 1], &tmS, &sm.sfull, 0, p.n0, bh * nch_all + c);
-          tma_load_3d(sm.SL[it & 1] + BIG, &tmS, &sm.sfull, 64, p.n0, bh * nch_all + c);
-          si = it + 1;
-        }
-        for (int it = xi > NS ? xi - NS : 0; it < xi; ++it)
-          mbar_drain(&sm.xfull[it % NS], (it / NS) & 1, wc, W_TMA_DRAIN);
-        if (si > 0) mbar_drain(&sm.sfull, (si - 1) & 1, wc, W_TMA_DRAIN);
-      }
-    } else if (warp == 1) {
-      // ---------------------------------------------------------- MMA issuer
-      if (lane == 0) {
-        const uint32_t id_cc = idesc_bf16(64, 64, false, false);      // X X^T, U G^T, G U^T
-        const uint32_t id_w = idesc_bf16(128, 128, true, true);       // U^T X, U^T Xg
-        const uint32_t id_tb = idesc_bf16(64, 128, false, true);      // U S_in, U W0, Ar U, ...
-        const uint32_t id_r1 = idesc_bf16(64, 128, false, false);     // X Lam^T
-        const uint32_t id_v = idesc_bf16(64, 64, false, true);        // Bm Q^T
-        const uint32_t sW0 = smem_u32(sm.W0);
-        // Issue order per chunk: K, Kug and dW0 as soon as X, G, U land (their accumulators
-        // were last read by the previous chunk's matrix build); KugT and R1 once the previous
-        // chunk's output phase has read its accumulators and left the bf16 Lam; DXb when S_in
-        // lands; the Lam update once the math warps have scaled Lam; the dx terms that need
-        // only scaled G and DXb; and last the three products that need the chunk matrices.
-        auto xgu = [&](int it, uint32_t& sX, uint32_t& sG, uint32_t& sU) {
-          const int st = it % NS;
-          sX = smem_u32(sm.X[st]);
-          sG = smem_u32(sm.G[st]);
-          sU = smem_u32(sm.U[st]);
-        };
-        // this chunk's S_in / chunk-matrix region, and the bf16 Lam of the chunk before
-        auto region_s = [&](int it) { return smem_u32(sm.SL[it & 1]); };
-        auto region_l = [&](int it) { return smem_u32(sm.SL[(it & 1) ^ 1]); };
-        auto phase1a = [&](int it) -> bool {  // K = X X^T, Kug = U G^T, dW0 += U^T X
-          uint32_t sX, sG, sU;
-          xgu(it, sX, sG, sU);
-          if (!mbar_wait(&sm.xfull[it % NS], (it / NS) & 1, wc, W_MMA_XFULL)) return false;
-          tc_fence_after();
-          #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * TILE + (kk & 3) * 32;
-            const uint64_t dX = desc_at(sw128_desc(sX, 16, 1024), off);
-            umma_bf16(tbase + COL_KK, dX, dX, id_cc, kk > 0);
-            umma_bf16(tbase + COL_KK + LANE16, desc_at(sw128_desc(sU, 16, 1024), off),
-                      desc_at(sw128_desc(sG, 16, 1024), off), id_cc, kk > 0);
-          }
-          #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_bf16(tbase + COL_W, desc_at(sw128_desc(sU, TILE, 1024), kk * 2048),
-                      desc_at(sw128_desc(sX, TILE, 1024), kk * 2048), id_w, (it > 0 || kk > 0));
-          return true;
-        };
-        auto phase1r = [&](int it) -> bool {  // KugT = G U^T, R1 = X Lam^T
-          uint32_t sX, sG, sU;
-          xgu(it, sX, sG, sU);
-          // KugT, R1 (and DXb after them) overwrite accumulators that the previous chunk's
-          // output phase reads until m2done: V^T's neighbour lanes, r and dx
-          if (it > 0 && !mbar_wait(&sm.m2done, (it - 1) & 1, wc, W_MMA_M2)) return false;
-          if (it > 0 && !mbar_wait(&sm.lbready, (it - 1) & 1, wc, W_MMA_LB)) return false;
-          tc_fence_after();
-          const uint32_t sL = region_l(it);
-          #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * TILE + (kk & 3) * 32;
-            umma_bf16(tbase + COL_KT, desc_at(sw128_desc(sG, 16, 1024), off),
-                      desc_at(sw128_desc(sU, 16, 1024), off), id_cc, kk > 0);
-          }
-          umma_commit(&sm.ccfull);  // the Gram products (the last readers of unscaled G)
-          #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            umma_bf16(tbase + COL_RX, desc_at(sw128_desc(sX, 16, 1024), (kk >> 2) * TILE + (kk & 3) * 32),
-                      desc_at(sw128_desc(sL, 16, 1024), (kk >> 2) * BIG + (kk & 3) * 32), id_r1, kk > 0);
-          return true;
-        };
-        auto phase1b = [&](int it) -> bool {  // DXb = U S_in, once S_in has landed
-          uint32_t sX, sG, sU;
-          xgu(it, sX, sG, sU);
-          if (!mbar_wait(&sm.sfull, it & 1, wc, W_MMA_SFULL)) return false;
-          tc_fence_after();
-          const uint32_t sS = region_s(it);
-          #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)  // DXb = U S_in
-            umma_bf16(tbase + COL_RX + LANE16, desc_at(sw128_desc(sU, 16, 1024), (kk >> 2) * TILE + (kk & 3) * 32),
-                      desc_at(sw128_desc(sS, BIG, 1024), kk * 2048), id_tb, kk > 0);
-          if (!(p.inject == 2 && it == 1)) umma_commit(&sm.b1full);  // R1, Gram, dW0, DXb
-          return true;
-        };
-        auto phase2a = [&](int it) -> bool {  // dx terms that need only Gs and gam (.) DXb
-          uint32_t sX, sG, sU;
-          xgu(it, sX, sG, sU);
-          if (!mbar_wait(&sm.m1a, it & 1, wc, W_MMA_M1A)) return false;
-          tc_fence_after();
-          const uint32_t sL = region_l(it);
-          #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)  // dx = gam (.) DXb + U W0
-            umma_bf16(tbase + COL_RX + LANE16, desc_at(sw128_desc(sU, 16, 1024), (kk >> 2) * TILE + (kk & 3) * 32),
-                      desc_at(sw128_desc(sW0, BIG, 1024), kk * 2048), id_tb, 1);
-          if (!p.local) {
-            #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)  //      + Gs Lam
-              umma_bf16(tbase + COL_RX + LANE16, desc_at(sw128_desc(sG, 16, 1024), (kk >> 2) * TILE + (kk & 3) * 32),
-                        desc_at(sw128_desc(sL, BIG, 1024), kk * 2048), id_tb, 1);
-          }
-          umma_commit(&sm.lbfree);  // the last product reading the bf16 Lam of the chunk before
-          return true;
-        };
-        auto phase2b = [&](int it) -> bool {  // the products of the chunk matrices
-          uint32_t sX, sG, sU;
-          xgu(it, sX, sG, sU);
-          if (!mbar_wait(&sm.m1done, it & 1, wc, W_MMA_M1)) return false;
-          tc_fence_after();
-          const uint32_t sS = region_s(it);
-          #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)  // V^T = Bm Q^T
-            umma_bf16(tbase + COL_KT + LANE16, desc_at(sw128_desc(sS, 16, 1024), CC_BM + kk * 32),
-                      desc_at(sw128_desc(sS, TILE, 1024), CC_QT + kk * 2048), id_v, kk > 0);
-          #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)  // r = del (.) R1 + Ar U
-            umma_bf16(tbase + COL_RX, desc_at(sw128_desc(sS, 16, 1024), CC_AR + kk * 32),
-                      desc_at(sw128_desc(sU, TILE, 1024), kk * 2048), id_tb, 1);
-          #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)  // dx += Z X
-            umma_bf16(tbase + COL_RX + LANE16, desc_at(sw128_desc(sS, 16, 1024), CC_Z + kk * 32),
-                      desc_at(sw128_desc(sX, TILE, 1024), kk * 2048), id_tb, 1);
-          umma_commit(&sm.b2full);           // every product of this chunk, the Lam update included
-          umma_commit(&sm.xempty[it % NS]);  // the last products reading X, G and U
-          return true;
-        };
-        auto phase3 = [&](int it) -> bool {  // Lam += U^T Xg (Lam pre-scaled by the math warps)
-          uint32_t sX, sG, sU;
-          xgu(it, sX, sG, sU);
-          if (!mbar_wait(&sm.lscaled, it & 1, wc, W_MMA_XS)) return false;
-          if (!mbar_wait(&sm.xgready, it & 1, wc, W_MMA_XS)) return false;
-          tc_fence_after();
-          const uint32_t sXg = smem_u32(sm.Xg);
-          #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_bf16(tbase + COL_L, desc_at(sw128_desc(sU, TILE, 1024), kk * 2048),
-                      desc_at(sw128_desc(sXg, TILE, 1024), kk * 2048), id_w, 1);
-          umma_commit(&sm.xgfree);
-          return true;
-        };
-        // K, Kug and dW0 run while the previous chunk's output phase reads its accumulators;
-        // R1 and DXb follow, and the Lam update is issued as soon as the math warps have
-        // scaled Lam, so that it runs while they build the chunk matrices.
-        bool ok = true;
-        for (int it = 0; it < nch && ok; ++it)
-          ok = phase1a(it) && phase1r(it) && phase1b(it) && phase3(it) && phase2a(it) &&
-               phase2b(it);
-        umma_commit(&sm.done);
-        mbar_drain(&sm.done, 0, wc, W_MMA_DONE);
-      }
-    } else if (warp == 3) {
-      // ---------------------------------------------------------- Xg = diag(gam) X
-      bool ok = true;
-      for (int it = 0; it < nch && ok; ++it) {
-        const int st = it % NS, g = it % GS;
-        ok = ok && mbar_wait_warp(&sm.xfull[st], (it / NS) & 1, wc, W_XG_FULL);
-        ok = ok && mbar_wait_warp(&sm.gfull[g], (it / GS) & 1, wc, W_XG_GFULL);
-        ok = ok && (it == 0 || mbar_wait_warp(&sm.xgfree, (it - 1) & 1, wc, W_XG_FREE));
-        if (!ok) break;
-        const GateSlot& gs = sm.gates[g];
-        const uint32_t src = smem_u32(sm.X[st]), dst = smem_u32(sm.Xg);
-#pragma unroll 4
-        for (int idx = lane; idx < 2 * TILE / 16; idx += 32) {
-          const uint32_t off = (uint32_t)idx * 16;
-          const int sr = (off & (TILE - 1)) >> 7;  // token row
-          const __nv_bfloat162 f2 = __float2bfloat162_rn(gs.gam[sr]);
-          const uint32_t fv = *reinterpret_cast<const uint32_t*>(&f2);
-          const uint4 v = ld_shared_v4(src + off);
-          st_shared_v4(dst + off, hmul2_bf16(v.x, fv), hmul2_bf16(v.y, fv), hmul2_bf16(v.z, fv),
-                       hmul2_bf16(v.w, fv));
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.xgready);
-      }
-    } else if (warp == 2) {
-      // ---------------------------------------------------------- gate prep
+      // ---------------------------------------------------------- TMA producer + gate prep
+      // Per chunk: lane 0 issues the tile loads (X, G, U into the stage, then S_in into
+      // the region the chunk before left its bf16 Lam in), then the warp prepares the
+      // gates, whose alpha / eta were loaded one chunk ahead.
       const size_t gbase = (size_t)bh * T;
-      for (int it = 0; it < nch; ++it) {
-        const int c = c1 - 1 - it, g = it % GS;
-        if (!mbar_wait_warp(&sm.gempty[g], ((it / GS) & 1) ^ 1, wc, W_GATE_EMPTY)) break;
+      int xi = 0, si = 0;
+      bool ok = true;
+      float a0 = 1.f, a1 = 1.f, e0 = 0.f, e1 = 0.f;  // gates of the chunk prepared next
+      auto gate_load = [&](int it, float& x0, float& x1, float& y0, float& y1) {
+        const int c = c1 - 1 - it, t0 = c * C + lane, t1 = t0 + 32;
+        const bool in = it < nch;
+        x0 = in && t0 < T ? p.alpha[gbase + t0] : 1.f;
+        x1 = in && t1 < T ? p.alpha[gbase + t1] : 1.f;
+        y0 = in && t0 < T ? p.eta[gbase + t0] : 0.f;
+        y1 = in && t1 < T ? p.eta[gbase + t1] : 0.f;
+      };
+      auto store_staged = [&](int j) -> bool {
+        const int sj = j % NS, t0j = (c1 - 1 - j) * C;
+        if (!mbar_wait(&sm.staged[sj], (j / NS) & 1, wc, W_TMA_STAGED)) return false;
+        tma_store_3d(&tmDG, sm.G[sj], p.n0, t0j, bh);
+        tma_store_3d(&tmDG, sm.G[sj] + TILE, p.n0 + 64, t0j, bh);
+        tma_store_3d(&tmDX, sm.U[sj], 0, t0j, bh);
+        tma_store_3d(&tmDX, sm.U[sj] + TILE, 64, t0j, bh);
+        tma_store_commit();
+        tma_store_wait_read();
+        mbar_arrive(&sm.xempty[sj]);
+        return true;
+      };
+      gate_load(0, a0, a1, e0, e1);
+      for (int it = 0; it < nch && ok; ++it) {
+        const int c = c1 - 1 - it, st = it % NS, g = it % GS;
+        int tok = 1;
+        if (lane == 0) {
+          // dg and dx of chunk it - NS, staged in this stage's G and U tiles; the stage is
+          // free for chunk it once the stores have read them (rows past T are clipped)
+          if (it >= NS && !store_staged(it - NS)) {
+            tok = 0;
+          } else if (!mbar_wait(&sm.xempty[st], ((it / NS) & 1) ^ 1, wc, W_TMA_XEMPTY)) {
+            tok = 0;
+          } else {
+            mbar_arrive_expect_tx(&sm.xfull[st], 6 * TILE);
+            tma_load_3d(sm.X[st], &tmX, &sm.xfull[st], 0, c * C, bh);
+            tma_load_3d(sm.X[st] + TILE, &tmX, &sm.xfull[st], 64, c * C, bh);
+            tma_load_3d(sm.G[st], &tmG, &sm.xfull[st], p.n0, c * C, bh);
+            tma_load_3d(sm.G[st] + TILE, &tmG, &sm.xfull[st], p.n0 + 64, c * C, bh);
+            tma_load_3d(sm.U[st], &tmU, &sm.xfull[st], p.n0, c * C, bh);
+            tma_load_3d(sm.U[st] + TILE, &tmU, &sm.xfull[st], p.n0 + 64, c * C, bh);
+            xi = it + 1;
+            // S_in goes to SL[it & 1], which last held the bf16 Lam that chunk it - 1 read:
+            // load once that chunk's last products on it have completed
+            if (it > 0 && !mbar_wait(&sm.lbfree, (it - 1) & 1, wc, W_TMA_SEMPTY)) {
+              tok = 0;
+            } else {
+              mbar_arrive_expect_tx(&sm.sfull, 2 * BIG);
+              tma_load_3d(sm.SL[it & 1], &tmS, &sm.sfull, 0, p.n0, bh * nch_all + c);
+              tma_load_3d(sm.SL[it & 1] + BIG, &tmS, &sm.sfull, 64, p.n0, bh * nch_all + c);
+              si = it + 1;
+            }
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, tok, 0) != 0;
+        ok = ok && mbar_wait_warp(&sm.gempty[g], ((it / GS) & 1) ^ 1, wc, W_GATE_EMPTY);
+        if (!ok) break;
         GateSlot& gs = sm.gates[g];
-        const int t0 = c * C + lane, t1 = t0 + 32;
-        const float a0 = t0 < T ? p.alpha[gbase + t0] : 1.f;
-        const float a1 = t1 < T ? p.alpha[gbase + t1] : 1.f;
-        const float e0 = t0 < T ? p.eta[gbase + t0] : 0.f;
-        const float e1 = t1 < T ? p.eta[gbase + t1] : 0.f;
-        float l0 = fmaxf(log2f(a0), -100.f), l1 = fmaxf(log2f(a1), -100.f);
+        const float x0 = a0, x1 = a1, y0 = e0, y1 = e1;
+        gate_load(it + 1, a0, a1, e0, e1);  // the next chunk's gates, in flight meanwhile
+        float l0 = fmaxf(log2f(x0), -100.f), l1 = fmaxf(log2f(x1), -100.f);
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
           const float u0 = __shfl_up_sync(0xffffffffu, l0, o);
@@ -457,8 +326,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const float pm1 = __shfl_up_sync(0xffffffffu, l1, 1);
         gs.L[lane] = l0;
         gs.L[lane + 32] = l1;
-        gs.eta[lane] = e0;
-        gs.eta[lane + 32] = e1;
+        gs.eta[lane] = y0;
+        gs.eta[lane + 32] = y1;
         gs.gam[lane] = lane == 0 ? 1.f : exp2f(pm0);
         gs.gam[lane + 32] = exp2f(lane == 0 ? last0 : pm1);
         gs.del[lane] = exp2f(Lend - l0);
@@ -468,8 +337,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const float lm0 = lane == 0 ? 0.f : pm0, lm1 = lane == 0 ? last0 : pm1;  // L_{i-1}
           gs.ra[lane] = exp2f(lm0 - Mid);
           gs.ra[lane + 32] = exp2f(lm1 - Mid);
-          gs.ca[lane] = -e0 * exp2f(Mid - l0);
-          gs.ca[lane + 32] = -e1 * exp2f(Mid - l1);
+          gs.ca[lane] = -y0 * exp2f(Mid - l0);
+          gs.ca[lane + 32] = -y1 * exp2f(Mid - l1);
           gs.rb[lane] = exp2f(Mid - l0);
           gs.rb[lane + 32] = exp2f(Mid - l1);
           gs.cb[lane] = exp2f(lm0 - Mid);
@@ -482,6 +351,142 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         __syncwarp();
         mbar_arrive(&sm.gfull[g]);
       }
+      if (lane == 0) {
+        // the last chunks' dg and dx
+        for (int j = nch > NS ? nch - NS : 0; ok && j < nch; ++j) ok = store_staged(j);
+        tma_store_wait_all();
+        for (int it = xi > NS ? xi - NS : 0; it < xi; ++it)
+          mbar_drain(&sm.xfull[it % NS], (it / NS) & 1, wc, W_TMA_DRAIN);
+        if (si > 0) mbar_drain(&sm.sfull, (si - 1) & 1, wc, W_TMA_DRAIN);
+      }
+    } else if (lane == 0) {
+      // ---------------------------------------------------------- MMA issuers
+      // A (warp 1): the Gram products K | Kug and KugT, dW0, and V^T = Bm Q^T.
+      // B (warp 2): the r accumulator (R1 = X Lam^T, then + Ar U) and the Lam update.
+      // C (warp 3): the dx accumulator (DXb = U S_in, then + U W0 + Gs Lam + Z X).
+      // Each accumulator has one issuer; where one issuer's product follows another's
+      // (a scaling pass of the math warps in between), the math warps' barrier orders them.
+      const int ii = warp - 1;
+      const uint32_t id_cc = idesc_bf16(64, 64, false, false);      // X X^T, U G^T, G U^T
+      const uint32_t id_w = idesc_bf16(128, 128, true, true);       // U^T X, U^T Xg
+      const uint32_t id_tb = idesc_bf16(64, 128, false, true);      // U S_in, U W0, Ar U, ...
+      const uint32_t id_r1 = idesc_bf16(64, 128, false, false);     // X Lam^T
+      const uint32_t id_v = idesc_bf16(64, 64, false, true);        // Bm Q^T
+      const uint32_t sW0 = smem_u32(sm.W0);
+      bool ok = true;
+      for (int it = 0; it < nch && ok; ++it) {
+        const int st = it % NS;
+        const uint32_t sX = smem_u32(sm.X[st]), sG = smem_u32(sm.G[st]), sU = smem_u32(sm.U[st]);
+        const uint32_t sS = smem_u32(sm.SL[it & 1]);        // S_in, then the chunk matrices
+        const uint32_t sL = smem_u32(sm.SL[(it & 1) ^ 1]);  // the bf16 Lam of the chunk before
+        ok = mbar_wait(&sm.xfull[st], (it / NS) & 1, wc, W_MMA_XFULL);
+        if (!ok) break;
+        if (ii == 0) {
+          // K | Kug and dW0: the previous chunk's matrix build has read K | Kug
+          ok = it == 0 || mbar_wait(&sm.m1done, (it - 1) & 1, wc, W_MMA_M1);
+          if (!ok) break;
+          tc_fence_after();
+          #pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * TILE + (kk & 3) * 32;
+            const uint64_t dX = desc_at(sw128_desc(sX, 16, 1024), off);
+            umma_bf16(tbase + COL_KK, dX, dX, id_cc, kk > 0);
+            umma_bf16(tbase + COL_KK + LANE16, desc_at(sw128_desc(sU, 16, 1024), off),
+                      desc_at(sw128_desc(sG, 16, 1024), off), id_cc, kk > 0);
+          }
+          #pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tbase + COL_W, desc_at(sw128_desc(sU, TILE, 1024), kk * 2048),
+                      desc_at(sw128_desc(sX, TILE, 1024), kk * 2048), id_w, (it > 0 || kk > 0));
+          // KugT: its columns neighbour V^T, which the previous output phase reads until m2done
+          ok = it == 0 || mbar_wait(&sm.m2done, (it - 1) & 1, wc, W_MMA_M2);
+          if (!ok) break;
+          tc_fence_after();
+          #pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * TILE + (kk & 3) * 32;
+            umma_bf16(tbase + COL_KT, desc_at(sw128_desc(sG, 16, 1024), off),
+                      desc_at(sw128_desc(sU, 16, 1024), off), id_cc, kk > 0);
+          }
+          umma_commit(&sm.ccfull);  // the Gram products (the last readers of unscaled G)
+          // V^T = Bm Q^T from the chunk matrices
+          ok = mbar_wait(&sm.m1done, it & 1, wc, W_MMA_M1);
+          if (!ok) break;
+          tc_fence_after();
+          #pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tbase + COL_KT + LANE16, desc_at(sw128_desc(sS, 16, 1024), CC_BM + kk * 32),
+                      desc_at(sw128_desc(sS, TILE, 1024), CC_QT + kk * 2048), id_v, kk > 0);
+        } else if (ii == 1) {
+          // R1 = X Lam^T: r was read by the previous output phase, the bf16 Lam is in place
+          ok = it == 0 || (mbar_wait(&sm.m2done, (it - 1) & 1, wc, W_MMA_M2) &&
+                           mbar_wait(&sm.lbready, (it - 1) & 1, wc, W_MMA_LB));
+          if (!ok) break;
+          tc_fence_after();
+          #pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_bf16(tbase + COL_RX, desc_at(sw128_desc(sX, 16, 1024), (kk >> 2) * TILE + (kk & 3) * 32),
+                      desc_at(sw128_desc(sL, 16, 1024), (kk >> 2) * BIG + (kk & 3) * 32), id_r1, kk > 0);
+          if (!(p.inject == 2 && it == 1)) umma_commit(&sm.b1full);
+          umma_commit(&sm.lbfree);  // one of the two products reading the bf16 Lam
+          // Lam += U^T Xg once the math warps have scaled Lam and written Xg
+          ok = mbar_wait(&sm.lscaled, it & 1, wc, W_MMA_XS) && mbar_wait(&sm.xgready, it & 1, wc, W_MMA_XS);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t sXg = smem_u32(sm.Xg);
+          #pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tbase + COL_L, desc_at(sw128_desc(sU, TILE, 1024), kk * 2048),
+                      desc_at(sw128_desc(sXg, TILE, 1024), kk * 2048), id_w, 1);
+          // r = del (.) R1 + Ar U
+          ok = mbar_wait(&sm.m1done, it & 1, wc, W_MMA_M1);
+          if (!ok) break;
+          tc_fence_after();
+          #pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tbase + COL_RX, desc_at(sw128_desc(sS, 16, 1024), CC_AR + kk * 32),
+                      desc_at(sw128_desc(sU, TILE, 1024), kk * 2048), id_tb, 1);
+        } else {
+          // DXb = U S_in: dx was read by the previous output phase, S_in has landed
+          ok = (it == 0 || mbar_wait(&sm.m2done, (it - 1) & 1, wc, W_MMA_M2)) &&
+               mbar_wait(&sm.sfull, it & 1, wc, W_MMA_SFULL);
+          if (!ok) break;
+          tc_fence_after();
+          #pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_bf16(tbase + COL_RX + LANE16, desc_at(sw128_desc(sU, 16, 1024), (kk >> 2) * TILE + (kk & 3) * 32),
+                      desc_at(sw128_desc(sS, BIG, 1024), kk * 2048), id_tb, kk > 0);
+          umma_commit(&sm.b1full);
+          // dx = gam (.) DXb + U W0 + Gs Lam, once DXb is scaled and G is scaled in place
+          ok = mbar_wait(&sm.m1a, it & 1, wc, W_MMA_M1A);
+          if (!ok) break;
+          tc_fence_after();
+          #pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_bf16(tbase + COL_RX + LANE16, desc_at(sw128_desc(sU, 16, 1024), (kk >> 2) * TILE + (kk & 3) * 32),
+                      desc_at(sw128_desc(sW0, BIG, 1024), kk * 2048), id_tb, 1);
+          if (!p.local) {
+            #pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              umma_bf16(tbase + COL_RX + LANE16, desc_at(sw128_desc(sG, 16, 1024), (kk >> 2) * TILE + (kk & 3) * 32),
+                        desc_at(sw128_desc(sL, BIG, 1024), kk * 2048), id_tb, 1);
+          }
+          umma_commit(&sm.lbfree);  // the other product reading the bf16 Lam
+          // dx += Z X
+          ok = mbar_wait(&sm.m1done, it & 1, wc, W_MMA_M1);
+          if (!ok) break;
+          tc_fence_after();
+          #pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tbase + COL_RX + LANE16, desc_at(sw128_desc(sS, 16, 1024), CC_Z + kk * 32),
+                      desc_at(sw128_desc(sX, TILE, 1024), kk * 2048), id_tb, 1);
+        }
+        umma_commit(&sm.b2full);      // this issuer's products of the chunk
+        umma_commit(&sm.xempty[st]);  // its last reads of X, G and U
+      }
+      // teardown: every MMA this thread issued completes before TMEM is released
+      umma_commit(&sm.done[ii]);
+      mbar_drain(&sm.done[ii], 0, wc, W_MMA_DONE);
     }
   } else {
     // ------------------------------------------------------------ math warpgroups
@@ -532,6 +537,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       ok = ok && mbar_wait_warp(&sm.sfull, it & 1, wc, W_M_GFULL);
       tc_fence_after();
 
+      if (ok) {
+        // ---- Xg = diag(gam) X for the Lam update (the previous update has read Xg: the
+        //      previous chunk's b2full covers it); two 16-byte pieces per thread
+        const uint32_t dst = smem_u32(sm.Xg);
+#pragma unroll
+        for (int k = 0; k < (2 * TILE / 16) / (32 * NMATH); ++k) {
+          const uint32_t off = (uint32_t)(mt + 32 * NMATH * k) * 16;
+          const int sr = (off & (TILE - 1)) >> 7;  // token row
+          const __nv_bfloat162 f2 = __float2bfloat162_rn(gs.gam[sr]);
+          const uint32_t fv = *reinterpret_cast<const uint32_t*>(&f2);
+          const uint4 v = ld_shared_v4(sX + off);
+          st_shared_v4(dst + off, hmul2_bf16(v.x, fv), hmul2_bf16(v.y, fv), hmul2_bf16(v.z, fv),
+                       hmul2_bf16(v.w, fv));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.xgready);
+      }
       if (ok) {
         // ---- <Lam_end, S_in>, then Lam <- 2^{L_{C-1}} Lam in place (Lam_end is complete
         //      since the previous chunk's b2full; this overlaps the R1 and DXb products)
@@ -904,13 +927,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
       named_sync_math();  // (B4) t, hv of all warpgroups and the dg / dx staging tiles written
-      if (ok && mt == 0) {  // rows past T are clipped by the tensor maps
-        tma_store_3d(&tmDG, sm.G[st], p.n0, t0, bh);
-        tma_store_3d(&tmDG, sm.G[st] + TILE, p.n0 + 64, t0, bh);
-        tma_store_3d(&tmDX, sm.U[st], 0, t0, bh);
-        tma_store_3d(&tmDX, sm.U[st] + TILE, 64, t0, bh);
-        tma_store_commit();
-      }
+      if (ok && mt == 0) mbar_arrive(&sm.staged[st]);  // warp 0 stores dg and dx from here
       if (ok && mt < C) {  // d_eta_j = -(del_j q_j + t_j)
         const int j = mt;
         const float deta =
@@ -932,11 +949,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (t0 + i < T) p.d_alpha[tokbase + i] = p.accumulate ? p.d_alpha[tokbase + i] + da : da;
       }
 
-      // ---- the staging tiles are read: the stage may take the X, G, U of chunk it + NS
-      if (mt == 0) {
-        tma_store_wait_read();
-        mbar_arrive(&sm.xempty[st]);
-      }
       __syncwarp();
       if (ok && lane == 0) mbar_arrive(&sm.gempty[g]);  // this chunk's gates are read
       // No barrier is needed here. Faster warps may start the next chunk while warps
@@ -947,7 +959,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // this stage land in the staging tiles only after their stores have read them.
     }
 
-    if (mt == 0) tma_store_wait_all();
     // ---- this scan's dW0 partial: the last b2full wait covered every product
     if (ok) {
       float v[32];
