@@ -793,9 +793,62 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             store_pair(cc, v0, v1);
           }
         };
+        // A diagonal block with the factored decays: the lane pair of row i splits the
+        // 16 columns (lo: the first 8, hi: the last 8) and each lane produces all four
+        // matrices for its columns. Lo holds K and KugT of the row, hi holds Kug; one
+        // exchange per column gives lo the Kug and hi the K of its own columns, a second
+        // gives hi the KugT.
+        auto build_diag = [&]() {
+          const int h = lo ? 0 : 1;
+          const int jb = j0w + 8 * h;
+          const float neti = -zb * eti;
+          float cbv[8], cav[8], qvv[8], pvv[8];
+#pragma unroll
+          for (int e4 = 0; e4 < 8; e4 += 4) {
+            const float4 cb4 = *reinterpret_cast<const float4*>(&gs.cb[jb + e4]);
+            const float4 ca4 = *reinterpret_cast<const float4*>(&gs.ca[jb + e4]);
+            const float4 q4 = *reinterpret_cast<const float4*>(&sm.qv[jb + e4]);
+            const float4 p4 = *reinterpret_cast<const float4*>(&sm.pv[jb + e4]);
+            cbv[e4] = cb4.x; cbv[e4 + 1] = cb4.y; cbv[e4 + 2] = cb4.z; cbv[e4 + 3] = cb4.w;
+            cav[e4] = ca4.x; cav[e4 + 1] = ca4.y; cav[e4 + 2] = ca4.z; cav[e4 + 3] = ca4.w;
+            qvv[e4] = q4.x; qvv[e4 + 1] = q4.y; qvv[e4 + 2] = q4.z; qvv[e4 + 3] = q4.w;
+            pvv[e4] = p4.x; pvv[e4 + 1] = p4.y; pvv[e4 + 2] = p4.z; pvv[e4 + 3] = p4.w;
+          }
+          float ar[8], zz[8], qq[8], bm[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            // lo sends K of column 8+e and receives Kug of column e; hi the reverse
+            const float x1 = __shfl_xor_sync(0xffffffffu, lo ? vkk[8 + e] : vkk[e], 16);
+            // lo sends KugT of column 8+e (hi's value is not used)
+            const float x2 = __shfl_xor_sync(0xffffffffu, vkt[8 + e], 16);
+            const float kr = lo ? vkk[e] : x1;      // x_i . x_j
+            const float kg = lo ? x1 : vkk[8 + e];  // u_i . g_j
+            const float kt = lo ? vkt[e] : x2;      // g_i . u_j
+            const int j = jb + e;
+            const float bij = cbv[e] * rbi, aij = rai * cav[e];
+            const bool up = j > i, dn = j < i;
+            const float bu = up ? bij : 0.f, ad = dn ? aij : 0.f;
+            ar[e] = bu * kr;                               // Ar = b K (j > i)
+            zz[e] = fmaf(ad, kg, neti * bu * kt);          // Z = a Kug (j < i) - eta_i b KugT (j > i)
+            qq[e] = dn ? kr * kg : 0.f;                    // Q^T: K Kug (j < i)
+            bm[e] = bu;                                    // Bm = b (j > i)
+            t2part = fmaf(ad, qvv[e], t2part);
+            tpart = fmaf(ar[e], kt, tpart);
+            t3part = fmaf(bu, pvv[e], t3part);
+          }
+          const uint32_t cidx = 2 * wg + h;
+          st_shared_v4(sS + CC_AR + sw128_off(i, cidx), pack_bf16(ar[0], ar[1]), pack_bf16(ar[2], ar[3]),
+                       pack_bf16(ar[4], ar[5]), pack_bf16(ar[6], ar[7]));
+          st_shared_v4(sS + CC_Z + sw128_off(i, cidx), pack_bf16(zz[0], zz[1]), pack_bf16(zz[2], zz[3]),
+                       pack_bf16(zz[4], zz[5]), pack_bf16(zz[6], zz[7]));
+          st_shared_v4(sS + CC_QT + sw128_off(i, cidx), pack_bf16(qq[0], qq[1]), pack_bf16(qq[2], qq[3]),
+                       pack_bf16(qq[4], qq[5]), pack_bf16(qq[6], qq[7]));
+          st_shared_v4(sS + CC_BM + sw128_off(i, cidx), pack_bf16(bm[0], bm[1]), pack_bf16(bm[2], bm[3]),
+                       pack_bf16(bm[4], bm[5]), pack_bf16(bm[6], bm[7]));
+        };
         if (gs.fac && wg > q) build_above();
         else if (gs.fac && wg < q) build_below();
-        else if (gs.fac) build(std::true_type{});
+        else if (gs.fac) build_diag();
         else build(std::false_type{});
         // each partial is nonzero in one lane half only; combine the pair
         tpart += __shfl_xor_sync(0xffffffffu, tpart, 16);
