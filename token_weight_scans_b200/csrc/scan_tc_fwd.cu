@@ -22,7 +22,8 @@
 // The fp32 state lives in TMEM: the state warps scale it by 2^{L_{C-1}} in place
 // and the tensor core accumulates G^T Xhat onto it, so no thread carries it.
 //
-// Warp roles (20 warps): 0 TMA producer, 1 and 2 MMA issuers (1 owns TMEM),
+// Warp roles (20 warps): 0 TMA producer (X and G tiles three chunks ahead: a tile
+// takes about 2 us to land), 1 and 2 MMA issuers (1 owns TMEM),
 // 3 gate prep (log2 alpha cumulative sums, prefetched), 4..11 two state
 // warpgroups (bf16 copy of the chunk-start state for the S X^T product and the
 // checkpoint, then the in-place decay, then the scaled-X tile of the next chunk,
@@ -34,9 +35,10 @@
 // with the math warps of its TMEM lane quadrant; its issue rate drops several-
 // fold while they are busy. So the products are split between two issuers on
 // different schedulers: warp 1 issues K, the state update (right after K, so
-// that nothing queues ahead of it on the state chain), X W0^T and P G; warp 2
-// issues X S^T. Y is complete when both have committed, a stage is free when
-// both have read it.
+// that nothing queues ahead of it on the state chain) and P G; warp 2 issues
+// X W0^T and X S^T. P G accumulates onto X W0^T, so warp 1 waits for warp 2's
+// commit of that product first. Y is complete when both have committed, a
+// stage is free when both have read it.
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -57,7 +59,7 @@ using namespace sm100;
 namespace {
 
 constexpr int C = 64;          // tokens per chunk
-constexpr int NS = 2;          // TMA stages (X and G tiles)
+constexpr int NS = 3;          // TMA stages (X and G tiles)
 constexpr int GS = 4;          // gate slots
 constexpr int NTHREADS = 640;  // 20 warps
 constexpr int TILE = C * 128;  // bytes of one [64 rows x 128 B] swizzled block
@@ -92,7 +94,7 @@ struct Smem {
   uint8_t X[NS][2 * TILE];     // k-blocks [0,64), [64,128): 64 token rows x 128 B
   uint8_t G[NS][2 * TILE];     // n-blocks of the slice: 64 token rows x 128 B
   uint8_t W0[2][BIG];          // k-blocks: 128 n rows x 128 B (bf16 W0 slice)
-  uint8_t S[2][2][BIG];        // [buffer][k-block]: 128 n rows x 128 B (bf16 chunk-start state)
+  uint8_t S[2][BIG];           // [k-block]: 128 n rows x 128 B (bf16 chunk-start state)
   uint8_t Xh[2][2 * TILE];     // [buffer] scaled X, same layout as X
   uint8_t P[TILE];             // 64 token rows (i) x 128 B (j)
   uint8_t Ys[2 * TILE];        // y staging: n-blocks of 64 token rows x 128 B (TMA store)
@@ -101,8 +103,9 @@ struct Smem {
   uint64_t gfull[GS], gempty[GS];
   uint64_t kfull[2], kfree[2];
   uint64_t xhready[2], xhfree[2];  // per scaled-X buffer
-  uint64_t sready[2], sfree[2];    // per bf16 state buffer
+  uint64_t sready, sfree;          // the bf16 state tile
   uint64_t yfull[2], yfree[2];     // per Y1 | Y2 buffer
+  uint64_t y1full[2];              // per Y buffer: X W0^T (issuer 1) is complete
   uint64_t pready, dsfull, sscaled, done[2];
   uint32_t tmem_base;
   int abort;
@@ -115,7 +118,7 @@ static_assert(kSmemBytes <= 227 * 1024, "over the 227 KB of shared memory a CTA 
 enum : uint32_t {
   W_TMA_EMPTY = 0x001, W_TMA_DRAIN = 0x002,
   W_MMA_FULL = 0x101, W_MMA_KFREE, W_MMA_YFREE, W_MMA_XREADY, W_MMA_SSCALED, W_MMA_PREADY,
-  W_MMA_SREADY, W_MMA_DONE,
+  W_MMA_SREADY, W_MMA_DONE, W_MMA_Y1FULL,
   W_GATE_EMPTY = 0x201,
   W_XH_FULL = 0x301, W_XH_GFULL, W_XH_FREE,
   W_M_GFULL = 0x401, W_M_KFULL, W_M_YFULL,
@@ -164,14 +167,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&sm.kfree[b], 8);
       mbar_init(&sm.xhready[b], 8);  // the state warps
       mbar_init(&sm.xhfree[b], 1);
-      mbar_init(&sm.sready[b], 8);
-      mbar_init(&sm.sfree[b], 1);
       mbar_init(&sm.yfull[b], 2);  // both issuers write Y
       mbar_init(&sm.yfree[b], 8);
     }
     mbar_init(&sm.pready, 8);
+    mbar_init(&sm.sready, 8);
+    mbar_init(&sm.sfree, 1);
     mbar_init(&sm.dsfull, 1);
     mbar_init(&sm.sscaled, 8);
+    mbar_init(&sm.y1full[0], 1);
+    mbar_init(&sm.y1full[1], 1);
     mbar_init(&sm.done[0], 1);
     mbar_init(&sm.done[1], 1);
     fence_mbar_init();
@@ -226,7 +231,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
   } else if (warp == 1 || warp == 2) {
     // ------------------------------------------------------------ MMA issuers
-    const int ii = warp - 1;  // 0: K, the state update, X W0^T, P G; 1: X S^T
+    const int ii = warp - 1;  // 0: K, the state update, P G; 1: X W0^T, X S^T
     // (the state carry alone has no work for issuer 1)
     if (lane == 0 && (ii == 0 || full)) {
       const uint32_t id_k = idesc_bf16(64, 64, false, false);    // X X^T
@@ -237,7 +242,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int c = 0; c < nch; ++c) {
         const int s = c % NS, b = c & 1;
         const uint32_t sX = smem_u32(sm.X[s]), sG = smem_u32(sm.G[s]);
-        const uint32_t sXh = smem_u32(sm.Xh[b]), sS = smem_u32(sm.S[b][0]);
+        const uint32_t sXh = smem_u32(sm.Xh[b]), sS = smem_u32(sm.S[0]);
         const uint32_t tY1 = tbase + COL_Y + 128 * b, tY2 = tY1 + LANE16;
         if (!mbar_wait(&sm.full[s], (c / NS) & 1, wc, W_MMA_FULL)) break;
         if (ii == 0) {
@@ -267,6 +272,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             umma_commit(&sm.empty[s]);
             continue;
           }
+          // Y1 += P G onto X W0^T (issuer 1). The mask of chunk c + 1 overwrites P only
+          // after the K product of chunk c + 1 has completed, which this thread commits
+          // after these.
+          if (!mbar_wait(&sm.pready, c & 1, wc, W_MMA_PREADY)) break;
+          if (!mbar_wait(&sm.y1full[b], (c >> 1) & 1, wc, W_MMA_Y1FULL)) break;
+          tc_fence_after();
+          #pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tY1, desc_at(sw128_desc(sP, 16, 1024), kk * 32),
+                      desc_at(sw128_desc(sG, TILE, 1024), kk * 2048), id_pg, 1);
+          umma_commit(&sm.yfull[b]);
+          umma_commit(&sm.empty[s]);
+        } else {
           // Y1 = X W0^T into buffer b (the epilogue of chunk c - 2 has read it)
           if (!mbar_wait(&sm.yfree[b], ((c >> 1) & 1) ^ 1, wc, W_MMA_YFREE)) break;
           tc_fence_after();
@@ -277,20 +295,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             umma_bf16(tY1, desc_at(sw128_desc(sX, 16, 1024), aoff),
                       desc_at(sw128_desc(sW0, 16, 1024), boff), id_y, kk > 0);
           }
-          // Y1 += P G. The mask of chunk c + 1 overwrites P only after the K product
-          // of chunk c + 1 has completed, which this thread commits after these.
-          if (!mbar_wait(&sm.pready, c & 1, wc, W_MMA_PREADY)) break;
-          tc_fence_after();
-          #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_bf16(tY1, desc_at(sw128_desc(sP, 16, 1024), kk * 32),
-                      desc_at(sw128_desc(sG, TILE, 1024), kk * 2048), id_pg, 1);
-          umma_commit(&sm.yfull[b]);
-          umma_commit(&sm.empty[s]);
-        } else {
-          // Y2 = X S^T (bf16 chunk-start state in buffer b) into buffer b
-          if (!mbar_wait(&sm.sready[b], (c >> 1) & 1, wc, W_MMA_SREADY)) break;
-          if (!mbar_wait(&sm.yfree[b], ((c >> 1) & 1) ^ 1, wc, W_MMA_YFREE)) break;
+          umma_commit(&sm.y1full[b]);
+          // Y2 = X S^T (bf16 chunk-start state) into buffer b
+          if (!mbar_wait(&sm.sready, c & 1, wc, W_MMA_SREADY)) break;
           tc_fence_after();
           #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
@@ -299,7 +306,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             umma_bf16(tY2, desc_at(sw128_desc(sX, 16, 1024), aoff),
                       desc_at(sw128_desc(sS, 16, 1024), boff), id_y, kk > 0);
           }
-          umma_commit(&sm.sfree[b]);
+          umma_commit(&sm.sfree);
           umma_commit(&sm.yfull[b]);
           umma_commit(&sm.empty[s]);
         }
@@ -413,7 +420,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tmem_st_wait();
     }
     // Each warp TMA-stores what it wrote itself: its 32 rows of one k-block of the
-    // bf16 chunk-start state (bf16 [bh][chunk][dout][din], box of 32 rows).
+    // bf16 chunk-start state (bf16 [bh][chunk][dout][din], box of 32 rows). The tile is
+    // single-buffered; the store has a chunk to read it before the tile is rewritten.
     const uint32_t s_part = (uint32_t)(32 * q) * 128;  // byte offset of the warp's state rows
     // Xhat of the c-th walked chunk, w_j x_j (forward) or 2^{L_{j-1}} x_j (adjoint
     // summary), with packed bf16 multiplies; each state thread writes 4 of its 1024
@@ -443,14 +451,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     };
     bool ok = nch > 0 ? scaled_x(0) : true;
     for (int c = 0; c < nch && ok; ++c) {
-      const int g = c % GS, b = c & 1;
+      const int g = c % GS;
       const GateSlot& gs = sm.gates[g];
       ok = ok && mbar_wait_warp(&sm.gfull[g], (c / GS) & 1, wc, W_S_GFULL);
       // S_c is complete: the update of chunk c - 1 has accumulated onto it
       ok = ok && (c == 0 || mbar_wait_warp(&sm.dsfull, (c - 1) & 1, wc, W_S_DSFULL));
-      // buffer b was last read by the S X^T product and the checkpoint store of chunk c - 2
-      ok = ok && (!full || c < 2 || mbar_wait_warp(&sm.sfree[b], ((c - 2) >> 1) & 1, wc, W_S_SFREE));
-      if (lane == 0 && has_ck) tma_store_wait_read_n<1>();
+      // the bf16 state tile was last read by the S X^T product and the checkpoint store
+      // of chunk c - 1
+      ok = ok && (!full || c < 1 || mbar_wait_warp(&sm.sfree, (c - 1) & 1, wc, W_S_SFREE));
+      if (lane == 0 && has_ck) tma_store_wait_read_n<0>();
       __syncwarp();
       if (!ok) break;
       tc_fence_after();
@@ -474,20 +483,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.sscaled);  // the update of chunk c may accumulate
       if (full) {
-        const uint32_t srow = smem_u32(sm.S[b][hh]);
+        const uint32_t srow = smem_u32(sm.S[hh]);
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc)
           st_shared_v4(srow + sw128_off(n, cc), pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
         fence_proxy_async_smem();
       }
       __syncwarp();
-      if (lane == 0) {
-        if (full) {
-          mbar_arrive(&sm.sready[b]);  // the S X^T product of chunk c may read buffer b
-          if (has_ck) {  // the checkpoint of chunk c: the state at its first token
-            tma_store_3d(&tmS, sm.S[b][hh] + s_part, 64 * hh, n0 + 32 * q, bh * nch_all + cg(c));
-            tma_store_commit();
-          }
+      if (lane == 0 && full) {
+        mbar_arrive(&sm.sready);  // the S X^T product of chunk c may read the tile
+        if (has_ck) {  // the checkpoint of chunk c: the state at its first token
+          tma_store_3d(&tmS, sm.S[hh] + s_part, 64 * hh, n0 + 32 * q, bh * nch_all + cg(c));
+          tma_store_commit();
         }
       }
       // the scaled X of the next chunk, while the update of this one runs
