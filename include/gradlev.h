@@ -321,8 +321,8 @@ GRADLEV_API gradlev_status gradlev_mlp2_recon(int B, int H, int T, int d_x, int 
  * nothing (no cudaMalloc, cudaFree or allocating library routine).
  *   - Limit: the call needs gradlev_scan_bwd_noalloc_scratch_bytes() of
  *     scratch. That is the status word and the per-scan dW0 partials
- *     (B*H*d_out*d_in*4 bytes, times the number of segments per scan when the
- *     tensor-core path cuts few long scans into segments, plus the segment
+ *     (B*H*d_out*d_in*4 bytes, times the number of segments per scan when
+ *     either kernel family cuts few long scans into segments, plus the segment
  *     summaries), and, when ckpt is NULL, the chunk-start states as well; with
  *     ckpt NULL it equals gradlev_scan_workspace_bytes(.., is_bwd = 1). A
  *     problem that needs more than GRADLEV_NOALLOC_SCRATCH_BYTES returns

@@ -66,7 +66,7 @@ static size_t ckpt_bytes_of(int B, int H, int T, int din, int dout, gradlev_dtyp
                                : ffma::ckpt_bytes(B, H, T, din, dout);
 }
 
-// ---- segmented long scans (tensor-core path)
+// ---- segmented long scans (both kernel families)
 //
 // When the scans of a call cannot fill the GPU, each scan is cut into segments
 // that separate CTAs walk at the same time. Forward: a summary pass gives each
@@ -90,6 +90,13 @@ static SegPlan bwd_plan(int B, int H, int T) {
   return s;
 }
 
+// The CUDA-core kernels: one CTA per (scan, segment) in both directions.
+static SegPlan ffma_plan(int B, int H, int T) {
+  SegPlan s;
+  tc::segment_plan(B * H, (T + ffma::kChunk - 1) / ffma::kChunk, &s.nseg, &s.seg_chunks);
+  return s;
+}
+
 // Scratch of the segment passes: local summaries and combined states
 // ([B*H][nseg][dout][din] fp32 each) and the segment log-decays ([B*H][nseg]).
 static size_t seg_bytes(int B, int H, int din, int dout, int nseg) {
@@ -109,12 +116,12 @@ static SegBufs seg_bufs(char* base, int B, int H, int din, int dout, int nseg) {
 }
 
 static size_t fwd_scratch_bytes(int B, int H, int T, int din, int dout, gradlev_dtype dt) {
-  if (!use_tc(din, dout, dt)) return kStatusBytes;
+  if (!use_tc(din, dout, dt)) return kStatusBytes + seg_bytes(B, H, din, dout, ffma_plan(B, H, T).nseg);
   return kStatusBytes + seg_bytes(B, H, din, dout, fwd_plan(B, H, T, dout).nseg);
 }
 
 static size_t dW0_part_bytes(int B, int H, int T, int din, int dout, gradlev_dtype dt) {
-  const int nseg = use_tc(din, dout, dt) ? bwd_plan(B, H, T).nseg : 1;
+  const int nseg = use_tc(din, dout, dt) ? bwd_plan(B, H, T).nseg : ffma_plan(B, H, T).nseg;
   return align_up((size_t)B * H * nseg * din * dout * sizeof(float), 256);
 }
 
@@ -126,6 +133,8 @@ size_t bwd_scratch_bytes(int B, int H, int T, int din, int dout, gradlev_dtype d
     const size_t fseg = own_states ? seg_bytes(B, H, din, dout, fwd_plan(B, H, T, dout).nseg) : 0;
     const size_t bseg = seg_bytes(B, H, din, dout, bwd_plan(B, H, T).nseg);
     ws += fseg > bseg ? fseg : bseg;
+  } else {  // the same plan in both directions
+    ws += seg_bytes(B, H, din, dout, ffma_plan(B, H, T).nseg);
   }
   return ws;
 }
@@ -167,7 +176,28 @@ static gradlev_status launch_fwd_impl(int B, int H, int T, int din, int dout, gr
     return tc::launch_fwd(prm, x, g, st) == cudaSuccess ? GRADLEV_OK : GRADLEV_ERR_CUDA;
   }
   ffma::FwdArgs a{B, H, T, din, dout, x, g, eta, alpha, W0, y, static_cast<float*>(ckpt)};
-  a.S0 = S0;
+  const SegPlan sp = ffma_plan(B, H, T);
+  a.S0 = S0;  // [B*H][1][dout][din]: the one segment's start state
+  if (sp.nseg > 1) {
+    const SegBufs sb = seg_bufs(seg_ws, B, H, din, dout, sp.nseg);
+    ffma::FwdArgs sum = a;  // each segment's local state and log-decay, from zero
+    sum.y = nullptr;
+    sum.ckpt = nullptr;
+    sum.S0 = nullptr;
+    sum.nseg = sp.nseg;
+    sum.seg_chunks = sp.seg_chunks;
+    sum.summary = 1;
+    sum.Sloc = sb.loc;
+    sum.segL = sb.L;
+    if (ffma::launch_fwd(sum, dt == GRADLEV_BF16, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
+    // the first segment starts from the carried state S0
+    if (tc::combine_segments(sb.loc, sb.L, S0, sb.comb, B * H, sp.nseg, dout * din, 0, st) !=
+        cudaSuccess)
+      return GRADLEV_ERR_CUDA;
+    a.nseg = sp.nseg;
+    a.seg_chunks = sp.seg_chunks;
+    a.S0 = sb.comb;
+  }
   a.ST = ST;
   return ffma::launch_fwd(a, dt == GRADLEV_BF16, st) == cudaSuccess ? GRADLEV_OK
                                                                    : GRADLEV_ERR_CUDA;
@@ -233,7 +263,29 @@ gradlev_status bwd_run(int B, int H, int T, int din, int dout, gradlev_dtype dt,
   }
   ffma::BwdArgs a{B, H, T, din, dout, x, g, eta, alpha, W0, dy, dx, dg, d_eta, d_alpha, dW0,
                   static_cast<const float*>(states), dW0_part};
-  a.LamT = io.LamT;
+  const SegPlan sp = ffma_plan(B, H, T);
+  a.LamT = io.LamT;  // one segment: it ends where the adjoint flows in
+  if (sp.nseg > 1) {
+    // each segment's local adjoint (walked backwards from zero) and log-decay, then the
+    // adjoint at each segment's end
+    const SegBufs sb = seg_bufs(seg_ws, B, H, din, dout, sp.nseg);
+    ffma::BwdArgs sum = a;
+    sum.LamT = nullptr;
+    sum.dS0 = nullptr;
+    sum.nseg = sp.nseg;
+    sum.seg_chunks = sp.seg_chunks;
+    sum.summary = 1;
+    sum.Lloc = sb.loc;
+    sum.segL = sb.L;
+    if (ffma::launch_bwd(sum, dt == GRADLEV_BF16, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
+    // the last segment ends where the adjoint LamT flows in
+    if (tc::combine_segments(sb.loc, sb.L, io.LamT, sb.comb, B * H, sp.nseg, dout * din, 1,
+                             st) != cudaSuccess)
+      return GRADLEV_ERR_CUDA;
+    a.nseg = sp.nseg;
+    a.seg_chunks = sp.seg_chunks;
+    a.LamT = sb.comb;
+  }
   a.dS0 = io.dS0;
   return ffma::launch_bwd(a, dt == GRADLEV_BF16, st) == cudaSuccess ? GRADLEV_OK
                                                                    : GRADLEV_ERR_CUDA;

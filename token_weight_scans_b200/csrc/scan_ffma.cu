@@ -32,7 +32,7 @@
 namespace gradlev {
 namespace ffma {
 
-constexpr int FC = 32;    // tokens per chunk
+constexpr int FC = kChunk;  // tokens per chunk
 constexpr int FT = 256;   // threads per CTA
 constexpr int LDD = FC + 2;  // row stride of the decay table
 constexpr int LDC = FC + 1;  // row stride of FC x FC tables
@@ -97,23 +97,27 @@ __global__ void __launch_bounds__(FT, 1) fwd_kernel(FwdArgs a) {
   float* et = Dt + (FC + 1) * LDD;
   float* al = et + FC;
 
-  const int bh = blockIdx.x, h = bh % a.H;
+  // one CTA per (scan, segment); the segment walks chunks [c0, c1)
+  const int bh = blockIdx.x / a.nseg, seg = blockIdx.x - bh * a.nseg, h = bh % a.H;
   const size_t tok0 = (size_t)bh * a.T;
-  const int nch = (a.T + FC - 1) / FC;
+  const int nch = (a.T + FC - 1) / FC;  // chunks of the whole scan (checkpoint indexing)
+  const int c0 = seg * a.seg_chunks, c1 = min(nch, c0 + a.seg_chunks);
+  const size_t seg_row = (size_t)bh * a.nseg + seg;
   const Tio* xg = static_cast<const Tio*>(a.x);
   const Tio* gg = static_cast<const Tio*>(a.g);
   Tio* yg = static_cast<Tio*>(a.y);
   const float* W0 = a.W0 + (size_t)h * dout * din;
 
-  const float* S0 = a.S0 ? a.S0 + (size_t)bh * dout * din : nullptr;
+  const float* S0 = a.S0 ? a.S0 + seg_row * dout * din : nullptr;
   for (int e = tid; e < dout * din; e += FT) {
     const int n = e / din, k = e - n * din;
     S[n * LDI + k] = S0 ? S0[e] : 0.f;
     W[n * LDI + k] = W0[e];
   }
   const int NG = dout / 4, NK4 = din / 4, NB = dout / 8;
+  float lseg = 0.f;  // log2 of the product of alpha over the walked chunks (summary)
 
-  for (int c = 0; c < nch; ++c) {
+  for (int c = c0; c < c1; ++c) {
     const int t0 = c * FC;
     const int nt = min(FC, a.T - t0);
     __syncthreads();
@@ -200,6 +204,7 @@ __global__ void __launch_bounds__(FT, 1) fwd_kernel(FwdArgs a) {
 
     // carry: S <- D[FC][-1] S + sum_j (-eta_j D[FC][j]) g_j x_j^T
     const float gC = Dt[FC * LDD];
+    lseg += log2f(gC);
     for (int item = tid; item < NB * NK4; item += FT) {
       const int nb = item / NK4, k4 = item - nb * NK4;
       float4 acc[8];
@@ -218,7 +223,16 @@ __global__ void __launch_bounds__(FT, 1) fwd_kernel(FwdArgs a) {
       for (int r = 0; r < 8; ++r) *reinterpret_cast<float4*>(&S[(nb * 8 + r) * LDI + 4 * k4]) = acc[r];
     }
   }
-  if (a.ST) {  // the state after the last token (padded tokens left it unchanged)
+  if (a.summary) {  // this segment's local end state and log-decay
+    __syncthreads();
+    float* dst = a.Sloc + seg_row * dout * din;
+    for (int e = tid; e < dout * din; e += FT) {
+      const int n = e / din, k = e - n * din;
+      dst[e] = S[n * LDI + k];
+    }
+    if (tid == 0) a.segL[seg_row] = lseg;
+  }
+  if (a.ST && seg == a.nseg - 1) {  // the state after the last token (padded tokens left it unchanged)
     __syncthreads();
     float* dst = a.ST + (size_t)bh * dout * din;
     for (int e = tid; e < dout * din; e += FT) {
@@ -266,9 +280,13 @@ __global__ void __launch_bounds__(FT, 1) bwd_kernel(BwdArgs a) {
   float* pv = qv + FC;              // [FC]
   float* Esh = pv + FC;             // [1]
 
-  const int bh = blockIdx.x, h = bh % a.H;
+  // one CTA per (scan, segment); the segment walks chunks c1 - 1 down to c0
+  const int bh = blockIdx.x / a.nseg, seg = blockIdx.x - bh * a.nseg, h = bh % a.H;
   const size_t tok0 = (size_t)bh * a.T;
-  const int nch = (a.T + FC - 1) / FC;
+  const int nch = (a.T + FC - 1) / FC;  // chunks of the whole scan (checkpoint indexing)
+  const int c0 = seg * a.seg_chunks, c1 = min(nch, c0 + a.seg_chunks);
+  const size_t seg_row = (size_t)bh * a.nseg + seg;
+  const bool full = !a.summary;  // outputs, not just the adjoint carry
   const Tio* xg = static_cast<const Tio*>(a.x);
   const Tio* gg = static_cast<const Tio*>(a.g);
   const Tio* ug = static_cast<const Tio*>(a.dy);
@@ -276,7 +294,7 @@ __global__ void __launch_bounds__(FT, 1) bwd_kernel(BwdArgs a) {
   Tio* dgg = static_cast<Tio*>(a.dg);
   const float* W0 = a.W0 + (size_t)h * dout * din;
 
-  const float* LamT = a.LamT ? a.LamT + (size_t)bh * dout * din : nullptr;
+  const float* LamT = a.LamT ? a.LamT + seg_row * dout * din : nullptr;
   for (int e = tid; e < dout * din; e += FT) {
     const int n = e / din, k = e - n * din;
     L[n * LDI + k] = LamT ? LamT[e] : 0.f;
@@ -287,14 +305,15 @@ __global__ void __launch_bounds__(FT, 1) bwd_kernel(BwdArgs a) {
 #pragma unroll
     for (int r = 0; r < 8; ++r) dw[it][r] = make_float4(0.f, 0.f, 0.f, 0.f);
 
-  for (int c = nch - 1; c >= 0; --c) {
+  float lseg = 0.f;  // log2 of the product of alpha over the walked chunks (summary)
+  for (int c = c1 - 1; c >= c0; --c) {
     const int t0 = c * FC;
     const int nt = min(FC, a.T - t0);
     __syncthreads();
     load_rows(X, LDI, xg + (tok0 + t0) * din, FC, nt, din, tid);
-    load_rows(G, LDO, gg + (tok0 + t0) * dout, FC, nt, dout, tid);
     load_rows(U, LDO, ug + (tok0 + t0) * dout, FC, nt, dout, tid);
-    {
+    if (full) {
+      load_rows(G, LDO, gg + (tok0 + t0) * dout, FC, nt, dout, tid);
       const float* src = a.ckpt + ((size_t)bh * nch + c) * dout * din;
       for (int e = tid; e < dout * din; e += FT) {
         const int n = e / din, k = e - n * din;
@@ -307,6 +326,7 @@ __global__ void __launch_bounds__(FT, 1) bwd_kernel(BwdArgs a) {
     }
     __syncthreads();
     decay_table(Dt, al, tid);
+    if (full) {
     // Gram matrices of the chunk
     for (int e = tid; e < 2 * FC * FC; e += FT) {
       const int which = e / (FC * FC), ij = e - which * FC * FC;
@@ -487,8 +507,12 @@ __global__ void __launch_bounds__(FT, 1) bwd_kernel(BwdArgs a) {
       const float h = gam * dl * Esh[0] + dl * t2 + gam * t3 + t4;
       if (i < nt) a.d_alpha[tok0 + t0 + i] = h;
     }
+    } else {
+      __syncthreads();  // the decay table is complete
+    }
     // Lam <- D[FC][-1] Lam + sum_s D[s][-1] u_s x_s^T ; dW0 += sum_s u_s x_s^T
     const float gC = Dt[FC * LDD];
+    lseg += log2f(gC);
 #pragma unroll
     for (int it = 0; it < 2; ++it) {
       const int item = tid + it * FT;
@@ -507,7 +531,7 @@ __global__ void __launch_bounds__(FT, 1) bwd_kernel(BwdArgs a) {
           for (int r = 0; r < 8; ++r) {
             const float uv = U[s * LDO + nb * 8 + r];
             fma4(acc[r], gs * uv, xv);
-            fma4(dw[it][r], uv, xv);
+            if (full) fma4(dw[it][r], uv, xv);
           }
         }
 #pragma unroll
@@ -515,7 +539,17 @@ __global__ void __launch_bounds__(FT, 1) bwd_kernel(BwdArgs a) {
       }
     }
   }
-  if (a.dS0) {  // the adjoint at the first token
+  if (!full) {  // this segment's local adjoint and log-decay
+    __syncthreads();
+    float* dl = a.Lloc + seg_row * dout * din;
+    for (int e = tid; e < dout * din; e += FT) {
+      const int n = e / din, k = e - n * din;
+      dl[e] = L[n * LDI + k];
+    }
+    if (tid == 0) a.segL[seg_row] = lseg;
+    return;
+  }
+  if (a.dS0 && seg == 0) {  // the adjoint at the first token
     __syncthreads();
     float* ds = a.dS0 + (size_t)bh * dout * din;
     for (int e = tid; e < dout * din; e += FT) {
@@ -523,8 +557,9 @@ __global__ void __launch_bounds__(FT, 1) bwd_kernel(BwdArgs a) {
       ds[e] = L[n * LDI + k];
     }
   }
-  // this pair's dW0 partial
-  float* dst = a.dW0_part + (size_t)bh * dout * din;
+  // this (scan, segment)'s dW0 partial: [b][seg][h], summed over b and seg in a fixed order
+  const int bb = bh / a.H;
+  float* dst = a.dW0_part + (((size_t)bb * a.nseg + seg) * a.H + h) * dout * din;
 #pragma unroll
   for (int it = 0; it < 2; ++it) {
     const int item = tid + it * FT;
@@ -555,7 +590,7 @@ static cudaError_t launch_fwd_t(const FwdArgs& a, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(fwd_kernel<Tio>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  fwd_kernel<Tio><<<a.B * a.H, FT, smem, st>>>(a);
+  fwd_kernel<Tio><<<a.B * a.H * a.nseg, FT, smem, st>>>(a);
   count_launch();
   return cudaGetLastError();
 }
@@ -566,14 +601,14 @@ static cudaError_t launch_bwd_t(const BwdArgs& a, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(bwd_kernel<Tio>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  bwd_kernel<Tio><<<a.B * a.H, FT, smem, st>>>(a);
+  bwd_kernel<Tio><<<a.B * a.H * a.nseg, FT, smem, st>>>(a);
   count_launch();
   e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess || a.summary) return e;
   const int dd = a.din * a.dout;
   const size_t n = (size_t)a.H * dd;
   const int blocks = (int)((n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184);
-  reduce_dW0_kernel<<<blocks, 256, 0, st>>>(a.dW0_part, a.dW0, a.B, a.H, dd);
+  reduce_dW0_kernel<<<blocks, 256, 0, st>>>(a.dW0_part, a.dW0, a.B * a.nseg, a.H, dd);
   count_launch();
   return cudaGetLastError();
 }
