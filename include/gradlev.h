@@ -381,6 +381,18 @@ GRADLEV_API int gradlev_last_launch_count(void);
  * Host-global, one-shot, not thread-safe; for tests only. */
 GRADLEV_API void gradlev_debug_inject_timeout(int site, int timeout_ms);
 
+/* Test hook for the segment-summary passes of the bf16 tensor-core path (few
+ * long scans, cut into segments). Those passes carry only the state or the
+ * adjoint across each segment; they keep the decay accumulated since the last
+ * rescale as a scale factor 2^E outside tensor memory (folded into the
+ * scaled inputs of each update) and rescale the stored matrix in place once E
+ * would fall below -log2_bound. The default bound is 64. A smaller bound in
+ * [0, 126] makes the in-place rescale run more often (0: at every chunk that
+ * decays), so that tests can reach it on short inputs; a negative or NaN value
+ * restores the default, and values above 126 are clamped to 126. Results agree
+ * for every bound up to rounding. Host-global, not thread-safe; for tests only. */
+GRADLEV_API void gradlev_debug_summary_rescale(float log2_bound);
+
 #ifdef __cplusplus
 }
 #endif

@@ -112,13 +112,22 @@ def _gpu(d):
     return {k: to_numpy(v) for k, v in out.items()}
 
 
-@pytest.mark.parametrize("shape", [(8, 16, 200), (1, 2, 400)],
-                         ids=["one-CTA-per-scan", "segmented"])
-def test_decay_path_bit_exact(shape):
+@pytest.mark.parametrize("shape,bound", [((8, 16, 200), -1.0), ((1, 2, 400), -1.0),
+                                         ((1, 2, 400), 0.0)],
+                         ids=["one-CTA-per-scan", "segmented", "segmented-rescale-every-chunk"])
+def test_decay_path_bit_exact(shape, bound):
+    """bound: that of the summary passes' deferred decay (-1: the default; 0: the carried
+    matrix is rescaled in place at every chunk that decays). The scales are powers of two
+    here, so the result is bit-exact either way."""
+    import token_weight_scans_b200 as tw
     B, H, T = shape
     d, ref = _find(B, H, T, p_half=1 / 64, seed0=1000 + T)
     assert np.any(d["alpha"] == 0.5)
-    got = _gpu(d)
+    tw.lib().gradlev_debug_summary_rescale(bound)
+    try:
+        got = _gpu(d)
+    finally:
+        tw.lib().gradlev_debug_summary_rescale(-1.0)
     for k in ("y",) + OUTS:
         assert np.array_equal(got[k], ref[k]), (k, rel_err(got[k], ref[k]))
     # the decays are exercised: some outputs differ from the alpha = 1 problem

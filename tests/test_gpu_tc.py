@@ -12,7 +12,7 @@ import pytest
 
 import oracle
 from token_weight_scans_b200 import inputs
-from tests.helpers import TOL, rel_err, to_device, to_numpy
+from tests.helpers import TOL, heads_slice, rel_err, to_device, to_numpy
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -215,6 +215,38 @@ def test_tc_segmented_scan_matches_unsegmented():
     assert rel_err(a["dW0"], b["dW0"][:1]) <= 1e-2
     ref = oracle_fwd_bwd(lone)
     check_all(a, ref, "segmented lone scan")
+
+
+@pytest.fixture
+def summary_rescale():
+    """Sets the bound of the summary passes' deferred decay; restores the default after."""
+    import token_weight_scans_b200 as tw
+    yield tw.lib().gradlev_debug_summary_rescale
+    tw.lib().gradlev_debug_summary_rescale(-1.0)
+
+
+@pytest.mark.parametrize("bound", [64.0, 4.0, 0.0],
+                         ids=["default", "every-few-chunks", "every-chunk"])
+def test_tc_segment_summary_deferred_decay(bound, summary_rescale):
+    """The summary passes keep the decay since the last in-place rescale of the carried
+    matrix as a scale 2^E outside tensor memory and rescale the matrix once E would drop
+    below -bound. Sixteen scans of 72 chunks are cut into 9 segments of 8 chunks; the
+    same scans run unsegmented as heads of a batch of 80 (no summary pass). With these
+    gates (about -1.3 of log2 decay per chunk) the rescale never runs at the default
+    bound, every few chunks at 4 and at every chunk at 0; the results agree with the
+    unsegmented run and with the oracle whatever the bound."""
+    summary_rescale(bound)
+    H, T = 80, 72 * 64
+    big = inputs.draw(1, H, T, 128, 128, dtype="bf16", alpha_mode="log_uniform", seed=62)
+    lone = {k: (v[:16] if k == "W0" else v[:, :16]) for k, v in big.items()}
+    a = gpu_fwd_bwd(lone)
+    b = gpu_fwd_bwd(big)
+    for k in ("y", "dx", "dg", "deta", "dalpha"):
+        err = rel_err(a[k], b[k][:, :16])
+        assert err <= 1e-2, (k, err)
+    assert rel_err(a["dW0"], b["dW0"][:16]) <= 1e-2
+    got = {k: (a[k][5:6] if k == "dW0" else a[k][:, 5:6]) for k in ("y",) + BWD_OUTS}
+    check_all(got, oracle_fwd_bwd(heads_slice(lone, 0, 5)), f"segmented, bound {bound}")
 
 
 # ------------------------------------------------------------------ bounded-wait failure path

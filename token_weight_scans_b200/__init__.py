@@ -90,6 +90,10 @@ def lib():
     L.gradlev_device_status.restype = I
     L.gradlev_last_launch_count.argtypes = []
     L.gradlev_last_launch_count.restype = I
+    L.gradlev_debug_inject_timeout.argtypes = [I, I]
+    L.gradlev_debug_inject_timeout.restype = None
+    L.gradlev_debug_summary_rescale.argtypes = [ctypes.c_float]
+    L.gradlev_debug_summary_rescale.restype = None
     _lib = L
     return L
 

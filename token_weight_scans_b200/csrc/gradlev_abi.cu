@@ -35,6 +35,8 @@ void reset_launch_count() { t_launches = 0; }
 enum InjectSite { INJ_NONE = 0, INJ_FWD = 1, INJ_BWD = 2, INJ_FWD_SUMMARY = 3, INJ_BWD_SUMMARY = 4 };
 static int g_inject = INJ_NONE;
 static uint64_t g_inject_timeout_ns = 0;
+// Test hook state (gradlev_debug_summary_rescale): bound of the summary passes' deferred decay
+static float g_rescale_log2 = tc::kSummaryRescaleLog2;
 
 // The kernel's inject code and wait bound for a launch at `site` (one-shot).
 static int take_inject(int site, int code, uint64_t* timeout_ns) {
@@ -161,6 +163,7 @@ static gradlev_status launch_fwd_impl(int B, int H, int T, int din, int dout, gr
       sum.S_final = sb.loc;
       sum.seg_L = sb.L;
       sum.summary = 1;
+      sum.rescale_log2 = g_rescale_log2;
       if (tc::launch_fwd(sum, x, g, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
       // the first segment starts from the carried state S0
       if (tc::combine_segments(sb.loc, sb.L, S0, sb.comb, B * H, sp.nseg, dout * din, 0, st) !=
@@ -237,6 +240,7 @@ gradlev_status bwd_run(int B, int H, int T, int din, int dout, gradlev_dtype dt,
       sum.seg_L = sb.L;
       sum.summary = 1;
       sum.reverse = 1;
+      sum.rescale_log2 = g_rescale_log2;
       if (tc::launch_fwd(sum, x, dy, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
       // the last segment ends where the adjoint LamT flows in
       if (tc::combine_segments(sb.loc, sb.L, io.LamT, sb.comb, B * H, sp.nseg, dout * din, 1,
@@ -612,6 +616,10 @@ int gradlev_last_launch_count(void) { return t_launches; }
 void gradlev_debug_inject_timeout(int site, int timeout_ms) {
   g_inject = (site >= INJ_FWD && site <= INJ_BWD_SUMMARY) ? site : INJ_NONE;
   g_inject_timeout_ns = (uint64_t)(timeout_ms > 0 ? timeout_ms : 1) * 1000000ull;
+}
+
+void gradlev_debug_summary_rescale(float log2_bound) {
+  g_rescale_log2 = !(log2_bound >= 0.f) ? tc::kSummaryRescaleLog2 : fminf(log2_bound, 126.f);
 }
 
 }  // extern "C"

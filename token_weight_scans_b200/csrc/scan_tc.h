@@ -18,6 +18,8 @@ namespace tc {
 // reverse = 1 walks the segment backwards and weights row j of the G-operand by
 // 2^{L_{j-1}} instead of -eta_j 2^{L_{C-1}-L_j}: with dy in place of g, that is the
 // adjoint recursion Lam <- 2^{L_{C-1}} Lam + sum_j 2^{L_{j-1}} u_j x_j^T.
+constexpr float kSummaryRescaleLog2 = 64.f;  // default bound of the summary passes' deferred decay
+
 struct TcFwdParams {
   int B, H, T, din, dout;   // din == 128, dout % 128 == 0
   const float* eta;         // [B,H,T]
@@ -38,6 +40,9 @@ struct TcFwdParams {
   int reverse = 0;          // 1: adjoint summary (see above)
   float* S_last = nullptr;  // [B*H][dout][din] the state after the scan's last token, or null
                             // (written by the last segment's CTAs; not in summary mode)
+  // summary mode: the decay since the last in-place rescale of the state is kept as a
+  // scale 2^E, and the state is rescaled once E would drop below -rescale_log2 (0..126)
+  float rescale_log2 = kSummaryRescaleLog2;
 };
 
 // The reverse scan of one 128-row slice [n0, n0+128) of d_out: the rows of the

@@ -39,6 +39,17 @@
 // X W0^T and X S^T. P G accumulates onto X W0^T, so warp 1 waits for warp 2's
 // commit of that product first. Y is complete when both have committed, a
 // stage is free when both have read it.
+//
+// The state carry alone (the segment summary passes: FULL = false) has no output
+// and no bf16 copy of the state, so it keeps the decay out of the state chain:
+// TMEM holds A with S = 2^E A, where E is the log2 decay since the last in-place
+// rescale, and the gate warp folds 2^{-E_{c+1}} into the weights of the scaled X,
+// so the update of chunk c adds G^T (2^{-E_{c+1}} Xhat) onto A without waiting for
+// the state warps. Only when E would drop below -rescale_log2 (64 by default) do
+// the state warps rescale A in place (by 2^{E_c + L_{C-1}}, after which E = 0),
+// and the final state is 2^E A. Every scaled weight stays below eta 2^64, far inside
+// the bf16 and fp32 ranges. Without the bf16 state tile and W0, that shared memory
+// holds two more TMA stages.
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -60,6 +71,7 @@ namespace {
 
 constexpr int C = 64;          // tokens per chunk
 constexpr int NS = 3;          // TMA stages (X and G tiles)
+constexpr int NS_SUM = 5;      // stages of the state carry alone: the W0 and S tiles hold two more
 constexpr int GS = 4;          // gate slots
 constexpr int NTHREADS = 640;  // 20 warps
 constexpr int TILE = C * 128;  // bytes of one [64 rows x 128 B] swizzled block
@@ -86,7 +98,11 @@ struct GateSlot {
   float ca[C];    // -eta_j 2^{M - L_j}
   float gC;       // 2^{L_{C-1}}
   int fac;
-  float pad[2];
+  // state carry alone: w and gam above already carry the factor 2^{-E_{c+1}}
+  float rs;       // rescale of A before this chunk's update (when renorm)
+  float Eout;     // E after this chunk
+  int renorm;
+  float pad[3];
 };
 
 struct Smem {
@@ -99,7 +115,7 @@ struct Smem {
   uint8_t P[TILE];             // 64 token rows (i) x 128 B (j)
   uint8_t Ys[2 * TILE];        // y staging: n-blocks of 64 token rows x 128 B (TMA store)
   GateSlot gates[GS];
-  uint64_t full[NS], empty[NS];
+  uint64_t full[NS_SUM], empty[NS_SUM];
   uint64_t gfull[GS], gempty[GS];
   uint64_t kfull[2], kfree[2];
   uint64_t xhready[2], xhfree[2];  // per scaled-X buffer
@@ -118,15 +134,25 @@ static_assert(kSmemBytes <= 227 * 1024, "over the 227 KB of shared memory a CTA 
 enum : uint32_t {
   W_TMA_EMPTY = 0x001, W_TMA_DRAIN = 0x002,
   W_MMA_FULL = 0x101, W_MMA_KFREE, W_MMA_YFREE, W_MMA_XREADY, W_MMA_SSCALED, W_MMA_PREADY,
-  W_MMA_SREADY, W_MMA_DONE, W_MMA_Y1FULL,
+  W_MMA_SREADY, W_MMA_DONE, W_MMA_Y1FULL, W_MMA_GFULL,
   W_GATE_EMPTY = 0x201,
   W_XH_FULL = 0x301, W_XH_GFULL, W_XH_FREE,
   W_M_GFULL = 0x401, W_M_KFULL, W_M_YFULL,
-  W_S_GFULL = 0x501, W_S_DSFULL, W_S_SFREE,
+  W_S_GFULL = 0x501, W_S_DSFULL, W_S_SFREE, W_S_UPD,
 };
+
+// X and G tiles of stage s; stages NS.. (state carry alone) use the W0 and S tiles
+__device__ __forceinline__ uint8_t* stage_x(Smem& sm, int s) {
+  return s < NS ? sm.X[s] : (s == NS ? sm.W0[0] : sm.S[0]);
+}
+__device__ __forceinline__ uint8_t* stage_g(Smem& sm, int s) {
+  return s < NS ? sm.G[s] : (s == NS ? sm.W0[1] : sm.S[1]);
+}
 
 }  // namespace
 
+// FULL: outputs (y, checkpoints); otherwise the state carry alone (summary passes).
+template <bool FULL>
 __global__ void __launch_bounds__(NTHREADS, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmG,
                const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmS,
@@ -149,18 +175,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   auto cg = [&](int c) { return p.reverse ? c1 - 1 - c : c0 + c; };
   const size_t seg_row = (size_t)bh * p.nseg + seg;  // [bh][seg] index of the segment states
   const WaitCtx wc{&sm.abort, p.status, p.timeout_ns};
-  const bool full = !p.summary;  // outputs, not just the state carry
+  constexpr bool full = FULL;
+  constexpr int ns = FULL ? NS : NS_SUM;  // TMA stages
 
   if (threadIdx.x == 0) {
     sm.abort = 0;
-    for (int s = 0; s < NS; ++s) {
+    for (int s = 0; s < ns; ++s) {
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], full ? 2 : 1);  // the issuers that read the stage
     }
     for (int g = 0; g < GS; ++g) {
       mbar_init(&sm.gfull[g], 32);
-      // 8 state warps (+ 8 output warps when there are outputs)
-      mbar_init(&sm.gempty[g], full ? 16 : 8);
+      // 8 state warps + 8 output warps, or 8 state warps + the update's issuer
+      mbar_init(&sm.gempty[g], full ? 16 : 9);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.kfull[b], 1);
@@ -215,19 +242,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     int issued = 0;
     if (lane == 0) {
       for (int c = 0; c < nch; ++c) {
-        const int s = c % NS;
-        if (!mbar_wait(&sm.empty[s], ((c / NS) & 1) ^ 1, wc, W_TMA_EMPTY)) break;
+        const int s = c % ns;
+        if (!mbar_wait(&sm.empty[s], ((c / ns) & 1) ^ 1, wc, W_TMA_EMPTY)) break;
         mbar_arrive_expect_tx(&sm.full[s], 4 * TILE);
         const int t0 = cg(c) * C;
-        tma_load_3d(sm.X[s], &tmX, &sm.full[s], 0, t0, bh);
-        tma_load_3d(sm.X[s] + TILE, &tmX, &sm.full[s], 64, t0, bh);
-        tma_load_3d(sm.G[s], &tmG, &sm.full[s], n0, t0, bh);
-        tma_load_3d(sm.G[s] + TILE, &tmG, &sm.full[s], n0 + 64, t0, bh);
+        uint8_t* sx = stage_x(sm, s);
+        uint8_t* sg = stage_g(sm, s);
+        tma_load_3d(sx, &tmX, &sm.full[s], 0, t0, bh);
+        tma_load_3d(sx + TILE, &tmX, &sm.full[s], 64, t0, bh);
+        tma_load_3d(sg, &tmG, &sm.full[s], n0, t0, bh);
+        tma_load_3d(sg + TILE, &tmG, &sm.full[s], n0 + 64, t0, bh);
         issued = c + 1;
       }
       // teardown: let every load this thread issued land before the CTA exits
-      for (int c = issued > NS ? issued - NS : 0; c < issued; ++c)
-        mbar_drain(&sm.full[c % NS], (c / NS) & 1, wc, W_TMA_DRAIN);
+      for (int c = issued > ns ? issued - ns : 0; c < issued; ++c)
+        mbar_drain(&sm.full[c % ns], (c / ns) & 1, wc, W_TMA_DRAIN);
     }
   } else if (warp == 1 || warp == 2) {
     // ------------------------------------------------------------ MMA issuers
@@ -239,12 +268,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint32_t id_pg = idesc_bf16(64, 128, false, true);   // P G (G n-contiguous)
       const uint32_t id_ds = idesc_bf16(128, 128, true, true);   // G^T Xhat
       const uint32_t sW0 = smem_u32(sm.W0[0]), sP = smem_u32(sm.P);
+      int nrn = 0;  // rescaled chunks so far (state carry alone)
       for (int c = 0; c < nch; ++c) {
-        const int s = c % NS, b = c & 1;
-        const uint32_t sX = smem_u32(sm.X[s]), sG = smem_u32(sm.G[s]);
+        const int s = c % ns, b = c & 1;
+        const uint32_t sX = smem_u32(stage_x(sm, s)), sG = smem_u32(stage_g(sm, s));
         const uint32_t sXh = smem_u32(sm.Xh[b]), sS = smem_u32(sm.S[0]);
         const uint32_t tY1 = tbase + COL_Y + 128 * b, tY2 = tY1 + LANE16;
-        if (!mbar_wait(&sm.full[s], (c / NS) & 1, wc, W_MMA_FULL)) break;
+        if (!mbar_wait(&sm.full[s], (c / ns) & 1, wc, W_MMA_FULL)) break;
         if (ii == 0) {
           if (full) {
             // K = X X^T into buffer b (the mask of chunk c - 2 has read it)
@@ -258,16 +288,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             if (!(p.inject == 1 && c == 1)) umma_commit(&sm.kfull[b]);
           }
-          // S += G^T Xhat onto the state that the state warps have scaled in place
+          // S += G^T Xhat onto the state that the state warps have scaled in place. The
+          // state carry alone waits for them only on the chunks where they rescale A.
+          bool wait_scaled = true;
+          if (!full) {
+            const int g = c % GS;
+            if (!mbar_wait(&sm.gfull[g], (c / GS) & 1, wc, W_MMA_GFULL)) break;
+            wait_scaled = *reinterpret_cast<volatile int*>(&sm.gates[g].renorm) != 0;
+            mbar_arrive(&sm.gempty[g]);
+          }
           if (!mbar_wait(&sm.xhready[b], (c >> 1) & 1, wc, W_MMA_XREADY)) break;
-          if (!mbar_wait(&sm.sscaled, c & 1, wc, W_MMA_SSCALED)) break;
+          if (wait_scaled && !mbar_wait(&sm.sscaled, (full ? c : nrn) & 1, wc, W_MMA_SSCALED)) break;
+          nrn += wait_scaled ? 1 : 0;
           tc_fence_after();
           #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             umma_bf16(tbase + COL_S, desc_at(sw128_desc(sG, TILE, 1024), kk * 2048),
                       desc_at(sw128_desc(sXh, TILE, 1024), kk * 2048), id_ds, 1);
-          if (!(p.inject == 3 && c == 1)) umma_commit(&sm.dsfull);
-          umma_commit(&sm.xhfree[b]);
+          umma_commit(&sm.dsfull);
+          if (!(p.inject == 3 && c == 1)) umma_commit(&sm.xhfree[b]);
           if (!full) {  // state carry only: the stage is free once the update has read it
             umma_commit(&sm.empty[s]);
             continue;
@@ -324,6 +363,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     constexpr bool gate_warp = true;
     float ra[PD][2], re[PD][2];
     float Lseg = 0.f;  // sum of log2 alpha over the walked chunks (lane-uniform)
+    float Erun = 0.f;  // state carry alone: log2 of the deferred scale, S = 2^E A (lane-uniform)
     // gates of the c-th walked chunk (alpha = 1, eta = 0 past the walk or past T)
     auto gate_load = [&](int c, float (&a)[2], float (&e)[2]) {
       const bool in = c < nch;
@@ -365,14 +405,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           Lseg += Lend;
           const float pm0 = __shfl_up_sync(0xffffffffu, l0, 1);
           const float pm1 = __shfl_up_sync(0xffffffffu, l1, 1);
+          // state carry alone: E_{c+1} = E_c + L_{C-1} unless that falls below -kDeferLog2,
+          // in which case A is rescaled by 2^{E_c + L_{C-1}} and E restarts at 0
+          const float Enext = Erun + Lend;
+          const bool rn = !full && Enext < -p.rescale_log2;
+          const float m = (full || rn) ? 1.f : exp2f(-Enext);
           gs.L[lane] = l0;
           gs.L[lane + 32] = l1;
           gs.eta[lane] = e0;
           gs.eta[lane + 32] = e1;
-          gs.gam[lane] = lane == 0 ? 1.f : exp2f(pm0);
-          gs.gam[lane + 32] = exp2f(lane == 0 ? last0 : pm1);
-          gs.w[lane] = -e0 * exp2f(Lend - l0);
-          gs.w[lane + 32] = -e1 * exp2f(Lend - l1);
+          gs.gam[lane] = m * (lane == 0 ? 1.f : exp2f(pm0));
+          gs.gam[lane + 32] = m * exp2f(lane == 0 ? last0 : pm1);
+          gs.w[lane] = m * (-e0 * exp2f(Lend - l0));
+          gs.w[lane + 32] = m * (-e1 * exp2f(Lend - l1));
           gs.ra[lane] = exp2f((lane == 0 ? 0.f : pm0) - last0);
           gs.ra[lane + 32] = exp2f((lane == 0 ? last0 : pm1) - last0);
           gs.ca[lane] = -e0 * exp2f(last0 - l0);
@@ -380,7 +425,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (lane == 0) {
             gs.gC = exp2f(Lend);
             gs.fac = (Lend >= -120.f) ? 1 : 0;
+            gs.rs = exp2f(Enext);
+            gs.renorm = rn ? 1 : 0;
+            gs.Eout = rn ? 0.f : Enext;
           }
+          Erun = rn ? 0.f : Enext;
           __syncwarp();
           mbar_arrive(&sm.gfull[g]);
         }
@@ -418,6 +467,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tmem_st32(tS + 32 * hf, v);
       }
       tmem_st_wait();
+      tc_fence_before();  // the state carry alone: the first update may follow xhready alone
     }
     // Each warp TMA-stores what it wrote itself: its 32 rows of one k-block of the
     // bf16 chunk-start state (bf16 [bh][chunk][dout][din], box of 32 rows). The tile is
@@ -428,12 +478,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // 16-byte pieces. Written a chunk ahead, into the buffer the update of chunk c - 2 read.
     const int st = threadIdx.x - 128;  // 0..255 over the state warps
     auto scaled_x = [&](int c) -> bool {
-      const int s = c % NS, g = c % GS, b = c & 1;
-      if (!mbar_wait_warp(&sm.full[s], (c / NS) & 1, wc, W_XH_FULL)) return false;
+      const int s = c % ns, g = c % GS, b = c & 1;
+      if (!mbar_wait_warp(&sm.full[s], (c / ns) & 1, wc, W_XH_FULL)) return false;
       if (!mbar_wait_warp(&sm.gfull[g], (c / GS) & 1, wc, W_XH_GFULL)) return false;
       if (!mbar_wait_warp(&sm.xhfree[b], ((c >> 1) & 1) ^ 1, wc, W_XH_FREE)) return false;
       const GateSlot& gs = sm.gates[g];
-      const uint32_t src = smem_u32(sm.X[s]), dst = smem_u32(sm.Xh[b]);
+      const uint32_t src = smem_u32(stage_x(sm, s)), dst = smem_u32(sm.Xh[b]);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const uint32_t off = (uint32_t)(st + 256 * k) * 16;
@@ -449,79 +499,132 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (lane == 0) mbar_arrive(&sm.xhready[b]);
       return true;
     };
-    bool ok = nch > 0 ? scaled_x(0) : true;
-    for (int c = 0; c < nch && ok; ++c) {
-      const int g = c % GS;
-      const GateSlot& gs = sm.gates[g];
-      ok = ok && mbar_wait_warp(&sm.gfull[g], (c / GS) & 1, wc, W_S_GFULL);
-      // S_c is complete: the update of chunk c - 1 has accumulated onto it
-      ok = ok && (c == 0 || mbar_wait_warp(&sm.dsfull, (c - 1) & 1, wc, W_S_DSFULL));
-      // the bf16 state tile was last read by the S X^T product and the checkpoint store
-      // of chunk c - 1
-      ok = ok && (!full || c < 1 || mbar_wait_warp(&sm.sfree, (c - 1) & 1, wc, W_S_SFREE));
-      if (lane == 0 && has_ck) tma_store_wait_read_n<0>();
-      __syncwarp();
-      if (!ok) break;
-      tc_fence_after();
-      // S_c -> bf16 (kept packed), S <- 2^{L_{C-1}} S in place; the update of chunk c
-      // may then accumulate, and the bf16 copy goes to buffer b (outputs only)
-      const float gC = gs.gC;
-      uint32_t pk[32];
+    if (!full) {
+      // ---- the state carry alone: S = 2^E A, A rescaled in place only where the gates
+      //      say so (the weights of the scaled X carry 2^{-E})
+      // the update of chunk c has accumulated: its commit to xhfree[c & 1] (the update of
+      // chunk c - 2, the phase before, is known complete wherever this is called)
+      auto upd_done = [&](int c) {
+        return mbar_wait_warp(&sm.xhfree[c & 1], (c >> 1) & 1, wc, W_S_UPD);
+      };
+      float E = 0.f;  // after the chunks walked so far
+      bool ok = nch > 0 ? scaled_x(0) : true;
+      for (int c = 0; c < nch && ok; ++c) {
+        const int g = c % GS;
+        const GateSlot& gs = sm.gates[g];
+        if (!mbar_wait_warp(&sm.gfull[g], (c / GS) & 1, wc, W_S_GFULL)) { ok = false; break; }
+        E = gs.Eout;
+        if (gs.renorm) {
+          if (c > 0 && !upd_done(c - 1)) { ok = false; break; }
+          tc_fence_after();
+          const float rs = gs.rs;
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        float v[32];
-        tmem_ld32(tS + 32 * hf, v);
-        tmem_ld_wait();
+          for (int hf = 0; hf < 2; ++hf) {
+            float v[32];
+            tmem_ld32(tS + 32 * hf, v);
+            tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) pk[16 * hf + e] = pack_bf16(v[2 * e], v[2 * e + 1]);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] *= gC;
-        tmem_st32(tS + 32 * hf, v);
+            for (int e = 0; e < 32; ++e) v[e] *= rs;
+            tmem_st32(tS + 32 * hf, v);
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.sscaled);  // the update of chunk c may accumulate
+        }
+        if (c + 1 < nch && !scaled_x(c + 1)) ok = false;
+        if (lane == 0) mbar_arrive(&sm.gempty[g]);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.sscaled);  // the update of chunk c may accumulate
-      if (full) {
-        const uint32_t srow = smem_u32(sm.S[hh]);
+      if (ok && p.S_final && (nch == 0 || upd_done(nch - 1))) {
+        tc_fence_after();
+        const float sc = exp2f(E);
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc)
-          st_shared_v4(srow + sw128_off(n, cc), pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
-        fence_proxy_async_smem();
-      }
-      __syncwarp();
-      if (lane == 0 && full) {
-        mbar_arrive(&sm.sready);  // the S X^T product of chunk c may read the tile
-        if (has_ck) {  // the checkpoint of chunk c: the state at its first token
-          tma_store_3d(&tmS, sm.S[hh] + s_part, 64 * hh, n0 + 32 * q, bh * nch_all + cg(c));
-          tma_store_commit();
+        for (int hf = 0; hf < 2; ++hf) {
+          float v[32];
+          tmem_ld32(tS + 32 * hf, v);
+          tmem_ld_wait();
+          float4* so = reinterpret_cast<float4*>(p.S_final + (seg_row * p.dout + n0 + n) * 128 +
+                                                 64 * hh + 32 * hf);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            so[e] = make_float4(sc * v[4 * e], sc * v[4 * e + 1], sc * v[4 * e + 2], sc * v[4 * e + 3]);
         }
       }
-      // the scaled X of the next chunk, while the update of this one runs
-      if (c + 1 < nch && !scaled_x(c + 1)) ok = false;
-      if (lane == 0) mbar_arrive(&sm.gempty[g]);
-    }
-    if (lane == 0) tma_store_wait_all();
-    // the state after the walked chunks, fp32
-    const bool last = full && p.S_last && seg == p.nseg - 1;  // S_T: padded tokens left it unchanged
-    if (ok && (p.S_final || last) &&
-        (nch == 0 || mbar_wait_warp(&sm.dsfull, (nch - 1) & 1, wc, W_S_DSFULL))) {
-      tc_fence_after();
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        float v[32];
-        tmem_ld32(tS + 32 * hf, v);
-        tmem_ld_wait();
-        const size_t col = (size_t)64 * hh + 32 * hf;
-        if (p.S_final) {
-          float4* so = reinterpret_cast<float4*>(p.S_final + (seg_row * p.dout + n0 + n) * 128 + col);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) so[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+    } else {
+      bool ok = nch > 0 ? scaled_x(0) : true;
+      for (int c = 0; c < nch && ok; ++c) {
+        const int g = c % GS;
+        const GateSlot& gs = sm.gates[g];
+        ok = ok && mbar_wait_warp(&sm.gfull[g], (c / GS) & 1, wc, W_S_GFULL);
+        // S_c is complete: the update of chunk c - 1 has accumulated onto it
+        ok = ok && (c == 0 || mbar_wait_warp(&sm.dsfull, (c - 1) & 1, wc, W_S_DSFULL));
+        // the bf16 state tile was last read by the S X^T product and the checkpoint store
+        // of chunk c - 1
+        ok = ok && (!full || c < 1 || mbar_wait_warp(&sm.sfree, (c - 1) & 1, wc, W_S_SFREE));
+        if (lane == 0 && has_ck) tma_store_wait_read_n<0>();
+        __syncwarp();
+        if (!ok) break;
+        tc_fence_after();
+        // S_c -> bf16 (kept packed), S <- 2^{L_{C-1}} S in place; the update of chunk c
+        // may then accumulate, and the bf16 copy goes to buffer b (outputs only)
+        const float gC = gs.gC;
+        uint32_t pk[32];
+  #pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          float v[32];
+          tmem_ld32(tS + 32 * hf, v);
+          tmem_ld_wait();
+  #pragma unroll
+          for (int e = 0; e < 16; ++e) pk[16 * hf + e] = pack_bf16(v[2 * e], v[2 * e + 1]);
+  #pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] *= gC;
+          tmem_st32(tS + 32 * hf, v);
         }
-        if (last) {
-          float4* so = reinterpret_cast<float4*>(p.S_last + ((size_t)bh * p.dout + n0 + n) * 128 + col);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) so[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.sscaled);  // the update of chunk c may accumulate
+        if (full) {
+          const uint32_t srow = smem_u32(sm.S[hh]);
+  #pragma unroll
+          for (int cc = 0; cc < 8; ++cc)
+            st_shared_v4(srow + sw128_off(n, cc), pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0 && full) {
+          mbar_arrive(&sm.sready);  // the S X^T product of chunk c may read the tile
+          if (has_ck) {  // the checkpoint of chunk c: the state at its first token
+            tma_store_3d(&tmS, sm.S[hh] + s_part, 64 * hh, n0 + 32 * q, bh * nch_all + cg(c));
+            tma_store_commit();
+          }
+        }
+        // the scaled X of the next chunk, while the update of this one runs
+        if (c + 1 < nch && !scaled_x(c + 1)) ok = false;
+        if (lane == 0) mbar_arrive(&sm.gempty[g]);
+      }
+      if (lane == 0) tma_store_wait_all();
+      // the state after the walked chunks, fp32
+      const bool last = full && p.S_last && seg == p.nseg - 1;  // S_T: padded tokens left it unchanged
+      if (ok && (p.S_final || last) &&
+          (nch == 0 || mbar_wait_warp(&sm.dsfull, (nch - 1) & 1, wc, W_S_DSFULL))) {
+        tc_fence_after();
+  #pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          float v[32];
+          tmem_ld32(tS + 32 * hf, v);
+          tmem_ld_wait();
+          const size_t col = (size_t)64 * hh + 32 * hf;
+          if (p.S_final) {
+            float4* so = reinterpret_cast<float4*>(p.S_final + (seg_row * p.dout + n0 + n) * 128 + col);
+  #pragma unroll
+            for (int e = 0; e < 8; ++e) so[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+          }
+          if (last) {
+            float4* so = reinterpret_cast<float4*>(p.S_last + ((size_t)bh * p.dout + n0 + n) * 128 + col);
+  #pragma unroll
+            for (int e = 0; e < 8; ++e) so[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+          }
         }
       }
     }
@@ -702,13 +805,19 @@ cudaError_t launch_fwd(const TcFwdParams& prm, const void* x, const void* g, cud
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
   if (!bit || !(attr_set.load() & bit)) {
-    cudaError_t e = cudaFuncSetAttribute(fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(fwd_kernel<true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(fwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set.fetch_or(bit);
   }
   const int grid = prm.B * prm.H * (prm.dout / 128) * prm.nseg;
-  fwd_kernel<<<grid, NTHREADS, kSmemBytes, st>>>(mx, mg, my, ms, prm);
+  if (prm.summary)
+    fwd_kernel<false><<<grid, NTHREADS, kSmemBytes, st>>>(mx, mg, my, ms, prm);
+  else
+    fwd_kernel<true><<<grid, NTHREADS, kSmemBytes, st>>>(mx, mg, my, ms, prm);
   count_launch();
   return cudaGetLastError();
 }
