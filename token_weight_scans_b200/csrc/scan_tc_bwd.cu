@@ -48,6 +48,12 @@
 // therefore split over three issuers on three schedulers (A: the Gram products,
 // dW0, V^T; B: the r accumulator and the Lam update; C: the dx accumulator), so
 // that each accumulator has a single issuer.
+//
+// A later slice of d_out (accumulate) adds its dx to the earlier slices' by one bulk
+// reduction per chunk in L2 (staged row-major) and its d_eta and d_alpha by atomic
+// adds, one per element, so that no load of the earlier values sits on its chain;
+// with one add per element onto a completed launch's result, the sums do not depend
+// on timing.
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -264,8 +270,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (!mbar_wait(&sm.staged[sj], (j / NS) & 1, wc, W_TMA_STAGED)) return false;
         tma_store_3d(&tmDG, sm.G[sj], p.n0, t0j, bh);
         tma_store_3d(&tmDG, sm.G[sj] + TILE, p.n0 + 64, t0j, bh);
-        tma_store_3d(&tmDX, sm.U[sj], 0, t0j, bh);
-        tma_store_3d(&tmDX, sm.U[sj] + TILE, 64, t0j, bh);
+        if (!p.accumulate) {
+          tma_store_3d(&tmDX, sm.U[sj], 0, t0j, bh);
+          tma_store_3d(&tmDX, sm.U[sj] + TILE, 64, t0j, bh);
+        } else {  // later slices: the staged rows (row-major) are added onto dx in L2
+          const int rows = min(C, T - t0j);
+          bulk_reduce_add_bf16(p.dx + ((size_t)bh * T + t0j) * 128, sm.U[sj], (uint32_t)rows * 256u);
+        }
         tma_store_commit();
         tma_store_wait_read();
         mbar_arrive(&sm.xempty[sj]);
@@ -954,28 +965,27 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               }
             }
           }
-          if (!lo && p.accumulate && t0 + i < T) {  // add the dx of the slices already done
-            const uint4* dxo = reinterpret_cast<const uint4*>(p.dx + (tokbase + i) * 128 + 32 * wg);
+          if (!lo && p.accumulate) {
+            // this slice's dx is added onto that of the slices already done by one bulk
+            // reduction of the chunk's rows (issued with the stores of the stage), so it is
+            // staged row-major: row i at 256 i bytes
+            const uint32_t trow = smem_u32(sm.U[st]) + (uint32_t)i * 256u + 64u * wg;
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
-              const uint4 o = dxo[cc];
-              v[8 * cc + 0] += bf16_lo(o.x);
-              v[8 * cc + 1] += bf16_hi(o.x);
-              v[8 * cc + 2] += bf16_lo(o.y);
-              v[8 * cc + 3] += bf16_hi(o.y);
-              v[8 * cc + 4] += bf16_lo(o.z);
-              v[8 * cc + 5] += bf16_hi(o.z);
-              v[8 * cc + 6] += bf16_lo(o.w);
-              v[8 * cc + 7] += bf16_hi(o.w);
+              st_shared_v4(trow + 16u * cc, pack_bf16(v[8 * cc], v[8 * cc + 1]),
+                           pack_bf16(v[8 * cc + 2], v[8 * cc + 3]),
+                           pack_bf16(v[8 * cc + 4], v[8 * cc + 5]),
+                           pack_bf16(v[8 * cc + 6], v[8 * cc + 7]));
             }
-          }
-          const uint32_t trow = smem_u32(lo ? sm.G[st] : sm.U[st]) + (wg >> 1) * TILE;
+          } else {
+            const uint32_t trow = smem_u32(lo ? sm.G[st] : sm.U[st]) + (wg >> 1) * TILE;
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc)
-            st_shared_v4(trow + sw128_off(i, 4 * (wg & 1) + cc), pack_bf16(v[8 * cc], v[8 * cc + 1]),
-                         pack_bf16(v[8 * cc + 2], v[8 * cc + 3]),
-                         pack_bf16(v[8 * cc + 4], v[8 * cc + 5]),
-                         pack_bf16(v[8 * cc + 6], v[8 * cc + 7]));
+            for (int cc = 0; cc < 4; ++cc)
+              st_shared_v4(trow + sw128_off(i, 4 * (wg & 1) + cc), pack_bf16(v[8 * cc], v[8 * cc + 1]),
+                           pack_bf16(v[8 * cc + 2], v[8 * cc + 3]),
+                           pack_bf16(v[8 * cc + 4], v[8 * cc + 5]),
+                           pack_bf16(v[8 * cc + 6], v[8 * cc + 7]));
+          }
           fence_proxy_async_smem();
         }
       }
@@ -985,7 +995,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int j = mt;
         const float deta =
             -(gs.del[j] * sm.qv[j] + sm.tv[0][j] + sm.tv[1][j] + sm.tv[2][j] + sm.tv[3][j]);
-        if (t0 + j < T) p.d_eta[tokbase + j] = p.accumulate ? p.d_eta[tokbase + j] + deta : deta;
+        if (t0 + j < T) {  // later slices add (one fire-and-forget add per element)
+          if (p.accumulate)
+            atomicAdd(p.d_eta + tokbase + j, deta);
+          else
+            p.d_eta[tokbase + j] = deta;
+        }
       }
       if (ok && mt >= C && mt < 2 * C) {
         const int i = mt - C;
@@ -999,7 +1014,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           E += (e4.x + e4.y) + (e4.z + e4.w);
         }
         const float da = gs.gam[i] * gs.del[i] * E + gs.del[i] * t2 + gs.gam[i] * t3 + h4;
-        if (t0 + i < T) p.d_alpha[tokbase + i] = p.accumulate ? p.d_alpha[tokbase + i] + da : da;
+        if (t0 + i < T) {
+          if (p.accumulate)
+            atomicAdd(p.d_alpha + tokbase + i, da);
+          else
+            p.d_alpha[tokbase + i] = da;
+        }
       }
 
       __syncwarp();
