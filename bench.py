@@ -160,9 +160,10 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def kernel_traffic():
+def kernel_traffic(cfg, dom):
     """DRAM bytes per launch of the dominant kernel from the committed ncu summary, or
-    None when the kernel source changed since the counters were taken."""
+    None when the kernel source changed since the counters were taken, or when the
+    record is for another call or workload."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(path):
         return None, None
@@ -173,6 +174,10 @@ def kernel_traffic():
         return None, None
     h = hashlib.sha256(open(src, "rb").read()).hexdigest()
     if h != d.get("source_sha256"):
+        return None, d.get("kernel")
+    w = d.get("workload", {})
+    shape = {"B": cfg.B, "H": cfg.H, "T": cfg.T, "d_in": cfg.d_in, "d_out": cfg.d_out}
+    if d.get("call") != dom or w != shape:
         return None, d.get("kernel")
     return d.get("bytes_per_launch"), d.get("kernel")
 
@@ -673,7 +678,7 @@ def main():
         dom = "bwd" if do_bwd else "fwd"
         dom_ms = bwd_ms if do_bwd else fwd_ms
         achieved = ab[dom] / (dom_ms * 1e-3) / 1e9
-        traffic, tkernel = kernel_traffic()
+        traffic, tkernel = kernel_traffic(cfg, dom)
         step_bytes = ab["fwd"] + (ab["bwd"] if do_bwd else 0)
         step_flops = af["fwd"] + (af["bwd"] if do_bwd else 0)
         t_roof = max(step_bytes / (peaks["hbm_gbs"] * 1e9),
