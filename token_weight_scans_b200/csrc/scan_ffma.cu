@@ -252,24 +252,25 @@ __global__ void __launch_bounds__(FT, 1) fwd_kernel(FwdArgs a) {
           }
       }
       __syncthreads();
-      // y_i = W0 x_i + D[i][-1] S_in x_i + sum_j P_ij g_j; thread tile 2 tokens x 4 outputs
-      for (int tile = tid; tile < (FC / 2) * NG; tile += FT) {
+      // y_i = W0 x_i + D[i][-1] S_in x_i + sum_j P_ij g_j; thread tile 4 tokens x 4 outputs
+      // (a wider tile than the reverse's: each W0 and S row it loads serves 4 tokens)
+      for (int tile = tid; tile < (FC / 4) * NG; tile += FT) {
         const int ig = tile / NG, ng = tile - ig * NG;
-        float a1[2][4], a2[2][4], a3[2][4];
+        float a1[4][4], a2[4][4], a3[4][4];
 #pragma unroll
-        for (int q = 0; q < 2; ++q)
+        for (int q = 0; q < 4; ++q)
 #pragma unroll
           for (int r = 0; r < 4; ++r) a1[q][r] = a2[q][r] = a3[q][r] = 0.f;
         for (int k = 0; k < din; k += 4) {
-          float4 xv[2];
+          float4 xv[4];
 #pragma unroll
-          for (int q = 0; q < 2; ++q) xv[q] = *reinterpret_cast<const float4*>(&X[(ig * 2 + q) * LDI + k]);
+          for (int q = 0; q < 4; ++q) xv[q] = *reinterpret_cast<const float4*>(&X[(ig * 4 + q) * LDI + k]);
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
             const float4 wv = *reinterpret_cast<const float4*>(&W[(ng + NG * r) * LDI + k]);
             const float4 sv = *reinterpret_cast<const float4*>(&S[(ng + NG * r) * LDI + k]);
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
+            for (int q = 0; q < 4; ++q) {
               a1[q][r] += dot4(xv[q], wv);
               a2[q][r] += dot4(xv[q], sv);
             }
@@ -280,15 +281,15 @@ __global__ void __launch_bounds__(FT, 1) fwd_kernel(FwdArgs a) {
 #pragma unroll
           for (int r = 0; r < 4; ++r) gv[r] = G[j * LDO + ng + NG * r];
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const float pv = P[(ig * 2 + q) * LDC + j];
+          for (int q = 0; q < 4; ++q) {
+            const float pv = P[(ig * 4 + q) * LDC + j];
 #pragma unroll
             for (int r = 0; r < 4; ++r) a3[q][r] = fmaf(pv, gv[r], a3[q][r]);
           }
         }
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const int i = ig * 2 + q;
+        for (int q = 0; q < 4; ++q) {
+          const int i = ig * 4 + q;
           if (i < nt) {
             const float gam = Dt[i * LDD];
 #pragma unroll
