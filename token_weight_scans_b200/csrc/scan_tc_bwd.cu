@@ -545,9 +545,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint32_t sS = smem_u32(sm.SL[it & 1]);  // S_in, then the chunk matrices
       ok = ok && mbar_wait_warp(&sm.gfull[g], (it / GS) & 1, wc, W_M_GFULL);
       ok = ok && mbar_wait_warp(&sm.xfull[st], (it / NS) & 1, wc, W_M_GFULL);
-      ok = ok && mbar_wait_warp(&sm.sfull, it & 1, wc, W_M_GFULL);
-      tc_fence_after();
-
       if (ok) {
         // ---- Xg = diag(gam) X for the Lam update (the previous update has read Xg: the
         //      previous chunk's b2full covers it); two 16-byte pieces per thread
@@ -566,6 +563,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.xgready);
       }
+      // S_in has landed (Xg above needs only the X tile, so it goes first)
+      ok = ok && mbar_wait_warp(&sm.sfull, it & 1, wc, W_M_GFULL);
+      tc_fence_after();
       if (ok) {
         // ---- <Lam_end, S_in>, then Lam <- 2^{L_{C-1}} Lam in place (Lam_end is complete
         //      since the previous chunk's b2full; this overlaps the R1 and DXb products)
@@ -575,19 +575,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           float v[32];
           tmem_ld32(tL, v);
           tmem_ld_wait();
-          float acc = 0.f;
+          float ac4[4] = {0.f, 0.f, 0.f, 0.f};  // four chains, summed in a fixed order
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) {
             const uint4 sv = ld_shared_v4(row + sw128_off(n, 4 * (wg & 1) + cc));
-            acc = fmaf(v[8 * cc + 0], bf16_lo(sv.x), acc);
-            acc = fmaf(v[8 * cc + 1], bf16_hi(sv.x), acc);
-            acc = fmaf(v[8 * cc + 2], bf16_lo(sv.y), acc);
-            acc = fmaf(v[8 * cc + 3], bf16_hi(sv.y), acc);
-            acc = fmaf(v[8 * cc + 4], bf16_lo(sv.z), acc);
-            acc = fmaf(v[8 * cc + 5], bf16_hi(sv.z), acc);
-            acc = fmaf(v[8 * cc + 6], bf16_lo(sv.w), acc);
-            acc = fmaf(v[8 * cc + 7], bf16_hi(sv.w), acc);
+            ac4[cc] = fmaf(v[8 * cc + 0], bf16_lo(sv.x), ac4[cc]);
+            ac4[cc] = fmaf(v[8 * cc + 1], bf16_hi(sv.x), ac4[cc]);
+            ac4[cc] = fmaf(v[8 * cc + 2], bf16_lo(sv.y), ac4[cc]);
+            ac4[cc] = fmaf(v[8 * cc + 3], bf16_hi(sv.y), ac4[cc]);
+            ac4[cc] = fmaf(v[8 * cc + 4], bf16_lo(sv.z), ac4[cc]);
+            ac4[cc] = fmaf(v[8 * cc + 5], bf16_hi(sv.z), ac4[cc]);
+            ac4[cc] = fmaf(v[8 * cc + 6], bf16_lo(sv.w), ac4[cc]);
+            ac4[cc] = fmaf(v[8 * cc + 7], bf16_hi(sv.w), ac4[cc]);
           }
+          float acc = (ac4[0] + ac4[1]) + (ac4[2] + ac4[3]);
 #pragma unroll
           for (int e = 0; e < 32; ++e) v[e] *= gC;
           tmem_st32(tL, v);
