@@ -614,19 +614,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tmem_ld_wait();
           const int i = ir;
           const uint32_t row = (lo ? sG : sX) + (wg >> 1) * TILE;
-          float acc = 0.f;
+          float ac4[4] = {0.f, 0.f, 0.f, 0.f};  // four chains, summed in a fixed order
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) {
             const uint4 sv = ld_shared_v4(row + sw128_off(i, 4 * (wg & 1) + cc));
-            acc = fmaf(v[8 * cc + 0], bf16_lo(sv.x), acc);
-            acc = fmaf(v[8 * cc + 1], bf16_hi(sv.x), acc);
-            acc = fmaf(v[8 * cc + 2], bf16_lo(sv.y), acc);
-            acc = fmaf(v[8 * cc + 3], bf16_hi(sv.y), acc);
-            acc = fmaf(v[8 * cc + 4], bf16_lo(sv.z), acc);
-            acc = fmaf(v[8 * cc + 5], bf16_hi(sv.z), acc);
-            acc = fmaf(v[8 * cc + 6], bf16_lo(sv.w), acc);
-            acc = fmaf(v[8 * cc + 7], bf16_hi(sv.w), acc);
+            ac4[cc] = fmaf(v[8 * cc + 0], bf16_lo(sv.x), ac4[cc]);
+            ac4[cc] = fmaf(v[8 * cc + 1], bf16_hi(sv.x), ac4[cc]);
+            ac4[cc] = fmaf(v[8 * cc + 2], bf16_lo(sv.y), ac4[cc]);
+            ac4[cc] = fmaf(v[8 * cc + 3], bf16_hi(sv.y), ac4[cc]);
+            ac4[cc] = fmaf(v[8 * cc + 4], bf16_lo(sv.z), ac4[cc]);
+            ac4[cc] = fmaf(v[8 * cc + 5], bf16_hi(sv.z), ac4[cc]);
+            ac4[cc] = fmaf(v[8 * cc + 6], bf16_lo(sv.w), ac4[cc]);
+            ac4[cc] = fmaf(v[8 * cc + 7], bf16_hi(sv.w), ac4[cc]);
           }
+          const float acc = (ac4[0] + ac4[1]) + (ac4[2] + ac4[3]);
           const float sc = lo ? gs.del[i] : gs.gam[i];
 #pragma unroll
           for (int e = 0; e < 32; ++e) v[e] *= sc;
@@ -637,6 +638,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tmem_st_wait();
       }
       named_sync_math();  // (B1) S_in read; partial sums of q, p and E written; G read
+      if (ok && mt < C) {
+        const int j = mt;
+        sm.qv[j] = sm.redq[0][j] + sm.redq[1][j] + sm.redq[2][j] + sm.redq[3][j];
+        sm.pv[j] = sm.redp[0][j] + sm.redp[1][j] + sm.redp[2][j] + sm.redp[3][j];
+      }
       // the Gram products (which read G) are complete before G is scaled in place
       ok = ok && mbar_wait_warp(&sm.ccfull, it & 1, wc, W_M_CC);
       tc_fence_after();
@@ -656,11 +662,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.m1a);
-      }
-      if (ok && mt < C) {
-        const int j = mt;
-        sm.qv[j] = sm.redq[0][j] + sm.redq[1][j] + sm.redq[2][j] + sm.redq[3][j];
-        sm.pv[j] = sm.redp[0][j] + sm.redp[1][j] + sm.redp[2][j] + sm.redp[3][j];
       }
       named_sync_math();  // (B2) q and p complete; the S_in buffer may be overwritten
 
