@@ -57,3 +57,29 @@ def test_algorithmic_bytes_match_the_stated_per_unit_figures():
     assert ab["fwd"] == N * 776 + w
     assert ab["bwd"] == N * 1296 + 2 * w
     assert ab["bwd"] == pytest.approx(681.6e6, rel=1e-3)
+
+
+def test_traffic_record_applies_to_its_call_and_workload_only():
+    """The committed DRAM-traffic record is reported only for the call and workload it was
+    taken on, and only while the kernel source is the one it was taken from."""
+    import dataclasses
+    import hashlib
+    sys.path.insert(0, ROOT)
+    import bench
+    from token_weight_scans_b200 import inputs
+    with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
+        rec = json.load(f)
+    src = open(os.path.join(ROOT, rec["source"]), "rb").read()
+    current = hashlib.sha256(src).hexdigest() == rec["source_sha256"]
+    w = rec["workload"]
+    match = [c for c in inputs.CONFIGS
+             if {"B": c.B, "H": c.H, "T": c.T, "d_in": c.d_in, "d_out": c.d_out} == w]
+    assert match, "the record names a workload that no configuration has"
+    cfg = match[0]
+    got, kernel = bench.kernel_traffic(cfg, rec["call"])
+    assert kernel == rec["kernel"]
+    assert got == (rec["bytes_per_launch"] if current else None)
+    other = "fwd" if rec["call"] == "bwd" else "bwd"
+    assert bench.kernel_traffic(cfg, other)[0] is None
+    reduced = dataclasses.replace(cfg, B=cfg.B // 2)
+    assert bench.kernel_traffic(reduced, rec["call"])[0] is None
