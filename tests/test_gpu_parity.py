@@ -99,7 +99,10 @@ def test_mid_size_several_chunks(dtype):
     assert_close(gpu, ref, dtype, ("y",) + OUTS, "B2H3T300d128")
 
 
-@pytest.mark.parametrize("shape", [(1, 2, 70, 8, 64), (2, 1, 45, 96, 16), (1, 1, 40, 128, 64)])
+# the last three have tile loops of several passes per thread (d_in = 512: 2048 dx tiles;
+# d_out = 256: 1024 r tiles and a 256-wide Gram product)
+@pytest.mark.parametrize("shape", [(1, 2, 70, 8, 64), (2, 1, 45, 96, 16), (1, 1, 40, 128, 64),
+                                   (1, 1, 70, 512, 16), (1, 1, 45, 32, 256), (1, 2, 40, 256, 32)])
 def test_rectangular(shape):
     B, H, T, di, do = shape
     d = inputs.draw(B, H, T, di, do, dtype="f32", seed=sum(shape))
