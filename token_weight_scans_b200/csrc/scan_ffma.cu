@@ -24,7 +24,11 @@
 // + intra-chunk state), which avoids any division by alpha.
 
 #include <cuda_bf16.h>
+
+#include <atomic>
 #include <cuda_runtime.h>
+
+#include <type_traits>
 
 #include "common.cuh"
 #include "scan_ffma.h"
@@ -708,11 +712,28 @@ __global__ void reduce_dW0_kernel(const float* __restrict__ part, float* __restr
   }
 }
 
+// The dynamic shared-memory opt-in is per kernel and device; it is raised only when a launch
+// needs more than the largest size set so far (kernel k, device dev < 64).
+static cudaError_t ensure_smem(const void* kernel, int k, size_t smem) {
+  static std::atomic<int> set[4][64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  if (dev >= 0 && dev < 64 && set[k][dev].load() >= (int)smem) return cudaSuccess;
+  const cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) {
+    int cur = set[k][dev].load();
+    while (cur < (int)smem && !set[k][dev].compare_exchange_weak(cur, (int)smem)) {
+    }
+  }
+  return e;
+}
+
 template <typename Tio>
 static cudaError_t launch_fwd_t(const FwdArgs& a, cudaStream_t st) {
   const size_t smem = fwd_smem_bytes(a.din, a.dout);
-  cudaError_t e = cudaFuncSetAttribute(fwd_kernel<Tio>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(fwd_kernel<Tio>),
+                              std::is_same<Tio, float>::value ? 0 : 1, smem);
   if (e != cudaSuccess) return e;
   fwd_kernel<Tio><<<a.B * a.H * a.nseg, FT, smem, st>>>(a);
   count_launch();
@@ -722,8 +743,8 @@ static cudaError_t launch_fwd_t(const FwdArgs& a, cudaStream_t st) {
 template <typename Tio>
 static cudaError_t launch_bwd_t(const BwdArgs& a, cudaStream_t st) {
   const size_t smem = bwd_smem_bytes(a.din, a.dout);
-  cudaError_t e = cudaFuncSetAttribute(bwd_kernel<Tio>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(bwd_kernel<Tio>),
+                              std::is_same<Tio, float>::value ? 2 : 3, smem);
   if (e != cudaSuccess) return e;
   bwd_kernel<Tio><<<a.B * a.H * a.nseg, FT, smem, st>>>(a);
   count_launch();
