@@ -225,19 +225,21 @@ def summary_rescale():
     tw.lib().gradlev_debug_summary_rescale(-1.0)
 
 
+@pytest.mark.parametrize("dout", [128, 256])
 @pytest.mark.parametrize("bound", [64.0, 4.0, 0.0],
                          ids=["default", "every-few-chunks", "every-chunk"])
-def test_tc_segment_summary_deferred_decay(bound, summary_rescale):
+def test_tc_segment_summary_deferred_decay(bound, dout, summary_rescale):
     """The summary passes keep the decay since the last in-place rescale of the carried
     matrix as a scale 2^E outside tensor memory and rescale the matrix once E would drop
     below -bound. Sixteen scans of 72 chunks are cut into 9 segments of 8 chunks; the
     same scans run unsegmented as heads of a batch of 80 (no summary pass). With these
     gates (about -1.3 of log2 decay per chunk) the rescale never runs at the default
     bound, every few chunks at 4 and at every chunk at 0; the results agree with the
-    unsegmented run and with the oracle whatever the bound."""
+    unsegmented run and with the oracle whatever the bound. At d_out = 256 the reverse's
+    summary pass carries both 128-row slices of the adjoint in one CTA."""
     summary_rescale(bound)
     H, T = 80, 72 * 64
-    big = inputs.draw(1, H, T, 128, 128, dtype="bf16", alpha_mode="log_uniform", seed=62)
+    big = inputs.draw(1, H, T, 128, dout, dtype="bf16", alpha_mode="log_uniform", seed=62)
     lone = {k: (v[:16] if k == "W0" else v[:, :16]) for k, v in big.items()}
     a = gpu_fwd_bwd(lone)
     b = gpu_fwd_bwd(big)
@@ -246,7 +248,7 @@ def test_tc_segment_summary_deferred_decay(bound, summary_rescale):
         assert err <= 1e-2, (k, err)
     assert rel_err(a["dW0"], b["dW0"][:16]) <= 1e-2
     got = {k: (a[k][5:6] if k == "dW0" else a[k][:, 5:6]) for k in ("y",) + BWD_OUTS}
-    check_all(got, oracle_fwd_bwd(heads_slice(lone, 0, 5)), f"segmented, bound {bound}")
+    check_all(got, oracle_fwd_bwd(heads_slice(lone, 0, 5)), f"segmented, bound {bound}, d_out {dout}")
 
 
 # ------------------------------------------------------------------ bounded-wait failure path

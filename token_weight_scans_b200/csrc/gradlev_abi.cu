@@ -241,6 +241,7 @@ gradlev_status bwd_run(int B, int H, int T, int din, int dout, gradlev_dtype dt,
       sum.summary = 1;
       sum.reverse = 1;
       sum.rescale_log2 = g_rescale_log2;
+      sum.two_slices = dout == 256 ? 1 : 0;  // one CTA per (scan, segment): one wave
       if (tc::launch_fwd(sum, x, dy, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
       // the last segment ends where the adjoint LamT flows in
       if (tc::combine_segments(sb.loc, sb.L, io.LamT, sb.comb, B * H, sp.nseg, dout * din, 1,

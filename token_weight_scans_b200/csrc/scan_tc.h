@@ -43,6 +43,8 @@ struct TcFwdParams {
   // summary mode: the decay since the last in-place rescale of the state is kept as a
   // scale 2^E, and the state is rescaled once E would drop below -rescale_log2 (0..126)
   float rescale_log2 = kSummaryRescaleLog2;
+  // summary mode at d_out = 256: 1 = one CTA carries both 128-row slices (grid B*H*nseg)
+  int two_slices = 0;
 };
 
 // The reverse scan of one 128-row slice [n0, n0+128) of d_out: the rows of the

@@ -85,6 +85,7 @@ constexpr int BIG = 128 * 128; // bytes of one [128 rows x 128 B] swizzled block
 constexpr uint32_t COL_K0 = 0, COL_K1 = 64;      // K = X X^T, double buffer (lanes 0-15)
 constexpr uint32_t COL_Y = 128;                  // + 128 * buffer: Y1 | Y2 (128 columns)
 constexpr uint32_t COL_S = 384;                  // fp32 state (128 columns, all 128 lanes)
+constexpr uint32_t COL_S2 = 128;                 // state carry alone with two slices: the second
 constexpr uint32_t LANE16 = 16u << 16;
 
 // With M = L_{31}, the mask factor -eta_j 2^{L_{i-1} - L_j} = ra_i ca_j whenever
@@ -148,6 +149,10 @@ __device__ __forceinline__ uint8_t* stage_x(Smem& sm, int s) {
 __device__ __forceinline__ uint8_t* stage_g(Smem& sm, int s) {
   return s < NS ? sm.G[s] : (s == NS ? sm.W0[1] : sm.S[1]);
 }
+// the second slice's G tile of stage s < NS (state carry alone with two slices)
+__device__ __forceinline__ uint8_t* stage_g2(Smem& sm, int s) {
+  return s == 0 ? sm.W0[0] : (s == 1 ? sm.W0[1] : sm.S[0]);
+}
 
 }  // namespace
 
@@ -161,7 +166,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   Smem& sm = *reinterpret_cast<Smem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nslice = p.dout >> 7;
+  // the state carry alone at d_out = 256 may carry both 128-row slices in one CTA (the grid
+  // then has no slice dimension): one scaled X tile and one X load serve both
+  const bool two = !FULL && p.two_slices;
+  const int nslice = two ? 1 : p.dout >> 7;
   const int unit = blockIdx.x / p.nseg, seg = blockIdx.x - unit * p.nseg;
   const int bh = unit / nslice, slice = unit - bh * nslice;
   const int h = bh % p.H;
@@ -176,7 +184,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const size_t seg_row = (size_t)bh * p.nseg + seg;  // [bh][seg] index of the segment states
   const WaitCtx wc{&sm.abort, p.status, p.timeout_ns};
   constexpr bool full = FULL;
-  constexpr int ns = FULL ? NS : NS_SUM;  // TMA stages
+  const int ns = FULL ? NS : (two ? NS : NS_SUM);  // TMA stages
 
   if (threadIdx.x == 0) {
     sm.abort = 0;
@@ -244,7 +252,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int c = 0; c < nch; ++c) {
         const int s = c % ns;
         if (!mbar_wait(&sm.empty[s], ((c / ns) & 1) ^ 1, wc, W_TMA_EMPTY)) break;
-        mbar_arrive_expect_tx(&sm.full[s], 4 * TILE);
+        mbar_arrive_expect_tx(&sm.full[s], (two ? 6 : 4) * TILE);
         const int t0 = cg(c) * C;
         uint8_t* sx = stage_x(sm, s);
         uint8_t* sg = stage_g(sm, s);
@@ -252,6 +260,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tma_load_3d(sx + TILE, &tmX, &sm.full[s], 64, t0, bh);
         tma_load_3d(sg, &tmG, &sm.full[s], n0, t0, bh);
         tma_load_3d(sg + TILE, &tmG, &sm.full[s], n0 + 64, t0, bh);
+        if (two) {
+          uint8_t* sg2 = stage_g2(sm, s);
+          tma_load_3d(sg2, &tmG, &sm.full[s], 128, t0, bh);
+          tma_load_3d(sg2 + TILE, &tmG, &sm.full[s], 192, t0, bh);
+        }
         issued = c + 1;
       }
       // teardown: let every load this thread issued land before the CTA exits
@@ -305,6 +318,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int kk = 0; kk < 4; ++kk)
             umma_bf16(tbase + COL_S, desc_at(sw128_desc(sG, TILE, 1024), kk * 2048),
                       desc_at(sw128_desc(sXh, TILE, 1024), kk * 2048), id_ds, 1);
+          if (two) {  // the second slice, from its own G tile and the same scaled X
+            const uint32_t sG2 = smem_u32(stage_g2(sm, s));
+            #pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16(tbase + COL_S2, desc_at(sw128_desc(sG2, TILE, 1024), kk * 2048),
+                        desc_at(sw128_desc(sXh, TILE, 1024), kk * 2048), id_ds, 1);
+          }
           umma_commit(&sm.dsfull);
           if (!(p.inject == 3 && c == 1)) umma_commit(&sm.xhfree[b]);
           if (!full) {  // state carry only: the stage is free once the update has read it
@@ -443,15 +463,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
     const int n = 32 * q + lane;     // row of the d_out slice owned by this thread
     const uint32_t tS = tbase + COL_S + lane_off + 64 * hh;
+    const uint32_t tS2 = tbase + COL_S2 + lane_off + 64 * hh;  // two slices: the second
+    const int nsl = two ? 2 : 1;                                // slices this CTA carries
     const bool has_ck = full && p.ckpt != nullptr;
     // S_0 (the segment's start state, or zero) into TMEM
-    {
+    for (int sl = 0; sl < nsl; ++sl) {
       float v[32];
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         if (p.S_init) {
           const float4* si = reinterpret_cast<const float4*>(
-              p.S_init + (seg_row * p.dout + n0 + n) * 128 + 64 * hh + 32 * hf);
+              p.S_init + (seg_row * p.dout + n0 + 128 * sl + n) * 128 + 64 * hh + 32 * hf);
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const float4 u = si[e];
@@ -464,7 +486,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) v[e] = 0.f;
         }
-        tmem_st32(tS + 32 * hf, v);
+        tmem_st32((sl ? tS2 : tS) + 32 * hf, v);
       }
       tmem_st_wait();
       tc_fence_before();  // the state carry alone: the first update may follow xhready alone
@@ -518,14 +540,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (c > 0 && !upd_done(c - 1)) { ok = false; break; }
           tc_fence_after();
           const float rs = gs.rs;
+          for (int sl = 0; sl < nsl; ++sl) {
 #pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            float v[32];
-            tmem_ld32(tS + 32 * hf, v);
-            tmem_ld_wait();
+            for (int hf = 0; hf < 2; ++hf) {
+              float v[32];
+              tmem_ld32((sl ? tS2 : tS) + 32 * hf, v);
+              tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] *= rs;
-            tmem_st32(tS + 32 * hf, v);
+              for (int e = 0; e < 32; ++e) v[e] *= rs;
+              tmem_st32((sl ? tS2 : tS) + 32 * hf, v);
+            }
           }
           tmem_st_wait();
           tc_fence_before();
@@ -538,16 +562,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (ok && p.S_final && (nch == 0 || upd_done(nch - 1))) {
         tc_fence_after();
         const float sc = exp2f(E);
+        for (int sl = 0; sl < nsl; ++sl) {
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          float v[32];
-          tmem_ld32(tS + 32 * hf, v);
-          tmem_ld_wait();
-          float4* so = reinterpret_cast<float4*>(p.S_final + (seg_row * p.dout + n0 + n) * 128 +
-                                                 64 * hh + 32 * hf);
+          for (int hf = 0; hf < 2; ++hf) {
+            float v[32];
+            tmem_ld32((sl ? tS2 : tS) + 32 * hf, v);
+            tmem_ld_wait();
+            float4* so = reinterpret_cast<float4*>(
+                p.S_final + (seg_row * p.dout + n0 + 128 * sl + n) * 128 + 64 * hh + 32 * hf);
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            so[e] = make_float4(sc * v[4 * e], sc * v[4 * e + 1], sc * v[4 * e + 2], sc * v[4 * e + 3]);
+            for (int e = 0; e < 8; ++e)
+              so[e] = make_float4(sc * v[4 * e], sc * v[4 * e + 1], sc * v[4 * e + 2], sc * v[4 * e + 3]);
+          }
         }
       }
     } else {
@@ -813,7 +839,7 @@ cudaError_t launch_fwd(const TcFwdParams& prm, const void* x, const void* g, cud
     if (e != cudaSuccess) return e;
     attr_set.fetch_or(bit);
   }
-  const int grid = prm.B * prm.H * (prm.dout / 128) * prm.nseg;
+  const int grid = prm.B * prm.H * (prm.two_slices ? 1 : prm.dout / 128) * prm.nseg;
   if (prm.summary)
     fwd_kernel<false><<<grid, NTHREADS, kSmemBytes, st>>>(mx, mg, my, ms, prm);
   else
