@@ -86,6 +86,30 @@ static SegPlan fwd_plan(int B, int H, int T, int dout) {
   return s;
 }
 
+// The forward's summary pass at d_out = 256 carries both 128-row slices in one CTA, so it has
+// half the units of the main pass and may cut each main segment into `ratio` equal pieces
+// (the main segments' boundaries stay segment boundaries, and the combine keeps their start
+// states). Without such a split it runs as the main pass does, one slice per CTA.
+struct SumPlan {
+  SegPlan seg;
+  int two = 0, ratio = 1;
+};
+
+static SumPlan fwd_summary_plan(int B, int H, int T, int dout, const SegPlan& m) {
+  SumPlan p;
+  p.seg = m;
+  if (dout != 256 || m.nseg <= 1) return p;
+  const int n_chunks = (T + tc::kChunk - 1) / tc::kChunk;
+  int r = (148 / (B * H)) / m.nseg;  // pieces per main segment that still fit one wave
+  while (r > 1 && m.seg_chunks % r) --r;
+  if (r < 2) return p;
+  p.seg.seg_chunks = m.seg_chunks / r;
+  p.seg.nseg = (n_chunks + p.seg.seg_chunks - 1) / p.seg.seg_chunks;
+  p.two = 1;
+  p.ratio = r;
+  return p;
+}
+
 static SegPlan bwd_plan(int B, int H, int T) {
   SegPlan s;
   tc::segment_plan(B * H, (T + tc::kChunk - 1) / tc::kChunk, &s.nseg, &s.seg_chunks);
@@ -117,9 +141,15 @@ static SegBufs seg_bufs(char* base, int B, int H, int din, int dout, int nseg) {
           reinterpret_cast<float*>(base + 2 * mats)};
 }
 
+// segments of the forward's summary pass (at least as many as the main pass's)
+static int fwd_seg_count(int B, int H, int T, int dout) {
+  const SegPlan m = fwd_plan(B, H, T, dout);
+  return fwd_summary_plan(B, H, T, dout, m).seg.nseg;
+}
+
 static size_t fwd_scratch_bytes(int B, int H, int T, int din, int dout, gradlev_dtype dt) {
   if (!use_tc(din, dout, dt)) return kStatusBytes + seg_bytes(B, H, din, dout, ffma_plan(B, H, T).nseg);
-  return kStatusBytes + seg_bytes(B, H, din, dout, fwd_plan(B, H, T, dout).nseg);
+  return kStatusBytes + seg_bytes(B, H, din, dout, fwd_seg_count(B, H, T, dout));
 }
 
 static size_t dW0_part_bytes(int B, int H, int T, int din, int dout, gradlev_dtype dt) {
@@ -132,7 +162,7 @@ size_t bwd_scratch_bytes(int B, int H, int T, int din, int dout, gradlev_dtype d
   size_t ws = kStatusBytes + dW0_part_bytes(B, H, T, din, dout, dt);
   if (own_states) ws += align_up(ckpt_bytes_of(B, H, T, din, dout, dt), 256);
   if (use_tc(din, dout, dt)) {
-    const size_t fseg = own_states ? seg_bytes(B, H, din, dout, fwd_plan(B, H, T, dout).nseg) : 0;
+    const size_t fseg = own_states ? seg_bytes(B, H, din, dout, fwd_seg_count(B, H, T, dout)) : 0;
     const size_t bseg = seg_bytes(B, H, din, dout, bwd_plan(B, H, T).nseg);
     ws += fseg > bseg ? fseg : bseg;
   } else {  // the same plan in both directions
@@ -153,21 +183,24 @@ static gradlev_status launch_fwd_impl(int B, int H, int T, int din, int dout, gr
     tc::TcFwdParams prm{B, H, T, din, dout, eta, alpha, W0, static_cast<__nv_bfloat16*>(y),
                         static_cast<__nv_bfloat16*>(ckpt), status, tmo, inject};
     if (sp.nseg > 1) {
-      const SegBufs sb = seg_bufs(seg_ws, B, H, din, dout, sp.nseg);
+      const SumPlan ss = fwd_summary_plan(B, H, T, dout, sp);
+      const SegBufs sb = seg_bufs(seg_ws, B, H, din, dout, ss.seg.nseg);
       tc::TcFwdParams sum = prm;  // each segment's local state and log-decay
       sum.y = nullptr;
       sum.ckpt = nullptr;
       sum.inject = take_inject(INJ_FWD_SUMMARY, 3, &sum.timeout_ns);
-      sum.nseg = sp.nseg;
-      sum.seg_chunks = sp.seg_chunks;
+      sum.nseg = ss.seg.nseg;
+      sum.seg_chunks = ss.seg.seg_chunks;
       sum.S_final = sb.loc;
       sum.seg_L = sb.L;
       sum.summary = 1;
       sum.rescale_log2 = g_rescale_log2;
+      sum.two_slices = ss.two;
       if (tc::launch_fwd(sum, x, g, st) != cudaSuccess) return GRADLEV_ERR_CUDA;
-      // the first segment starts from the carried state S0
-      if (tc::combine_segments(sb.loc, sb.L, S0, sb.comb, B * H, sp.nseg, dout * din, 0, st) !=
-          cudaSuccess)
+      // the first segment starts from the carried state S0; the main pass's segments start
+      // at every ratio-th summary segment
+      if (tc::combine_segments(sb.loc, sb.L, S0, sb.comb, B * H, ss.seg.nseg, dout * din, 0, st,
+                               ss.ratio) != cudaSuccess)
         return GRADLEV_ERR_CUDA;
       prm.nseg = sp.nseg;
       prm.seg_chunks = sp.seg_chunks;

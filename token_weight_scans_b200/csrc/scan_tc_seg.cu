@@ -11,6 +11,8 @@
 //   forward (state S):    S_start(0) = 0,  S_start(k) = 2^{L_{k-1}} S_start(k-1) + Sloc_{k-1}
 //   reverse (adjoint Lam): Lam_end(nseg-1) = 0,
 //                          Lam_end(k) = 2^{L_{k+1}} Lam_end(k+1) + Lloc_{k+1}
+// The forward may keep only every out_every-th start state (the summary pass then cut each
+// segment of the main pass into out_every pieces): out holds [scan][ceil(nseg / out_every)].
 // The recursion runs element by element in fp32: one thread per element of the
 // d_out x d_in matrix, looping over the segments of its scan. A carried start
 // state (forward) or an adjoint flowing in at the sequence's end (reverse)
@@ -26,25 +28,28 @@ namespace tc {
 
 __global__ void combine_kernel(const float* __restrict__ loc, const float* __restrict__ segL,
                                const float* __restrict__ init, float* __restrict__ out, int nseg,
-                               int per_scan, int reverse) {
+                               int per_scan, int reverse, int out_every) {
   const int scan = blockIdx.y;
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= per_scan) return;
   const size_t base = (size_t)scan * nseg;
+  const size_t obase = (size_t)scan * ((nseg + out_every - 1) / out_every);
   float acc = init ? init[(size_t)scan * per_scan + e] : 0.f;
   for (int i = 0; i < nseg; ++i) {
     const int k = reverse ? nseg - 1 - i : i;
     const size_t at = (base + k) * per_scan + e;
     const float l = loc[at];  // read before the write below when loc and out alias
-    out[at] = acc;
+    if (k % out_every == 0) out[(obase + k / out_every) * per_scan + e] = acc;
     acc = fmaf(exp2f(segL[base + k]), acc, l);
   }
 }
 
 cudaError_t combine_segments(const float* loc, const float* segL, const float* init, float* out,
-                             int scans, int nseg, int per_scan, int reverse, cudaStream_t st) {
+                             int scans, int nseg, int per_scan, int reverse, cudaStream_t st,
+                             int out_every) {
+  if (out_every < 1 || (reverse && out_every != 1)) return cudaErrorInvalidValue;
   const dim3 grid((per_scan + 255) / 256, scans);
-  combine_kernel<<<grid, 256, 0, st>>>(loc, segL, init, out, nseg, per_scan, reverse);
+  combine_kernel<<<grid, 256, 0, st>>>(loc, segL, init, out, nseg, per_scan, reverse, out_every);
   count_launch();
   return cudaGetLastError();
 }
