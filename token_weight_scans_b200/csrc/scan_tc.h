@@ -98,7 +98,8 @@ void segment_plan(int units, int n_chunks, int* nseg, int* seg_chunks);
 // ([scans][per_scan], or null for zero) is the value entering the first segment walked:
 // the carried start state forward, the adjoint flowing in at the end in reverse.
 // out_every > 1 (forward only): out keeps the start states of segments 0, out_every,
-// 2 out_every, ... as [scans][ceil(nseg / out_every)].
+// 2 out_every, ... as [scans][ceil(nseg / out_every)]. out may alias loc only when
+// out_every == 1.
 cudaError_t combine_segments(const float* loc, const float* segL, const float* init, float* out,
                              int scans, int nseg, int per_scan, int reverse, cudaStream_t st,
                              int out_every = 1);
