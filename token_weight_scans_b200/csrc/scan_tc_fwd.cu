@@ -49,7 +49,10 @@
 // the state warps rescale A in place (by 2^{E_c + L_{C-1}}, after which E = 0),
 // and the final state is 2^E A. Every scaled weight stays below eta 2^64, far inside
 // the bf16 and fp32 ranges. Without the bf16 state tile and W0, that shared memory
-// holds two more TMA stages.
+// holds two more TMA stages. At d_out = 256 the state carry alone may instead hold both
+// 128-row slices in one CTA (two_slices): the second slice's state in the TMEM columns the
+// outputs use in the main pass, its G tiles in the W0 and S tiles (three stages), and one
+// X tile and one scaled X tile serving both slices' updates.
 
 #include <cuda.h>
 #include <cuda_bf16.h>
