@@ -10,7 +10,7 @@
 //   deta_t = -g_t . Lam_{t+1} x_t,  dalpha_t = <Lam_{t+1}, S_t>,  dW0 = sum u_t x_t^T.
 //
 // One CTA per (b, h) walks the 64-token chunks backwards, carrying Lam (fp32 in
-// registers, bf16 copy in shared memory). The chunk-start state S_in comes from
+// TMEM, a bf16 copy in shared memory). The chunk-start state S_in comes from
 // the bf16 checkpoints of the forward scan. Inside a chunk (local i, with
 // L_j = sum_{r<=j} log2 alpha, gam_i = 2^{L_{i-1}}, del_i = 2^{L_{C-1}-L_i},
 // a_ij = -eta_j 2^{L_{i-1}-L_j} (j<i), b_is = 2^{L_{s-1}-L_i} (s>i)):
