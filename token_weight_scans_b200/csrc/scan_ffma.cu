@@ -1,7 +1,9 @@
 // CUDA-core (FFMA) chunkwise GradLev scans: the float32 path of the library.
 //
-// Per (b, h) scan one CTA walks the sequence in chunks of FC = 32 tokens and
-// keeps the d_out x d_in float32 state in shared memory. Within a chunk the
+// Per (b, h) scan one CTA walks the sequence in chunks of FC = 32 tokens (or, when
+// few long scans cannot fill the GPU, one CTA per segment of it: a summary pass from
+// a zero start, the segment combine, then the main pass from the combined start
+// state) and keeps the d_out x d_in float32 state in shared memory. Within a chunk the
 // recurrence S_{t+1} = alpha_t S_t - eta_t g_t x_t^T (Cognaptus, "Parallelize
 // the Training, Keep the Learning Serial", section "Once the gradient signals
 // are known, the weight trajectory becomes parallelizable") is unrolled into
